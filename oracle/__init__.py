@@ -1,0 +1,158 @@
+"""CKDA oracle: a plain fp64 CPU implementation of the recurrence.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg import this package. The CUDA library never
+imports, links or calls it, and this package imports nothing from the CUDA
+library: the two share only the seeded input generators, which hold none of
+the method's arithmetic.
+
+The arithmetic lives in ``ckda_oracle.c`` (one token at a time, fp64, the
+recurrence of "Semidirect Fourier Delta Attention" §1 eq. (1) / §2.2 eq. (9)
+with the readout of §3 eq. (14); ranges from "Complex KDA", abstract). This
+module only compiles it with gcc (no fast-math) and marshals numpy arrays.
+
+Every function here is pinned by ``tests/test_oracle_pins.py`` against the
+lesson's worked traces, closed forms and the dense affine composition
+(§2.2 eq. (10)); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ckda_oracle.c")
+_LIB = os.path.join(_HERE, "libckda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ckda_oracle.c into libckda_oracle.so (gcc -O2 -fopenmp, IEEE fp64)."""
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    tmp = _LIB + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared",
+           "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC]
+    subprocess.check_call(cmd)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _bind(path: str):
+    """Load a compiled oracle library and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    ip = ctypes.POINTER(ctypes.c_int32)
+    lp = ctypes.POINTER(ctypes.c_int64)
+    i32 = ctypes.c_int32
+    lib.ckda_oracle_fwd.restype = ctypes.c_int
+    lib.ckda_oracle_fwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, ip,
+                                    i32, i32, i32, i32, ctypes.c_double, i32]
+    lib.ckda_oracle_decode.restype = ctypes.c_int
+    lib.ckda_oracle_decode.argtypes = [dp, dp, dp, dp, dp, dp, dp,
+                                       i32, i32, i32, i32, ctypes.c_double,
+                                       lp, ctypes.c_int64, i32]
+    lib.ckda_oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load(lib=None):
+    global _lib
+    if lib is not None:
+        return lib
+    if _lib is None:
+        _lib = _bind(build())
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor (CPU); upcast exactly
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a, ty=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ty))
+
+
+def max_threads() -> int:
+    return int(_load().ckda_oracle_max_threads())
+
+
+def fwd(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None,
+        scale: float = 1.0, nthreads: int = 0, lib=None):
+    """Token-by-token fp64 forward.
+
+    q, k: [total_T, H, d_k]; v: [total_T, H, d_v]; alpha: [total_T, H, d_k];
+    beta: [total_T, H]; initial_state: [N, H, d_k, d_v] or None (zero);
+    cu_seqlens: [N+1] int (None = one sequence of total_T tokens).
+    Returns (o [total_T, H, d_v], final_state [N, H, d_k, d_v]) in fp64.
+    ``lib`` selects another compiled copy of the oracle (the mutation tests
+    load deliberately broken copies to show the pins catch them).
+    """
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    s0 = _f64(initial_state)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int32)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    N = cu.shape[0] - 1
+    if int(cu[-1]) != T:
+        raise ValueError("cu_seqlens[-1] must equal total_T")
+    if s0 is not None and s0.shape != (N, H, dk, dv):
+        raise ValueError("initial_state shape mismatch")
+    o = np.zeros((T, H, dv), dtype=np.float64)
+    sf = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load(lib).ckda_oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                 _ptr(beta), _ptr(s0), _ptr(sf), _ptr(o),
+                                 _ptr(cu, ctypes.c_int32), N, H, dk, dv,
+                                 float(scale), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("ckda_oracle_fwd failed (%d)" % rc)
+    return o, sf
+
+
+def decode(q, k, v, alpha, beta, state, scale: float = 1.0, pairs=None,
+           nthreads: int = 0, lib=None):
+    """One fp64 decode step, in place on ``state`` (an fp64 numpy array).
+
+    q, k: [N, H, d_k]; v: [N, H, d_v]; alpha: [N, H, d_k]; beta: [N, H];
+    state: [N, H, d_k, d_v] float64, C-contiguous, updated in place.
+    pairs: optional int64 array of flattened (n*H + h) indices to step; the
+    other pairs' state and output are left untouched (output rows zero).
+    Returns o [N, H, d_v] (fp64).
+    """
+    q, k, v, alpha, beta = map(_f64, (q, k, v, alpha, beta))
+    if not (isinstance(state, np.ndarray) and state.dtype == np.float64
+            and state.flags.c_contiguous):
+        raise TypeError("state must be a C-contiguous float64 numpy array")
+    N, H, dk = q.shape
+    dv = v.shape[2]
+    if state.shape != (N, H, dk, dv):
+        raise ValueError("state shape mismatch")
+    o = np.zeros((N, H, dv), dtype=np.float64)
+    pp = None
+    npairs = 0
+    if pairs is not None:
+        pp = np.ascontiguousarray(pairs, dtype=np.int64)
+        npairs = pp.shape[0]
+    rc = _load(lib).ckda_oracle_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha),
+                                    _ptr(beta), _ptr(state), _ptr(o), N, H, dk,
+                                    dv, float(scale),
+                                    _ptr(pp, ctypes.c_int64), npairs,
+                                    int(nthreads))
+    if rc != 0:
+        raise RuntimeError("ckda_oracle_decode failed (%d)" % rc)
+    return o

@@ -1,0 +1,33 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line(
+        "markers", "gpu: needs a CUDA GPU (sm_100a) and the built CUDA library")
+    config.addinivalue_line(
+        "markers", "slow: long CPU test (oracle at full workload size)")
+
+
+def gpu_available() -> bool:
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.fixture(scope="session")
+def cuda_lib():
+    """The CUDA library binding; a GPU test must never fall back to anything."""
+    if not gpu_available():
+        pytest.fail("a test marked gpu ran without a CUDA device")
+    from gated_delta_rule_114_b200 import ckda
+    ckda.load()
+    return ckda
