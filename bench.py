@@ -1,0 +1,392 @@
+"""Benchmark of the CKDA hot path on B200: chunked prefill forward + decode step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One JSON line on rank 0. A "step" is one chunked forward (every step of the
+chunkwise path: load, gate cumulant, Grams, UT solve, WY factors, state
+propagation and output) over the CKDA long-prefill batch (B=1, H=32,
+T=8192, d_k=d_v=128, bf16 I/O, fp32 state), inputs resident in HBM. The decode
+step (256 sequences x 32 heads, fp32 state in HBM) is timed in the same run
+and reported under "decode". N>1 (torchrun, one rank per GPU): every rank runs
+its own copy of the batch (heads and sequences are independent, so no
+collective sits on the data path); value = all ranks' tokens / max time.
+
+--impl reference runs the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_114_b200 import ckda  # noqa: E402
+from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,  # noqa: E402
+                                              make_decode_tokens,
+                                              make_fwd_inputs)
+
+METRIC = ("CKDA prefill tokens/s (H=32, d=128, T=8192) + % bf16 roofline; "
+          "decode tok/s, HBM GB/s")
+PREFILL = "ckda_B1_H32_T8192_d128"
+DECODE = "decode_N256_H32_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def esize(dt):
+    return 2 if dt == torch.bfloat16 else 4
+
+
+def prefill_bytes(inp) -> int:
+    """Algorithmic HBM bytes of one forward: every input read once, every
+    output written once (q, k, v, alpha, beta, o per token-head; states)."""
+    T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[2]
+    es = esize(inp["q"].dtype)
+    per_th = (2 * dk + dv) * es + dk * 4 + 4 + dv * es
+    N = inp["cu_seqlens"].numel() - 1
+    st = N * H * dk * dv * 4
+    return T * H * per_th + (st if inp["initial_state"] is not None else 0) + st
+
+
+def prefill_flops(inp, C=64) -> float:
+    """Useful flops of the chunked form: per chunk 2.5 C^2 d + 3 C d^2 + C^3/6
+    multiply-adds (Grams, WY factors, state/output contractions, UT solve)."""
+    T, H, d = inp["q"].shape
+    cu = inp["cu_seqlens"].tolist()
+    mac = 0.0
+    for n in range(len(cu) - 1):
+        L = cu[n + 1] - cu[n]
+        full, rem = divmod(L, C)
+        for c in [C] * full + ([rem] if rem else []):
+            mac += 2.5 * c * c * d + 3 * c * d * d + c ** 3 / 6.0
+    return 2.0 * mac * H
+
+
+def decode_bytes(N, H, dk, dv, dt) -> int:
+    es = esize(dt)
+    return N * H * (2 * dk * dv * 4 + (2 * dk + dv) * es + dk * 4 + 4 + dv * es)
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons while the timed region runs."""
+
+    REASONS = {  # NVML clocks-event-reason bits
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period: float = 0.02):
+        self.index = index
+        self.period = period
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self._nvml = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for b, name in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples)}
+
+
+def time_loop(fn, steps: int, warmup: int, stream, barrier=None):
+    """W untimed calls, then K calls between CUDA events on `stream`."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    return start.elapsed_time(end) / steps  # ms per step
+
+
+def cpu_baseline_prefill(w, inp_cpu, target_s=12.0):
+    """Oracle (as it stands) on a bounded sample: the first h heads of the
+    prefill batch, h grown until one run takes about target_s seconds."""
+    import oracle
+    cores = oracle.max_threads()
+    T = inp_cpu["q"].shape[0]
+    H = inp_cpu["q"].shape[1]
+    h = 1
+    while True:
+        sub = {key: inp_cpu[key][:, :h].contiguous() for key in
+               ("q", "k", "v", "alpha", "beta")}
+        s0 = inp_cpu["initial_state"][:, :h].contiguous()
+        t0 = time.perf_counter()
+        oracle.fwd(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"], s0,
+                   inp_cpu["cu_seqlens"])
+        dt = time.perf_counter() - t0
+        if dt >= target_s / 3 or h >= H:
+            break
+        h = min(H, max(h + 1, int(h * target_s / max(dt, 1e-3))))
+    tok_heads = T * h
+    return {"value": tok_heads / dt / H, "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": ("fp64 token-by-token oracle on %d of %d heads x %d tokens "
+                       "(%d token-heads, %.2f s); tokens/s = token-heads/s / %d heads"
+                       % (h, H, T, tok_heads, dt, H))}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    w = WORKLOADS[PREFILL]
+    inp = make_fwd_inputs(w)
+    cores = oracle.max_threads()
+    T, H = inp["q"].shape[:2]
+    h = 1  # one head of the batch per step: ~0.5-2 s of CPU work
+    sub = {key: inp[key][:, :h].contiguous() for key in ("q", "k", "v", "alpha", "beta")}
+    s0 = inp["initial_state"][:, :h].contiguous()
+
+    def step():
+        oracle.fwd(sub["q"], sub["k"], sub["v"], sub["alpha"], sub["beta"], s0,
+                   inp["cu_seqlens"])
+
+    for _ in range(args.warmup):
+        step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        step()
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * sum(times) / len(times)
+    value = T * h / (ms / 1e3) / H
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PREFILL, "global_batch": 1, "seq_len": T,
+                   "heads": H, "d_k": 128, "d_v": 128, "chunk": 64,
+                   "sample_heads_per_step": h},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": "fp64 oracle on %d of %d heads x %d tokens per step; "
+                                   "tokens/s = token-heads/s / %d heads" % (h, H, T, H)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    barrier = (lambda: dist.barrier()) if dist else None
+    ckda.load()
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+
+    # ---------------- prefill (the headline step)
+    w = WORKLOADS[PREFILL]
+    inp_cpu = make_fwd_inputs(w)
+    dev = {key: (val.cuda() if isinstance(val, torch.Tensor) else val)
+           for key, val in inp_cpu.items()}
+    T_total, H, dk = dev["q"].shape
+    dv = dev["v"].shape[2]
+    N = dev["cu_seqlens"].numel() - 1
+    o = torch.empty((T_total, H, dv), dtype=dev["q"].dtype, device="cuda")
+    sf = torch.empty((N, H, dk, dv), dtype=torch.float32, device="cuda")
+
+    def prefill():
+        ckda.ckda_fwd_chunked(dev["q"], dev["k"], dev["v"], dev["alpha"],
+                              dev["beta"], dev["initial_state"], sf, o,
+                              dev["cu_seqlens"], None, chunk=w.chunk,
+                              stream=stream)
+
+    with ClockSampler(local) as clk:
+        ms = time_loop(prefill, args.steps, args.warmup, stream, barrier)
+    if ckda.ckda_last_error() != ckda.CKDA_OK:
+        raise RuntimeError("kernel reported an error")
+    ms_max = ms
+    if dist:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    tokens = T_total * world
+    value = tokens / (ms_max / 1e3)
+    nbytes = prefill_bytes(inp_cpu)
+    flops = prefill_flops(inp_cpu, w.chunk)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                "traffic": None, "peak_source": pk["source"],
+                "algorithmic_bytes_per_launch": nbytes,
+                "tensor": {"achieved_tflops": flops / (ms / 1e3) / 1e12,
+                           "peak_tflops": pk["bf16_tflops"],
+                           "frac": flops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                           "useful_flops_per_launch": flops}}
+
+    # ---------------- end to end through the C ABI with host buffers
+    pinned = {key: (val.pin_memory() if isinstance(val, torch.Tensor) else val)
+              for key, val in inp_cpu.items()}
+    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    sf_host = torch.empty(sf.shape, dtype=sf.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for k_, v in pinned.items()
+              if isinstance(v, torch.Tensor))
+    d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * 4
+
+    def e2e_step():
+        for key, val in pinned.items():
+            if isinstance(val, torch.Tensor):
+                dev[key].copy_(val, non_blocking=True)
+        prefill()
+        o_host.copy_(o, non_blocking=True)
+        sf_host.copy_(sf, non_blocking=True)
+
+    e2e_ms = time_loop(e2e_step, args.e2e_steps, 3, stream, barrier)
+    e2e = {"value": T_total * world / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": e2e_ms}
+
+    # ---------------- decode step
+    wd = WORKLOADS[DECODE]
+    state = make_decode_state(wd).cuda()
+    toks = [{key: val.cuda() for key, val in make_decode_tokens(wd, s).items()}
+            for s in range(4)]
+    od = torch.empty((wd.B, wd.H, wd.d_v), dtype=toks[0]["q"].dtype, device="cuda")
+    it = [0]
+
+    def dstep():
+        tk = toks[it[0] % len(toks)]
+        it[0] += 1
+        ckda.ckda_decode_step(tk["q"], tk["k"], tk["v"], tk["alpha"], tk["beta"],
+                              state, od, stream=stream)
+
+    with ClockSampler(local) as dclk:
+        dms = time_loop(dstep, args.decode_steps, args.warmup, stream, barrier)
+    dbytes = decode_bytes(wd.B, wd.H, wd.d_k, wd.d_v, toks[0]["q"].dtype)
+    dgbs = dbytes / (dms / 1e3) / 1e9
+    decode = {"workload": DECODE, "ms_per_step": dms,
+              "tokens_per_s": wd.B * world / (dms / 1e3),
+              "token_heads_per_s": wd.B * wd.H * world / (dms / 1e3),
+              "steps": args.decode_steps,
+              "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"],
+                           "unit": "GB/s", "frac": dgbs / pk["hbm_gbs"],
+                           "traffic": None, "algorithmic_bytes_per_launch": dbytes},
+              "gpu_launches": args.decode_steps, "clocks": dclk.summary()}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_prefill(w, inp_cpu)
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PREFILL, "global_batch": world, "seq_len": T_total,
+                   "heads": H, "d_k": dk, "d_v": dv, "chunk": w.chunk,
+                   "io": "bf16 q/k/v/o, fp32 alpha/beta/state",
+                   "l2": "inputs larger than L2 (%.0f MB per step)" % (nbytes / 1e6),
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,198 @@
+"""Python binding of the CKDA C ABI (include/ckda.h).
+
+Argument marshalling only: every step of the forward and the decode step runs
+in the CUDA kernels of ``libckda.so``. PyTorch supplies device memory and
+streams. There is no fallback of any kind: if the library cannot be loaded,
+every call raises.
+
+The functions named like the C entry points take caller-allocated tensors
+(like the C ABI); ``fwd_chunked`` and ``decode_step`` are conveniences that
+allocate the outputs with torch and then call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libckda.so")
+
+CKDA_OK, CKDA_ERR_ARG, CKDA_ERR_UNSUPPORTED, CKDA_ERR_CUDA, CKDA_ERR_DEVICE = range(5)
+CKDA_BF16, CKDA_F32 = 0, 1
+_DT = {torch.bfloat16: CKDA_BF16, torch.float32: CKDA_F32}
+
+_lib = None
+
+
+class CkdaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = _lib.ckda_status_string(status).decode() if _lib else str(status)
+        super().__init__("%s: %s" % (where, msg))
+
+
+def load(path: str | None = None):
+    """Load libckda.so (built in-tree by build.py). Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(
+            "libckda.so not found at %s: build it with "
+            "`python -m gated_delta_rule_114_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    lib.ckda_fwd_chunked.restype = ctypes.c_int
+    lib.ckda_fwd_chunked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                     i32, i32, i32, i32, i32, i32, f32,
+                                     ctypes.c_int, vp]
+    lib.ckda_decode_step.restype = ctypes.c_int
+    lib.ckda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                     i32, f32, ctypes.c_int, vp]
+    lib.ckda_status_string.restype = ctypes.c_char_p
+    lib.ckda_status_string.argtypes = [ctypes.c_int]
+    lib.ckda_last_error.restype = ctypes.c_int
+    lib.ckda_last_error.argtypes = [vp]
+    lib.ckda_version.restype = ctypes.c_int32
+    lib.ckda_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def _p(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, where: str):
+    if status != CKDA_OK:
+        raise CkdaError(status, where)
+
+
+def _need(t, name, dtype=None, dims=None):
+    if t is None:
+        raise ValueError("%s is required" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s" % (name, dtype))
+    if dims is not None and t.dim() != dims:
+        raise ValueError("%s must have %d dims" % (name, dims))
+
+
+def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
+                     cu_seqlens=None, cu_seqlens_host=None, N=None, T=None,
+                     chunk: int = 0, scale: float = 1.0, stream=None):
+    """Marshal tensors into ckda_fwd_chunked (see include/ckda.h).
+
+    q, k [T_total, H, d_k]; v, o [T_total, H, d_v] (bf16 or fp32, one dtype);
+    alpha [T_total, H, d_k] fp32; beta [T_total, H] fp32; states
+    [N, H, d_k, d_v] fp32 or None. With cu_seqlens (int32 CUDA [N+1]) the
+    sequences are packed; otherwise give N and T (N sequences of T tokens).
+    cu_seqlens_host: optional CPU int32 copy, validated by the library.
+    """
+    lib = load()
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, nme, q.dtype, 3)
+    _need(alpha, "alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v, o must be bfloat16 or float32")
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+        T = T_total
+    elif N is None or T is None:
+        raise ValueError("give cu_seqlens, or N and T")
+    for t, nme in ((initial_state, "initial_state"), (final_state, "final_state")):
+        if t is not None:
+            _need(t, nme, torch.float32, 4)
+    host_ptr = None
+    if cu_seqlens_host is not None:
+        if cu_seqlens_host.is_cuda or cu_seqlens_host.dtype != torch.int32 \
+                or not cu_seqlens_host.is_contiguous():
+            raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
+        host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    st = lib.ckda_fwd_chunked(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                              _p(initial_state), _p(final_state), _p(o),
+                              _p(cu_seqlens), host_ptr, int(N), int(T), int(H),
+                              int(d_k), int(d_v), int(chunk), float(scale),
+                              _DT[q.dtype], _stream(stream))
+    _check(st, "ckda_fwd_chunked")
+
+
+def ckda_decode_step(q, k, v, alpha, beta, state, o, scale: float = 1.0,
+                     stream=None):
+    """Marshal tensors into ckda_decode_step (state updated in place).
+
+    q, k [N, H, d_k]; v, o [N, H, d_v] (bf16 or fp32); alpha [N, H, d_k] fp32;
+    beta [N, H] fp32; state [N, H, d_k, d_v] fp32.
+    """
+    lib = load()
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, nme, q.dtype, 3)
+    _need(alpha, "alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(state, "state", torch.float32, 4)
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v, o must be bfloat16 or float32")
+    N, H, d_k = q.shape
+    d_v = v.shape[2]
+    st = lib.ckda_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                              _p(state), _p(o), int(N), int(H), int(d_k),
+                              int(d_v), float(scale), _DT[q.dtype],
+                              _stream(stream))
+    _check(st, "ckda_decode_step")
+
+
+def ckda_last_error(stream=None) -> int:
+    """Synchronise the stream; return and clear the device error status."""
+    return int(load().ckda_last_error(_stream(stream)))
+
+
+def version() -> int:
+    return int(load().ckda_version())
+
+
+def fwd_chunked(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None,
+                cu_seqlens_host=None, N=None, T=None, chunk: int = 0,
+                scale: float = 1.0, output_final_state: bool = True,
+                stream=None):
+    """Allocate o (and the final state) with torch, then call ckda_fwd_chunked."""
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+    elif N is None:
+        N, T = 1, T_total
+    o = torch.empty((T_total, H, d_v), dtype=q.dtype, device=q.device)
+    sf = None
+    if output_final_state:
+        sf = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=q.device)
+    ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, sf, o, cu_seqlens,
+                     cu_seqlens_host, N, T, chunk, scale, stream)
+    return o, sf
+
+
+def decode_step(q, k, v, alpha, beta, state, scale: float = 1.0, stream=None):
+    """Allocate o with torch, then call ckda_decode_step (state in place)."""
+    N, H, _ = q.shape
+    o = torch.empty((N, H, v.shape[2]), dtype=q.dtype, device=q.device)
+    ckda_decode_step(q, k, v, alpha, beta, state, o, scale, stream)
+    return o

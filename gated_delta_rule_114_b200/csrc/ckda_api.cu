@@ -1,0 +1,198 @@
+// C ABI of the CKDA library: host-side validation, dispatch, error word.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "ckda.h"
+#include "ckda_common.cuh"
+
+namespace ckda {
+template <typename IOT>
+cudaError_t launch_decode(int dk, int dv, const void *q, const void *k,
+                          const void *v, const float *alpha, const float *beta,
+                          float *state, void *o, int N, int H, float scale,
+                          cudaStream_t st);
+template <typename IOT>
+cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
+                            const void *k, const void *v, const float *alpha,
+                            const float *beta, const float *s0, float *sf,
+                            void *o, const int32_t *cu, int N, int T,
+                            int T_total, int H, float scale, unsigned int *err,
+                            cudaStream_t st);
+bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt);
+cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v,
+                          const float *alpha, const float *beta,
+                          const float *s0, float *sf, void *o,
+                          const int32_t *cu, int N, int T, int T_total, int H,
+                          float scale, unsigned int *err, cudaStream_t st);
+}  // namespace ckda
+
+// The per-device error word. Each device context gets its own instance.
+__device__ unsigned int g_ckda_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+unsigned int *g_err_addr[kMaxDevices] = {};
+
+// Device address of the error word on the current device (cached).
+unsigned int *error_word_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+    return nullptr;
+  std::lock_guard<std::mutex> lk(g_err_mu);
+  if (!g_err_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ckda_error_word) != cudaSuccess) return nullptr;
+    g_err_addr[dev] = static_cast<unsigned int *>(p);
+  }
+  return g_err_addr[dev];
+}
+
+bool supported_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+bool aligned16(const void *p) {
+  return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// [a, a+na) and [b, b+nb) overlap (byte ranges; empty ranges never overlap)
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a);
+  const uintptr_t y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+size_t esize(ckda_dtype dt) { return dt == CKDA_F32 ? 4 : 2; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t ckda_version(void) { return 100; }
+
+const char *ckda_status_string(ckda_status s) {
+  switch (s) {
+    case CKDA_OK: return "CKDA_OK";
+    case CKDA_ERR_ARG: return "CKDA_ERR_ARG: invalid argument";
+    case CKDA_ERR_UNSUPPORTED: return "CKDA_ERR_UNSUPPORTED: unsupported size, chunk or dtype";
+    case CKDA_ERR_CUDA: return "CKDA_ERR_CUDA: CUDA runtime or launch failure";
+    case CKDA_ERR_DEVICE: return "CKDA_ERR_DEVICE: a kernel reported an error";
+  }
+  return "CKDA_UNKNOWN_STATUS";
+}
+
+ckda_status ckda_last_error(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return CKDA_ERR_CUDA;
+  unsigned int w = 0;
+  const unsigned int zero = 0;
+  if (cudaMemcpyFromSymbol(&w, g_ckda_error_word, sizeof(w)) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  if (w != 0 &&
+      cudaMemcpyToSymbol(g_ckda_error_word, &zero, sizeof(zero)) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  return w ? CKDA_ERR_DEVICE : CKDA_OK;
+}
+
+ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta,
+                             const float *initial_state, float *final_state,
+                             void *o, const int32_t *cu_seqlens,
+                             const int32_t *cu_seqlens_host, int32_t N,
+                             int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                             int32_t chunk, float scale, ckda_dtype dt,
+                             cudaStream_t stream) {
+  if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (chunk == 0) chunk = 64;
+  if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_UNSUPPORTED;
+  if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!q || !k || !v || !alpha || !beta || !o) return CKDA_ERR_ARG;
+  const void *ptrs[] = {q, k, v, alpha, beta, o, initial_state, final_state,
+                        cu_seqlens};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return CKDA_ERR_ARG;
+
+  int64_t T_total;
+  if (cu_seqlens == nullptr) {
+    if (cu_seqlens_host) return CKDA_ERR_ARG;
+    T_total = (int64_t)N * T;
+  } else {
+    T_total = T;
+    if (cu_seqlens_host) {
+      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return CKDA_ERR_ARG;
+      for (int32_t n = 0; n < N; ++n)
+        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return CKDA_ERR_ARG;
+    }
+  }
+  if (T_total > INT32_MAX) return CKDA_ERR_ARG;
+
+  // the output must not overlap any input or state
+  const size_t es = esize(dt);
+  const size_t th = (size_t)T_total * H;
+  const size_t ob = th * d_v * es;
+  const size_t sb = (size_t)N * H * d_k * d_v * sizeof(float);
+  if (overlaps(o, ob, q, th * d_k * es) || overlaps(o, ob, k, th * d_k * es) ||
+      overlaps(o, ob, v, th * d_v * es) ||
+      overlaps(o, ob, alpha, th * d_k * sizeof(float)) ||
+      overlaps(o, ob, beta, th * sizeof(float)) ||
+      overlaps(o, ob, initial_state, sb) || overlaps(o, ob, final_state, sb))
+    return CKDA_ERR_ARG;
+  if (final_state && initial_state && final_state != initial_state &&
+      overlaps(final_state, sb, initial_state, sb))
+    return CKDA_ERR_ARG;
+
+  if (N == 0) return CKDA_OK;
+  unsigned int *err = error_word_ptr();
+  cudaError_t e;
+  if (ckda::fwd_tc_supported(d_k, d_v, chunk, dt)) {
+    e = ckda::launch_fwd_tc(q, k, v, alpha, beta, initial_state, final_state, o,
+                            cu_seqlens, N, T, (int)T_total, H, scale, err,
+                            stream);
+  } else if (dt == CKDA_F32) {
+    e = ckda::launch_fwd_simt<float>(d_k, d_v, chunk, q, k, v, alpha, beta,
+                                     initial_state, final_state, o, cu_seqlens,
+                                     N, T, (int)T_total, H, scale, err, stream);
+  } else {
+    e = ckda::launch_fwd_simt<__nv_bfloat16>(
+        d_k, d_v, chunk, q, k, v, alpha, beta, initial_state, final_state, o,
+        cu_seqlens, N, T, (int)T_total, H, scale, err, stream);
+  }
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta,
+                             float *state, void *o, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, float scale,
+                             ckda_dtype dt, cudaStream_t stream) {
+  if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (N < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!q || !k || !v || !alpha || !beta || !state || !o) return CKDA_ERR_ARG;
+  const void *ptrs[] = {q, k, v, alpha, beta, state, o};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return CKDA_ERR_ARG;
+  const size_t es = esize(dt);
+  const size_t nh = (size_t)N * H;
+  const size_t ob = nh * d_v * es;
+  if (overlaps(o, ob, state, nh * d_k * d_v * sizeof(float)) ||
+      overlaps(o, ob, q, nh * d_k * es) || overlaps(o, ob, k, nh * d_k * es) ||
+      overlaps(o, ob, v, nh * d_v * es) ||
+      overlaps(o, ob, alpha, nh * d_k * sizeof(float)) ||
+      overlaps(o, ob, beta, nh * sizeof(float)))
+    return CKDA_ERR_ARG;
+  if (nh > 0x7fffffffu) return CKDA_ERR_ARG;
+  if (N == 0) return CKDA_OK;
+  cudaError_t e =
+      dt == CKDA_F32
+          ? ckda::launch_decode<float>(d_k, d_v, q, k, v, alpha, beta, state, o,
+                                       N, H, scale, stream)
+          : ckda::launch_decode<__nv_bfloat16>(d_k, d_v, q, k, v, alpha, beta,
+                                               state, o, N, H, scale, stream);
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+// Shared device helpers for the CKDA kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ckda {
+
+// Bits of the per-device error word (read and cleared by ckda_last_error).
+enum : unsigned int {
+  kErrBadSeqlens = 1u << 0,   // device cu_seqlens out of range / decreasing
+  kErrMbarTimeout = 1u << 1,  // a bounded mbarrier wait gave up
+  kErrTmemAlloc = 1u << 2,    // tensor-memory allocation returned garbage
+};
+
+// Kernels receive the device address of the per-device error word (defined
+// in ckda_api.cu) as an argument; nullptr disables reporting.
+__device__ __forceinline__ void flag_error(unsigned int *err, unsigned int bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// Element-type traits for q, k, v, o.
+template <typename T> struct IO;
+template <> struct IO<float> {
+  static __device__ __forceinline__ float ld(const float *p) { return *p; }
+  static __device__ __forceinline__ void st(float *p, float x) { *p = x; }
+  // 4 consecutive elements (16-byte aligned for float)
+  static __device__ __forceinline__ float4 ld4(const float *p) {
+    return *reinterpret_cast<const float4 *>(p);
+  }
+  static __device__ __forceinline__ void st4(float *p, float4 x) {
+    *reinterpret_cast<float4 *>(p) = x;
+  }
+};
+template <> struct IO<__nv_bfloat16> {
+  static __device__ __forceinline__ float ld(const __nv_bfloat16 *p) {
+    return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16 *p, float x) {
+    *p = __float2bfloat16_rn(x);
+  }
+  // 4 consecutive elements (8-byte aligned)
+  static __device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+    uint2 raw = *reinterpret_cast<const uint2 *>(p);
+    __nv_bfloat162 a = *reinterpret_cast<__nv_bfloat162 *>(&raw.x);
+    __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162 *>(&raw.y);
+    float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    return make_float4(fa.x, fa.y, fb.x, fb.y);
+  }
+  static __device__ __forceinline__ void st4(__nv_bfloat16 *p, float4 x) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(x.x, x.y);
+    __nv_bfloat162 b = __floats2bfloat162_rn(x.z, x.w);
+    uint2 raw;
+    raw.x = *reinterpret_cast<unsigned int *>(&a);
+    raw.y = *reinterpret_cast<unsigned int *>(&b);
+    *reinterpret_cast<uint2 *>(p) = raw;
+  }
+};
+
+// Sequence bounds for sequence n: [bos, eos). With cu == nullptr every
+// sequence has T tokens. A malformed device cu_seqlens entry flags an error
+// and yields an empty range, so no kernel ever indexes outside [0, T_total).
+__device__ __forceinline__ void seq_bounds(const int32_t *cu, int n, int T,
+                                           int T_total, unsigned int *err,
+                                           int &bos, int &eos) {
+  if (cu == nullptr) {
+    bos = n * T;
+    eos = bos + T;
+    return;
+  }
+  bos = __ldg(cu + n);
+  eos = __ldg(cu + n + 1);
+  if (bos < 0 || eos < bos || eos > T_total) {
+    bos = 0;
+    eos = 0;
+    flag_error(err, kErrBadSeqlens);
+  }
+}
+
+}  // namespace ckda

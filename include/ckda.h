@@ -1,0 +1,137 @@
+/*
+ * ckda.h: C ABI of the CKDA (Complex Kimi Delta Attention) CUDA library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (Semidirect Fourier Delta Attention, §1 eq. (1) and §2.2
+ * eq. (9); readout §3 eq. (14); value ranges from Complex KDA, abstract):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t        (the state after the update is read)
+ *
+ * per sequence and head, with a channel-wise gate alpha_t in [-1,1]^{d_k}
+ * (negative and exactly-zero gates allowed; KDA's (0,1) is a special case), a
+ * scalar beta_t in [0,2], and a d_k x d_v fp32 state carried across tokens.
+ * The library does not clamp or check the ranges of alpha and beta; values
+ * outside them are computed as given.
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor pointers are DEVICE pointers on the current CUDA device unless
+ *    a parameter says "host". The caller owns every buffer; the library never
+ *    allocates device memory and keeps no pointer after a call returns.
+ *  - Layouts are dense, row-major (C order), last dimension contiguous:
+ *      q, k     [T, H, d_k]     v, o      [T, H, d_v]
+ *      alpha    [T, H, d_k] fp32          beta      [T, H]  fp32
+ *      states   [N, H, d_k, d_v] fp32 (d_v contiguous)
+ *    q, k, v and o share one element type (ckda_dtype); alpha, beta and the
+ *    states are always fp32. Every pointer must be 16-byte aligned.
+ *  - Supported sizes: d_k, d_v in {16, 32, 64, 128}; H >= 1.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream). Argument
+ *    errors are detected on the host and returned before anything is
+ *    launched. Launch failures return CKDA_ERR_CUDA. Errors found by a kernel
+ *    (e.g. a malformed device-only cu_seqlens) are recorded in a per-device
+ *    error word and reported by ckda_last_error().
+ *  - Deterministic: no atomics in any reduction, so results are bitwise
+ *    reproducible run to run on the same GPU and arguments.
+ */
+#ifndef CKDA_H
+#define CKDA_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CKDA_OK = 0,
+  CKDA_ERR_ARG = 1,          /* null/misaligned pointer, bad size, bad cu_seqlens */
+  CKDA_ERR_UNSUPPORTED = 2,  /* d_k, d_v, chunk or dtype outside the supported set */
+  CKDA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+  CKDA_ERR_DEVICE = 4        /* a kernel flagged an error (see ckda_last_error) */
+} ckda_status;
+
+typedef enum {
+  CKDA_BF16 = 0,             /* q, k, v, o are bfloat16 */
+  CKDA_F32 = 1               /* q, k, v, o are float32 (fp32 check mode) */
+} ckda_dtype;
+
+/*
+ * ckda_fwd_chunked: chunkwise-parallel forward (prefill) of the recurrence
+ * over packed sequences.
+ *
+ * Chunking is an execution strategy only: inside each chunk of `chunk`
+ * tokens the kernels build the chunk's WY / UT-transform factors (the
+ * compact representation of the product of diagonal-plus-rank-one
+ * transitions and its triangular solve, Semidirect Fourier Delta Attention
+ * §2.2) and carry the state from chunk to chunk through the affine chunk
+ * transfer (§1, contribution 4); the results equal the token recurrence up to
+ * rounding ("chunkwise execution changes cost, never the numbers": Kimi Delta
+ * Attention: a bounded case study, Exercise 2).
+ *
+ * q, k          [T_total, H, d_k] (dt)      token-major, packed sequences
+ * v             [T_total, H, d_v] (dt)
+ * alpha         [T_total, H, d_k] fp32      channel-wise gate
+ * beta          [T_total, H]      fp32      delta coefficient
+ * initial_state [N, H, d_k, d_v]  fp32 or NULL (NULL = zero state)
+ * final_state   [N, H, d_k, d_v]  fp32 or NULL (NULL = not written); may be
+ *               the same buffer as initial_state (read before written)
+ * o             [T_total, H, d_v] (dt)      output; must not alias any input
+ * cu_seqlens    device int32 [N+1] or NULL. NULL: N sequences of T tokens
+ *               each (T_total = N*T). Otherwise sequence n owns tokens
+ *               [cu[n], cu[n+1]), with cu[0]=0, non-decreasing, cu[N]=T and
+ *               T = T_total. Zero-length sequences are allowed (their final
+ *               state equals their initial state).
+ * cu_seqlens_host optional host copy of cu_seqlens (may be NULL). When given
+ *               it is validated on the host (CKDA_ERR_ARG if malformed).
+ *               When NULL the kernels validate the device copy and record
+ *               CKDA_ERR_DEVICE (skipping the bad sequence) instead.
+ * N, T, H, d_k, d_v  sizes as above (N >= 0, T >= 0).
+ * chunk         chunk length: 0 (default 64), 16, 32 or 64.
+ * scale         multiplies every output (o_t = scale * S_t^T q_t).
+ * dt            element type of q, k, v and o.
+ */
+ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta,
+                             const float *initial_state, float *final_state,
+                             void *o, const int32_t *cu_seqlens,
+                             const int32_t *cu_seqlens_host, int32_t N,
+                             int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                             int32_t chunk, float scale, ckda_dtype dt,
+                             cudaStream_t stream);
+
+/*
+ * ckda_decode_step: one recurrent step for N sequences x H heads, one new
+ * token each, updating the state in place (the recurrence above applied once;
+ * Semidirect Fourier Delta Attention §1 eq. (1), readout §3 eq. (14)).
+ *
+ * q, k   [N, H, d_k] (dt)      v, o [N, H, d_v] (dt)
+ * alpha  [N, H, d_k] fp32      beta [N, H] fp32
+ * state  [N, H, d_k, d_v] fp32, read and written in place
+ * o      must not alias state or any input.
+ */
+ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta,
+                             float *state, void *o, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, float scale,
+                             ckda_dtype dt, cudaStream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *ckda_status_string(ckda_status s);
+
+/*
+ * ckda_last_error: synchronises `stream`, then reads and clears the current
+ * device's error word. Returns CKDA_OK if no kernel recorded an error since
+ * the last call, CKDA_ERR_DEVICE if one did, CKDA_ERR_CUDA if the
+ * synchronisation or the read failed.
+ */
+ckda_status ckda_last_error(cudaStream_t stream);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int32_t ckda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKDA_H */

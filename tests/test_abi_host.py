@@ -1,0 +1,129 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+include/ckda.h declares, and rejects bad arguments before any launch.
+
+No GPU: every call below fails host-side validation, so nothing is launched
+and no device pointer is ever dereferenced (the fake pointers are never
+reached by a kernel).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_114_b200 import build as ckda_build
+from gated_delta_rule_114_b200 import ckda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ckda.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ckda_build.build()
+    return ckda.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ckda_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_status_string",
+                 "ckda_last_error", "ckda_version"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert lib.ckda_status_string(s).decode().startswith("CKDA_")
+    assert b"UNKNOWN" in lib.ckda_status_string(99)
+    assert lib.ckda_version() >= 100
+
+
+# fake, 16-byte aligned, never dereferenced: every call fails validation first
+P = ctypes.c_void_p(0x10000)
+P2 = ctypes.c_void_p(0x20000)
+P3 = ctypes.c_void_p(0x30000)
+P4 = ctypes.c_void_p(0x40000)
+P5 = ctypes.c_void_p(0x50000)
+P6 = ctypes.c_void_p(0x60000)
+ODD = ctypes.c_void_p(0x10004)
+NULL = None
+
+
+def fwd(lib, q=P, k=P2, v=P3, a=P4, b=P5, s0=NULL, sf=NULL, o=P6, cu=NULL,
+        cuh=NULL, N=1, T=8, H=1, dk=16, dv=16, chunk=0, dt=ckda.CKDA_F32):
+    return lib.ckda_fwd_chunked(q, k, v, a, b, s0, sf, o, cu, cuh, N, T, H, dk,
+                                dv, chunk, 1.0, dt, None)
+
+
+def dec(lib, q=P, k=P2, v=P3, a=P4, b=P5, s=P6, o=ctypes.c_void_p(0x70000),
+        N=1, H=1, dk=16, dv=16, dt=ckda.CKDA_F32):
+    return lib.ckda_decode_step(q, k, v, a, b, s, o, N, H, dk, dv, 1.0, dt, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=NULL), ckda.CKDA_ERR_ARG),
+    (dict(o=NULL), ckda.CKDA_ERR_ARG),
+    (dict(b=NULL), ckda.CKDA_ERR_ARG),
+    (dict(q=ODD), ckda.CKDA_ERR_ARG),
+    (dict(H=0), ckda.CKDA_ERR_ARG),
+    (dict(N=-1), ckda.CKDA_ERR_ARG),
+    (dict(T=-5), ckda.CKDA_ERR_ARG),
+    (dict(dk=48), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(dv=256), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(chunk=24), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(dt=7), ckda.CKDA_ERR_UNSUPPORTED),
+    # output aliasing an input
+    (dict(o=P), ckda.CKDA_ERR_ARG),
+    # host cu_seqlens without a device copy
+    (dict(cuh=ctypes.cast((ctypes.c_int32 * 2)(0, 8), ctypes.c_void_p)),
+     ckda.CKDA_ERR_ARG),
+])
+def test_fwd_rejects(lib, kw, want):
+    assert fwd(lib, **kw) == want
+
+
+@pytest.mark.parametrize("cu_host", [(1, 8), (0, 9), (0, 5, 3, 8)])
+def test_fwd_rejects_bad_host_seqlens(lib, cu_host):
+    arr = (ctypes.c_int32 * len(cu_host))(*cu_host)
+    st = fwd(lib, cu=P, cuh=ctypes.cast(arr, ctypes.c_void_p),
+             N=len(cu_host) - 1, T=8, q=P2, k=P3, v=P4, a=P5, b=P6,
+             o=ctypes.c_void_p(0x70000))
+    assert st == ckda.CKDA_ERR_ARG
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(s=NULL), ckda.CKDA_ERR_ARG),
+    (dict(o=P6), ckda.CKDA_ERR_ARG),  # o aliases the state
+    (dict(a=ODD), ckda.CKDA_ERR_ARG),
+    (dict(H=0), ckda.CKDA_ERR_ARG),
+    (dict(N=-2), ckda.CKDA_ERR_ARG),
+    (dict(dk=8), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(dt=3), ckda.CKDA_ERR_UNSUPPORTED),
+])
+def test_decode_rejects(lib, kw, want):
+    assert dec(lib, **kw) == want
+
+
+def test_python_binding_requires_cuda_tensors(lib):
+    import torch
+    x = torch.zeros(4, 1, 16)
+    with pytest.raises(ValueError):
+        ckda.ckda_fwd_chunked(x, x, x, x, torch.zeros(4, 1), None, None, x,
+                              N=1, T=4)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    monkeypatch.setattr(ckda, "_lib", None)
+    with pytest.raises(RuntimeError):
+        ckda.load(str(tmp_path / "nope.so"))

@@ -1,0 +1,295 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Every test here runs the kernels on cuda:0 and compares element by element
+with the oracle on the same seeded inputs, within the tolerances of
+parity_util (1e-5 rms in the fp32 check mode; 1e-2 rms plus the bf16 store
+rounding in bf16 mode).
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_114_b200 import ckda
+from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,
+                                              make_decode_tokens,
+                                              make_fwd_inputs, seqlens)
+from parity_util import as_f64, check_bf16_out, check_close, check_fp32, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_fwd(inp, chunk=0, scale=1.0, init=True, host_cu=True, cu=True):
+    d = to_dev(inp)
+    s0 = d["initial_state"] if init else None
+    cu_d = d["cu_seqlens"] if cu else None
+    N = inp["cu_seqlens"].numel() - 1
+    T_total = inp["q"].shape[0]
+    o, sf = ckda.fwd_chunked(
+        d["q"], d["k"], d["v"], d["alpha"], d["beta"], s0, cu_seqlens=cu_d,
+        cu_seqlens_host=inp["cu_seqlens"] if (cu and host_cu) else None,
+        N=None if cu else N, T=None if cu else T_total // max(N, 1),
+        chunk=chunk, scale=scale)
+    torch.cuda.synchronize()
+    assert ckda.ckda_last_error() == ckda.CKDA_OK
+    return o, sf
+
+
+def ref_fwd(inp, scale=1.0, init=True):
+    return oracle.fwd(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                      inp["initial_state"] if init else None,
+                      inp["cu_seqlens"], scale)
+
+
+def custom(base, **kw):
+    return dataclasses.replace(WORKLOADS[base], **kw)
+
+
+def lens_cu(lens):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return torch.from_numpy(cu)
+
+
+# ------------------------------------------------------------ fp32 check mode
+
+def test_tiny_config_fp32(cuda_lib):
+    """B=1, H=1, T=64, d=16, chunk 16, fp32: o and final state to 1e-5 rms."""
+    w = WORKLOADS["tiny_T64_d16_f32"]
+    inp = make_fwd_inputs(w)
+    inp["initial_state"] = None
+    o, sf = run_fwd(inp, chunk=w.chunk, init=False)
+    o_ref, sf_ref = ref_fwd(inp, init=False)
+    check_fp32(o, o_ref, "o")
+    check_fp32(sf, sf_ref, "final_state")
+
+
+@pytest.mark.parametrize("d_k,d_v", [(16, 16), (32, 64), (64, 32), (128, 128),
+                                     (128, 16), (16, 128)])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_fp32_shapes_and_ragged_varlen(cuda_lib, d_k, d_v, chunk):
+    """Several tiles and a ragged tail per sequence; zero-length and 1-token
+    sequences; CKDA gates with exact +-1 and 0; random initial states."""
+    w = custom("ckda_B1_H32_T8192_d128", d_k=d_k, d_v=d_v, dtype="f32",
+               seed=5000 + d_k + 3 * d_v + chunk)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([0, 1, chunk - 1, chunk,
+                                                 3 * chunk + 5, 0, 2 * chunk + 1]),
+                          H=3)
+    o, sf = run_fwd(inp, chunk=chunk, scale=0.75)
+    o_ref, sf_ref = ref_fwd(inp, scale=0.75)
+    check_fp32(o, o_ref, "o")
+    check_fp32(sf, sf_ref, "final_state")
+
+
+def test_fp32_long_sequence(cuda_lib):
+    """One 1000-token sequence (15 full chunks + a ragged tail), d=128."""
+    w = custom("ckda_B1_H32_T8192_d128", dtype="f32", seed=777)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([1000]), H=2)
+    o, sf = run_fwd(inp)
+    o_ref, sf_ref = ref_fwd(inp)
+    check_fp32(o, o_ref, "o")
+    check_fp32(sf, sf_ref, "final_state")
+
+
+@pytest.mark.parametrize("kind", ["zero", "sign", "orthogonal"])
+def test_fp32_degenerate_gates(cuda_lib, kind):
+    """All-zero gates; all -1 gates with beta = 0; |alpha| = 1 random signs
+    with beta in {0, 2} (orthogonal transitions)."""
+    w = custom("ckda_B1_H32_T8192_d128", d_k=64, d_v=64, dtype="f32", seed=31)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([150, 70]), H=2)
+    g = torch.Generator().manual_seed(3)
+    if kind == "zero":
+        inp["alpha"].zero_()
+    elif kind == "sign":
+        inp["alpha"].fill_(-1.0)
+        inp["beta"].zero_()
+    else:
+        inp["alpha"] = torch.where(torch.rand(inp["alpha"].shape, generator=g) < 0.5,
+                                   -1.0, 1.0).float()
+        inp["beta"] = torch.where(torch.rand(inp["beta"].shape, generator=g) < 0.5,
+                                  0.0, 2.0).float()
+    o, sf = run_fwd(inp)
+    o_ref, sf_ref = ref_fwd(inp)
+    check_fp32(o, o_ref, "o")
+    check_fp32(sf, sf_ref, "final_state")
+
+
+def test_fp32_equal_length_without_cu_seqlens(cuda_lib):
+    w = custom("kda_B4_H16_T2048_d128", dtype="f32", seed=91)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([200, 200, 200]), H=2)
+    inp["initial_state"] = None
+    o, sf = run_fwd(inp, init=False, cu=False)
+    o_ref, sf_ref = ref_fwd(inp, init=False)
+    check_fp32(o, o_ref, "o")
+    check_fp32(sf, sf_ref, "final_state")
+
+
+# ------------------------------------------------------------ bf16 workloads
+
+def test_kda_range_prefill_full(cuda_lib):
+    """B=4, H=16, T=2048, d=128, KDA ranges, zero initial state (full size)."""
+    w = WORKLOADS["kda_B4_H16_T2048_d128"]
+    inp = make_fwd_inputs(w)
+    o, sf = run_fwd(inp, chunk=w.chunk, init=False)
+    o_ref, sf_ref = ref_fwd(inp, init=False)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
+def test_ckda_long_prefill_full(cuda_lib):
+    """B=1, H=32, T=8192, d=128, CKDA ranges with exact +-1 / 0 gates and a
+    random initial state (full size, every output compared)."""
+    w = WORKLOADS["ckda_B1_H32_T8192_d128"]
+    inp = make_fwd_inputs(w)
+    o, sf = run_fwd(inp, chunk=w.chunk)
+    o_ref, sf_ref = ref_fwd(inp)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
+def test_ckda_varlen_full_sampled(cuda_lib):
+    """32 packed sequences, U[128,4096] tokens, H=32 at full size on the GPU;
+    the oracle recomputes a seeded sample of 6 sequences (all heads),
+    including the longest and the shortest."""
+    w = WORKLOADS["ckda_varlen_N32_H32_d128"]
+    inp = make_fwd_inputs(w)
+    o, sf = run_fwd(inp, chunk=w.chunk)
+    cu = inp["cu_seqlens"].numpy()
+    lens = np.diff(cu)
+    rng = np.random.default_rng(4)
+    pick = sorted(set([int(lens.argmax()), int(lens.argmin())] +
+                      list(rng.choice(len(lens), 4, replace=False))))
+    sub_rows = np.concatenate([np.arange(cu[n], cu[n + 1]) for n in pick])
+    sub = {key: inp[key][sub_rows] for key in ("q", "k", "v", "alpha", "beta")}
+    sub["initial_state"] = inp["initial_state"][pick]
+    sub["cu_seqlens"] = lens_cu(lens[pick])
+    o_ref, sf_ref = ref_fwd(sub)
+    check_bf16_out(o.cpu()[torch.from_numpy(sub_rows)], o_ref)
+    check_close(sf.cpu()[pick], sf_ref, 1e-2, 0.0, "final_state")
+
+
+def test_bf16_ragged_small(cuda_lib):
+    """bf16 path on ragged lengths (partial chunks, empty and 1-token
+    sequences), scale != 1."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=4242)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([0, 1, 63, 64, 65, 200, 0, 130]),
+                          H=4)
+    o, sf = run_fwd(inp, chunk=64, scale=1.5)
+    o_ref, sf_ref = ref_fwd(inp, scale=1.5)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
+def test_split_resume_equals_single_call(cuda_lib):
+    """fwd(x[:a]) then fwd(x[a:], init = final) equals fwd(x): the state is
+    the checkpoint (chunk-to-chunk carry). fp32 mode, split mid-chunk."""
+    w = custom("ckda_B1_H32_T8192_d128", dtype="f32", seed=99)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([300]), H=2)
+    o, sf = run_fwd(inp)
+    a = 137
+    first = {key: inp[key][:a] for key in ("q", "k", "v", "alpha", "beta")}
+    first.update(initial_state=inp["initial_state"], cu_seqlens=lens_cu([a]))
+    o1, sf1 = run_fwd(first)
+    second = {key: inp[key][a:] for key in ("q", "k", "v", "alpha", "beta")}
+    second.update(initial_state=sf1.cpu(), cu_seqlens=lens_cu([300 - a]))
+    o2, sf2 = run_fwd(second)
+    check_fp32(torch.cat([o1, o2]).cpu(), as_f64(o), "o")
+    check_fp32(sf2, as_f64(sf), "final_state")
+
+
+def test_final_state_in_place_and_deterministic(cuda_lib):
+    """final_state may alias initial_state; two identical calls agree bitwise."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=5)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([100, 260]), H=2)
+    d = to_dev(inp)
+    o1, sf1 = ckda.fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                               d["initial_state"], d["cu_seqlens"])
+    o2, sf2 = ckda.fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                               d["initial_state"], d["cu_seqlens"])
+    assert torch.equal(o1, o2) and torch.equal(sf1, sf2)
+    s = d["initial_state"].clone()
+    o3 = torch.empty_like(o1)
+    ckda.ckda_fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"], s, s,
+                          o3, d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert torch.equal(o3, o1) and torch.equal(s, sf1)
+
+
+def test_device_seqlens_error_is_reported(cuda_lib):
+    """A malformed device cu_seqlens (no host copy) is clamped in the kernel
+    (no out-of-range access) and reported by ckda_last_error."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=6)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([40, 40]), H=1)
+    d = to_dev(inp)
+    assert ckda.ckda_last_error() == ckda.CKDA_OK
+    bad = torch.tensor([0, 50, 30], dtype=torch.int32, device="cuda")
+    o = torch.zeros_like(d["v"])
+    ckda.ckda_fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"], None,
+                          None, o, bad)
+    assert ckda.ckda_last_error() == ckda.CKDA_ERR_DEVICE
+    assert ckda.ckda_last_error() == ckda.CKDA_OK  # cleared by the read
+
+
+# ------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("d_k,d_v,dtype", [(16, 16, "f32"), (64, 128, "f32"),
+                                           (128, 32, "f32"), (128, 128, "bf16")])
+def test_decode_small(cuda_lib, d_k, d_v, dtype):
+    """20 decode steps on 5 x 3 (sequence, head) pairs, every pair checked."""
+    w = custom("decode_N256_H32_d128", d_k=d_k, d_v=d_v, dtype=dtype, seed=2000 + d_k)
+    N, H = 5, 3
+    state = make_decode_state(w, N=N, H=H)
+    st_ref = state.double().numpy().copy()
+    st_dev = state.cuda()
+    for step in range(20):
+        tok = make_decode_tokens(w, step, N=N, H=H)
+        d = to_dev(tok)
+        o = ckda.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                             st_dev, scale=0.9)
+        o_ref = oracle.decode(tok["q"], tok["k"], tok["v"], tok["alpha"],
+                              tok["beta"], st_ref, scale=0.9)
+        if dtype == "f32":
+            check_fp32(o, o_ref, "o step %d" % step)
+        else:
+            check_bf16_out(o, o_ref, "o step %d" % step)
+    if dtype == "f32":
+        check_fp32(st_dev, st_ref, "state")
+    else:
+        check_close(st_dev, st_ref, 1e-2, 0.0, "state")
+
+
+def test_decode_workload_1000_steps(cuda_lib):
+    """256 sequences x 32 heads, d=128, bf16 tokens, fp32 state, 1000
+    consecutive steps with fresh tokens. Every pair is checked after step 1;
+    a seeded sample of 256 pairs is stepped in lockstep by the oracle and
+    checked at every step (o) and after steps 1, 10, 100, 1000 (state)."""
+    w = WORKLOADS["decode_N256_H32_d128"]
+    N, H = w.B, w.H
+    state = make_decode_state(w)
+    st_dev = state.cuda()
+    rng = np.random.default_rng(12)
+    pairs = np.sort(rng.choice(N * H, 256, replace=False)).astype(np.int64)
+    st_ref = state.reshape(N * H, w.d_k, w.d_v)[torch.from_numpy(pairs)].double().numpy().copy()
+    full_ref = None
+    pidx = torch.from_numpy(pairs).cuda()
+    for step in range(1000):
+        tok = make_decode_tokens(w, step)
+        d = to_dev(tok)
+        if step == 0:
+            full_ref = state.double().numpy().copy()
+            o_full_ref = oracle.decode(tok["q"], tok["k"], tok["v"],
+                                       tok["alpha"], tok["beta"], full_ref)
+        o = ckda.decode_step(d["q"], d["k"], d["v"], d["alpha"], d["beta"], st_dev)
+        sub = {key: val.reshape(N * H, *val.shape[2:])[torch.from_numpy(pairs)]
+               .unsqueeze(1) for key, val in tok.items()}
+        o_ref = oracle.decode(sub["q"], sub["k"], sub["v"], sub["alpha"],
+                              sub["beta"], st_ref.reshape(256, 1, w.d_k, w.d_v))
+        o_sub = o.reshape(N * H, w.d_v)[pidx]
+        check_bf16_out(o_sub.unsqueeze(1), o_ref, "o step %d" % step)
+        if step == 0:
+            check_bf16_out(o, o_full_ref, "o step 0 (all pairs)")
+            check_close(st_dev, full_ref, 1e-2, 0.0, "state step 1 (all pairs)")
+        if step + 1 in (1, 10, 100, 1000):
+            s_sub = st_dev.reshape(N * H, w.d_k, w.d_v)[pidx]
+            check_close(s_sub, st_ref, 1e-2, 0.0, "state after %d" % (step + 1))
