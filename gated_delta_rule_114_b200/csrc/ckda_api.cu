@@ -21,7 +21,7 @@ cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
                             int T_total, int H, float scale, unsigned int *err,
                             cudaStream_t st);
 bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt);
-cudaError_t launch_fwd_tc(const void *q, const void *k, const void *v,
+cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
                           const float *alpha, const float *beta,
                           const float *s0, float *sf, void *o,
                           const int32_t *cu, int N, int T, int T_total, int H,
@@ -148,7 +148,7 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
   unsigned int *err = error_word_ptr();
   cudaError_t e;
   if (ckda::fwd_tc_supported(d_k, d_v, chunk, dt)) {
-    e = ckda::launch_fwd_tc(q, k, v, alpha, beta, initial_state, final_state, o,
+    e = ckda::launch_fwd_tc(d_v, q, k, v, alpha, beta, initial_state, final_state, o,
                             cu_seqlens, N, T, (int)T_total, H, scale, err,
                             stream);
   } else if (dt == CKDA_F32) {
