@@ -56,18 +56,21 @@ constexpr int AS = 65;     // fp32 row stride of A, M, T
 constexpr uint32_t OFF_GA = 0;        // 49152 Lk/Lq (96 rows x 128, K-major sw128)
                                       //       -> [beta Khat | beta V] (N160 x K64 MN-sw128b32)
 constexpr uint32_t OFF_GB = 49152;    // 49152 R stack (96 rows x 128, K-major sw128)
-                                      //       -> solve scratch
+                                      //       -> [M ; I] (128 x 64 K-major) + T operand
+constexpr uint32_t OFF_A0 = OFF_GB;           // 32768 [M ; I], A of D0
+constexpr uint32_t OFF_B0 = OFF_GB + 32768;   // 16384 T, B of D0 (K64 x N64 MN-sw128b32)
 constexpr uint32_t OFF_SB = 98304;    // 16384 S, B of D1 (K128 x N32 MN-sw128b32)
 constexpr uint32_t OFF_UB = 114688;   //  8192 U, B of D2 (K64 x N32 MN-sw128b32)
 constexpr uint32_t OFF_Q = 122880;    // 16384 raw q bf16 [64][128] -> T fp32 [64][65]
 constexpr uint32_t OFF_K = 139264;    // 16384 raw k bf16 [64][128]    (T spills in)
+constexpr uint32_t OFF_XT = OFF_K + 4096;     //  3072 solve scratch (after raw k is dead)
 constexpr uint32_t OFF_AL = 155648;   // 33792 alpha fp32 [64][132] -> Qhat fp32
 constexpr uint32_t OFF_V = 189440;    //  4096 raw v bf16 [64][32]
 constexpr uint32_t OFF_A = 193536;    // 16640 A fp32 [64][65]
 constexpr uint32_t OFF_M = 210176;    // 16640 M fp32 [64][65]
 constexpr uint32_t OFF_B = 226816;    //   256 beta
 constexpr uint32_t OFF_GC = 227072;   //   512 gamma over the chunk
-constexpr uint32_t OFF_BAR = 227584;  //    64 mbarriers + TMEM address + flags
+constexpr uint32_t OFF_BAR = 227584;  //    64 mbarriers [0..4] + TMEM address + flags
 constexpr uint32_t SMEM_USED = 227648;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
 
@@ -82,6 +85,7 @@ constexpr uint32_t TM_D2 = 416;   //  32
 constexpr uint32_t TM_COLS = 512;
 
 constexpr uint32_t ID_G = idesc_tf32(128, 96, 0, 0);
+constexpr uint32_t ID_D0 = idesc_tf32(128, 64, 0, 1);
 constexpr uint32_t ID_D5 = idesc_tf32(128, 160, 0, 1);
 constexpr uint32_t ID_D1 = idesc_tf32(128, 32, 0, 1);
 constexpr uint32_t ID_D2 = idesc_tf32(128, 32, 0, 1);
@@ -123,12 +127,12 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
   float *sA = reinterpret_cast<float *>(sm + OFF_A);
   float *sM = reinterpret_cast<float *>(sm + OFF_M);
   float *sT = reinterpret_cast<float *>(sm + OFF_Q);
-  float *sXT = reinterpret_cast<float *>(sm + OFF_GB);
+  float *sXT = reinterpret_cast<float *>(sm + OFF_XT);
   float *sB = reinterpret_cast<float *>(sm + OFF_B);
   float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [0..3]
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 32);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + OFF_BAR + 36);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [0..4]
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 48);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + OFF_BAR + 52);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vt = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
@@ -142,7 +146,7 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
+    for (int i = 0; i < 5; ++i) mbar_init(&bar[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -169,53 +173,107 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
 
   for (int t0 = bos; t0 < eos; t0 += C, phase ^= 1u) {
     const int L = min(C, eos - t0);
-    // ---------------- 1. load the chunk
-    for (int idx = tid; idx < C * 16; idx += NT) {  // q, k: 16-byte pieces
-      const int i = idx >> 4, ch = idx & 15;
-      uint4 qv = make_uint4(0, 0, 0, 0), kv = qv;
-      if (i < L) {
-        const size_t off = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
-        qv = *reinterpret_cast<const uint4 *>(q + off);
-        kv = *reinterpret_cast<const uint4 *>(k + off);
+    // ---------------- 1. load the chunk: all global loads in flight at once
+    {
+      uint4 qv[4], kv[4], vv;
+      float4 av[8];
+      float bv = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // q, k: 64 rows x 16 pieces of 16 bytes
+        const int idx = tid + u * NT, i = idx >> 4, ch = idx & 15;
+        qv[u] = kv[u] = make_uint4(0, 0, 0, 0);
+        if (i < L) {
+          const size_t off = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
+          qv[u] = __ldg(reinterpret_cast<const uint4 *>(q + off));
+          kv[u] = __ldg(reinterpret_cast<const uint4 *>(k + off));
+        }
       }
-      *reinterpret_cast<uint4 *>(sm + OFF_Q + i * 256 + ch * 16) = qv;
-      *reinterpret_cast<uint4 *>(sm + OFF_K + i * 256 + ch * 16) = kv;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {  // alpha: 64 rows x 32 float4
+        const int idx = tid + u * NT, i = idx >> 5, c4 = (idx & 31) * 4;
+        av[u] = make_float4(1.f, 1.f, 1.f, 1.f);
+        if (i < L)
+          av[u] = __ldg(reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4));
+      }
+      {  // v tile: 64 rows x 64 bytes
+        const int i = tid >> 2, ch = tid & 3;
+        vv = make_uint4(0, 0, 0, 0);
+        if (i < L) vv = __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + i) * H + h) * DV + c0 + ch * 8));
+      }
+      if (tid < L) bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int idx = tid + u * NT, i = idx >> 4, ch = idx & 15;
+        *reinterpret_cast<uint4 *>(sm + OFF_Q + i * 256 + ch * 16) = qv[u];
+        *reinterpret_cast<uint4 *>(sm + OFF_K + i * 256 + ch * 16) = kv[u];
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int idx = tid + u * NT, i = idx >> 5, c4 = (idx & 31) * 4;
+        *reinterpret_cast<float4 *>(sAl + i * AL_S + c4) = av[u];
+      }
+      *reinterpret_cast<uint4 *>(sm + OFF_V + (tid >> 2) * 64 + (tid & 3) * 16) = vv;
+      if (tid < C) sB[tid] = bv;
     }
-    for (int idx = tid; idx < C * 32; idx += NT) {  // alpha: float4 pieces
-      const int i = idx >> 5, c4 = (idx & 31) * 4;
-      float4 av = make_float4(1.f, 1.f, 1.f, 1.f);
-      if (i < L) av = *reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4);
-      *reinterpret_cast<float4 *>(sAl + i * AL_S + c4) = av;
+    if (tid < C && t0 + C + tid < eos) {  // next chunk's rows into L2
+      const size_t th = (size_t)(t0 + C + tid) * H + h;
+      prefetch_l2(q + th * DK, DK * 2);
+      prefetch_l2(k + th * DK, DK * 2);
+      prefetch_l2(alpha + th * DK, DK * 4);
+      prefetch_l2(v + th * DV + c0, DVT * 2);
     }
-    {  // v tile: 64 rows x 64 bytes
-      const int i = tid >> 2, ch = tid & 3;
-      uint4 vv = make_uint4(0, 0, 0, 0);
-      if (i < L) vv = *reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + i) * H + h) * DV + c0 + ch * 8);
-      *reinterpret_cast<uint4 *>(sm + OFF_V + i * 64 + ch * 16) = vv;
-    }
-    if (tid < C) sB[tid] = (tid < L) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
     __syncthreads();
 
     // ---------------- 2. Gram operands (tf32, K-major 128B swizzle, 96 rows)
+    // Each thread owns one channel; a sub-block's 16 rows are read into
+    // registers before the running product walks them.
     if (tid < DK) {
       const int c = tid;
+#pragma unroll 1
       for (int I = 1; I < 4; ++I) {
-        float g = 1.f;
+        float a[16], kk_[16], qq[16];
+#pragma unroll
         for (int ii = 0; ii < 16; ++ii) {
           const int i = 16 * I + ii;
-          g *= sAl[i * AL_S + c];
-          st_f32(GA + off_k_sw128_f32((I - 1) * 32 + ii, c, 96), g * bf(sKr + i * DK + c));
-          st_f32(GA + off_k_sw128_f32((I - 1) * 32 + 16 + ii, c, 96), g * bf(sQr + i * DK + c));
+          a[ii] = sAl[i * AL_S + c];
+          kk_[ii] = bf(sKr + i * DK + c);
+          qq[ii] = bf(sQr + i * DK + c);
+        }
+        float g = 1.f;
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) {
+          g *= a[ii];
+          st_f32(GA + off_k_sw128_f32((I - 1) * 32 + ii, c, 96), g * kk_[ii]);
+          st_f32(GA + off_k_sw128_f32((I - 1) * 32 + 16 + ii, c, 96), g * qq[ii]);
         }
       }
     } else {
+      // R^(I)_j = k_j G_{16I-1<-j}: one backward sweep over j = 47..0 carries
+      // the three running products (each starts at its own 16I-1)
       const int c = tid - DK;
-      for (int I = 1; I < 4; ++I) {
-        const int off = 8 * I * (I - 1);
-        float g = 1.f;
-        for (int j = 16 * I - 1; j >= 0; --j) {
-          st_f32(GB + off_k_sw128_f32(off + j, c, 96), g * bf(sKr + j * DK + c));
-          g *= sAl[j * AL_S + c];
+      float g1 = 1.f, g2 = 1.f, g3 = 1.f;
+#pragma unroll 1
+      for (int b = 2; b >= 0; --b) {
+        float a[16], kk_[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int j = 16 * b + u;
+          a[u] = sAl[j * AL_S + c];
+          kk_[u] = bf(sKr + j * DK + c);
+        }
+#pragma unroll
+        for (int u = 15; u >= 0; --u) {
+          const int j = 16 * b + u;
+          st_f32(GB + off_k_sw128_f32(48 + j, c, 96), g3 * kk_[u]);
+          g3 *= a[u];
+          if (b <= 1) {
+            st_f32(GB + off_k_sw128_f32(16 + j, c, 96), g2 * kk_[u]);
+            g2 *= a[u];
+          }
+          if (b == 0) {
+            st_f32(GB + off_k_sw128_f32(j, c, 96), g1 * kk_[u]);
+            g1 *= a[u];
+          }
         }
       }
     }
@@ -231,39 +289,73 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
                     desc_k_sw128_f32(sb + OFF_GB, 96, kk), ID_G, kk > 0);
       mma_commit(&bar[0]);
     }
-    // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile
+    // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile: thread (column
+    // j, lane sl) runs the gate product over channels 8 sl .. 8 sl + 7; the 16
+    // lanes of a half-warp are then reduced with a reduce-scatter butterfly
+    // that leaves entries 2 sl, 2 sl + 1 of [A column | M column] in lane sl.
     for (int I = 0; I < 4; ++I) {
       const int r0 = 16 * I;
-      const int j = tid >> 4, sl = tid & 15;
-      float accA[16], accM[16];
+      const int j = tid >> 4, sl = tid & 15, c8 = 8 * sl;
+      float vv[32];
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) accA[ii] = accM[ii] = 0.f;
-      for (int c = sl; c < DK; c += 16) {
-        const float kj = bf(sKr + (r0 + j) * DK + c);
-        float g = 1.f;
+      for (int e = 0; e < 32; ++e) vv[e] = 0.f;
+      float kj[8], g[8];
+      {
+        const uint4 raw = *reinterpret_cast<const uint4 *>(sKr + (r0 + j) * DK + c8);
+        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          if (ii >= j) {
-            if (ii > j) g *= sAl[(r0 + ii) * AL_S + c];
-            const float x = g * kj;
-            accA[ii] += bf(sKr + (r0 + ii) * DK + c) * x;
-            accM[ii] += bf(sQr + (r0 + ii) * DK + c) * x;
-          }
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(p2[e]);
+          kj[2 * e] = f.x;
+          kj[2 * e + 1] = f.y;
         }
       }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = 1.f;
 #pragma unroll
       for (int ii = 0; ii < 16; ++ii) {
+        if (ii >= j) {
+          const float4 a0 = *reinterpret_cast<const float4 *>(sAl + (r0 + ii) * AL_S + c8);
+          const float4 a1 = *reinterpret_cast<const float4 *>(sAl + (r0 + ii) * AL_S + c8 + 4);
+          const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + (r0 + ii) * DK + c8);
+          const uint4 qr = *reinterpret_cast<const uint4 *>(sQr + (r0 + ii) * DK + c8);
+          const float al[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
+          const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
+          float sa = 0.f, sq = 0.f;
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) {
-          accA[ii] += __shfl_xor_sync(0xffffffffu, accA[ii], off);
-          accM[ii] += __shfl_xor_sync(0xffffffffu, accM[ii], off);
+          for (int e = 0; e < 4; ++e) {
+            const float2 kf = __bfloat1622float2(k2[e]), qf = __bfloat1622float2(q2[e]);
+            if (ii > j) {
+              g[2 * e] *= al[2 * e];
+              g[2 * e + 1] *= al[2 * e + 1];
+            }
+            const float x0 = g[2 * e] * kj[2 * e], x1 = g[2 * e + 1] * kj[2 * e + 1];
+            sa += kf.x * x0 + kf.y * x1;
+            sq += qf.x * x0 + qf.y * x1;
+          }
+          vv[ii] += sa;
+          vv[16 + ii] += sq;
         }
       }
-      if (sl == 0) {
+      // reduce-scatter over the 16 lanes sharing column j
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          if (ii > j) sA[(r0 + ii) * AS + r0 + j] = sB[r0 + ii] * accA[ii];
-          if (ii >= j) sM[(r0 + ii) * AS + r0 + j] = accM[ii];
+      for (int m = 8, n = 32; m > 0; m >>= 1, n >>= 1) {
+        const bool up = (sl & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+          const float keep = up ? vv[n / 2 + i] : vv[i];
+          const float send = up ? vv[i] : vv[n / 2 + i];
+          vv[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int idx = 2 * sl + e, ii = idx & 15;
+        if (idx >= 16) {
+          if (ii >= j) sM[(r0 + ii) * AS + r0 + j] = vv[e];
+        } else if (ii > j) {
+          sA[(r0 + ii) * AS + r0 + j] = sB[r0 + ii] * vv[e];
         }
       }
     }
@@ -292,22 +384,43 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
       float kb0[32], kb1[32];
       float g = 1.f;
 #pragma unroll
-      for (int j = C - 1; j >= 32; --j) {  // sigma_j = prod_{s>j} alpha_s
-        kb1[j - 32] = to_tf32(g * bf(sKr + j * DK + c));
-        g *= sAl[j * AL_S + c];
-      }
+      for (int b = 3; b >= 0; --b) {  // sigma_j = prod_{s>j} alpha_s, j = 63..0
+        float a[16], kk_[16];
 #pragma unroll
-      for (int j = 31; j >= 0; --j) {
-        kb0[j] = to_tf32(g * bf(sKr + j * DK + c));
-        g *= sAl[j * AL_S + c];
+        for (int u = 0; u < 16; ++u) {
+          a[u] = sAl[(16 * b + u) * AL_S + c];
+          kk_[u] = bf(sKr + (16 * b + u) * DK + c);
+        }
+#pragma unroll
+        for (int u = 15; u >= 0; --u) {
+          const int j = 16 * b + u;
+          const float x = to_tf32(g * kk_[u]);
+          if (j >= 32) kb1[j - 32] = x;
+          else kb0[j] = x;
+          g *= a[u];
+        }
       }
       tmem_st32(tm + lane_base + TM_AD2, kb0);
       tmem_st32(tm + lane_base + TM_AD2 + 32, kb1);
       g = 1.f;
-      for (int i = 0; i < C; ++i) {       // gamma_i = prod_{s<=i} alpha_s
-        g *= sAl[i * AL_S + c];
-        st_f32(GA + off_mn_sw128b32_f32(i, c, C), sB[i] * g * bf(sKr + i * DK + c));
-        sAl[i * AL_S + c] = g * bf(sQr + i * DK + c);  // Qhat (fp32, in place)
+#pragma unroll 1
+      for (int b = 0; b < 4; ++b) {       // gamma_i = prod_{s<=i} alpha_s
+        float a[16], kk_[16], qq[16], bb[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = 16 * b + u;
+          a[u] = sAl[i * AL_S + c];
+          kk_[u] = bf(sKr + i * DK + c);
+          qq[u] = bf(sQr + i * DK + c);
+          bb[u] = sB[i];
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = 16 * b + u;
+          g *= a[u];
+          st_f32(GA + off_mn_sw128b32_f32(i, c, C), bb[u] * g * kk_[u]);
+          sAl[i * AL_S + c] = g * qq[u];  // Qhat (fp32, in place)
+        }
       }
       sGC[c] = g;
     } else {
@@ -367,27 +480,42 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
       }
       __syncthreads();
     }
-    {  // thread = TMEM lane = row of [M T ; T]; warp halves take column halves
-      const int qw = warp & 3, hf = warp >> 2, Lr = 32 * qw + lane, j0 = 32 * hf;
-      float x[32];
+    // [M T ; T] = [M ; I] x T on the tensor cores, straight into TMEM
+    for (int task = tid; task < 128 * 16; task += NT) {  // A0 = [M ; I]
+      const int row = task >> 4, k4 = (task & 15) * 4;
+      float x[4];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] = 0.f;
-      if (Lr < C) {  // (M T)[i][j] = sum_{l=j}^{i} M[i][l] T[l][j]
-        const int i = Lr;
-        for (int l = j0; l <= i; ++l) {
-          const float m = sM[i * AS + l];
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (j0 + e <= l) x[e] += m * sT[l * AS + j0 + e];
-        }
-      } else {
-        const int i = Lr - C;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[e] = (j0 + e <= i) ? sT[i * AS + j0 + e] : 0.f;
+      for (int e = 0; e < 4; ++e) {
+        const int l = k4 + e;
+        x[e] = (row < C) ? ((l <= row) ? sM[row * AS + l] : 0.f) : ((l == row - C) ? 1.f : 0.f);
       }
+      st4_f32(sm + OFF_A0 + off_k_sw128_f32(row, k4, 128), x[0], x[1], x[2], x[3]);
+    }
+    for (int task = tid; task < C * 16; task += NT) {  // B0 = T (row l, columns j)
+      const int l = task >> 4, j4 = (task & 15) * 4;
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x[e] = (j4 + e <= l) ? sT[l * AS + j4 + e] : 0.f;
+      st4_f32(sm + OFF_B0 + off_mn_sw128b32_f32(l, j4, C), x[0], x[1], x[2], x[3]);
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < C / 8; ++kk)
+        mma_tf32_ss(tm + TM_AD5, desc_k_sw128_f32(sb + OFF_A0, 128, kk),
+                    desc_mn_sw128b32_f32(sb + OFF_B0, C, kk), ID_D0, kk > 0);
+      mma_commit(&bar[4]);
+    }
+    if (!wait_all(&bar[4], phase, s_abort)) break;
+    if ((warp & 3) < 2) {  // rows of M T: round the fp32 accumulator to tf32
+      const uint32_t ta = tm + lane_base + TM_AD5 + (uint32_t)(32 * (warp >> 2));
+      float x[32];
+      tmem_ld32(ta, x);
 #pragma unroll
       for (int e = 0; e < 32; ++e) x[e] = to_tf32(x[e]);
-      tmem_st32(tm + lane_base + TM_AD5 + (uint32_t)j0, x);
+      tmem_st32(ta, x);
     }
     tmem_wait_st();
     fence_before_sync();
@@ -489,7 +617,7 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
   if (*s_abort) {
     if (tid == 0) flag_error(err, kErrMbarTimeout);
     // give in-flight MMAs a bounded chance to drain before TMEM is released
-    for (int i = 0; i < 4; ++i) (void)mbar_wait(&bar[i], phase, 100000000LL);
+    for (int i = 0; i < 5; ++i) (void)mbar_wait(&bar[i], phase, 100000000LL);
   } else if (sfin && warp < 4) {
     const int r = tid;
 #pragma unroll

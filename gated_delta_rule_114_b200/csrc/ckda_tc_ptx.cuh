@@ -266,6 +266,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t phase,
   return true;
 }
 
+// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)
+               : "memory");
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (MMA).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -1,0 +1,54 @@
+"""Run one kernel of the library on one workload a few times (for profilers).
+
+    python -m gated_delta_rule_114_b200.run_case --case prefill [--T 4096] [--iters 3]
+    python -m gated_delta_rule_114_b200.run_case --case decode [--N 64] [--iters 3]
+
+The prefill case uses the CKDA long-prefill recipe (H=32, d=128, bf16 I/O,
+CKDA gates, random initial state) with T tokens per head; the decode case
+uses the decode recipe with N sequences. It prints nothing but a line with
+the shapes; it is meant to be wrapped by a profiler, not to time anything.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from gated_delta_rule_114_b200 import ckda
+from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,
+                                              make_decode_tokens,
+                                              make_fwd_inputs)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=["prefill", "decode"], default="prefill")
+    ap.add_argument("--T", type=int, default=4096)
+    ap.add_argument("--H", type=int, default=32)
+    ap.add_argument("--N", type=int, default=64)
+    ap.add_argument("--iters", type=int, default=3)
+    args = ap.parse_args()
+    ckda.load()
+    if args.case == "prefill":
+        w = WORKLOADS["ckda_B1_H32_T8192_d128"]
+        cu = torch.tensor([0, args.T], dtype=torch.int32)
+        inp = make_fwd_inputs(w, cu_seqlens=cu, H=args.H)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        for _ in range(args.iters):
+            ckda.fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                             d["initial_state"], d["cu_seqlens"], chunk=w.chunk)
+        shape = "T=%d H=%d d=128" % (args.T, args.H)
+    else:
+        w = WORKLOADS["decode_N256_H32_d128"]
+        state = make_decode_state(w, N=args.N).cuda()
+        tok = {k: v.cuda() for k, v in make_decode_tokens(w, 0, N=args.N).items()}
+        for _ in range(args.iters):
+            ckda.decode_step(tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"], state)
+        shape = "N=%d H=32 d=128" % args.N
+    torch.cuda.synchronize()
+    assert ckda.ckda_last_error() == ckda.CKDA_OK
+    print("run_case %s %s iters=%d ok" % (args.case, shape, args.iters))
+
+
+if __name__ == "__main__":
+    main()
