@@ -283,12 +283,15 @@ def main():
     N = dev["cu_seqlens"].numel() - 1
     o = torch.empty((T_total, H, dv), dtype=dev["q"].dtype, device="cuda")
     sf = torch.empty((N, H, dk, dv), dtype=torch.float32, device="cuda")
+    ws_bytes = ckda.ckda_fwd_workspace_bytes(N, T_total, H, dk, dv, w.chunk,
+                                             True, dev["q"].dtype)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
 
     def prefill():
         ckda.ckda_fwd_chunked(dev["q"], dev["k"], dev["v"], dev["alpha"],
                               dev["beta"], dev["initial_state"], sf, o,
                               dev["cu_seqlens"], None, chunk=w.chunk,
-                              stream=stream)
+                              stream=stream, workspace=ws)
 
     with ClockSampler(local) as clk:
         ms = time_loop(prefill, args.steps, args.warmup, stream, barrier)

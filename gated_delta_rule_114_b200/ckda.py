@@ -48,7 +48,10 @@ def load(path: str | None = None):
     lib.ckda_fwd_chunked.restype = ctypes.c_int
     lib.ckda_fwd_chunked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                      i32, i32, i32, i32, i32, i32, f32,
-                                     ctypes.c_int, vp]
+                                     ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.ckda_fwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.ckda_fwd_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32,
+                                             ctypes.c_int]
     lib.ckda_decode_step.restype = ctypes.c_int
     lib.ckda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
                                      i32, f32, ctypes.c_int, vp]
@@ -94,9 +97,18 @@ def _need(t, name, dtype=None, dims=None):
         raise ValueError("%s must have %d dims" % (name, dims))
 
 
+def ckda_fwd_workspace_bytes(N, T, H, d_k, d_v, chunk=0, varlen=False,
+                             dtype=torch.bfloat16) -> int:
+    """Scratch bytes ckda_fwd_chunked needs (see include/ckda.h)."""
+    return int(load().ckda_fwd_workspace_bytes(int(N), int(T), int(H), int(d_k),
+                                               int(d_v), int(chunk), int(bool(varlen)),
+                                               _DT[dtype]))
+
+
 def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
                      cu_seqlens=None, cu_seqlens_host=None, N=None, T=None,
-                     chunk: int = 0, scale: float = 1.0, stream=None):
+                     chunk: int = 0, scale: float = 1.0, stream=None,
+                     workspace=None):
     """Marshal tensors into ckda_fwd_chunked (see include/ckda.h).
 
     q, k [T_total, H, d_k]; v, o [T_total, H, d_v] (bf16 or fp32, one dtype);
@@ -104,6 +116,8 @@ def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
     [N, H, d_k, d_v] fp32 or None. With cu_seqlens (int32 CUDA [N+1]) the
     sequences are packed; otherwise give N and T (N sequences of T tokens).
     cu_seqlens_host: optional CPU int32 copy, validated by the library.
+    workspace: optional uint8 CUDA tensor of at least ckda_fwd_workspace_bytes
+    bytes; allocated with torch here when it is needed and not given.
     """
     lib = load()
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
@@ -129,11 +143,17 @@ def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
                 or not cu_seqlens_host.is_contiguous():
             raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
         host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    need = ckda_fwd_workspace_bytes(N, T, H, d_k, d_v, chunk,
+                                    cu_seqlens is not None, q.dtype)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib.ckda_fwd_chunked(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
                               _p(initial_state), _p(final_state), _p(o),
                               _p(cu_seqlens), host_ptr, int(N), int(T), int(H),
                               int(d_k), int(d_v), int(chunk), float(scale),
-                              _DT[q.dtype], _stream(stream))
+                              _DT[q.dtype], _p(workspace), ws_bytes,
+                              _stream(stream))
     _check(st, "ckda_fwd_chunked")
 
 
@@ -173,7 +193,7 @@ def version() -> int:
 def fwd_chunked(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None,
                 cu_seqlens_host=None, N=None, T=None, chunk: int = 0,
                 scale: float = 1.0, output_final_state: bool = True,
-                stream=None):
+                stream=None, workspace=None):
     """Allocate o (and the final state) with torch, then call ckda_fwd_chunked."""
     T_total, H, d_k = q.shape
     d_v = v.shape[2]
@@ -186,7 +206,7 @@ def fwd_chunked(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None,
     if output_final_state:
         sf = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=q.device)
     ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, sf, o, cu_seqlens,
-                     cu_seqlens_host, N, T, chunk, scale, stream)
+                     cu_seqlens_host, N, T, chunk, scale, stream, workspace)
     return o, sf
 
 

@@ -21,11 +21,13 @@ cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
                             int T_total, int H, float scale, unsigned int *err,
                             cudaStream_t st);
 bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt);
+size_t fwd_tc_workspace_bytes(int N, int T_total, int H, int dv);
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
                           const float *alpha, const float *beta,
                           const float *s0, float *sf, void *o,
                           const int32_t *cu, int N, int T, int T_total, int H,
-                          float scale, unsigned int *err, cudaStream_t st);
+                          float scale, void *ws, unsigned int *err,
+                          cudaStream_t st);
 }  // namespace ckda
 
 // The per-device error word. Each device context gets its own instance.
@@ -96,6 +98,17 @@ ckda_status ckda_last_error(cudaStream_t stream) {
   return w ? CKDA_ERR_DEVICE : CKDA_OK;
 }
 
+size_t ckda_fwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                int32_t d_v, int32_t chunk, int32_t varlen,
+                                ckda_dtype dt) {
+  if (chunk == 0) chunk = 64;
+  if (N <= 0 || T < 0 || H <= 0) return 0;
+  if (!ckda::fwd_tc_supported(d_k, d_v, chunk, dt)) return 0;
+  const int64_t T_total = varlen ? (int64_t)T : (int64_t)N * T;
+  if (T_total > INT32_MAX) return 0;
+  return ckda::fwd_tc_workspace_bytes(N, (int)T_total, H, d_v);
+}
+
 ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
                              const float *alpha, const float *beta,
                              const float *initial_state, float *final_state,
@@ -103,6 +116,7 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
                              const int32_t *cu_seqlens_host, int32_t N,
                              int32_t T, int32_t H, int32_t d_k, int32_t d_v,
                              int32_t chunk, float scale, ckda_dtype dt,
+                             void *workspace, size_t workspace_bytes,
                              cudaStream_t stream) {
   if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
@@ -111,7 +125,7 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
   if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
   if (!q || !k || !v || !alpha || !beta || !o) return CKDA_ERR_ARG;
   const void *ptrs[] = {q, k, v, alpha, beta, o, initial_state, final_state,
-                        cu_seqlens};
+                        cu_seqlens, workspace};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return CKDA_ERR_ARG;
 
@@ -144,13 +158,29 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
       overlaps(final_state, sb, initial_state, sb))
     return CKDA_ERR_ARG;
 
+  const size_t need = ckda_fwd_workspace_bytes(N, T, H, d_k, d_v, chunk,
+                                               cu_seqlens != nullptr, dt);
+  if (need > 0) {
+    if (!workspace || workspace_bytes < need) return CKDA_ERR_ARG;
+    const size_t ib = th * d_k * es;
+    if (overlaps(workspace, need, q, ib) || overlaps(workspace, need, k, ib) ||
+        overlaps(workspace, need, v, th * d_v * es) ||
+        overlaps(workspace, need, alpha, th * d_k * sizeof(float)) ||
+        overlaps(workspace, need, beta, th * sizeof(float)) ||
+        overlaps(workspace, need, o, ob) ||
+        overlaps(workspace, need, initial_state, sb) ||
+        overlaps(workspace, need, final_state, sb) ||
+        overlaps(workspace, need, cu_seqlens, (size_t)(N + 1) * sizeof(int32_t)))
+      return CKDA_ERR_ARG;
+  }
+
   if (N == 0) return CKDA_OK;
   unsigned int *err = error_word_ptr();
   cudaError_t e;
   if (ckda::fwd_tc_supported(d_k, d_v, chunk, dt)) {
     e = ckda::launch_fwd_tc(d_v, q, k, v, alpha, beta, initial_state, final_state, o,
-                            cu_seqlens, N, T, (int)T_total, H, scale, err,
-                            stream);
+                            cu_seqlens, N, T, (int)T_total, H, scale, workspace,
+                            err, stream);
   } else if (dt == CKDA_F32) {
     e = ckda::launch_fwd_simt<float>(d_k, d_v, chunk, q, k, v, alpha, beta,
                                      initial_state, final_state, o, cu_seqlens,

@@ -1,40 +1,42 @@
 // Chunkwise CKDA forward with tcgen05 tensor cores (sm_100a): bf16 I/O,
 // fp32 state, tf32 tensor-core operands with fp32 accumulation. d_k = 128,
-// chunk 64, d_v tiled by 32.
+// chunk 64, d_v in {32, 64, 128}.
 //
-// Operand precision: with bf16 operands the per-term rounding (2^-9) of the
-// chunk products adds up to about 2-3% of rms(o) on the CKDA and KDA
-// workloads (o is a difference of larger terms: Qhat S + M U), above the
-// 1e-2 rms bound; tf32 operands (2^-11) keep it near 2e-3. Every MMA here is
-// therefore kind::tf32, with operands rounded to tf32 when they are written.
+// Two kernels, split where the work changes character:
 //
-// One CTA per (sequence, head, 32-column d_v tile), 256 threads. The CTA
-// walks its sequence chunk by chunk; the state tile S (128 x 32) stays fp32 in
-// the registers of warps 0-3 (thread = state row) and is mirrored in shared
-// memory as an MMA operand.
+//  * ckda_chunk_prep_kernel: one CTA per (chunk, head), all chunks of all
+//    sequences in parallel. It builds everything about a chunk that does not
+//    depend on the state entering it (the chunk-WY / UT-transform factors of
+//    the product of diagonal-plus-rank-one transitions, Semidirect Fourier
+//    Delta Attention §2.2, and the affine chunk transfer's write summary, §1
+//    contribution 4), and stores the serial step's operands in a workspace:
+//        [Qtil ; W]   = [Qhat - M W ; T diag(beta) Khat]       128 x d_k
+//        Kbar^T                                                d_k x 64
+//        [M Ut ; Ut]  = [M T ; T] diag(beta) V                 128 x d_v
+//        gamma        = prod of the chunk's gates, per channel
+//  * ckda_chunk_scan_kernel: one CTA per (sequence, head, 32-column d_v tile)
+//    walks the chunks in order and only carries the state:
+//        D1 = [Qtil ; W] S  ->  O = scale (Qtil S + M Ut)   (rows 0..63)
+//                           ->  U = Ut - W S                (rows 64..127)
+//        D2 = Kbar^T U      ->  S <- diag(gamma) S + D2
+//    with the next chunk's operands bulk-copied into a second buffer while
+//    the current one is used.
+// O = Qhat S + M U with U = Ut - W S, so O = (Qhat - M W) S + M Ut: the output
+// costs no MMA of its own on the serial chain.
 //
-// Per chunk (positions i, j in 0..63; chunk-WY derivation in
-// ckda_fwd_simt.cu; Semidirect Fourier Delta Attention §2.2 and the affine
-// chunk transfer of §1 contribution 4):
+// Chunk factors (positions i, j in 0..63; G_{i<-j} = prod_{s=j+1..i} alpha_s;
+// gamma_i = G_{i<-0}; sigma_j = G_{63<-j}; see ckda_fwd_simt.cu):
+//   A_ij = beta_i k_i^T G_{i<-j} k_j (j<i), M_ij = q_i^T G_{i<-j} k_j (j<=i),
+//   T = (I + A)^{-1}, Khat_i = gamma_i k_i, Qhat_i = gamma_i q_i, Kbar_j = sigma_j k_j.
+// Gate factors are bounded running products (exact for negative and zero
+// gates; no logarithm, no division). Off-diagonal 16x16 sub-blocks of A and
+// M factor through the sub-block boundary and run as one MMA; the diagonal
+// sub-blocks use per-pair running products on CUDA cores.
 //
-//   1. load q, k, alpha, beta, v-tile into shared memory
-//   2. gate operands (bounded running products, exact for alpha <= 0):
-//        Lk_I = k * F, Lq_I = q * F  (F = G_{i<-16I-1}, rows of sub-block I)
-//        R^(I)_j = k_j * G_{16I-1<-j}  (j < 16 I)
-//   3. Grams A (beta-scaled, strictly lower) and M (lower):
-//        off-diagonal sub-blocks: one MMA  [Lk_1;Lq_1;..;Lq_3] x [R^(1);R^(2);R^(3)]^T
-//        diagonal 16x16 sub-blocks: running products on CUDA cores
-//   4. T = (I + A)^{-1} by blocked forward substitution (fp32), and M T;
-//      [M T ; T] is written straight into tensor memory (A operand)
-//   5. one MMA  [M T ; T] x [beta Khat | beta V]  gives  [M W | M Utilde ; W | Utilde]
-//        (W = T diag(beta) Khat, Utilde = T diag(beta) V); Qtil = Qhat - M W is
-//        formed in place in tensor memory: [Qtil ; W] is the next A operand
-//   6. serial state step (two dependent MMAs, A operands in tensor memory):
-//        D1 = [Qtil ; W] x S        -> O = scale (Qtil S + M Utilde)  (rows 0..63)
-//                                   -> U = Utilde - W S              (rows 64..127)
-//        D2 = Kbar^T x U            -> S <- diag(gamma_L) S + D2
-//   Since O = Qhat S + M U = (Qhat - M W) S + M Utilde, the output needs no MMA
-//   of its own on the serial chain.
+// Operand precision: with bf16 operands the rounding of the chunk products
+// adds up to about 2-3% of rms(o) on the CKDA and KDA workloads, above the
+// 1e-2 rms bound; tf32 operands keep it near 2e-3. Every MMA is kind::tf32,
+// operands rounded to tf32 when they are written.
 #include <cuda_bf16.h>
 
 #include "ckda.h"
@@ -46,49 +48,56 @@ namespace {
 
 using namespace tc;
 
-constexpr int C = 64, DK = 128, DVT = 32, NT = 256;
+constexpr int C = 64, DK = 128, DVT = 32;
 constexpr int AL_S = 132;  // fp32 row stride of alpha / Qhat
 constexpr int AS = 65;     // fp32 row stride of A, M, T
 
+// ---------------------------------------------------------------- workspace
+// One block per (chunk slot, head); chunk c of sequence n sits in slot
+// floor(cu[n] / 64) + n + c, which never collides and is below
+// floor(T_total / 64) + N.
+constexpr uint32_t WS_A1 = 0;       // [Qtil ; W]: 128 x 128 tf32, K-major sw128 image
+constexpr uint32_t WS_A2 = 65536;   // Kbar^T:     128 x 64 tf32, K-major sw128 image
+constexpr uint32_t WS_OU = 98304;   // [M Ut ; Ut]: 128 rows x d_v fp32, row-major
+__host__ __device__ constexpr uint32_t ws_gamma_off(int dv) { return WS_OU + 128u * dv * 4u; }
+__host__ __device__ constexpr uint32_t ws_block_bytes(int dv) {
+  return ws_gamma_off(dv) + 1024u;  // gamma: 128 fp32, block kept 1 KB aligned
+}
+
+// first slot of sequence n
+__device__ __forceinline__ int slot_base(const int32_t *cu, int n, int T) {
+  const int b = cu ? __ldg(cu + n) : n * T;
+  return b / C + n;
+}
+
+// ---------------------------------------------------------------- prep kernel
 // shared-memory map (byte offsets from a 1024-aligned base); fp32 operands.
 // MN-major tf32 operands use the 128B-swizzle / 32B-atom form (the only
 // MN-major form tcgen05 accepts for 32-bit elements).
-constexpr uint32_t OFF_GA = 0;        // 49152 Lk/Lq (96 rows x 128, K-major sw128)
-                                      //       -> [beta Khat | beta V] (N160 x K64 MN-sw128b32)
-constexpr uint32_t OFF_GB = 49152;    // 49152 R stack (96 rows x 128, K-major sw128)
-                                      //       -> [M ; I] (128 x 64 K-major) + T operand
-constexpr uint32_t OFF_A0 = OFF_GB;           // 32768 [M ; I], A of D0
-constexpr uint32_t OFF_B0 = OFF_GB + 32768;   // 16384 T, B of D0 (K64 x N64 MN-sw128b32)
-constexpr uint32_t OFF_SB = 98304;    // 16384 S, B of D1 (K128 x N32 MN-sw128b32)
-constexpr uint32_t OFF_UB = 114688;   //  8192 U, B of D2 (K64 x N32 MN-sw128b32)
-constexpr uint32_t OFF_Q = 122880;    // 16384 raw q bf16 [64][128] -> T fp32 [64][65]
-constexpr uint32_t OFF_K = 139264;    // 16384 raw k bf16 [64][128]    (T spills in)
-constexpr uint32_t OFF_XT = OFF_K + 4096;     //  3072 solve scratch (after raw k is dead)
-constexpr uint32_t OFF_AL = 155648;   // 33792 alpha fp32 [64][132] -> Qhat fp32
-constexpr uint32_t OFF_V = 189440;    //  4096 raw v bf16 [64][32]
-constexpr uint32_t OFF_A = 193536;    // 16640 A fp32 [64][65]
-constexpr uint32_t OFF_M = 210176;    // 16640 M fp32 [64][65]
-constexpr uint32_t OFF_B = 226816;    //   256 beta
-constexpr uint32_t OFF_GC = 227072;   //   512 gamma over the chunk
-constexpr uint32_t OFF_BAR = 227584;  //    64 mbarriers [0..4] + TMEM address + flags
-constexpr uint32_t SMEM_USED = 227648;
-constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // alignment slack
+constexpr int NTP = 256;
+constexpr uint32_t P_GA = 0;          // 49152 Lk/Lq (96 rows x 128, K-major)
+                                      //   -> [beta Khat | beta V] (K64 x N(128+dv) MN) 65536
+constexpr uint32_t P_GB = 49152;      // 49152 R stack (96 rows x 128, K-major)
+constexpr uint32_t P_A0 = 65536;      // 32768 [M ; I] (128 x 64 K-major), after the Grams
+constexpr uint32_t P_B0 = 98304;      // 16384 T (K64 x N64 MN)
+constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128] -> T fp32 [64][65]
+constexpr uint32_t P_K = 131072;      // 16384 raw k bf16 [64][128]    (T spills in)
+constexpr uint32_t P_XT = P_K + 4096; //  3072 solve scratch (after raw k is dead)
+constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
+constexpr uint32_t P_A = 181248;      // 16640 A fp32 [64][65]
+constexpr uint32_t P_M = 197888;      // 16640 M fp32 [64][65]
+constexpr uint32_t P_B = 214528;      //   256 beta
+constexpr uint32_t P_BAR = 214784;    //    64 mbarriers [0..2] + TMEM address + flag
+constexpr uint32_t P_SMEM = 214848 + 1024;
 
-// TMEM columns (512 allocated; one CTA per SM)
-constexpr uint32_t TM_G = 0;      //  96 Gram accumulator
-constexpr uint32_t TM_AD2 = 96;   //  64 Kbar^T (A of D2; lane = channel)
-constexpr uint32_t TM_D5 = 160;   // 160 [M W | M Ut ; W | Ut] -> [Qtil ; W] (A of D1)
-constexpr uint32_t TM_UT = 288;   //     (the M Ut / Ut columns of D5)
-constexpr uint32_t TM_AD5 = 320;  //  64 [M T ; T] (A of D5)
-constexpr uint32_t TM_D1 = 384;   //  32
-constexpr uint32_t TM_D2 = 416;   //  32
-constexpr uint32_t TM_COLS = 512;
+// TMEM columns of the prep kernel (512 allocated; one CTA per SM)
+constexpr uint32_t TP_G = 0;      //  96 Gram accumulator
+constexpr uint32_t TP_AD5 = 96;   //  64 [M T ; T] (A of D5)
+constexpr uint32_t TP_D5 = 160;   // 256 [M W | M Ut ; W | Ut]
+constexpr uint32_t TP_COLS = 512;
 
 constexpr uint32_t ID_G = idesc_tf32(128, 96, 0, 0);
 constexpr uint32_t ID_D0 = idesc_tf32(128, 64, 0, 1);
-constexpr uint32_t ID_D5 = idesc_tf32(128, 160, 0, 1);
-constexpr uint32_t ID_D1 = idesc_tf32(128, 32, 0, 1);
-constexpr uint32_t ID_D2 = idesc_tf32(128, 32, 0, 1);
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 __device__ __forceinline__ void st_f32(uint8_t *p, float x) {
@@ -108,45 +117,59 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase,
   return *s_abort == 0;
 }
 
-__global__ void __launch_bounds__(NT, 1)
-fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-              const __nv_bfloat16 *__restrict__ v, const float *__restrict__ alpha,
-              const float *__restrict__ beta, const float *__restrict__ s0,
-              float *__restrict__ sfin, __nv_bfloat16 *__restrict__ o,
-              const int32_t *__restrict__ cu, int T, int T_total, int H, int DV,
-              float scale, unsigned int *err) {
+__global__ void __launch_bounds__(NTP, 1)
+ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
+                       const __nv_bfloat16 *__restrict__ k,
+                       const __nv_bfloat16 *__restrict__ v,
+                       const float *__restrict__ alpha,
+                       const float *__restrict__ beta,
+                       const int32_t *__restrict__ cu, int N, int T, int T_total,
+                       int H, int DV, uint8_t *__restrict__ ws,
+                       unsigned int *err) {
+  // ---- which (sequence, chunk) this slot holds; empty slots leave at once
+  const int slot = blockIdx.x, h = blockIdx.y;
+  int n = 0;
+  {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (slot_base(cu, mid, T) <= slot) lo = mid;
+      else hi = mid - 1;
+    }
+    n = lo;
+  }
+  int bos, eos;
+  seq_bounds(cu, n, T, T_total, err, bos, eos);
+  const int cidx = slot - slot_base(cu, n, T);
+  const int t0 = bos + C * cidx;
+  if (cidx < 0 || t0 >= eos) return;
+  const int L = min(C, eos - t0);
+
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  uint8_t *GA = sm + OFF_GA, *GB = sm + OFF_GB, *SB = sm + OFF_SB, *UB = sm + OFF_UB;
-  const __nv_bfloat16 *sQr = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_Q);
-  const __nv_bfloat16 *sKr = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_K);
-  const __nv_bfloat16 *sVr = reinterpret_cast<const __nv_bfloat16 *>(sm + OFF_V);
-  float *sAl = reinterpret_cast<float *>(sm + OFF_AL);
-  float *sA = reinterpret_cast<float *>(sm + OFF_A);
-  float *sM = reinterpret_cast<float *>(sm + OFF_M);
-  float *sT = reinterpret_cast<float *>(sm + OFF_Q);
-  float *sXT = reinterpret_cast<float *>(sm + OFF_XT);
-  float *sB = reinterpret_cast<float *>(sm + OFF_B);
-  float *sGC = reinterpret_cast<float *>(sm + OFF_GC);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);  // [0..4]
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 48);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + OFF_BAR + 52);
+  uint8_t *GA = sm + P_GA, *GB = sm + P_GB;
+  const __nv_bfloat16 *sQr = reinterpret_cast<const __nv_bfloat16 *>(sm + P_Q);
+  const __nv_bfloat16 *sKr = reinterpret_cast<const __nv_bfloat16 *>(sm + P_K);
+  float *sAl = reinterpret_cast<float *>(sm + P_AL);
+  float *sA = reinterpret_cast<float *>(sm + P_A);
+  float *sM = reinterpret_cast<float *>(sm + P_M);
+  float *sT = reinterpret_cast<float *>(sm + P_Q);
+  float *sXT = reinterpret_cast<float *>(sm + P_XT);
+  float *sB = reinterpret_cast<float *>(sm + P_B);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..2]
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
+  uint8_t *wsb = ws + ((size_t)slot * H + h) * ws_block_bytes(DV);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int vt = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
-  const int c0 = vt * DVT;
-  int bos, eos;
-  seq_bounds(cu, n, T, T_total, err, bos, eos);
-  const size_t st_base = ((size_t)n * H + h) * DK * DV;
-
   if (warp == 0) {
-    tmem_alloc(s_tmem, TM_COLS);
+    tmem_alloc(s_tmem, TP_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 5; ++i) mbar_init(&bar[i], 1);
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -156,31 +179,15 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
-  // state rows in registers of warps 0..3 (thread = row r of the 128 x 32 tile)
-  float S[DVT];
-  if (warp < 4) {
-    const int r = tid;
-#pragma unroll
-    for (int e = 0; e < DVT; e += 4) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (s0) x = *reinterpret_cast<const float4 *>(s0 + st_base + (size_t)r * DV + c0 + e);
-      S[e] = x.x; S[e + 1] = x.y; S[e + 2] = x.z; S[e + 3] = x.w;
-      st4_f32(SB + off_mn_sw128b32_f32(r, e, DK), x.x, x.y, x.z, x.w);
-    }
-  }
-  float ut[DVT];  // rows of the D5 [M Ut ; Ut] columns (warps 0..3)
-  uint32_t phase = 0;
-
-  for (int t0 = bos; t0 < eos; t0 += C, phase ^= 1u) {
-    const int L = min(C, eos - t0);
+  do {  // one pass; `break` leaves on a timed-out wait
     // ---------------- 1. load the chunk: all global loads in flight at once
     {
-      uint4 qv[4], kv[4], vv;
+      uint4 qv[4], kv[4];
       float4 av[8];
       float bv = 0.f;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {  // q, k: 64 rows x 16 pieces of 16 bytes
-        const int idx = tid + u * NT, i = idx >> 4, ch = idx & 15;
+        const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
         qv[u] = kv[u] = make_uint4(0, 0, 0, 0);
         if (i < L) {
           const size_t off = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
@@ -190,43 +197,28 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {  // alpha: 64 rows x 32 float4
-        const int idx = tid + u * NT, i = idx >> 5, c4 = (idx & 31) * 4;
+        const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
         av[u] = make_float4(1.f, 1.f, 1.f, 1.f);
         if (i < L)
           av[u] = __ldg(reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4));
       }
-      {  // v tile: 64 rows x 64 bytes
-        const int i = tid >> 2, ch = tid & 3;
-        vv = make_uint4(0, 0, 0, 0);
-        if (i < L) vv = __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + i) * H + h) * DV + c0 + ch * 8));
-      }
       if (tid < L) bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int idx = tid + u * NT, i = idx >> 4, ch = idx & 15;
-        *reinterpret_cast<uint4 *>(sm + OFF_Q + i * 256 + ch * 16) = qv[u];
-        *reinterpret_cast<uint4 *>(sm + OFF_K + i * 256 + ch * 16) = kv[u];
+        const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
+        *reinterpret_cast<uint4 *>(sm + P_Q + i * 256 + ch * 16) = qv[u];
+        *reinterpret_cast<uint4 *>(sm + P_K + i * 256 + ch * 16) = kv[u];
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int idx = tid + u * NT, i = idx >> 5, c4 = (idx & 31) * 4;
+        const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
         *reinterpret_cast<float4 *>(sAl + i * AL_S + c4) = av[u];
       }
-      *reinterpret_cast<uint4 *>(sm + OFF_V + (tid >> 2) * 64 + (tid & 3) * 16) = vv;
       if (tid < C) sB[tid] = bv;
-    }
-    if (tid < C && t0 + C + tid < eos) {  // next chunk's rows into L2
-      const size_t th = (size_t)(t0 + C + tid) * H + h;
-      prefetch_l2(q + th * DK, DK * 2);
-      prefetch_l2(k + th * DK, DK * 2);
-      prefetch_l2(alpha + th * DK, DK * 4);
-      prefetch_l2(v + th * DV + c0, DVT * 2);
     }
     __syncthreads();
 
     // ---------------- 2. Gram operands (tf32, K-major 128B swizzle, 96 rows)
-    // Each thread owns one channel; a sub-block's 16 rows are read into
-    // registers before the running product walks them.
     if (tid < DK) {
       const int c = tid;
 #pragma unroll 1
@@ -285,8 +277,8 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < DK / 8; ++kk)
-        mma_tf32_ss(tm + TM_G, desc_k_sw128_f32(sb + OFF_GA, 96, kk),
-                    desc_k_sw128_f32(sb + OFF_GB, 96, kk), ID_G, kk > 0);
+        mma_tf32_ss(tm + TP_G, desc_k_sw128_f32(sb + P_GA, 96, kk),
+                    desc_k_sw128_f32(sb + P_GB, 96, kk), ID_G, kk > 0);
       mma_commit(&bar[0]);
     }
     // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile: thread (column
@@ -338,14 +330,13 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
           vv[16 + ii] += sq;
         }
       }
-      // reduce-scatter over the 16 lanes sharing column j
 #pragma unroll
-      for (int m = 8, n = 32; m > 0; m >>= 1, n >>= 1) {
+      for (int m = 8, nn = 32; m > 0; m >>= 1, nn >>= 1) {
         const bool up = (sl & m) != 0;
 #pragma unroll
-        for (int i = 0; i < n / 2; ++i) {
-          const float keep = up ? vv[n / 2 + i] : vv[i];
-          const float send = up ? vv[i] : vv[n / 2 + i];
+        for (int i = 0; i < nn / 2; ++i) {
+          const float keep = up ? vv[nn / 2 + i] : vv[i];
+          const float send = up ? vv[i] : vv[nn / 2 + i];
           vv[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
         }
       }
@@ -359,12 +350,12 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
         }
       }
     }
-    if (!wait_all(&bar[0], phase, s_abort)) break;
+    if (!wait_all(&bar[0], 0, s_abort)) break;
     // off-diagonal blocks out of TMEM: warp quarter qw <-> sub-block row I = qw+1
     if (warp == 0 || warp == 1 || warp == 6) {
       const int qw = warp & 3, I = qw + 1, ii = lane & 15, isM = lane >> 4;
       const int i = 16 * I + ii, off = 8 * I * (I - 1), ncols = 16 * I;
-      const uint32_t ta = tm + lane_base + TM_G + (uint32_t)off;
+      const uint32_t ta = tm + lane_base + TP_G + (uint32_t)off;
       for (int cb = 0; cb < ncols; cb += 16) {
         float x[16];
         tmem_ld16(ta + (uint32_t)cb, x);
@@ -378,10 +369,10 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
     fence_before_sync();
     __syncthreads();
 
-    // ---------------- 2b. Kbar^T (into TMEM), beta Khat | beta V, Qhat, gamma
+    // ---------------- 4. Kbar^T (to the workspace), beta Khat | beta V, Qhat, gamma
     if (tid < DK) {
-      const int c = tid;  // = TMEM lane of this thread
-      float kb0[32], kb1[32];
+      const int c = tid;
+      float kb[C];
       float g = 1.f;
 #pragma unroll
       for (int b = 3; b >= 0; --b) {  // sigma_j = prod_{s>j} alpha_s, j = 63..0
@@ -393,15 +384,14 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
         }
 #pragma unroll
         for (int u = 15; u >= 0; --u) {
-          const int j = 16 * b + u;
-          const float x = to_tf32(g * kk_[u]);
-          if (j >= 32) kb1[j - 32] = x;
-          else kb0[j] = x;
+          kb[16 * b + u] = to_tf32(g * kk_[u]);
           g *= a[u];
         }
       }
-      tmem_st32(tm + lane_base + TM_AD2, kb0);
-      tmem_st32(tm + lane_base + TM_AD2 + 32, kb1);
+#pragma unroll
+      for (int j = 0; j < C; j += 4)  // row c of Kbar^T (K-major sw128 image)
+        *reinterpret_cast<float4 *>(wsb + WS_A2 + off_k_sw128_f32(c, j, DK)) =
+            make_float4(kb[j], kb[j + 1], kb[j + 2], kb[j + 3]);
       g = 1.f;
 #pragma unroll 1
       for (int b = 0; b < 4; ++b) {       // gamma_i = prod_{s<=i} alpha_s
@@ -422,22 +412,34 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
           sAl[i * AL_S + c] = g * qq[u];  // Qhat (fp32, in place)
         }
       }
-      sGC[c] = g;
+      reinterpret_cast<float *>(wsb + ws_gamma_off(DV))[c] = g;
     } else {
-      for (int task = tid - DK; task < C * 8; task += NT - DK) {  // beta V columns
-        const int j = task >> 3, g4 = task & 7;
-        const float b = sB[j];
-        const __nv_bfloat16 *vr = sVr + j * DVT + 4 * g4;
-        st4_f32(GA + off_mn_sw128b32_f32(j, DK + 4 * g4, C), b * bf(vr), b * bf(vr + 1),
-                b * bf(vr + 2), b * bf(vr + 3));
+      // beta V columns 128 .. 128+DV of the D5 B operand, straight from global
+      const int nq = DV / 4;  // 4-column groups per row
+      for (int task0 = tid - DK; task0 < C * nq; task0 += 16 * (NTP - DK)) {
+        uint2 raw[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int task = task0 + u * (NTP - DK), j = task / nq, g4 = task % nq;
+          raw[u] = make_uint2(0, 0);
+          if (task < C * nq && j < L)
+            raw[u] = __ldg(reinterpret_cast<const uint2 *>(v + ((size_t)(t0 + j) * H + h) * DV + 4 * g4));
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int task = task0 + u * (NTP - DK), j = task / nq, g4 = task % nq;
+          if (task < C * nq) {
+            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u]);
+            const float2 x = __bfloat1622float2(p2[0]), y = __bfloat1622float2(p2[1]);
+            const float b = sB[j];
+            st4_f32(GA + off_mn_sw128b32_f32(j, DK + 4 * g4, C), b * x.x, b * x.y, b * y.x, b * y.y);
+          }
+        }
       }
     }
-    tmem_wait_st();
-    fence_async_smem();
-    fence_before_sync();
     __syncthreads();
 
-    // ---------------- 4. T = (I + A)^{-1}; then [M T ; T] into TMEM
+    // ---------------- 5. T = (I + A)^{-1} by blocked forward substitution
     if (tid < C) {
       const int b = tid >> 4, j = tid & 15, ob = b * 16;
       float t[16];
@@ -458,7 +460,7 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
     }
     __syncthreads();
     for (int d = 1; d < 4; ++d) {
-      for (int idx = tid; idx < (4 - d) * 256; idx += NT) {
+      for (int idx = tid; idx < (4 - d) * 256; idx += NTP) {
         const int p = idx >> 8, e = idx & 255, ii = e >> 4, jj = e & 15;
         const int I = d + p, J = p;
         float s = 0.f;
@@ -469,7 +471,7 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
         sXT[p * 256 + ii * 16 + jj] = s;
       }
       __syncthreads();
-      for (int idx = tid; idx < (4 - d) * 256; idx += NT) {
+      for (int idx = tid; idx < (4 - d) * 256; idx += NTP) {
         const int p = idx >> 8, e = idx & 255, ii = e >> 4, jj = e & 15;
         const int I = d + p, J = p;
         float s = 0.f;
@@ -480,8 +482,9 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
       }
       __syncthreads();
     }
-    // [M T ; T] = [M ; I] x T on the tensor cores, straight into TMEM
-    for (int task = tid; task < 128 * 16; task += NT) {  // A0 = [M ; I]
+
+    // ---------------- 6. [M T ; T] = [M ; I] x T on the tensor cores, into TMEM
+    for (int task = tid; task < 128 * 16; task += NTP) {  // A0 = [M ; I]
       const int row = task >> 4, k4 = (task & 15) * 4;
       float x[4];
 #pragma unroll
@@ -489,14 +492,14 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
         const int l = k4 + e;
         x[e] = (row < C) ? ((l <= row) ? sM[row * AS + l] : 0.f) : ((l == row - C) ? 1.f : 0.f);
       }
-      st4_f32(sm + OFF_A0 + off_k_sw128_f32(row, k4, 128), x[0], x[1], x[2], x[3]);
+      st4_f32(sm + P_A0 + off_k_sw128_f32(row, k4, 128), x[0], x[1], x[2], x[3]);
     }
-    for (int task = tid; task < C * 16; task += NT) {  // B0 = T (row l, columns j)
+    for (int task = tid; task < C * 16; task += NTP) {  // B0 = T (row l, columns j)
       const int l = task >> 4, j4 = (task & 15) * 4;
       float x[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) x[e] = (j4 + e <= l) ? sT[l * AS + j4 + e] : 0.f;
-      st4_f32(sm + OFF_B0 + off_mn_sw128b32_f32(l, j4, C), x[0], x[1], x[2], x[3]);
+      st4_f32(sm + P_B0 + off_mn_sw128b32_f32(l, j4, C), x[0], x[1], x[2], x[3]);
     }
     fence_async_smem();
     __syncthreads();
@@ -504,13 +507,13 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < C / 8; ++kk)
-        mma_tf32_ss(tm + TM_AD5, desc_k_sw128_f32(sb + OFF_A0, 128, kk),
-                    desc_mn_sw128b32_f32(sb + OFF_B0, C, kk), ID_D0, kk > 0);
-      mma_commit(&bar[4]);
+        mma_tf32_ss(tm + TP_AD5, desc_k_sw128_f32(sb + P_A0, 128, kk),
+                    desc_mn_sw128b32_f32(sb + P_B0, C, kk), ID_D0, kk > 0);
+      mma_commit(&bar[1]);
     }
-    if (!wait_all(&bar[4], phase, s_abort)) break;
+    if (!wait_all(&bar[1], 0, s_abort)) break;
     if ((warp & 3) < 2) {  // rows of M T: round the fp32 accumulator to tf32
-      const uint32_t ta = tm + lane_base + TM_AD5 + (uint32_t)(32 * (warp >> 2));
+      const uint32_t ta = tm + lane_base + TP_AD5 + (uint32_t)(32 * (warp >> 2));
       float x[32];
       tmem_ld32(ta, x);
 #pragma unroll
@@ -521,52 +524,166 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
     fence_before_sync();
     __syncthreads();
 
-    // ---------------- 5. [M T ; T] x [beta Khat | beta V]
+    // ---------------- 7. [M T ; T] x [beta Khat | beta V] -> workspace
     if (tid == 0) {
       fence_after_sync();
+      const uint32_t id5 = idesc_tf32(128, DK + DV, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < C / 8; ++kk)
-        mma_tf32_ts(tm + TM_D5, tm + TM_AD5 + (uint32_t)(8 * kk),
-                    desc_mn_sw128b32_f32(sb + OFF_GA, C, kk), ID_D5, kk > 0);
-      mma_commit(&bar[1]);
+        mma_tf32_ts(tm + TP_D5, tm + TP_AD5 + (uint32_t)(8 * kk),
+                    desc_mn_sw128b32_f32(sb + P_GA, C, kk), id5, kk > 0);
+      mma_commit(&bar[2]);
     }
-    if (!wait_all(&bar[1], phase, s_abort)) break;
-    {  // [M W ; W] -> [Qtil ; W] in place (tf32); keep [M Ut ; Ut] rows
-      const int qw = warp & 3, hf = warp >> 2, Lr = 32 * qw + lane;
+    if (!wait_all(&bar[2], 0, s_abort)) break;
+    {
+      const int qw = warp & 3, hw = warp >> 2, row = 32 * qw + lane;
+      if (hw == 0) {  // [Qtil ; W] rows, tf32, K-major sw128 image
+        for (int cb = 0; cb < DK; cb += 32) {
+          float x[32];
+          tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)cb, x);
+          if (row < C) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int cb = 64 * hf + 32 * half;
-        float x[32];
-        tmem_ld32(tm + lane_base + TM_D5 + (uint32_t)cb, x);
-        if (Lr < C) {
+            for (int e = 0; e < 32; ++e) x[e] = sAl[row * AL_S + cb + e] - x[e];
+          }
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = to_tf32(sAl[Lr * AL_S + cb + e] - x[e]);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) x[e] = to_tf32(x[e]);
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4 *>(wsb + WS_A1 + off_k_sw128_f32(row, cb + e, DK)) =
+                make_float4(to_tf32(x[e]), to_tf32(x[e + 1]), to_tf32(x[e + 2]), to_tf32(x[e + 3]));
         }
-        tmem_st32(tm + lane_base + TM_D5 + (uint32_t)cb, x);
+      } else {  // [M Ut ; Ut] rows, fp32 row-major
+        float *dst = reinterpret_cast<float *>(wsb + WS_OU) + (size_t)row * DV;
+        for (int cb = 0; cb < DV; cb += 32) {
+          float x[32];
+          tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)(DK + cb), x);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4 *>(dst + cb + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+        }
       }
-      if (hf == 0) tmem_ld32(tm + lane_base + TM_UT, ut);
     }
-    tmem_wait_st();
-    fence_before_sync();
-    __syncthreads();
+  } while (0);
 
-    // ---------------- 6. serial state step
+  if (*s_abort && tid == 0) flag_error(err, kErrMbarTimeout);
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after_sync();
+    tmem_dealloc(tm, TP_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- scan kernel
+constexpr int NTS = 128;
+constexpr uint32_t S_A1 = 0;          // 2 x 65536 [Qtil ; W] buffers
+constexpr uint32_t S_A2 = 131072;     // 2 x 32768 Kbar^T buffers
+constexpr uint32_t S_S = 196608;      // 16384 S, B of D1 (K128 x N32 MN)
+constexpr uint32_t S_U = 212992;      //  8192 U, B of D2 (K64 x N32 MN)
+constexpr uint32_t S_BAR = 221184;    //    64 mbarriers [0..2] + TMEM address + flag
+constexpr uint32_t S_SMEM = 221248 + 1024;
+constexpr uint32_t TS_D1 = 0, TS_D2 = 32, TS_COLS = 64;
+constexpr uint32_t ID_D1 = idesc_tf32(128, 32, 0, 1);
+constexpr uint32_t ID_D2 = idesc_tf32(128, 32, 0, 1);
+constexpr uint32_t LOAD_BYTES = 65536 + 32768;
+
+__global__ void __launch_bounds__(NTS, 1)
+ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
+                       __nv_bfloat16 *__restrict__ o, const int32_t *__restrict__ cu,
+                       int T, int T_total, int H, int DV, float scale,
+                       const uint8_t *__restrict__ ws, unsigned int *err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(sm);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S_BAR);  // [0..1] loads, [2] MMAs
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + S_BAR + 32);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + S_BAR + 36);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int vt = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int c0 = vt * DVT;
+  int bos, eos;
+  seq_bounds(cu, n, T, T_total, err, bos, eos);
+  const int nch = (eos - bos + C - 1) / C;
+  const int base = slot_base(cu, n, T);
+  const size_t st_base = ((size_t)n * H + h) * DK * DV;
+  const uint32_t wsz = ws_block_bytes(DV);
+
+  if (warp == 0) {
+    tmem_alloc(s_tmem, TS_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+    *s_abort = 0;
+    fence_mbar_init();
+    if (nch > 0) {  // chunk 0 into buffer 0
+      const uint8_t *blk = ws + ((size_t)base * H + h) * wsz;
+      mbar_arrive_expect_tx(&bar[0], LOAD_BYTES);
+      bulk_g2s(sm + S_A1, blk + WS_A1, 65536, &bar[0]);
+      bulk_g2s(sm + S_A2, blk + WS_A2, 32768, &bar[0]);
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tm = *s_tmem;
+  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+
+  // state row r = tid of the 128 x 32 tile, fp32 in registers
+  float S[DVT];
+  {
+    const int r = tid;
+#pragma unroll
+    for (int e = 0; e < DVT; e += 4) {
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (s0) x = *reinterpret_cast<const float4 *>(s0 + st_base + (size_t)r * DV + c0 + e);
+      S[e] = x.x; S[e + 1] = x.y; S[e + 2] = x.z; S[e + 3] = x.w;
+      st4_f32(sm + S_S + off_mn_sw128b32_f32(r, e, DK), x.x, x.y, x.z, x.w);
+    }
+  }
+  fence_async_smem();
+  __syncthreads();
+
+  for (int c = 0; c < nch; ++c) {
+    const int buf = c & 1;
+    const int t0 = bos + C * c, L = min(C, eos - t0);
+    // next chunk's operands into the other buffer (free: chunk c-1 is done)
+    if (tid == 0 && c + 1 < nch) {
+      const uint8_t *nb = ws + ((size_t)(base + c + 1) * H + h) * wsz;
+      mbar_arrive_expect_tx(&bar[buf ^ 1], LOAD_BYTES);
+      bulk_g2s(sm + S_A1 + (buf ^ 1) * 65536, nb + WS_A1, 65536, &bar[buf ^ 1]);
+      bulk_g2s(sm + S_A2 + (buf ^ 1) * 32768, nb + WS_A2, 32768, &bar[buf ^ 1]);
+    }
+    // this thread's row of [M Ut ; Ut] (d_v tile) and gamma of its state row
+    const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
+    float ou[DVT];
+    {
+      const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV + c0;
+#pragma unroll
+      for (int e = 0; e < DVT; e += 4) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(src + e));
+        ou[e] = x.x; ou[e + 1] = x.y; ou[e + 2] = x.z; ou[e + 3] = x.w;
+      }
+    }
+    const float gc = __ldg(reinterpret_cast<const float *>(blk + ws_gamma_off(DV)) + tid);
+    if (!mbar_wait(&bar[buf], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
+    __syncthreads();
+    if (*s_abort) break;
+
+    // D1 = [Qtil ; W] x S
     if (tid == 0) {
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < DK / 8; ++kk)
-        mma_tf32_ts(tm + TM_D1, tm + TM_D5 + (uint32_t)(8 * kk),
-                    desc_mn_sw128b32_f32(sb + OFF_SB, DK, kk), ID_D1, kk > 0);
+        mma_tf32_ss(tm + TS_D1, desc_k_sw128_f32(sb + S_A1 + buf * 65536, 128, kk),
+                    desc_mn_sw128b32_f32(sb + S_S, DK, kk), ID_D1, kk > 0);
       mma_commit(&bar[2]);
     }
-    if (!wait_all(&bar[2], phase, s_abort)) break;
-    if (warp < 4) {
+    if (!wait_all(&bar[2], 0, s_abort)) break;
+    {
       float d1[32];
-      tmem_ld32(tm + lane_base + TM_D1, d1);
-      if (warp < 2) {  // output rows
+      tmem_ld32(tm + lane_base + TS_D1, d1);
+      if (tid < C) {  // output rows
         const int i = tid;
         if (i < L) {
           __nv_bfloat16 *dst = o + ((size_t)(t0 + i) * H + h) * DV + c0;
@@ -574,40 +691,39 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
           for (int g8 = 0; g8 < 4; ++g8) {
             float y[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = scale * (d1[8 * g8 + e] + ut[8 * g8 + e]);
+            for (int e = 0; e < 8; ++e) y[e] = scale * (d1[8 * g8 + e] + ou[8 * g8 + e]);
             *reinterpret_cast<uint4 *>(dst + 8 * g8) = pack8_bf16(y);
           }
         }
-      } else {  // U = Utilde - W S
+      } else {  // U = Ut - W S
         const int j = tid - C;
 #pragma unroll
         for (int e = 0; e < DVT; e += 4)
-          st4_f32(UB + off_mn_sw128b32_f32(j, e, C), ut[e] - d1[e], ut[e + 1] - d1[e + 1],
-                  ut[e + 2] - d1[e + 2], ut[e + 3] - d1[e + 3]);
+          st4_f32(sm + S_U + off_mn_sw128b32_f32(j, e, C), ou[e] - d1[e], ou[e + 1] - d1[e + 1],
+                  ou[e + 2] - d1[e + 2], ou[e + 3] - d1[e + 3]);
       }
     }
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
+    // D2 = Kbar^T x U
     if (tid == 0) {
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < C / 8; ++kk)
-        mma_tf32_ts(tm + TM_D2, tm + TM_AD2 + (uint32_t)(8 * kk),
-                    desc_mn_sw128b32_f32(sb + OFF_UB, C, kk), ID_D2, kk > 0);
-      mma_commit(&bar[3]);
+        mma_tf32_ss(tm + TS_D2, desc_k_sw128_f32(sb + S_A2 + buf * 32768, 128, kk),
+                    desc_mn_sw128b32_f32(sb + S_U, C, kk), ID_D2, kk > 0);
+      mma_commit(&bar[2]);
     }
-    if (!wait_all(&bar[3], phase, s_abort)) break;
-    if (warp < 4) {
-      const int r = tid;
+    if (!wait_all(&bar[2], 1, s_abort)) break;
+    {
       float d2[32];
-      tmem_ld32(tm + lane_base + TM_D2, d2);
-      const float gc = sGC[r];
+      tmem_ld32(tm + lane_base + TS_D2, d2);
 #pragma unroll
       for (int e = 0; e < DVT; ++e) S[e] = gc * S[e] + d2[e];
 #pragma unroll
       for (int e = 0; e < DVT; e += 4)
-        st4_f32(SB + off_mn_sw128b32_f32(r, e, DK), S[e], S[e + 1], S[e + 2], S[e + 3]);
+        st4_f32(sm + S_S + off_mn_sw128b32_f32(tid, e, DK), S[e], S[e + 1], S[e + 2], S[e + 3]);
     }
     fence_async_smem();
     fence_before_sync();
@@ -616,9 +732,13 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
 
   if (*s_abort) {
     if (tid == 0) flag_error(err, kErrMbarTimeout);
-    // give in-flight MMAs a bounded chance to drain before TMEM is released
-    for (int i = 0; i < 5; ++i) (void)mbar_wait(&bar[i], phase, 100000000LL);
-  } else if (sfin && warp < 4) {
+    // let in-flight copies and MMAs drain (bounded) before shared memory and
+    // tensor memory are released
+    for (int i = 0; i < 3; ++i) {
+      (void)mbar_wait(&bar[i], 0, 100000000LL);
+      (void)mbar_wait(&bar[i], 1, 100000000LL);
+    }
+  } else if (sfin) {
     const int r = tid;
 #pragma unroll
     for (int e = 0; e < DVT; e += 4)
@@ -629,29 +749,45 @@ fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restri
   __syncthreads();
   if (warp == 0) {
     fence_after_sync();
-    tmem_dealloc(tm, TM_COLS);
+    tmem_dealloc(tm, TS_COLS);
   }
 }
 
 }  // namespace
 
 bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt) {
-  return dt == CKDA_BF16 && dk == 128 && chunk == 64 && (dv % DVT) == 0;
+  return dt == CKDA_BF16 && dk == 128 && chunk == 64 &&
+         (dv == 32 || dv == 64 || dv == 128);
+}
+
+size_t fwd_tc_workspace_bytes(int N, int T_total, int H, int dv) {
+  const size_t slots = (size_t)T_total / C + (size_t)N;
+  return slots * (size_t)H * ws_block_bytes(dv);
 }
 
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
                           const float *alpha, const float *beta,
                           const float *s0, float *sf, void *o,
                           const int32_t *cu, int N, int T, int T_total, int H,
-                          float scale, unsigned int *err, cudaStream_t st) {
-  if (dv % DVT != 0) return cudaErrorInvalidValue;
+                          float scale, void *ws, unsigned int *err,
+                          cudaStream_t st) {
+  if (!fwd_tc_supported(DK, dv, C, CKDA_BF16)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(
-      fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      ckda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
   if (e != cudaSuccess) return e;
-  const dim3 grid(dv / DVT, H, N);
-  fwd_tc_kernel<<<grid, NT, SMEM_BYTES, st>>>(
-      (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-      alpha, beta, s0, sf, (__nv_bfloat16 *)o, cu, T, T_total, H, dv, scale, err);
+  e = cudaFuncSetAttribute(ckda_chunk_scan_kernel,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
+  if (e != cudaSuccess) return e;
+  const int slots = T_total / C + N;
+  if (slots > 0 && T_total > 0) {
+    ckda_chunk_prep_kernel<<<dim3(slots, H), NTP, P_SMEM, st>>>(
+        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
+        alpha, beta, cu, N, T, T_total, H, dv, (uint8_t *)ws, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  ckda_chunk_scan_kernel<<<dim3(dv / DVT, H, N), NTS, S_SMEM, st>>>(
+      s0, sf, (__nv_bfloat16 *)o, cu, T, T_total, H, dv, scale, (const uint8_t *)ws, err);
   return cudaGetLastError();
 }
 

@@ -266,6 +266,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t phase,
   return true;
 }
 
+// Expect `bytes` of asynchronous transactions on an mbarrier (one arrival).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(mbar)),
+               "r"(bytes)
+               : "memory");
+}
+// Bulk copy global -> shared (this CTA), completion counted on an mbarrier.
+// Both addresses 16-byte aligned, bytes % 16 == 0. No multicast.
+__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32_t bytes,
+                                         uint64_t *mbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst_smem)),
+      "l"(src), "r"(bytes), "r"(smem_u32(mbar))
+      : "memory");
+}
+
 // Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
 __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)

@@ -16,8 +16,9 @@
  *
  * Conventions shared by every entry point:
  *  - All tensor pointers are DEVICE pointers on the current CUDA device unless
- *    a parameter says "host". The caller owns every buffer; the library never
- *    allocates device memory and keeps no pointer after a call returns.
+ *    a parameter says "host". The caller owns every buffer, scratch included
+ *    (ckda_fwd_workspace_bytes says how much); the library never allocates
+ *    device memory and keeps no pointer after a call returns.
  *  - Layouts are dense, row-major (C order), last dimension contiguous:
  *      q, k     [T, H, d_k]     v, o      [T, H, d_v]
  *      alpha    [T, H, d_k] fp32          beta      [T, H]  fp32
@@ -36,6 +37,7 @@
 #ifndef CKDA_H
 #define CKDA_H
 
+#include <stddef.h>
 #include <stdint.h>
 #include <cuda_runtime_api.h>
 
@@ -90,6 +92,13 @@ typedef enum {
  * chunk         chunk length: 0 (default 64), 16, 32 or 64.
  * scale         multiplies every output (o_t = scale * S_t^T q_t).
  * dt            element type of q, k, v and o.
+ * workspace     device scratch of at least workspace_bytes bytes, 16-byte
+ *               aligned, owned by the caller, or NULL when
+ *               ckda_fwd_workspace_bytes() returns 0 for these arguments.
+ *               Its contents on entry are ignored; it must not overlap any
+ *               other argument, and two calls running at the same time on
+ *               the GPU must not share it.
+ * workspace_bytes  size of workspace (CKDA_ERR_ARG if too small).
  */
 ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
                              const float *alpha, const float *beta,
@@ -98,7 +107,20 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
                              const int32_t *cu_seqlens_host, int32_t N,
                              int32_t T, int32_t H, int32_t d_k, int32_t d_v,
                              int32_t chunk, float scale, ckda_dtype dt,
+                             void *workspace, size_t workspace_bytes,
                              cudaStream_t stream);
+
+/*
+ * ckda_fwd_workspace_bytes: scratch that ckda_fwd_chunked needs for these
+ * arguments (same meaning as there; varlen != 0 means cu_seqlens is given, so
+ * T is the total token count). The tensor-core path (bf16, d_k = 128, chunk
+ * 64, d_v in {32, 64, 128}) keeps each chunk's state-independent factors
+ * there between its two kernels: about 160 KB per (chunk, head) for d_v = 128,
+ * for floor(T_total / 64) + N chunk slots. Other arguments need none (0).
+ */
+size_t ckda_fwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                int32_t d_v, int32_t chunk, int32_t varlen,
+                                ckda_dtype dt);
 
 /*
  * ckda_decode_step: one recurrent step for N sequences x H heads, one new

@@ -61,9 +61,10 @@ NULL = None
 
 
 def fwd(lib, q=P, k=P2, v=P3, a=P4, b=P5, s0=NULL, sf=NULL, o=P6, cu=NULL,
-        cuh=NULL, N=1, T=8, H=1, dk=16, dv=16, chunk=0, dt=ckda.CKDA_F32):
+        cuh=NULL, N=1, T=8, H=1, dk=16, dv=16, chunk=0, dt=ckda.CKDA_F32,
+        ws=NULL, wsb=0):
     return lib.ckda_fwd_chunked(q, k, v, a, b, s0, sf, o, cu, cuh, N, T, H, dk,
-                                dv, chunk, 1.0, dt, None)
+                                dv, chunk, 1.0, dt, ws, wsb, None)
 
 
 def dec(lib, q=P, k=P2, v=P3, a=P4, b=P5, s=P6, o=ctypes.c_void_p(0x70000),
@@ -91,6 +92,29 @@ def dec(lib, q=P, k=P2, v=P3, a=P4, b=P5, s=P6, o=ctypes.c_void_p(0x70000),
 ])
 def test_fwd_rejects(lib, kw, want):
     assert fwd(lib, **kw) == want
+
+
+def test_workspace_query(lib):
+    # tensor-core path (bf16, d_k=128, chunk 64): one block per (slot, head)
+    # 1 sequence of 64 tokens: floor(64/64) + 1 = 2 chunk slots
+    block = ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 128) // 2
+    assert block > 0 and block % 1024 == 0
+    assert ckda.ckda_fwd_workspace_bytes(2, 8192, 32, 128, 128) == (2 * 8192 // 64 + 2) * 32 * block
+    assert ckda.ckda_fwd_workspace_bytes(1, 100, 1, 128, 128, varlen=True) == 2 * block
+    assert ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 32) < 2 * block
+    # CUDA-core path and unsupported arguments need none
+    assert ckda.ckda_fwd_workspace_bytes(1, 64, 1, 64, 64) == 0
+    assert ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 128, dtype=__import__("torch").float32) == 0
+    assert ckda.ckda_fwd_workspace_bytes(0, 64, 1, 128, 128) == 0
+
+
+def test_fwd_rejects_missing_workspace(lib):
+    # bf16, d=128, chunk 64 needs scratch: none given -> argument error
+    st = fwd(lib, dk=128, dv=128, dt=ckda.CKDA_BF16, T=64)
+    assert st == ckda.CKDA_ERR_ARG
+    st = fwd(lib, dk=128, dv=128, dt=ckda.CKDA_BF16, T=64,
+             ws=ctypes.c_void_p(0x1000000), wsb=16)
+    assert st == ckda.CKDA_ERR_ARG
 
 
 @pytest.mark.parametrize("cu_host", [(1, 8), (0, 9), (0, 5, 3, 8)])
