@@ -52,6 +52,10 @@ def load(path: str | None = None):
     lib.ckda_fwd_workspace_bytes.restype = ctypes.c_size_t
     lib.ckda_fwd_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32,
                                              ctypes.c_int]
+    lib.ckda_fwd_chunked_noalloc.restype = ctypes.c_int
+    lib.ckda_fwd_chunked_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                             i32, i32, i32, i32, i32, i32, f32,
+                                             ctypes.c_int, vp]
     lib.ckda_decode_step.restype = ctypes.c_int
     lib.ckda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
                                      i32, f32, ctypes.c_int, vp]
@@ -155,6 +159,52 @@ def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
                               _DT[q.dtype], _p(workspace), ws_bytes,
                               _stream(stream))
     _check(st, "ckda_fwd_chunked")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20  # CKDA_NOALLOC_SCRATCH_BYTES in include/ckda.h
+
+
+def ckda_fwd_chunked_noalloc(q, k, v, alpha, beta, initial_state, final_state,
+                             o, cu_seqlens=None, cu_seqlens_host=None, N=None,
+                             T=None, chunk: int = 0, scale: float = 1.0,
+                             stream=None):
+    """Marshal tensors into ckda_fwd_chunked_noalloc (see include/ckda.h).
+
+    For callers that cannot provide device scratch: the library uses its own
+    fixed array of NOALLOC_SCRATCH_BYTES per device, shared by all calls, so
+    calls must not overlap on the GPU. Arguments as in ckda_fwd_chunked.
+    Nothing is allocated here either.
+    """
+    lib = load()
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, nme, q.dtype, 3)
+    _need(alpha, "alpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v, o must be bfloat16 or float32")
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+        T = T_total
+    elif N is None or T is None:
+        raise ValueError("give cu_seqlens, or N and T")
+    for t, nme in ((initial_state, "initial_state"), (final_state, "final_state")):
+        if t is not None:
+            _need(t, nme, torch.float32, 4)
+    host_ptr = None
+    if cu_seqlens_host is not None:
+        if cu_seqlens_host.is_cuda or cu_seqlens_host.dtype != torch.int32 \
+                or not cu_seqlens_host.is_contiguous():
+            raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
+        host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    st = lib.ckda_fwd_chunked_noalloc(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
+                                      _p(initial_state), _p(final_state), _p(o),
+                                      _p(cu_seqlens), host_ptr, int(N), int(T),
+                                      int(H), int(d_k), int(d_v), int(chunk),
+                                      float(scale), _DT[q.dtype], _stream(stream))
+    _check(st, "ckda_fwd_chunked_noalloc")
 
 
 def ckda_decode_step(q, k, v, alpha, beta, state, o, scale: float = 1.0,

@@ -123,6 +123,40 @@ size_t ckda_fwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
                                 ckda_dtype dt);
 
 /*
+ * ckda_fwd_chunked_noalloc: ckda_fwd_chunked for callers that cannot give the
+ * library any device memory. It has no counterpart in the paper; it exists
+ * because some callers have no device allocator to draw a workspace from
+ * (a plain C program) or must not call cudaMalloc while they run (a serving
+ * loop, where cudaMalloc may synchronise the device and stall other work).
+ *
+ * Same arguments and results as ckda_fwd_chunked, without the workspace: the
+ * scratch is one array of CKDA_NOALLOC_SCRATCH_BYTES bytes of device memory
+ * inside the library, which every GPU that loads the library keeps until the
+ * process exits. The function allocates nothing.
+ *  - Limit: calls whose ckda_fwd_workspace_bytes() exceeds
+ *    CKDA_NOALLOC_SCRATCH_BYTES return CKDA_ERR_UNSUPPORTED and launch
+ *    nothing (with d_v = 128, 64 MiB holds about 400 (chunk slot, head)
+ *    pairs, e.g. 32 heads x 768 tokens). Calls that need no scratch run as in
+ *    ckda_fwd_chunked.
+ *  - The first call on each device looks up the array's device address (a
+ *    cudaGetSymbolAddress on the current device); make that first call before
+ *    any stream capture.
+ *  - All calls on a device share the one array, which keeps what the last
+ *    call left in it (nothing in it has to start at zero). Calls whose kernels
+ *    overlap on the GPU (different streams, or different host threads) race on
+ *    it: run them one after another.
+ */
+#define CKDA_NOALLOC_SCRATCH_BYTES (64u << 20)
+ckda_status ckda_fwd_chunked_noalloc(const void *q, const void *k, const void *v,
+                                     const float *alpha, const float *beta,
+                                     const float *initial_state, float *final_state,
+                                     void *o, const int32_t *cu_seqlens,
+                                     const int32_t *cu_seqlens_host, int32_t N,
+                                     int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                     int32_t chunk, float scale, ckda_dtype dt,
+                                     cudaStream_t stream);
+
+/*
  * ckda_decode_step: one recurrent step for N sequences x H heads, one new
  * token each, updating the state in place (the recurrence above applied once;
  * Semidirect Fourier Delta Attention §1 eq. (1), readout §3 eq. (14)).
