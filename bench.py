@@ -59,6 +59,18 @@ def esize(dt):
     return 2 if dt == torch.bfloat16 else 4
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of the current kernels, scaled by the units processed; the
+# capture, its command and the scaling are in profiles/. Set to None whenever
+# a kernel changes after its capture.
+NCU_TRAFFIC = {
+    # prep + scan at T=2048, H=32 (1024 chunk-heads): 383.0 MB, x4 for T=8192
+    "prefill": 4 * 383.0e6,
+    # N=64 (2048 pairs): 212.8 MB, x4 for N=256
+    "decode": 4 * 212.8e6,
+}
+
+
 def prefill_bytes(inp) -> int:
     """Algorithmic HBM bytes of one forward: every input read once, every
     output written once (q, k, v, alpha, beta, o per token-head; states)."""
@@ -309,7 +321,7 @@ def main():
     achieved = nbytes / (ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
                 "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
-                "traffic": None, "peak_source": pk["source"],
+                "traffic": NCU_TRAFFIC["prefill"], "peak_source": pk["source"],
                 "algorithmic_bytes_per_launch": nbytes,
                 "tensor": {"achieved_tflops": flops / (ms / 1e3) / 1e12,
                            "peak_tflops": pk["bf16_tflops"],
@@ -362,7 +374,8 @@ def main():
               "steps": args.decode_steps,
               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": pk["hbm_gbs"],
                            "unit": "GB/s", "frac": dgbs / pk["hbm_gbs"],
-                           "traffic": None, "algorithmic_bytes_per_launch": dbytes},
+                           "traffic": NCU_TRAFFIC["decode"],
+                           "algorithmic_bytes_per_launch": dbytes},
               "gpu_launches": args.decode_steps, "clocks": dclk.summary()}
 
     cpu = None
@@ -385,7 +398,8 @@ def main():
                    "l2": "inputs larger than L2 (%.0f MB per step)" % (nbytes / 1e6),
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": args.steps, "clocks": clk.summary(), "decode": decode,
+        # each forward call launches the prep and the scan kernel
+        "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "decode": decode,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -644,6 +644,21 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   fence_async_smem();
   __syncthreads();
 
+  // this thread's row of [M Ut ; Ut] (d_v tile) and gamma of its state row,
+  // read one chunk ahead so the loads overlap the previous chunk's MMAs
+  float ou_next[DVT], gc_next = 0.f;
+  auto load_rows = [&](int c) {
+    const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
+    const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV + c0;
+#pragma unroll
+    for (int e = 0; e < DVT; e += 4) {
+      const float4 x = __ldg(reinterpret_cast<const float4 *>(src + e));
+      ou_next[e] = x.x; ou_next[e + 1] = x.y; ou_next[e + 2] = x.z; ou_next[e + 3] = x.w;
+    }
+    gc_next = __ldg(reinterpret_cast<const float *>(blk + ws_gamma_off(DV)) + tid);
+  };
+  if (nch > 0) load_rows(0);
+
   for (int c = 0; c < nch; ++c) {
     const int buf = c & 1;
     const int t0 = bos + C * c, L = min(C, eos - t0);
@@ -654,18 +669,11 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
       bulk_g2s(sm + S_A1 + (buf ^ 1) * 65536, nb + WS_A1, 65536, &bar[buf ^ 1]);
       bulk_g2s(sm + S_A2 + (buf ^ 1) * 32768, nb + WS_A2, 32768, &bar[buf ^ 1]);
     }
-    // this thread's row of [M Ut ; Ut] (d_v tile) and gamma of its state row
-    const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
     float ou[DVT];
-    {
-      const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV + c0;
 #pragma unroll
-      for (int e = 0; e < DVT; e += 4) {
-        const float4 x = __ldg(reinterpret_cast<const float4 *>(src + e));
-        ou[e] = x.x; ou[e + 1] = x.y; ou[e + 2] = x.z; ou[e + 3] = x.w;
-      }
-    }
-    const float gc = __ldg(reinterpret_cast<const float *>(blk + ws_gamma_off(DV)) + tid);
+    for (int e = 0; e < DVT; ++e) ou[e] = ou_next[e];
+    const float gc = gc_next;
+    if (c + 1 < nch) load_rows(c + 1);
     if (!mbar_wait(&bar[buf], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
     __syncthreads();
     if (*s_abort) break;

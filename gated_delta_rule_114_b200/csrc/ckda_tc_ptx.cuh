@@ -266,6 +266,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t phase,
   return true;
 }
 
+// Plain arrival of this thread on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t *mbar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(mbar)) : "memory");
+}
+// Barrier among the `count` threads (a multiple of 32) that use named barrier `id`.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // Expect `bytes` of asynchronous transactions on an mbarrier (one arrival).
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *mbar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(mbar)),
