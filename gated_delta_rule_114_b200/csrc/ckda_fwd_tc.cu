@@ -4,8 +4,9 @@
 //
 // Two kernels, split where the work changes character:
 //
-//  * ckda_chunk_prep_kernel: one CTA per (chunk, head), all chunks of all
-//    sequences in parallel. It builds everything about a chunk that does not
+//  * ckda_chunk_prep_kernel: persistent, one CTA per SM, walking the (chunk,
+//    head) items of all sequences (a small kernel first tabulates which
+//    chunk each slot holds). For each item it builds everything that does not
 //    depend on the state entering it (the chunk-WY / UT-transform factors of
 //    the product of diagonal-plus-rank-one transitions, Semidirect Fourier
 //    Delta Attention §2.2, and the affine chunk transfer's write summary, §1
@@ -39,6 +40,9 @@
 // operands rounded to tf32 when they are written.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+#include <mutex>
+
 #include "ckda.h"
 #include "ckda_common.cuh"
 #include "ckda_tc_ptx.cuh"
@@ -50,7 +54,15 @@ using namespace tc;
 
 constexpr int C = 64, DK = 128, DVT = 32;
 constexpr int AL_S = 132;  // fp32 row stride of alpha / Qhat
-constexpr int AS = 65;     // fp32 row stride of A, M, T
+
+// Float offset of (row i, channel c) in the alpha / Qhat buffer: the 16-byte
+// piece p = c / 4 of a row sits at p ^ ((p >> 3) & 1), so that the 16 lanes
+// of a half-warp reading pieces 2 sl (or 2 sl + 1) of one row hit every bank
+// group twice, not half of them four times.
+__device__ __forceinline__ int al_off(int i, int c) {
+  const int p = c >> 2;
+  return i * AL_S + 4 * (p ^ ((p >> 3) & 1)) + (c & 3);
+}
 
 // ---------------------------------------------------------------- workspace
 // One block per (chunk slot, head); chunk c of sequence n sits in slot
@@ -58,7 +70,7 @@ constexpr int AS = 65;     // fp32 row stride of A, M, T
 // floor(T_total / 64) + N.
 constexpr uint32_t WS_A1 = 0;       // [Qtil ; W]: 128 x 128 tf32, K-major sw128 image
 constexpr uint32_t WS_A2 = 65536;   // Kbar^T:     128 x 64 tf32, K-major sw128 image
-constexpr uint32_t WS_OU = 98304;   // [M Ut ; Ut]: 128 rows x d_v fp32, row-major
+constexpr uint32_t WS_OU = 98304;   // [M Ut ; Ut]: 128 rows x d_v fp32, 16-byte pieces swizzled by row
 __host__ __device__ constexpr uint32_t ws_gamma_off(int dv) { return WS_OU + 128u * dv * 4u; }
 __host__ __device__ constexpr uint32_t ws_block_bytes(int dv) {
   return ws_gamma_off(dv) + 1024u;  // gamma: 128 fp32, block kept 1 KB aligned
@@ -70,25 +82,62 @@ __device__ __forceinline__ int slot_base(const int32_t *cu, int n, int T) {
   return b / C + n;
 }
 
+// Slot table (after the blocks): per slot, {first token, tokens} of the chunk
+// it holds ({0, 0} for an empty slot).
+__host__ __device__ constexpr size_t slot_table_off(size_t slots, size_t H, int dv) {
+  return slots * H * ws_block_bytes(dv);
+}
+__host__ __device__ constexpr size_t slot_table_bytes(size_t slots) {
+  return (slots * sizeof(int2) + 1023) & ~size_t(1023);
+}
+
+// One thread per slot: which (sequence, chunk) the slot holds. Every slot is
+// written, and a malformed device cu_seqlens only ever yields token ranges
+// inside [0, T_total) (seq_bounds flags it).
+__global__ void ckda_slot_table_kernel(const int32_t *__restrict__ cu, int N, int T,
+                                       int T_total, int slots, int2 *__restrict__ tab,
+                                       unsigned int *err) {
+  const int slot = blockIdx.x * blockDim.x + threadIdx.x;
+  if (slot >= slots) return;
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (slot_base(cu, mid, T) <= slot) lo = mid;
+    else hi = mid - 1;
+  }
+  int bos, eos;
+  seq_bounds(cu, lo, T, T_total, err, bos, eos);
+  const int cidx = slot - slot_base(cu, lo, T);
+  const long long t0 = (long long)bos + (long long)C * cidx;
+  int2 e = make_int2(0, 0);
+  if (cidx >= 0 && t0 < eos) e = make_int2((int)t0, min(C, eos - (int)t0));
+  tab[slot] = e;
+}
+
 // ---------------------------------------------------------------- prep kernel
 // shared-memory map (byte offsets from a 1024-aligned base); fp32 operands.
 // MN-major tf32 operands use the 128B-swizzle / 32B-atom form (the only
 // MN-major form tcgen05 accepts for 32-bit elements).
-constexpr int NTP = 256;
-constexpr uint32_t P_GA = 0;          // 49152 Lk/Lq (96 rows x 128, K-major)
-                                      //   -> [beta Khat | beta V] (K64 x N(128+dv) MN) 65536
+constexpr int NTP = 512;
+constexpr int RS = 68;                // fp32 row stride of A, M, T (16-byte aligned rows)
+constexpr uint32_t P_GA = 0;          // 65536 Lk/Lq (96 rows x 128, K-major)
+                                      //   -> [beta Khat | beta V] (K64 x N(128+dv), MN)
+                                      //   -> staged [Qtil ; W] image (epilogue)
 constexpr uint32_t P_GB = 49152;      // 49152 R stack (96 rows x 128, K-major)
-constexpr uint32_t P_A0 = 65536;      // 32768 [M ; I] (128 x 64 K-major), after the Grams
+constexpr uint32_t P_A0 = 65536;      // 32768 [M ; I] (128 x 64 K-major)
+constexpr uint32_t P_OU = 65536;      // <=65536 staged [M Ut ; Ut] rows (epilogue)
+constexpr uint32_t P_V = 98304;       // 16384 raw v bf16 [64][dv] (until beta V is built)
 constexpr uint32_t P_B0 = 98304;      // 16384 T (K64 x N64 MN)
-constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128] -> T fp32 [64][65]
+constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128] -> T fp32 [64][68]
 constexpr uint32_t P_K = 131072;      // 16384 raw k bf16 [64][128]    (T spills in)
 constexpr uint32_t P_XT = P_K + 4096; //  3072 solve scratch (after raw k is dead)
 constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
-constexpr uint32_t P_A = 181248;      // 16640 A fp32 [64][65]
-constexpr uint32_t P_M = 197888;      // 16640 M fp32 [64][65]
-constexpr uint32_t P_B = 214528;      //   256 beta
-constexpr uint32_t P_BAR = 214784;    //    64 mbarriers [0..2] + TMEM address + flag
-constexpr uint32_t P_SMEM = 214848 + 1024;
+constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68]
+constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
+constexpr uint32_t P_B = 216064;      //   256 beta
+constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..2] + TMEM address + flag
+constexpr uint32_t P_P = 216384;      //  2048 gate products of whole sub-blocks [4][128]
+constexpr uint32_t P_SMEM = 218432 + 1024;
 
 // TMEM columns of the prep kernel (512 allocated; one CTA per SM)
 constexpr uint32_t TP_G = 0;      //  96 Gram accumulator
@@ -107,6 +156,11 @@ __device__ __forceinline__ void st4_f32(uint8_t *p, float a, float b, float c, f
   *reinterpret_cast<float4 *>(p) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
+// Row r of [M Ut ; Ut] keeps its 16-byte piece p at p ^ (r mod 8), in the
+// workspace as in shared memory, so that the row-per-thread writes of the
+// prep epilogue hit distinct banks.
+__device__ __forceinline__ int ou_piece(int row, int piece) { return piece ^ (row & 7); }
+
 // Bounded wait of all threads on one mbarrier; false (and the abort flag set)
 // if it timed out. Ends with every thread past a CTA barrier.
 __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase,
@@ -123,28 +177,9 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                        const __nv_bfloat16 *__restrict__ v,
                        const float *__restrict__ alpha,
                        const float *__restrict__ beta,
-                       const int32_t *__restrict__ cu, int N, int T, int T_total,
+                       const int2 *__restrict__ slot_tab, int n_items,
                        int H, int DV, uint8_t *__restrict__ ws,
                        unsigned int *err) {
-  // ---- which (sequence, chunk) this slot holds; empty slots leave at once
-  const int slot = blockIdx.x, h = blockIdx.y;
-  int n = 0;
-  {
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (slot_base(cu, mid, T) <= slot) lo = mid;
-      else hi = mid - 1;
-    }
-    n = lo;
-  }
-  int bos, eos;
-  seq_bounds(cu, n, T, T_total, err, bos, eos);
-  const int cidx = slot - slot_base(cu, n, T);
-  const int t0 = bos + C * cidx;
-  if (cidx < 0 || t0 >= eos) return;
-  const int L = min(C, eos - t0);
-
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -158,10 +193,10 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   float *sT = reinterpret_cast<float *>(sm + P_Q);
   float *sXT = reinterpret_cast<float *>(sm + P_XT);
   float *sB = reinterpret_cast<float *>(sm + P_B);
+  float *sP = reinterpret_cast<float *>(sm + P_P);
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..2]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
-  uint8_t *wsb = ws + ((size_t)slot * H + h) * ws_block_bytes(DV);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (warp == 0) {
@@ -179,14 +214,33 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
+  // Persistent: items (slot, head) = it / H, it % H, strided by the grid.
+  // Each mbarrier completes once per non-empty item: parity `ph`.
+  uint32_t ph = 0;
+  int2 cur = make_int2(0, 0);
+  if ((int)blockIdx.x < n_items) cur = __ldg(slot_tab + blockIdx.x / H);
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+  const int slot = it / H, h = it - slot * H;
+  const int t0 = cur.x, L = cur.y;
+  const int nit = it + gridDim.x;
+  int2 nxt = make_int2(0, 0);
+  if (nit < n_items) nxt = __ldg(slot_tab + nit / H);
+  if (L <= 0) {  // empty slot (CTA-uniform)
+    cur = nxt;
+    continue;
+  }
+  uint8_t *wsb = ws + ((size_t)slot * H + h) * ws_block_bytes(DV);
+
   do {  // one pass; `break` leaves on a timed-out wait
     // ---------------- 1. load the chunk: all global loads in flight at once
     {
-      uint4 qv[4], kv[4];
-      float4 av[8];
+      uint4 qv[2], kv[2];
+      float4 av[4];
+      uint4 vr[2];
       float bv = 0.f;
+      const int nv = DV / 8;  // 16-byte pieces of a v row
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // q, k: 64 rows x 16 pieces of 16 bytes
+      for (int u = 0; u < 2; ++u) {  // q, k: 64 rows x 16 pieces of 16 bytes
         const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
         qv[u] = kv[u] = make_uint4(0, 0, 0, 0);
         if (i < L) {
@@ -196,78 +250,128 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         }
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // alpha: 64 rows x 32 float4
+      for (int u = 0; u < 4; ++u) {  // alpha: 64 rows x 32 float4
         const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
         av[u] = make_float4(1.f, 1.f, 1.f, 1.f);
         if (i < L)
           av[u] = __ldg(reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4));
       }
-      if (tid < L) bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {  // v: 64 rows x DV/8 pieces of 16 bytes
+        const int idx = tid + u * NTP, i = idx / nv, p8 = idx % nv;
+        vr[u] = make_uint4(0, 0, 0, 0);
+        if (idx < C * nv && i < L)
+          vr[u] = __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + i) * H + h) * DV + 8 * p8));
+      }
+      if (tid < L) bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
+      // the previous item's bulk stores read staging that overlaps v and q
+      if (tid == 0) bulk_wait_read0();
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
         const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
         *reinterpret_cast<uint4 *>(sm + P_Q + i * 256 + ch * 16) = qv[u];
         *reinterpret_cast<uint4 *>(sm + P_K + i * 256 + ch * 16) = kv[u];
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 4; ++u) {
         const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
-        *reinterpret_cast<float4 *>(sAl + i * AL_S + c4) = av[u];
+        *reinterpret_cast<float4 *>(sAl + al_off(i, c4)) = av[u];
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int idx = tid + u * NTP;
+        if (idx < C * nv) *reinterpret_cast<uint4 *>(sm + P_V + idx * 16) = vr[u];
       }
       if (tid < C) sB[tid] = bv;
     }
     __syncthreads();
 
-    // ---------------- 2. Gram operands (tf32, K-major 128B swizzle, 96 rows)
-    if (tid < DK) {
-      const int c = tid;
-#pragma unroll 1
-      for (int I = 1; I < 4; ++I) {
-        float a[16], kk_[16], qq[16];
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          const int i = 16 * I + ii;
-          a[ii] = sAl[i * AL_S + c];
-          kk_[ii] = bf(sKr + i * DK + c);
-          qq[ii] = bf(sQr + i * DK + c);
-        }
-        float g = 1.f;
-#pragma unroll
-        for (int ii = 0; ii < 16; ++ii) {
-          g *= a[ii];
-          st_f32(GA + off_k_sw128_f32((I - 1) * 32 + ii, c, 96), g * kk_[ii]);
-          st_f32(GA + off_k_sw128_f32((I - 1) * 32 + 16 + ii, c, 96), g * qq[ii]);
-        }
+    // the next item's rows into L2 (one 128-byte line per thread and step;
+    // plain prefetches, which leave the bulk-copy unit to the workspace
+    // stores), while this item is computed
+    if (nxt.y > 0) {
+      const int nh = nit % H;
+      const int lq = DK * 2 / 128, la = DK * 4 / 128, lv = (DV * 2 + 127) / 128;
+      const int per = 2 * lq + la + lv;  // lines per token row
+      for (int t = tid; t < nxt.y * per; t += NTP) {
+        const int r = t / per, w = t % per;
+        const size_t tok = (size_t)(nxt.x + r) * H + nh;
+        const char *p;
+        if (w < lq) p = reinterpret_cast<const char *>(q + tok * DK) + 128 * w;
+        else if (w < 2 * lq) p = reinterpret_cast<const char *>(k + tok * DK) + 128 * (w - lq);
+        else if (w < 2 * lq + la) p = reinterpret_cast<const char *>(alpha + tok * DK) + 128 * (w - 2 * lq);
+        else p = reinterpret_cast<const char *>(v + tok * DV) + 128 * (w - 2 * lq - la);
+        prefetch_line_l2(p);
+        if (w == 0) prefetch_line_l2(beta + tok);
       }
-    } else {
-      // R^(I)_j = k_j G_{16I-1<-j}: one backward sweep over j = 47..0 carries
-      // the three running products (each starts at its own 16I-1)
-      const int c = tid - DK;
-      float g1 = 1.f, g2 = 1.f, g3 = 1.f;
-#pragma unroll 1
-      for (int b = 2; b >= 0; --b) {
-        float a[16], kk_[16];
+    }
+
+    // ---------------- 2. gate pass: thread (16-token sub-block g, channel c)
+    // forms the sub-block prefix products p_u = prod_{s=16g..16g+u} alpha_s
+    // and suffix products prod_{s=16g+u+1..16g+15} alpha_s, and the product
+    // P_g of the whole sub-block; with the P of the other sub-blocks
+    //   Lk_i = k_i G_{i<-16g-1} = k_i p_u, Lq_i = q_i p_u      (Gram rows, g >= 1)
+    //   R^(I)_j = k_j G_{16I-1<-j} = (k_j suffix_u) P_{g+1} .. P_{I-1}   (I > g)
+    //   Kbar_j = k_j sigma_j = (k_j suffix_u) P_{g+1} .. P_3
+    //   gamma_i = P_0 .. P_{g-1} p_u                           (kept for phase 4)
+    const int gq = tid >> 7, gc = tid & 127;
+    float pp[16], pre = 1.f;
+    {
+      float a[16], kr[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        a[u] = sAl[al_off(16 * gq + u, gc)];
+        kr[u] = bf(sKr + (16 * gq + u) * DK + gc);
+      }
+      float p = 1.f;
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        p *= a[u];
+        pp[u] = p;
+      }
+      float sfx = 1.f;
+#pragma unroll
+      for (int u = 15; u >= 0; --u) {
+        kr[u] *= sfx;  // k_j times the suffix product of its sub-block
+        sfx *= a[u];
+      }
+      sP[gq * DK + gc] = p;
+      __syncthreads();
+      float P[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) P[b] = sP[b * DK + gc];
+      float suf = 1.f;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        if (b < gq) pre *= P[b];
+        if (b > gq) suf *= P[b];
+      }
+      if (gq >= 1) {
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          const int j = 16 * b + u;
-          a[u] = sAl[j * AL_S + c];
-          kk_[u] = bf(sKr + j * DK + c);
-        }
-#pragma unroll
-        for (int u = 15; u >= 0; --u) {
-          const int j = 16 * b + u;
-          st_f32(GB + off_k_sw128_f32(48 + j, c, 96), g3 * kk_[u]);
-          g3 *= a[u];
-          if (b <= 1) {
-            st_f32(GB + off_k_sw128_f32(16 + j, c, 96), g2 * kk_[u]);
-            g2 *= a[u];
-          }
-          if (b == 0) {
-            st_f32(GB + off_k_sw128_f32(j, c, 96), g1 * kk_[u]);
-            g1 *= a[u];
-          }
+          const int i = 16 * gq + u;
+          const float kk = bf(sKr + i * DK + gc), qq = bf(sQr + i * DK + gc);
+          st_f32(GA + off_k_sw128_f32((gq - 1) * 32 + u, gc, 96), pp[u] * kk);
+          st_f32(GA + off_k_sw128_f32((gq - 1) * 32 + 16 + u, gc, 96), pp[u] * qq);
         }
       }
+      float f = 1.f;
+#pragma unroll
+      for (int I = 1; I < 4; ++I) {
+        if (I > gq) {
+          if (I > gq + 1) f *= P[I - 1];
+#pragma unroll
+          for (int u = 0; u < 16; ++u)
+            st_f32(GB + off_k_sw128_f32(8 * I * (I - 1) + 16 * gq + u, gc, 96), f * kr[u]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 16; u += 4)  // row c of Kbar^T (K-major sw128 image)
+        *reinterpret_cast<float4 *>(wsb + WS_A2 + off_k_sw128_f32(gc, 16 * gq + u, DK)) =
+            make_float4(to_tf32(suf * kr[u]), to_tf32(suf * kr[u + 1]),
+                        to_tf32(suf * kr[u + 2]), to_tf32(suf * kr[u + 3]));
+      if (gq == 3) reinterpret_cast<float *>(wsb + ws_gamma_off(DV))[gc] = pre * pp[15];
     }
     fence_async_smem();
     __syncthreads();
@@ -281,165 +385,123 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                     desc_k_sw128_f32(sb + P_GB, 96, kk), ID_G, kk > 0);
       mma_commit(&bar[0]);
     }
-    // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile: thread (column
-    // j, lane sl) runs the gate product over channels 8 sl .. 8 sl + 7; the 16
-    // lanes of a half-warp are then reduced with a reduce-scatter butterfly
-    // that leaves entries 2 sl, 2 sl + 1 of [A column | M column] in lane sl.
-    for (int I = 0; I < 4; ++I) {
-      const int r0 = 16 * I;
-      const int j = tid >> 4, sl = tid & 15, c8 = 8 * sl;
-      float vv[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) vv[e] = 0.f;
-      float kj[8], g[8];
-      {
-        const uint4 raw = *reinterpret_cast<const uint4 *>(sKr + (r0 + j) * DK + c8);
-        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(p2[e]);
-          kj[2 * e] = f.x;
-          kj[2 * e + 1] = f.y;
+    // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile. A half-warp
+    // owns one row i (lane sl: channels 8 sl .. 8 sl + 7) and walks j = i,
+    // i-1, ... down the sub-block carrying G_{i<-j} (paired fp32); the 16
+    // lanes are then reduced with a reduce-scatter butterfly that leaves
+    // entries 2 sl, 2 sl + 1 of [A row | M row] in lane sl. Warp w takes rows
+    // w mod 8 and 15 - (w mod 8) of two sub-blocks (one per half), so every
+    // warp walks 17 steps.
+    {
+      const int sl = lane & 15, c8 = 8 * sl, rp = warp & 7;
+      const int r0 = 16 * (2 * (warp >> 3) + (lane >> 4));
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int ii = pass ? 15 - rp : rp, i = r0 + ii;
+        uint64_t ki[4], qi[4], g[4];
+        {
+          const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + i * DK + c8);
+          const uint4 qr = *reinterpret_cast<const uint4 *>(sQr + i * DK + c8);
+          ki[0] = bf2_to_f2(kr.x); ki[1] = bf2_to_f2(kr.y);
+          ki[2] = bf2_to_f2(kr.z); ki[3] = bf2_to_f2(kr.w);
+          qi[0] = bf2_to_f2(qr.x); qi[1] = bf2_to_f2(qr.y);
+          qi[2] = bf2_to_f2(qr.z); qi[3] = bf2_to_f2(qr.w);
         }
-      }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) g[e] = 1.f;
+        for (int e = 0; e < 4; ++e) g[e] = f2pack(1.f, 1.f);
+        float vv[32];
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) {
-        if (ii >= j) {
-          const float4 a0 = *reinterpret_cast<const float4 *>(sAl + (r0 + ii) * AL_S + c8);
-          const float4 a1 = *reinterpret_cast<const float4 *>(sAl + (r0 + ii) * AL_S + c8 + 4);
-          const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + (r0 + ii) * DK + c8);
-          const uint4 qr = *reinterpret_cast<const uint4 *>(sQr + (r0 + ii) * DK + c8);
-          const float al[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-          const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-          const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qr);
-          float sa = 0.f, sq = 0.f;
+        for (int e = 0; e < 32; ++e) vv[e] = 0.f;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 kf = __bfloat1622float2(k2[e]), qf = __bfloat1622float2(q2[e]);
-            if (ii > j) {
-              g[2 * e] *= al[2 * e];
-              g[2 * e + 1] *= al[2 * e + 1];
-            }
-            const float x0 = g[2 * e] * kj[2 * e], x1 = g[2 * e + 1] * kj[2 * e + 1];
-            sa += kf.x * x0 + kf.y * x1;
-            sq += qf.x * x0 + qf.y * x1;
+        for (int jj = 15; jj >= 0; --jj) {
+          if (jj <= ii) {
+            const int j = r0 + jj;
+            const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + j * DK + c8);
+            const float4 a0 = *reinterpret_cast<const float4 *>(sAl + al_off(j, c8));
+            const float4 a1 = *reinterpret_cast<const float4 *>(sAl + al_off(j, c8 + 4));
+            const uint64_t x0 = f2mul(g[0], bf2_to_f2(kr.x)), x1 = f2mul(g[1], bf2_to_f2(kr.y));
+            const uint64_t x2 = f2mul(g[2], bf2_to_f2(kr.z)), x3 = f2mul(g[3], bf2_to_f2(kr.w));
+            uint64_t sa = f2mul(ki[0], x0), sq = f2mul(qi[0], x0);
+            sa = f2fma(ki[1], x1, sa); sq = f2fma(qi[1], x1, sq);
+            sa = f2fma(ki[2], x2, sa); sq = f2fma(qi[2], x2, sq);
+            sa = f2fma(ki[3], x3, sa); sq = f2fma(qi[3], x3, sq);
+            const float2 fa = f2unpack(sa), fq = f2unpack(sq);
+            vv[jj] = fa.x + fa.y;
+            vv[16 + jj] = fq.x + fq.y;
+            g[0] = f2mul(g[0], f2pack(a0.x, a0.y));
+            g[1] = f2mul(g[1], f2pack(a0.z, a0.w));
+            g[2] = f2mul(g[2], f2pack(a1.x, a1.y));
+            g[3] = f2mul(g[3], f2pack(a1.z, a1.w));
           }
-          vv[ii] += sa;
-          vv[16 + ii] += sq;
         }
-      }
 #pragma unroll
-      for (int m = 8, nn = 32; m > 0; m >>= 1, nn >>= 1) {
-        const bool up = (sl & m) != 0;
+        for (int m = 8, nn = 32; m > 0; m >>= 1, nn >>= 1) {
+          const bool up = (sl & m) != 0;
 #pragma unroll
-        for (int i = 0; i < nn / 2; ++i) {
-          const float keep = up ? vv[nn / 2 + i] : vv[i];
-          const float send = up ? vv[i] : vv[nn / 2 + i];
-          vv[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+          for (int e = 0; e < nn / 2; ++e) {
+            const float keep = up ? vv[nn / 2 + e] : vv[e];
+            const float send = up ? vv[e] : vv[nn / 2 + e];
+            vv[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+          }
         }
-      }
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int idx = 2 * sl + e, ii = idx & 15;
-        if (idx >= 16) {
-          if (ii >= j) sM[(r0 + ii) * AS + r0 + j] = vv[e];
-        } else if (ii > j) {
-          sA[(r0 + ii) * AS + r0 + j] = sB[r0 + ii] * vv[e];
+        for (int e = 0; e < 2; ++e) {
+          const int idx = 2 * sl + e, jj = idx & 15;
+          if (idx >= 16) {
+            if (jj <= ii) sM[i * RS + r0 + jj] = vv[e];
+          } else if (jj < ii) {
+            sA[i * RS + r0 + jj] = sB[i] * vv[e];
+          }
         }
       }
     }
-    if (!wait_all(&bar[0], 0, s_abort)) break;
-    // off-diagonal blocks out of TMEM: warp quarter qw <-> sub-block row I = qw+1
-    if (warp == 0 || warp == 1 || warp == 6) {
-      const int qw = warp & 3, I = qw + 1, ii = lane & 15, isM = lane >> 4;
-      const int i = 16 * I + ii, off = 8 * I * (I - 1), ncols = 16 * I;
-      const uint32_t ta = tm + lane_base + TP_G + (uint32_t)off;
-      for (int cb = 0; cb < ncols; cb += 16) {
+    if (!wait_all(&bar[0], ph, s_abort)) break;
+
+    // ---------------- 4. off-diagonal Gram blocks out of TMEM; beta Khat |
+    // beta V (B operand of the last MMA, over the consumed Gram operands);
+    // Qhat over alpha (no longer read)
+    {
+      // sub-block row I = qw + 1 sits in lane quarter qw (lanes 0-15 Lk rows,
+      // 16-31 Lq rows); warp part takes columns 16 part .. 16 part + 15
+      const int qw = warp & 3, part = warp >> 2;
+      if (qw < 3 && part <= qw) {
+        const int I = qw + 1, ii = lane & 15, i = 16 * I + ii;
+        const int cb = 16 * part;
         float x[16];
-        tmem_ld16(ta + (uint32_t)cb, x);
+        tmem_ld16(tm + lane_base + TP_G + (uint32_t)(8 * I * (I - 1) + cb), x);
+        const float b = (lane >> 4) ? 1.f : sB[i];
+        float *dst = ((lane >> 4) ? sM : sA) + i * RS + cb;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          if (isM) sM[i * AS + cb + e] = x[e];
-          else sA[i * AS + cb + e] = sB[i] * x[e];
-        }
+        for (int e = 0; e < 16; e += 4)
+          *reinterpret_cast<float4 *>(dst + e) =
+              make_float4(b * x[e], b * x[e + 1], b * x[e + 2], b * x[e + 3]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {  // thread (g, c): gamma_i = pre * p_u
+      const int i = 16 * gq + u;
+      const float gmm = pre * pp[u];
+      const float kk = bf(sKr + i * DK + gc), qq = bf(sQr + i * DK + gc);
+      st_f32(GA + off_mn_sw128b32_f32(i, gc, C), sB[i] * gmm * kk);
+      sAl[al_off(i, gc)] = gmm * qq;  // Qhat (fp32, in place)
+    }
+    {
+      const int nq = DV / 4;
+      for (int task = tid; task < C * nq; task += NTP) {  // beta V columns 128 .. 128+DV
+        const int j = task / nq, g4 = task % nq;
+        const uint2 raw = *reinterpret_cast<const uint2 *>(sm + P_V + task * 8);
+        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+        const float2 x = __bfloat1622float2(p2[0]), y = __bfloat1622float2(p2[1]);
+        const float b = sB[j];
+        st4_f32(GA + off_mn_sw128b32_f32(j, DK + 4 * g4, C), b * x.x, b * x.y, b * y.x, b * y.y);
       }
     }
     fence_before_sync();
-    __syncthreads();
-
-    // ---------------- 4. Kbar^T (to the workspace), beta Khat | beta V, Qhat, gamma
-    if (tid < DK) {
-      const int c = tid;
-      float kb[C];
-      float g = 1.f;
-#pragma unroll
-      for (int b = 3; b >= 0; --b) {  // sigma_j = prod_{s>j} alpha_s, j = 63..0
-        float a[16], kk_[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          a[u] = sAl[(16 * b + u) * AL_S + c];
-          kk_[u] = bf(sKr + (16 * b + u) * DK + c);
-        }
-#pragma unroll
-        for (int u = 15; u >= 0; --u) {
-          kb[16 * b + u] = to_tf32(g * kk_[u]);
-          g *= a[u];
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < C; j += 4)  // row c of Kbar^T (K-major sw128 image)
-        *reinterpret_cast<float4 *>(wsb + WS_A2 + off_k_sw128_f32(c, j, DK)) =
-            make_float4(kb[j], kb[j + 1], kb[j + 2], kb[j + 3]);
-      g = 1.f;
-#pragma unroll 1
-      for (int b = 0; b < 4; ++b) {       // gamma_i = prod_{s<=i} alpha_s
-        float a[16], kk_[16], qq[16], bb[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = 16 * b + u;
-          a[u] = sAl[i * AL_S + c];
-          kk_[u] = bf(sKr + i * DK + c);
-          qq[u] = bf(sQr + i * DK + c);
-          bb[u] = sB[i];
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = 16 * b + u;
-          g *= a[u];
-          st_f32(GA + off_mn_sw128b32_f32(i, c, C), bb[u] * g * kk_[u]);
-          sAl[i * AL_S + c] = g * qq[u];  // Qhat (fp32, in place)
-        }
-      }
-      reinterpret_cast<float *>(wsb + ws_gamma_off(DV))[c] = g;
-    } else {
-      // beta V columns 128 .. 128+DV of the D5 B operand, straight from global
-      const int nq = DV / 4;  // 4-column groups per row
-      for (int task0 = tid - DK; task0 < C * nq; task0 += 16 * (NTP - DK)) {
-        uint2 raw[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int task = task0 + u * (NTP - DK), j = task / nq, g4 = task % nq;
-          raw[u] = make_uint2(0, 0);
-          if (task < C * nq && j < L)
-            raw[u] = __ldg(reinterpret_cast<const uint2 *>(v + ((size_t)(t0 + j) * H + h) * DV + 4 * g4));
-        }
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int task = task0 + u * (NTP - DK), j = task / nq, g4 = task % nq;
-          if (task < C * nq) {
-            const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u]);
-            const float2 x = __bfloat1622float2(p2[0]), y = __bfloat1622float2(p2[1]);
-            const float b = sB[j];
-            st4_f32(GA + off_mn_sw128b32_f32(j, DK + 4 * g4, C), b * x.x, b * x.y, b * y.x, b * y.y);
-          }
-        }
-      }
-    }
+    fence_async_smem();
     __syncthreads();
 
     // ---------------- 5. T = (I + A)^{-1} by blocked forward substitution
+    // diagonal 16x16 blocks: thread (block b, column j), row by row
     if (tid < C) {
       const int b = tid >> 4, j = tid & 15, ob = b * 16;
       float t[16];
@@ -451,34 +513,48 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           float s = 0.f;
 #pragma unroll
           for (int l = 0; l < ii; ++l)
-            if (l >= j) s += sA[(ob + ii) * AS + ob + l] * t[l];
+            if (l >= j) s += sA[(ob + ii) * RS + ob + l] * t[l];
           t[ii] = -s;
         }
       }
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) sT[(ob + ii) * AS + ob + j] = t[ii];
+      for (int ii = 0; ii < 16; ++ii) sT[(ob + ii) * RS + ob + j] = t[ii];
     }
     __syncthreads();
+    // block (I, J = I - d): X = sum_{J <= Lb < I} A_{I,Lb} T_{Lb,J}, then
+    // T_{I,J} = -T_{I,I} X; thread = 2x2 tile (ti, tj) of one block
     for (int d = 1; d < 4; ++d) {
-      for (int idx = tid; idx < (4 - d) * 256; idx += NTP) {
-        const int p = idx >> 8, e = idx & 255, ii = e >> 4, jj = e & 15;
-        const int I = d + p, J = p;
-        float s = 0.f;
-        for (int Lb = J; Lb < I; ++Lb)
+      const int ntask = (4 - d) * 64;
+      const int p = tid >> 6, ti = (tid & 63) >> 3, tj = tid & 7;
+      const int J = p, I = p + d;
+      const int r = 16 * I + 2 * ti, cc = 16 * J + 2 * tj;
+      if (tid < ntask) {
+        float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+        for (int Lb = J; Lb < I; ++Lb) {
 #pragma unroll
-          for (int l = 0; l < 16; ++l)
-            s += sA[(I * 16 + ii) * AS + Lb * 16 + l] * sT[(Lb * 16 + l) * AS + J * 16 + jj];
-        sXT[p * 256 + ii * 16 + jj] = s;
+          for (int l = 0; l < 16; ++l) {
+            const int col = 16 * Lb + l;
+            const float a0 = sA[r * RS + col], a1 = sA[(r + 1) * RS + col];
+            const float2 tv = *reinterpret_cast<const float2 *>(sT + col * RS + cc);
+            x00 += a0 * tv.x; x01 += a0 * tv.y;
+            x10 += a1 * tv.x; x11 += a1 * tv.y;
+          }
+        }
+        *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti) * 16 + 2 * tj) = make_float2(x00, x01);
+        *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti + 1) * 16 + 2 * tj) = make_float2(x10, x11);
       }
       __syncthreads();
-      for (int idx = tid; idx < (4 - d) * 256; idx += NTP) {
-        const int p = idx >> 8, e = idx & 255, ii = e >> 4, jj = e & 15;
-        const int I = d + p, J = p;
-        float s = 0.f;
+      if (tid < ntask) {
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
 #pragma unroll
-        for (int m = 0; m < 16; ++m)
-          if (m <= ii) s += sT[(I * 16 + ii) * AS + I * 16 + m] * sXT[p * 256 + m * 16 + jj];
-        sT[(I * 16 + ii) * AS + J * 16 + jj] = -s;
+        for (int m = 0; m < 16; ++m) {  // T_{I,I} is zero above its diagonal
+          const float t0 = sT[r * RS + 16 * I + m], t1 = sT[(r + 1) * RS + 16 * I + m];
+          const float2 xv = *reinterpret_cast<const float2 *>(sXT + p * 256 + m * 16 + 2 * tj);
+          y00 += t0 * xv.x; y01 += t0 * xv.y;
+          y10 += t1 * xv.x; y11 += t1 * xv.y;
+        }
+        *reinterpret_cast<float2 *>(sT + r * RS + cc) = make_float2(-y00, -y01);
+        *reinterpret_cast<float2 *>(sT + (r + 1) * RS + cc) = make_float2(-y10, -y11);
       }
       __syncthreads();
     }
@@ -487,18 +563,23 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     for (int task = tid; task < 128 * 16; task += NTP) {  // A0 = [M ; I]
       const int row = task >> 4, k4 = (task & 15) * 4;
       float x[4];
+      if (row < C) {
+        const float4 mv = *reinterpret_cast<const float4 *>(sM + row * RS + k4);
+        x[0] = mv.x; x[1] = mv.y; x[2] = mv.z; x[3] = mv.w;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int l = k4 + e;
-        x[e] = (row < C) ? ((l <= row) ? sM[row * AS + l] : 0.f) : ((l == row - C) ? 1.f : 0.f);
+        for (int e = 0; e < 4; ++e) if (k4 + e > row) x[e] = 0.f;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = (k4 + e == row - C) ? 1.f : 0.f;
       }
       st4_f32(sm + P_A0 + off_k_sw128_f32(row, k4, 128), x[0], x[1], x[2], x[3]);
     }
     for (int task = tid; task < C * 16; task += NTP) {  // B0 = T (row l, columns j)
       const int l = task >> 4, j4 = (task & 15) * 4;
-      float x[4];
+      const float4 tv = *reinterpret_cast<const float4 *>(sT + l * RS + j4);
+      float x[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) x[e] = (j4 + e <= l) ? sT[l * AS + j4 + e] : 0.f;
+      for (int e = 0; e < 4; ++e) if (j4 + e > l) x[e] = 0.f;
       st4_f32(sm + P_B0 + off_mn_sw128b32_f32(l, j4, C), x[0], x[1], x[2], x[3]);
     }
     fence_async_smem();
@@ -511,8 +592,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                     desc_mn_sw128b32_f32(sb + P_B0, C, kk), ID_D0, kk > 0);
       mma_commit(&bar[1]);
     }
-    if (!wait_all(&bar[1], 0, s_abort)) break;
-    if ((warp & 3) < 2) {  // rows of M T: round the fp32 accumulator to tf32
+    if (!wait_all(&bar[1], ph, s_abort)) break;
+    if ((warp & 3) < 2 && warp < 8) {  // rows of M T: round the fp32 accumulator to tf32
       const uint32_t ta = tm + lane_base + TP_AD5 + (uint32_t)(32 * (warp >> 2));
       float x[32];
       tmem_ld32(ta, x);
@@ -524,7 +605,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     fence_before_sync();
     __syncthreads();
 
-    // ---------------- 7. [M T ; T] x [beta Khat | beta V] -> workspace
+    // ---------------- 7. [M T ; T] x [beta Khat | beta V], staged, -> workspace
     if (tid == 0) {
       fence_after_sync();
       const uint32_t id5 = idesc_tf32(128, DK + DV, 0, 1);
@@ -534,36 +615,51 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                     desc_mn_sw128b32_f32(sb + P_GA, C, kk), id5, kk > 0);
       mma_commit(&bar[2]);
     }
-    if (!wait_all(&bar[2], 0, s_abort)) break;
+    if (!wait_all(&bar[2], ph, s_abort)) break;
     {
-      const int qw = warp & 3, hw = warp >> 2, row = 32 * qw + lane;
-      if (hw == 0) {  // [Qtil ; W] rows, tf32, K-major sw128 image
-        for (int cb = 0; cb < DK; cb += 32) {
-          float x[32];
-          tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)cb, x);
+      const int qw = warp & 3, cg = warp >> 2, row = 32 * qw + lane;
+      for (int cb = 32 * cg; cb < DK + DV; cb += 128) {
+        float x[32];
+        tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)cb, x);
+        if (cb < DK) {  // [Qtil ; W] rows, tf32, K-major sw128 image
           if (row < C) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = sAl[row * AL_S + cb + e] - x[e];
+            for (int e = 0; e < 32; e += 4) {
+              const float4 qh = *reinterpret_cast<const float4 *>(sAl + al_off(row, cb + e));
+              x[e] = qh.x - x[e]; x[e + 1] = qh.y - x[e + 1];
+              x[e + 2] = qh.z - x[e + 2]; x[e + 3] = qh.w - x[e + 3];
+            }
           }
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4 *>(wsb + WS_A1 + off_k_sw128_f32(row, cb + e, DK)) =
-                make_float4(to_tf32(x[e]), to_tf32(x[e + 1]), to_tf32(x[e + 2]), to_tf32(x[e + 3]));
-        }
-      } else {  // [M Ut ; Ut] rows, fp32 row-major
-        float *dst = reinterpret_cast<float *>(wsb + WS_OU) + (size_t)row * DV;
-        for (int cb = 0; cb < DV; cb += 32) {
-          float x[32];
-          tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)(DK + cb), x);
+            st4_f32(sm + P_GA + off_k_sw128_f32(row, cb + e, DK), x[e], x[e + 1], x[e + 2], x[e + 3]);
+        } else {  // [M Ut ; Ut] rows, fp32, pieces swizzled by row
+          uint8_t *dst = sm + P_OU + (size_t)row * DV * 4;
+          const int pc0 = (cb - DK) >> 2;
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4 *>(dst + cb + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+            *reinterpret_cast<float4 *>(dst + 16 * ou_piece(row, pc0 + (e >> 2))) =
+                make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
         }
       }
     }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_s2g(wsb + WS_A1, sm + P_GA, 65536);
+      bulk_s2g(wsb + WS_OU, sm + P_OU, 128u * DV * 4u);
+      bulk_commit();
+    }
   } while (0);
+  if (*s_abort) break;  // CTA-uniform: read after a barrier
+  ph ^= 1u;
+  cur = nxt;
+  }  // item loop
 
-  if (*s_abort && tid == 0) flag_error(err, kErrMbarTimeout);
+  if (tid == 0) {
+    if (*s_abort) flag_error(err, kErrMbarTimeout);
+    bulk_wait_read0();  // shared memory stays valid until the stores read it
+  }
   fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -649,10 +745,10 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   float ou_next[DVT], gc_next = 0.f;
   auto load_rows = [&](int c) {
     const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
-    const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV + c0;
+    const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV;
 #pragma unroll
     for (int e = 0; e < DVT; e += 4) {
-      const float4 x = __ldg(reinterpret_cast<const float4 *>(src + e));
+      const float4 x = __ldg(reinterpret_cast<const float4 *>(src + 4 * ou_piece(tid, (c0 + e) >> 2)));
       ou_next[e] = x.x; ou_next[e + 1] = x.y; ou_next[e + 2] = x.z; ou_next[e + 3] = x.w;
     }
     gc_next = __ldg(reinterpret_cast<const float *>(blk + ws_gamma_off(DV)) + tid);
@@ -770,7 +866,23 @@ bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt) {
 
 size_t fwd_tc_workspace_bytes(int N, int T_total, int H, int dv) {
   const size_t slots = (size_t)T_total / C + (size_t)N;
-  return slots * (size_t)H * ws_block_bytes(dv);
+  return slot_table_off(slots, (size_t)H, dv) + slot_table_bytes(slots);
+}
+
+// SM count of the current device (looked up once per device).
+static int sm_count() {
+  static std::mutex mu;
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
 }
 
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
@@ -788,9 +900,17 @@ cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
   if (e != cudaSuccess) return e;
   const int slots = T_total / C + N;
   if (slots > 0 && T_total > 0) {
-    ckda_chunk_prep_kernel<<<dim3(slots, H), NTP, P_SMEM, st>>>(
+    int2 *tab = reinterpret_cast<int2 *>((uint8_t *)ws + slot_table_off(slots, H, dv));
+    ckda_slot_table_kernel<<<(slots + 255) / 256, 256, 0, st>>>(cu, N, T, T_total, slots,
+                                                               tab, err);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const long long items = (long long)slots * H;
+    if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int grid = (int)std::min<long long>(items, (long long)sm_count());
+    ckda_chunk_prep_kernel<<<grid, NTP, P_SMEM, st>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-        alpha, beta, cu, N, T, T_total, H, dv, (uint8_t *)ws, err);
+        alpha, beta, tab, (int)items, H, dv, (uint8_t *)ws, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -292,15 +292,58 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32
       : "memory");
 }
 
-// Bulk prefetch of [p, p + bytes) into L2 (16-byte aligned, bytes % 16 == 0).
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes)
+// Bulk copy shared (this CTA) -> global, tracked in this thread's bulk
+// async-group. Both addresses 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_s2g(void *dst, const void *src_smem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src_smem)), "r"(bytes)
                : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until every bulk store this thread committed has finished reading its
+// shared-memory source (the source may then be overwritten).
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Prefetch the cache line holding p into L2 (no data returned).
+__device__ __forceinline__ void prefetch_line_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (MMA).
 __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ------------------------------------------------------------ packed fp32 pairs
+// Two fp32 values in one 64-bit register pair, for the sm_100 paired fp32
+// instructions (each rounds like its scalar form).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+// a bf16 pair (element 0 in the low half) -> the fp32 pair (exact)
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t w) {
+  return f2pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
 // 8 floats -> 8 bf16 packed in 16 bytes.

@@ -91,6 +91,9 @@ def _alpha(kind: str, shape, g: torch.Generator) -> torch.Tensor:
         a = torch.where((u >= 0.025) & (u < 0.05), -torch.ones_like(a), a)
         a = torch.where((u >= 0.05) & (u < 0.06), torch.zeros_like(a), a)
         return a
+    if kind == "slow":  # long memory: |alpha| = 1 - 0.01 |N(0,1)|, 10% negative
+        a = 1.0 - 0.01 * x.abs()
+        return torch.where(u < 0.1, -a, a)
     raise ValueError(kind)
 
 

@@ -96,11 +96,17 @@ def test_fwd_rejects(lib, kw, want):
 
 def test_workspace_query(lib):
     # tensor-core path (bf16, d_k=128, chunk 64): one block per (slot, head)
+    # plus a table of 8 bytes per slot (rounded up to 1 KB);
     # 1 sequence of 64 tokens: floor(64/64) + 1 = 2 chunk slots
-    block = ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 128) // 2
+    def table(slots):
+        return (slots * 8 + 1023) // 1024 * 1024
+    block = (ckda.ckda_fwd_workspace_bytes(1, 64, 2, 128, 128)
+             - ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 128)) // 2
     assert block > 0 and block % 1024 == 0
-    assert ckda.ckda_fwd_workspace_bytes(2, 8192, 32, 128, 128) == (2 * 8192 // 64 + 2) * 32 * block
-    assert ckda.ckda_fwd_workspace_bytes(1, 100, 1, 128, 128, varlen=True) == 2 * block
+    assert ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 128) == 2 * block + table(2)
+    slots = 2 * 8192 // 64 + 2
+    assert ckda.ckda_fwd_workspace_bytes(2, 8192, 32, 128, 128) == slots * 32 * block + table(slots)
+    assert ckda.ckda_fwd_workspace_bytes(1, 100, 1, 128, 128, varlen=True) == 2 * block + table(2)
     assert ckda.ckda_fwd_workspace_bytes(1, 64, 1, 128, 32) < 2 * block
     # CUDA-core path and unsupported arguments need none
     assert ckda.ckda_fwd_workspace_bytes(1, 64, 1, 64, 64) == 0

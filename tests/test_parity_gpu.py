@@ -181,6 +181,18 @@ def test_bf16_ragged_small(cuda_lib):
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
 
 
+def test_bf16_long_memory_gates(cuda_lib):
+    """bf16 path with |alpha| close to 1 and 10% negative gates: the gate
+    products over a whole chunk stay O(1), so every row of every chunk
+    reaches the output and the final state (full, partial and short chunks)."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=515, alpha_kind="slow")
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([64, 1000, 130, 7]), H=4)
+    o, sf = run_fwd(inp, chunk=64)
+    o_ref, sf_ref = ref_fwd(inp)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
 def test_split_resume_equals_single_call(cuda_lib):
     """fwd(x[:a]) then fwd(x[a:], init = final) equals fwd(x): the state is
     the checkpoint (chunk-to-chunk carry). fp32 mode, split mid-chunk."""
