@@ -674,7 +674,7 @@ constexpr uint32_t S_A1 = 0;          // 2 x 65536 [Qtil ; W] buffers
 constexpr uint32_t S_A2 = 131072;     // 2 x 32768 Kbar^T buffers
 constexpr uint32_t S_S = 196608;      // 16384 S, B of D1 (K128 x N32 MN)
 constexpr uint32_t S_U = 212992;      //  8192 U, B of D2 (K64 x N32 MN)
-constexpr uint32_t S_BAR = 221184;    //    64 mbarriers [0..2] + TMEM address + flag
+constexpr uint32_t S_BAR = 221184;    //    64 mbarriers [0..3] + TMEM address + flag
 constexpr uint32_t S_SMEM = 221248 + 1024;
 constexpr uint32_t TS_D1 = 0, TS_D2 = 32, TS_COLS = 64;
 constexpr uint32_t ID_D1 = idesc_tf32(128, 32, 0, 1);
@@ -690,7 +690,7 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S_BAR);  // [0..1] loads, [2] MMAs
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S_BAR);  // [0..1] loads, [2] D1, [3] D2
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + S_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + S_BAR + 36);
 
@@ -703,14 +703,15 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   const int base = slot_base(cu, n, T);
   const size_t st_base = ((size_t)n * H + h) * DK * DV;
   const uint32_t wsz = ws_block_bytes(DV);
+  // Thread ISS (first thread of the U half) issues the copies and the MMAs.
+  constexpr int ISS = C;
 
   if (warp == 0) {
     tmem_alloc(s_tmem, TS_COLS);
     tmem_relinquish();
   }
-  if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
-    *s_abort = 0;
+  if (tid == ISS) {
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
     if (nch > 0) {  // chunk 0 into buffer 0
       const uint8_t *blk = ws + ((size_t)base * H + h) * wsz;
@@ -719,6 +720,7 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
       bulk_g2s(sm + S_A2, blk + WS_A2, 32768, &bar[0]);
     }
   }
+  if (tid == 0) *s_abort = 0;
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -755,27 +757,29 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   };
   if (nch > 0) load_rows(0);
 
+  // Per chunk one CTA barrier (the state tile is complete in shared memory);
+  // the U half hands D2 over through named barrier 1 while the output half
+  // stores O. A timed-out wait only sets the abort flag, read after the
+  // chunk's CTA barrier.
   for (int c = 0; c < nch; ++c) {
     const int buf = c & 1;
     const int t0 = bos + C * c, L = min(C, eos - t0);
-    // next chunk's operands into the other buffer (free: chunk c-1 is done)
-    if (tid == 0 && c + 1 < nch) {
-      const uint8_t *nb = ws + ((size_t)(base + c + 1) * H + h) * wsz;
-      mbar_arrive_expect_tx(&bar[buf ^ 1], LOAD_BYTES);
-      bulk_g2s(sm + S_A1 + (buf ^ 1) * 65536, nb + WS_A1, 65536, &bar[buf ^ 1]);
-      bulk_g2s(sm + S_A2 + (buf ^ 1) * 32768, nb + WS_A2, 32768, &bar[buf ^ 1]);
-    }
     float ou[DVT];
 #pragma unroll
     for (int e = 0; e < DVT; ++e) ou[e] = ou_next[e];
     const float gc = gc_next;
     if (c + 1 < nch) load_rows(c + 1);
-    if (!mbar_wait(&bar[buf], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
-    __syncthreads();
-    if (*s_abort) break;
 
-    // D1 = [Qtil ; W] x S
-    if (tid == 0) {
+    if (tid == ISS) {
+      // next chunk's operands into the other buffer (free: chunk c-1 is done)
+      if (c + 1 < nch) {
+        const uint8_t *nb = ws + ((size_t)(base + c + 1) * H + h) * wsz;
+        mbar_arrive_expect_tx(&bar[buf ^ 1], LOAD_BYTES);
+        bulk_g2s(sm + S_A1 + (buf ^ 1) * 65536, nb + WS_A1, 65536, &bar[buf ^ 1]);
+        bulk_g2s(sm + S_A2 + (buf ^ 1) * 32768, nb + WS_A2, 32768, &bar[buf ^ 1]);
+      }
+      // D1 = [Qtil ; W] x S once this chunk's operands have landed
+      if (!mbar_wait(&bar[buf], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < DK / 8; ++kk)
@@ -783,43 +787,43 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
                     desc_mn_sw128b32_f32(sb + S_S, DK, kk), ID_D1, kk > 0);
       mma_commit(&bar[2]);
     }
-    if (!wait_all(&bar[2], 0, s_abort)) break;
-    {
-      float d1[32];
-      tmem_ld32(tm + lane_base + TS_D1, d1);
-      if (tid < C) {  // output rows
-        const int i = tid;
-        if (i < L) {
-          __nv_bfloat16 *dst = o + ((size_t)(t0 + i) * H + h) * DV + c0;
+    // D1 and D2 complete once per chunk each, on their own mbarriers, so no
+    // thread can fall a full phase behind the one it waits for
+    if (!mbar_wait(&bar[2], (uint32_t)c & 1u)) *s_abort = 1;
+    fence_after_sync();
+    float d1[32];
+    tmem_ld32(tm + lane_base + TS_D1, d1);
+    if (tid >= C) {  // U = Ut - W S, then D2 = Kbar^T x U
+      const int j = tid - C;
 #pragma unroll
-          for (int g8 = 0; g8 < 4; ++g8) {
-            float y[8];
+      for (int e = 0; e < DVT; e += 4)
+        st4_f32(sm + S_U + off_mn_sw128b32_f32(j, e, C), ou[e] - d1[e], ou[e + 1] - d1[e + 1],
+                ou[e + 2] - d1[e + 2], ou[e + 3] - d1[e + 3]);
+      fence_async_smem();
+      named_bar_sync(1, NTS - C);
+      if (tid == ISS) {
+        fence_after_sync();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = scale * (d1[8 * g8 + e] + ou[8 * g8 + e]);
-            *reinterpret_cast<uint4 *>(dst + 8 * g8) = pack8_bf16(y);
-          }
+        for (int kk = 0; kk < C / 8; ++kk)
+          mma_tf32_ss(tm + TS_D2, desc_k_sw128_f32(sb + S_A2 + buf * 32768, 128, kk),
+                      desc_mn_sw128b32_f32(sb + S_U, C, kk), ID_D2, kk > 0);
+        mma_commit(&bar[3]);
+      }
+    } else {  // output rows, while D2 runs
+      const int i = tid;
+      if (i < L) {
+        __nv_bfloat16 *dst = o + ((size_t)(t0 + i) * H + h) * DV + c0;
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = scale * (d1[8 * g8 + e] + ou[8 * g8 + e]);
+          *reinterpret_cast<uint4 *>(dst + 8 * g8) = pack8_bf16(y);
         }
-      } else {  // U = Ut - W S
-        const int j = tid - C;
-#pragma unroll
-        for (int e = 0; e < DVT; e += 4)
-          st4_f32(sm + S_U + off_mn_sw128b32_f32(j, e, C), ou[e] - d1[e], ou[e + 1] - d1[e + 1],
-                  ou[e + 2] - d1[e + 2], ou[e + 3] - d1[e + 3]);
       }
     }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    // D2 = Kbar^T x U
-    if (tid == 0) {
-      fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < C / 8; ++kk)
-        mma_tf32_ss(tm + TS_D2, desc_k_sw128_f32(sb + S_A2 + buf * 32768, 128, kk),
-                    desc_mn_sw128b32_f32(sb + S_U, C, kk), ID_D2, kk > 0);
-      mma_commit(&bar[2]);
-    }
-    if (!wait_all(&bar[2], 1, s_abort)) break;
+    if (!mbar_wait(&bar[3], (uint32_t)c & 1u)) *s_abort = 1;
+    fence_after_sync();
     {
       float d2[32];
       tmem_ld32(tm + lane_base + TS_D2, d2);
@@ -832,13 +836,14 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
+    if (*s_abort) break;
   }
 
   if (*s_abort) {
     if (tid == 0) flag_error(err, kErrMbarTimeout);
     // let in-flight copies and MMAs drain (bounded) before shared memory and
     // tensor memory are released
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
       (void)mbar_wait(&bar[i], 0, 100000000LL);
       (void)mbar_wait(&bar[i], 1, 100000000LL);
     }
