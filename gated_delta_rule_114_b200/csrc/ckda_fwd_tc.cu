@@ -669,14 +669,26 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
 }
 
 // ---------------------------------------------------------------- scan kernel
-constexpr int NTS = 128;
-constexpr uint32_t S_A1 = 0;          // 2 x 65536 [Qtil ; W] buffers
-constexpr uint32_t S_A2 = 131072;     // 2 x 32768 Kbar^T buffers
+// 4 consumer warps (thread r = state row r of the 128 x 32 tile) and one
+// producer warp. The producer bulk-copies each chunk's [Qtil ; W] and Kbar^T
+// images into a shared-memory landing buffer two chunks ahead and moves them
+// into tensor memory (tcgen05.cp, 128 lanes x 8 columns per K-step), so both
+// MMAs of the state chain take their A operand from tensor memory and read
+// only the small B operand (S or U) from shared memory.
+constexpr int NTS = 160, NCONS = 128;
+constexpr uint32_t S_A1 = 0;          // 2 x 65536 [Qtil ; W] landing buffers
+constexpr uint32_t S_A2 = 131072;     // 2 x 32768 Kbar^T landing buffers
 constexpr uint32_t S_S = 196608;      // 16384 S, B of D1 (K128 x N32 MN)
 constexpr uint32_t S_U = 212992;      //  8192 U, B of D2 (K64 x N32 MN)
-constexpr uint32_t S_BAR = 221184;    //    64 mbarriers [0..3] + TMEM address + flag
-constexpr uint32_t S_SMEM = 221248 + 1024;
-constexpr uint32_t TS_D1 = 0, TS_D2 = 32, TS_COLS = 64;
+constexpr uint32_t S_BAR = 221184;    //   128 mbarriers [0..9] + TMEM address + flag
+constexpr uint32_t S_SMEM = 221312 + 1024;
+// mbarriers: landed[2] (bulk copy into landing buffer b), ready[2] (buffer b
+// in tensor memory), free[2] (the MMAs that read tensor-memory buffer b are
+// done), D1, D2. Each completes once per use of its buffer or chunk, and no
+// waiter can be two completions behind, so parity waits are exact.
+enum { B_LANDED = 0, B_READY = 2, B_FREE = 4, B_D1 = 6, B_D2 = 7, NBAR = 8 };
+// tensor memory: D1, D2 accumulators; [Qtil ; W] and Kbar^T, two buffers each
+constexpr uint32_t TS_D1 = 0, TS_D2 = 32, TS_A1 = 64, TS_A2 = 320, TS_COLS = 512;
 constexpr uint32_t ID_D1 = idesc_tf32(128, 32, 0, 1);
 constexpr uint32_t ID_D2 = idesc_tf32(128, 32, 0, 1);
 constexpr uint32_t LOAD_BYTES = 65536 + 32768;
@@ -690,11 +702,11 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(sm);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S_BAR);  // [0..1] loads, [2] D1, [3] D2
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + S_BAR + 32);
-  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + S_BAR + 36);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + S_BAR);
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + S_BAR + 8 * NBAR);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(sm + S_BAR + 8 * NBAR + 4);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int vt = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
   const int c0 = vt * DVT;
   int bos, eos;
@@ -703,159 +715,198 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   const int base = slot_base(cu, n, T);
   const size_t st_base = ((size_t)n * H + h) * DK * DV;
   const uint32_t wsz = ws_block_bytes(DV);
-  // Thread ISS (first thread of the U half) issues the copies and the MMAs.
+  // Consumer thread ISS (first thread of the U half) issues the MMAs.
   constexpr int ISS = C;
+  constexpr int PROD = NCONS;  // producer thread (lane 0 of warp 4)
 
   if (warp == 0) {
     tmem_alloc(s_tmem, TS_COLS);
     tmem_relinquish();
   }
-  if (tid == ISS) {
-    for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
+  if (tid == PROD) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(&bar[i], 1);
     fence_mbar_init();
-    if (nch > 0) {  // chunk 0 into buffer 0
-      const uint8_t *blk = ws + ((size_t)base * H + h) * wsz;
-      mbar_arrive_expect_tx(&bar[0], LOAD_BYTES);
-      bulk_g2s(sm + S_A1, blk + WS_A1, 65536, &bar[0]);
-      bulk_g2s(sm + S_A2, blk + WS_A2, 32768, &bar[0]);
-    }
   }
   if (tid == 0) *s_abort = 0;
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tm = *s_tmem;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
 
-  // state row r = tid of the 128 x 32 tile, fp32 in registers
-  float S[DVT];
-  {
-    const int r = tid;
-#pragma unroll
-    for (int e = 0; e < DVT; e += 4) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (s0) x = *reinterpret_cast<const float4 *>(s0 + st_base + (size_t)r * DV + c0 + e);
-      S[e] = x.x; S[e + 1] = x.y; S[e + 2] = x.z; S[e + 3] = x.w;
-      st4_f32(sm + S_S + off_mn_sw128b32_f32(r, e, DK), x.x, x.y, x.z, x.w);
-    }
-  }
-  fence_async_smem();
-  __syncthreads();
-
-  // this thread's row of [M Ut ; Ut] (d_v tile) and gamma of its state row,
-  // read one chunk ahead so the loads overlap the previous chunk's MMAs
-  float ou_next[DVT], gc_next = 0.f;
-  auto load_rows = [&](int c) {
-    const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
-    const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV;
-#pragma unroll
-    for (int e = 0; e < DVT; e += 4) {
-      const float4 x = __ldg(reinterpret_cast<const float4 *>(src + 4 * ou_piece(tid, (c0 + e) >> 2)));
-      ou_next[e] = x.x; ou_next[e + 1] = x.y; ou_next[e + 2] = x.z; ou_next[e + 3] = x.w;
-    }
-    gc_next = __ldg(reinterpret_cast<const float *>(blk + ws_gamma_off(DV)) + tid);
-  };
-  if (nch > 0) load_rows(0);
-
-  // Per chunk one CTA barrier (the state tile is complete in shared memory);
-  // the U half hands D2 over through named barrier 1 while the output half
-  // stores O. A timed-out wait only sets the abort flag, read after the
-  // chunk's CTA barrier.
-  for (int c = 0; c < nch; ++c) {
-    const int buf = c & 1;
-    const int t0 = bos + C * c, L = min(C, eos - t0);
-    float ou[DVT];
-#pragma unroll
-    for (int e = 0; e < DVT; ++e) ou[e] = ou_next[e];
-    const float gc = gc_next;
-    if (c + 1 < nch) load_rows(c + 1);
-
-    if (tid == ISS) {
-      // next chunk's operands into the other buffer (free: chunk c-1 is done)
-      if (c + 1 < nch) {
-        const uint8_t *nb = ws + ((size_t)(base + c + 1) * H + h) * wsz;
-        mbar_arrive_expect_tx(&bar[buf ^ 1], LOAD_BYTES);
-        bulk_g2s(sm + S_A1 + (buf ^ 1) * 65536, nb + WS_A1, 65536, &bar[buf ^ 1]);
-        bulk_g2s(sm + S_A2 + (buf ^ 1) * 32768, nb + WS_A2, 32768, &bar[buf ^ 1]);
-      }
-      // D1 = [Qtil ; W] x S once this chunk's operands have landed
-      if (!mbar_wait(&bar[buf], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
-      fence_after_sync();
-#pragma unroll
-      for (int kk = 0; kk < DK / 8; ++kk)
-        mma_tf32_ss(tm + TS_D1, desc_k_sw128_f32(sb + S_A1 + buf * 65536, 128, kk),
-                    desc_mn_sw128b32_f32(sb + S_S, DK, kk), ID_D1, kk > 0);
-      mma_commit(&bar[2]);
-    }
-    // D1 and D2 complete once per chunk each, on their own mbarriers, so no
-    // thread can fall a full phase behind the one it waits for
-    if (!mbar_wait(&bar[2], (uint32_t)c & 1u)) *s_abort = 1;
-    fence_after_sync();
-    float d1[32];
-    tmem_ld32(tm + lane_base + TS_D1, d1);
-    if (tid >= C) {  // U = Ut - W S, then D2 = Kbar^T x U
-      const int j = tid - C;
-#pragma unroll
-      for (int e = 0; e < DVT; e += 4)
-        st4_f32(sm + S_U + off_mn_sw128b32_f32(j, e, C), ou[e] - d1[e], ou[e + 1] - d1[e + 1],
-                ou[e + 2] - d1[e + 2], ou[e + 3] - d1[e + 3]);
-      fence_async_smem();
-      named_bar_sync(1, NTS - C);
-      if (tid == ISS) {
+  if (warp == NCONS / 32) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      auto load = [&](int c) {
+        const int b = c & 1;
+        const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
+        mbar_arrive_expect_tx(&bar[B_LANDED + b], LOAD_BYTES);
+        bulk_g2s(sm + S_A1 + b * 65536, blk + WS_A1, 65536, &bar[B_LANDED + b]);
+        bulk_g2s(sm + S_A2 + b * 32768, blk + WS_A2, 32768, &bar[B_LANDED + b]);
+      };
+      if (nch > 0) load(0);
+      if (nch > 1) load(1);
+      for (int c = 0; c < nch; ++c) {
+        const int b = c & 1;
+        const uint32_t use = (uint32_t)(c >> 1);  // how often buffer b was used before
+        bool ok = mbar_wait(&bar[B_LANDED + b], use & 1u);
+        if (ok && c >= 2) ok = mbar_wait(&bar[B_FREE + b], (use - 1) & 1u);
+        if (!ok) {
+          *s_abort = 1;
+          break;
+        }
         fence_after_sync();
 #pragma unroll
+        for (int kk = 0; kk < DK / 8; ++kk)
+          tmem_cp_128x256b(tm + TS_A1 + b * 128 + 8 * kk,
+                           desc_k_sw128_f32(sb + S_A1 + b * 65536, 128, kk));
+#pragma unroll
         for (int kk = 0; kk < C / 8; ++kk)
-          mma_tf32_ss(tm + TS_D2, desc_k_sw128_f32(sb + S_A2 + buf * 32768, 128, kk),
-                      desc_mn_sw128b32_f32(sb + S_U, C, kk), ID_D2, kk > 0);
-        mma_commit(&bar[3]);
-      }
-    } else {  // output rows, while D2 runs
-      const int i = tid;
-      if (i < L) {
-        __nv_bfloat16 *dst = o + ((size_t)(t0 + i) * H + h) * DV + c0;
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-          float y[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = scale * (d1[8 * g8 + e] + ou[8 * g8 + e]);
-          *reinterpret_cast<uint4 *>(dst + 8 * g8) = pack8_bf16(y);
+          tmem_cp_128x256b(tm + TS_A2 + b * 64 + 8 * kk,
+                           desc_k_sw128_f32(sb + S_A2 + b * 32768, 128, kk));
+        mma_commit(&bar[B_READY + b]);
+        if (c + 2 < nch) {  // landing buffer b again, once the copies have read it
+          if (!mbar_wait(&bar[B_READY + b], use & 1u)) {
+            *s_abort = 1;
+            break;
+          }
+          load(c + 2);
         }
+        if (*s_abort) break;
       }
     }
-    if (!mbar_wait(&bar[3], (uint32_t)c & 1u)) *s_abort = 1;
-    fence_after_sync();
+  } else {
+    // ------------------------------------------------------------ consumers
+    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
+    // state row r = tid of the 128 x 32 tile, fp32 in registers
+    float S[DVT];
     {
-      float d2[32];
-      tmem_ld32(tm + lane_base + TS_D2, d2);
+      const int r = tid;
 #pragma unroll
-      for (int e = 0; e < DVT; ++e) S[e] = gc * S[e] + d2[e];
-#pragma unroll
-      for (int e = 0; e < DVT; e += 4)
-        st4_f32(sm + S_S + off_mn_sw128b32_f32(tid, e, DK), S[e], S[e + 1], S[e + 2], S[e + 3]);
+      for (int e = 0; e < DVT; e += 4) {
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (s0) x = *reinterpret_cast<const float4 *>(s0 + st_base + (size_t)r * DV + c0 + e);
+        S[e] = x.x; S[e + 1] = x.y; S[e + 2] = x.z; S[e + 3] = x.w;
+        st4_f32(sm + S_S + off_mn_sw128b32_f32(r, e, DK), x.x, x.y, x.z, x.w);
+      }
     }
     fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    if (*s_abort) break;
+    named_bar_sync(2, NCONS);
+
+    // this thread's row of [M Ut ; Ut] (d_v tile) and gamma of its state row,
+    // read one chunk ahead so the loads overlap the previous chunk's MMAs
+    float ou_next[DVT], gc_next = 0.f;
+    auto load_rows = [&](int c) {
+      const uint8_t *blk = ws + ((size_t)(base + c) * H + h) * wsz;
+      const float *src = reinterpret_cast<const float *>(blk + WS_OU) + (size_t)tid * DV;
+#pragma unroll
+      for (int e = 0; e < DVT; e += 4) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(src + 4 * ou_piece(tid, (c0 + e) >> 2)));
+        ou_next[e] = x.x; ou_next[e + 1] = x.y; ou_next[e + 2] = x.z; ou_next[e + 3] = x.w;
+      }
+      gc_next = __ldg(reinterpret_cast<const float *>(blk + ws_gamma_off(DV)) + tid);
+    };
+    if (nch > 0) load_rows(0);
+
+    // Per chunk one barrier of the consumers (the state tile is complete in
+    // shared memory); the U half hands D2 over through named barrier 1 while
+    // the output half stores O. A timed-out wait only sets the abort flag,
+    // read after the chunk's barrier.
+    for (int c = 0; c < nch; ++c) {
+      const int b = c & 1;
+      const int t0 = bos + C * c, L = min(C, eos - t0);
+      float ou[DVT];
+#pragma unroll
+      for (int e = 0; e < DVT; ++e) ou[e] = ou_next[e];
+      const float gc = gc_next;
+      if (c + 1 < nch) load_rows(c + 1);
+
+      if (tid == ISS) {  // D1 = [Qtil ; W] x S, A from tensor memory
+        if (!mbar_wait(&bar[B_READY + b], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < DK / 8; ++kk)
+          mma_tf32_ts(tm + TS_D1, tm + TS_A1 + b * 128 + 8 * kk,
+                      desc_mn_sw128b32_f32(sb + S_S, DK, kk), ID_D1, kk > 0);
+        mma_commit(&bar[B_D1]);
+      }
+      if (!mbar_wait(&bar[B_D1], (uint32_t)c & 1u)) *s_abort = 1;
+      fence_after_sync();
+      float d1[32];
+      tmem_ld32(tm + lane_base + TS_D1, d1);
+      if (tid >= C) {  // U = Ut - W S, then D2 = Kbar^T x U
+        const int j = tid - C;
+#pragma unroll
+        for (int e = 0; e < DVT; e += 4)
+          st4_f32(sm + S_U + off_mn_sw128b32_f32(j, e, C), ou[e] - d1[e], ou[e + 1] - d1[e + 1],
+                  ou[e + 2] - d1[e + 2], ou[e + 3] - d1[e + 3]);
+        fence_async_smem();
+        named_bar_sync(1, NCONS - C);
+        if (tid == ISS) {
+          fence_after_sync();
+#pragma unroll
+          for (int kk = 0; kk < C / 8; ++kk)
+            mma_tf32_ts(tm + TS_D2, tm + TS_A2 + b * 64 + 8 * kk,
+                        desc_mn_sw128b32_f32(sb + S_U, C, kk), ID_D2, kk > 0);
+          mma_commit(&bar[B_D2]);
+          mma_commit(&bar[B_FREE + b]);  // tensor-memory buffer b may be refilled
+        }
+      } else {  // output rows, while D2 runs
+        const int i = tid;
+        if (i < L) {
+          __nv_bfloat16 *dst = o + ((size_t)(t0 + i) * H + h) * DV + c0;
+#pragma unroll
+          for (int g8 = 0; g8 < 4; ++g8) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = scale * (d1[8 * g8 + e] + ou[8 * g8 + e]);
+            *reinterpret_cast<uint4 *>(dst + 8 * g8) = pack8_bf16(y);
+          }
+        }
+      }
+      if (!mbar_wait(&bar[B_D2], (uint32_t)c & 1u)) *s_abort = 1;
+      fence_after_sync();
+      {
+        float d2[32];
+        tmem_ld32(tm + lane_base + TS_D2, d2);
+#pragma unroll
+        for (int e = 0; e < DVT; ++e) S[e] = gc * S[e] + d2[e];
+#pragma unroll
+        for (int e = 0; e < DVT; e += 4)
+          st4_f32(sm + S_S + off_mn_sw128b32_f32(tid, e, DK), S[e], S[e + 1], S[e + 2], S[e + 3]);
+      }
+      fence_async_smem();
+      fence_before_sync();
+      named_bar_sync(2, NCONS);
+      if (*s_abort) break;
+    }
+    // the last two buffer-free commits are never waited for by the producer:
+    // let their arrivals land before shared memory is released
+    if (tid == ISS && !*s_abort) {
+      for (int c = max(nch - 2, 0); c < nch; ++c)
+        if (!mbar_wait(&bar[B_FREE + (c & 1)], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
+    }
+    if (!*s_abort && sfin) {
+      const int r = tid;
+#pragma unroll
+      for (int e = 0; e < DVT; e += 4)
+        *reinterpret_cast<float4 *>(sfin + st_base + (size_t)r * DV + c0 + e) =
+            make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    }
   }
 
+  fence_before_sync();
+  __syncthreads();
   if (*s_abort) {
     if (tid == 0) flag_error(err, kErrMbarTimeout);
     // let in-flight copies and MMAs drain (bounded) before shared memory and
     // tensor memory are released
-    for (int i = 0; i < 4; ++i) {
-      (void)mbar_wait(&bar[i], 0, 100000000LL);
-      (void)mbar_wait(&bar[i], 1, 100000000LL);
-    }
-  } else if (sfin) {
-    const int r = tid;
-#pragma unroll
-    for (int e = 0; e < DVT; e += 4)
-      *reinterpret_cast<float4 *>(sfin + st_base + (size_t)r * DV + c0 + e) =
-          make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    if (tid == PROD)
+      for (int i = 0; i < NBAR; ++i) {
+        (void)mbar_wait(&bar[i], 0, 100000000LL);
+        (void)mbar_wait(&bar[i], 1, 100000000LL);
+      }
+    __syncthreads();
   }
-  fence_before_sync();
-  __syncthreads();
   if (warp == 0) {
     fence_after_sync();
     tmem_dealloc(tm, TS_COLS);

@@ -147,7 +147,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
       "r"(m3));
 }
 
-// Arrive on an mbarrier when every MMA issued so far by this thread is done.
+// Copy a 128-row x 256-bit (8 x 32-bit) matrix from shared memory, described
+// like an MMA operand, into 128 lanes x 8 columns of tensor memory (lane =
+// row). Completion is tracked by tcgen05.commit like an MMA.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Arrive on an mbarrier when every MMA (or tensor-memory copy) issued so far
+// by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t *mbar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
