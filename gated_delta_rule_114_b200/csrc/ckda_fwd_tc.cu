@@ -120,10 +120,10 @@ __global__ void ckda_slot_table_kernel(const int32_t *__restrict__ cu, int N, in
 // MN-major form tcgen05 accepts for 32-bit elements).
 constexpr int NTP = 512;
 constexpr int RS = 68;                // fp32 row stride of A, M, T (16-byte aligned rows)
-constexpr uint32_t P_GA = 0;          // 65536 Lk/Lq (96 rows x 128, K-major)
-                                      //   -> [beta Khat | beta V] (K64 x N(128+dv), MN)
+constexpr uint32_t P_GA = 0;          // 65536 Lk/Lq (M128 x K128, MN-major; rows 96.. unused)
+                                      //   -> [beta Khat | beta V] (N(128+dv) x K64, K-major)
                                       //   -> staged [Qtil ; W] image (epilogue)
-constexpr uint32_t P_GB = 49152;      // 49152 R stack (96 rows x 128, K-major)
+constexpr uint32_t P_GB = 49152;      // 49152 R stack (N96 x K128, MN-major)
 constexpr uint32_t P_A0 = 65536;      // 32768 [M ; I] (128 x 64 K-major)
 constexpr uint32_t P_OU = 65536;      // <=65536 staged [M Ut ; Ut] rows (epilogue)
 constexpr uint32_t P_V = 98304;       // 16384 raw v bf16 [64][dv] (until beta V is built)
@@ -145,13 +145,10 @@ constexpr uint32_t TP_AD5 = 96;   //  64 [M T ; T] (A of D5)
 constexpr uint32_t TP_D5 = 160;   // 256 [M W | M Ut ; W | Ut]
 constexpr uint32_t TP_COLS = 512;
 
-constexpr uint32_t ID_G = idesc_tf32(128, 96, 0, 0);
+constexpr uint32_t ID_G = idesc_tf32(128, 96, 1, 1);
 constexpr uint32_t ID_D0 = idesc_tf32(128, 64, 0, 1);
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
-__device__ __forceinline__ void st_f32(uint8_t *p, float x) {
-  *reinterpret_cast<float *>(p) = to_tf32(x);
-}
 __device__ __forceinline__ void st4_f32(uint8_t *p, float a, float b, float c, float d) {
   *reinterpret_cast<float4 *>(p) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
@@ -347,13 +344,20 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         if (b < gq) pre *= P[b];
         if (b > gq) suf *= P[b];
       }
+      // Gram operands are MN-major (rows contiguous): a thread's 16 rows of
+      // one channel are four 16-byte stores
       if (gq >= 1) {
+        float lk[16], lq[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
           const int i = 16 * gq + u;
-          const float kk = bf(sKr + i * DK + gc), qq = bf(sQr + i * DK + gc);
-          st_f32(GA + off_k_sw128_f32((gq - 1) * 32 + u, gc, 96), pp[u] * kk);
-          st_f32(GA + off_k_sw128_f32((gq - 1) * 32 + 16 + u, gc, 96), pp[u] * qq);
+          lk[u] = pp[u] * bf(sKr + i * DK + gc);
+          lq[u] = pp[u] * bf(sQr + i * DK + gc);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; u += 4) {
+          st4_f32(GA + off_mn_sw128b32_f32(gc, (gq - 1) * 32 + u, DK), lk[u], lk[u + 1], lk[u + 2], lk[u + 3]);
+          st4_f32(GA + off_mn_sw128b32_f32(gc, (gq - 1) * 32 + 16 + u, DK), lq[u], lq[u + 1], lq[u + 2], lq[u + 3]);
         }
       }
       float f = 1.f;
@@ -362,8 +366,9 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         if (I > gq) {
           if (I > gq + 1) f *= P[I - 1];
 #pragma unroll
-          for (int u = 0; u < 16; ++u)
-            st_f32(GB + off_k_sw128_f32(8 * I * (I - 1) + 16 * gq + u, gc, 96), f * kr[u]);
+          for (int u = 0; u < 16; u += 4)
+            st4_f32(GB + off_mn_sw128b32_f32(gc, 8 * I * (I - 1) + 16 * gq + u, DK),
+                    f * kr[u], f * kr[u + 1], f * kr[u + 2], f * kr[u + 3]);
         }
       }
 #pragma unroll
@@ -381,8 +386,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
       fence_after_sync();
 #pragma unroll
       for (int kk = 0; kk < DK / 8; ++kk)
-        mma_tf32_ss(tm + TP_G, desc_k_sw128_f32(sb + P_GA, 96, kk),
-                    desc_k_sw128_f32(sb + P_GB, 96, kk), ID_G, kk > 0);
+        mma_tf32_ss(tm + TP_G, desc_mn_sw128b32_f32(sb + P_GA, DK, kk),
+                    desc_mn_sw128b32_f32(sb + P_GB, DK, kk), ID_G, kk > 0);
       mma_commit(&bar[0]);
     }
     // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile. A half-warp
@@ -477,23 +482,30 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
               make_float4(b * x[e], b * x[e + 1], b * x[e + 2], b * x[e + 3]);
       }
     }
+    // The last MMA's B operand [beta Khat | beta V] is K-major (row n =
+    // output column, 4 tokens per 16-byte store), 128 + DV rows.
+    {
+      float bk[16];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) {  // thread (g, c): gamma_i = pre * p_u
-      const int i = 16 * gq + u;
-      const float gmm = pre * pp[u];
-      const float kk = bf(sKr + i * DK + gc), qq = bf(sQr + i * DK + gc);
-      st_f32(GA + off_mn_sw128b32_f32(i, gc, C), sB[i] * gmm * kk);
-      sAl[al_off(i, gc)] = gmm * qq;  // Qhat (fp32, in place)
+      for (int u = 0; u < 16; ++u) {  // thread (g, c): gamma_i = pre * p_u
+        const int i = 16 * gq + u;
+        const float gmm = pre * pp[u];
+        const float kk = bf(sKr + i * DK + gc), qq = bf(sQr + i * DK + gc);
+        bk[u] = sB[i] * gmm * kk;
+        sAl[al_off(i, gc)] = gmm * qq;  // Qhat (fp32, in place)
+      }
+#pragma unroll
+      for (int u = 0; u < 16; u += 4)
+        st4_f32(GA + off_k_sw128_f32(gc, 16 * gq + u, DK + DV), bk[u], bk[u + 1], bk[u + 2], bk[u + 3]);
     }
     {
-      const int nq = DV / 4;
-      for (int task = tid; task < C * nq; task += NTP) {  // beta V columns 128 .. 128+DV
-        const int j = task / nq, g4 = task % nq;
-        const uint2 raw = *reinterpret_cast<const uint2 *>(sm + P_V + task * 8);
-        const __nv_bfloat162 *p2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-        const float2 x = __bfloat1622float2(p2[0]), y = __bfloat1622float2(p2[1]);
-        const float b = sB[j];
-        st4_f32(GA + off_mn_sw128b32_f32(j, DK + 4 * g4, C), b * x.x, b * x.y, b * y.x, b * y.y);
+      const __nv_bfloat16 *sV = reinterpret_cast<const __nv_bfloat16 *>(sm + P_V);
+      for (int task = tid; task < DV * (C / 4); task += NTP) {  // beta V rows 128 .. 128+DV
+        const int cv = task % DV, j4 = 4 * (task / DV);
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = sB[j4 + e] * bf(sV + (j4 + e) * DV + cv);
+        st4_f32(GA + off_k_sw128_f32(DK + cv, j4, DK + DV), x[0], x[1], x[2], x[3]);
       }
     }
     fence_before_sync();
@@ -608,11 +620,11 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     // ---------------- 7. [M T ; T] x [beta Khat | beta V], staged, -> workspace
     if (tid == 0) {
       fence_after_sync();
-      const uint32_t id5 = idesc_tf32(128, DK + DV, 0, 1);
+      const uint32_t id5 = idesc_tf32(128, DK + DV, 0, 0);
 #pragma unroll
       for (int kk = 0; kk < C / 8; ++kk)
         mma_tf32_ts(tm + TP_D5, tm + TP_AD5 + (uint32_t)(8 * kk),
-                    desc_mn_sw128b32_f32(sb + P_GA, C, kk), id5, kk > 0);
+                    desc_k_sw128_f32(sb + P_GA, DK + DV, kk), id5, kk > 0);
       mma_commit(&bar[2]);
     }
     if (!wait_all(&bar[2], ph, s_abort)) break;
