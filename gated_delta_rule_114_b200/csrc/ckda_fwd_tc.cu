@@ -124,13 +124,14 @@ constexpr uint32_t P_GA = 0;          // 65536 Lk/Lq (M128 x K128, MN-major; row
                                       //   -> [beta Khat | beta V] (N(128+dv) x K64, K-major)
                                       //   -> staged [Qtil ; W] image (epilogue)
 constexpr uint32_t P_GB = 49152;      // 49152 R stack (N96 x K128, MN-major)
-constexpr uint32_t P_A0 = 65536;      // 32768 [M ; I] (128 x 64 K-major)
+constexpr uint32_t P_T = 65536;       // 17408 T fp32 [64][68] (after the Grams)
+constexpr uint32_t P_XT = P_T + 17408; //  3072 solve scratch
 constexpr uint32_t P_OU = 65536;      // <=65536 staged [M Ut ; Ut] rows (epilogue)
 constexpr uint32_t P_V = 98304;       // 16384 raw v bf16 [64][dv] (until beta V is built)
 constexpr uint32_t P_B0 = 98304;      // 16384 T (K64 x N64 MN)
-constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128] -> T fp32 [64][68]
-constexpr uint32_t P_K = 131072;      // 16384 raw k bf16 [64][128]    (T spills in)
-constexpr uint32_t P_XT = P_K + 4096; //  3072 solve scratch (after raw k is dead)
+constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128]
+constexpr uint32_t P_K = 131072;      // 16384 raw k bf16 [64][128]
+constexpr uint32_t P_A0 = 114688;     // 32768 [M ; I] (128 x 64 K-major), over raw q and k
 constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
 constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68]
 constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
@@ -187,7 +188,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   float *sAl = reinterpret_cast<float *>(sm + P_AL);
   float *sA = reinterpret_cast<float *>(sm + P_A);
   float *sM = reinterpret_cast<float *>(sm + P_M);
-  float *sT = reinterpret_cast<float *>(sm + P_Q);
+  float *sT = reinterpret_cast<float *>(sm + P_T);
   float *sXT = reinterpret_cast<float *>(sm + P_XT);
   float *sB = reinterpret_cast<float *>(sm + P_B);
   float *sP = reinterpret_cast<float *>(sm + P_P);
@@ -462,9 +463,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     }
     if (!wait_all(&bar[0], ph, s_abort)) break;
 
-    // ---------------- 4. off-diagonal Gram blocks out of TMEM; beta Khat |
-    // beta V (B operand of the last MMA, over the consumed Gram operands);
-    // Qhat over alpha (no longer read)
+    // ---------------- 4. off-diagonal Gram blocks out of TMEM; gamma over
+    // alpha (no longer read)
     {
       // sub-block row I = qw + 1 sits in lane quarter qw (lanes 0-15 Lk rows,
       // 16-31 Lq rows); warp part takes columns 16 part .. 16 part + 15
@@ -482,25 +482,89 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
               make_float4(b * x[e], b * x[e + 1], b * x[e + 2], b * x[e + 3]);
       }
     }
-    // The last MMA's B operand [beta Khat | beta V] is K-major (row n =
-    // output column, 4 tokens per 16-byte store), 128 + DV rows.
-    {
-      float bk[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {  // thread (g, c): gamma_i = pre * p_u
-        const int i = 16 * gq + u;
-        const float gmm = pre * pp[u];
-        const float kk = bf(sKr + i * DK + gc), qq = bf(sQr + i * DK + gc);
-        bk[u] = sB[i] * gmm * kk;
-        sAl[al_off(i, gc)] = gmm * qq;  // Qhat (fp32, in place)
+    for (int u = 0; u < 16; ++u) sAl[al_off(16 * gq + u, gc)] = pre * pp[u];  // gamma_i
+    fence_before_sync();
+    __syncthreads();
+
+    if (warp < NTP / 64) {  // warps 0..7 invert; named barrier 1 among them
+      // ---------------- 5. T = (I + A)^{-1} by blocked forward substitution
+      // diagonal 16x16 blocks: thread (block b, column j), row by row
+      if (tid < C) {
+        const int b = tid >> 4, j = tid & 15, ob = b * 16;
+        float t[16];
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) t[ii] = (ii == j) ? 1.f : 0.f;
+#pragma unroll
+        for (int ii = 1; ii < 16; ++ii) {
+          if (ii > j) {
+            float s = 0.f;
+#pragma unroll
+            for (int l = 0; l < ii; ++l)
+              if (l >= j) s += sA[(ob + ii) * RS + ob + l] * t[l];
+            t[ii] = -s;
+          }
+        }
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) sT[(ob + ii) * RS + ob + j] = t[ii];
       }
+      named_bar_sync(1, NTP / 2);
+      // block (I, J = I - d): X = sum_{J <= Lb < I} A_{I,Lb} T_{Lb,J}, then
+      // T_{I,J} = -T_{I,I} X; thread = 2x2 tile (ti, tj) of one block
+      for (int d = 1; d < 4; ++d) {
+        const int ntask = (4 - d) * 64;
+        const int p = tid >> 6, ti = (tid & 63) >> 3, tj = tid & 7;
+        const int J = p, I = p + d;
+        const int r = 16 * I + 2 * ti, cc = 16 * J + 2 * tj;
+        if (tid < ntask) {
+          float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+          for (int Lb = J; Lb < I; ++Lb) {
 #pragma unroll
-      for (int u = 0; u < 16; u += 4)
-        st4_f32(GA + off_k_sw128_f32(gc, 16 * gq + u, DK + DV), bk[u], bk[u + 1], bk[u + 2], bk[u + 3]);
-    }
-    {
+            for (int l = 0; l < 16; ++l) {
+              const int col = 16 * Lb + l;
+              const float a0 = sA[r * RS + col], a1 = sA[(r + 1) * RS + col];
+              const float2 tv = *reinterpret_cast<const float2 *>(sT + col * RS + cc);
+              x00 += a0 * tv.x; x01 += a0 * tv.y;
+              x10 += a1 * tv.x; x11 += a1 * tv.y;
+            }
+          }
+          *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti) * 16 + 2 * tj) = make_float2(x00, x01);
+          *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti + 1) * 16 + 2 * tj) = make_float2(x10, x11);
+        }
+        named_bar_sync(1, NTP / 2);
+        if (tid < ntask) {
+          float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+          for (int m = 0; m < 16; ++m) {  // T_{I,I} is zero above its diagonal
+            const float t0 = sT[r * RS + 16 * I + m], t1 = sT[(r + 1) * RS + 16 * I + m];
+            const float2 xv = *reinterpret_cast<const float2 *>(sXT + p * 256 + m * 16 + 2 * tj);
+            y00 += t0 * xv.x; y01 += t0 * xv.y;
+            y10 += t1 * xv.x; y11 += t1 * xv.y;
+          }
+          *reinterpret_cast<float2 *>(sT + r * RS + cc) = make_float2(-y00, -y01);
+          *reinterpret_cast<float2 *>(sT + (r + 1) * RS + cc) = make_float2(-y10, -y11);
+        }
+        named_bar_sync(1, NTP / 2);
+      }
+    } else {
+      // ---------------- 5'. meanwhile (warps 8..15): the last MMA's B operand
+      // [beta Khat | beta V], K-major (row n = output column, 4 tokens per
+      // 16-byte store, 128 + DV rows), and Qhat over gamma
+      const int t = tid - NTP / 2, c = t & (DK - 1), i0 = 32 * (t >> 7);
+#pragma unroll
+      for (int u = 0; u < 32; u += 4) {
+        float bk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = i0 + u + e;
+          const float gmm = sAl[al_off(i, c)];
+          bk[e] = sB[i] * gmm * bf(sKr + i * DK + c);
+          sAl[al_off(i, c)] = gmm * bf(sQr + i * DK + c);  // Qhat (fp32, in place)
+        }
+        st4_f32(GA + off_k_sw128_f32(c, i0 + u, DK + DV), bk[0], bk[1], bk[2], bk[3]);
+      }
       const __nv_bfloat16 *sV = reinterpret_cast<const __nv_bfloat16 *>(sm + P_V);
-      for (int task = tid; task < DV * (C / 4); task += NTP) {  // beta V rows 128 .. 128+DV
+      for (int task = t; task < DV * (C / 4); task += NTP / 2) {  // beta V rows 128 .. 128+DV
         const int cv = task % DV, j4 = 4 * (task / DV);
         float x[4];
 #pragma unroll
@@ -508,68 +572,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         st4_f32(GA + off_k_sw128_f32(DK + cv, j4, DK + DV), x[0], x[1], x[2], x[3]);
       }
     }
-    fence_before_sync();
-    fence_async_smem();
     __syncthreads();
-
-    // ---------------- 5. T = (I + A)^{-1} by blocked forward substitution
-    // diagonal 16x16 blocks: thread (block b, column j), row by row
-    if (tid < C) {
-      const int b = tid >> 4, j = tid & 15, ob = b * 16;
-      float t[16];
-#pragma unroll
-      for (int ii = 0; ii < 16; ++ii) t[ii] = (ii == j) ? 1.f : 0.f;
-#pragma unroll
-      for (int ii = 1; ii < 16; ++ii) {
-        if (ii > j) {
-          float s = 0.f;
-#pragma unroll
-          for (int l = 0; l < ii; ++l)
-            if (l >= j) s += sA[(ob + ii) * RS + ob + l] * t[l];
-          t[ii] = -s;
-        }
-      }
-#pragma unroll
-      for (int ii = 0; ii < 16; ++ii) sT[(ob + ii) * RS + ob + j] = t[ii];
-    }
-    __syncthreads();
-    // block (I, J = I - d): X = sum_{J <= Lb < I} A_{I,Lb} T_{Lb,J}, then
-    // T_{I,J} = -T_{I,I} X; thread = 2x2 tile (ti, tj) of one block
-    for (int d = 1; d < 4; ++d) {
-      const int ntask = (4 - d) * 64;
-      const int p = tid >> 6, ti = (tid & 63) >> 3, tj = tid & 7;
-      const int J = p, I = p + d;
-      const int r = 16 * I + 2 * ti, cc = 16 * J + 2 * tj;
-      if (tid < ntask) {
-        float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-        for (int Lb = J; Lb < I; ++Lb) {
-#pragma unroll
-          for (int l = 0; l < 16; ++l) {
-            const int col = 16 * Lb + l;
-            const float a0 = sA[r * RS + col], a1 = sA[(r + 1) * RS + col];
-            const float2 tv = *reinterpret_cast<const float2 *>(sT + col * RS + cc);
-            x00 += a0 * tv.x; x01 += a0 * tv.y;
-            x10 += a1 * tv.x; x11 += a1 * tv.y;
-          }
-        }
-        *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti) * 16 + 2 * tj) = make_float2(x00, x01);
-        *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti + 1) * 16 + 2 * tj) = make_float2(x10, x11);
-      }
-      __syncthreads();
-      if (tid < ntask) {
-        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {  // T_{I,I} is zero above its diagonal
-          const float t0 = sT[r * RS + 16 * I + m], t1 = sT[(r + 1) * RS + 16 * I + m];
-          const float2 xv = *reinterpret_cast<const float2 *>(sXT + p * 256 + m * 16 + 2 * tj);
-          y00 += t0 * xv.x; y01 += t0 * xv.y;
-          y10 += t1 * xv.x; y11 += t1 * xv.y;
-        }
-        *reinterpret_cast<float2 *>(sT + r * RS + cc) = make_float2(-y00, -y01);
-        *reinterpret_cast<float2 *>(sT + (r + 1) * RS + cc) = make_float2(-y10, -y11);
-      }
-      __syncthreads();
-    }
 
     // ---------------- 6. [M T ; T] = [M ; I] x T on the tensor cores, into TMEM
     for (int task = tid; task < 128 * 16; task += NTP) {  // A0 = [M ; I]
