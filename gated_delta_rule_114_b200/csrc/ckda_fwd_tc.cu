@@ -608,13 +608,13 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
       mma_commit(&bar[1]);
     }
     if (!wait_all(&bar[1], ph, s_abort)) break;
-    if ((warp & 3) < 2 && warp < 8) {  // rows of M T: round the fp32 accumulator to tf32
-      const uint32_t ta = tm + lane_base + TP_AD5 + (uint32_t)(32 * (warp >> 2));
-      float x[32];
-      tmem_ld32(ta, x);
+    if ((warp & 3) < 2) {  // rows of M T: round the fp32 accumulator to tf32
+      const uint32_t ta = tm + lane_base + TP_AD5 + (uint32_t)(16 * (warp >> 2));
+      float x[16];
+      tmem_ld16(ta, x);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) x[e] = to_tf32(x[e]);
-      tmem_st32(ta, x);
+      for (int e = 0; e < 16; ++e) x[e] = to_tf32(x[e]);
+      tmem_st16(ta, x);
     }
     tmem_wait_st();
     fence_before_sync();

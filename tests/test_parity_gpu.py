@@ -181,6 +181,19 @@ def test_bf16_ragged_small(cuda_lib):
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
 
 
+@pytest.mark.parametrize("d_k,d_v,chunk", [(128, 32, 64), (128, 64, 64), (64, 64, 64),
+                                           (128, 128, 32), (32, 128, 16)])
+def test_bf16_shapes_ragged(cuda_lib, d_k, d_v, chunk):
+    """bf16 I/O on every d_v the tensor-core path takes (d_k=128, chunk 64)
+    and on the CUDA-core fallback (other d_k or chunk), ragged lengths."""
+    w = custom("ckda_B1_H32_T8192_d128", d_k=d_k, d_v=d_v, seed=7000 + d_k + d_v + chunk)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([200, 64, 1, 130, 0, 77]), H=3)
+    o, sf = run_fwd(inp, chunk=chunk, scale=0.75)
+    o_ref, sf_ref = ref_fwd(inp, scale=0.75)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
 def test_bf16_long_memory_gates(cuda_lib):
     """bf16 path with |alpha| close to 1 and 10% negative gates: the gate
     products over a whole chunk stay O(1), so every row of every chunk
