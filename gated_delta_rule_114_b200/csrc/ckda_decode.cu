@@ -29,7 +29,7 @@ struct DecodeShape {
 };
 
 template <int DK, int DV, int DVS, typename IOT>
-__global__ void __launch_bounds__(DecodeShape<DK, DVS>::THREADS)
+__global__ void __launch_bounds__(DecodeShape<DK, DVS>::THREADS, 4)
 decode_step_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
                    const IOT *__restrict__ v, const float *__restrict__ alpha,
                    const float *__restrict__ beta, float *__restrict__ state,
