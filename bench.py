@@ -33,7 +33,8 @@ sys.path.insert(0, ROOT)
 from gated_delta_rule_114_b200 import ckda  # noqa: E402
 from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,  # noqa: E402
                                               make_decode_tokens,
-                                              make_fwd_inputs)
+                                              make_fwd_inputs,
+                                              make_gated_fwd_inputs)
 
 METRIC = ("CKDA prefill tokens/s (H=32, d=128, T=8192) + % bf16 roofline; "
           "decode tok/s, HBM GB/s")
@@ -95,6 +96,18 @@ def prefill_flops(inp, C=64) -> float:
         for c in [C] * full + ([rem] if rem else []):
             mac += 2.5 * c * c * d + 3 * c * d * d + c ** 3 / 6.0
     return 2.0 * mac * H
+
+
+def prefill_gated_bytes(inp) -> int:
+    """Algorithmic HBM bytes of one forward with the fused input prologue:
+    q, k_raw, v, a_logit (I/O dtype), c_logit (fp32), o per token-head; states."""
+    T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[2]
+    es = esize(inp["q"].dtype)
+    per_th = (3 * dk + dv) * es + 4 + dv * es
+    N = inp["cu_seqlens"].numel() - 1
+    st = N * H * dk * dv * 4
+    return T * H * per_th + (st if inp["initial_state"] is not None else 0) + st
 
 
 def decode_bytes(N, H, dk, dv, dt) -> int:
@@ -350,6 +363,29 @@ def main():
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": e2e_ms}
 
+    # ---------------- the same workload through the fused input prologue
+    ginp = make_gated_fwd_inputs(w)
+    gdev = {key: (val.cuda() if isinstance(val, torch.Tensor) else val)
+            for key, val in ginp.items()}
+    gates = ckda.GateParams(**ckda.CKDA_GATES, k_eps=1e-6)
+
+    def prefill_gated():
+        ckda.ckda_fwd_chunked_gated(gdev["q"], gdev["k_raw"], gdev["v"], gdev["a_logit"],
+                                    gdev["c_logit"], gdev["initial_state"], sf, o, gates,
+                                    gdev["cu_seqlens"], None, chunk=w.chunk,
+                                    stream=stream, workspace=ws)
+
+    gms = time_loop(prefill_gated, args.steps, args.warmup, stream, barrier)
+    gbytes = prefill_gated_bytes(ginp)
+    gated = {"ms_per_step": gms, "tokens_per_s": T_total * world / (gms / 1e3),
+             "roofline": {"bound": "hbm", "achieved": gbytes / (gms / 1e3) / 1e9,
+                          "peak": pk["hbm_gbs"], "unit": "GB/s",
+                          "frac": gbytes / (gms / 1e3) / 1e9 / pk["hbm_gbs"],
+                          "traffic": None, "algorithmic_bytes_per_launch": gbytes},
+             "inputs": "bf16 q, raw k, v, gate logits a; fp32 logits c; CKDA ranges",
+             "gpu_launches": 3 * args.steps}
+    del gdev
+
     # ---------------- decode step
     wd = WORKLOADS[DECODE]
     state = make_decode_state(wd).cuda()
@@ -400,6 +436,7 @@ def main():
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         # each forward call launches the slot-table, prep and scan kernels
         "gpu_launches": 3 * args.steps, "clocks": clk.summary(), "decode": decode,
+        "prefill_fused_prologue": gated,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -26,6 +26,18 @@ _DT = {torch.bfloat16: CKDA_BF16, torch.float32: CKDA_F32}
 _lib = None
 
 
+class GateParams(ctypes.Structure):
+    """ckda_gate_params (include/ckda.h): the fused input prologue's
+    alpha = alpha_min + (alpha_max - alpha_min) sigmoid(a),
+    beta = beta_max sigmoid(c), k = k_raw / (||k_raw|| + k_eps)."""
+    _fields_ = [("alpha_min", ctypes.c_float), ("alpha_max", ctypes.c_float),
+                ("beta_max", ctypes.c_float), ("k_eps", ctypes.c_float)]
+
+
+CKDA_GATES = dict(alpha_min=-1.0, alpha_max=1.0, beta_max=2.0)  # CKDA ranges
+KDA_GATES = dict(alpha_min=0.0, alpha_max=1.0, beta_max=1.0)    # KDA ranges
+
+
 class CkdaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -59,6 +71,14 @@ def load(path: str | None = None):
     lib.ckda_decode_step.restype = ctypes.c_int
     lib.ckda_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
                                      i32, f32, ctypes.c_int, vp]
+    lib.ckda_fwd_chunked_gated.restype = ctypes.c_int
+    lib.ckda_fwd_chunked_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                           i32, i32, i32, i32, i32, i32, f32,
+                                           ctypes.c_int, GateParams, vp,
+                                           ctypes.c_size_t, vp]
+    lib.ckda_decode_step_gated.restype = ctypes.c_int
+    lib.ckda_decode_step_gated.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32,
+                                           i32, f32, ctypes.c_int, GateParams, vp]
     lib.ckda_status_string.restype = ctypes.c_char_p
     lib.ckda_status_string.argtypes = [ctypes.c_int]
     lib.ckda_last_error.restype = ctypes.c_int
@@ -123,11 +143,31 @@ def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
     workspace: optional uint8 CUDA tensor of at least ckda_fwd_workspace_bytes
     bytes; allocated with torch here when it is needed and not given.
     """
+    _fwd_call(q, k, v, alpha, beta, initial_state, final_state, o, cu_seqlens,
+              cu_seqlens_host, N, T, chunk, scale, stream, workspace, None)
+
+
+def ckda_fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, initial_state, final_state,
+                           o, gates: GateParams, cu_seqlens=None, cu_seqlens_host=None,
+                           N=None, T=None, chunk: int = 0, scale: float = 1.0,
+                           stream=None, workspace=None):
+    """Marshal tensors into ckda_fwd_chunked_gated (fused input prologue).
+
+    As ckda_fwd_chunked with k_raw (unnormalised keys), a_logit
+    [T_total, H, d_k] in q's dtype and c_logit [T_total, H] fp32 in place of
+    k, alpha and beta; `gates` is a GateParams."""
+    _fwd_call(q, k_raw, v, a_logit, c_logit, initial_state, final_state, o, cu_seqlens,
+              cu_seqlens_host, N, T, chunk, scale, stream, workspace, gates)
+
+
+def _fwd_call(q, k, v, alpha, beta, initial_state, final_state, o, cu_seqlens,
+              cu_seqlens_host, N, T, chunk, scale, stream, workspace, gates):
     lib = load()
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, nme, q.dtype, 3)
-    _need(alpha, "alpha", torch.float32, 3)
-    _need(beta, "beta", torch.float32, 2)
+    _need(alpha, "a_logit" if gates is not None else "alpha",
+          q.dtype if gates is not None else torch.float32, 3)
+    _need(beta, "c_logit" if gates is not None else "beta", torch.float32, 2)
     if q.dtype not in _DT:
         raise ValueError("q, k, v, o must be bfloat16 or float32")
     T_total, H, d_k = q.shape
@@ -152,13 +192,16 @@ def ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, final_state, o,
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.ckda_fwd_chunked(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
-                              _p(initial_state), _p(final_state), _p(o),
-                              _p(cu_seqlens), host_ptr, int(N), int(T), int(H),
-                              int(d_k), int(d_v), int(chunk), float(scale),
-                              _DT[q.dtype], _p(workspace), ws_bytes,
-                              _stream(stream))
-    _check(st, "ckda_fwd_chunked")
+    args = (_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(initial_state),
+            _p(final_state), _p(o), _p(cu_seqlens), host_ptr, int(N), int(T), int(H),
+            int(d_k), int(d_v), int(chunk), float(scale), _DT[q.dtype])
+    if gates is None:
+        st = lib.ckda_fwd_chunked(*args, _p(workspace), ws_bytes, _stream(stream))
+        _check(st, "ckda_fwd_chunked")
+    else:
+        st = lib.ckda_fwd_chunked_gated(*args, gates, _p(workspace), ws_bytes,
+                                        _stream(stream))
+        _check(st, "ckda_fwd_chunked_gated")
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # CKDA_NOALLOC_SCRATCH_BYTES in include/ckda.h
@@ -214,21 +257,35 @@ def ckda_decode_step(q, k, v, alpha, beta, state, o, scale: float = 1.0,
     q, k [N, H, d_k]; v, o [N, H, d_v] (bf16 or fp32); alpha [N, H, d_k] fp32;
     beta [N, H] fp32; state [N, H, d_k, d_v] fp32.
     """
+    _decode_call(q, k, v, alpha, beta, state, o, scale, stream, None)
+
+
+def ckda_decode_step_gated(q, k_raw, v, a_logit, c_logit, state, o, gates: GateParams,
+                           scale: float = 1.0, stream=None):
+    """Marshal tensors into ckda_decode_step_gated (fused input prologue):
+    k_raw [N, H, d_k], a_logit [N, H, d_k] in q's dtype, c_logit [N, H] fp32."""
+    _decode_call(q, k_raw, v, a_logit, c_logit, state, o, scale, stream, gates)
+
+
+def _decode_call(q, k, v, alpha, beta, state, o, scale, stream, gates):
     lib = load()
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, nme, q.dtype, 3)
-    _need(alpha, "alpha", torch.float32, 3)
-    _need(beta, "beta", torch.float32, 2)
+    _need(alpha, "a_logit" if gates is not None else "alpha",
+          q.dtype if gates is not None else torch.float32, 3)
+    _need(beta, "c_logit" if gates is not None else "beta", torch.float32, 2)
     _need(state, "state", torch.float32, 4)
     if q.dtype not in _DT:
         raise ValueError("q, k, v, o must be bfloat16 or float32")
     N, H, d_k = q.shape
     d_v = v.shape[2]
-    st = lib.ckda_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta),
-                              _p(state), _p(o), int(N), int(H), int(d_k),
-                              int(d_v), float(scale), _DT[q.dtype],
-                              _stream(stream))
-    _check(st, "ckda_decode_step")
+    args = (_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(state), _p(o), int(N), int(H),
+            int(d_k), int(d_v), float(scale), _DT[q.dtype])
+    if gates is None:
+        _check(lib.ckda_decode_step(*args, _stream(stream)), "ckda_decode_step")
+    else:
+        _check(lib.ckda_decode_step_gated(*args, gates, _stream(stream)),
+               "ckda_decode_step_gated")
 
 
 def ckda_last_error(stream=None) -> int:
@@ -257,6 +314,26 @@ def fwd_chunked(q, k, v, alpha, beta, initial_state=None, cu_seqlens=None,
         sf = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=q.device)
     ckda_fwd_chunked(q, k, v, alpha, beta, initial_state, sf, o, cu_seqlens,
                      cu_seqlens_host, N, T, chunk, scale, stream, workspace)
+    return o, sf
+
+
+def fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, gates: GateParams,
+                      initial_state=None, cu_seqlens=None, cu_seqlens_host=None,
+                      N=None, T=None, chunk: int = 0, scale: float = 1.0,
+                      stream=None, workspace=None):
+    """Allocate o and the final state with torch, then call
+    ckda_fwd_chunked_gated."""
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+    elif N is None:
+        N, T = 1, T_total
+    o = torch.empty((T_total, H, d_v), dtype=q.dtype, device=q.device)
+    sf = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=q.device)
+    ckda_fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, initial_state, sf, o, gates,
+                           cu_seqlens, cu_seqlens_host, N, T, chunk, scale, stream,
+                           workspace)
     return o, sf
 
 

@@ -8,25 +8,27 @@
 #include "ckda_common.cuh"
 
 namespace ckda {
+// With g.on, `alpha` points to the gate logits a (I/O element type), `beta`
+// to the fp32 logits c and `k` to the raw keys (the fused input prologue).
 template <typename IOT>
 cudaError_t launch_decode(int dk, int dv, const void *q, const void *k,
-                          const void *v, const float *alpha, const float *beta,
+                          const void *v, const void *alpha, const float *beta,
                           float *state, void *o, int N, int H, float scale,
-                          cudaStream_t st);
+                          GateArgs g, cudaStream_t st);
 template <typename IOT>
 cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
-                            const void *k, const void *v, const float *alpha,
+                            const void *k, const void *v, const void *alpha,
                             const float *beta, const float *s0, float *sf,
                             void *o, const int32_t *cu, int N, int T,
-                            int T_total, int H, float scale, unsigned int *err,
-                            cudaStream_t st);
+                            int T_total, int H, float scale, GateArgs g,
+                            unsigned int *err, cudaStream_t st);
 bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt);
 size_t fwd_tc_workspace_bytes(int N, int T_total, int H, int dv);
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
-                          const float *alpha, const float *beta,
+                          const void *alpha, const float *beta,
                           const float *s0, float *sf, void *o,
                           const int32_t *cu, int N, int T, int T_total, int H,
-                          float scale, void *ws, unsigned int *err,
+                          float scale, GateArgs g, void *ws, unsigned int *err,
                           cudaStream_t st);
 }  // namespace ckda
 
@@ -68,6 +70,39 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 }
 
 size_t esize(ckda_dtype dt) { return dt == CKDA_F32 ? 4 : 2; }
+
+bool finite(float x) { return x == x && x - x == 0.f; }
+
+// ckda_gate_params -> kernel arguments; false if outside the documented ranges
+bool gate_args(const ckda_gate_params &gp, ckda::GateArgs &g) {
+  if (!finite(gp.alpha_min) || !finite(gp.alpha_max) || !finite(gp.beta_max) ||
+      !finite(gp.k_eps))
+    return false;
+  if (gp.alpha_min < -1.f || gp.alpha_max > 1.f || gp.alpha_min > gp.alpha_max) return false;
+  if (gp.beta_max < 0.f || gp.beta_max > 2.f || gp.k_eps < 0.f) return false;
+  g.on = 1;
+  g.amin = gp.alpha_min;
+  g.arange = gp.alpha_max - gp.alpha_min;
+  g.bmax = gp.beta_max;
+  g.keps = gp.k_eps;
+  return true;
+}
+
+// The forward behind both entry points; with g.on, alpha is the logits a
+// (element size es) and beta the logits c.
+ckda_status fwd_impl(const void *q, const void *k, const void *v,
+                     const void *alpha, const float *beta,
+                     const float *initial_state, float *final_state, void *o,
+                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                     int32_t N, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                     int32_t chunk, float scale, ckda_dtype dt, ckda::GateArgs g,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+ckda_status decode_impl(const void *q, const void *k, const void *v,
+                        const void *alpha, const float *beta, float *state,
+                        void *o, int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                        float scale, ckda_dtype dt, ckda::GateArgs g,
+                        cudaStream_t stream);
 
 }  // namespace
 
@@ -118,6 +153,59 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
                              int32_t chunk, float scale, ckda_dtype dt,
                              void *workspace, size_t workspace_bytes,
                              cudaStream_t stream) {
+  return fwd_impl(q, k, v, alpha, beta, initial_state, final_state, o, cu_seqlens,
+                  cu_seqlens_host, N, T, H, d_k, d_v, chunk, scale, dt,
+                  ckda::GateArgs{0, 0.f, 0.f, 0.f, 0.f}, workspace, workspace_bytes, stream);
+}
+
+ckda_status ckda_fwd_chunked_gated(const void *q, const void *k_raw, const void *v,
+                                   const void *a_logit, const float *c_logit,
+                                   const float *initial_state, float *final_state,
+                                   void *o, const int32_t *cu_seqlens,
+                                   const int32_t *cu_seqlens_host, int32_t N,
+                                   int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                   int32_t chunk, float scale, ckda_dtype dt,
+                                   ckda_gate_params gp, void *workspace,
+                                   size_t workspace_bytes, cudaStream_t stream) {
+  ckda::GateArgs g;
+  if (!gate_args(gp, g)) return CKDA_ERR_ARG;
+  return fwd_impl(q, k_raw, v, a_logit, c_logit, initial_state, final_state, o,
+                  cu_seqlens, cu_seqlens_host, N, T, H, d_k, d_v, chunk, scale, dt, g,
+                  workspace, workspace_bytes, stream);
+}
+
+ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta,
+                             float *state, void *o, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, float scale,
+                             ckda_dtype dt, cudaStream_t stream) {
+  return decode_impl(q, k, v, alpha, beta, state, o, N, H, d_k, d_v, scale, dt,
+                     ckda::GateArgs{0, 0.f, 0.f, 0.f, 0.f}, stream);
+}
+
+ckda_status ckda_decode_step_gated(const void *q, const void *k_raw, const void *v,
+                                   const void *a_logit, const float *c_logit,
+                                   float *state, void *o, int32_t N, int32_t H,
+                                   int32_t d_k, int32_t d_v, float scale,
+                                   ckda_dtype dt, ckda_gate_params gp,
+                                   cudaStream_t stream) {
+  ckda::GateArgs g;
+  if (!gate_args(gp, g)) return CKDA_ERR_ARG;
+  return decode_impl(q, k_raw, v, a_logit, c_logit, state, o, N, H, d_k, d_v, scale,
+                     dt, g, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+ckda_status fwd_impl(const void *q, const void *k, const void *v,
+                     const void *alpha, const float *beta,
+                     const float *initial_state, float *final_state, void *o,
+                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                     int32_t N, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                     int32_t chunk, float scale, ckda_dtype dt, ckda::GateArgs g,
+                     void *workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (chunk == 0) chunk = 64;
@@ -148,9 +236,10 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
   const size_t th = (size_t)T_total * H;
   const size_t ob = th * d_v * es;
   const size_t sb = (size_t)N * H * d_k * d_v * sizeof(float);
+  const size_t ab = th * d_k * (g.on ? es : sizeof(float));  // alpha or its logits
   if (overlaps(o, ob, q, th * d_k * es) || overlaps(o, ob, k, th * d_k * es) ||
       overlaps(o, ob, v, th * d_v * es) ||
-      overlaps(o, ob, alpha, th * d_k * sizeof(float)) ||
+      overlaps(o, ob, alpha, ab) ||
       overlaps(o, ob, beta, th * sizeof(float)) ||
       overlaps(o, ob, initial_state, sb) || overlaps(o, ob, final_state, sb))
     return CKDA_ERR_ARG;
@@ -165,7 +254,7 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
     const size_t ib = th * d_k * es;
     if (overlaps(workspace, need, q, ib) || overlaps(workspace, need, k, ib) ||
         overlaps(workspace, need, v, th * d_v * es) ||
-        overlaps(workspace, need, alpha, th * d_k * sizeof(float)) ||
+        overlaps(workspace, need, alpha, ab) ||
         overlaps(workspace, need, beta, th * sizeof(float)) ||
         overlaps(workspace, need, o, ob) ||
         overlaps(workspace, need, initial_state, sb) ||
@@ -179,25 +268,25 @@ ckda_status ckda_fwd_chunked(const void *q, const void *k, const void *v,
   cudaError_t e;
   if (ckda::fwd_tc_supported(d_k, d_v, chunk, dt)) {
     e = ckda::launch_fwd_tc(d_v, q, k, v, alpha, beta, initial_state, final_state, o,
-                            cu_seqlens, N, T, (int)T_total, H, scale, workspace,
+                            cu_seqlens, N, T, (int)T_total, H, scale, g, workspace,
                             err, stream);
   } else if (dt == CKDA_F32) {
     e = ckda::launch_fwd_simt<float>(d_k, d_v, chunk, q, k, v, alpha, beta,
                                      initial_state, final_state, o, cu_seqlens,
-                                     N, T, (int)T_total, H, scale, err, stream);
+                                     N, T, (int)T_total, H, scale, g, err, stream);
   } else {
     e = ckda::launch_fwd_simt<__nv_bfloat16>(
         d_k, d_v, chunk, q, k, v, alpha, beta, initial_state, final_state, o,
-        cu_seqlens, N, T, (int)T_total, H, scale, err, stream);
+        cu_seqlens, N, T, (int)T_total, H, scale, g, err, stream);
   }
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
-ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
-                             const float *alpha, const float *beta,
-                             float *state, void *o, int32_t N, int32_t H,
-                             int32_t d_k, int32_t d_v, float scale,
-                             ckda_dtype dt, cudaStream_t stream) {
+ckda_status decode_impl(const void *q, const void *k, const void *v,
+                        const void *alpha, const float *beta, float *state,
+                        void *o, int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                        float scale, ckda_dtype dt, ckda::GateArgs g,
+                        cudaStream_t stream) {
   if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (N < 0 || H <= 0) return CKDA_ERR_ARG;
@@ -211,7 +300,7 @@ ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
   if (overlaps(o, ob, state, nh * d_k * d_v * sizeof(float)) ||
       overlaps(o, ob, q, nh * d_k * es) || overlaps(o, ob, k, nh * d_k * es) ||
       overlaps(o, ob, v, nh * d_v * es) ||
-      overlaps(o, ob, alpha, nh * d_k * sizeof(float)) ||
+      overlaps(o, ob, alpha, nh * d_k * (g.on ? es : sizeof(float))) ||
       overlaps(o, ob, beta, nh * sizeof(float)))
     return CKDA_ERR_ARG;
   if (nh > 0x7fffffffu) return CKDA_ERR_ARG;
@@ -219,10 +308,10 @@ ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
   cudaError_t e =
       dt == CKDA_F32
           ? ckda::launch_decode<float>(d_k, d_v, q, k, v, alpha, beta, state, o,
-                                       N, H, scale, stream)
+                                       N, H, scale, g, stream)
           : ckda::launch_decode<__nv_bfloat16>(d_k, d_v, q, k, v, alpha, beta,
-                                               state, o, N, H, scale, stream);
+                                               state, o, N, H, scale, g, stream);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
-}  // extern "C"
+}  // namespace

@@ -20,6 +20,32 @@ __device__ __forceinline__ void flag_error(unsigned int *err, unsigned int bit) 
   if (err) atomicOr(err, bit);
 }
 
+// Fused input prologue (see ckda_gate_params in ckda.h). When `on`, the
+// kernels read gate logits a (I/O element type) and c (fp32) in place of
+// alpha and beta and raw keys in place of k, and form
+//   alpha = amin + arange * sigmoid(a), beta = bmax * sigmoid(c),
+//   k = k_raw * rn with rn = 1 / (||k_raw|| + keps) (0 when that sum is 0).
+struct GateArgs {
+  int on;
+  float amin, arange, bmax, keps;
+};
+__device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + expf(-x)); }
+__device__ __forceinline__ float gate_alpha(const GateArgs &g, float a) {
+  return g.amin + g.arange * sigmoidf(a);
+}
+__device__ __forceinline__ float gate_beta(const GateArgs &g, float c) {
+  return g.bmax * sigmoidf(c);
+}
+// The tensor-core path (tf32 products) takes the hardware exp2 and
+// reciprocal approximations, a few ulp from the accurate forms above.
+__device__ __forceinline__ float gate_alpha_fast(const GateArgs &g, float a) {
+  return g.amin + g.arange * __fdividef(1.f, 1.f + __expf(-a));
+}
+__device__ __forceinline__ float key_rnorm(const GateArgs &g, float sumsq) {
+  const float d = sqrtf(sumsq) + g.keps;
+  return d > 0.f ? 1.f / d : 0.f;
+}
+
 // Element-type traits for q, k, v, o.
 template <typename T> struct IO;
 template <> struct IO<float> {

@@ -28,17 +28,23 @@ struct DecodeShape {
   static_assert(DK % RG == 0, "row groups must tile d_k");
 };
 
-template <int DK, int DV, int DVS, typename IOT>
+// GATED: the fused input prologue (GateArgs): alpha_in holds gate logits
+// (IOT), beta logits, k raw keys; with rn = 1 / (||k|| + eps),
+// p = rn S'^T k, k.q = rn (k.q) and the update adds (rn k) u^T.
+template <int DK, int DV, int DVS, typename IOT, bool GATED>
 __global__ void __launch_bounds__(DecodeShape<DK, DVS>::THREADS, 4)
 decode_step_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
-                   const IOT *__restrict__ v, const float *__restrict__ alpha,
+                   const IOT *__restrict__ v, const void *__restrict__ alpha_in,
                    const float *__restrict__ beta, float *__restrict__ state,
-                   IOT *__restrict__ o, float scale) {
+                   IOT *__restrict__ o, float scale, GateArgs ga) {
   using Sh = DecodeShape<DK, DVS>;
   constexpr int TPR = Sh::TPR, RG = Sh::RG, RPT = Sh::RPT;
   __shared__ float4 red_p[RG][TPR];
   __shared__ float4 red_r[RG][TPR];
   __shared__ float red_kq[RG];
+  __shared__ float red_kk[GATED ? RG : 1];
+  const float *__restrict__ alpha = reinterpret_cast<const float *>(alpha_in);
+  const IOT *__restrict__ alogit = reinterpret_cast<const IOT *>(alpha_in);
 
   const size_t nh = blockIdx.x;
   const int tid = threadIdx.x;
@@ -58,16 +64,18 @@ decode_step_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
 #pragma unroll
   for (int m = 0; m < RPT; ++m) {
     const int r = rg + m * RG;
-    a[m] = __ldg(alpha + nh * DK + r);
+    if constexpr (GATED) a[m] = gate_alpha(ga, IO<IOT>::ld(alogit + nh * DK + r));
+    else a[m] = __ldg(alpha + nh * DK + r);
     kk[m] = IO<IOT>::ld(k + nh * DK + r);
     qq[m] = IO<IOT>::ld(q + nh * DK + r);
   }
 
   float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 rq = p;
-  float kq = 0.f;
+  float kq = 0.f, kk2 = 0.f;
 #pragma unroll
   for (int m = 0; m < RPT; ++m) {
+    if constexpr (GATED) kk2 += kk[m] * kk[m];
     s[m].x *= a[m];
     s[m].y *= a[m];
     s[m].z *= a[m];
@@ -84,11 +92,15 @@ decode_step_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
   }
   red_p[rg][cg] = p;
   red_r[rg][cg] = rq;
-  if (cg == 0) red_kq[rg] = kq;
+  if (cg == 0) {
+    red_kq[rg] = kq;
+    if constexpr (GATED) red_kk[rg] = kk2;
+  }
   __syncthreads();
   p = make_float4(0.f, 0.f, 0.f, 0.f);
   rq = p;
   kq = 0.f;
+  kk2 = 0.f;
 #pragma unroll
   for (int g = 0; g < RG; ++g) {
     const float4 x = red_p[g][cg], y = red_r[g][cg];
@@ -101,9 +113,18 @@ decode_step_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
     rq.z += y.z;
     rq.w += y.w;
     kq += red_kq[g];
+    if constexpr (GATED) kk2 += red_kk[g];
+  }
+  if constexpr (GATED) {  // normalised key: scale what k entered
+    const float rn = key_rnorm(ga, kk2);
+    p.x *= rn; p.y *= rn; p.z *= rn; p.w *= rn;
+    kq *= rn;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) kk[m] *= rn;
   }
 
-  const float b = __ldg(beta + nh);
+  float b = __ldg(beta + nh);
+  if constexpr (GATED) b = gate_beta(ga, b);
   const float4 vv = IO<IOT>::ld4(v + nh * DV + col);
   float4 u;
   u.x = b * (vv.x - p.x);
@@ -131,52 +152,58 @@ decode_step_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
 
 template <int DK, int DV, typename IOT>
 static cudaError_t launch_decode_dv(const void *q, const void *k, const void *v,
-                                    const float *alpha, const float *beta,
+                                    const void *alpha, const float *beta,
                                     float *state, void *o, int N, int H,
-                                    float scale, cudaStream_t st) {
+                                    float scale, GateArgs g, cudaStream_t st) {
   constexpr int DVS = DV >= 64 ? 64 : DV;
   using Sh = DecodeShape<DK, DVS>;
   const dim3 grid((unsigned)((size_t)N * H), DV / DVS);
-  decode_step_kernel<DK, DV, DVS, IOT><<<grid, Sh::THREADS, 0, st>>>(
-      (const IOT *)q, (const IOT *)k, (const IOT *)v, alpha, beta, state,
-      (IOT *)o, scale);
+  if (g.on)
+    decode_step_kernel<DK, DV, DVS, IOT, true><<<grid, Sh::THREADS, 0, st>>>(
+        (const IOT *)q, (const IOT *)k, (const IOT *)v, alpha, beta, state,
+        (IOT *)o, scale, g);
+  else
+    decode_step_kernel<DK, DV, DVS, IOT, false><<<grid, Sh::THREADS, 0, st>>>(
+        (const IOT *)q, (const IOT *)k, (const IOT *)v, alpha, beta, state,
+        (IOT *)o, scale, g);
   return cudaGetLastError();
 }
 
 template <int DK, typename IOT>
 static cudaError_t launch_decode_dk(int dv, const void *q, const void *k,
-                                    const void *v, const float *alpha,
+                                    const void *v, const void *alpha,
                                     const float *beta, float *state, void *o,
-                                    int N, int H, float scale, cudaStream_t st) {
+                                    int N, int H, float scale, GateArgs g,
+                                    cudaStream_t st) {
   switch (dv) {
-    case 16: return launch_decode_dv<DK, 16, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, st);
-    case 32: return launch_decode_dv<DK, 32, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, st);
-    case 64: return launch_decode_dv<DK, 64, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, st);
-    case 128: return launch_decode_dv<DK, 128, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, st);
+    case 16: return launch_decode_dv<DK, 16, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, g, st);
+    case 32: return launch_decode_dv<DK, 32, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, g, st);
+    case 64: return launch_decode_dv<DK, 64, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, g, st);
+    case 128: return launch_decode_dv<DK, 128, IOT>(q, k, v, alpha, beta, state, o, N, H, scale, g, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template <typename IOT>
 cudaError_t launch_decode(int dk, int dv, const void *q, const void *k,
-                          const void *v, const float *alpha, const float *beta,
+                          const void *v, const void *alpha, const float *beta,
                           float *state, void *o, int N, int H, float scale,
-                          cudaStream_t st) {
+                          GateArgs g, cudaStream_t st) {
   switch (dk) {
-    case 16: return launch_decode_dk<16, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, st);
-    case 32: return launch_decode_dk<32, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, st);
-    case 64: return launch_decode_dk<64, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, st);
-    case 128: return launch_decode_dk<128, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, st);
+    case 16: return launch_decode_dk<16, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, g, st);
+    case 32: return launch_decode_dk<32, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, g, st);
+    case 64: return launch_decode_dk<64, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, g, st);
+    case 128: return launch_decode_dk<128, IOT>(dv, q, k, v, alpha, beta, state, o, N, H, scale, g, st);
   }
   return cudaErrorInvalidValue;
 }
 
 template cudaError_t launch_decode<float>(int, int, const void *, const void *,
-                                          const void *, const float *,
+                                          const void *, const void *,
                                           const float *, float *, void *, int,
-                                          int, float, cudaStream_t);
+                                          int, float, GateArgs, cudaStream_t);
 template cudaError_t launch_decode<__nv_bfloat16>(
-    int, int, const void *, const void *, const void *, const float *,
-    const float *, float *, void *, int, int, float, cudaStream_t);
+    int, int, const void *, const void *, const void *, const void *,
+    const float *, float *, void *, int, int, float, GateArgs, cudaStream_t);
 
 }  // namespace ckda

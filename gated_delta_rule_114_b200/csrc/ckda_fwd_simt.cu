@@ -65,11 +65,15 @@ struct SimtShape {
 template <int DK, int DVT, int C, typename IOT>
 __global__ void __launch_bounds__(256, 1)
 fwd_simt_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
-                const IOT *__restrict__ v, const float *__restrict__ alpha,
+                const IOT *__restrict__ v, const void *__restrict__ alpha_in,
                 const float *__restrict__ beta, const float *__restrict__ s0,
                 float *__restrict__ sfin, IOT *__restrict__ o,
                 const int32_t *__restrict__ cu, int T, int T_total, int H,
-                int DV, float scale, unsigned int *err) {
+                int DV, float scale, GateArgs ga, unsigned int *err) {
+  // ga.on: alpha_in holds gate logits (IOT), beta logits, k raw keys (the
+  // fused input prologue); the keys are normalised in shared memory
+  const float *__restrict__ alpha = reinterpret_cast<const float *>(alpha_in);
+  const IOT *__restrict__ alogit = reinterpret_cast<const IOT *>(alpha_in);
   using Sh = SimtShape<DK, DVT, C>;
   constexpr int KS = Sh::KS, VS = Sh::VS, AS = Sh::AS, NB = Sh::NB;
   constexpr int CPT = Sh::CPT, TC = Sh::TC, TR = Sh::TR, RPT = Sh::RPT,
@@ -114,7 +118,13 @@ fwd_simt_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
         const size_t off = ((size_t)(t0 + i) * H + h) * DK + c4;
         kv = IO<IOT>::ld4(k + off);
         qv = IO<IOT>::ld4(q + off);
-        av = *reinterpret_cast<const float4 *>(alpha + off);
+        if (ga.on) {
+          const float4 x = IO<IOT>::ld4(alogit + off);
+          av = make_float4(gate_alpha(ga, x.x), gate_alpha(ga, x.y), gate_alpha(ga, x.z),
+                           gate_alpha(ga, x.w));
+        } else {
+          av = *reinterpret_cast<const float4 *>(alpha + off);
+        }
       }
       *reinterpret_cast<float4 *>(sK + i * KS + c4) = kv;
       *reinterpret_cast<float4 *>(sQ + i * KS + c4) = qv;
@@ -126,9 +136,23 @@ fwd_simt_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
       if (i < L) vv = IO<IOT>::ld4(v + ((size_t)(t0 + i) * H + h) * DV + c0 + c4);
       *reinterpret_cast<float4 *>(sV + i * VS + c4) = vv;
     }
-    for (int i = tid; i < C; i += Sh::NT)
-      sB[i] = (i < L) ? beta[(size_t)(t0 + i) * H + h] : 0.f;
+    for (int i = tid; i < C; i += Sh::NT) {
+      float b = (i < L) ? beta[(size_t)(t0 + i) * H + h] : 0.f;
+      if (ga.on && i < L) b = gate_beta(ga, b);
+      sB[i] = b;
+    }
     __syncthreads();
+    if (ga.on) {  // k_i <- k_i / (||k_i|| + eps), a warp per row
+      for (int i = tid >> 5; i < C; i += Sh::NT / 32) {
+        float ss = 0.f;
+        for (int c = tid & 31; c < DK; c += 32) ss += sK[i * KS + c] * sK[i * KS + c];
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        const float rn = key_rnorm(ga, ss);
+        for (int c = tid & 31; c < DK; c += 32) sK[i * KS + c] *= rn;
+      }
+      __syncthreads();
+    }
 
     // ---- 2. gated Grams A and M, one 16-row sub-block at a time
     for (int I = 0; I < NB; ++I) {
@@ -384,10 +408,10 @@ fwd_simt_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k,
 
 template <int DK, int DVT, int C, typename IOT>
 static cudaError_t launch_simt_cfg(const void *q, const void *k, const void *v,
-                                   const float *alpha, const float *beta,
+                                   const void *alpha, const float *beta,
                                    const float *s0, float *sf, void *o,
                                    const int32_t *cu, int N, int T, int T_total,
-                                   int H, int DV, float scale,
+                                   int H, int DV, float scale, GateArgs g,
                                    unsigned int *err, cudaStream_t st) {
   using Sh = SimtShape<DK, DVT, C>;
   auto kern = fwd_simt_kernel<DK, DVT, C, IOT>;
@@ -398,22 +422,22 @@ static cudaError_t launch_simt_cfg(const void *q, const void *k, const void *v,
   kern<<<grid, Sh::NT, Sh::BYTES, st>>>((const IOT *)q, (const IOT *)k,
                                         (const IOT *)v, alpha, beta, s0, sf,
                                         (IOT *)o, cu, T, T_total, H, DV, scale,
-                                        err);
+                                        g, err);
   return cudaGetLastError();
 }
 
 template <int DK, int DVT, typename IOT>
 static cudaError_t launch_simt_chunk(int chunk, const void *q, const void *k,
-                                     const void *v, const float *alpha,
+                                     const void *v, const void *alpha,
                                      const float *beta, const float *s0,
                                      float *sf, void *o, const int32_t *cu,
                                      int N, int T, int T_total, int H, int DV,
-                                     float scale, unsigned int *err,
+                                     float scale, GateArgs g, unsigned int *err,
                                      cudaStream_t st) {
   switch (chunk) {
-    case 16: return launch_simt_cfg<DK, DVT, 16, IOT>(q, k, v, alpha, beta, s0, sf, o, cu, N, T, T_total, H, DV, scale, err, st);
-    case 32: return launch_simt_cfg<DK, DVT, 32, IOT>(q, k, v, alpha, beta, s0, sf, o, cu, N, T, T_total, H, DV, scale, err, st);
-    case 64: return launch_simt_cfg<DK, DVT, 64, IOT>(q, k, v, alpha, beta, s0, sf, o, cu, N, T, T_total, H, DV, scale, err, st);
+    case 16: return launch_simt_cfg<DK, DVT, 16, IOT>(q, k, v, alpha, beta, s0, sf, o, cu, N, T, T_total, H, DV, scale, g, err, st);
+    case 32: return launch_simt_cfg<DK, DVT, 32, IOT>(q, k, v, alpha, beta, s0, sf, o, cu, N, T, T_total, H, DV, scale, g, err, st);
+    case 64: return launch_simt_cfg<DK, DVT, 64, IOT>(q, k, v, alpha, beta, s0, sf, o, cu, N, T, T_total, H, DV, scale, g, err, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -421,20 +445,20 @@ static cudaError_t launch_simt_chunk(int chunk, const void *q, const void *k,
 // d_v is tiled by DVT = min(d_v, 32) columns per CTA.
 template <typename IOT>
 cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
-                            const void *k, const void *v, const float *alpha,
+                            const void *k, const void *v, const void *alpha,
                             const float *beta, const float *s0, float *sf,
                             void *o, const int32_t *cu, int N, int T,
-                            int T_total, int H, float scale, unsigned int *err,
-                            cudaStream_t st) {
+                            int T_total, int H, float scale, GateArgs g,
+                            unsigned int *err, cudaStream_t st) {
 #define CKDA_SIMT_DK(DKV)                                                       \
   case DKV:                                                                     \
     if (dv == 16)                                                               \
       return launch_simt_chunk<DKV, 16, IOT>(chunk, q, k, v, alpha, beta, s0,   \
                                              sf, o, cu, N, T, T_total, H, dv,   \
-                                             scale, err, st);                   \
+                                             scale, g, err, st);                \
     return launch_simt_chunk<DKV, 32, IOT>(chunk, q, k, v, alpha, beta, s0, sf, \
                                            o, cu, N, T, T_total, H, dv, scale,  \
-                                           err, st);
+                                           g, err, st);
   switch (dk) {
     CKDA_SIMT_DK(16)
     CKDA_SIMT_DK(32)
@@ -447,13 +471,14 @@ cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
 
 template cudaError_t launch_fwd_simt<float>(int, int, int, const void *,
                                             const void *, const void *,
-                                            const float *, const float *,
+                                            const void *, const float *,
                                             const float *, float *, void *,
                                             const int32_t *, int, int, int, int,
-                                            float, unsigned int *, cudaStream_t);
+                                            float, GateArgs, unsigned int *,
+                                            cudaStream_t);
 template cudaError_t launch_fwd_simt<__nv_bfloat16>(
-    int, int, int, const void *, const void *, const void *, const float *,
+    int, int, int, const void *, const void *, const void *, const void *,
     const float *, const float *, float *, void *, const int32_t *, int, int,
-    int, int, float, unsigned int *, cudaStream_t);
+    int, int, float, GateArgs, unsigned int *, cudaStream_t);
 
 }  // namespace ckda

@@ -138,7 +138,8 @@ constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
 constexpr uint32_t P_B = 216064;      //   256 beta
 constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..2] + TMEM address + flag
 constexpr uint32_t P_P = 216384;      //  2048 gate products of whole sub-blocks [4][128]
-constexpr uint32_t P_SMEM = 218432 + 1024;
+constexpr uint32_t P_RN = 218432;     //   256 key row inverse norms (fused prologue)
+constexpr uint32_t P_SMEM = 218688 + 1024;
 
 // TMEM columns of the prep kernel (512 allocated; one CTA per SM)
 constexpr uint32_t TP_G = 0;      //  96 Gram accumulator
@@ -169,15 +170,22 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase,
   return *s_abort == 0;
 }
 
+// GATED: the fused input prologue (GateArgs): `alpha` holds bf16 gate
+// logits, `beta` fp32 logits and `k` raw keys; the key row inverse norms rn
+// are applied to every product k enters (Gram rows, R, Kbar, beta Khat and
+// the diagonal sub-blocks), which is the same as using the normalised keys.
+template <bool GATED>
 __global__ void __launch_bounds__(NTP, 1)
 ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                        const __nv_bfloat16 *__restrict__ k,
                        const __nv_bfloat16 *__restrict__ v,
-                       const float *__restrict__ alpha,
+                       const void *__restrict__ alpha_in,
                        const float *__restrict__ beta,
                        const int2 *__restrict__ slot_tab, int n_items,
-                       int H, int DV, uint8_t *__restrict__ ws,
+                       int H, int DV, GateArgs ga, uint8_t *__restrict__ ws,
                        unsigned int *err) {
+  const float *__restrict__ alpha = reinterpret_cast<const float *>(alpha_in);
+  const __nv_bfloat16 *__restrict__ alogit = reinterpret_cast<const __nv_bfloat16 *>(alpha_in);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -192,6 +200,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   float *sXT = reinterpret_cast<float *>(sm + P_XT);
   float *sB = reinterpret_cast<float *>(sm + P_B);
   float *sP = reinterpret_cast<float *>(sm + P_P);
+  float *sRN = reinterpret_cast<float *>(sm + P_RN);
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..2]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
@@ -234,6 +243,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     {
       uint4 qv[2], kv[2];
       float4 av[4];
+      (void)av;
       uint4 vr[2];
       float bv = 0.f;
       const int nv = DV / 8;  // 16-byte pieces of a v row
@@ -247,12 +257,23 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           kv[u] = __ldg(reinterpret_cast<const uint4 *>(k + off));
         }
       }
+      uint4 al[2];  // GATED: 64 rows x 16 pieces of 8 bf16 logits
+      if constexpr (GATED) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // alpha: 64 rows x 32 float4
-        const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
-        av[u] = make_float4(1.f, 1.f, 1.f, 1.f);
-        if (i < L)
-          av[u] = __ldg(reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4));
+        for (int u = 0; u < 2; ++u) {
+          const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
+          al[u] = make_uint4(0, 0, 0, 0);
+          if (i < L)
+            al[u] = __ldg(reinterpret_cast<const uint4 *>(alogit + ((size_t)(t0 + i) * H + h) * DK + ch * 8));
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {  // alpha: 64 rows x 32 float4
+          const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
+          av[u] = make_float4(1.f, 1.f, 1.f, 1.f);
+          if (i < L)
+            av[u] = __ldg(reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4));
+        }
       }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {  // v: 64 rows x DV/8 pieces of 16 bytes
@@ -261,7 +282,10 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         if (idx < C * nv && i < L)
           vr[u] = __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + i) * H + h) * DV + 8 * p8));
       }
-      if (tid < L) bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
+      if (tid < L) {
+        bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
+        if constexpr (GATED) bv = gate_beta(ga, bv);
+      }
       // the previous item's bulk stores read staging that overlaps v and q
       if (tid == 0) bulk_wait_read0();
       __syncthreads();
@@ -271,10 +295,40 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         *reinterpret_cast<uint4 *>(sm + P_Q + i * 256 + ch * 16) = qv[u];
         *reinterpret_cast<uint4 *>(sm + P_K + i * 256 + ch * 16) = kv[u];
       }
+      if constexpr (GATED) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
-        *reinterpret_cast<float4 *>(sAl + al_off(i, c4)) = av[u];
+        for (int u = 0; u < 2; ++u) {
+          const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
+          // alpha from the logits (1 on padded rows)
+          float x[8];
+          const uint32_t w[4] = {al[u].x, al[u].y, al[u].z, al[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x[2 * e] = __uint_as_float(w[e] << 16);
+            x[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = (i < L) ? gate_alpha_fast(ga, x[e]) : 1.f;
+          *reinterpret_cast<float4 *>(sAl + al_off(i, 8 * ch)) = make_float4(x[0], x[1], x[2], x[3]);
+          *reinterpret_cast<float4 *>(sAl + al_off(i, 8 * ch + 4)) = make_float4(x[4], x[5], x[6], x[7]);
+          // key row inverse norm: 16 lanes hold row i's 128 channels
+          const uint32_t kw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(kw[e] << 16), hi = __uint_as_float(kw[e] & 0xffff0000u);
+            ss += lo * lo + hi * hi;
+          }
+#pragma unroll
+          for (int m = 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+          if (ch == 0) sRN[i] = (i < L) ? key_rnorm(ga, ss) : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
+          *reinterpret_cast<float4 *>(sAl + al_off(i, c4)) = av[u];
+        }
       }
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -321,6 +375,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
       for (int u = 0; u < 16; ++u) {
         a[u] = sAl[al_off(16 * gq + u, gc)];
         kr[u] = bf(sKr + (16 * gq + u) * DK + gc);
+        if constexpr (GATED) kr[u] *= sRN[16 * gq + u];
       }
       float p = 1.f;
 #pragma unroll
@@ -353,6 +408,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         for (int u = 0; u < 16; ++u) {
           const int i = 16 * gq + u;
           lk[u] = pp[u] * bf(sKr + i * DK + gc);
+          if constexpr (GATED) lk[u] *= sRN[i];
           lq[u] = pp[u] * bf(sQr + i * DK + gc);
         }
 #pragma unroll
@@ -412,6 +468,11 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           ki[2] = bf2_to_f2(kr.z); ki[3] = bf2_to_f2(kr.w);
           qi[0] = bf2_to_f2(qr.x); qi[1] = bf2_to_f2(qr.y);
           qi[2] = bf2_to_f2(qr.z); qi[3] = bf2_to_f2(qr.w);
+          if constexpr (GATED) {
+            const uint64_t rn2 = f2pack(sRN[i], sRN[i]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ki[e] = f2mul(ki[e], rn2);
+          }
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) g[e] = f2pack(1.f, 1.f);
@@ -453,10 +514,11 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int idx = 2 * sl + e, jj = idx & 15;
+          const float rj = GATED ? sRN[r0 + jj] : 1.f;  // column j's key norm
           if (idx >= 16) {
-            if (jj <= ii) sM[i * RS + r0 + jj] = vv[e];
+            if (jj <= ii) sM[i * RS + r0 + jj] = rj * vv[e];
           } else if (jj < ii) {
-            sA[i * RS + r0 + jj] = sB[i] * vv[e];
+            sA[i * RS + r0 + jj] = sB[i] * rj * vv[e];
           }
         }
       }
@@ -559,6 +621,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           const int i = i0 + u + e;
           const float gmm = sAl[al_off(i, c)];
           bk[e] = sB[i] * gmm * bf(sKr + i * DK + c);
+          if constexpr (GATED) bk[e] *= sRN[i];
           sAl[al_off(i, c)] = gmm * bf(sQr + i * DK + c);  // Qhat (fp32, in place)
         }
         st4_f32(GA + off_k_sw128_f32(c, i0 + u, DK + DV), bk[0], bk[1], bk[2], bk[3]);
@@ -957,14 +1020,15 @@ static int sm_count() {
 }
 
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
-                          const float *alpha, const float *beta,
+                          const void *alpha, const float *beta,
                           const float *s0, float *sf, void *o,
                           const int32_t *cu, int N, int T, int T_total, int H,
-                          float scale, void *ws, unsigned int *err,
+                          float scale, GateArgs g, void *ws, unsigned int *err,
                           cudaStream_t st) {
   if (!fwd_tc_supported(DK, dv, C, CKDA_BF16)) return cudaErrorInvalidValue;
+  auto prep = g.on ? ckda_chunk_prep_kernel<true> : ckda_chunk_prep_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(
-      ckda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
+      prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(ckda_chunk_scan_kernel,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S_SMEM);
@@ -979,9 +1043,9 @@ cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
     const long long items = (long long)slots * H;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(items, (long long)sm_count());
-    ckda_chunk_prep_kernel<<<grid, NTP, P_SMEM, st>>>(
+    prep<<<grid, NTP, P_SMEM, st>>>(
         (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-        alpha, beta, tab, (int)items, H, dv, (uint8_t *)ws, err);
+        alpha, beta, tab, (int)items, H, dv, g, (uint8_t *)ws, err);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

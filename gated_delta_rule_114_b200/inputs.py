@@ -181,3 +181,60 @@ def make_decode_tokens(w: Workload, step: int, N: int | None = None,
 def token_heads(w: Workload) -> int:
     cu = seqlens(w)
     return int(cu[-1]) * w.H
+
+
+def _gate_logits(shape, g: torch.Generator) -> torch.Tensor:
+    """Gate logits a ~ N(0, 2); 1% exactly 0 and 5% +-30 (fair sign), which
+    the fused prologue with the CKDA ranges maps to alpha = 0 and, in fp32,
+    alpha = +-1 exactly."""
+    x = 2.0 * torch.randn(shape, generator=g, dtype=torch.float32)
+    u = torch.rand(shape, generator=g, dtype=torch.float32)
+    x = torch.where(u < 0.025, torch.full_like(x, 30.0), x)
+    x = torch.where((u >= 0.025) & (u < 0.05), torch.full_like(x, -30.0), x)
+    return torch.where((u >= 0.05) & (u < 0.06), torch.zeros_like(x), x)
+
+
+def _raw_keys(shape, g: torch.Generator) -> torch.Tensor:
+    """Unnormalised keys: N(0, 1) rows scaled by U(0.2, 3) per row."""
+    x = torch.randn(shape, generator=g, dtype=torch.float32)
+    s = 0.2 + 2.8 * torch.rand(shape[:-1] + (1,), generator=g, dtype=torch.float32)
+    return x * s
+
+
+def make_gated_fwd_inputs(w: Workload, cu_seqlens: torch.Tensor | None = None,
+                          H: int | None = None) -> dict:
+    """CPU tensors for one forward with the fused input prologue: q (unit
+    rows), k_raw, v, a_logit (I/O dtype), c_logit ~ N(0, 1.5) (fp32),
+    initial_state, cu_seqlens; shapes as make_fwd_inputs."""
+    g = _gen(w.seed + 31337)
+    cu = seqlens(w) if cu_seqlens is None else cu_seqlens.to(torch.int32)
+    H = w.H if H is None else H
+    N = cu.numel() - 1
+    T = int(cu[-1])
+    dt = TORCH_DTYPE[w.dtype]
+    q = _unit(torch.randn(T, H, w.d_k, generator=g, dtype=torch.float32))
+    k = _raw_keys((T, H, w.d_k), g)
+    v = torch.randn(T, H, w.d_v, generator=g, dtype=torch.float32)
+    a = _gate_logits((T, H, w.d_k), g)
+    c = 1.5 * torch.randn(T, H, generator=g, dtype=torch.float32)
+    s0 = None
+    if w.init_state:
+        s0 = 0.1 * torch.randn(N, H, w.d_k, w.d_v, generator=g, dtype=torch.float32)
+    return dict(q=q.to(dt), k_raw=k.to(dt), v=v.to(dt), a_logit=a.to(dt).contiguous(),
+                c_logit=c.contiguous(), initial_state=s0, cu_seqlens=cu)
+
+
+def make_gated_decode_tokens(w: Workload, step: int, N: int | None = None,
+                             H: int | None = None) -> dict:
+    """Fresh seeded tokens with logits for a gated decode step."""
+    g = _gen(w.seed * 100003 + 7777 + int(step))
+    N = w.B if N is None else N
+    H = w.H if H is None else H
+    dt = TORCH_DTYPE[w.dtype]
+    q = _unit(torch.randn(N, H, w.d_k, generator=g, dtype=torch.float32))
+    k = _raw_keys((N, H, w.d_k), g)
+    v = torch.randn(N, H, w.d_v, generator=g, dtype=torch.float32)
+    a = _gate_logits((N, H, w.d_k), g)
+    c = 1.5 * torch.randn(N, H, generator=g, dtype=torch.float32)
+    return dict(q=q.to(dt), k_raw=k.to(dt), v=v.to(dt), a_logit=a.to(dt).contiguous(),
+                c_logit=c.contiguous())

@@ -172,6 +172,62 @@ ckda_status ckda_decode_step(const void *q, const void *k, const void *v,
                              int32_t d_k, int32_t d_v, float scale,
                              ckda_dtype dt, cudaStream_t stream);
 
+/*
+ * Fused input prologue: the gates and the key normalisation computed inside
+ * the kernels from per-token logits, in the stable parameterisation of
+ * Semidirect Fourier Delta Attention §3 eqs. (15), (17), (18):
+ *
+ *     alpha = alpha_min + (alpha_max - alpha_min) * sigmoid(a)   (per channel)
+ *     beta  = beta_max * sigmoid(c)                              (per token)
+ *     k     = k_raw / (||k_raw||_2 + k_eps)                      (per token)
+ *
+ * with sigmoid(x) = 1 / (1 + exp(-x)). alpha_min = -1, alpha_max = 1,
+ * beta_max = 2 give the CKDA ranges (alpha = tanh(a / 2), exactly 0 at a = 0;
+ * Complex KDA, abstract); alpha_min = 0, alpha_max = 1, beta_max = 1 give
+ * KDA's. A key row whose ||k_raw|| + k_eps is 0 is taken as k = 0.
+ * Requirements (CKDA_ERR_ARG otherwise): -1 <= alpha_min <= alpha_max <= 1,
+ * 0 <= beta_max <= 2, k_eps >= 0, all finite.
+ */
+typedef struct {
+  float alpha_min;
+  float alpha_max;
+  float beta_max;
+  float k_eps;
+} ckda_gate_params;
+
+/*
+ * ckda_fwd_chunked_gated: ckda_fwd_chunked with the fused input prologue.
+ * Same arguments, results and workspace (ckda_fwd_workspace_bytes) as
+ * ckda_fwd_chunked, except:
+ *   k_raw    [T_total, H, d_k] (dt)   keys before normalisation
+ *   a_logit  [T_total, H, d_k] (dt)   gate logits, in the I/O element type
+ *                                     (half the bytes of fp32 gates in bf16)
+ *   c_logit  [T_total, H]      fp32   delta-coefficient logits
+ *   gp       the gate parameters above
+ * q is used as given (the pages normalise only k).
+ */
+ckda_status ckda_fwd_chunked_gated(const void *q, const void *k_raw, const void *v,
+                                   const void *a_logit, const float *c_logit,
+                                   const float *initial_state, float *final_state,
+                                   void *o, const int32_t *cu_seqlens,
+                                   const int32_t *cu_seqlens_host, int32_t N,
+                                   int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                   int32_t chunk, float scale, ckda_dtype dt,
+                                   ckda_gate_params gp, void *workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * ckda_decode_step_gated: ckda_decode_step with the fused input prologue
+ * (k_raw [N, H, d_k] (dt), a_logit [N, H, d_k] (dt), c_logit [N, H] fp32 in
+ * place of k, alpha, beta); otherwise as ckda_decode_step.
+ */
+ckda_status ckda_decode_step_gated(const void *q, const void *k_raw, const void *v,
+                                   const void *a_logit, const float *c_logit,
+                                   float *state, void *o, int32_t N, int32_t H,
+                                   int32_t d_k, int32_t d_v, float scale,
+                                   ckda_dtype dt, ckda_gate_params gp,
+                                   cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char *ckda_status_string(ckda_status s);
 

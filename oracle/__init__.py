@@ -11,7 +11,8 @@ recurrence of "Semidirect Fourier Delta Attention" §1 eq. (1) / §2.2 eq. (9)
 with the readout of §3 eq. (14); ranges from "Complex KDA", abstract). This
 module only compiles it with gcc (no fast-math) and marshals numpy arrays.
 
-Every function here is pinned by ``tests/test_oracle_pins.py`` against the
+Every function here is pinned by ``tests/test_oracle_pins.py`` and
+``tests/test_oracle_prologue.py`` against the
 lesson's worked traces, closed forms and the dense affine composition
 (§2.2 eq. (10)); none is "parity unpinned".
 """
@@ -156,3 +157,43 @@ def decode(q, k, v, alpha, beta, state, scale: float = 1.0, pairs=None,
     if rc != 0:
         raise RuntimeError("ckda_oracle_decode failed (%d)" % rc)
     return o
+
+
+def sigmoid(x):
+    """1 / (1 + exp(-x)) in fp64, without overflow for large |x|."""
+    x = _f64(x)
+    e = np.exp(-np.abs(x))
+    return np.where(x >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def gate_prologue(a_logit, c_logit, k_raw, alpha_min: float, alpha_max: float,
+                  beta_max: float, k_eps: float):
+    """The fused input prologue in fp64, the stable parameterisation of
+    "Semidirect Fourier Delta Attention" §3, eqs. (15), (17), (18):
+
+        alpha = alpha_min + (alpha_max - alpha_min) * sigmoid(a)   per channel
+        beta  = beta_max * sigmoid(c)                              per token
+        k     = k_raw / (||k_raw||_2 + k_eps)                      per token
+
+    with k = 0 where ||k_raw|| + k_eps is 0. Returns (alpha, beta, k)."""
+    a, c, kr = _f64(a_logit), _f64(c_logit), _f64(k_raw)
+    alpha = alpha_min + (alpha_max - alpha_min) * sigmoid(a)
+    beta = beta_max * sigmoid(c)
+    den = np.sqrt((kr * kr).sum(axis=-1, keepdims=True)) + k_eps
+    k = np.where(den > 0, kr / np.where(den > 0, den, 1.0), 0.0)
+    return alpha, beta, k
+
+
+def fwd_gated(q, k_raw, v, a_logit, c_logit, gates: dict, initial_state=None,
+              cu_seqlens=None, scale: float = 1.0):
+    """The forward with the fused input prologue: gate_prologue, then fwd."""
+    alpha, beta, k = gate_prologue(a_logit, c_logit, k_raw, **gates)
+    return fwd(q, k, v, alpha, beta, initial_state, cu_seqlens, scale)
+
+
+def decode_gated(q, k_raw, v, a_logit, c_logit, state, gates: dict,
+                 scale: float = 1.0, pairs=None):
+    """One decode step with the fused input prologue: gate_prologue, then
+    decode (state updated in place)."""
+    alpha, beta, k = gate_prologue(a_logit, c_logit, k_raw, **gates)
+    return decode(q, k, v, alpha, beta, state, scale, pairs)

@@ -157,3 +157,36 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(ckda, "_lib", None)
     with pytest.raises(RuntimeError):
         ckda.load(str(tmp_path / "nope.so"))
+
+
+@pytest.mark.parametrize("gp,ok", [((-1.0, 1.0, 2.0, 0.0), True), ((0.0, 1.0, 1.0, 1e-6), True),
+                                   ((-1.5, 1.0, 2.0, 0.0), False), ((0.0, 1.2, 1.0, 0.0), False),
+                                   ((0.5, 0.2, 1.0, 0.0), False), ((0.0, 1.0, 2.5, 0.0), False),
+                                   ((0.0, 1.0, -0.1, 0.0), False), ((0.0, 1.0, 1.0, -1.0), False),
+                                   ((0.0, float("nan"), 1.0, 0.0), False),
+                                   ((0.0, 1.0, float("inf"), 0.0), False)])
+def test_gate_params_are_validated_first(lib, gp, ok):
+    # d_k = 48 is unsupported: valid gate parameters reach that check
+    # (CKDA_ERR_UNSUPPORTED), invalid ones are rejected before it (CKDA_ERR_ARG)
+    g = ckda.GateParams(*gp)
+    want = ckda.CKDA_ERR_UNSUPPORTED if ok else ckda.CKDA_ERR_ARG
+    st = lib.ckda_fwd_chunked_gated(P, P2, P3, P4, P5, NULL, NULL, P6, NULL, NULL, 1, 8, 1,
+                                    48, 16, 0, 1.0, ckda.CKDA_F32, g, NULL, 0, None)
+    assert st == want
+    st = lib.ckda_decode_step_gated(P, P2, P3, P4, P5, P6, ctypes.c_void_p(0x70000), 1, 1,
+                                    48, 16, 1.0, ckda.CKDA_F32, g, None)
+    assert st == want
+
+
+def test_gated_forward_rejects_like_the_plain_one(lib):
+    g = ckda.GateParams(-1.0, 1.0, 2.0, 1e-6)
+    # missing logits, misaligned logits, output aliasing the raw keys
+    assert lib.ckda_fwd_chunked_gated(P, P2, P3, NULL, P5, NULL, NULL, P6, NULL, NULL, 1, 8,
+                                      1, 16, 16, 0, 1.0, ckda.CKDA_F32, g, NULL, 0,
+                                      None) == ckda.CKDA_ERR_ARG
+    assert lib.ckda_fwd_chunked_gated(P, P2, P3, ODD, P5, NULL, NULL, P6, NULL, NULL, 1, 8,
+                                      1, 16, 16, 0, 1.0, ckda.CKDA_F32, g, NULL, 0,
+                                      None) == ckda.CKDA_ERR_ARG
+    assert lib.ckda_fwd_chunked_gated(P, P2, P3, P4, P5, NULL, NULL, P2, NULL, NULL, 1, 8,
+                                      1, 16, 16, 0, 1.0, ckda.CKDA_F32, g, NULL, 0,
+                                      None) == ckda.CKDA_ERR_ARG
