@@ -53,6 +53,7 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64, DK = 128, DVT = 32;
+constexpr int PF_STEP = 128;  // bytes per L2 prefetch of the next item's rows
 constexpr int AL_S = 132;  // fp32 row stride of alpha / Qhat
 
 // Float offset of (row i, channel c) in the alpha / Qhat buffer: the 16-byte
@@ -339,21 +340,25 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     }
     __syncthreads();
 
-    // the next item's rows into L2 (one 128-byte line per thread and step;
-    // plain prefetches, which leave the bulk-copy unit to the workspace
-    // stores), while this item is computed
+    // the next item's rows into L2 (one PF_STEP-byte piece per thread and
+    // step; plain prefetches, which leave the bulk-copy unit to the workspace
+    // stores), while this item is computed. Every address lies inside its
+    // row: q, k bf16, the gate input (fp32 alpha or bf16 logits), v bf16.
     if (nxt.y > 0) {
       const int nh = nit % H;
-      const int lq = DK * 2 / 128, la = DK * 4 / 128, lv = (DV * 2 + 127) / 128;
-      const int per = 2 * lq + la + lv;  // lines per token row
+      constexpr int AW = GATED ? 2 : 4;  // bytes per gate element
+      constexpr int lq = DK * 2 / PF_STEP, la = DK * AW / PF_STEP;
+      const int lv = (DV * 2 + PF_STEP - 1) / PF_STEP;
+      const int per = 2 * lq + la + lv;  // pieces per token row
+      const char *gate_in = reinterpret_cast<const char *>(alpha_in);
       for (int t = tid; t < nxt.y * per; t += NTP) {
         const int r = t / per, w = t % per;
         const size_t tok = (size_t)(nxt.x + r) * H + nh;
         const char *p;
-        if (w < lq) p = reinterpret_cast<const char *>(q + tok * DK) + 128 * w;
-        else if (w < 2 * lq) p = reinterpret_cast<const char *>(k + tok * DK) + 128 * (w - lq);
-        else if (w < 2 * lq + la) p = reinterpret_cast<const char *>(alpha + tok * DK) + 128 * (w - 2 * lq);
-        else p = reinterpret_cast<const char *>(v + tok * DV) + 128 * (w - 2 * lq - la);
+        if (w < lq) p = reinterpret_cast<const char *>(q + tok * DK) + PF_STEP * w;
+        else if (w < 2 * lq) p = reinterpret_cast<const char *>(k + tok * DK) + PF_STEP * (w - lq);
+        else if (w < 2 * lq + la) p = gate_in + tok * DK * AW + PF_STEP * (w - 2 * lq);
+        else p = reinterpret_cast<const char *>(v + tok * DV) + PF_STEP * (w - 2 * lq - la);
         prefetch_line_l2(p);
         if (w == 0) prefetch_line_l2(beta + tok);
       }
