@@ -137,7 +137,7 @@ constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
 constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68]
 constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
 constexpr uint32_t P_B = 216064;      //   256 beta
-constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..2] + TMEM address + flag
+constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..3] + TMEM address + flag
 constexpr uint32_t P_P = 216384;      //  2048 gate products of whole sub-blocks [4][128]
 constexpr uint32_t P_RN = 218432;     //   256 key row inverse norms (fused prologue)
 constexpr uint32_t P_SMEM = 218688 + 1024;
@@ -146,6 +146,7 @@ constexpr uint32_t P_SMEM = 218688 + 1024;
 constexpr uint32_t TP_G = 0;      //  96 Gram accumulator
 constexpr uint32_t TP_AD5 = 96;   //  64 [M T ; T] (A of D5)
 constexpr uint32_t TP_D5 = 160;   // 256 [M W | M Ut ; W | Ut]
+constexpr uint32_t TP_G4 = 416;   //  96 Gram inside the 16-token sub-blocks
 constexpr uint32_t TP_COLS = 512;
 
 constexpr uint32_t ID_G = idesc_tf32(128, 96, 1, 1);
@@ -154,6 +155,24 @@ constexpr uint32_t ID_D0 = idesc_tf32(128, 64, 0, 1);
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
 __device__ __forceinline__ void st4_f32(uint8_t *p, float a, float b, float c, float d) {
   *reinterpret_cast<float4 *>(p) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
+}
+
+// Two 16-byte stores of one channel into an MN-major image, rows mn0 and
+// mn0 + 4 (the two 16-byte halves of one 32-byte swizzle chunk). `swap`
+// (lane bit 2, independent of the channel's swizzle chunk k mod 4) reverses
+// their order in half of the lanes, so that each store instruction of a warp
+// (32 consecutive channels) covers all 32 banks instead of half of them.
+__device__ __forceinline__ void st4x2_mn(uint8_t *base, int k, int mn0, int ktot,
+                                         const float *v0, const float *v1, bool swap) {
+  const uint32_t o0 = off_mn_sw128b32_f32(k, mn0, ktot), o1 = off_mn_sw128b32_f32(k, mn0 + 4, ktot);
+  float a[4], b[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    a[e] = swap ? v1[e] : v0[e];
+    b[e] = swap ? v0[e] : v1[e];
+  }
+  st4_f32(base + (swap ? o1 : o0), a[0], a[1], a[2], a[3]);
+  st4_f32(base + (swap ? o0 : o1), b[0], b[1], b[2], b[3]);
 }
 
 // Row r of [M Ut ; Ut] keeps its 16-byte piece p at p ^ (r mod 8), in the
@@ -202,7 +221,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   float *sB = reinterpret_cast<float *>(sm + P_B);
   float *sP = reinterpret_cast<float *>(sm + P_P);
   float *sRN = reinterpret_cast<float *>(sm + P_RN);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..2]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..3]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
 
@@ -212,7 +231,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bar[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -371,10 +390,9 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     //   Lk_i = k_i G_{i<-16g-1} = k_i p_u, Lq_i = q_i p_u      (Gram rows, g >= 1)
     //   R^(I)_j = k_j G_{16I-1<-j} = (k_j suffix_u) P_{g+1} .. P_{I-1}   (I > g)
     //   Kbar_j = k_j sigma_j = (k_j suffix_u) P_{g+1} .. P_3
-    //   gamma_i = P_0 .. P_{g-1} p_u                           (kept for phase 4)
     const int gq = tid >> 7, gc = tid & 127;
-    float pp[16], pre = 1.f;
     {
+      float pre = 1.f;
       float a[16], kr[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
@@ -382,12 +400,25 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         kr[u] = bf(sKr + (16 * gq + u) * DK + gc);
         if constexpr (GATED) kr[u] *= sRN[16 * gq + u];
       }
+      // Gram rows, MN-major (rows contiguous): a thread's 16 rows of one
+      // channel are four 16-byte stores per operand
+      if (gq >= 1) {
+        float lk[16], lq[16], pu = 1.f;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          pu *= a[u];
+          lk[u] = pu * kr[u];
+          lq[u] = pu * bf(sQr + (16 * gq + u) * DK + gc);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; u += 8) {
+          st4x2_mn(GA, gc, (gq - 1) * 32 + u, DK, lk + u, lk + u + 4, (lane >> 2) & 1);
+          st4x2_mn(GA, gc, (gq - 1) * 32 + 16 + u, DK, lq + u, lq + u + 4, (lane >> 2) & 1);
+        }
+      }
       float p = 1.f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        p *= a[u];
-        pp[u] = p;
-      }
+      for (int u = 0; u < 16; ++u) p *= a[u];
       float sfx = 1.f;
 #pragma unroll
       for (int u = 15; u >= 0; --u) {
@@ -405,32 +436,17 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         if (b < gq) pre *= P[b];
         if (b > gq) suf *= P[b];
       }
-      // Gram operands are MN-major (rows contiguous): a thread's 16 rows of
-      // one channel are four 16-byte stores
-      if (gq >= 1) {
-        float lk[16], lq[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int i = 16 * gq + u;
-          lk[u] = pp[u] * bf(sKr + i * DK + gc);
-          if constexpr (GATED) lk[u] *= sRN[i];
-          lq[u] = pp[u] * bf(sQr + i * DK + gc);
-        }
-#pragma unroll
-        for (int u = 0; u < 16; u += 4) {
-          st4_f32(GA + off_mn_sw128b32_f32(gc, (gq - 1) * 32 + u, DK), lk[u], lk[u + 1], lk[u + 2], lk[u + 3]);
-          st4_f32(GA + off_mn_sw128b32_f32(gc, (gq - 1) * 32 + 16 + u, DK), lq[u], lq[u + 1], lq[u + 2], lq[u + 3]);
-        }
-      }
       float f = 1.f;
 #pragma unroll
       for (int I = 1; I < 4; ++I) {
         if (I > gq) {
           if (I > gq + 1) f *= P[I - 1];
 #pragma unroll
-          for (int u = 0; u < 16; u += 4)
-            st4_f32(GB + off_mn_sw128b32_f32(gc, 8 * I * (I - 1) + 16 * gq + u, DK),
-                    f * kr[u], f * kr[u + 1], f * kr[u + 2], f * kr[u + 3]);
+          for (int u = 0; u < 16; u += 8) {
+            const float r0[4] = {f * kr[u], f * kr[u + 1], f * kr[u + 2], f * kr[u + 3]};
+            const float r1[4] = {f * kr[u + 4], f * kr[u + 5], f * kr[u + 6], f * kr[u + 7]};
+            st4x2_mn(GB, gc, 8 * I * (I - 1) + 16 * gq + u, DK, r0, r1, (lane >> 2) & 1);
+          }
         }
       }
 #pragma unroll
@@ -438,7 +454,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         *reinterpret_cast<float4 *>(wsb + WS_A2 + off_k_sw128_f32(gc, 16 * gq + u, DK)) =
             make_float4(to_tf32(suf * kr[u]), to_tf32(suf * kr[u + 1]),
                         to_tf32(suf * kr[u + 2]), to_tf32(suf * kr[u + 3]));
-      if (gq == 3) reinterpret_cast<float *>(wsb + ws_gamma_off(DV))[gc] = pre * pp[15];
+      if (gq == 3) reinterpret_cast<float *>(wsb + ws_gamma_off(DV))[gc] = pre * p;
     }
     fence_async_smem();
     __syncthreads();
@@ -452,19 +468,19 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                     desc_mn_sw128b32_f32(sb + P_GB, DK, kk), ID_G, kk > 0);
       mma_commit(&bar[0]);
     }
-    // ... diagonal 16x16 sub-blocks on CUDA cores, meanwhile. A half-warp
-    // owns one row i (lane sl: channels 8 sl .. 8 sl + 7) and walks j = i,
-    // i-1, ... down the sub-block carrying G_{i<-j} (paired fp32); the 16
-    // lanes are then reduced with a reduce-scatter butterfly that leaves
-    // entries 2 sl, 2 sl + 1 of [A row | M row] in lane sl. Warp w takes rows
-    // w mod 8 and 15 - (w mod 8) of two sub-blocks (one per half), so every
-    // warp walks 17 steps.
+    // ... and, meanwhile on CUDA cores, the pairs inside each 4-token group
+    // (j <= i, same group). A half-warp owns row i (lane sl: channels
+    // 8 sl .. 8 sl + 7) and walks j = i, i-1, ... down the group carrying
+    // G_{i<-j} (paired fp32); a reduce-scatter butterfly over the 16 lanes
+    // then leaves entry sl / 2 of [A row | M row] (4 + 4 entries) in lanes
+    // sl. Warp w takes group 2 (w / 2) + half and its rows {0, 3} (w even) or
+    // {1, 2} (w odd), so every half-warp walks 5 steps.
     {
-      const int sl = lane & 15, c8 = 8 * sl, rp = warp & 7;
-      const int r0 = 16 * (2 * (warp >> 3) + (lane >> 4));
+      const int sl = lane & 15, c8 = 8 * sl;
+      const int r0 = 4 * (2 * (warp >> 1) + (lane >> 4));
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
-        const int ii = pass ? 15 - rp : rp, i = r0 + ii;
+        const int ii = (warp & 1) ? 1 + pass : 3 * pass, i = r0 + ii;
         uint64_t ki[4], qi[4], g[4];
         {
           const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + i * DK + c8);
@@ -481,11 +497,11 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) g[e] = f2pack(1.f, 1.f);
-        float vv[32];
+        float vv[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) vv[e] = 0.f;
+        for (int e = 0; e < 8; ++e) vv[e] = 0.f;
 #pragma unroll
-        for (int jj = 15; jj >= 0; --jj) {
+        for (int jj = 3; jj >= 0; --jj) {
           if (jj <= ii) {
             const int j = r0 + jj;
             const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + j * DK + c8);
@@ -499,7 +515,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
             sa = f2fma(ki[3], x3, sa); sq = f2fma(qi[3], x3, sq);
             const float2 fa = f2unpack(sa), fq = f2unpack(sq);
             vv[jj] = fa.x + fa.y;
-            vv[16 + jj] = fq.x + fq.y;
+            vv[4 + jj] = fq.x + fq.y;
             g[0] = f2mul(g[0], f2pack(a0.x, a0.y));
             g[1] = f2mul(g[1], f2pack(a0.z, a0.w));
             g[2] = f2mul(g[2], f2pack(a1.x, a1.y));
@@ -507,7 +523,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           }
         }
 #pragma unroll
-        for (int m = 8, nn = 32; m > 0; m >>= 1, nn >>= 1) {
+        for (int m = 8, nn = 8; m > 1; m >>= 1, nn >>= 1) {
           const bool up = (sl & m) != 0;
 #pragma unroll
           for (int e = 0; e < nn / 2; ++e) {
@@ -516,22 +532,84 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
             vv[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
           }
         }
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int idx = 2 * sl + e, jj = idx & 15;
+        vv[0] += __shfl_xor_sync(0xffffffffu, vv[0], 1);
+        if ((sl & 1) == 0) {
+          const int idx = sl >> 1, jj = idx & 3;
           const float rj = GATED ? sRN[r0 + jj] : 1.f;  // column j's key norm
-          if (idx >= 16) {
-            if (jj <= ii) sM[i * RS + r0 + jj] = rj * vv[e];
+          if (idx >= 4) {
+            if (jj <= ii) sM[i * RS + r0 + jj] = rj * vv[0];
           } else if (jj < ii) {
-            sA[i * RS + r0 + jj] = sB[i] * rj * vv[e];
+            sA[i * RS + r0 + jj] = sB[i] * rj * vv[0];
           }
         }
       }
     }
-    if (!wait_all(&bar[0], ph, s_abort)) break;
+    if (!wait_all(&bar[0], ph, s_abort)) break;  // the first Gram has read its operands
 
-    // ---------------- 4. off-diagonal Gram blocks out of TMEM; gamma over
-    // alpha (no longer read)
+    // ---------------- 3b. inside each 16-token sub-block b, a pair of
+    // different 4-token groups factors at the boundary before i's group m:
+    //   G_{i<-j} = G_{i<-4m-1} G_{4m-1<-j}          (token indices local to b)
+    // with both factors bounded products, so the rows
+    //   Lk4_i = k_i G_{i<-4m-1},  Lq4_i = q_i G_{i<-4m-1}           (m >= 1)
+    // and the columns R4^(m)_j = k_j G_{4m-1<-j} (j < 4m) give all of them
+    // as one more tensor-core product, in the buffers of the first: row
+    // 32 (m - 1) + 8 b + 4 kind + u (kind 0: Lk4, 1: Lq4; u = i - 4m),
+    // column off_m + 4 m b + j with off_m = 0, 16, 48. Thread (b = gq,
+    // channel gc), which also writes gamma_i over its own alpha column.
+    {
+      float a[16], kr[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        a[u] = sAl[al_off(16 * gq + u, gc)];
+        kr[u] = bf(sKr + (16 * gq + u) * DK + gc);
+        if constexpr (GATED) kr[u] *= sRN[16 * gq + u];
+      }
+#pragma unroll
+      for (int m = 1; m < 4; ++m) {
+        float lk[4], lq[4], p = 1.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = 4 * m + u;
+          p *= a[i];
+          lk[u] = p * kr[i];
+          lq[u] = p * bf(sQr + (16 * gq + i) * DK + gc);
+        }
+        st4x2_mn(GA, gc, 32 * (m - 1) + 8 * gq, DK, lk, lq, (lane >> 2) & 1);
+      }
+#pragma unroll
+      for (int m = 1; m < 4; ++m) {
+        float r[12], sfx = 1.f;
+#pragma unroll
+        for (int j = 4 * m - 1; j >= 0; --j) {
+          r[j] = sfx * kr[j];
+          sfx *= a[j];
+        }
+        const int col = (m == 1 ? 0 : (m == 2 ? 16 : 48)) + 4 * m * gq;
+        if (m == 1) st4_f32(GB + off_mn_sw128b32_f32(gc, col, DK), r[0], r[1], r[2], r[3]);
+        else st4x2_mn(GB, gc, col, DK, r, r + 4, (lane >> 2) & 1);
+        if (m == 3) st4_f32(GB + off_mn_sw128b32_f32(gc, col + 8, DK), r[8], r[9], r[10], r[11]);
+      }
+      float gam = 1.f;  // gamma_i = prod_{s <= i} alpha_s, over alpha (read only here from now on)
+      for (int b = 0; b < gq; ++b) gam *= sP[b * DK + gc];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        gam *= a[u];
+        sAl[al_off(16 * gq + u, gc)] = gam;
+      }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      fence_after_sync();
+#pragma unroll
+      for (int kk = 0; kk < DK / 8; ++kk)
+        mma_tf32_ss(tm + TP_G4, desc_mn_sw128b32_f32(sb + P_GA, DK, kk),
+                    desc_mn_sw128b32_f32(sb + P_GB, DK, kk), ID_G, kk > 0);
+      mma_commit(&bar[3]);
+    }
+
+    // ---------------- 4. Gram blocks out of TMEM: first the pairs of
+    // different 16-token sub-blocks (while the second product runs) ...
     {
       // sub-block row I = qw + 1 sits in lane quarter qw (lanes 0-15 Lk rows,
       // 16-31 Lq rows); warp part takes columns 16 part .. 16 part + 15
@@ -549,8 +627,36 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
               make_float4(b * x[e], b * x[e + 1], b * x[e + 2], b * x[e + 3]);
       }
     }
+    if (!wait_all(&bar[3], ph, s_abort)) break;
+    // ... then those of different 4-token groups of one sub-block: warp
+    // (lane quarter m - 1, sub-block b = warp / 4) reads the 4 m columns of
+    // R4^(m) of block b; its lanes 8 b .. 8 b + 7 hold rows (kind, u).
+    {
+      const int qw = warp & 3, b = warp >> 2;
+      if (qw < 3) {
+        const int m = qw + 1;
+        const uint32_t ta = tm + lane_base + TP_G4 + (uint32_t)((m == 1 ? 0 : (m == 2 ? 16 : 48)) + 4 * m * b);
+        float x[12];
 #pragma unroll
-    for (int u = 0; u < 16; ++u) sAl[al_off(16 * gq + u, gc)] = pre * pp[u];  // gamma_i
+        for (int e = 0; e < 12; ++e) x[e] = 0.f;
+        if (m == 1) {
+          tmem_ld4(ta, x);
+        } else {
+          tmem_ld8(ta, x);
+          if (m == 3) tmem_ld4(ta + 8, x + 8);
+        }
+        if ((lane >> 3) == b) {
+          const int kind = (lane >> 2) & 1, u = lane & 3, i = 16 * b + 4 * m + u;
+          const float sc = kind ? 1.f : sB[i];
+          float *dst = (kind ? sM : sA) + i * RS + 16 * b;
+#pragma unroll
+          for (int e = 0; e < 12; e += 4)
+            if (e < 4 * m)
+              *reinterpret_cast<float4 *>(dst + e) =
+                  make_float4(sc * x[e], sc * x[e + 1], sc * x[e + 2], sc * x[e + 3]);
+        }
+      }
+    }
     fence_before_sync();
     __syncthreads();
 
@@ -869,8 +975,9 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
         float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
         if (s0) x = *reinterpret_cast<const float4 *>(s0 + st_base + (size_t)r * DV + c0 + e);
         S[e] = x.x; S[e + 1] = x.y; S[e + 2] = x.z; S[e + 3] = x.w;
-        st4_f32(sm + S_S + off_mn_sw128b32_f32(r, e, DK), x.x, x.y, x.z, x.w);
       }
+#pragma unroll
+      for (int e = 0; e < DVT; e += 8) st4x2_mn(sm + S_S, r, e, DK, S + e, S + e + 4, (lane >> 2) & 1);
     }
     fence_async_smem();
     named_bar_sync(2, NCONS);
@@ -918,10 +1025,11 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
       tmem_ld32(tm + lane_base + TS_D1, d1);
       if (tid >= C) {  // U = Ut - W S, then D2 = Kbar^T x U
         const int j = tid - C;
+        float u[DVT];
 #pragma unroll
-        for (int e = 0; e < DVT; e += 4)
-          st4_f32(sm + S_U + off_mn_sw128b32_f32(j, e, C), ou[e] - d1[e], ou[e + 1] - d1[e + 1],
-                  ou[e + 2] - d1[e + 2], ou[e + 3] - d1[e + 3]);
+        for (int e = 0; e < DVT; ++e) u[e] = ou[e] - d1[e];
+#pragma unroll
+        for (int e = 0; e < DVT; e += 8) st4x2_mn(sm + S_U, j, e, C, u + e, u + e + 4, (lane >> 2) & 1);
         fence_async_smem();
         named_bar_sync(1, NCONS - C);
         if (tid == ISS) {
@@ -954,8 +1062,7 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
 #pragma unroll
         for (int e = 0; e < DVT; ++e) S[e] = gc * S[e] + d2[e];
 #pragma unroll
-        for (int e = 0; e < DVT; e += 4)
-          st4_f32(sm + S_S + off_mn_sw128b32_f32(tid, e, DK), S[e], S[e + 1], S[e + 2], S[e + 3]);
+        for (int e = 0; e < DVT; e += 8) st4x2_mn(sm + S_S, tid, e, DK, S + e, S + e + 4, (lane >> 2) & 1);
       }
       fence_async_smem();
       fence_before_sync();
