@@ -863,7 +863,10 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
 // images into a shared-memory landing buffer two chunks ahead and moves them
 // into tensor memory (tcgen05.cp, 128 lanes x 8 columns per K-step), so both
 // MMAs of the state chain take their A operand from tensor memory and read
-// only the small B operand (S or U) from shared memory.
+// only the small B operand (S or U) from shared memory. Each product is
+// issued by two threads in different warps, each taking half of the K-steps
+// into its own accumulator (the chain is bound by how fast MMAs are issued,
+// not by the tensor pipe); readers add the two halves.
 constexpr int NTS = 160, NCONS = 128;
 constexpr uint32_t S_A1 = 0;          // 2 x 65536 [Qtil ; W] landing buffers
 constexpr uint32_t S_A2 = 131072;     // 2 x 32768 Kbar^T landing buffers
@@ -873,11 +876,14 @@ constexpr uint32_t S_BAR = 221184;    //   128 mbarriers [0..9] + TMEM address +
 constexpr uint32_t S_SMEM = 221312 + 1024;
 // mbarriers: landed[2] (bulk copy into landing buffer b), ready[2] (buffer b
 // in tensor memory), free[2] (the MMAs that read tensor-memory buffer b are
-// done), D1, D2. Each completes once per use of its buffer or chunk, and no
-// waiter can be two completions behind, so parity waits are exact.
+// done), D1, D2. Each completes once per use of its buffer or chunk (free,
+// D1 and D2 after one commit from each of the two issuers), and no waiter
+// can be two completions behind, so parity waits are exact.
 enum { B_LANDED = 0, B_READY = 2, B_FREE = 4, B_D1 = 6, B_D2 = 7, NBAR = 8 };
-// tensor memory: D1, D2 accumulators; [Qtil ; W] and Kbar^T, two buffers each
-constexpr uint32_t TS_D1 = 0, TS_D2 = 32, TS_A1 = 64, TS_A2 = 320, TS_COLS = 512;
+// tensor memory: D1, D2 accumulators (first issuer's halves); [Qtil ; W] and
+// Kbar^T, two buffers each; the second issuer's D1, D2 halves
+constexpr uint32_t TS_D1 = 0, TS_D2 = 32, TS_A1 = 64, TS_A2 = 320, TS_D1B = 448, TS_D2B = 480;
+constexpr uint32_t TS_COLS = 512;
 constexpr uint32_t ID_D1 = idesc_tf32(128, 32, 0, 1);
 constexpr uint32_t ID_D2 = idesc_tf32(128, 32, 0, 1);
 constexpr uint32_t LOAD_BYTES = 65536 + 32768;
@@ -904,8 +910,9 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
   const int base = slot_base(cu, n, T);
   const size_t st_base = ((size_t)n * H + h) * DK * DV;
   const uint32_t wsz = ws_block_bytes(DV);
-  // Consumer thread ISS (first thread of the U half) issues the MMAs.
-  constexpr int ISS = C;
+  // Consumer threads ISS and ISS2 (lane 0 of the two U-half warps) issue the
+  // MMAs, K-steps 0 .. K/2-1 and K/2 .. K-1 respectively.
+  constexpr int ISS = C, ISS2 = C + 32;
   constexpr int PROD = NCONS;  // producer thread (lane 0 of warp 4)
 
   if (warp == 0) {
@@ -913,7 +920,7 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
     tmem_relinquish();
   }
   if (tid == PROD) {
-    for (int i = 0; i < NBAR; ++i) mbar_init(&bar[i], 1);
+    for (int i = 0; i < NBAR; ++i) mbar_init(&bar[i], i >= B_FREE ? 2 : 1);  // free, D1, D2: two issuers
     fence_mbar_init();
   }
   if (tid == 0) *s_abort = 0;
@@ -1010,19 +1017,26 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
       const float gc = gc_next;
       if (c + 1 < nch) load_rows(c + 1);
 
-      if (tid == ISS) {  // D1 = [Qtil ; W] x S, A from tensor memory
+      if (tid == ISS || tid == ISS2) {  // D1 = [Qtil ; W] x S, K split over two issuers
+        const int h2 = tid == ISS2;
         if (!mbar_wait(&bar[B_READY + b], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
         fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < DK / 8; ++kk)
-          mma_tf32_ts(tm + TS_D1, tm + TS_A1 + b * 128 + 8 * kk,
-                      desc_mn_sw128b32_f32(sb + S_S, DK, kk), ID_D1, kk > 0);
+        for (int kk = 0; kk < DK / 16; ++kk)
+          mma_tf32_ts(tm + (h2 ? TS_D1B : TS_D1), tm + TS_A1 + b * 128 + 8 * (kk + 8 * h2),
+                      desc_mn_sw128b32_f32(sb + S_S, DK, kk + 8 * h2), ID_D1, kk > 0);
         mma_commit(&bar[B_D1]);
       }
       if (!mbar_wait(&bar[B_D1], (uint32_t)c & 1u)) *s_abort = 1;
       fence_after_sync();
       float d1[32];
-      tmem_ld32(tm + lane_base + TS_D1, d1);
+      {
+        float d1b[32];
+        tmem_ld32(tm + lane_base + TS_D1, d1);
+        tmem_ld32(tm + lane_base + TS_D1B, d1b);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) d1[e] += d1b[e];
+      }
       if (tid >= C) {  // U = Ut - W S, then D2 = Kbar^T x U
         const int j = tid - C;
         float u[DVT];
@@ -1032,12 +1046,13 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
         for (int e = 0; e < DVT; e += 8) st4x2_mn(sm + S_U, j, e, C, u + e, u + e + 4, (lane >> 2) & 1);
         fence_async_smem();
         named_bar_sync(1, NCONS - C);
-        if (tid == ISS) {
+        if (tid == ISS || tid == ISS2) {
+          const int h2 = tid == ISS2;
           fence_after_sync();
 #pragma unroll
-          for (int kk = 0; kk < C / 8; ++kk)
-            mma_tf32_ts(tm + TS_D2, tm + TS_A2 + b * 64 + 8 * kk,
-                        desc_mn_sw128b32_f32(sb + S_U, C, kk), ID_D2, kk > 0);
+          for (int kk = 0; kk < C / 16; ++kk)
+            mma_tf32_ts(tm + (h2 ? TS_D2B : TS_D2), tm + TS_A2 + b * 64 + 8 * (kk + 4 * h2),
+                        desc_mn_sw128b32_f32(sb + S_U, C, kk + 4 * h2), ID_D2, kk > 0);
           mma_commit(&bar[B_D2]);
           mma_commit(&bar[B_FREE + b]);  // tensor-memory buffer b may be refilled
         }
@@ -1058,7 +1073,13 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
       fence_after_sync();
       {
         float d2[32];
-        tmem_ld32(tm + lane_base + TS_D2, d2);
+        {
+          float d2b[32];
+          tmem_ld32(tm + lane_base + TS_D2, d2);
+          tmem_ld32(tm + lane_base + TS_D2B, d2b);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) d2[e] += d2b[e];
+        }
 #pragma unroll
         for (int e = 0; e < DVT; ++e) S[e] = gc * S[e] + d2[e];
 #pragma unroll
