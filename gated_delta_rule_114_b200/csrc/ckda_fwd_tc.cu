@@ -662,24 +662,59 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
 
     if (warp < NTP / 64) {  // warps 0..7 invert; named barrier 1 among them
       // ---------------- 5. T = (I + A)^{-1} by blocked forward substitution
-      // diagonal 16x16 blocks: thread (block b, column j), row by row
+      // diagonal 16x16 blocks T_II in two levels of 8: first the 8x8 diagonal
+      // sub-blocks by forward substitution, thread (block b, half h, column
+      // j), with row ii + 1 loaded while row ii is solved ...
       if (tid < C) {
-        const int b = tid >> 4, j = tid & 15, ob = b * 16;
-        float t[16];
+        const int b = tid >> 4, h = (tid >> 3) & 1, j = tid & 7, o8 = 16 * b + 8 * h;
+        const float *Ab = sA + o8 * RS + o8;
+        float t[8], ar[8];
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) t[ii] = (ii == j) ? 1.f : 0.f;
+        for (int ii = 0; ii < 8; ++ii) t[ii] = (ii == j) ? 1.f : 0.f;
+        {
+          const float4 v = *reinterpret_cast<const float4 *>(Ab + RS);
+          ar[0] = v.x; ar[1] = v.y; ar[2] = v.z; ar[3] = v.w;
+        }
 #pragma unroll
-        for (int ii = 1; ii < 16; ++ii) {
+        for (int ii = 1; ii < 8; ++ii) {
+          float cur[8];
+#pragma unroll
+          for (int l = 0; l < ii; ++l) cur[l] = ar[l];
+          if (ii + 1 < 8) {
+#pragma unroll
+            for (int q4 = 0; q4 < (ii + 4) / 4; ++q4) {  // columns 0 .. ii of row ii + 1
+              const float4 v = *reinterpret_cast<const float4 *>(Ab + (ii + 1) * RS + 4 * q4);
+              ar[4 * q4] = v.x; ar[4 * q4 + 1] = v.y; ar[4 * q4 + 2] = v.z; ar[4 * q4 + 3] = v.w;
+            }
+          }
           if (ii > j) {
             float s = 0.f;
 #pragma unroll
             for (int l = 0; l < ii; ++l)
-              if (l >= j) s += sA[(ob + ii) * RS + ob + l] * t[l];
+              if (l >= j) s += cur[l] * t[l];
             t[ii] = -s;
           }
         }
 #pragma unroll
-        for (int ii = 0; ii < 16; ++ii) sT[(ob + ii) * RS + ob + j] = t[ii];
+        for (int ii = 0; ii < 8; ++ii) sT[(o8 + ii) * RS + o8 + j] = t[ii];
+      }
+      named_bar_sync(1, NTP / 2);
+      // ... then the lower-left 8x8 block T21 = -T22 (A21 T11), thread
+      // (block b, row r, column c); the upper-right block is zero
+      {
+        const int b = tid >> 6, r = (tid >> 3) & 7, c = tid & 7, ob = 16 * b;
+        float x = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          if (m >= c) x += sA[(ob + 8 + r) * RS + ob + m] * sT[(ob + m) * RS + ob + c];
+        sXT[b * 64 + r * 8 + c] = x;
+        named_bar_sync(1, NTP / 2);
+        float y = 0.f;
+#pragma unroll
+        for (int m = 0; m < 8; ++m)
+          if (m <= r) y += sT[(ob + 8 + r) * RS + ob + 8 + m] * sXT[b * 64 + m * 8 + c];
+        sT[(ob + 8 + r) * RS + ob + c] = -y;
+        sT[(ob + r) * RS + ob + 8 + c] = 0.f;
       }
       named_bar_sync(1, NTP / 2);
       // block (I, J = I - d): X = sum_{J <= Lb < I} A_{I,Lb} T_{Lb,J}, then
@@ -692,10 +727,18 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         if (tid < ntask) {
           float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
           for (int Lb = J; Lb < I; ++Lb) {
+            float ra[16], rb[16];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              const float4 u0 = *reinterpret_cast<const float4 *>(sA + r * RS + 16 * Lb + 4 * q4);
+              const float4 u1 = *reinterpret_cast<const float4 *>(sA + (r + 1) * RS + 16 * Lb + 4 * q4);
+              ra[4 * q4] = u0.x; ra[4 * q4 + 1] = u0.y; ra[4 * q4 + 2] = u0.z; ra[4 * q4 + 3] = u0.w;
+              rb[4 * q4] = u1.x; rb[4 * q4 + 1] = u1.y; rb[4 * q4 + 2] = u1.z; rb[4 * q4 + 3] = u1.w;
+            }
 #pragma unroll
             for (int l = 0; l < 16; ++l) {
               const int col = 16 * Lb + l;
-              const float a0 = sA[r * RS + col], a1 = sA[(r + 1) * RS + col];
+              const float a0 = ra[l], a1 = rb[l];
               const float2 tv = *reinterpret_cast<const float2 *>(sT + col * RS + cc);
               x00 += a0 * tv.x; x01 += a0 * tv.y;
               x10 += a1 * tv.x; x11 += a1 * tv.y;
@@ -737,13 +780,37 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         }
         st4_f32(GA + off_k_sw128_f32(c, i0 + u, DK + DV), bk[0], bk[1], bk[2], bk[3]);
       }
+      // beta V rows 128 .. 128 + DV: thread (channel pair cp, 16-token quarter);
+      // the two rows' stores alternate their order on lane bit 2 (rows 2 cp
+      // and 2 cp + 1 then cover all eight 16-byte slots of a swizzle line)
       const __nv_bfloat16 *sV = reinterpret_cast<const __nv_bfloat16 *>(sm + P_V);
-      for (int task = t; task < DV * (C / 4); task += NTP / 2) {  // beta V rows 128 .. 128+DV
-        const int cv = task % DV, j4 = 4 * (task / DV);
-        float x[4];
+      const int npair = DV / 2;
+      if (t < 4 * npair) {
+        const int cv = 2 * (t % npair), j0 = 16 * (t / npair);
+        float lo[16], hi[16], bb[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = sB[j4 + e] * bf(sV + (j4 + e) * DV + cv);
-        st4_f32(GA + off_k_sw128_f32(DK + cv, j4, DK + DV), x[0], x[1], x[2], x[3]);
+        for (int e = 0; e < 16; ++e) {
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(sV + (j0 + e) * DV + cv);
+          lo[e] = __uint_as_float(w << 16);
+          hi[e] = __uint_as_float(w & 0xffff0000u);
+        }
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const float4 b4 = *reinterpret_cast<const float4 *>(sB + j0 + e);
+          bb[e] = b4.x; bb[e + 1] = b4.y; bb[e + 2] = b4.z; bb[e + 3] = b4.w;
+        }
+        const bool sw = (lane >> 2) & 1;
+#pragma unroll
+        for (int g = 0; g < 16; g += 4) {
+          float x0[4], x1[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x0[e] = bb[g + e] * (sw ? hi[g + e] : lo[g + e]);
+            x1[e] = bb[g + e] * (sw ? lo[g + e] : hi[g + e]);
+          }
+          st4_f32(GA + off_k_sw128_f32(DK + cv + (sw ? 1 : 0), j0 + g, DK + DV), x0[0], x0[1], x0[2], x0[3]);
+          st4_f32(GA + off_k_sw128_f32(DK + cv + (sw ? 0 : 1), j0 + g, DK + DV), x1[0], x1[1], x1[2], x1[3]);
+        }
       }
     }
     __syncthreads();
