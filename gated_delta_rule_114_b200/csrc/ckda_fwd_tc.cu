@@ -717,68 +717,142 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         sT[(ob + r) * RS + ob + 8 + c] = 0.f;
       }
       named_bar_sync(1, NTP / 2);
-      // block (I, J = I - d): X = sum_{J <= Lb < I} A_{I,Lb} T_{Lb,J}, then
-      // T_{I,J} = -T_{I,I} X; thread = 2x2 tile (ti, tj) of one block
-      for (int d = 1; d < 4; ++d) {
-        const int ntask = (4 - d) * 64;
-        const int p = tid >> 6, ti = (tid & 63) >> 3, tj = tid & 7;
-        const int J = p, I = p + d;
-        const int r = 16 * I + 2 * ti, cc = 16 * J + 2 * tj;
-        if (tid < ntask) {
-          float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-          for (int Lb = J; Lb < I; ++Lb) {
-            float ra[16], rb[16];
+      // off-diagonal blocks by doubling. Level 1 (16 -> 32): T_10 =
+      // -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22), thread (block pair q,
+      // row r, column pair cp); the upper-right blocks T_01, T_23 are zero.
+      {
+        const int q = tid >> 7, r = (tid >> 3) & 15, cp = tid & 7;
+        const int J = 2 * q, I = 2 * q + 1, c = 16 * J + 2 * cp;
+        float a[16];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              const float4 u0 = *reinterpret_cast<const float4 *>(sA + r * RS + 16 * Lb + 4 * q4);
-              const float4 u1 = *reinterpret_cast<const float4 *>(sA + (r + 1) * RS + 16 * Lb + 4 * q4);
-              ra[4 * q4] = u0.x; ra[4 * q4 + 1] = u0.y; ra[4 * q4 + 2] = u0.z; ra[4 * q4 + 3] = u0.w;
-              rb[4 * q4] = u1.x; rb[4 * q4 + 1] = u1.y; rb[4 * q4 + 2] = u1.z; rb[4 * q4 + 3] = u1.w;
-            }
-#pragma unroll
-            for (int l = 0; l < 16; ++l) {
-              const int col = 16 * Lb + l;
-              const float a0 = ra[l], a1 = rb[l];
-              const float2 tv = *reinterpret_cast<const float2 *>(sT + col * RS + cc);
-              x00 += a0 * tv.x; x01 += a0 * tv.y;
-              x10 += a1 * tv.x; x11 += a1 * tv.y;
-            }
-          }
-          *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti) * 16 + 2 * tj) = make_float2(x00, x01);
-          *reinterpret_cast<float2 *>(sXT + p * 256 + (2 * ti + 1) * 16 + 2 * tj) = make_float2(x10, x11);
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float4 u = *reinterpret_cast<const float4 *>(sA + (16 * I + r) * RS + 16 * J + 4 * q4);
+          a[4 * q4] = u.x; a[4 * q4 + 1] = u.y; a[4 * q4 + 2] = u.z; a[4 * q4 + 3] = u.w;
         }
-        named_bar_sync(1, NTP / 2);
-        if (tid < ntask) {
-          float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+        float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-          for (int m = 0; m < 16; ++m) {  // T_{I,I} is zero above its diagonal
-            const float t0 = sT[r * RS + 16 * I + m], t1 = sT[(r + 1) * RS + 16 * I + m];
-            const float2 xv = *reinterpret_cast<const float2 *>(sXT + p * 256 + m * 16 + 2 * tj);
-            y00 += t0 * xv.x; y01 += t0 * xv.y;
-            y10 += t1 * xv.x; y11 += t1 * xv.y;
-          }
-          *reinterpret_cast<float2 *>(sT + r * RS + cc) = make_float2(-y00, -y01);
-          *reinterpret_cast<float2 *>(sT + (r + 1) * RS + cc) = make_float2(-y10, -y11);
+        for (int m = 0; m < 16; ++m) {
+          const float2 tv = *reinterpret_cast<const float2 *>(sT + (16 * J + m) * RS + c);
+          x0 += a[m] * tv.x; x1 += a[m] * tv.y;
         }
+        *reinterpret_cast<float2 *>(sXT + q * 256 + r * 16 + 2 * cp) = make_float2(x0, x1);
         named_bar_sync(1, NTP / 2);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {  // row r of T_II (zero above its diagonal)
+          const float4 u = *reinterpret_cast<const float4 *>(sT + (16 * I + r) * RS + 16 * I + 4 * q4);
+          a[4 * q4] = u.x; a[4 * q4 + 1] = u.y; a[4 * q4 + 2] = u.z; a[4 * q4 + 3] = u.w;
+        }
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+          const float2 xv = *reinterpret_cast<const float2 *>(sXT + q * 256 + m * 16 + 2 * cp);
+          y0 += a[m] * xv.x; y1 += a[m] * xv.y;
+        }
+        *reinterpret_cast<float2 *>(sT + (16 * I + r) * RS + c) = make_float2(-y0, -y1);
+        *reinterpret_cast<float2 *>(sT + (16 * J + r) * RS + 16 * I + 2 * cp) = make_float2(0.f, 0.f);
       }
+      named_bar_sync(1, NTP / 2);
+      // Level 2 (32 -> 64): T_hl = -T_hi (A_hl T_lo) over 32x32 blocks (rows
+      // 32 .. 63, columns 0 .. 31). X = A_hl T_lo is kept in the unused
+      // upper-right 32x32 block of T (rows 0 .. 31, columns 32 .. 63).
+      // Thread = 2x2 tile; the zero block of T_lo (rows < 16, columns >= 16)
+      // and that of T_hi (rows < 16, columns >= 16) are skipped.
+      {
+        const int ch = tid >> 7, tr = (tid >> 3) & 15, tc = tid & 7;
+        const int r = 2 * tr, c = 16 * ch + 2 * tc;
+        float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+        for (int Lb = ch; Lb < 2; ++Lb) {
+          float ra[16], rb[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 u0 = *reinterpret_cast<const float4 *>(sA + (32 + r) * RS + 16 * Lb + 4 * q4);
+            const float4 u1 = *reinterpret_cast<const float4 *>(sA + (33 + r) * RS + 16 * Lb + 4 * q4);
+            ra[4 * q4] = u0.x; ra[4 * q4 + 1] = u0.y; ra[4 * q4 + 2] = u0.z; ra[4 * q4 + 3] = u0.w;
+            rb[4 * q4] = u1.x; rb[4 * q4 + 1] = u1.y; rb[4 * q4 + 2] = u1.z; rb[4 * q4 + 3] = u1.w;
+          }
+#pragma unroll
+          for (int l = 0; l < 16; ++l) {
+            const float2 tv = *reinterpret_cast<const float2 *>(sT + (16 * Lb + l) * RS + c);
+            x00 += ra[l] * tv.x; x01 += ra[l] * tv.y;
+            x10 += rb[l] * tv.x; x11 += rb[l] * tv.y;
+          }
+        }
+        *reinterpret_cast<float2 *>(sT + r * RS + 32 + c) = make_float2(x00, x01);
+        *reinterpret_cast<float2 *>(sT + (r + 1) * RS + 32 + c) = make_float2(x10, x11);
+      }
+      named_bar_sync(1, NTP / 2);
+      {
+        const int rh = tid >> 7, tr = (tid >> 4) & 7, tc = tid & 15;
+        const int r = 16 * rh + 2 * tr, c = 2 * tc;
+        float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+        for (int Lb = 0; Lb <= rh; ++Lb) {
+          float ta[16], tb[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 u0 = *reinterpret_cast<const float4 *>(sT + (32 + r) * RS + 32 + 16 * Lb + 4 * q4);
+            const float4 u1 = *reinterpret_cast<const float4 *>(sT + (33 + r) * RS + 32 + 16 * Lb + 4 * q4);
+            ta[4 * q4] = u0.x; ta[4 * q4 + 1] = u0.y; ta[4 * q4 + 2] = u0.z; ta[4 * q4 + 3] = u0.w;
+            tb[4 * q4] = u1.x; tb[4 * q4 + 1] = u1.y; tb[4 * q4 + 2] = u1.z; tb[4 * q4 + 3] = u1.w;
+          }
+#pragma unroll
+          for (int l = 0; l < 16; ++l) {
+            const float2 xv = *reinterpret_cast<const float2 *>(sT + (16 * Lb + l) * RS + 32 + c);
+            y00 += ta[l] * xv.x; y01 += ta[l] * xv.y;
+            y10 += tb[l] * xv.x; y11 += tb[l] * xv.y;
+          }
+        }
+        *reinterpret_cast<float2 *>(sT + (32 + r) * RS + c) = make_float2(-y00, -y01);
+        *reinterpret_cast<float2 *>(sT + (33 + r) * RS + c) = make_float2(-y10, -y11);
+      }
+      named_bar_sync(1, NTP / 2);
     } else {
       // ---------------- 5'. meanwhile (warps 8..15): the last MMA's B operand
       // [beta Khat | beta V], K-major (row n = output column, 4 tokens per
       // 16-byte store, 128 + DV rows), and Qhat over gamma
-      const int t = tid - NTP / 2, c = t & (DK - 1), i0 = 32 * (t >> 7);
+      // thread (channel pair cp, 16-token quarter), 8 tokens at a time, every
+      // load ahead of the stores; the two rows' stores alternate on lane bit 2
+      const int t = tid - NTP / 2;
+      const bool sw = (lane >> 2) & 1;
+      {
+        const int c = 2 * (t & 63), j0 = 16 * (t >> 6);
 #pragma unroll
-      for (int u = 0; u < 32; u += 4) {
-        float bk[4];
+        for (int h8 = 0; h8 < 16; h8 += 8) {
+          float g0[8], g1[8], k0[8], k1[8], q0[8], q1[8], bb[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = i0 + u + e;
-          const float gmm = sAl[al_off(i, c)];
-          bk[e] = sB[i] * gmm * bf(sKr + i * DK + c);
-          if constexpr (GATED) bk[e] *= sRN[i];
-          sAl[al_off(i, c)] = gmm * bf(sQr + i * DK + c);  // Qhat (fp32, in place)
+          for (int e = 0; e < 8; ++e) {
+            const int i = j0 + h8 + e;
+            const float2 gm = *reinterpret_cast<const float2 *>(sAl + al_off(i, c));
+            const uint32_t kw = *reinterpret_cast<const uint32_t *>(sKr + i * DK + c);
+            const uint32_t qw = *reinterpret_cast<const uint32_t *>(sQr + i * DK + c);
+            g0[e] = gm.x; g1[e] = gm.y;
+            k0[e] = __uint_as_float(kw << 16); k1[e] = __uint_as_float(kw & 0xffff0000u);
+            q0[e] = __uint_as_float(qw << 16); q1[e] = __uint_as_float(qw & 0xffff0000u);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; e += 4) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(sB + j0 + h8 + e);
+            bb[e] = b4.x; bb[e + 1] = b4.y; bb[e + 2] = b4.z; bb[e + 3] = b4.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e)  // Qhat (fp32, in place)
+            *reinterpret_cast<float2 *>(sAl + al_off(j0 + h8 + e, c)) = make_float2(g0[e] * q0[e], g1[e] * q1[e]);
+#pragma unroll
+          for (int g = 0; g < 8; g += 4) {
+            float x0[4], x1[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float b0 = bb[g + e] * g0[g + e] * k0[g + e], b1 = bb[g + e] * g1[g + e] * k1[g + e];
+              if constexpr (GATED) {
+                b0 *= sRN[j0 + h8 + g + e];
+                b1 *= sRN[j0 + h8 + g + e];
+              }
+              x0[e] = sw ? b1 : b0;
+              x1[e] = sw ? b0 : b1;
+            }
+            st4_f32(GA + off_k_sw128_f32(c + (sw ? 1 : 0), j0 + h8 + g, DK + DV), x0[0], x0[1], x0[2], x0[3]);
+            st4_f32(GA + off_k_sw128_f32(c + (sw ? 0 : 1), j0 + h8 + g, DK + DV), x1[0], x1[1], x1[2], x1[3]);
+          }
         }
-        st4_f32(GA + off_k_sw128_f32(c, i0 + u, DK + DV), bk[0], bk[1], bk[2], bk[3]);
       }
       // beta V rows 128 .. 128 + DV: thread (channel pair cp, 16-token quarter);
       // the two rows' stores alternate their order on lane bit 2 (rows 2 cp
@@ -799,7 +873,6 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           const float4 b4 = *reinterpret_cast<const float4 *>(sB + j0 + e);
           bb[e] = b4.x; bb[e + 1] = b4.y; bb[e + 2] = b4.z; bb[e + 3] = b4.w;
         }
-        const bool sw = (lane >> 2) & 1;
 #pragma unroll
         for (int g = 0; g < 16; g += 4) {
           float x0[4], x1[4];
