@@ -127,14 +127,14 @@ constexpr uint32_t P_GA = 0;          // 65536 Lk/Lq (M128 x K128, MN-major; row
 constexpr uint32_t P_GB = 49152;      // 49152 R stack (N96 x K128, MN-major)
 constexpr uint32_t P_T = 65536;       // 17408 T fp32 [64][68] (after the Grams)
 constexpr uint32_t P_XT = P_T + 17408; //  3072 solve scratch
-constexpr uint32_t P_OU = 65536;      // <=65536 staged [M Ut ; Ut] rows (epilogue)
+constexpr uint32_t P_OU = 65536;      // <=32768 staged M Ut rows (epilogue; Ut rows at P_A)
 constexpr uint32_t P_V = 98304;       // 16384 raw v bf16 [64][dv] (until beta V is built)
 constexpr uint32_t P_B0 = 98304;      // 16384 T (K64 x N64 MN)
 constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128]
 constexpr uint32_t P_K = 131072;      // 16384 raw k bf16 [64][128]
 constexpr uint32_t P_A0 = 114688;     // 32768 [M ; I] (128 x 64 K-major), over raw q and k
 constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
-constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68]
+constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68] (with P_M: staged Ut rows, epilogue)
 constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
 constexpr uint32_t P_B = 216064;      //   256 beta
 constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..3] + TMEM address + flag
@@ -306,9 +306,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
         if constexpr (GATED) bv = gate_beta(ga, bv);
       }
-      // the previous item's bulk stores read staging that overlaps v and q
-      if (tid == 0) bulk_wait_read0();
-      __syncthreads();
+      // (the previous item's bulk stores may still read its staging, which
+      // lies outside every buffer written here)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
@@ -356,6 +355,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
         if (idx < C * nv) *reinterpret_cast<uint4 *>(sm + P_V + idx * 16) = vr[u];
       }
       if (tid < C) sB[tid] = bv;
+      // the gate pass writes over the staging: the stores must have read it
+      if (tid == 0) bulk_wait_read0();
     }
     __syncthreads();
 
@@ -962,8 +963,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
             st4_f32(sm + P_GA + off_k_sw128_f32(row, cb + e, DK), x[e], x[e + 1], x[e + 2], x[e + 3]);
-        } else {  // [M Ut ; Ut] rows, fp32, pieces swizzled by row
-          uint8_t *dst = sm + P_OU + (size_t)row * DV * 4;
+        } else {  // [M Ut ; Ut] rows, fp32, pieces swizzled by row (Ut rows over A, M)
+          uint8_t *dst = row < C ? sm + P_OU + (size_t)row * DV * 4 : sm + P_A + (size_t)(row - C) * DV * 4;
           const int pc0 = (cb - DK) >> 2;
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
@@ -976,7 +977,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     __syncthreads();
     if (tid == 0) {
       bulk_s2g(wsb + WS_A1, sm + P_GA, 65536);
-      bulk_s2g(wsb + WS_OU, sm + P_OU, 128u * DV * 4u);
+      bulk_s2g(wsb + WS_OU, sm + P_OU, 64u * DV * 4u);
+      bulk_s2g(wsb + WS_OU + 64u * DV * 4u, sm + P_A, 64u * DV * 4u);
       bulk_commit();
     }
   } while (0);
