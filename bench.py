@@ -65,8 +65,8 @@ def esize(dt):
 # capture, its command and the scaling are in profiles/. Set to None whenever
 # a kernel changes after its capture.
 NCU_TRAFFIC = {
-    # prep + scan at T=2048, H=32 (1024 chunk-heads): 376.8 MB, x4 for T=8192
-    "prefill": 4 * 376.8e6,
+    # prep + scan at T=2048, H=32 (1024 chunk-heads): 375.9 MB, x4 for T=8192
+    "prefill": 4 * 375.9e6,
     # N=64 (2048 pairs): 214.8 MB, x4 for N=256
     "decode": 4 * 214.8e6,
 }
