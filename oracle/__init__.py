@@ -11,10 +11,11 @@ recurrence of "Semidirect Fourier Delta Attention" §1 eq. (1) / §2.2 eq. (9)
 with the readout of §3 eq. (14); ranges from "Complex KDA", abstract). This
 module only compiles it with gcc (no fast-math) and marshals numpy arrays.
 
-Every function here is pinned by ``tests/test_oracle_pins.py`` and
-``tests/test_oracle_prologue.py`` against the
-lesson's worked traces, closed forms and the dense affine composition
-(§2.2 eq. (10)); none is "parity unpinned".
+Every function here is pinned by ``tests/test_oracle_pins.py``,
+``tests/test_oracle_prologue.py`` and ``tests/test_oracle_bwd.py`` against
+the lesson's worked traces, closed forms, the dense affine composition
+(§2.2 eq. (10)) and, for the backward pass, central finite differences of
+the forward; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -197,3 +198,86 @@ def decode_gated(q, k_raw, v, a_logit, c_logit, state, gates: dict,
     decode (state updated in place)."""
     alpha, beta, k = gate_prologue(a_logit, c_logit, k_raw, **gates)
     return decode(q, k, v, alpha, beta, state, scale, pairs)
+
+
+def _bwd_head(q, k, v, alpha, beta, do, s0, g_final, scale):
+    """Reverse-mode gradients of one (sequence, head) token recurrence, fp64.
+
+    Forward step (state S_prev before token t):
+        S' = diag(alpha_t) S_prev,  w = v_t - S'^T k_t,  S_t = S' + beta_t k_t w^T,
+        o_t = scale S_t^T q_t.
+    Backward step, G = dL/dS_t coming from the later tokens:
+        G += scale q_t do_t^T;  dq_t = scale S_t do_t;  g = G^T k_t;
+        dv_t = beta_t g;  dbeta_t = g . w;  dk_t = beta_t (G w - S' g);
+        dS' = G - beta_t k_t g^T;  dalpha_t = rowsum(dS' * S_prev);
+        G <- diag(alpha_t) dS'  (= dL/dS_prev).
+    """
+    L = q.shape[0]
+    S = s0.copy()
+    prev, ws = [], []
+    for t in range(L):
+        prev.append(S)
+        Sp = alpha[t][:, None] * S
+        w = v[t] - Sp.T @ k[t]
+        S = Sp + beta[t] * np.outer(k[t], w)
+        ws.append(w)
+    dq = np.zeros_like(q); dk = np.zeros_like(k); dv = np.zeros_like(v)
+    dal = np.zeros_like(alpha); dbe = np.zeros_like(beta)
+    G = g_final.copy()
+    for t in range(L - 1, -1, -1):
+        S_prev, w = prev[t], ws[t]
+        Sp = alpha[t][:, None] * S_prev
+        St = Sp + beta[t] * np.outer(k[t], w)
+        G = G + scale * np.outer(q[t], do[t])
+        dq[t] = scale * (St @ do[t])
+        g = G.T @ k[t]
+        dv[t] = beta[t] * g
+        dbe[t] = g @ w
+        dk[t] = beta[t] * (G @ w - Sp @ g)
+        dSp = G - beta[t] * np.outer(k[t], g)
+        dal[t] = (dSp * S_prev).sum(axis=1)
+        G = alpha[t][:, None] * dSp
+    return dq, dk, dv, dal, dbe, G
+
+
+def bwd(q, k, v, alpha, beta, d_o, initial_state=None, d_final_state=None,
+        cu_seqlens=None, scale: float = 1.0, _head=None):
+    """Gradients of the forward (``fwd``) for a loss L with dL/do = d_o and
+    dL/d(final state) = d_final_state (None = 0), in fp64.
+
+    The pages state the forward recurrence only ("Semidirect Fourier Delta
+    Attention" §1 eq. (1), §3 eq. (14)); the backward here is its adjoint,
+    one token at a time in reverse (``_bwd_head``). Shapes as ``fwd``; d_o
+    is [total_T, H, d_v]. Returns (dq, dk, dv, dalpha, dbeta,
+    d_initial_state), the last [N, H, d_k, d_v]. ``_head`` replaces the
+    per-head routine (the mutation tests pass deliberately broken copies).
+    """
+    q, k, v, alpha, beta, d_o = map(_f64, (q, k, v, alpha, beta, d_o))
+    s0 = _f64(initial_state)
+    gf = _f64(d_final_state)
+    T, H, dk_ = q.shape
+    dv_ = v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    if int(cu[-1]) != T:
+        raise ValueError("cu_seqlens[-1] must equal total_T")
+    head = _head or _bwd_head
+    out = [np.zeros_like(q), np.zeros_like(k), np.zeros_like(v),
+           np.zeros_like(alpha), np.zeros_like(beta),
+           np.zeros((N, H, dk_, dv_), dtype=np.float64)]
+    for n in range(N):
+        a, b = int(cu[n]), int(cu[n + 1])
+        for h in range(H):
+            st0 = s0[n, h] if s0 is not None else np.zeros((dk_, dv_))
+            g0 = gf[n, h] if gf is not None else np.zeros((dk_, dv_))
+            r = head(q[a:b, h], k[a:b, h], v[a:b, h], alpha[a:b, h], beta[a:b, h],
+                     d_o[a:b, h], st0, g0, float(scale))
+            for i in range(5):
+                out[i][a:b, h] = r[i]
+            out[5][n, h] = r[5]
+    return tuple(out)
