@@ -81,6 +81,10 @@ def load(path: str | None = None):
                                            i32, f32, ctypes.c_int, GateParams, vp]
     lib.ckda_status_string.restype = ctypes.c_char_p
     lib.ckda_status_string.argtypes = [ctypes.c_int]
+    lib.ckda_bwd.restype = ctypes.c_int
+    lib.ckda_bwd.argtypes = [vp] * 16 + [i32] * 5 + [f32, ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.ckda_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.ckda_bwd_workspace_bytes.argtypes = [i32] * 6
     lib.ckda_last_error.restype = ctypes.c_int
     lib.ckda_last_error.argtypes = [vp]
     lib.ckda_version.restype = ctypes.c_int32
@@ -202,6 +206,60 @@ def _fwd_call(q, k, v, alpha, beta, initial_state, final_state, o, cu_seqlens,
         st = lib.ckda_fwd_chunked_gated(*args, gates, _p(workspace), ws_bytes,
                                         _stream(stream))
         _check(st, "ckda_fwd_chunked_gated")
+
+
+def ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, varlen=False) -> int:
+    """Scratch bytes ckda_bwd needs (see include/ckda.h)."""
+    return int(load().ckda_bwd_workspace_bytes(int(N), int(T), int(H), int(d_k), int(d_v),
+                                               int(bool(varlen))))
+
+
+def ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv,
+             dalpha, dbeta, d_initial_state, cu_seqlens=None, cu_seqlens_host=None,
+             N=None, T=None, scale: float = 1.0, stream=None, workspace=None):
+    """Marshal tensors into ckda_bwd (see include/ckda.h): gradients of
+    ckda_fwd_chunked for dL/do = d_o and dL/d(final state) = d_final_state
+    (None = zero). dq, dk [T_total, H, d_k] and dv [T_total, H, d_v] in q's
+    dtype, dalpha [T_total, H, d_k] and dbeta [T_total, H] fp32 and
+    d_initial_state [N, H, d_k, d_v] fp32 (or None) are written."""
+    lib = load()
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o"), (dq, "dq"), (dk, "dk"),
+                   (dv, "dv")):
+        _need(t, nme, q.dtype, 3)
+    _need(alpha, "alpha", torch.float32, 3)
+    _need(dalpha, "dalpha", torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    _need(dbeta, "dbeta", torch.float32, 2)
+    if q.dtype not in _DT:
+        raise ValueError("q, k, v must be bfloat16 or float32")
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+        T = T_total
+    elif N is None or T is None:
+        raise ValueError("give cu_seqlens, or N and T")
+    for t, nme in ((initial_state, "initial_state"), (d_final_state, "d_final_state"),
+                   (d_initial_state, "d_initial_state")):
+        if t is not None:
+            _need(t, nme, torch.float32, 4)
+    host_ptr = None
+    if cu_seqlens_host is not None:
+        if cu_seqlens_host.is_cuda or cu_seqlens_host.dtype != torch.int32 \
+                or not cu_seqlens_host.is_contiguous():
+            raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
+        host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    need = ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens is not None)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.ckda_bwd(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(initial_state), _p(d_o),
+                      _p(d_final_state), _p(dq), _p(dk), _p(dv), _p(dalpha), _p(dbeta),
+                      _p(d_initial_state), _p(cu_seqlens), host_ptr, int(N), int(T), int(H),
+                      int(d_k), int(d_v), float(scale), _DT[q.dtype], _p(workspace), ws_bytes,
+                      _stream(stream))
+    _check(st, "ckda_bwd")
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # CKDA_NOALLOC_SCRATCH_BYTES in include/ckda.h
@@ -335,6 +393,26 @@ def fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, gates: GateParams,
                            cu_seqlens, cu_seqlens_host, N, T, chunk, scale, stream,
                            workspace)
     return o, sf
+
+
+def bwd(q, k, v, alpha, beta, d_o, initial_state=None, d_final_state=None,
+        cu_seqlens=None, cu_seqlens_host=None, N=None, T=None, scale: float = 1.0,
+        stream=None, workspace=None):
+    """Allocate the gradients with torch, then call ckda_bwd. Returns
+    (dq, dk, dv, dalpha, dbeta, d_initial_state)."""
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+    elif N is None:
+        N, T = 1, T_total
+    dq, dk = torch.empty_like(q), torch.empty_like(k)
+    dv = torch.empty_like(v)
+    dalpha, dbeta = torch.empty_like(alpha), torch.empty_like(beta)
+    ds0 = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=q.device)
+    ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv, dalpha,
+             dbeta, ds0, cu_seqlens, cu_seqlens_host, N, T, scale, stream, workspace)
+    return dq, dk, dv, dalpha, dbeta, ds0
 
 
 def decode_step(q, k, v, alpha, beta, state, scale: float = 1.0, stream=None):

@@ -22,6 +22,14 @@ cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
                             void *o, const int32_t *cu, int N, int T,
                             int T_total, int H, float scale, GateArgs g,
                             unsigned int *err, cudaStream_t st);
+size_t bwd_workspace_bytes(int N, int T_total, int H, int dk, int dv);
+template <typename IOT>
+cudaError_t launch_bwd(int dk, int dv, const void *q, const void *k, const void *v,
+                       const float *alpha, const float *beta, const float *s0,
+                       const void *d_o, const float *dsf, void *dq, void *dk_, void *dv_,
+                       float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
+                       int T, int T_total, int H, float scale, void *ws,
+                       unsigned int *err, cudaStream_t st);
 bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt);
 size_t fwd_tc_workspace_bytes(int N, int T_total, int H, int dv);
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
@@ -131,6 +139,78 @@ ckda_status ckda_last_error(cudaStream_t stream) {
       cudaMemcpyToSymbol(g_ckda_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return CKDA_ERR_CUDA;
   return w ? CKDA_ERR_DEVICE : CKDA_OK;
+}
+
+size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                int32_t d_v, int32_t varlen) {
+  if (N <= 0 || T < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v)) return 0;
+  const int64_t T_total = varlen ? (int64_t)T : (int64_t)N * T;
+  if (T_total > INT32_MAX) return 0;
+  return ckda::bwd_workspace_bytes(N, (int)T_total, H, d_k, d_v);
+}
+
+ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *alpha,
+                     const float *beta, const float *initial_state, const void *d_o,
+                     const float *d_final_state, void *dq, void *dk, void *dv,
+                     float *dalpha, float *dbeta, float *d_initial_state,
+                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, int32_t N,
+                     int32_t T, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                     ckda_dtype dt, void *workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
+  if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!q || !k || !v || !alpha || !beta || !d_o || !dq || !dk || !dv || !dalpha || !dbeta)
+    return CKDA_ERR_ARG;
+  const void *ptrs[] = {q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk,
+                        dv, dalpha, dbeta, d_initial_state, cu_seqlens, workspace};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return CKDA_ERR_ARG;
+  int64_t T_total;
+  if (cu_seqlens == nullptr) {
+    if (cu_seqlens_host) return CKDA_ERR_ARG;
+    T_total = (int64_t)N * T;
+  } else {
+    T_total = T;
+    if (cu_seqlens_host) {
+      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return CKDA_ERR_ARG;
+      for (int32_t n = 0; n < N; ++n)
+        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return CKDA_ERR_ARG;
+    }
+  }
+  if (T_total > INT32_MAX) return CKDA_ERR_ARG;
+  // no output may overlap an input, another output or the workspace
+  const size_t es = esize(dt), th = (size_t)T_total * H;
+  const size_t kb = th * d_k * es, vb = th * d_v * es, ab = th * d_k * sizeof(float);
+  const size_t bb = th * sizeof(float), sb = (size_t)N * H * d_k * d_v * sizeof(float);
+  const size_t need = ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens != nullptr);
+  struct R { const void *p; size_t n; };
+  const R ins[] = {{q, kb}, {k, kb}, {v, vb}, {alpha, ab}, {beta, bb}, {initial_state, sb},
+                   {d_o, vb}, {d_final_state, sb},
+                   {cu_seqlens, cu_seqlens ? (size_t)(N + 1) * sizeof(int32_t) : 0}};
+  const R outs[] = {{dq, kb}, {dk, kb}, {dv, vb}, {dalpha, ab}, {dbeta, bb},
+                    {d_initial_state, sb}, {workspace, need}};
+  for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+    for (const R &x : ins)
+      if (overlaps(outs[i].p, outs[i].n, x.p, x.n)) return CKDA_ERR_ARG;
+    for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+      if (overlaps(outs[i].p, outs[i].n, outs[j].p, outs[j].n)) return CKDA_ERR_ARG;
+  }
+  if (N == 0) return CKDA_OK;
+  if (!workspace || workspace_bytes < need) return CKDA_ERR_ARG;
+  unsigned int *err = error_word_ptr();
+  cudaError_t e;
+  if (dt == CKDA_F32)
+    e = ckda::launch_bwd<float>(d_k, d_v, q, k, v, alpha, beta, initial_state, d_o,
+                                d_final_state, dq, dk, dv, dalpha, dbeta, d_initial_state,
+                                cu_seqlens, N, T, (int)T_total, H, scale, workspace, err,
+                                stream);
+  else
+    e = ckda::launch_bwd<__nv_bfloat16>(d_k, d_v, q, k, v, alpha, beta, initial_state, d_o,
+                                        d_final_state, dq, dk, dv, dalpha, dbeta,
+                                        d_initial_state, cu_seqlens, N, T, (int)T_total, H,
+                                        scale, workspace, err, stream);
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
 size_t ckda_fwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,

@@ -1,0 +1,356 @@
+// Backward pass of the CKDA recurrence on CUDA cores (sm_100a).
+//
+// The forward, per (sequence, head) and token t, with S_prev the state before
+// the step ("Semidirect Fourier Delta Attention" §1 eq. (1), readout §3 eq. (14)):
+//   S' = diag(alpha_t) S_prev,  w = v_t - S'^T k_t,  S_t = S' + beta_t k_t w^T,
+//   o_t = scale S_t^T q_t.
+// Its adjoint, going backwards with G = dL/dS_t (d_final_state at the end):
+//   G += scale q_t do_t^T;  dq_t = scale S_t do_t;  g = G^T k_t;
+//   dv_t = beta_t g;  dbeta_t = g . w;  dk_t = beta_t (G w - S' g);
+//   dS' = G - beta_t k_t g^T;  dalpha_t = rowsum(dS' * S_prev);
+//   G <- diag(alpha_t) dS'   (and d_initial_state = G after the first token).
+//
+// One CTA per (sequence, head); thread (row r, column quarter cq) keeps
+// d_v/4 columns of row r of the state (forward) or of G (backward) in
+// registers. Pass 1 runs the forward and stores the state every CK = 16
+// tokens (checkpoint slots in the workspace). Pass 2 walks the 16-token
+// chunks backwards: it reloads the chunk's checkpoint, recomputes the
+// chunk's pre-step states into a per-CTA buffer (w into shared memory), then
+// runs the chunk's reverse steps. Every chunk's inputs are staged in shared
+// memory once. The only reduction across rows (a column sum: p = S'^T k
+// forward, g = G^T k backward) is a reduce-scatter over the 8 row lanes of a
+// warp followed by a fixed-order sum across warps, so results are
+// deterministic; sums across a row are shuffles among 4 lanes.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "ckda.h"
+#include "ckda_common.cuh"
+
+namespace ckda {
+namespace {
+
+constexpr int CK = 16;  // tokens between checkpoints
+
+// first checkpoint slot of sequence n; chunk c of it sits at slot + c, which
+// never collides and stays below floor(T_total / CK) + N
+__device__ __forceinline__ int bwd_slot_base(const int32_t *cu, int n, int T) {
+  const int b = cu ? __ldg(cu + n) : n * T;
+  return b / CK + n;
+}
+
+template <int DK, int DV>
+struct BwdShape {
+  static constexpr int NT = 4 * DK;     // threads
+  static constexpr int NW = NT / 32;    // warps
+  static constexpr int CPT = DV / 4;    // columns per thread
+  // shared memory (floats): chunk inputs q, k, alpha [CK][DK]; v, do, w
+  // [CK][DV]; beta [CK]; column-sum partials [NW][DV] and sums [DV]
+  static constexpr int OFF_Q = 0, OFF_K = OFF_Q + CK * DK, OFF_A = OFF_K + CK * DK;
+  static constexpr int OFF_V = OFF_A + CK * DK, OFF_DO = OFF_V + CK * DV;
+  static constexpr int OFF_W = OFF_DO + CK * DV, OFF_B = OFF_W + CK * DV;
+  static constexpr int OFF_P = OFF_B + CK, OFF_CS = OFF_P + NW * DV;
+  static constexpr int FLOATS = OFF_CS + DV;
+};
+
+// Column sums of x (this thread's CPT columns of row r) over all DK rows;
+// x is replaced by the sums of the same columns. Two CTA barriers.
+template <int DK, int DV>
+__device__ __forceinline__ void col_sum(float (&x)[DV / 4], float *sm, int tid) {
+  using B = BwdShape<DK, DV>;
+  constexpr int CPT = B::CPT;
+  const int lane = tid & 31, warp = tid >> 5, cq = lane & 3;
+  // reduce-scatter over lane bits 4, 3, 2 (the row lanes) while a lane holds
+  // two values or more; all-reduce after that
+  int off = 0;
+  bool writer = true;
+  constexpr int n1 = CPT, n2 = n1 >= 2 ? n1 / 2 : 1, n3 = n2 >= 2 ? n2 / 2 : 1;
+  constexpr int nf = n3 >= 2 ? n3 / 2 : 1;
+#pragma unroll
+  for (int level = 0; level < 3; ++level) {
+    const int m = 16 >> level;
+    const int n = level == 0 ? n1 : (level == 1 ? n2 : n3);
+    const bool up = (lane & m) != 0;
+    if (n >= 2) {
+      const int half = n / 2;
+#pragma unroll
+      for (int e = 0; e < CPT / 2; ++e) {
+        if (e < half) {
+          const float keep = up ? x[half + e] : x[e];
+          const float send = up ? x[e] : x[half + e];
+          x[e] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+        }
+      }
+      off += up ? half : 0;
+    } else {
+      x[0] += __shfl_xor_sync(0xffffffffu, x[0], m);
+      writer = writer && !up;
+    }
+  }
+  float *part = sm + B::OFF_P, *cs = sm + B::OFF_CS;
+  if (writer) {
+#pragma unroll
+    for (int e = 0; e < nf; ++e) part[warp * DV + cq * CPT + off + e] = x[e];
+  }
+  __syncthreads();
+  for (int c = tid; c < DV; c += B::NT) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < B::NW; ++w) s += part[w * DV + c];
+    cs[c] = s;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) x[j] = cs[cq * CPT + j];
+}
+
+// sum over the 4 lanes of one row
+__device__ __forceinline__ float row_sum4(float x) {
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  return x;
+}
+
+// stage tokens [t0, t0 + L) of head h into shared memory as fp32
+template <typename IOT, int DK, int DV>
+__device__ __forceinline__ void stage_chunk(float *sm, const IOT *q, const IOT *k, const IOT *v,
+                                            const float *alpha, const float *beta,
+                                            const IOT *d_o, int t0, int L, int H, int h,
+                                            int tid) {
+  using B = BwdShape<DK, DV>;
+  for (int i = tid; i < L * DK; i += B::NT) {
+    const int t = i / DK, r = i - t * DK;
+    const size_t g = ((size_t)(t0 + t) * H + h) * DK + r;
+    sm[B::OFF_Q + t * DK + r] = IO<IOT>::ld(q + g);
+    sm[B::OFF_K + t * DK + r] = IO<IOT>::ld(k + g);
+    sm[B::OFF_A + t * DK + r] = __ldg(alpha + g);
+  }
+  for (int i = tid; i < L * DV; i += B::NT) {
+    const int t = i / DV, c = i - t * DV;
+    const size_t g = ((size_t)(t0 + t) * H + h) * DV + c;
+    sm[B::OFF_V + t * DV + c] = IO<IOT>::ld(v + g);
+    sm[B::OFF_DO + t * DV + c] = d_o ? IO<IOT>::ld(d_o + g) : 0.f;
+  }
+  for (int t = tid; t < L; t += B::NT) sm[B::OFF_B + t] = __ldg(beta + (size_t)(t0 + t) * H + h);
+}
+
+// one forward step on this thread's columns of row r; w (column values) is
+// written to shared memory row tl by the row-0 threads
+template <int DK, int DV>
+__device__ __forceinline__ void fwd_step(float (&S)[DV / 4], float *sm, int tl, int r, int cq,
+                                         int tid, bool store_w) {
+  using B = BwdShape<DK, DV>;
+  constexpr int CPT = B::CPT;
+  const float kr = sm[B::OFF_K + tl * DK + r], ar = sm[B::OFF_A + tl * DK + r];
+  const float bt = sm[B::OFF_B + tl];
+  float x[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) x[j] = (ar * S[j]) * kr;
+  col_sum<DK, DV>(x, sm, tid);  // p = S'^T k
+  const float *vv = sm + B::OFF_V + tl * DV + cq * CPT;
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) {
+    const float w = vv[j] - x[j];
+    S[j] = ar * S[j] + kr * (bt * w);
+    x[j] = w;
+  }
+  if (store_w && r == 0) {
+#pragma unroll
+    for (int j = 0; j < CPT; ++j) sm[B::OFF_W + tl * DV + cq * CPT + j] = x[j];
+  }
+}
+
+template <typename IOT, int DK, int DV>
+__global__ void __launch_bounds__(4 * DK, 1)
+ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT *__restrict__ v,
+                const float *__restrict__ alpha, const float *__restrict__ beta,
+                const float *__restrict__ s0, const IOT *__restrict__ d_o,
+                const float *__restrict__ dsf, IOT *__restrict__ dq, IOT *__restrict__ dk,
+                IOT *__restrict__ dv, float *__restrict__ dalpha, float *__restrict__ dbeta,
+                float *__restrict__ ds0, const int32_t *__restrict__ cu, int T, int T_total,
+                int H, float scale, float *__restrict__ ck, float *__restrict__ buf,
+                unsigned int *err) {
+  using B = BwdShape<DK, DV>;
+  constexpr int CPT = B::CPT;
+  extern __shared__ float sm[];
+  const int tid = threadIdx.x, r = tid >> 2, cq = tid & 3;
+  const int h = blockIdx.x, n = blockIdx.y;
+  int bos, eos;
+  seq_bounds(cu, n, T, T_total, err, bos, eos);
+  const int len = eos - bos, nck = (len + CK - 1) / CK;
+  const int slot0 = bwd_slot_base(cu, n, T);
+  const size_t st_off = ((size_t)n * H + h) * DK * DV + (size_t)r * DV + cq * CPT;
+  const size_t row_off = (size_t)r * DV + cq * CPT;  // within one DK x DV state
+  float *mybuf = buf + ((size_t)n * H + h) * CK * DK * DV;
+
+  // ---- pass 1: forward, a checkpoint at the start of every chunk
+  float S[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) S[j] = s0 ? s0[st_off + j] : 0.f;
+  for (int i = 0; i < nck; ++i) {
+    const int t0 = bos + CK * i, L = min(CK, eos - t0);
+    float *cp = ck + ((size_t)(slot0 + i) * H + h) * DK * DV + row_off;
+#pragma unroll
+    for (int j = 0; j < CPT; j += 4)
+      *reinterpret_cast<float4 *>(cp + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    __syncthreads();  // the previous chunk's readers of the staged inputs are done
+    stage_chunk<IOT, DK, DV>(sm, q, k, v, alpha, beta, nullptr, t0, L, H, h, tid);
+    __syncthreads();
+    for (int tl = 0; tl < L; ++tl) fwd_step<DK, DV>(S, sm, tl, r, cq, tid, false);
+  }
+
+  // ---- pass 2: chunks in reverse; recompute the pre-step states, then the
+  // reverse steps
+  float G[CPT];
+#pragma unroll
+  for (int j = 0; j < CPT; ++j) G[j] = dsf ? dsf[st_off + j] : 0.f;
+  for (int i = nck - 1; i >= 0; --i) {
+    const int t0 = bos + CK * i, L = min(CK, eos - t0);
+    const float *cp = ck + ((size_t)(slot0 + i) * H + h) * DK * DV + row_off;
+#pragma unroll
+    for (int j = 0; j < CPT; j += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(cp + j);
+      S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+    }
+    __syncthreads();
+    stage_chunk<IOT, DK, DV>(sm, q, k, v, alpha, beta, d_o, t0, L, H, h, tid);
+    __syncthreads();
+    for (int tl = 0; tl < L; ++tl) {
+      float *bp = mybuf + (size_t)tl * DK * DV + row_off;
+#pragma unroll
+      for (int j = 0; j < CPT; j += 4)
+        *reinterpret_cast<float4 *>(bp + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+      fwd_step<DK, DV>(S, sm, tl, r, cq, tid, true);
+    }
+    __syncthreads();  // w rows in shared memory
+    for (int tl = L - 1; tl >= 0; --tl) {
+      const size_t tok = (size_t)(t0 + tl) * H + h;
+      const float qr = sm[B::OFF_Q + tl * DK + r], kr = sm[B::OFF_K + tl * DK + r];
+      const float ar = sm[B::OFF_A + tl * DK + r], bt = sm[B::OFF_B + tl];
+      const float *wv = sm + B::OFF_W + tl * DV + cq * CPT;
+      const float *dov = sm + B::OFF_DO + tl * DV + cq * CPT;
+      const float *bp = mybuf + (size_t)tl * DK * DV + row_off;
+      float sp[CPT];
+#pragma unroll
+      for (int j = 0; j < CPT; j += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(bp + j);
+        sp[j] = x.x; sp[j + 1] = x.y; sp[j + 2] = x.z; sp[j + 3] = x.w;
+      }
+      float dqp = 0.f;
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        G[j] += scale * qr * dov[j];
+        const float st = ar * sp[j] + kr * (bt * wv[j]);  // S_t
+        dqp += st * dov[j];
+      }
+      const float dqr = scale * row_sum4(dqp);
+      float g[CPT];
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) g[j] = G[j] * kr;
+      col_sum<DK, DV>(g, sm, tid);  // g = G^T k
+      float dkp = 0.f, dap = 0.f, dbp = 0.f;
+#pragma unroll
+      for (int j = 0; j < CPT; ++j) {
+        const float spj = ar * sp[j];  // S'
+        dkp += G[j] * wv[j] - spj * g[j];
+        const float dspj = G[j] - bt * kr * g[j];  // dS'
+        dap += dspj * sp[j];
+        G[j] = ar * dspj;
+        dbp += g[j] * wv[j];
+      }
+      const float dkr = bt * row_sum4(dkp), dar = row_sum4(dap), dbt = row_sum4(dbp);
+      if (cq == 0) {
+        IO<IOT>::st(dq + tok * DK + r, dqr);
+        IO<IOT>::st(dk + tok * DK + r, dkr);
+        dalpha[tok * DK + r] = dar;
+      }
+      if (r == 0) {
+#pragma unroll
+        for (int j = 0; j < CPT; ++j) IO<IOT>::st(dv + tok * DV + cq * CPT + j, bt * g[j]);
+        if (cq == 0) dbeta[tok] = dbt;
+      }
+    }
+  }
+  if (ds0) {
+#pragma unroll
+    for (int j = 0; j < CPT; j += 4)
+      *reinterpret_cast<float4 *>(ds0 + st_off + j) = make_float4(G[j], G[j + 1], G[j + 2], G[j + 3]);
+  }
+}
+
+template <typename IOT, int DK, int DV>
+cudaError_t launch_bwd_dims(const void *q, const void *k, const void *v, const float *alpha,
+                            const float *beta, const float *s0, const void *d_o,
+                            const float *dsf, void *dq, void *dk, void *dv, float *dalpha,
+                            float *dbeta, float *ds0, const int32_t *cu, int N, int T,
+                            int T_total, int H, float scale, float *ck, float *buf,
+                            unsigned int *err, cudaStream_t st) {
+  using B = BwdShape<DK, DV>;
+  auto kern = ckda_bwd_kernel<IOT, DK, DV>;
+  const size_t smem = (size_t)B::FLOATS * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(H, N), B::NT, smem, st>>>(
+      static_cast<const IOT *>(q), static_cast<const IOT *>(k), static_cast<const IOT *>(v),
+      alpha, beta, s0, static_cast<const IOT *>(d_o), dsf, static_cast<IOT *>(dq),
+      static_cast<IOT *>(dk), static_cast<IOT *>(dv), dalpha, dbeta, ds0, cu, T, T_total, H,
+      scale, ck, buf, err);
+  return cudaGetLastError();
+}
+
+template <typename IOT, int DK>
+cudaError_t launch_bwd_dv(int dv_, const void *q, const void *k, const void *v,
+                          const float *alpha, const float *beta, const float *s0,
+                          const void *d_o, const float *dsf, void *dq, void *dk, void *dv,
+                          float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
+                          int T, int T_total, int H, float scale, float *ck, float *buf,
+                          unsigned int *err, cudaStream_t st) {
+#define CKDA_BWD_DV(X)                                                                          \
+  if (dv_ == X)                                                                                 \
+    return launch_bwd_dims<IOT, DK, X>(q, k, v, alpha, beta, s0, d_o, dsf, dq, dk, dv, dalpha, \
+                                       dbeta, ds0, cu, N, T, T_total, H, scale, ck, buf, err, st);
+  CKDA_BWD_DV(16) CKDA_BWD_DV(32) CKDA_BWD_DV(64) CKDA_BWD_DV(128)
+#undef CKDA_BWD_DV
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t bwd_workspace_bytes(int N, int T_total, int H, int dk, int dv) {
+  const size_t slots = (size_t)T_total / CK + (size_t)N;
+  const size_t state = (size_t)dk * dv * sizeof(float);
+  return slots * H * state + (size_t)N * H * CK * state;
+}
+
+template <typename IOT>
+cudaError_t launch_bwd(int dk_, int dv_, const void *q, const void *k, const void *v,
+                       const float *alpha, const float *beta, const float *s0,
+                       const void *d_o, const float *dsf, void *dq, void *dk, void *dv,
+                       float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
+                       int T, int T_total, int H, float scale, void *ws,
+                       unsigned int *err, cudaStream_t st) {
+  float *ck = static_cast<float *>(ws);
+  const size_t slots = (size_t)T_total / CK + (size_t)N;
+  float *buf = ck + slots * H * (size_t)dk_ * dv_;
+#define CKDA_BWD_DK(X)                                                                        \
+  if (dk_ == X)                                                                               \
+    return launch_bwd_dv<IOT, X>(dv_, q, k, v, alpha, beta, s0, d_o, dsf, dq, dk, dv, dalpha, \
+                                 dbeta, ds0, cu, N, T, T_total, H, scale, ck, buf, err, st);
+  CKDA_BWD_DK(16) CKDA_BWD_DK(32) CKDA_BWD_DK(64) CKDA_BWD_DK(128)
+#undef CKDA_BWD_DK
+  return cudaErrorInvalidValue;
+}
+
+template cudaError_t launch_bwd<float>(int, int, const void *, const void *, const void *,
+                                       const float *, const float *, const float *,
+                                       const void *, const float *, void *, void *, void *,
+                                       float *, float *, float *, const int32_t *, int, int,
+                                       int, int, float, void *, unsigned int *, cudaStream_t);
+template cudaError_t launch_bwd<__nv_bfloat16>(int, int, const void *, const void *,
+                                               const void *, const float *, const float *,
+                                               const float *, const void *, const float *,
+                                               void *, void *, void *, float *, float *,
+                                               float *, const int32_t *, int, int, int, int,
+                                               float, void *, unsigned int *, cudaStream_t);
+
+}  // namespace ckda

@@ -238,3 +238,13 @@ def make_gated_decode_tokens(w: Workload, step: int, N: int | None = None,
     c = 1.5 * torch.randn(N, H, generator=g, dtype=torch.float32)
     return dict(q=q.to(dt), k_raw=k.to(dt), v=v.to(dt), a_logit=a.to(dt).contiguous(),
                 c_logit=c.contiguous())
+
+
+def make_bwd_grads(w: Workload, T_total: int, H: int, N: int, seed_offset: int = 0) -> dict:
+    """Seeded upstream gradients for a backward pass: d_o ~ N(0, 1)
+    [T_total, H, d_v] in the I/O dtype and d_final_state ~ N(0, 1)
+    [N, H, d_k, d_v] fp32."""
+    g = _gen(w.seed + 4242 + seed_offset)
+    d_o = torch.randn(T_total, H, w.d_v, generator=g, dtype=torch.float32)
+    dsf = torch.randn(N, H, w.d_k, w.d_v, generator=g, dtype=torch.float32)
+    return dict(d_o=d_o.to(TORCH_DTYPE[w.dtype]), d_final_state=dsf)

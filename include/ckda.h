@@ -228,6 +228,55 @@ ckda_status ckda_decode_step_gated(const void *q, const void *k_raw, const void 
                                    ckda_dtype dt, ckda_gate_params gp,
                                    cudaStream_t stream);
 
+/*
+ * ckda_bwd: gradients of ckda_fwd_chunked's outputs with respect to its
+ * inputs, for a scalar loss L with dL/do = d_o and dL/d(final state) =
+ * d_final_state. The pages state the forward recurrence only ("Semidirect
+ * Fourier Delta Attention" §1 eq. (1), §3 eq. (14)); this is its adjoint, one
+ * token at a time in reverse, with S_prev the state before token t:
+ *   S' = diag(alpha_t) S_prev,  w = v_t - S'^T k_t,  S_t = S' + beta_t k_t w^T;
+ *   G += scale q_t do_t^T;  dq_t = scale S_t do_t;  g = G^T k_t;
+ *   dv_t = beta_t g;  dbeta_t = g . w;  dk_t = beta_t (G w - S' g);
+ *   dS' = G - beta_t k_t g^T;  dalpha_t = rowsum(dS' * S_prev);  G <- diag(alpha_t) dS'
+ * starting from G = d_final_state, ending with d_initial_state = G.
+ *
+ *   q, k, v, alpha, beta, initial_state, cu_seqlens, cu_seqlens_host, N, T,
+ *               H, d_k, d_v, scale, dt: as for ckda_fwd_chunked (the same
+ *               call's inputs; initial_state NULL = zero).
+ *   d_o         [total_T, H, d_v], dtype dt: gradient of the output.
+ *   d_final_state [N, H, d_k, d_v] fp32, or NULL (= zero).
+ *   dq, dk      [total_T, H, d_k], dtype dt (outputs).
+ *   dv          [total_T, H, d_v], dtype dt (output).
+ *   dalpha      [total_T, H, d_k] fp32 (output).
+ *   dbeta       [total_T, H] fp32 (output).
+ *   d_initial_state [N, H, d_k, d_v] fp32 (output), or NULL (not written).
+ *   workspace   device scratch of at least ckda_bwd_workspace_bytes() bytes,
+ *               owned by the caller (state checkpoints every 16 tokens and a
+ *               16-state buffer per (sequence, head)); required when N > 0.
+ * Every pointer must be 16-byte aligned; no output may overlap an input,
+ * another output or the workspace (CKDA_ERR_ARG). d_k, d_v in {16, 32, 64,
+ * 128}, dt in {CKDA_BF16, CKDA_F32} (else CKDA_ERR_UNSUPPORTED). The call is
+ * asynchronous on `stream`; device-side errors (malformed device cu_seqlens)
+ * surface through ckda_last_error(). Results are deterministic (no atomics).
+ * One CTA per (sequence, head) walks the tokens on CUDA cores.
+ */
+ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *alpha,
+                     const float *beta, const float *initial_state, const void *d_o,
+                     const float *d_final_state, void *dq, void *dk, void *dv,
+                     float *dalpha, float *dbeta, float *d_initial_state,
+                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, int32_t N,
+                     int32_t T, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                     ckda_dtype dt, void *workspace, size_t workspace_bytes,
+                     cudaStream_t stream);
+
+/*
+ * ckda_bwd_workspace_bytes: scratch ckda_bwd needs (T as in ckda_bwd; varlen
+ * nonzero when cu_seqlens is given, so that T is total_T). 0 for unsupported
+ * or invalid sizes.
+ */
+size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                int32_t d_v, int32_t varlen);
+
 /* Static description of a status code (never NULL). */
 const char *ckda_status_string(ckda_status s);
 

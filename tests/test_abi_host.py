@@ -190,3 +190,68 @@ def test_gated_forward_rejects_like_the_plain_one(lib):
     assert lib.ckda_fwd_chunked_gated(P, P2, P3, P4, P5, NULL, NULL, P2, NULL, NULL, 1, 8,
                                       1, 16, 16, 0, 1.0, ckda.CKDA_F32, g, NULL, 0,
                                       None) == ckda.CKDA_ERR_ARG
+
+
+def declared_arities():
+    """Parameter count of every function include/ckda.h declares."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(ckda_[a-z_0-9]+)\s*\(([^)]*)\)\s*;", src):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_argument_counts_match_the_header(lib):
+    """Every ctypes signature the binding declares has the header's arity."""
+    ar = declared_arities()
+    assert "ckda_bwd" in ar and "ckda_bwd_workspace_bytes" in ar
+    for name, n in ar.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is not None:
+            assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+
+
+def bwd(lib, q=P, k=P2, v=P3, a=P4, b=P5, do=P6, dq=ctypes.c_void_p(0x70000),
+        dk=ctypes.c_void_p(0x80000), dv=ctypes.c_void_p(0x90000),
+        da=ctypes.c_void_p(0xA0000), db=ctypes.c_void_p(0xB0000), N=1, T=8, H=1, dkd=16,
+        dvd=16, dt=ckda.CKDA_F32, ws=ctypes.c_void_p(0x100000), wsb=1 << 30):
+    return lib.ckda_bwd(q, k, v, a, b, NULL, do, NULL, dq, dk, dv, da, db, NULL, NULL, NULL,
+                        N, T, H, dkd, dvd, 1.0, dt, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=NULL), ckda.CKDA_ERR_ARG),
+    (dict(do=NULL), ckda.CKDA_ERR_ARG),
+    (dict(db=NULL), ckda.CKDA_ERR_ARG),
+    (dict(k=ODD), ckda.CKDA_ERR_ARG),
+    (dict(H=0), ckda.CKDA_ERR_ARG),
+    (dict(N=-1), ckda.CKDA_ERR_ARG),
+    (dict(dkd=48), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(dvd=256), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(dt=7), ckda.CKDA_ERR_UNSUPPORTED),
+    # a gradient aliasing an input, two gradients aliasing each other
+    (dict(dq=P), ckda.CKDA_ERR_ARG),
+    (dict(dk=ctypes.c_void_p(0x70000)), ckda.CKDA_ERR_ARG),
+    # workspace missing or too small
+    (dict(ws=NULL), ckda.CKDA_ERR_ARG),
+    (dict(wsb=1024), ckda.CKDA_ERR_ARG),
+])
+def test_bwd_rejects(lib, kw, want):
+    assert bwd(lib, **kw) == want
+
+
+def test_bwd_workspace_query(lib):
+    # checkpoints every 16 tokens: floor(T_total / 16) + N slots per head, plus
+    # a 16-state buffer per (sequence, head); fp32 d_k x d_v states
+    st = 32 * 64 * 4
+    assert lib.ckda_bwd_workspace_bytes(2, 40, 3, 32, 64, 0) == ((80 // 16 + 2) * 3 + 2 * 3 * 16) * st
+    assert lib.ckda_bwd_workspace_bytes(2, 40, 3, 32, 64, 1) == ((40 // 16 + 2) * 3 + 2 * 3 * 16) * st
+    assert lib.ckda_bwd_workspace_bytes(1, 8, 1, 48, 16, 0) == 0
+    assert lib.ckda_bwd_workspace_bytes(0, 8, 1, 16, 16, 0) == 0
+
+
+def test_bwd_zero_sequences_is_a_noop(lib):
+    """N = 0: validated, nothing launched, CKDA_OK (the fake pointers are
+    never dereferenced)."""
+    assert bwd(lib, N=0, T=0, ws=NULL, wsb=0) == ckda.CKDA_OK
