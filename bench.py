@@ -31,7 +31,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from gated_delta_rule_114_b200 import ckda  # noqa: E402
-from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,  # noqa: E402
+from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_bwd_grads,  # noqa: E402
+                                              make_decode_state,
                                               make_decode_tokens,
                                               make_fwd_inputs,
                                               make_gated_fwd_inputs)
@@ -108,6 +109,19 @@ def prefill_gated_bytes(inp) -> int:
     N = inp["cu_seqlens"].numel() - 1
     st = N * H * dk * dv * 4
     return T * H * per_th + (st if inp["initial_state"] is not None else 0) + st
+
+
+def bwd_bytes(inp) -> int:
+    """Algorithmic HBM bytes of one backward call: the forward's inputs and
+    do read once, dq, dk, dv, dalpha, dbeta written once per token-head;
+    initial state and final-state gradient read, initial-state gradient
+    written once per (sequence, head)."""
+    T, H, dk = inp["q"].shape
+    dv = inp["v"].shape[2]
+    es = esize(inp["q"].dtype)
+    per_th = ((2 * dk + dv) * es + dk * 4 + 4 + dv * es) + ((2 * dk + dv) * es + dk * 4 + 4)
+    N = inp["cu_seqlens"].numel() - 1
+    return T * H * per_th + 3 * N * H * dk * dv * 4
 
 
 def decode_bytes(N, H, dk, dv, dt) -> int:
@@ -275,6 +289,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=200)
+    ap.add_argument("--bwd-steps", type=int, default=5)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -386,6 +401,34 @@ def main():
              "gpu_launches": 3 * args.steps}
     del gdev
 
+    # ---------------- backward pass of the same workload
+    bg = make_bwd_grads(w, T_total, H, N)
+    bdo, bdsf = bg["d_o"].cuda(), bg["d_final_state"].cuda()
+    bout = [torch.empty_like(dev["q"]), torch.empty_like(dev["k"]), torch.empty_like(dev["v"]),
+            torch.empty_like(dev["alpha"]), torch.empty_like(dev["beta"]),
+            torch.empty((N, H, dk, dv), dtype=torch.float32, device="cuda")]
+    bws = torch.empty(ckda.ckda_bwd_workspace_bytes(N, T_total, H, dk, dv, True),
+                      dtype=torch.uint8, device="cuda")
+
+    def bwd_step():
+        ckda.ckda_bwd(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"],
+                      dev["initial_state"], bdo, bdsf, *bout, dev["cu_seqlens"], None,
+                      stream=stream, workspace=bws)
+
+    bms = time_loop(bwd_step, args.bwd_steps, 3, stream, barrier)
+    if ckda.ckda_last_error() != ckda.CKDA_OK:
+        raise RuntimeError("kernel reported an error")
+    bbytes = bwd_bytes(inp_cpu)
+    backward = {"ms_per_step": bms, "tokens_per_s": T_total * world / (bms / 1e3),
+                "steps": args.bwd_steps, "warmup": 3,
+                "roofline": {"bound": "hbm", "achieved": bbytes / (bms / 1e3) / 1e9,
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": bbytes / (bms / 1e3) / 1e9 / pk["hbm_gbs"],
+                             "traffic": None, "algorithmic_bytes_per_launch": bbytes},
+                "kernel": "token-serial adjoint on CUDA cores, one CTA per (sequence, head)",
+                "gpu_launches": args.bwd_steps}
+    del bws, bout
+
     # ---------------- decode step
     wd = WORKLOADS[DECODE]
     state = make_decode_state(wd).cuda()
@@ -436,7 +479,7 @@ def main():
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         # each forward call launches the slot-table, prep and scan kernels
         "gpu_launches": 3 * args.steps, "clocks": clk.summary(), "decode": decode,
-        "prefill_fused_prologue": gated,
+        "prefill_fused_prologue": gated, "backward": backward,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -44,14 +44,29 @@ struct BwdShape {
   static constexpr int NT = 4 * DK;     // threads
   static constexpr int NW = NT / 32;    // warps
   static constexpr int CPT = DV / 4;    // columns per thread
+  // Per-column vectors keep each column quarter 4 floats apart from the next
+  // (column c at pc(c) = c + 4 (c / CPT), row length DVP): the four quarter
+  // groups of a warp then read four different banks instead of one.
+  static constexpr int DVP = DV + 16;
   // shared memory (floats): chunk inputs q, k, alpha [CK][DK]; v, do, w
-  // [CK][DV]; beta [CK]; column-sum partials [NW][DV] and sums [DV]
+  // [CK][DVP]; beta [CK]; column-sum partials [NW][DVP] and sums [DVP]
   static constexpr int OFF_Q = 0, OFF_K = OFF_Q + CK * DK, OFF_A = OFF_K + CK * DK;
-  static constexpr int OFF_V = OFF_A + CK * DK, OFF_DO = OFF_V + CK * DV;
-  static constexpr int OFF_W = OFF_DO + CK * DV, OFF_B = OFF_W + CK * DV;
-  static constexpr int OFF_P = OFF_B + CK, OFF_CS = OFF_P + NW * DV;
-  static constexpr int FLOATS = OFF_CS + DV;
+  static constexpr int OFF_V = OFF_A + CK * DK, OFF_DO = OFF_V + CK * DVP;
+  static constexpr int OFF_W = OFF_DO + CK * DVP, OFF_B = OFF_W + CK * DVP;
+  static constexpr int OFF_P = OFF_B + CK, OFF_CS = OFF_P + NW * DVP;
+  static constexpr int FLOATS = OFF_CS + DVP;
+  static __device__ __forceinline__ int pc(int c) { return c + 4 * (c / CPT); }
 };
+
+// n (a multiple of 4) consecutive floats of shared memory into registers
+template <int N>
+__device__ __forceinline__ void lds_vec(float *dst, const float *src) {
+#pragma unroll
+  for (int j = 0; j < N; j += 4) {
+    const float4 x = *reinterpret_cast<const float4 *>(src + j);
+    dst[j] = x.x; dst[j + 1] = x.y; dst[j + 2] = x.z; dst[j + 3] = x.w;
+  }
+}
 
 // Column sums of x (this thread's CPT columns of row r) over all DK rows;
 // x is replaced by the sums of the same columns. Two CTA barriers.
@@ -90,18 +105,18 @@ __device__ __forceinline__ void col_sum(float (&x)[DV / 4], float *sm, int tid) 
   float *part = sm + B::OFF_P, *cs = sm + B::OFF_CS;
   if (writer) {
 #pragma unroll
-    for (int e = 0; e < nf; ++e) part[warp * DV + cq * CPT + off + e] = x[e];
+    for (int e = 0; e < nf; ++e) part[warp * B::DVP + cq * (CPT + 4) + off + e] = x[e];
   }
   __syncthreads();
   for (int c = tid; c < DV; c += B::NT) {
     float s = 0.f;
+    const int cp = B::pc(c);
 #pragma unroll
-    for (int w = 0; w < B::NW; ++w) s += part[w * DV + c];
-    cs[c] = s;
+    for (int w = 0; w < B::NW; ++w) s += part[w * B::DVP + cp];
+    cs[cp] = s;
   }
   __syncthreads();
-#pragma unroll
-  for (int j = 0; j < CPT; ++j) x[j] = cs[cq * CPT + j];
+  lds_vec<CPT>(x, cs + cq * (CPT + 4));
 }
 
 // sum over the 4 lanes of one row
@@ -128,8 +143,8 @@ __device__ __forceinline__ void stage_chunk(float *sm, const IOT *q, const IOT *
   for (int i = tid; i < L * DV; i += B::NT) {
     const int t = i / DV, c = i - t * DV;
     const size_t g = ((size_t)(t0 + t) * H + h) * DV + c;
-    sm[B::OFF_V + t * DV + c] = IO<IOT>::ld(v + g);
-    sm[B::OFF_DO + t * DV + c] = d_o ? IO<IOT>::ld(d_o + g) : 0.f;
+    sm[B::OFF_V + t * B::DVP + B::pc(c)] = IO<IOT>::ld(v + g);
+    sm[B::OFF_DO + t * B::DVP + B::pc(c)] = d_o ? IO<IOT>::ld(d_o + g) : 0.f;
   }
   for (int t = tid; t < L; t += B::NT) sm[B::OFF_B + t] = __ldg(beta + (size_t)(t0 + t) * H + h);
 }
@@ -147,7 +162,8 @@ __device__ __forceinline__ void fwd_step(float (&S)[DV / 4], float *sm, int tl, 
 #pragma unroll
   for (int j = 0; j < CPT; ++j) x[j] = (ar * S[j]) * kr;
   col_sum<DK, DV>(x, sm, tid);  // p = S'^T k
-  const float *vv = sm + B::OFF_V + tl * DV + cq * CPT;
+  float vv[CPT];
+  lds_vec<CPT>(vv, sm + B::OFF_V + tl * B::DVP + cq * (CPT + 4));
 #pragma unroll
   for (int j = 0; j < CPT; ++j) {
     const float w = vv[j] - x[j];
@@ -155,8 +171,10 @@ __device__ __forceinline__ void fwd_step(float (&S)[DV / 4], float *sm, int tl, 
     x[j] = w;
   }
   if (store_w && r == 0) {
+    float *wd = sm + B::OFF_W + tl * B::DVP + cq * (CPT + 4);
 #pragma unroll
-    for (int j = 0; j < CPT; ++j) sm[B::OFF_W + tl * DV + cq * CPT + j] = x[j];
+    for (int j = 0; j < CPT; j += 4)
+      *reinterpret_cast<float4 *>(wd + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
   }
 }
 
@@ -227,8 +245,7 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
       const size_t tok = (size_t)(t0 + tl) * H + h;
       const float qr = sm[B::OFF_Q + tl * DK + r], kr = sm[B::OFF_K + tl * DK + r];
       const float ar = sm[B::OFF_A + tl * DK + r], bt = sm[B::OFF_B + tl];
-      const float *wv = sm + B::OFF_W + tl * DV + cq * CPT;
-      const float *dov = sm + B::OFF_DO + tl * DV + cq * CPT;
+      const float *wrow = sm + B::OFF_W + tl * B::DVP + cq * (CPT + 4);
       const float *bp = mybuf + (size_t)tl * DK * DV + row_off;
       float sp[CPT];
 #pragma unroll
@@ -237,11 +254,18 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
         sp[j] = x.x; sp[j + 1] = x.y; sp[j + 2] = x.z; sp[j + 3] = x.w;
       }
       float dqp = 0.f;
+      const float *dorow = sm + B::OFF_DO + tl * B::DVP + cq * (CPT + 4);
 #pragma unroll
-      for (int j = 0; j < CPT; ++j) {
-        G[j] += scale * qr * dov[j];
-        const float st = ar * sp[j] + kr * (bt * wv[j]);  // S_t
-        dqp += st * dov[j];
+      for (int j = 0; j < CPT; j += 4) {
+        float w4[4], d4[4];
+        lds_vec<4>(w4, wrow + j);
+        lds_vec<4>(d4, dorow + j);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          G[j + e] += scale * qr * d4[e];
+          const float st = ar * sp[j + e] + kr * (bt * w4[e]);  // S_t
+          dqp += st * d4[e];
+        }
       }
       const float dqr = scale * row_sum4(dqp);
       float g[CPT];
@@ -250,13 +274,18 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
       col_sum<DK, DV>(g, sm, tid);  // g = G^T k
       float dkp = 0.f, dap = 0.f, dbp = 0.f;
 #pragma unroll
-      for (int j = 0; j < CPT; ++j) {
-        const float spj = ar * sp[j];  // S'
-        dkp += G[j] * wv[j] - spj * g[j];
-        const float dspj = G[j] - bt * kr * g[j];  // dS'
-        dap += dspj * sp[j];
-        G[j] = ar * dspj;
-        dbp += g[j] * wv[j];
+      for (int j = 0; j < CPT; j += 4) {
+        float w4[4];
+        lds_vec<4>(w4, wrow + j);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float spj = ar * sp[j + e];  // S'
+          dkp += G[j + e] * w4[e] - spj * g[j + e];
+          const float dspj = G[j + e] - bt * kr * g[j + e];  // dS'
+          dap += dspj * sp[j + e];
+          G[j + e] = ar * dspj;
+          dbp += g[j + e] * w4[e];
+        }
       }
       const float dkr = bt * row_sum4(dkp), dar = row_sum4(dap), dbt = row_sum4(dbp);
       if (cq == 0) {
