@@ -70,6 +70,8 @@ NCU_TRAFFIC = {
     "prefill": 4 * 375.9e6,
     # N=64 (2048 pairs): 214.8 MB, x4 for N=256
     "decode": 4 * 214.8e6,
+    # backward at T=512, H=32: 153.5 MB, x16 for T=8192
+    "backward": 16 * 153.5e6,
 }
 
 
@@ -424,7 +426,8 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": bbytes / (bms / 1e3) / 1e9,
                              "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": bbytes / (bms / 1e3) / 1e9 / pk["hbm_gbs"],
-                             "traffic": None, "algorithmic_bytes_per_launch": bbytes},
+                             "traffic": NCU_TRAFFIC["backward"],
+                             "algorithmic_bytes_per_launch": bbytes},
                 "kernel": "token-serial adjoint on CUDA cores, one CTA per (sequence, head)",
                 "gpu_launches": args.bwd_steps}
     del bws, bout
