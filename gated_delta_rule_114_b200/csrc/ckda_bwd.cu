@@ -10,9 +10,13 @@
 //   dS' = G - beta_t k_t g^T;  dalpha_t = rowsum(dS' * S_prev);
 //   G <- diag(alpha_t) dS'   (and d_initial_state = G after the first token).
 //
-// One CTA per (sequence, head); thread (row r, column quarter cq) keeps
-// d_v/4 columns of row r of the state (forward) or of G (backward) in
-// registers. Pass 1 runs the forward and stores the state every CK = 16
+// The columns of S (and of G) evolve independently, so one CTA takes one
+// (sequence, head, tile of DVT columns); thread (row r, column quarter cq)
+// keeps DVT/4 columns of row r of the state (forward) or of G (backward) in
+// registers. dv and the initial-state gradient are per column and written by
+// the tile that owns them; dq, dk, dalpha and dbeta sum over all columns, so
+// every tile writes fp32 partials and a second kernel adds the tiles in a
+// fixed order. Pass 1 runs the forward and stores the state every CK = 16
 // tokens (checkpoint slots in the workspace). Pass 2 walks the 16-token
 // chunks backwards: it reloads the chunk's checkpoint, recomputes the
 // chunk's pre-step states into a per-CTA buffer (w into shared memory), then
@@ -23,6 +27,8 @@
 // deterministic; sums across a row are shuffles among 4 lanes.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "ckda.h"
 #include "ckda_common.cuh"
@@ -131,8 +137,8 @@ template <typename IOT, int DK, int DV>
 __device__ __forceinline__ void stage_chunk(float *sm, const IOT *q, const IOT *k, const IOT *v,
                                             const float *alpha, const float *beta,
                                             const IOT *d_o, int t0, int L, int H, int h,
-                                            int tid) {
-  using B = BwdShape<DK, DV>;
+                                            int tid, int DVF, int c0) {
+  using B = BwdShape<DK, DV>;  // DV: the tile width here; DVF: the full d_v
   for (int i = tid; i < L * DK; i += B::NT) {
     const int t = i / DK, r = i - t * DK;
     const size_t g = ((size_t)(t0 + t) * H + h) * DK + r;
@@ -142,7 +148,7 @@ __device__ __forceinline__ void stage_chunk(float *sm, const IOT *q, const IOT *
   }
   for (int i = tid; i < L * DV; i += B::NT) {
     const int t = i / DV, c = i - t * DV;
-    const size_t g = ((size_t)(t0 + t) * H + h) * DV + c;
+    const size_t g = ((size_t)(t0 + t) * H + h) * DVF + c0 + c;
     sm[B::OFF_V + t * B::DVP + B::pc(c)] = IO<IOT>::ld(v + g);
     sm[B::OFF_DO + t * B::DVP + B::pc(c)] = d_o ? IO<IOT>::ld(d_o + g) : 0.f;
   }
@@ -183,23 +189,27 @@ __global__ void __launch_bounds__(4 * DK, 1)
 ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT *__restrict__ v,
                 const float *__restrict__ alpha, const float *__restrict__ beta,
                 const float *__restrict__ s0, const IOT *__restrict__ d_o,
-                const float *__restrict__ dsf, IOT *__restrict__ dq, IOT *__restrict__ dk,
-                IOT *__restrict__ dv, float *__restrict__ dalpha, float *__restrict__ dbeta,
-                float *__restrict__ ds0, const int32_t *__restrict__ cu, int T, int T_total,
-                int H, float scale, float *__restrict__ ck, float *__restrict__ buf,
+                const float *__restrict__ dsf, IOT *__restrict__ dv,
+                float *__restrict__ pq, float *__restrict__ pk, float *__restrict__ pa,
+                float *__restrict__ pb, float *__restrict__ ds0,
+                const int32_t *__restrict__ cu, int T, int T_total, int H, int DVF,
+                float scale, float *__restrict__ ck, float *__restrict__ buf,
                 unsigned int *err) {
-  using B = BwdShape<DK, DV>;
+  using B = BwdShape<DK, DV>;  // DV: the tile width; DVF: the full d_v
   constexpr int CPT = B::CPT;
   extern __shared__ float sm[];
   const int tid = threadIdx.x, r = tid >> 2, cq = tid & 3;
-  const int h = blockIdx.x, n = blockIdx.y;
+  const int h = blockIdx.x, n = blockIdx.y, tile = blockIdx.z, ntile = gridDim.z;
+  const int c0 = tile * DV;
+  const size_t TH = (size_t)T_total * H;
   int bos, eos;
   seq_bounds(cu, n, T, T_total, err, bos, eos);
   const int len = eos - bos, nck = (len + CK - 1) / CK;
   const int slot0 = bwd_slot_base(cu, n, T);
-  const size_t st_off = ((size_t)n * H + h) * DK * DV + (size_t)r * DV + cq * CPT;
-  const size_t row_off = (size_t)r * DV + cq * CPT;  // within one DK x DV state
-  float *mybuf = buf + ((size_t)n * H + h) * CK * DK * DV;
+  const size_t row_off = (size_t)r * DVF + c0 + cq * CPT;  // within one DK x DVF state
+  const size_t st_off = ((size_t)n * H + h) * DK * DVF + row_off;
+  float *mybuf = buf + (((size_t)n * H + h) * ntile + tile) * CK * DK * DV;
+  const size_t brow = (size_t)r * DV + cq * CPT;  // within one buffered DK x DV tile
 
   // ---- pass 1: forward, a checkpoint at the start of every chunk
   float S[CPT];
@@ -207,12 +217,12 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
   for (int j = 0; j < CPT; ++j) S[j] = s0 ? s0[st_off + j] : 0.f;
   for (int i = 0; i < nck; ++i) {
     const int t0 = bos + CK * i, L = min(CK, eos - t0);
-    float *cp = ck + ((size_t)(slot0 + i) * H + h) * DK * DV + row_off;
+    float *cp = ck + ((size_t)(slot0 + i) * H + h) * DK * DVF + row_off;
 #pragma unroll
     for (int j = 0; j < CPT; j += 4)
       *reinterpret_cast<float4 *>(cp + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
     __syncthreads();  // the previous chunk's readers of the staged inputs are done
-    stage_chunk<IOT, DK, DV>(sm, q, k, v, alpha, beta, nullptr, t0, L, H, h, tid);
+    stage_chunk<IOT, DK, DV>(sm, q, k, v, alpha, beta, nullptr, t0, L, H, h, tid, DVF, c0);
     __syncthreads();
     for (int tl = 0; tl < L; ++tl) fwd_step<DK, DV>(S, sm, tl, r, cq, tid, false);
   }
@@ -224,17 +234,17 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
   for (int j = 0; j < CPT; ++j) G[j] = dsf ? dsf[st_off + j] : 0.f;
   for (int i = nck - 1; i >= 0; --i) {
     const int t0 = bos + CK * i, L = min(CK, eos - t0);
-    const float *cp = ck + ((size_t)(slot0 + i) * H + h) * DK * DV + row_off;
+    const float *cp = ck + ((size_t)(slot0 + i) * H + h) * DK * DVF + row_off;
 #pragma unroll
     for (int j = 0; j < CPT; j += 4) {
       const float4 x = *reinterpret_cast<const float4 *>(cp + j);
       S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
     }
     __syncthreads();
-    stage_chunk<IOT, DK, DV>(sm, q, k, v, alpha, beta, d_o, t0, L, H, h, tid);
+    stage_chunk<IOT, DK, DV>(sm, q, k, v, alpha, beta, d_o, t0, L, H, h, tid, DVF, c0);
     __syncthreads();
     for (int tl = 0; tl < L; ++tl) {
-      float *bp = mybuf + (size_t)tl * DK * DV + row_off;
+      float *bp = mybuf + (size_t)tl * DK * DV + brow;
 #pragma unroll
       for (int j = 0; j < CPT; j += 4)
         *reinterpret_cast<float4 *>(bp + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
@@ -246,7 +256,7 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
       const float qr = sm[B::OFF_Q + tl * DK + r], kr = sm[B::OFF_K + tl * DK + r];
       const float ar = sm[B::OFF_A + tl * DK + r], bt = sm[B::OFF_B + tl];
       const float *wrow = sm + B::OFF_W + tl * B::DVP + cq * (CPT + 4);
-      const float *bp = mybuf + (size_t)tl * DK * DV + row_off;
+      const float *bp = mybuf + (size_t)tl * DK * DV + brow;
       float sp[CPT];
 #pragma unroll
       for (int j = 0; j < CPT; j += 4) {
@@ -288,15 +298,16 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
         }
       }
       const float dkr = bt * row_sum4(dkp), dar = row_sum4(dap), dbt = row_sum4(dbp);
-      if (cq == 0) {
-        IO<IOT>::st(dq + tok * DK + r, dqr);
-        IO<IOT>::st(dk + tok * DK + r, dkr);
-        dalpha[tok * DK + r] = dar;
+      if (cq == 0) {  // this tile's share of the row sums
+        const size_t pi = (tile * TH + tok) * DK + r;
+        pq[pi] = dqr;
+        pk[pi] = dkr;
+        pa[pi] = dar;
       }
       if (r == 0) {
 #pragma unroll
-        for (int j = 0; j < CPT; ++j) IO<IOT>::st(dv + tok * DV + cq * CPT + j, bt * g[j]);
-        if (cq == 0) dbeta[tok] = dbt;
+        for (int j = 0; j < CPT; ++j) IO<IOT>::st(dv + tok * DVF + c0 + cq * CPT + j, bt * g[j]);
+        if (cq == 0) pb[tile * TH + tok] = dbt;
       }
     }
   }
@@ -307,48 +318,73 @@ ckda_bwd_kernel(const IOT *__restrict__ q, const IOT *__restrict__ k, const IOT 
   }
 }
 
-template <typename IOT, int DK, int DV>
+// dq, dk, dalpha (n_tk = T_total H d_k entries) and dbeta (n_t = T_total H):
+// the tiles' partials added in tile order
+template <typename IOT>
+__global__ void ckda_bwd_reduce_kernel(const float *__restrict__ pq, const float *__restrict__ pk,
+                                       const float *__restrict__ pa, const float *__restrict__ pb,
+                                       IOT *__restrict__ dq, IOT *__restrict__ dk,
+                                       float *__restrict__ dalpha, float *__restrict__ dbeta,
+                                       size_t n_tk, size_t n_t, int ntile) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_tk;
+       i += (size_t)gridDim.x * blockDim.x) {
+    float a = 0.f, b = 0.f, c = 0.f;
+    for (int t = 0; t < ntile; ++t) {
+      a += pq[t * n_tk + i];
+      b += pk[t * n_tk + i];
+      c += pa[t * n_tk + i];
+    }
+    IO<IOT>::st(dq + i, a);
+    IO<IOT>::st(dk + i, b);
+    dalpha[i] = c;
+    if (i < n_t) {
+      float e = 0.f;
+      for (int t = 0; t < ntile; ++t) e += pb[t * n_t + i];
+      dbeta[i] = e;
+    }
+  }
+}
+
+template <typename IOT, int DK, int DVT>
 cudaError_t launch_bwd_dims(const void *q, const void *k, const void *v, const float *alpha,
                             const float *beta, const float *s0, const void *d_o,
                             const float *dsf, void *dq, void *dk, void *dv, float *dalpha,
                             float *dbeta, float *ds0, const int32_t *cu, int N, int T,
-                            int T_total, int H, float scale, float *ck, float *buf,
-                            unsigned int *err, cudaStream_t st) {
-  using B = BwdShape<DK, DV>;
-  auto kern = ckda_bwd_kernel<IOT, DK, DV>;
+                            int T_total, int H, int DVF, float scale, float *ck, float *buf,
+                            float *pq, float *pk, float *pa, float *pb, unsigned int *err,
+                            cudaStream_t st) {
+  using B = BwdShape<DK, DVT>;
+  auto kern = ckda_bwd_kernel<IOT, DK, DVT>;
   const size_t smem = (size_t)B::FLOATS * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(H, N), B::NT, smem, st>>>(
+  const int ntile = DVF / DVT;
+  kern<<<dim3(H, N, ntile), B::NT, smem, st>>>(
       static_cast<const IOT *>(q), static_cast<const IOT *>(k), static_cast<const IOT *>(v),
-      alpha, beta, s0, static_cast<const IOT *>(d_o), dsf, static_cast<IOT *>(dq),
-      static_cast<IOT *>(dk), static_cast<IOT *>(dv), dalpha, dbeta, ds0, cu, T, T_total, H,
-      scale, ck, buf, err);
+      alpha, beta, s0, static_cast<const IOT *>(d_o), dsf, static_cast<IOT *>(dv), pq, pk, pa,
+      pb, ds0, cu, T, T_total, H, DVF, scale, ck, buf, err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t n_t = (size_t)T_total * H, n_tk = n_t * DK;
+  if (n_tk == 0) return cudaSuccess;
+  const unsigned grid = (unsigned)std::min<size_t>((n_tk + 255) / 256, 148 * 16);
+  ckda_bwd_reduce_kernel<IOT><<<grid, 256, 0, st>>>(pq, pk, pa, pb, static_cast<IOT *>(dq),
+                                                   static_cast<IOT *>(dk), dalpha, dbeta, n_tk,
+                                                   n_t, ntile);
   return cudaGetLastError();
-}
-
-template <typename IOT, int DK>
-cudaError_t launch_bwd_dv(int dv_, const void *q, const void *k, const void *v,
-                          const float *alpha, const float *beta, const float *s0,
-                          const void *d_o, const float *dsf, void *dq, void *dk, void *dv,
-                          float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
-                          int T, int T_total, int H, float scale, float *ck, float *buf,
-                          unsigned int *err, cudaStream_t st) {
-#define CKDA_BWD_DV(X)                                                                          \
-  if (dv_ == X)                                                                                 \
-    return launch_bwd_dims<IOT, DK, X>(q, k, v, alpha, beta, s0, d_o, dsf, dq, dk, dv, dalpha, \
-                                       dbeta, ds0, cu, N, T, T_total, H, scale, ck, buf, err, st);
-  CKDA_BWD_DV(16) CKDA_BWD_DV(32) CKDA_BWD_DV(64) CKDA_BWD_DV(128)
-#undef CKDA_BWD_DV
-  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
+// columns per CTA
+static int bwd_tile(int dv) { return dv < 32 ? dv : 32; }
+
 size_t bwd_workspace_bytes(int N, int T_total, int H, int dk, int dv) {
   const size_t slots = (size_t)T_total / CK + (size_t)N;
   const size_t state = (size_t)dk * dv * sizeof(float);
-  return slots * H * state + (size_t)N * H * CK * state;
+  const size_t ntile = (size_t)(dv / bwd_tile(dv)), th = (size_t)T_total * H;
+  return slots * H * state + (size_t)N * H * CK * state +
+         ntile * th * (3 * (size_t)dk + 1) * sizeof(float);
 }
 
 template <typename IOT>
@@ -358,13 +394,26 @@ cudaError_t launch_bwd(int dk_, int dv_, const void *q, const void *k, const voi
                        float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
                        int T, int T_total, int H, float scale, void *ws,
                        unsigned int *err, cudaStream_t st) {
+  // workspace: checkpoints | state buffers | partials dq, dk, dalpha [ntile][T_total H d_k],
+  // dbeta [ntile][T_total H]
   float *ck = static_cast<float *>(ws);
   const size_t slots = (size_t)T_total / CK + (size_t)N;
   float *buf = ck + slots * H * (size_t)dk_ * dv_;
-#define CKDA_BWD_DK(X)                                                                        \
-  if (dk_ == X)                                                                               \
-    return launch_bwd_dv<IOT, X>(dv_, q, k, v, alpha, beta, s0, d_o, dsf, dq, dk, dv, dalpha, \
-                                 dbeta, ds0, cu, N, T, T_total, H, scale, ck, buf, err, st);
+  const size_t ntile = (size_t)(dv_ / bwd_tile(dv_)), th = (size_t)T_total * H;
+  float *pq = buf + (size_t)N * H * CK * dk_ * dv_;
+  float *pk = pq + ntile * th * dk_;
+  float *pa = pk + ntile * th * dk_;
+  float *pb = pa + ntile * th * dk_;
+#define CKDA_BWD_DK(X)                                                                          \
+  if (dk_ == X) {                                                                               \
+    if (dv_ == 16)                                                                              \
+      return launch_bwd_dims<IOT, X, 16>(q, k, v, alpha, beta, s0, d_o, dsf, dq, dk, dv, dalpha, \
+                                         dbeta, ds0, cu, N, T, T_total, H, dv_, scale, ck, buf, \
+                                         pq, pk, pa, pb, err, st);                              \
+    return launch_bwd_dims<IOT, X, 32>(q, k, v, alpha, beta, s0, d_o, dsf, dq, dk, dv, dalpha,   \
+                                       dbeta, ds0, cu, N, T, T_total, H, dv_, scale, ck, buf,   \
+                                       pq, pk, pa, pb, err, st);                                \
+  }
   CKDA_BWD_DK(16) CKDA_BWD_DK(32) CKDA_BWD_DK(64) CKDA_BWD_DK(128)
 #undef CKDA_BWD_DK
   return cudaErrorInvalidValue;

@@ -243,10 +243,15 @@ def test_bwd_rejects(lib, kw, want):
 
 def test_bwd_workspace_query(lib):
     # checkpoints every 16 tokens: floor(T_total / 16) + N slots per head, plus
-    # a 16-state buffer per (sequence, head); fp32 d_k x d_v states
+    # a 16-state buffer per (sequence, head); fp32 d_k x d_v states; plus the
+    # fp32 partials of dq, dk, dalpha (d_k each) and dbeta per token-head for
+    # each 32-column tile (d_v = 64: 2 tiles)
     st = 32 * 64 * 4
-    assert lib.ckda_bwd_workspace_bytes(2, 40, 3, 32, 64, 0) == ((80 // 16 + 2) * 3 + 2 * 3 * 16) * st
-    assert lib.ckda_bwd_workspace_bytes(2, 40, 3, 32, 64, 1) == ((40 // 16 + 2) * 3 + 2 * 3 * 16) * st
+    part = lambda th: 2 * th * (3 * 32 + 1) * 4
+    assert lib.ckda_bwd_workspace_bytes(2, 40, 3, 32, 64, 0) == \
+        ((80 // 16 + 2) * 3 + 2 * 3 * 16) * st + part(80 * 3)
+    assert lib.ckda_bwd_workspace_bytes(2, 40, 3, 32, 64, 1) == \
+        ((40 // 16 + 2) * 3 + 2 * 3 * 16) * st + part(40 * 3)
     assert lib.ckda_bwd_workspace_bytes(1, 8, 1, 48, 16, 0) == 0
     assert lib.ckda_bwd_workspace_bytes(0, 8, 1, 16, 16, 0) == 0
 
