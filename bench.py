@@ -70,8 +70,8 @@ NCU_TRAFFIC = {
     "prefill": 4 * 375.9e6,
     # N=64 (2048 pairs): 214.8 MB, x4 for N=256
     "decode": 4 * 214.8e6,
-    # backward at T=512, H=32: 153.5 MB, x16 for T=8192
-    "backward": 16 * 153.5e6,
+    # backward (both kernels) at T=512, H=32: 356.3 MB, x16 for T=8192
+    "backward": 16 * 356.3e6,
 }
 
 
@@ -428,8 +428,9 @@ def main():
                              "frac": bbytes / (bms / 1e3) / 1e9 / pk["hbm_gbs"],
                              "traffic": NCU_TRAFFIC["backward"],
                              "algorithmic_bytes_per_launch": bbytes},
-                "kernel": "token-serial adjoint on CUDA cores, one CTA per (sequence, head)",
-                "gpu_launches": args.bwd_steps}
+                "kernel": "token-serial adjoint on CUDA cores, one CTA per (sequence, head, "
+                          "32-column tile), plus a tile reduction",
+                "gpu_launches": 2 * args.bwd_steps}
     del bws, bout
 
     # ---------------- decode step
