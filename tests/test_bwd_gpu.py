@@ -116,3 +116,17 @@ def test_bwd_is_deterministic(cuda_lib):
     b = run_gpu(inp, grads, 1.0)
     for name, x, y in zip(NAMES, a, b):
         assert torch.equal(x, y), name
+
+
+def test_bwd_equal_length_sequences_without_cu_seqlens(cuda_lib):
+    """N sequences of T tokens given by N and T alone (no cu_seqlens): the
+    checkpoint slots come from n T instead of the device offsets."""
+    w = custom("ckda_B1_H32_T8192_d128", dtype="f32", d_k=32, d_v=64, seed=813)
+    inp, grads = case(w, [40, 40], H=2)
+    d = to_dev(inp)
+    g = to_dev(grads)
+    got = ckda.bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], g["d_o"], d["initial_state"],
+                   g["d_final_state"], N=2, T=40, scale=0.7)
+    torch.cuda.synchronize()
+    assert ckda.ckda_last_error() == ckda.CKDA_OK
+    compare(got, run_ref(inp, grads, 0.7), bf16=False)
