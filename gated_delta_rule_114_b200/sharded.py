@@ -8,7 +8,9 @@ contiguous slice of the packed [T_total, H, d] inputs (no copy unless a slice
 would start off a 16-byte boundary), its
 cu_seqlens are the batch's entries rebased to 0, and the rank runs the same
 C-ABI forward on its slice. Gathering the outputs is optional and is the only
-collective (an all-gather of the per-rank o and final-state slices).
+collective (an all-gather of the per-rank o and final-state slices). The
+backward pass shards the same way: a rank's gradients depend only on its own
+sequences' rows (``bwd_sharded``).
 
 The host logic (the split, the slicing, the reassembly) is plain Python and
 runs under any torch.distributed backend; the forward itself is the CUDA
@@ -89,33 +91,89 @@ def fwd_chunked_sharded(q, k, v, alpha, beta, initial_state, cu_seqlens_host,
                                                      cu_seqlens_host, n0, n1)
     T, H, d_k = q.shape
     d_v = v.shape[2]
-    if n1 > n0:
+    if int(cu_local[-1]) > 0:
         o_loc, sf_loc = fwd(qs, ks, vs, as_, bs, s0, cu_local, chunk, scale)
-    else:
+    else:  # no token rows (no sequences, or only empty ones): nothing to launch
         o_loc = torch.empty((0, H, d_v), dtype=q.dtype, device=q.device)
-        sf_loc = torch.empty((0, H, d_k, d_v), dtype=torch.float32, device=q.device)
+        sf_loc = (s0.clone() if s0 is not None else
+                  torch.zeros((n1 - n0, H, d_k, d_v), dtype=torch.float32, device=q.device))
     if not gather:
         return o_loc, sf_loc, (n0, n1)
     return _gather(o_loc, sf_loc, cu_seqlens_host, world, group)
 
 
 def _gather(o_loc, sf_loc, cu_seqlens_host, world, group):
-    """All-gather the per-rank slices (padded to the largest) and reassemble."""
+    """All-gather the per-rank o and final-state slices and reassemble."""
+    return _gather_parts([(o_loc, "rows"), (sf_loc, "seqs")], cu_seqlens_host, world, group)
+
+
+def _gather_parts(parts, cu_seqlens_host, world, group):
+    """All-gather per-rank slices, each indexed by token rows ("rows") or by
+    sequences ("seqs"), padded to the largest rank's slice, and reassemble
+    them in rank order."""
     cu = [int(x) for x in cu_seqlens_host]
     plan = plan_shards(cu, world)
-    rows = [cu[n1] - cu[n0] for n0, n1 in plan]
-    seqs = [n1 - n0 for n0, n1 in plan]
-    mr, ms = max(rows), max(seqs)
+    sizes = {"rows": [cu[n1] - cu[n0] for n0, n1 in plan], "seqs": [n1 - n0 for n0, n1 in plan]}
 
     def padded(x, m):
         out = torch.zeros((m,) + tuple(x.shape[1:]), dtype=x.dtype, device=x.device)
         out[:x.shape[0]] = x
         return out
 
-    o_parts = [torch.empty_like(padded(o_loc, mr)) for _ in range(world)]
-    s_parts = [torch.empty_like(padded(sf_loc, ms)) for _ in range(world)]
-    dist.all_gather(o_parts, padded(o_loc, mr), group=group)
-    dist.all_gather(s_parts, padded(sf_loc, ms), group=group)
-    o = torch.cat([p[:r] for p, r in zip(o_parts, rows)])
-    sf = torch.cat([p[:s] for p, s in zip(s_parts, seqs)])
-    return o, sf
+    out = []
+    for x, kind in parts:
+        n = sizes[kind]
+        xs = [torch.empty_like(padded(x, max(n))) for _ in range(world)]
+        dist.all_gather(xs, padded(x, max(n)), group=group)
+        out.append(torch.cat([p[:c] for p, c in zip(xs, n)]))
+    return tuple(out)
+
+
+def _cuda_bwd(q, k, v, alpha, beta, s0, d_o, dsf, cu_local, scale):
+    return ckda.bwd(q, k, v, alpha, beta, d_o, s0, dsf, cu_seqlens=cu_local.to(q.device),
+                    cu_seqlens_host=cu_local, scale=scale)
+
+
+def bwd_sharded(q, k, v, alpha, beta, d_o, initial_state, d_final_state, cu_seqlens_host,
+                rank: int | None = None, world: int | None = None, *, scale: float = 1.0,
+                gather: bool = False, group=None, bwd: Callable | None = None):
+    """This rank's shard of a packed varlen backward pass.
+
+    Inputs are the whole batch (as for fwd_chunked_sharded, plus d_o
+    [T_total, H, d_v] and d_final_state [N, H, d_k, d_v] or None); each rank
+    reads only its own sequences' rows. Returns (dq, dk, dv, dalpha, dbeta,
+    d_initial_state) for this rank's token rows and sequences and (n0, n1);
+    with gather=True, the whole batch's gradients on every rank instead.
+    `bwd` replaces the CUDA backward (same arguments as the default) for
+    host-side tests."""
+    if rank is None:
+        rank = dist.get_rank(group) if dist.is_initialized() else 0
+    if world is None:
+        world = dist.get_world_size(group) if dist.is_initialized() else 1
+    bwd = bwd or _cuda_bwd
+    n0, n1 = plan_shards(cu_seqlens_host, world)[rank]
+    qs, ks, vs, as_, bs, s0, cu_local = shard_inputs(q, k, v, alpha, beta, initial_state,
+                                                     cu_seqlens_host, n0, n1)
+    cu = [int(x) for x in cu_seqlens_host]
+    t0, t1 = cu[n0], cu[n1]
+
+    def view(x):  # 16-byte aligned rows for the C ABI; copy a slice only if needed
+        return x if x.data_ptr() % 16 == 0 else x.clone()
+
+    dos = view(d_o[t0:t1])
+    dsf = view(d_final_state[n0:n1]) if d_final_state is not None else None
+    T, H, d_k = q.shape
+    d_v = v.shape[2]
+    if t1 > t0:
+        grads = bwd(qs, ks, vs, as_, bs, s0, dos, dsf, cu_local, scale)
+    else:  # no token rows: the initial-state gradient is the final-state one
+        rows = lambda d, dt: torch.empty((0, H, d), dtype=dt, device=q.device)
+        ds0 = (dsf.clone() if dsf is not None else
+               torch.zeros((n1 - n0, H, d_k, d_v), dtype=torch.float32, device=q.device))
+        grads = (rows(d_k, q.dtype), rows(d_k, q.dtype), rows(d_v, q.dtype),
+                 rows(d_k, torch.float32), torch.empty((0, H), dtype=torch.float32, device=q.device),
+                 ds0)
+    if not gather:
+        return tuple(grads) + ((n0, n1),)
+    kinds = ["rows"] * 5 + ["seqs"]
+    return _gather_parts(list(zip(grads, kinds)), cu_seqlens_host, world, group)
