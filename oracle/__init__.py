@@ -12,7 +12,8 @@ with the readout of §3 eq. (14); ranges from "Complex KDA", abstract). This
 module only compiles it with gcc (no fast-math) and marshals numpy arrays.
 
 Every function here is pinned by ``tests/test_oracle_pins.py``,
-``tests/test_oracle_prologue.py`` and ``tests/test_oracle_bwd.py`` against
+``tests/test_oracle_prologue.py``, ``tests/test_oracle_bwd.py`` and
+``tests/test_oracle_complex.py`` against
 the lesson's worked traces, closed forms, the dense affine composition
 (§2.2 eq. (10)) and, for the backward pass, central finite differences of
 the forward; none is "parity unpinned".
@@ -281,3 +282,51 @@ def bwd(q, k, v, alpha, beta, d_o, initial_state=None, d_final_state=None,
                 out[i][a:b, h] = r[i]
             out[5][n, h] = r[5]
     return tuple(out)
+
+
+def fwd_complex(q, k, v, alpha, theta, beta, initial_state=None, cu_seqlens=None,
+                scale: float = 1.0):
+    """The complex-phase gate of "Semidirect Fourier Delta Attention" §3,
+    eqs. (13)-(14), token by token in complex128:
+
+        S_t = (I - beta_t k_t k_t^*) Lambda_t S_{t-1} + beta_t k_t v_t^*,
+        Lambda_t = diag(alpha_t * exp(i theta_t)),   o_t = scale S_t^* q_t
+
+    (^* the conjugate transpose). q, k: [total_T, H, d_k] complex; v:
+    [total_T, H, d_v] complex; alpha, theta: [total_T, H, d_k] real; beta:
+    [total_T, H] real; states [N, H, d_k, d_v] complex. With theta = 0 and
+    real inputs this is ``fwd``. Returns (o, final_state) in complex128.
+    """
+    def c128(x):
+        if x is None:
+            return None
+        if hasattr(x, "detach"):
+            x = x.detach().to("cpu").numpy()
+        return np.ascontiguousarray(x, dtype=np.complex128)
+
+    q, k, v = c128(q), c128(k), c128(v)
+    alpha, theta, beta = _f64(alpha), _f64(theta), _f64(beta)
+    s0 = c128(initial_state)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.asarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    o = np.zeros((T, H, dv), dtype=np.complex128)
+    sf = np.zeros((N, H, dk, dv), dtype=np.complex128)
+    for n in range(N):
+        for h in range(H):
+            S = s0[n, h].copy() if s0 is not None else np.zeros((dk, dv), dtype=np.complex128)
+            for t in range(int(cu[n]), int(cu[n + 1])):
+                lam = alpha[t, h] * np.exp(1j * theta[t, h])
+                S = lam[:, None] * S                                  # Lambda_t S_{t-1}
+                kt = k[t, h]
+                S = S - beta[t, h] * np.outer(kt, kt.conj() @ S)       # (I - beta k k^*) .
+                S = S + beta[t, h] * np.outer(kt, v[t, h].conj())      # + beta k v^*
+                o[t, h] = scale * (S.conj().T @ q[t, h])               # S^* q
+            sf[n, h] = S
+    return o, sf
