@@ -32,6 +32,7 @@ sys.path.insert(0, ROOT)
 
 from gated_delta_rule_114_b200 import ckda  # noqa: E402
 from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_bwd_grads,  # noqa: E402
+                                              make_complex_inputs,
                                               make_decode_state,
                                               make_decode_tokens,
                                               make_fwd_inputs,
@@ -124,6 +125,13 @@ def bwd_bytes(inp) -> int:
     per_th = ((2 * dk + dv) * es + dk * 4 + 4 + dv * es) + ((2 * dk + dv) * es + dk * 4 + 4)
     N = inp["cu_seqlens"].numel() - 1
     return T * H * per_th + 3 * N * H * dk * dv * 4
+
+
+def complex_bytes(T, H, N, dk, dv) -> int:
+    """Algorithmic HBM bytes of one complex-phase-gate forward: q, k, v, o
+    complex64, alpha, theta, beta fp32 per token-head; initial and final
+    complex64 states per (sequence, head)."""
+    return T * H * ((2 * dk + 2 * dv) * 8 + 2 * dk * 4 + 4) + 2 * N * H * dk * dv * 8
 
 
 def decode_bytes(N, H, dk, dv, dt) -> int:
@@ -292,6 +300,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--bwd-steps", type=int, default=5)
+    ap.add_argument("--complex-steps", type=int, default=5)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -433,6 +442,31 @@ def main():
                 "gpu_launches": 2 * args.bwd_steps}
     del bws, bout
 
+    # ---------------- the complex-phase gate on the same shape (complex64)
+    cin = {key: val.cuda() for key, val in
+           make_complex_inputs(w, inp_cpu["cu_seqlens"], H).items()}
+    co = torch.empty((T_total, H, dv), dtype=torch.complex64, device="cuda")
+    csf = torch.empty((N, H, dk, dv), dtype=torch.complex64, device="cuda")
+
+    def complex_step():
+        ckda.ckda_fwd_complex(cin["q"], cin["k"], cin["v"], cin["alpha"], cin["theta"],
+                              cin["beta"], cin["initial_state"], csf, co, cin["cu_seqlens"],
+                              None, stream=stream)
+
+    cms = time_loop(complex_step, args.complex_steps, 3, stream, barrier)
+    if ckda.ckda_last_error() != ckda.CKDA_OK:
+        raise RuntimeError("kernel reported an error")
+    cbytes = complex_bytes(T_total, H, N, dk, dv)
+    complex_gate = {"ms_per_step": cms, "tokens_per_s": T_total * world / (cms / 1e3),
+                    "steps": args.complex_steps, "warmup": 3,
+                    "roofline": {"bound": "hbm", "achieved": cbytes / (cms / 1e3) / 1e9,
+                                 "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                 "frac": cbytes / (cms / 1e3) / 1e9 / pk["hbm_gbs"],
+                                 "traffic": None, "algorithmic_bytes_per_launch": cbytes},
+                    "kernel": "token-serial complex recurrence on CUDA cores, fp32",
+                    "gpu_launches": args.complex_steps}
+    del cin, co, csf
+
     # ---------------- decode step
     wd = WORKLOADS[DECODE]
     state = make_decode_state(wd).cuda()
@@ -483,7 +517,7 @@ def main():
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         # each forward call launches the slot-table, prep and scan kernels
         "gpu_launches": 3 * args.steps, "clocks": clk.summary(), "decode": decode,
-        "prefill_fused_prologue": gated, "backward": backward,
+        "prefill_fused_prologue": gated, "backward": backward, "complex_gate": complex_gate,
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -83,6 +83,8 @@ def load(path: str | None = None):
     lib.ckda_status_string.argtypes = [ctypes.c_int]
     lib.ckda_bwd.restype = ctypes.c_int
     lib.ckda_bwd.argtypes = [vp] * 16 + [i32] * 5 + [f32, ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.ckda_fwd_complex.restype = ctypes.c_int
+    lib.ckda_fwd_complex.argtypes = [vp] * 11 + [i32] * 5 + [f32, vp]
     lib.ckda_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.ckda_bwd_workspace_bytes.argtypes = [i32] * 6
     lib.ckda_last_error.restype = ctypes.c_int
@@ -392,6 +394,60 @@ def fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, gates: GateParams,
     ckda_fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, initial_state, sf, o, gates,
                            cu_seqlens, cu_seqlens_host, N, T, chunk, scale, stream,
                            workspace)
+    return o, sf
+
+
+def ckda_fwd_complex(q, k, v, alpha, theta, beta, initial_state, final_state, o,
+                     cu_seqlens=None, cu_seqlens_host=None, N=None, T=None,
+                     scale: float = 1.0, stream=None):
+    """Marshal tensors into ckda_fwd_complex (see include/ckda.h): q, k
+    [T_total, H, d_k] and v, o [T_total, H, d_v] complex64; alpha, theta
+    [T_total, H, d_k] and beta [T_total, H] fp32; states [N, H, d_k, d_v]
+    complex64 or None."""
+    lib = load()
+    for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, nme, torch.complex64, 3)
+    for t, nme in ((alpha, "alpha"), (theta, "theta")):
+        _need(t, nme, torch.float32, 3)
+    _need(beta, "beta", torch.float32, 2)
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+        N = cu_seqlens.numel() - 1
+        T = T_total
+    elif N is None or T is None:
+        raise ValueError("give cu_seqlens, or N and T")
+    for t, nme in ((initial_state, "initial_state"), (final_state, "final_state")):
+        if t is not None:
+            _need(t, nme, torch.complex64, 4)
+    host_ptr = None
+    if cu_seqlens_host is not None:
+        if cu_seqlens_host.is_cuda or cu_seqlens_host.dtype != torch.int32 \
+                or not cu_seqlens_host.is_contiguous():
+            raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
+        host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    st = lib.ckda_fwd_complex(_p(q), _p(k), _p(v), _p(alpha), _p(theta), _p(beta),
+                              _p(initial_state), _p(final_state), _p(o), _p(cu_seqlens), host_ptr,
+                              int(N), int(T), int(H), int(d_k), int(d_v), float(scale),
+                              _stream(stream))
+    _check(st, "ckda_fwd_complex")
+
+
+def fwd_complex(q, k, v, alpha, theta, beta, initial_state=None, cu_seqlens=None,
+                cu_seqlens_host=None, N=None, T=None, scale: float = 1.0, stream=None):
+    """The complex-phase gate: allocate o and the final state (complex64) with
+    torch, then call ckda_fwd_complex. Returns (o, final_state)."""
+    T_total, H, d_k = q.shape
+    d_v = v.shape[2]
+    if cu_seqlens is not None:
+        N = cu_seqlens.numel() - 1
+    elif N is None:
+        N, T = 1, T_total
+    o = torch.empty((T_total, H, d_v), dtype=torch.complex64, device=q.device)
+    sf = torch.empty((N, H, d_k, d_v), dtype=torch.complex64, device=q.device)
+    ckda_fwd_complex(q, k, v, alpha, theta, beta, initial_state, sf, o, cu_seqlens,
+                     cu_seqlens_host, N, T, scale, stream)
     return o, sf
 
 

@@ -23,6 +23,11 @@ cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
                             int T_total, int H, float scale, GateArgs g,
                             unsigned int *err, cudaStream_t st);
 size_t bwd_workspace_bytes(int N, int T_total, int H, int dk, int dv);
+cudaError_t launch_fwd_complex(int dk, int dv, const void *q, const void *k, const void *v,
+                               const float *alpha, const float *theta, const float *beta,
+                               const void *s0, void *sf, void *o, const int32_t *cu, int N,
+                               int T, int T_total, int H, float scale, unsigned int *err,
+                               cudaStream_t st);
 template <typename IOT>
 cudaError_t launch_bwd(int dk, int dv, const void *q, const void *k, const void *v,
                        const float *alpha, const float *beta, const float *s0,
@@ -139,6 +144,52 @@ ckda_status ckda_last_error(cudaStream_t stream) {
       cudaMemcpyToSymbol(g_ckda_error_word, &zero, sizeof(zero)) != cudaSuccess)
     return CKDA_ERR_CUDA;
   return w ? CKDA_ERR_DEVICE : CKDA_OK;
+}
+
+ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const float *alpha,
+                             const float *theta, const float *beta, const void *initial_state,
+                             void *final_state, void *o, const int32_t *cu_seqlens,
+                             const int32_t *cu_seqlens_host, int32_t N, int32_t T, int32_t H,
+                             int32_t d_k, int32_t d_v, float scale, cudaStream_t stream) {
+  if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!q || !k || !v || !alpha || !theta || !beta || !o) return CKDA_ERR_ARG;
+  const void *ptrs[] = {q, k, v, alpha, theta, beta, initial_state, final_state, o, cu_seqlens};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return CKDA_ERR_ARG;
+  int64_t T_total;
+  if (cu_seqlens == nullptr) {
+    if (cu_seqlens_host) return CKDA_ERR_ARG;
+    T_total = (int64_t)N * T;
+  } else {
+    T_total = T;
+    if (cu_seqlens_host) {
+      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return CKDA_ERR_ARG;
+      for (int32_t n = 0; n < N; ++n)
+        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return CKDA_ERR_ARG;
+    }
+  }
+  if (T_total > INT32_MAX) return CKDA_ERR_ARG;
+  // complex64 = 8 bytes per element; no output may overlap an input or the other output
+  const size_t th = (size_t)T_total * H;
+  const size_t kb = th * d_k * 8, vb = th * d_v * 8, rb = th * d_k * sizeof(float);
+  const size_t sb = (size_t)N * H * d_k * d_v * 8;
+  struct R { const void *p; size_t n; };
+  const R ins[] = {{q, kb}, {k, kb}, {v, vb}, {alpha, rb}, {theta, rb}, {beta, th * sizeof(float)},
+                   {initial_state, sb}};
+  for (const R &x : ins)
+    if (overlaps(o, vb, x.p, x.n)) return CKDA_ERR_ARG;
+  for (size_t i = 0; i + 1 < sizeof(ins) / sizeof(ins[0]); ++i)  // final state: any input but s0
+    if (overlaps(final_state, sb, ins[i].p, ins[i].n)) return CKDA_ERR_ARG;
+  if (overlaps(final_state, sb, o, vb)) return CKDA_ERR_ARG;
+  if (final_state && initial_state && final_state != initial_state &&
+      overlaps(final_state, sb, initial_state, sb))
+    return CKDA_ERR_ARG;
+  if (N == 0) return CKDA_OK;
+  const cudaError_t e = ckda::launch_fwd_complex(d_k, d_v, q, k, v, alpha, theta, beta,
+                                                 initial_state, final_state, o, cu_seqlens, N, T,
+                                                 (int)T_total, H, scale, error_word_ptr(), stream);
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
 size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,

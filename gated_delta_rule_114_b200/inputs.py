@@ -248,3 +248,35 @@ def make_bwd_grads(w: Workload, T_total: int, H: int, N: int, seed_offset: int =
     d_o = torch.randn(T_total, H, w.d_v, generator=g, dtype=torch.float32)
     dsf = torch.randn(N, H, w.d_k, w.d_v, generator=g, dtype=torch.float32)
     return dict(d_o=d_o.to(TORCH_DTYPE[w.dtype]), d_final_state=dsf)
+
+
+def make_complex_inputs(w: Workload, cu_seqlens: torch.Tensor, H: int, theta_max: float = 1.5,
+                        ranges: str = "sfda", seed_offset: int = 0) -> dict:
+    """Seeded inputs for the complex-phase gate: q, k (unit rows), v complex64
+    with N(0, 1) real and imaginary parts; theta = theta_max tanh(N(0, 1));
+    ranges "sfda": alpha = sigmoid(N(0, 1)) in (0, 1), beta = sigmoid(N(0, 1));
+    "ckda": alpha = tanh(N(0, 2)) in (-1, 1), beta = 2 sigmoid(N(0, 1.5));
+    initial state N(0, 0.1) complex64."""
+    g = _gen(w.seed + 9090 + seed_offset)
+    cu = cu_seqlens.to(torch.int32)
+    N, T = cu.numel() - 1, int(cu[-1])
+
+    def cn(*shape):
+        re = torch.randn(*shape, generator=g, dtype=torch.float32)
+        im = torch.randn(*shape, generator=g, dtype=torch.float32)
+        return torch.complex(re, im)
+
+    q = cn(T, H, w.d_k)
+    k = cn(T, H, w.d_k)
+    k = k / torch.linalg.vector_norm(k, dim=-1, keepdim=True)
+    v = cn(T, H, w.d_v)
+    theta = theta_max * torch.tanh(torch.randn(T, H, w.d_k, generator=g))
+    if ranges == "ckda":
+        alpha = torch.tanh(2.0 * torch.randn(T, H, w.d_k, generator=g))
+        beta = 2.0 * torch.sigmoid(1.5 * torch.randn(T, H, generator=g))
+    else:
+        alpha = torch.sigmoid(torch.randn(T, H, w.d_k, generator=g))
+        beta = torch.sigmoid(torch.randn(T, H, generator=g))
+    s0 = 0.1 * cn(N, H, w.d_k, w.d_v)
+    return dict(q=q, k=k, v=v, alpha=alpha.contiguous(), theta=theta.contiguous(),
+                beta=beta.contiguous(), initial_state=s0, cu_seqlens=cu)

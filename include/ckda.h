@@ -270,6 +270,31 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
                      cudaStream_t stream);
 
 /*
+ * ckda_fwd_complex: the complex-phase gate of "Semidirect Fourier Delta
+ * Attention" §3, eqs. (13)-(14), with complex q, k, v and state:
+ *   S_t = (I - beta_t k_t k_t^*) Lambda_t S_{t-1} + beta_t k_t v_t^*,
+ *   Lambda_t = diag(alpha_t exp(i theta_t)),   o_t = scale S_t^* q_t
+ * (^* the conjugate transpose; the page's real implementation of the gate is
+ * a 2x2 rotation-decay block on each (real, imaginary) pair).
+ *   q, k        [total_T, H, d_k] complex64 (interleaved real, imaginary fp32).
+ *   v, o        [total_T, H, d_v] complex64 (o written).
+ *   alpha, theta [total_T, H, d_k] fp32: decay and phase per channel.
+ *   beta        [total_T, H] fp32.
+ *   initial_state, final_state [N, H, d_k, d_v] complex64, or NULL (zero / not
+ *               written); final_state may equal initial_state (in place).
+ *   cu_seqlens, cu_seqlens_host, N, T, H, d_k, d_v, scale: as ckda_fwd_chunked.
+ * Every pointer 16-byte aligned; o must not overlap an input; d_k, d_v in {16,
+ * 32, 64, 128}. Token-serial on CUDA cores (one CTA per sequence, head and
+ * 32-column tile), fp32 arithmetic, deterministic; no workspace. Asynchronous
+ * on `stream`; device-side errors through ckda_last_error().
+ */
+ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const float *alpha,
+                             const float *theta, const float *beta, const void *initial_state,
+                             void *final_state, void *o, const int32_t *cu_seqlens,
+                             const int32_t *cu_seqlens_host, int32_t N, int32_t T, int32_t H,
+                             int32_t d_k, int32_t d_v, float scale, cudaStream_t stream);
+
+/*
  * ckda_bwd_workspace_bytes: scratch ckda_bwd needs (T as in ckda_bwd; varlen
  * nonzero when cu_seqlens is given, so that T is total_T). 0 for unsupported
  * or invalid sizes.
