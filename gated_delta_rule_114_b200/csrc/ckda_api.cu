@@ -86,6 +86,26 @@ size_t esize(ckda_dtype dt) { return dt == CKDA_F32 ? 4 : 2; }
 
 bool finite(float x) { return x == x && x - x == 0.f; }
 
+// Token rows of the packed [T_total, H, ...] tensors: N*T for fixed-length
+// sequences, T for varlen (cu_seqlens given). A host copy of the offsets, when
+// given, must start at 0, end at T and not decrease. False on any violation
+// or a row count above INT32_MAX.
+bool token_rows(const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, int32_t N,
+                int32_t T, int64_t &T_total) {
+  if (cu_seqlens == nullptr) {
+    if (cu_seqlens_host) return false;
+    T_total = (int64_t)N * T;
+  } else {
+    T_total = T;
+    if (cu_seqlens_host) {
+      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return false;
+      for (int32_t n = 0; n < N; ++n)
+        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return false;
+    }
+  }
+  return T_total <= INT32_MAX;
+}
+
 // ckda_gate_params -> kernel arguments; false if outside the documented ranges
 bool gate_args(const ckda_gate_params &gp, ckda::GateArgs &g) {
   if (!finite(gp.alpha_min) || !finite(gp.alpha_max) || !finite(gp.beta_max) ||
@@ -158,18 +178,7 @@ ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const 
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return CKDA_ERR_ARG;
   int64_t T_total;
-  if (cu_seqlens == nullptr) {
-    if (cu_seqlens_host) return CKDA_ERR_ARG;
-    T_total = (int64_t)N * T;
-  } else {
-    T_total = T;
-    if (cu_seqlens_host) {
-      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return CKDA_ERR_ARG;
-      for (int32_t n = 0; n < N; ++n)
-        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return CKDA_ERR_ARG;
-    }
-  }
-  if (T_total > INT32_MAX) return CKDA_ERR_ARG;
+  if (!token_rows(cu_seqlens, cu_seqlens_host, N, T, T_total)) return CKDA_ERR_ARG;
   // complex64 = 8 bytes per element; no output may overlap an input or the other output
   const size_t th = (size_t)T_total * H;
   const size_t kb = th * d_k * 8, vb = th * d_v * 8, rb = th * d_k * sizeof(float);
@@ -218,18 +227,7 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return CKDA_ERR_ARG;
   int64_t T_total;
-  if (cu_seqlens == nullptr) {
-    if (cu_seqlens_host) return CKDA_ERR_ARG;
-    T_total = (int64_t)N * T;
-  } else {
-    T_total = T;
-    if (cu_seqlens_host) {
-      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return CKDA_ERR_ARG;
-      for (int32_t n = 0; n < N; ++n)
-        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return CKDA_ERR_ARG;
-    }
-  }
-  if (T_total > INT32_MAX) return CKDA_ERR_ARG;
+  if (!token_rows(cu_seqlens, cu_seqlens_host, N, T, T_total)) return CKDA_ERR_ARG;
   // no output may overlap an input, another output or the workspace
   const size_t es = esize(dt), th = (size_t)T_total * H;
   const size_t kb = th * d_k * es, vb = th * d_v * es, ab = th * d_k * sizeof(float);
@@ -349,18 +347,7 @@ ckda_status fwd_impl(const void *q, const void *k, const void *v,
     if (p && !aligned16(p)) return CKDA_ERR_ARG;
 
   int64_t T_total;
-  if (cu_seqlens == nullptr) {
-    if (cu_seqlens_host) return CKDA_ERR_ARG;
-    T_total = (int64_t)N * T;
-  } else {
-    T_total = T;
-    if (cu_seqlens_host) {
-      if (cu_seqlens_host[0] != 0 || cu_seqlens_host[N] != T) return CKDA_ERR_ARG;
-      for (int32_t n = 0; n < N; ++n)
-        if (cu_seqlens_host[n + 1] < cu_seqlens_host[n]) return CKDA_ERR_ARG;
-    }
-  }
-  if (T_total > INT32_MAX) return CKDA_ERR_ARG;
+  if (!token_rows(cu_seqlens, cu_seqlens_host, N, T, T_total)) return CKDA_ERR_ARG;
 
   // the output must not overlap any input or state
   const size_t es = esize(dt);
