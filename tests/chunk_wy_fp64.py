@@ -26,9 +26,10 @@ import numpy as np
 def pair_gates(alpha: np.ndarray) -> np.ndarray:
     """G[i, j, :] = prod_{s=j+1..i} alpha[s] for j <= i (0 above the diagonal)."""
     L, d = alpha.shape
-    G = np.zeros((L, L, d))
+    dt = np.result_type(alpha, 1.0)            # real gates, or complex ones
+    G = np.zeros((L, L, d), dtype=dt)
     for j in range(L):
-        g = np.ones(d)
+        g = np.ones(d, dtype=dt)
         G[j, j] = g
         for i in range(j + 1, L):
             g = g * alpha[i]
@@ -74,3 +75,33 @@ def chunked_fwd(q, k, v, alpha, beta, S0, C, scale=1.0):
         o[s:e], S = chunk_step(S, q[s:e], k[s:e], v[s:e], alpha[s:e],
                                beta[s:e], scale)
     return o, S
+
+
+def chunk_step_complex(S, q, k, v, lam, beta, scale=1.0):
+    """One chunk of the complex-phase gate ("Semidirect Fourier Delta
+    Attention" §3, eqs. (13)-(14)): S' = Lambda S with complex diagonal
+    gates lam = alpha exp(i theta), S_i = S'_i + k_i u_i^T with
+    u_i^T = beta_i (v_i^* - k_i^* S'_i), and o_i = scale S_i^* q_i. The same
+    unrolling as the real case, with conjugates where k^* and q^* stand:
+        (I + A) U = diag(beta) (conj(V) - Khat S),  A_ij = beta_i k_i^* G_ij k_j (j < i)
+        conj(O)   = scale (Qhat S + M U),           M_ij = q_i^* G_ij k_j (j <= i)
+        S_L       = diag(gamma_L) S + Kbar^T U,
+    with Khat_i = gamma_i conj(k_i), Qhat_i = gamma_i conj(q_i),
+    Kbar_j = sigma_j k_j. Returns (O, S_L)."""
+    L = q.shape[0]
+    G = pair_gates(lam)
+    A = np.zeros((L, L), dtype=complex)
+    M = np.zeros((L, L), dtype=complex)
+    for i in range(L):
+        for j in range(i + 1):
+            gk = G[i, j] * k[j]
+            M[i, j] = q[i].conj() @ gk
+            if j < i:
+                A[i, j] = beta[i] * (k[i].conj() @ gk)
+    gamma = np.cumprod(lam, axis=0)
+    sigma = np.stack([G[L - 1, j] for j in range(L)])
+    T = np.linalg.inv(np.eye(L) + A)
+    U = T @ (beta[:, None] * (v.conj() - (gamma * k.conj()) @ S))
+    O = scale * ((gamma * q.conj()) @ S + M @ U).conj()
+    S_new = gamma[L - 1][:, None] * S + (sigma * k).T @ U
+    return O, S_new

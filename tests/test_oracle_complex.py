@@ -12,7 +12,9 @@ than itself:
     unitary, so ||S||_F is preserved exactly (this needs the conjugate in
     k k^*: with k k^T the beta = 2 step is not unitary);
   * with v = 0, alpha, beta in [0, 1] and ||k|| <= 1 the state norm never grows;
-  * the dense affine composition of the per-token maps S -> A_t S + B_t.
+  * the dense affine composition of the per-token maps S -> A_t S + B_t;
+  * the chunkwise (WY / UT) form in complex arithmetic (``chunk_wy_fp64``),
+    for several chunk lengths.
 Two planted mistakes (the projector without the conjugate, the readout without
 it) are each caught.
 """
@@ -22,6 +24,7 @@ import numpy as np
 import pytest
 
 import oracle
+from chunk_wy_fp64 import chunk_step_complex
 
 
 def cplx(rng, *shape):
@@ -130,6 +133,21 @@ def test_dense_affine_composition():
         st = Acc @ s0[0, 0] + Bcc
         np.testing.assert_allclose(o[t, 0], 0.9 * st.conj().T @ q[t, 0], rtol=0, atol=1e-12)
     np.testing.assert_allclose(sf[0, 0], Acc @ s0[0, 0] + Bcc, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("C", [1, 4, 16])
+def test_chunk_form_matches(C):
+    q, k, v, alpha, theta, beta, s0 = case(13, T=37, H=1, dk=5, dv=3)
+    alpha = np.where(np.random.default_rng(4).uniform(size=alpha.shape) < 0.1, 0.0, alpha)
+    beta = 2 * beta
+    o, sf = oracle.fwd_complex(q, k, v, alpha, theta, beta, s0, scale=0.7)
+    lam = alpha[:, 0] * np.exp(1j * theta[:, 0])
+    S = s0[0, 0]
+    for s in range(0, 37, C):
+        e = min(37, s + C)
+        oc, S = chunk_step_complex(S, q[s:e, 0], k[s:e, 0], v[s:e, 0], lam[s:e], beta[s:e, 0], 0.7)
+        np.testing.assert_allclose(oc, o[s:e, 0], rtol=0, atol=1e-11)
+    np.testing.assert_allclose(S, sf[0, 0], rtol=0, atol=1e-11)
 
 
 MUTATIONS = [
