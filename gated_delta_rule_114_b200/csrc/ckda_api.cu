@@ -70,6 +70,11 @@ unsigned int *error_word_ptr() {
 
 bool supported_dim(int32_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+// The sequence-parallel kernels put the sequence index, and the forward scan
+// also the head, on grid.y or grid.z, which hold at most 65535 blocks.
+constexpr int32_t kMaxGridYZ = 65535;
+bool grid_fits(int32_t N, int32_t H) { return N <= kMaxGridYZ && H <= kMaxGridYZ; }
+
 bool aligned16(const void *p) {
   return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
@@ -173,6 +178,7 @@ ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const 
                              int32_t d_k, int32_t d_v, float scale, cudaStream_t stream) {
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!grid_fits(N, H)) return CKDA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !alpha || !theta || !beta || !o) return CKDA_ERR_ARG;
   const void *ptrs[] = {q, k, v, alpha, theta, beta, initial_state, final_state, o, cu_seqlens};
   for (const void *p : ptrs)
@@ -220,6 +226,7 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
   if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!grid_fits(N, H)) return CKDA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !alpha || !beta || !d_o || !dq || !dk || !dv || !dalpha || !dbeta)
     return CKDA_ERR_ARG;
   const void *ptrs[] = {q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk,
@@ -340,6 +347,7 @@ ckda_status fwd_impl(const void *q, const void *k, const void *v,
   if (chunk == 0) chunk = 64;
   if (chunk != 16 && chunk != 32 && chunk != 64) return CKDA_ERR_UNSUPPORTED;
   if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
+  if (!grid_fits(N, H)) return CKDA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !alpha || !beta || !o) return CKDA_ERR_ARG;
   const void *ptrs[] = {q, k, v, alpha, beta, o, initial_state, final_state,
                         cu_seqlens, workspace};

@@ -25,7 +25,9 @@
  *      states   [N, H, d_k, d_v] fp32 (d_v contiguous)
  *    q, k, v and o share one element type (ckda_dtype); alpha, beta and the
  *    states are always fp32. Every pointer must be 16-byte aligned.
- *  - Supported sizes: d_k, d_v in {16, 32, 64, 128}; H >= 1.
+ *  - Supported sizes: d_k, d_v in {16, 32, 64, 128}; H >= 1. The chunked
+ *    forward, the backward and the complex-phase forward take N and H up to
+ *    65535 (CKDA_ERR_UNSUPPORTED beyond).
  *  - Calls are asynchronous on `stream` (0 = legacy default stream). Argument
  *    errors are detected on the host and returned before anything is
  *    launched. Launch failures return CKDA_ERR_CUDA. Errors found by a kernel
@@ -48,7 +50,7 @@ extern "C" {
 typedef enum {
   CKDA_OK = 0,
   CKDA_ERR_ARG = 1,          /* null/misaligned pointer, bad size, bad cu_seqlens */
-  CKDA_ERR_UNSUPPORTED = 2,  /* d_k, d_v, chunk or dtype outside the supported set */
+  CKDA_ERR_UNSUPPORTED = 2,  /* d_k, d_v, chunk, dtype or N, H outside the supported set */
   CKDA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
   CKDA_ERR_DEVICE = 4        /* a kernel flagged an error (see ckda_last_error) */
 } ckda_status;

@@ -84,6 +84,9 @@ def dec(lib, q=P, k=P2, v=P3, a=P4, b=P5, s=P6, o=ctypes.c_void_p(0x70000),
     (dict(dv=256), ckda.CKDA_ERR_UNSUPPORTED),
     (dict(chunk=24), ckda.CKDA_ERR_UNSUPPORTED),
     (dict(dt=7), ckda.CKDA_ERR_UNSUPPORTED),
+    # sequences or heads beyond a grid dimension
+    (dict(N=65536), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(H=65536), ckda.CKDA_ERR_UNSUPPORTED),
     # output aliasing an input
     (dict(o=P), ckda.CKDA_ERR_ARG),
     # host cu_seqlens without a device copy
@@ -230,6 +233,7 @@ def bwd(lib, q=P, k=P2, v=P3, a=P4, b=P5, do=P6, dq=ctypes.c_void_p(0x70000),
     (dict(dkd=48), ckda.CKDA_ERR_UNSUPPORTED),
     (dict(dvd=256), ckda.CKDA_ERR_UNSUPPORTED),
     (dict(dt=7), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(N=65536), ckda.CKDA_ERR_UNSUPPORTED),
     # a gradient aliasing an input, two gradients aliasing each other
     (dict(dq=P), ckda.CKDA_ERR_ARG),
     (dict(dk=ctypes.c_void_p(0x70000)), ckda.CKDA_ERR_ARG),
@@ -260,3 +264,31 @@ def test_bwd_zero_sequences_is_a_noop(lib):
     """N = 0: validated, nothing launched, CKDA_OK (the fake pointers are
     never dereferenced)."""
     assert bwd(lib, N=0, T=0, ws=NULL, wsb=0) == ckda.CKDA_OK
+
+
+def cplx(lib, q=P, k=P2, v=P3, a=P4, th=P5, b=P6, s0=NULL, sf=NULL,
+         o=ctypes.c_void_p(0x70000), cu=NULL, cuh=NULL, N=1, T=8, H=1, dk=16, dv=16):
+    return lib.ckda_fwd_complex(q, k, v, a, th, b, s0, sf, o, cu, cuh, N, T, H, dk, dv, 1.0,
+                                None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=NULL), ckda.CKDA_ERR_ARG),
+    (dict(th=NULL), ckda.CKDA_ERR_ARG),
+    (dict(v=ODD), ckda.CKDA_ERR_ARG),
+    (dict(H=0), ckda.CKDA_ERR_ARG),
+    (dict(T=-1), ckda.CKDA_ERR_ARG),
+    (dict(dk=24), ckda.CKDA_ERR_UNSUPPORTED),
+    (dict(N=65536), ckda.CKDA_ERR_UNSUPPORTED),
+    # output over an input; final state over the output
+    (dict(o=P3), ckda.CKDA_ERR_ARG),
+    (dict(sf=ctypes.c_void_p(0x70000)), ckda.CKDA_ERR_ARG),
+    # host cu_seqlens without a device copy
+    (dict(cuh=ctypes.cast((ctypes.c_int32 * 2)(0, 8), ctypes.c_void_p)), ckda.CKDA_ERR_ARG),
+])
+def test_complex_rejects(lib, kw, want):
+    assert cplx(lib, **kw) == want
+
+
+def test_complex_zero_sequences_is_a_noop(lib):
+    assert cplx(lib, N=0, T=0) == ckda.CKDA_OK
