@@ -257,6 +257,15 @@ __global__ void ckda_bwd_reduce_kernel(const float *__restrict__ pq, const float
   }
 }
 
+}  // namespace
+
+template <typename IOT>
+cudaError_t launch_bwd_reduce(const float *pq, const float *pk, const float *pa,
+                              const float *pb, void *dq, void *dk, float *dalpha, float *dbeta,
+                              size_t n_tk, size_t n_t, int ntile, cudaStream_t st);
+
+namespace {
+
 template <typename IOT, int DK, int DVT>
 cudaError_t launch_bwd_dims(const void *q, const void *k, const void *v, const float *alpha,
                             const float *beta, const float *s0, const void *d_o,
@@ -277,7 +286,16 @@ cudaError_t launch_bwd_dims(const void *q, const void *k, const void *v, const f
       pb, ds0, cu, T, T_total, H, DVF, scale, ck, buf, err);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t n_t = (size_t)T_total * H, n_tk = n_t * DK;
+  const size_t n_t = (size_t)T_total * H;
+  return launch_bwd_reduce<IOT>(pq, pk, pa, pb, dq, dk, dalpha, dbeta, n_t * DK, n_t, ntile, st);
+}
+
+}  // namespace
+
+template <typename IOT>
+cudaError_t launch_bwd_reduce(const float *pq, const float *pk, const float *pa,
+                              const float *pb, void *dq, void *dk, float *dalpha, float *dbeta,
+                              size_t n_tk, size_t n_t, int ntile, cudaStream_t st) {
   if (n_tk == 0) return cudaSuccess;
   const unsigned grid = (unsigned)std::min<size_t>((n_tk + 255) / 256, 148 * 16);
   ckda_bwd_reduce_kernel<IOT><<<grid, 256, 0, st>>>(pq, pk, pa, pb, static_cast<IOT *>(dq),
@@ -285,8 +303,13 @@ cudaError_t launch_bwd_dims(const void *q, const void *k, const void *v, const f
                                                    n_t, ntile);
   return cudaGetLastError();
 }
-
-}  // namespace
+template cudaError_t launch_bwd_reduce<float>(const float *, const float *, const float *,
+                                              const float *, void *, void *, float *, float *,
+                                              size_t, size_t, int, cudaStream_t);
+template cudaError_t launch_bwd_reduce<__nv_bfloat16>(const float *, const float *,
+                                                      const float *, const float *, void *,
+                                                      void *, float *, float *, size_t, size_t,
+                                                      int, cudaStream_t);
 
 // columns per CTA
 static int bwd_tile(int dv) { return dv < 32 ? dv : 32; }

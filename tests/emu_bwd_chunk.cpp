@@ -1,0 +1,126 @@
+// Test-only host build of the chunkwise backward's per-CTA program
+// (csrc/ckda_bwd_chunk.cuh): every CTA of the launch grid runs in turn, each
+// phase as a plain loop over its work items, which is the same set of calls
+// the GPU makes between two barriers. It checks the program's index
+// arithmetic and algebra on the CPU (built with AddressSanitizer by the
+// test); it is not a product path and no library calls it.
+//
+// usage: emu_bwd_chunk DIR N T H d_k d_v scale varlen has_s0 has_dsf
+// DIR holds float32 q k v alpha beta do [s0] [dsf] and int32 cu (varlen) as
+// raw .bin files; writes dq dk dv dalpha dbeta ds0 (.bin, float32) there.
+#include <cstdio>
+#include <cstdlib>
+#include <string>
+#include <vector>
+
+#include "ckda_bwd_chunk.cuh"
+
+namespace {
+
+struct HostExec {
+  template <class F>
+  void par(int n, F f) {
+    for (int i = 0; i < n; ++i) f(i);
+  }
+};
+
+struct HostIO {
+  static float ld(const float *p) { return *p; }
+  static void st(float *p, float x) { *p = x; }
+};
+
+std::vector<float> load(const std::string &path, size_t n) {
+  std::vector<float> x(n);
+  FILE *f = std::fopen(path.c_str(), "rb");
+  if (!f || std::fread(x.data(), sizeof(float), n, f) != n) {
+    std::fprintf(stderr, "cannot read %s\n", path.c_str());
+    std::exit(2);
+  }
+  std::fclose(f);
+  return x;
+}
+
+void save(const std::string &path, const std::vector<float> &x) {
+  FILE *f = std::fopen(path.c_str(), "wb");
+  if (!f || std::fwrite(x.data(), sizeof(float), x.size(), f) != x.size()) std::exit(3);
+  std::fclose(f);
+}
+
+template <int DK, int DVT>
+void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool varlen,
+         bool has_s0, bool has_dsf) {
+  using namespace ckda::bwdc;
+  std::vector<int> cu(N + 1);
+  int T_total = N * T;
+  if (varlen) {
+    FILE *f = std::fopen((dir + "/cu.bin").c_str(), "rb");
+    if (!f || std::fread(cu.data(), sizeof(int), N + 1, f) != (size_t)N + 1) std::exit(2);
+    std::fclose(f);
+    T_total = T;
+  }
+  const size_t TH = (size_t)T_total * H;
+  auto q = load(dir + "/q.bin", TH * DK), k = load(dir + "/k.bin", TH * DK);
+  auto v = load(dir + "/v.bin", TH * DV), al = load(dir + "/alpha.bin", TH * DK);
+  auto be = load(dir + "/beta.bin", TH), d_o = load(dir + "/do.bin", TH * DV);
+  const size_t st = (size_t)N * H * DK * DV;
+  std::vector<float> s0, dsf;
+  if (has_s0) s0 = load(dir + "/s0.bin", st);
+  if (has_dsf) dsf = load(dir + "/dsf.bin", st);
+  const int ntile = DV / DVT;
+  const size_t slots = (size_t)T_total / C + N;
+  std::vector<float> ck(slots * H * DK * DV), dv(TH * DV), ds0(st);
+  std::vector<float> pq(ntile * TH * DK), pk(ntile * TH * DK), pa(ntile * TH * DK),
+      pb(ntile * TH);
+  Args<float> a{q.data(), k.data(), v.data(), al.data(), be.data(),
+                has_s0 ? s0.data() : nullptr, d_o.data(), has_dsf ? dsf.data() : nullptr,
+                dv.data(), pq.data(), pk.data(), pa.data(), pb.data(), ds0.data(),
+                ck.data(), H, DV, TH, scale};
+  std::vector<float> sm(Layout<DK, DVT>::FLOATS);
+  HostExec x;
+  for (int tile = 0; tile < ntile; ++tile)
+    for (int n = 0; n < N; ++n)
+      for (int h = 0; h < H; ++h) {
+        const int bos = varlen ? cu[n] : n * T, eos = varlen ? cu[n + 1] : bos + T;
+        bwd_chunk_program<HostExec, HostIO, float, DK, DVT>(x, a, sm.data(), h, n, tile, bos,
+                                                           eos, bos / C + n);
+      }
+  std::vector<float> dq(TH * DK), dk(TH * DK), da(TH * DK), db(TH);
+  for (size_t i = 0; i < TH * DK; ++i)
+    for (int t = 0; t < ntile; ++t) {
+      dq[i] += pq[t * TH * DK + i];
+      dk[i] += pk[t * TH * DK + i];
+      da[i] += pa[t * TH * DK + i];
+    }
+  for (size_t i = 0; i < TH; ++i)
+    for (int t = 0; t < ntile; ++t) db[i] += pb[t * TH + i];
+  save(dir + "/dq.bin", dq);
+  save(dir + "/dk.bin", dk);
+  save(dir + "/dv.bin", dv);
+  save(dir + "/dalpha.bin", da);
+  save(dir + "/dbeta.bin", db);
+  save(dir + "/ds0.bin", ds0);
+}
+
+}  // namespace
+
+int main(int argc, char **argv) {
+  if (argc != 11) {
+    std::fprintf(stderr, "usage: %s DIR N T H d_k d_v scale varlen has_s0 has_dsf\n", argv[0]);
+    return 1;
+  }
+  const std::string dir = argv[1];
+  const int N = std::atoi(argv[2]), T = std::atoi(argv[3]), H = std::atoi(argv[4]);
+  const int dk = std::atoi(argv[5]), dv = std::atoi(argv[6]);
+  const float scale = (float)std::atof(argv[7]);
+  const bool varlen = std::atoi(argv[8]), s0 = std::atoi(argv[9]), dsf = std::atoi(argv[10]);
+#define EMU_CASE(DK, DVT)                                       \
+  if (dk == DK && (dv < 32 ? dv : 32) == DVT) {                 \
+    run<DK, DVT>(dir, N, T, H, dv, scale, varlen, s0, dsf);     \
+    return 0;                                                   \
+  }
+  EMU_CASE(16, 16) EMU_CASE(16, 32) EMU_CASE(32, 16) EMU_CASE(32, 32)
+  EMU_CASE(64, 16) EMU_CASE(64, 32) EMU_CASE(128, 16) EMU_CASE(128, 32)
+#undef EMU_CASE
+  std::fprintf(stderr, "unsupported d_k=%d d_v=%d\n", dk, dv);
+  return 1;
+}
