@@ -83,6 +83,8 @@ def load(path: str | None = None):
     lib.ckda_status_string.argtypes = [ctypes.c_int]
     lib.ckda_bwd.restype = ctypes.c_int
     lib.ckda_bwd.argtypes = [vp] * 16 + [i32] * 5 + [f32, ctypes.c_int, vp, ctypes.c_size_t, vp]
+    lib.ckda_bwd_chunked.restype = ctypes.c_int
+    lib.ckda_bwd_chunked.argtypes = lib.ckda_bwd.argtypes
     lib.ckda_fwd_complex.restype = ctypes.c_int
     lib.ckda_fwd_complex.argtypes = [vp] * 11 + [i32] * 5 + [f32, vp]
     lib.ckda_bwd_workspace_bytes.restype = ctypes.c_size_t
@@ -218,12 +220,14 @@ def ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, varlen=False) -> int:
 
 def ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv,
              dalpha, dbeta, d_initial_state, cu_seqlens=None, cu_seqlens_host=None,
-             N=None, T=None, scale: float = 1.0, stream=None, workspace=None):
-    """Marshal tensors into ckda_bwd (see include/ckda.h): gradients of
-    ckda_fwd_chunked for dL/do = d_o and dL/d(final state) = d_final_state
-    (None = zero). dq, dk [T_total, H, d_k] and dv [T_total, H, d_v] in q's
-    dtype, dalpha [T_total, H, d_k] and dbeta [T_total, H] fp32 and
-    d_initial_state [N, H, d_k, d_v] fp32 (or None) are written."""
+             N=None, T=None, scale: float = 1.0, stream=None, workspace=None,
+             chunked: bool = False):
+    """Marshal tensors into ckda_bwd, or ckda_bwd_chunked when ``chunked``
+    (see include/ckda.h): gradients of ckda_fwd_chunked for dL/do = d_o and
+    dL/d(final state) = d_final_state (None = zero). dq, dk [T_total, H, d_k]
+    and dv [T_total, H, d_v] in q's dtype, dalpha [T_total, H, d_k] and dbeta
+    [T_total, H] fp32 and d_initial_state [N, H, d_k, d_v] fp32 (or None) are
+    written."""
     lib = load()
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (d_o, "d_o"), (dq, "dq"), (dk, "dk"),
                    (dv, "dv")):
@@ -256,12 +260,12 @@ def ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    st = lib.ckda_bwd(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(initial_state), _p(d_o),
-                      _p(d_final_state), _p(dq), _p(dk), _p(dv), _p(dalpha), _p(dbeta),
-                      _p(d_initial_state), _p(cu_seqlens), host_ptr, int(N), int(T), int(H),
-                      int(d_k), int(d_v), float(scale), _DT[q.dtype], _p(workspace), ws_bytes,
-                      _stream(stream))
-    _check(st, "ckda_bwd")
+    fn = lib.ckda_bwd_chunked if chunked else lib.ckda_bwd
+    st = fn(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(initial_state), _p(d_o),
+            _p(d_final_state), _p(dq), _p(dk), _p(dv), _p(dalpha), _p(dbeta),
+            _p(d_initial_state), _p(cu_seqlens), host_ptr, int(N), int(T), int(H), int(d_k),
+            int(d_v), float(scale), _DT[q.dtype], _p(workspace), ws_bytes, _stream(stream))
+    _check(st, "ckda_bwd_chunked" if chunked else "ckda_bwd")
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20  # CKDA_NOALLOC_SCRATCH_BYTES in include/ckda.h
@@ -453,9 +457,9 @@ def fwd_complex(q, k, v, alpha, theta, beta, initial_state=None, cu_seqlens=None
 
 def bwd(q, k, v, alpha, beta, d_o, initial_state=None, d_final_state=None,
         cu_seqlens=None, cu_seqlens_host=None, N=None, T=None, scale: float = 1.0,
-        stream=None, workspace=None):
-    """Allocate the gradients with torch, then call ckda_bwd. Returns
-    (dq, dk, dv, dalpha, dbeta, d_initial_state)."""
+        stream=None, workspace=None, chunked: bool = False):
+    """Allocate the gradients with torch, then call ckda_bwd (ckda_bwd_chunked
+    when ``chunked``). Returns (dq, dk, dv, dalpha, dbeta, d_initial_state)."""
     T_total, H, d_k = q.shape
     d_v = v.shape[2]
     if cu_seqlens is not None:
@@ -467,7 +471,7 @@ def bwd(q, k, v, alpha, beta, d_o, initial_state=None, d_final_state=None,
     dalpha, dbeta = torch.empty_like(alpha), torch.empty_like(beta)
     ds0 = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=q.device)
     ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv, dalpha,
-             dbeta, ds0, cu_seqlens, cu_seqlens_host, N, T, scale, stream, workspace)
+             dbeta, ds0, cu_seqlens, cu_seqlens_host, N, T, scale, stream, workspace, chunked)
     return dq, dk, dv, dalpha, dbeta, ds0
 
 

@@ -35,6 +35,13 @@ cudaError_t launch_bwd(int dk, int dv, const void *q, const void *k, const void 
                        float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
                        int T, int T_total, int H, float scale, void *ws,
                        unsigned int *err, cudaStream_t st);
+template <typename IOT>
+cudaError_t launch_bwd_chunk(int dk, int dv, const void *q, const void *k, const void *v,
+                             const float *alpha, const float *beta, const float *s0,
+                             const void *d_o, const float *dsf, void *dq, void *dk_, void *dv_,
+                             float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
+                             int T, int T_total, int H, float scale, void *ws,
+                             unsigned int *err, cudaStream_t st);
 bool fwd_tc_supported(int dk, int dv, int chunk, ckda_dtype dt);
 size_t fwd_tc_workspace_bytes(int N, int T_total, int H, int dv);
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
@@ -215,14 +222,20 @@ size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
   return ckda::bwd_workspace_bytes(N, (int)T_total, H, d_k, d_v);
 }
 
-ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *alpha,
+}  // extern "C"
+
+namespace {
+
+// ckda_bwd (token-serial kernel) and ckda_bwd_chunked (chunkwise kernel):
+// one validation, then the chosen launch.
+ckda_status bwd_impl(const void *q, const void *k, const void *v, const float *alpha,
                      const float *beta, const float *initial_state, const void *d_o,
                      const float *d_final_state, void *dq, void *dk, void *dv,
                      float *dalpha, float *dbeta, float *d_initial_state,
                      const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, int32_t N,
                      int32_t T, int32_t H, int32_t d_k, int32_t d_v, float scale,
                      ckda_dtype dt, void *workspace, size_t workspace_bytes,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool chunked) {
   if (dt != CKDA_BF16 && dt != CKDA_F32) return CKDA_ERR_UNSUPPORTED;
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
@@ -255,18 +268,49 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
   if (N == 0) return CKDA_OK;
   if (!workspace || workspace_bytes < need) return CKDA_ERR_ARG;
   unsigned int *err = error_word_ptr();
-  cudaError_t e;
-  if (dt == CKDA_F32)
-    e = ckda::launch_bwd<float>(d_k, d_v, q, k, v, alpha, beta, initial_state, d_o,
-                                d_final_state, dq, dk, dv, dalpha, dbeta, d_initial_state,
-                                cu_seqlens, N, T, (int)T_total, H, scale, workspace, err,
-                                stream);
-  else
-    e = ckda::launch_bwd<__nv_bfloat16>(d_k, d_v, q, k, v, alpha, beta, initial_state, d_o,
-                                        d_final_state, dq, dk, dv, dalpha, dbeta,
-                                        d_initial_state, cu_seqlens, N, T, (int)T_total, H,
-                                        scale, workspace, err, stream);
+  auto launch = [&](auto io) {
+    using IOT = decltype(io);
+    return chunked ? ckda::launch_bwd_chunk<IOT>(d_k, d_v, q, k, v, alpha, beta, initial_state,
+                                                 d_o, d_final_state, dq, dk, dv, dalpha, dbeta,
+                                                 d_initial_state, cu_seqlens, N, T,
+                                                 (int)T_total, H, scale, workspace, err, stream)
+                   : ckda::launch_bwd<IOT>(d_k, d_v, q, k, v, alpha, beta, initial_state, d_o,
+                                           d_final_state, dq, dk, dv, dalpha, dbeta,
+                                           d_initial_state, cu_seqlens, N, T, (int)T_total, H,
+                                           scale, workspace, err, stream);
+  };
+  const cudaError_t e = dt == CKDA_F32 ? launch(float{}) : launch(__nv_bfloat16{});
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *alpha,
+                     const float *beta, const float *initial_state, const void *d_o,
+                     const float *d_final_state, void *dq, void *dk, void *dv,
+                     float *dalpha, float *dbeta, float *d_initial_state,
+                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host, int32_t N,
+                     int32_t T, int32_t H, int32_t d_k, int32_t d_v, float scale,
+                     ckda_dtype dt, void *workspace, size_t workspace_bytes,
+                     cudaStream_t stream) {
+  return bwd_impl(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv, dalpha,
+                  dbeta, d_initial_state, cu_seqlens, cu_seqlens_host, N, T, H, d_k, d_v, scale,
+                  dt, workspace, workspace_bytes, stream, false);
+}
+
+ckda_status ckda_bwd_chunked(const void *q, const void *k, const void *v, const float *alpha,
+                             const float *beta, const float *initial_state, const void *d_o,
+                             const float *d_final_state, void *dq, void *dk, void *dv,
+                             float *dalpha, float *dbeta, float *d_initial_state,
+                             const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                             int32_t N, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                             float scale, ckda_dtype dt, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+  return bwd_impl(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv, dalpha,
+                  dbeta, d_initial_state, cu_seqlens, cu_seqlens_host, N, T, H, d_k, d_v, scale,
+                  dt, workspace, workspace_bytes, stream, true);
 }
 
 size_t ckda_fwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,

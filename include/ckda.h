@@ -272,6 +272,29 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
                      cudaStream_t stream);
 
 /*
+ * ckda_bwd_chunked: the gradients of ckda_bwd (the same arguments, layouts,
+ * workspace query, errors and outputs) computed 16 tokens at a time in the
+ * chunk-WY form of the forward ("Semidirect Fourier Delta Attention" §2.2
+ * eqs. (9)-(10)) run in reverse: per chunk, dU = scale M^T dO + Kbar dS_C,
+ * dR = T^T dU, dv = diag(beta) dR, then dq, dk, dbeta from matrix products and
+ * the gated Gram terms, and dalpha per channel as the gate product with the
+ * one factor alpha_s left out (two running products, no logarithm and no
+ * division, so zero and negative gates are exact). Only the d_k x d_v state
+ * gradient dS = scale Qhat^T dO + diag(gamma) dS_C - Khat^T diag(beta) dR
+ * passes from chunk to chunk. One CTA per (sequence, head, tile of up to 32
+ * state columns), fp32 arithmetic on CUDA cores, deterministic (tile partials
+ * added in a fixed order).
+ */
+ckda_status ckda_bwd_chunked(const void *q, const void *k, const void *v, const float *alpha,
+                             const float *beta, const float *initial_state, const void *d_o,
+                             const float *d_final_state, void *dq, void *dk, void *dv,
+                             float *dalpha, float *dbeta, float *d_initial_state,
+                             const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                             int32_t N, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                             float scale, ckda_dtype dt, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * ckda_fwd_complex: the complex-phase gate of "Semidirect Fourier Delta
  * Attention" §3, eqs. (13)-(14), with complex q, k, v and state:
  *   S_t = (I - beta_t k_t k_t^*) Lambda_t S_{t-1} + beta_t k_t v_t^*,
@@ -297,7 +320,8 @@ ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const 
                              int32_t d_k, int32_t d_v, float scale, cudaStream_t stream);
 
 /*
- * ckda_bwd_workspace_bytes: scratch ckda_bwd needs (T as in ckda_bwd; varlen
+ * ckda_bwd_workspace_bytes: scratch ckda_bwd and ckda_bwd_chunked need (T as
+ * in ckda_bwd; varlen
  * nonzero when cu_seqlens is given, so that T is total_T). 0 for unsupported
  * or invalid sizes.
  */

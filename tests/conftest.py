@@ -13,6 +13,15 @@ def pytest_configure(config):
         "markers", "gpu: needs a CUDA GPU (sm_100a) and the built CUDA library")
     config.addinivalue_line(
         "markers", "slow: long CPU test (oracle at full workload size)")
+    config.addinivalue_line(
+        "markers", "last: run after every other collected test (newest GPU paths)")
+
+
+def pytest_collection_modifyitems(config, items):
+    """Tests marked ``last`` run after all others, in their collected order,
+    so that a run stopping at the first failure has already run the rest."""
+    items[:] = ([it for it in items if it.get_closest_marker("last") is None]
+                + [it for it in items if it.get_closest_marker("last") is not None])
 
 
 def gpu_available() -> bool:

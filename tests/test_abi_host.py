@@ -218,9 +218,9 @@ def test_binding_argument_counts_match_the_header(lib):
 def bwd(lib, q=P, k=P2, v=P3, a=P4, b=P5, do=P6, dq=ctypes.c_void_p(0x70000),
         dk=ctypes.c_void_p(0x80000), dv=ctypes.c_void_p(0x90000),
         da=ctypes.c_void_p(0xA0000), db=ctypes.c_void_p(0xB0000), N=1, T=8, H=1, dkd=16,
-        dvd=16, dt=ckda.CKDA_F32, ws=ctypes.c_void_p(0x100000), wsb=1 << 30):
-    return lib.ckda_bwd(q, k, v, a, b, NULL, do, NULL, dq, dk, dv, da, db, NULL, NULL, NULL,
-                        N, T, H, dkd, dvd, 1.0, dt, ws, wsb, None)
+        dvd=16, dt=ckda.CKDA_F32, ws=ctypes.c_void_p(0x100000), wsb=1 << 30, fn="ckda_bwd"):
+    return getattr(lib, fn)(q, k, v, a, b, NULL, do, NULL, dq, dk, dv, da, db, NULL, NULL, NULL,
+                            N, T, H, dkd, dvd, 1.0, dt, ws, wsb, None)
 
 
 @pytest.mark.parametrize("kw,want", [
@@ -241,8 +241,9 @@ def bwd(lib, q=P, k=P2, v=P3, a=P4, b=P5, do=P6, dq=ctypes.c_void_p(0x70000),
     (dict(ws=NULL), ckda.CKDA_ERR_ARG),
     (dict(wsb=1024), ckda.CKDA_ERR_ARG),
 ])
-def test_bwd_rejects(lib, kw, want):
-    assert bwd(lib, **kw) == want
+@pytest.mark.parametrize("fn", ["ckda_bwd", "ckda_bwd_chunked"])
+def test_bwd_rejects(lib, kw, want, fn):
+    assert bwd(lib, fn=fn, **kw) == want
 
 
 def test_bwd_workspace_query(lib):
@@ -264,6 +265,7 @@ def test_bwd_zero_sequences_is_a_noop(lib):
     """N = 0: validated, nothing launched, CKDA_OK (the fake pointers are
     never dereferenced)."""
     assert bwd(lib, N=0, T=0, ws=NULL, wsb=0) == ckda.CKDA_OK
+    assert bwd(lib, N=0, T=0, ws=NULL, wsb=0, fn="ckda_bwd_chunked") == ckda.CKDA_OK
 
 
 def cplx(lib, q=P, k=P2, v=P3, a=P4, th=P5, b=P6, s0=NULL, sf=NULL,

@@ -1,5 +1,8 @@
-"""GPU parity of the backward pass (ckda_bwd) against the oracle's fp64
-adjoint (oracle.bwd, pinned by finite differences in test_oracle_bwd.py).
+"""GPU parity of the backward pass against the oracle's fp64 adjoint
+(oracle.bwd, pinned by finite differences in test_oracle_bwd.py), for both
+entry points: ckda_bwd (token-serial kernel) and ckda_bwd_chunked (the
+chunkwise kernel, whose per-CTA program test_bwd_chunk_emu.py also runs on
+the CPU).
 
 Tolerances follow the forward's rule (parity_util): fp32 I/O check mode
 max|x - x_ref| <= BWD_FP32_REL * rms(x_ref) for every gradient; bf16 I/O
@@ -49,12 +52,17 @@ def case(w, lens, H, with_final=True, with_s0=True):
     return inp, grads
 
 
-def run_gpu(inp, grads, scale):
+# the chunkwise kernel's cases run after every other GPU test
+IMPLS = pytest.mark.parametrize(
+    "chunked", [False, pytest.param(True, marks=pytest.mark.last)], ids=["serial", "chunked"])
+
+
+def run_gpu(inp, grads, scale, chunked=False):
     d = to_dev(inp)
     g = to_dev(grads)
     out = ckda.bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], g["d_o"], d["initial_state"],
                    g["d_final_state"], cu_seqlens=d["cu_seqlens"],
-                   cu_seqlens_host=inp["cu_seqlens"], scale=scale)
+                   cu_seqlens_host=inp["cu_seqlens"], scale=scale, chunked=chunked)
     torch.cuda.synchronize()
     assert ckda.ckda_last_error() == ckda.CKDA_OK
     return out
@@ -83,10 +91,11 @@ def compare(got, ref, bf16):
     (64, 128, [31]),
     (128, 16, [48, 2]),
 ])
-def test_bwd_fp32(cuda_lib, d_k, d_v, lens):
+@IMPLS
+def test_bwd_fp32(cuda_lib, d_k, d_v, lens, chunked):
     w = custom("ckda_B1_H32_T8192_d128", dtype="f32", d_k=d_k, d_v=d_v, seed=600 + d_k + d_v)
     inp, grads = case(w, lens, H=2)
-    compare(run_gpu(inp, grads, 0.8), run_ref(inp, grads, 0.8), bf16=False)
+    compare(run_gpu(inp, grads, 0.8, chunked), run_ref(inp, grads, 0.8), bf16=False)
 
 
 @pytest.mark.parametrize("base,alpha_kind,lens,H", [
@@ -94,31 +103,35 @@ def test_bwd_fp32(cuda_lib, d_k, d_v, lens):
     ("kda_B4_H16_T2048_d128", None, [200, 1], 3),
     ("ckda_B1_H32_T8192_d128", "slow", [257], 2),
 ])
-def test_bwd_bf16(cuda_lib, base, alpha_kind, lens, H):
+@IMPLS
+def test_bwd_bf16(cuda_lib, base, alpha_kind, lens, H, chunked):
     kw = dict(seed=700 + sum(lens))
     if alpha_kind:
         kw["alpha_kind"] = alpha_kind
     w = custom(base, **kw)
     inp, grads = case(w, lens, H=H)
-    compare(run_gpu(inp, grads, 1.0), run_ref(inp, grads, 1.0), bf16=True)
+    compare(run_gpu(inp, grads, 1.0, chunked), run_ref(inp, grads, 1.0), bf16=True)
 
 
-def test_bwd_without_final_gradient_or_initial_state(cuda_lib):
+@IMPLS
+def test_bwd_without_final_gradient_or_initial_state(cuda_lib, chunked):
     w = custom("ckda_B1_H32_T8192_d128", dtype="f32", d_k=32, d_v=32, seed=811)
     inp, grads = case(w, [20, 45], H=2, with_final=False, with_s0=False)
-    compare(run_gpu(inp, grads, 1.0), run_ref(inp, grads, 1.0), bf16=False)
+    compare(run_gpu(inp, grads, 1.0, chunked), run_ref(inp, grads, 1.0), bf16=False)
 
 
-def test_bwd_is_deterministic(cuda_lib):
+@IMPLS
+def test_bwd_is_deterministic(cuda_lib, chunked):
     w = custom("ckda_B1_H32_T8192_d128", seed=812)
     inp, grads = case(w, [150, 30], H=2)
-    a = run_gpu(inp, grads, 1.0)
-    b = run_gpu(inp, grads, 1.0)
+    a = run_gpu(inp, grads, 1.0, chunked)
+    b = run_gpu(inp, grads, 1.0, chunked)
     for name, x, y in zip(NAMES, a, b):
         assert torch.equal(x, y), name
 
 
-def test_bwd_equal_length_sequences_without_cu_seqlens(cuda_lib):
+@IMPLS
+def test_bwd_equal_length_sequences_without_cu_seqlens(cuda_lib, chunked):
     """N sequences of T tokens given by N and T alone (no cu_seqlens): the
     checkpoint slots come from n T instead of the device offsets."""
     w = custom("ckda_B1_H32_T8192_d128", dtype="f32", d_k=32, d_v=64, seed=813)
@@ -126,7 +139,7 @@ def test_bwd_equal_length_sequences_without_cu_seqlens(cuda_lib):
     d = to_dev(inp)
     g = to_dev(grads)
     got = ckda.bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], g["d_o"], d["initial_state"],
-                   g["d_final_state"], N=2, T=40, scale=0.7)
+                   g["d_final_state"], N=2, T=40, scale=0.7, chunked=chunked)
     torch.cuda.synchronize()
     assert ckda.ckda_last_error() == ckda.CKDA_OK
     compare(got, run_ref(inp, grads, 0.7), bf16=False)

@@ -6,8 +6,9 @@ cudaMalloc while it runs): its scratch is a fixed array inside the library.
 These tests call it through the C ABI and compare with ckda_fwd_chunked run
 on a workspace from torch, on two calls in a row with different inputs (the
 shared array keeps the first call's contents when the second one starts).
-This file is collected last so that a run stopping at the first failure has
-already run every other test.
+This file is collected after the other test files (only tests marked ``last``
+follow it), so that a run stopping at the first failure has already run the
+rest.
 """
 import dataclasses
 
