@@ -300,6 +300,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--bwd-steps", type=int, default=5)
+    ap.add_argument("--bwd-impl", default="serial", choices=["serial", "chunked"],
+                    help="backward entry point: ckda_bwd (token-serial) or ckda_bwd_chunked")
     ap.add_argument("--complex-steps", type=int, default=5)
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -424,7 +426,7 @@ def main():
     def bwd_step():
         ckda.ckda_bwd(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"],
                       dev["initial_state"], bdo, bdsf, *bout, dev["cu_seqlens"], None,
-                      stream=stream, workspace=bws)
+                      stream=stream, workspace=bws, chunked=args.bwd_impl == "chunked")
 
     bms = time_loop(bwd_step, args.bwd_steps, 3, stream, barrier)
     if ckda.ckda_last_error() != ckda.CKDA_OK:
@@ -435,10 +437,15 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": bbytes / (bms / 1e3) / 1e9,
                              "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": bbytes / (bms / 1e3) / 1e9 / pk["hbm_gbs"],
-                             "traffic": NCU_TRAFFIC["backward"],
+                             # counters were taken on the token-serial kernel
+                             "traffic": (NCU_TRAFFIC["backward"] if args.bwd_impl == "serial"
+                                         else None),
                              "algorithmic_bytes_per_launch": bbytes},
-                "kernel": "token-serial adjoint on CUDA cores, one CTA per (sequence, head, "
-                          "32-column tile), plus a tile reduction",
+                "kernel": ("token-serial adjoint on CUDA cores, one CTA per (sequence, head, "
+                           "32-column tile), plus a tile reduction" if args.bwd_impl == "serial"
+                           else "chunkwise (16-token chunk-WY reverse) on CUDA cores, one CTA "
+                                "per (sequence, head, 32-column tile), plus a tile reduction"),
+                "entry_point": "ckda_bwd_chunked" if args.bwd_impl == "chunked" else "ckda_bwd",
                 "gpu_launches": 2 * args.bwd_steps}
     del bws, bout
 

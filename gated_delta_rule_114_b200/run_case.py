@@ -2,7 +2,7 @@
 
     python -m gated_delta_rule_114_b200.run_case --case prefill [--T 4096] [--iters 3]
     python -m gated_delta_rule_114_b200.run_case --case decode [--N 64] [--iters 3]
-    python -m gated_delta_rule_114_b200.run_case --case bwd [--T 2048] [--iters 2]
+    python -m gated_delta_rule_114_b200.run_case --case bwd [--T 2048] [--iters 2] [--chunked]
 
 The prefill case uses the CKDA long-prefill recipe (H=32, d=128, bf16 I/O,
 CKDA gates, random initial state) with T tokens per head; the decode case
@@ -31,6 +31,8 @@ def main():
     ap.add_argument("--H", type=int, default=32)
     ap.add_argument("--N", type=int, default=64)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--chunked", action="store_true",
+                    help="bwd case: ckda_bwd_chunked instead of ckda_bwd")
     args = ap.parse_args()
     ckda.load()
     if args.case == "prefill":
@@ -50,7 +52,8 @@ def main():
         g = {k: v.cuda() for k, v in make_bwd_grads(w, args.T, args.H, 1).items()}
         for _ in range(args.iters):
             ckda.bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], g["d_o"],
-                     d["initial_state"], g["d_final_state"], cu_seqlens=d["cu_seqlens"])
+                     d["initial_state"], g["d_final_state"], cu_seqlens=d["cu_seqlens"],
+                     chunked=args.chunked)
         shape = "T=%d H=%d d=128" % (args.T, args.H)
     else:
         w = WORKLOADS["decode_N256_H32_d128"]
