@@ -420,7 +420,8 @@ def main():
     bout = [torch.empty_like(dev["q"]), torch.empty_like(dev["k"]), torch.empty_like(dev["v"]),
             torch.empty_like(dev["alpha"]), torch.empty_like(dev["beta"]),
             torch.empty((N, H, dk, dv), dtype=torch.float32, device="cuda")]
-    bws = torch.empty(ckda.ckda_bwd_workspace_bytes(N, T_total, H, dk, dv, True),
+    bws = torch.empty(ckda.ckda_bwd_workspace_bytes(N, T_total, H, dk, dv, True,
+                                                    args.bwd_impl == "chunked"),
                       dtype=torch.uint8, device="cuda")
 
     def bwd_step():
@@ -443,10 +444,11 @@ def main():
                              "algorithmic_bytes_per_launch": bbytes},
                 "kernel": ("token-serial adjoint on CUDA cores, one CTA per (sequence, head, "
                            "32-column tile), plus a tile reduction" if args.bwd_impl == "serial"
-                           else "chunkwise (16-token chunk-WY reverse) on CUDA cores, one CTA "
-                                "per (sequence, head, 32-column tile), plus a tile reduction"),
+                           else "chunkwise (16-token chunk-WY reverse) on CUDA cores: prep and "
+                                "gradients over all chunks, two scans per (sequence, head, "
+                                "32-column tile), plus a tile reduction"),
                 "entry_point": "ckda_bwd_chunked" if args.bwd_impl == "chunked" else "ckda_bwd",
-                "gpu_launches": 2 * args.bwd_steps}
+                "gpu_launches": (2 if args.bwd_impl == "serial" else 5) * args.bwd_steps}
     del bws, bout
 
     # ---------------- the complex-phase gate on the same shape (complex64)

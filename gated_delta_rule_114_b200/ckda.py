@@ -89,6 +89,8 @@ def load(path: str | None = None):
     lib.ckda_fwd_complex.argtypes = [vp] * 11 + [i32] * 5 + [f32, vp]
     lib.ckda_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.ckda_bwd_workspace_bytes.argtypes = [i32] * 6
+    lib.ckda_bwd_chunked_workspace_bytes.restype = ctypes.c_size_t
+    lib.ckda_bwd_chunked_workspace_bytes.argtypes = [i32] * 6
     lib.ckda_last_error.restype = ctypes.c_int
     lib.ckda_last_error.argtypes = [vp]
     lib.ckda_version.restype = ctypes.c_int32
@@ -212,10 +214,11 @@ def _fwd_call(q, k, v, alpha, beta, initial_state, final_state, o, cu_seqlens,
         _check(st, "ckda_fwd_chunked_gated")
 
 
-def ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, varlen=False) -> int:
-    """Scratch bytes ckda_bwd needs (see include/ckda.h)."""
-    return int(load().ckda_bwd_workspace_bytes(int(N), int(T), int(H), int(d_k), int(d_v),
-                                               int(bool(varlen))))
+def ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, varlen=False, chunked=False) -> int:
+    """Scratch bytes ckda_bwd (ckda_bwd_chunked when ``chunked``) needs
+    (see include/ckda.h)."""
+    fn = load().ckda_bwd_chunked_workspace_bytes if chunked else load().ckda_bwd_workspace_bytes
+    return int(fn(int(N), int(T), int(H), int(d_k), int(d_v), int(bool(varlen))))
 
 
 def ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv,
@@ -256,7 +259,7 @@ def ckda_bwd(q, k, v, alpha, beta, initial_state, d_o, d_final_state, dq, dk, dv
                 or not cu_seqlens_host.is_contiguous():
             raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
         host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
-    need = ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens is not None)
+    need = ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens is not None, chunked)
     if need and workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()

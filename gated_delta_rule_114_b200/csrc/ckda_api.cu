@@ -35,8 +35,9 @@ cudaError_t launch_bwd(int dk, int dv, const void *q, const void *k, const void 
                        float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
                        int T, int T_total, int H, float scale, void *ws,
                        unsigned int *err, cudaStream_t st);
+size_t bwd_split_workspace_bytes(int N, int T_total, int H, int dk, int dv);
 template <typename IOT>
-cudaError_t launch_bwd_chunk(int dk, int dv, const void *q, const void *k, const void *v,
+cudaError_t launch_bwd_split(int dk, int dv, const void *q, const void *k, const void *v,
                              const float *alpha, const float *beta, const float *s0,
                              const void *d_o, const float *dsf, void *dq, void *dk_, void *dv_,
                              float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
@@ -222,6 +223,14 @@ size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
   return ckda::bwd_workspace_bytes(N, (int)T_total, H, d_k, d_v);
 }
 
+size_t ckda_bwd_chunked_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                        int32_t d_v, int32_t varlen) {
+  if (N <= 0 || T < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v)) return 0;
+  const int64_t T_total = varlen ? (int64_t)T : (int64_t)N * T;
+  if (T_total > INT32_MAX) return 0;
+  return ckda::bwd_split_workspace_bytes(N, (int)T_total, H, d_k, d_v);
+}
+
 }  // extern "C"
 
 namespace {
@@ -252,7 +261,9 @@ ckda_status bwd_impl(const void *q, const void *k, const void *v, const float *a
   const size_t es = esize(dt), th = (size_t)T_total * H;
   const size_t kb = th * d_k * es, vb = th * d_v * es, ab = th * d_k * sizeof(float);
   const size_t bb = th * sizeof(float), sb = (size_t)N * H * d_k * d_v * sizeof(float);
-  const size_t need = ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens != nullptr);
+  const size_t need = chunked
+                          ? ckda_bwd_chunked_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens != nullptr)
+                          : ckda_bwd_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens != nullptr);
   struct R { const void *p; size_t n; };
   const R ins[] = {{q, kb}, {k, kb}, {v, vb}, {alpha, ab}, {beta, bb}, {initial_state, sb},
                    {d_o, vb}, {d_final_state, sb},
@@ -270,7 +281,7 @@ ckda_status bwd_impl(const void *q, const void *k, const void *v, const float *a
   unsigned int *err = error_word_ptr();
   auto launch = [&](auto io) {
     using IOT = decltype(io);
-    return chunked ? ckda::launch_bwd_chunk<IOT>(d_k, d_v, q, k, v, alpha, beta, initial_state,
+    return chunked ? ckda::launch_bwd_split<IOT>(d_k, d_v, q, k, v, alpha, beta, initial_state,
                                                  d_o, d_final_state, dq, dk, dv, dalpha, dbeta,
                                                  d_initial_state, cu_seqlens, N, T,
                                                  (int)T_total, H, scale, workspace, err, stream)

@@ -1,4 +1,4 @@
-// The chunkwise backward pass of the CKDA recurrence: the per-CTA program.
+// The chunkwise backward pass of the CKDA recurrence: per-chunk pieces.
 //
 // Forward of one chunk of C tokens (rows i, j in 0..C-1; entry state S;
 // G_{i<-j} = prod_{s=j+1..i} diag(alpha_s); gamma_i = G_{i<-(-1)} the prefix
@@ -21,21 +21,21 @@
 // running products and no division, so zero and negative gates need nothing
 // special. Only dS crosses chunks.
 //
-// One CTA takes one (sequence, head, tile of DVT state columns). It first
-// runs the forward over the chunks and stores each chunk's entry state (a
-// checkpoint slot per chunk), then walks the chunks backwards carrying its
-// tile of dS. The columns of S and dS are independent; everything that sums
+// This file holds the pieces one chunk needs (staging, gate products, Grams
+// and the UT solve, Khat S and U, the gradients of a chunk from S, dS_C, U
+// and dR); ckda_bwd_split.cuh composes them into the four programs of the
+// backward. The columns of S and dS are independent; everything that sums
 // over columns (dq, dk, dalpha, dbeta) is linear in per-column terms, so each
-// tile writes fp32 partials that a second kernel adds in tile order.
+// column tile writes fp32 partials that a second kernel adds in tile order.
 //
-// The program is a fixed sequence of data-parallel phases. Executor X runs
+// Every program is a fixed sequence of data-parallel phases. Executor X runs
 // one phase, x.par(n, f): f(i) for every i in [0, n), the calls independent
 // of one another, then a barrier. Every value that outlives a phase sits in
-// the shared-memory block `sm`, so the same source runs as a CUDA kernel
-// (threads stride over i, __syncthreads between phases) and, for tests, as
-// plain host loops. Gate products inside a 16-token chunk are short running
-// products (at most 15 factors), so every factor keeps its sign and its
-// zeros exactly. fp32 throughout.
+// the shared-memory block `sm` (or in global memory), so the same source runs
+// as a CUDA kernel (threads stride over i, __syncthreads between phases) and,
+// for tests, as plain host loops. Gate products inside a 16-token chunk are
+// short running products (at most 15 factors), so every factor keeps its sign
+// and its zeros exactly. fp32 throughout.
 #pragma once
 
 #include <stddef.h>
@@ -56,11 +56,12 @@ namespace bwdc {
 
 constexpr int C = 16;  // tokens per chunk
 
-// Shared-memory layout (floats). Rows are padded to an odd stride so that a
-// warp reading down a column, or along rows indexed by its lanes, touches
-// distinct banks.
+// Shared-memory layout (floats) of the per-chunk gradient program. Rows are
+// padded to an odd stride so that a warp reading down a column, or along rows
+// indexed by its lanes, touches distinct banks.
 template <int DK, int DVT>
 struct Layout {
+  static constexpr int dk = DK, dvt = DVT;
   static constexpr int KS = DK + 1;   // C x DK rows
   static constexpr int VS = DVT + 1;  // C x DVT and DK x DVT rows
   static constexpr int CS = C + 1;    // C x C rows
@@ -69,14 +70,13 @@ struct Layout {
   static constexpr int Q = 0, K = Q + C * KS, AL = K + C * KS, GM = AL + C * KS,
                        SG = GM + C * KS, DQ = SG + C * KS, DKK = DQ + C * KS,
                        E0 = DKK + C * KS, EX = E0 + C * KS;
-  // C x DVT: v, dO, Khat S then w, R then dU, U, dR
-  static constexpr int V = EX + C * KS, DO = V + C * VS, KSW = DO + C * VS, RD = KSW + C * VS,
-                       U = RD + C * VS, DR = U + C * VS;
-  // DK x DVT: the state tile and its gradient
+  // C x DVT: v, dO, Khat S then w, U, dR
+  static constexpr int V = EX + C * KS, DO = V + C * VS, KSW = DO + C * VS, U = KSW + C * VS,
+                       DR = U + C * VS;
+  // DK x DVT: the entry state tile and the exit-state gradient tile
   static constexpr int S = DR + C * VS, DS = S + DK * VS;
-  // C x C: Abar, M, T, dM, dAbar
-  static constexpr int AB = DS + DK * VS, M = AB + C * CS, TT = M + C * CS, DM = TT + C * CS,
-                       DA = DM + C * CS;
+  // C x C: Abar, dM, dAbar
+  static constexpr int AB = DS + DK * VS, DM = AB + C * CS, DA = DM + C * CS;
   static constexpr int BE = DA + C * CS;  // beta [C]
   static constexpr int FLOATS = BE + C;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
@@ -84,7 +84,7 @@ struct Layout {
 
 // Pointers and sizes of one call. Token-major [T_total, H, .] tensors; states
 // [N, H, d_k, d_v]; partials [ntile, T_total H, d_k] (dq, dk, dalpha) and
-// [ntile, T_total H] (dbeta); checkpoints [slots, H, d_k, d_v].
+// [ntile, T_total H] (dbeta).
 template <typename IOT>
 struct Args {
   const IOT *q, *k, *v;
@@ -92,7 +92,7 @@ struct Args {
   const IOT *d_o;
   const float *dsf;
   IOT *dv;
-  float *pq, *pk, *pa, *pb, *ds0, *ck;
+  float *pq, *pk, *pa, *pb, *ds0;
   int H, DVF;   // heads; full d_v (the tiles' columns are c0 .. c0 + DVT - 1)
   size_t TH;    // T_total * H
   float scale;
@@ -100,10 +100,10 @@ struct Args {
 
 // Stage chunk rows [t0, t0 + L) of head h; rows L..C-1 are inert padding
 // (q = k = v = dO = 0, alpha = 1, beta = 0).
-template <class X, class IOL, typename IOT, int DK, int DVT>
+template <class X, class IOL, typename IOT, class Ly>
 CKDA_PROG void stage(X &x, const Args<IOT> &a, float *sm, int h, int c0, int t0, int L,
                      bool with_do) {
-  using Ly = Layout<DK, DVT>;
+  constexpr int DK = Ly::dk, DVT = Ly::dvt;
   constexpr int NW = DK > DVT ? DK : DVT;  // items per row: the wider of d_k and the tile
   x.par(C * NW, [&](int e) {
     const int i = e / NW, c = e - i * NW;
@@ -133,14 +133,11 @@ CKDA_PROG void stage(X &x, const Args<IOT> &a, float *sm, int h, int c0, int t0,
   });
 }
 
-// gamma_i = prod_{s<=i} alpha_s and sigma_j = prod_{s>j} alpha_s per channel;
-// Abar and M; T = (I + diag(beta) Abar)^-1; Khat S, R = diag(beta)(V - Khat S)
-// and U = T R.
-template <class X, int DK, int DVT>
-CKDA_PROG void chunk_forward_parts(X &x, float *sm, bool want_m) {
-  using Ly = Layout<DK, DVT>;
-  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
-  const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q, *be = sm + Ly::BE;
+// gamma_i = prod_{s<=i} alpha_s and sigma_j = prod_{s>j} alpha_s per channel
+template <class X, class Ly>
+CKDA_PROG void chunk_gates(X &x, float *sm) {
+  constexpr int DK = Ly::dk, KS = Ly::KS;
+  const float *al = sm + Ly::AL;
   x.par(DK, [&](int c) {
     float g = 1.f;
     for (int i = 0; i < C; ++i) {
@@ -153,6 +150,13 @@ CKDA_PROG void chunk_forward_parts(X &x, float *sm, bool want_m) {
       g *= al[j * KS + c];
     }
   });
+}
+
+// Abar and M (with M only when want_m); T = (I + diag(beta) Abar)^-1
+template <class X, class Ly>
+CKDA_PROG void chunk_grams_solve(X &x, float *sm, bool want_m) {
+  constexpr int DK = Ly::dk, KS = Ly::KS, CS = Ly::CS;
+  const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q, *be = sm + Ly::BE;
   x.par(C * C, [&](int e) {
     const int i = e / C, j = e - i * C;
     float ab = 0.f, m = 0.f;
@@ -180,19 +184,19 @@ CKDA_PROG void chunk_forward_parts(X &x, float *sm, bool want_m) {
       tt[i * CS + j] = -be[i] * s;
     }
   });
+}
+
+// Khat S (into the Khat S rows)
+template <class X, class Ly>
+CKDA_PROG void chunk_khat_s(X &x, float *sm) {
+  constexpr int DK = Ly::dk, DVT = Ly::dvt, KS = Ly::KS, VS = Ly::VS;
+  const float *kk = sm + Ly::K;
   x.par(C * DVT, [&](int e) {
     const int i = e / DVT, v = e - i * DVT;
     float ks = 0.f;
     for (int c = 0; c < DK; ++c)
       ks += sm[Ly::GM + i * KS + c] * kk[i * KS + c] * sm[Ly::S + c * VS + v];
     sm[Ly::KSW + i * VS + v] = ks;
-    sm[Ly::RD + i * VS + v] = be[i] * (sm[Ly::V + i * VS + v] - ks);
-  });
-  x.par(C * DVT, [&](int e) {
-    const int i = e / DVT, v = e - i * DVT;
-    float u = 0.f;
-    for (int m = 0; m <= i; ++m) u += sm[Ly::TT + i * CS + m] * sm[Ly::RD + m * VS + v];
-    sm[Ly::U + i * VS + v] = u;
   });
 }
 
@@ -234,168 +238,100 @@ CKDA_UNROLL
   }
 }
 
+// The gradients of one chunk from the staged inputs, gamma and sigma, Abar,
+// the entry state S, the exit-state gradient dS_C (in the DS rows), U, dR and
+// Khat S (in the Khat S rows): dv; dbeta, dq, dk and dalpha as this tile's
+// partials. Leaves Khat S replaced by w; S, dS_C, U and dR unchanged.
 template <class X, class IOL, typename IOT, int DK, int DVT>
-CKDA_PROG void bwd_chunk_program(X &x, const Args<IOT> &a, float *sm, int h, int n, int tile,
-                                 int bos, int eos, int slot0) {
+CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile, int t0,
+                            int L) {
   using Ly = Layout<DK, DVT>;
   constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
-  const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
-  const int nck = (eos - bos + C - 1) / C;
-  const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;  // this tile of an [N,H,DK,DVF] state
-  float *S = sm + Ly::S, *DS = sm + Ly::DS;
-
-  // ---- forward over the chunks: a checkpoint of the entry state per chunk
-  x.par(DK * DVT, [&](int e) {
-    const int c = e / DVT, v = e - c * DVT;
-    S[c * VS + v] = a.s0 ? a.s0[st_base + (size_t)c * DVF + v] : 0.f;
+  const int c0 = tile * DVT, H = a.H;
+  const float scale = a.scale;
+  const float *be = sm + Ly::BE;
+  const float *S = sm + Ly::S, *DS = sm + Ly::DS;
+  // w = V - Khat S - Abar U (over the Khat S rows); dv = diag(beta) dR
+  x.par(C * DVT, [&](int e) {
+    const int i = e / DVT, v = e - i * DVT;
+    float s = 0.f;
+    for (int m = 0; m < i; ++m) s += sm[Ly::AB + i * CS + m] * sm[Ly::U + m * VS + v];
+    sm[Ly::KSW + i * VS + v] = sm[Ly::V + i * VS + v] - sm[Ly::KSW + i * VS + v] - s;
+    if (i < L)
+      IOL::st(a.dv + ((size_t)(t0 + i) * H + h) * a.DVF + c0 + v,
+              be[i] * sm[Ly::DR + i * VS + v]);
   });
-  for (int ci = 0; ci < nck; ++ci) {
-    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
-    float *cp = a.ck + ((size_t)(slot0 + ci) * H + h) * DK * DVF + c0;
-    x.par(DK * DVT, [&](int e) {
-      const int c = e / DVT, v = e - c * DVT;
-      cp[(size_t)c * DVF + v] = S[c * VS + v];
-    });
-    stage<X, IOL, IOT, DK, DVT>(x, a, sm, h, c0, t0, L, false);
-    chunk_forward_parts<X, DK, DVT>(x, sm, false);
-    x.par(DK * DVT, [&](int e) {  // S <- diag(gamma_{C-1}) S + Kbar^T U
-      const int c = e / DVT, v = e - c * DVT;
-      float s = sm[Ly::GM + (C - 1) * KS + c] * S[c * VS + v];
-      for (int i = 0; i < C; ++i)
-        s += sm[Ly::SG + i * KS + c] * sm[Ly::K + i * KS + c] * sm[Ly::U + i * VS + v];
-      S[c * VS + v] = s;
-    });
-  }
-
-  // ---- the chunks in reverse, carrying dS
-  x.par(DK * DVT, [&](int e) {
-    const int c = e / DVT, v = e - c * DVT;
-    DS[c * VS + v] = a.dsf ? a.dsf[st_base + (size_t)c * DVF + v] : 0.f;
-  });
-  for (int ci = nck - 1; ci >= 0; --ci) {
-    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
-    const float *cp = a.ck + ((size_t)(slot0 + ci) * H + h) * DK * DVF + c0;
-    x.par(DK * DVT, [&](int e) {
-      const int c = e / DVT, v = e - c * DVT;
-      S[c * VS + v] = cp[(size_t)c * DVF + v];
-    });
-    stage<X, IOL, IOT, DK, DVT>(x, a, sm, h, c0, t0, L, true);
-    chunk_forward_parts<X, DK, DVT>(x, sm, true);
-    const float scale = a.scale;
-    const float *be = sm + Ly::BE;
-    // dU = scale M^T dO + Kbar dS_C (into the R rows, no longer needed)
-    x.par(C * DVT, [&](int e) {
-      const int j = e / DVT, v = e - j * DVT;
+  // dbeta (this tile's share); dM and dAbar
+  x.par(C * C, [&](int e) {
+    const int i = e / C, j = e - i * C;
+    if (j == 0 && i < L) {
       float s = 0.f;
-      for (int i = j; i < C; ++i) s += sm[Ly::M + i * CS + j] * sm[Ly::DO + i * VS + v];
-      float t = 0.f;
-      for (int c = 0; c < DK; ++c)
-        t += sm[Ly::SG + j * KS + c] * sm[Ly::K + j * KS + c] * DS[c * VS + v];
-      sm[Ly::RD + j * VS + v] = scale * s + t;
-    });
-    // dR = T^T dU; dv = diag(beta) dR
-    x.par(C * DVT, [&](int e) {
-      const int j = e / DVT, v = e - j * DVT;
-      float s = 0.f;
-      for (int i = j; i < C; ++i) s += sm[Ly::TT + i * CS + j] * sm[Ly::RD + i * VS + v];
-      sm[Ly::DR + j * VS + v] = s;
-      if (j < L)
-        IOL::st(a.dv + ((size_t)(t0 + j) * H + h) * DVF + c0 + v, be[j] * s);
-    });
-    // w = V - Khat S - Abar U (over the Khat S rows)
-    x.par(C * DVT, [&](int e) {
-      const int i = e / DVT, v = e - i * DVT;
-      float s = 0.f;
-      for (int m = 0; m < i; ++m) s += sm[Ly::AB + i * CS + m] * sm[Ly::U + m * VS + v];
-      sm[Ly::KSW + i * VS + v] = sm[Ly::V + i * VS + v] - sm[Ly::KSW + i * VS + v] - s;
-    });
-    // dbeta (this tile's share); dM and dAbar
-    x.par(C * C, [&](int e) {
-      const int i = e / C, j = e - i * C;
-      if (j == 0 && i < L) {
-        float s = 0.f;
-        for (int v = 0; v < DVT; ++v) s += sm[Ly::DR + i * VS + v] * sm[Ly::KSW + i * VS + v];
-        a.pb[(size_t)tile * a.TH + (size_t)(t0 + i) * H + h] = s;
-      }
-      float m = 0.f, d = 0.f;
-      if (j <= i) {
-        for (int v = 0; v < DVT; ++v) {
-          const float u = sm[Ly::U + j * VS + v];
-          m += sm[Ly::DO + i * VS + v] * u;
-          d += sm[Ly::DR + i * VS + v] * u;
-        }
-      }
-      sm[Ly::DM + i * CS + j] = scale * m;
-      sm[Ly::DA + i * CS + j] = j < i ? -be[i] * d : 0.f;
-    });
-    // the state-side terms: dQhat = scale dO S^T, dKhat = -diag(beta) dR S^T,
-    // dKbar = U dS_C^T; dq and dk start from them, E0 and EX keep the gate parts
-    x.par(C * DK, [&](int e) {
-      const int i = e / DK, c = e - i * DK;
-      float xq = 0.f, xk = 0.f, xb = 0.f;
+      for (int v = 0; v < DVT; ++v) s += sm[Ly::DR + i * VS + v] * sm[Ly::KSW + i * VS + v];
+      a.pb[(size_t)tile * a.TH + (size_t)(t0 + i) * H + h] = s;
+    }
+    float m = 0.f, d = 0.f;
+    if (j <= i) {
       for (int v = 0; v < DVT; ++v) {
-        const float s = S[c * VS + v];
-        xq += sm[Ly::DO + i * VS + v] * s;
-        xk += sm[Ly::DR + i * VS + v] * s;
-        xb += sm[Ly::U + i * VS + v] * DS[c * VS + v];
+        const float u = sm[Ly::U + j * VS + v];
+        m += sm[Ly::DO + i * VS + v] * u;
+        d += sm[Ly::DR + i * VS + v] * u;
       }
-      const float dqh = scale * xq, dkh = -be[i] * xk;
-      const float gm = sm[Ly::GM + i * KS + c], sg = sm[Ly::SG + i * KS + c];
-      sm[Ly::DQ + i * KS + c] = gm * dqh;
-      sm[Ly::DKK + i * KS + c] = gm * dkh + sg * xb;
-      sm[Ly::E0 + i * KS + c] = sm[Ly::Q + i * KS + c] * dqh + sm[Ly::K + i * KS + c] * dkh;
-      sm[Ly::EX + i * KS + c] = sm[Ly::K + i * KS + c] * xb;
-    });
-    // gated Gram terms of dq and dk; write this tile's dq, dk partials
-    x.par(C * DK, [&](int e) {
-      const int r = e / DK, c = e - r * DK;
-      const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
-      float dq = sm[Ly::DQ + r * KS + c], dk = sm[Ly::DKK + r * KS + c];
-      float g = 1.f;  // G_{r<-j}
-      dq += sm[Ly::DM + r * CS + r] * kk[r * KS + c];
-      for (int j = r - 1; j >= 0; --j) {
-        g *= al[(j + 1) * KS + c];
-        const float gk = g * kk[j * KS + c];
-        dq += sm[Ly::DM + r * CS + j] * gk;
-        dk += sm[Ly::DA + r * CS + j] * gk;
-      }
-      g = 1.f;  // G_{i<-r}
-      for (int i = r; i < C; ++i) {
-        if (i > r) g *= al[i * KS + c];
-        dk += g * (sm[Ly::DM + i * CS + r] * qq[i * KS + c] + sm[Ly::DA + i * CS + r] * kk[i * KS + c]);
-      }
-      if (r < L) {
-        const size_t pi = ((size_t)tile * a.TH + (size_t)(t0 + r) * H + h) * DK + c;
-        a.pq[pi] = dq;
-        a.pk[pi] = dk;
-      }
-    });
-    // dalpha (this tile's share), one channel per item
-    x.par(DK, [&](int c) {
-      float sds = 0.f;
-      for (int v = 0; v < DVT; ++v) sds += S[c * VS + v] * DS[c * VS + v];
-      float da[C];
-      gate_grad_channel<DK, DVT>(sm, c, sds, da);
-      for (int i = 0; i < L; ++i)
-        a.pa[((size_t)tile * a.TH + (size_t)(t0 + i) * H + h) * DK + c] = da[i];
-    });
-    // dS <- scale Qhat^T dO + diag(gamma_{C-1}) dS - Khat^T diag(beta) dR
-    x.par(DK * DVT, [&](int e) {
-      const int c = e / DVT, v = e - c * DVT;
-      float s = sm[Ly::GM + (C - 1) * KS + c] * DS[c * VS + v];
-      for (int i = 0; i < C; ++i)
-        s += sm[Ly::GM + i * KS + c] *
-             (scale * sm[Ly::Q + i * KS + c] * sm[Ly::DO + i * VS + v] -
-              be[i] * sm[Ly::K + i * KS + c] * sm[Ly::DR + i * VS + v]);
-      DS[c * VS + v] = s;
-    });
-  }
-  if (a.ds0) {
-    x.par(DK * DVT, [&](int e) {
-      const int c = e / DVT, v = e - c * DVT;
-      a.ds0[st_base + (size_t)c * DVF + v] = DS[c * VS + v];
-    });
-  }
+    }
+    sm[Ly::DM + i * CS + j] = scale * m;
+    sm[Ly::DA + i * CS + j] = j < i ? -be[i] * d : 0.f;
+  });
+  // the state-side terms: dQhat = scale dO S^T, dKhat = -diag(beta) dR S^T,
+  // dKbar = U dS_C^T; dq and dk start from them, E0 and EX keep the gate parts
+  x.par(C * DK, [&](int e) {
+    const int i = e / DK, c = e - i * DK;
+    float xq = 0.f, xk = 0.f, xb = 0.f;
+    for (int v = 0; v < DVT; ++v) {
+      const float s = S[c * VS + v];
+      xq += sm[Ly::DO + i * VS + v] * s;
+      xk += sm[Ly::DR + i * VS + v] * s;
+      xb += sm[Ly::U + i * VS + v] * DS[c * VS + v];
+    }
+    const float dqh = scale * xq, dkh = -be[i] * xk;
+    const float gm = sm[Ly::GM + i * KS + c], sg = sm[Ly::SG + i * KS + c];
+    sm[Ly::DQ + i * KS + c] = gm * dqh;
+    sm[Ly::DKK + i * KS + c] = gm * dkh + sg * xb;
+    sm[Ly::E0 + i * KS + c] = sm[Ly::Q + i * KS + c] * dqh + sm[Ly::K + i * KS + c] * dkh;
+    sm[Ly::EX + i * KS + c] = sm[Ly::K + i * KS + c] * xb;
+  });
+  // gated Gram terms of dq and dk; write this tile's dq, dk partials
+  x.par(C * DK, [&](int e) {
+    const int r = e / DK, c = e - r * DK;
+    const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
+    float dq = sm[Ly::DQ + r * KS + c], dk = sm[Ly::DKK + r * KS + c];
+    float g = 1.f;  // G_{r<-j}
+    dq += sm[Ly::DM + r * CS + r] * kk[r * KS + c];
+    for (int j = r - 1; j >= 0; --j) {
+      g *= al[(j + 1) * KS + c];
+      const float gk = g * kk[j * KS + c];
+      dq += sm[Ly::DM + r * CS + j] * gk;
+      dk += sm[Ly::DA + r * CS + j] * gk;
+    }
+    g = 1.f;  // G_{i<-r}
+    for (int i = r; i < C; ++i) {
+      if (i > r) g *= al[i * KS + c];
+      dk += g * (sm[Ly::DM + i * CS + r] * qq[i * KS + c] + sm[Ly::DA + i * CS + r] * kk[i * KS + c]);
+    }
+    if (r < L) {
+      const size_t pi = ((size_t)tile * a.TH + (size_t)(t0 + r) * H + h) * DK + c;
+      a.pq[pi] = dq;
+      a.pk[pi] = dk;
+    }
+  });
+  // dalpha (this tile's share), one channel per item
+  x.par(DK, [&](int c) {
+    float sds = 0.f;
+    for (int v = 0; v < DVT; ++v) sds += S[c * VS + v] * DS[c * VS + v];
+    float da[C];
+    gate_grad_channel<DK, DVT>(sm, c, sds, da);
+CKDA_UNROLL
+    for (int i = 0; i < C; ++i)  // static indices keep da in registers
+      if (i < L) a.pa[((size_t)tile * a.TH + (size_t)(t0 + i) * H + h) * DK + c] = da[i];
+  });
 }
 
 }  // namespace bwdc

@@ -1,0 +1,265 @@
+// The chunkwise backward pass, split by what depends on the carried state.
+//
+// Built from the per-chunk pieces of ckda_bwd_chunk.cuh (the chunk-WY reverse
+// of "Semidirect Fourier Delta Attention" §2.2 eqs. (9)-(10) in 16-token
+// chunks): the work that does not depend on S or dS runs in CTAs of its own,
+// in parallel over all chunks, and the two sequential scans keep only their
+// state products. With T = (I + diag(beta) Abar)^-1 and per chunk
+//   W = T diag(beta) Khat,  Utilde = T diag(beta) V,  Kbar = sigma * k,
+//   Wb = T^T Kbar,  X = T^T (scale M^T dO),  Qs = scale Qhat,  BK = diag(beta) Khat,
+// the forward over chunks is S <- diag(gamma_C) S + Kbar^T U with
+// U = Utilde - W S, and the reverse is dR = X + Wb dS_C,
+// dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR. Four programs:
+//   prep   (per chunk and head)            the factors above, Abar, gamma_C;
+//   scan1  (per sequence, head, col. tile) entry states S per chunk, and U;
+//   scan2  (per sequence, head, col. tile) exit-state gradients dS_C, and dR;
+//   grads  (per chunk, head, col. tile)    chunk_grads from (S, dS_C, U, dR).
+// Per-chunk values (S, dS_C, gamma_C, Abar) sit in checkpoint slots
+// (slot = floor(cu[n] / C) + n + chunk, at most floor(T_total / C) + N
+// slots); per-token values in token-major [T_total, H, .] fp32 arrays.
+#pragma once
+
+#include "ckda_bwd_chunk.cuh"
+
+namespace ckda {
+namespace bwdc {
+
+// Workspace arrays of the split form (all fp32).
+struct SplitWs {
+  float *cks, *ckd;              // [slots][H][DK][DVF]: S entering, dS leaving each chunk
+  float *gc;                     // [slots][H][DK]: gamma over the whole chunk
+  float *ab;                     // [slots][H][C][C]: Abar
+  float *wt, *kb, *wb, *qs, *bk; // [T_total H][DK]: W, Kbar, Wb, Qs, BK
+  float *ut, *xt, *uu, *dr;      // [T_total H][DVF]: Utilde, X, U, dR
+};
+
+// Sequence n and chunk ci of checkpoint slot g (slots of sequence n start at
+// floor(start_n / C) + n); false when no sequence starts a chunk there.
+CKDA_PROG bool slot_chunk(const int32_t *cu, int N, int T, int g, int &n, int &ci) {
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) / 2;
+    const int b = cu ? cu[mid] : mid * T;
+    if (b / C + mid <= g) lo = mid; else hi = mid - 1;
+  }
+  const int b = cu ? cu[lo] : lo * T;
+  n = lo;
+  ci = g - (b / C + lo);
+  return ci >= 0;
+}
+
+// Prep works on one (chunk, head) for all of d_v, one DVT tile of v and dO at a time.
+template <int DK, int DVT>
+struct PrepLayout {
+  static constexpr int dk = DK, dvt = DVT;
+  static constexpr int KS = DK + 1, VS = DVT + 1, CS = C + 1;
+  static constexpr int Q = 0, K = Q + C * KS, AL = K + C * KS, GM = AL + C * KS,
+                       SG = GM + C * KS;
+  static constexpr int V = SG + C * KS, DO = V + C * VS, RD = DO + C * VS;
+  static constexpr int AB = RD + C * VS, M = AB + C * CS, TT = M + C * CS;
+  static constexpr int BE = TT + C * CS;
+  static constexpr int FLOATS = BE + C;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+template <class X, class IOL, typename IOT, int DK, int DVT>
+CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
+                            int t0, int L, int slot) {
+  using Ly = PrepLayout<DK, DVT>;
+  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
+  const int H = a.H, DVF = a.DVF;
+  const float scale = a.scale;
+  const float *be = sm + Ly::BE, *tt = sm + Ly::TT;
+  stage<X, IOL, IOT, Ly>(x, a, sm, h, 0, t0, L, true);
+  chunk_gates<X, Ly>(x, sm);
+  chunk_grams_solve<X, Ly>(x, sm, true);
+  // the d_k-wide factors, gamma_C and Abar
+  x.par(C * DK, [&](int e) {
+    const int i = e / DK, c = e - i * DK;
+    if (e < DK) w.gc[((size_t)slot * H + h) * DK + c] = sm[Ly::GM + (C - 1) * KS + c];
+    if (e < C * C) w.ab[((size_t)slot * H + h) * C * C + e] = sm[Ly::AB + (e / C) * CS + e % C];
+    if (i >= L) return;
+    float wt = 0.f, wb = 0.f;
+    for (int m = 0; m <= i; ++m)
+      wt += tt[i * CS + m] * be[m] * sm[Ly::GM + m * KS + c] * sm[Ly::K + m * KS + c];
+    for (int j = i; j < C; ++j)
+      wb += tt[j * CS + i] * sm[Ly::SG + j * KS + c] * sm[Ly::K + j * KS + c];
+    const float gm = sm[Ly::GM + i * KS + c], kc = sm[Ly::K + i * KS + c];
+    const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
+    w.wt[o] = wt;
+    w.kb[o] = sm[Ly::SG + i * KS + c] * kc;
+    w.wb[o] = wb;
+    w.qs[o] = scale * gm * sm[Ly::Q + i * KS + c];
+    w.bk[o] = be[i] * gm * kc;
+  });
+  // Utilde = T diag(beta) V and X = T^T (scale M^T dO), one column tile at a time
+  for (int c0 = 0; c0 < DVF; c0 += DVT) {
+    if (c0 > 0) {
+      x.par(C * DVT, [&](int e) {
+        const int i = e / DVT, v = e - i * DVT;
+        float vv = 0.f, dd = 0.f;
+        if (i < L) {
+          const size_t g = ((size_t)(t0 + i) * H + h) * DVF + c0 + v;
+          vv = IOL::ld(a.v + g);
+          dd = IOL::ld(a.d_o + g);
+        }
+        sm[Ly::V + i * VS + v] = vv;
+        sm[Ly::DO + i * VS + v] = dd;
+      });
+    }
+    x.par(C * DVT, [&](int e) {  // Utilde; Y = scale M^T dO into the R rows
+      const int i = e / DVT, v = e - i * DVT;
+      float u = 0.f, y = 0.f;
+      for (int m = 0; m <= i; ++m) u += tt[i * CS + m] * be[m] * sm[Ly::V + m * VS + v];
+      for (int l = i; l < C; ++l) y += sm[Ly::M + l * CS + i] * sm[Ly::DO + l * VS + v];
+      sm[Ly::RD + i * VS + v] = scale * y;
+      if (i < L) w.ut[((size_t)(t0 + i) * H + h) * DVF + c0 + v] = u;
+    });
+    x.par(C * DVT, [&](int e) {  // X = T^T Y
+      const int j = e / DVT, v = e - j * DVT;
+      float s = 0.f;
+      for (int i = j; i < C; ++i) s += tt[i * CS + j] * sm[Ly::RD + i * VS + v];
+      if (j < L) w.xt[((size_t)(t0 + j) * H + h) * DVF + c0 + v] = s;
+    });
+  }
+}
+
+// Shared memory of the two scans: one state (or state gradient) tile and the
+// chunk's per-token factors.
+template <int DK, int DVT>
+struct ScanLayout {
+  static constexpr int KS = DK + 1, VS = DVT + 1;
+  static constexpr int S = 0, F0 = S + DK * VS, F1 = F0 + C * KS, F2 = F1 + C * KS,
+                       R0 = F2 + C * KS, R1 = R0 + C * VS, GC = R1 + C * VS;
+  static constexpr int FLOATS = GC + DK;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+// rows [t0, t0 + L) of a token-major [T_total H][width] array into C padded rows
+template <class X>
+CKDA_PROG void load_rows(X &x, float *dst, int stride, const float *src, int width, int col0,
+                         int ncol, int t0, int L, int H, int h) {
+  x.par(C * ncol, [&](int e) {
+    const int i = e / ncol, c = e - i * ncol;
+    dst[i * stride + c] = i < L ? src[((size_t)(t0 + i) * H + h) * width + col0 + c] : 0.f;
+  });
+}
+
+template <class X, class IOL, typename IOT, int DK, int DVT>
+CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
+                             int n, int tile, int bos, int eos, int slot0) {
+  using Ly = ScanLayout<DK, DVT>;
+  constexpr int KS = Ly::KS, VS = Ly::VS;
+  const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
+  const int nck = (eos - bos + C - 1) / C;
+  const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
+  float *S = sm + Ly::S, *WT = sm + Ly::F0, *KB = sm + Ly::F1, *U = sm + Ly::R0;
+  float *GC = sm + Ly::GC;
+  x.par(DK * DVT, [&](int e) {
+    const int c = e / DVT, v = e - c * DVT;
+    S[c * VS + v] = a.s0 ? a.s0[st_base + (size_t)c * DVF + v] : 0.f;
+  });
+  for (int ci = 0; ci < nck; ++ci) {
+    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
+    const size_t slot = (size_t)(slot0 + ci) * H + h;
+    x.par(DK * DVT, [&](int e) {
+      const int c = e / DVT, v = e - c * DVT;
+      w.cks[slot * DK * DVF + (size_t)c * DVF + c0 + v] = S[c * VS + v];
+      if (e < DK) GC[e] = w.gc[slot * DK + e];
+    });
+    load_rows(x, WT, KS, w.wt, DK, 0, DK, t0, L, H, h);
+    load_rows(x, KB, KS, w.kb, DK, 0, DK, t0, L, H, h);
+    load_rows(x, U, VS, w.ut, DVF, c0, DVT, t0, L, H, h);
+    x.par(C * DVT, [&](int e) {  // U = Utilde - W S
+      const int i = e / DVT, v = e - i * DVT;
+      float s = U[i * VS + v];
+      for (int c = 0; c < DK; ++c) s -= WT[i * KS + c] * S[c * VS + v];
+      U[i * VS + v] = s;
+      if (i < L) w.uu[((size_t)(t0 + i) * H + h) * DVF + c0 + v] = s;
+    });
+    x.par(DK * DVT, [&](int e) {  // S <- diag(gamma_C) S + Kbar^T U
+      const int c = e / DVT, v = e - c * DVT;
+      float s = GC[c] * S[c * VS + v];
+      for (int i = 0; i < C; ++i) s += KB[i * KS + c] * U[i * VS + v];
+      S[c * VS + v] = s;
+    });
+  }
+}
+
+template <class X, class IOL, typename IOT, int DK, int DVT>
+CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
+                             int n, int tile, int bos, int eos, int slot0) {
+  using Ly = ScanLayout<DK, DVT>;
+  constexpr int KS = Ly::KS, VS = Ly::VS;
+  const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
+  const int nck = (eos - bos + C - 1) / C;
+  const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
+  float *DS = sm + Ly::S, *WB = sm + Ly::F0, *QS = sm + Ly::F1, *BK = sm + Ly::F2;
+  float *DR = sm + Ly::R0, *DO = sm + Ly::R1, *GC = sm + Ly::GC;
+  x.par(DK * DVT, [&](int e) {
+    const int c = e / DVT, v = e - c * DVT;
+    DS[c * VS + v] = a.dsf ? a.dsf[st_base + (size_t)c * DVF + v] : 0.f;
+  });
+  for (int ci = nck - 1; ci >= 0; --ci) {
+    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
+    const size_t slot = (size_t)(slot0 + ci) * H + h;
+    x.par(DK * DVT, [&](int e) {
+      const int c = e / DVT, v = e - c * DVT;
+      w.ckd[slot * DK * DVF + (size_t)c * DVF + c0 + v] = DS[c * VS + v];
+      if (e < DK) GC[e] = w.gc[slot * DK + e];
+    });
+    load_rows(x, WB, KS, w.wb, DK, 0, DK, t0, L, H, h);
+    load_rows(x, QS, KS, w.qs, DK, 0, DK, t0, L, H, h);
+    load_rows(x, BK, KS, w.bk, DK, 0, DK, t0, L, H, h);
+    load_rows(x, DR, VS, w.xt, DVF, c0, DVT, t0, L, H, h);
+    x.par(C * DVT, [&](int e) {
+      const int i = e / DVT, v = e - i * DVT;
+      DO[i * VS + v] = i < L ? IOL::ld(a.d_o + ((size_t)(t0 + i) * H + h) * DVF + c0 + v) : 0.f;
+    });
+    x.par(C * DVT, [&](int e) {  // dR = X + Wb dS_C
+      const int j = e / DVT, v = e - j * DVT;
+      float s = DR[j * VS + v];
+      for (int c = 0; c < DK; ++c) s += WB[j * KS + c] * DS[c * VS + v];
+      DR[j * VS + v] = s;
+      if (j < L) w.dr[((size_t)(t0 + j) * H + h) * DVF + c0 + v] = s;
+    });
+    x.par(DK * DVT, [&](int e) {  // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
+      const int c = e / DVT, v = e - c * DVT;
+      float s = GC[c] * DS[c * VS + v];
+      for (int i = 0; i < C; ++i) s += QS[i * KS + c] * DO[i * VS + v] - BK[i * KS + c] * DR[i * VS + v];
+      DS[c * VS + v] = s;
+    });
+  }
+  if (a.ds0) {
+    x.par(DK * DVT, [&](int e) {
+      const int c = e / DVT, v = e - c * DVT;
+      a.ds0[st_base + (size_t)c * DVF + v] = DS[c * VS + v];
+    });
+  }
+}
+
+// The gradients of one (chunk, head, column tile) from the scans' outputs.
+template <class X, class IOL, typename IOT, int DK, int DVT>
+CKDA_PROG void grads_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
+                             int tile, int t0, int L, int slot) {
+  using Ly = Layout<DK, DVT>;
+  constexpr int VS = Ly::VS, CS = Ly::CS;
+  const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
+  const size_t sl = (size_t)slot * H + h;
+  stage<X, IOL, IOT, Ly>(x, a, sm, h, c0, t0, L, true);
+  chunk_gates<X, Ly>(x, sm);
+  x.par(DK * DVT, [&](int e) {
+    const int c = e / DVT, v = e - c * DVT;
+    const size_t o = sl * DK * DVF + (size_t)c * DVF + c0 + v;
+    sm[Ly::S + c * VS + v] = w.cks[o];
+    sm[Ly::DS + c * VS + v] = w.ckd[o];
+    if (e < C * C) sm[Ly::AB + (e / C) * CS + e % C] = w.ab[sl * C * C + e];
+  });
+  load_rows(x, sm + Ly::U, VS, w.uu, DVF, c0, DVT, t0, L, H, h);
+  load_rows(x, sm + Ly::DR, VS, w.dr, DVF, c0, DVT, t0, L, H, h);
+  chunk_khat_s<X, Ly>(x, sm);
+  chunk_grads<X, IOL, IOT, DK, DVT>(x, a, sm, h, tile, t0, L);
+}
+
+}  // namespace bwdc
+}  // namespace ckda

@@ -273,17 +273,23 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
 
 /*
  * ckda_bwd_chunked: the gradients of ckda_bwd (the same arguments, layouts,
- * workspace query, errors and outputs) computed 16 tokens at a time in the
- * chunk-WY form of the forward ("Semidirect Fourier Delta Attention" §2.2
- * eqs. (9)-(10)) run in reverse: per chunk, dU = scale M^T dO + Kbar dS_C,
- * dR = T^T dU, dv = diag(beta) dR, then dq, dk, dbeta from matrix products and
- * the gated Gram terms, and dalpha per channel as the gate product with the
- * one factor alpha_s left out (two running products, no logarithm and no
- * division, so zero and negative gates are exact). Only the d_k x d_v state
- * gradient dS = scale Qhat^T dO + diag(gamma) dS_C - Khat^T diag(beta) dR
- * passes from chunk to chunk. One CTA per (sequence, head, tile of up to 32
- * state columns), fp32 arithmetic on CUDA cores, deterministic (tile partials
- * added in a fixed order).
+ * errors and outputs) computed 16 tokens at a time in the chunk-WY form of the
+ * forward ("Semidirect Fourier Delta Attention" §2.2 eqs. (9)-(10)) run in
+ * reverse: per chunk, dU = scale M^T dO + Kbar dS_C, dR = T^T dU,
+ * dv = diag(beta) dR, then dq, dk, dbeta from matrix products and the gated
+ * Gram terms, and dalpha per channel as the gate product with the one factor
+ * alpha_s left out (two running products, no logarithm and no division, so
+ * zero and negative gates are exact). Only the d_k x d_v state gradient
+ * dS = scale Qhat^T dO + diag(gamma) dS_C - Khat^T diag(beta) dR passes from
+ * chunk to chunk. Four kernels: a prep over all chunks, a forward scan and a
+ * reverse scan per (sequence, head, tile of up to 32 state columns) that
+ * carry only the state products, and the per-chunk gradients over all
+ * chunks; then the tiles' partials are added in a fixed order. fp32
+ * arithmetic on CUDA cores, deterministic.
+ *   workspace   device scratch of at least ckda_bwd_chunked_workspace_bytes()
+ *               bytes, owned by the caller (one entry state and one exit-state
+ *               gradient per 16-token chunk, the chunks' factors, the tiles'
+ *               partials); required when N > 0.
  */
 ckda_status ckda_bwd_chunked(const void *q, const void *k, const void *v, const float *alpha,
                              const float *beta, const float *initial_state, const void *d_o,
@@ -320,13 +326,15 @@ ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const 
                              int32_t d_k, int32_t d_v, float scale, cudaStream_t stream);
 
 /*
- * ckda_bwd_workspace_bytes: scratch ckda_bwd and ckda_bwd_chunked need (T as
- * in ckda_bwd; varlen
- * nonzero when cu_seqlens is given, so that T is total_T). 0 for unsupported
- * or invalid sizes.
+ * ckda_bwd_workspace_bytes, ckda_bwd_chunked_workspace_bytes: scratch that
+ * ckda_bwd and ckda_bwd_chunked need (T as in ckda_bwd; varlen nonzero when
+ * cu_seqlens is given, so that T is total_T). 0 for unsupported or invalid
+ * sizes.
  */
 size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
                                 int32_t d_v, int32_t varlen);
+size_t ckda_bwd_chunked_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                        int32_t d_v, int32_t varlen);
 
 /* Static description of a status code (never NULL). */
 const char *ckda_status_string(ckda_status s);

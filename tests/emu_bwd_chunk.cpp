@@ -1,9 +1,10 @@
-// Test-only host build of the chunkwise backward's per-CTA program
-// (csrc/ckda_bwd_chunk.cuh): every CTA of the launch grid runs in turn, each
-// phase as a plain loop over its work items, which is the same set of calls
-// the GPU makes between two barriers. It checks the program's index
-// arithmetic and algebra on the CPU (built with AddressSanitizer by the
-// test); it is not a product path and no library calls it.
+// Test-only host build of the chunkwise backward's per-CTA programs
+// (csrc/ckda_bwd_split.cuh): every CTA of each of the four launch grids runs
+// in turn, the launches in their stream order, each phase as a plain loop over
+// its work items, which is the same set of calls the GPU makes between two
+// barriers. It checks the programs' index arithmetic and algebra on the
+// CPU (built with AddressSanitizer by the test, every workspace piece its own
+// allocation); it is not a product path and no library calls it.
 //
 // usage: emu_bwd_chunk DIR N T H d_k d_v scale varlen has_s0 has_dsf
 // DIR holds float32 q k v alpha beta do [s0] [dsf] and int32 cu (varlen) as
@@ -13,7 +14,7 @@
 #include <string>
 #include <vector>
 
-#include "ckda_bwd_chunk.cuh"
+#include "ckda_bwd_split.cuh"
 
 namespace {
 
@@ -68,22 +69,62 @@ void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool 
   if (has_dsf) dsf = load(dir + "/dsf.bin", st);
   const int ntile = DV / DVT;
   const size_t slots = (size_t)T_total / C + N;
-  std::vector<float> ck(slots * H * DK * DV), dv(TH * DV), ds0(st);
+  std::vector<float> dv(TH * DV), ds0(st);
   std::vector<float> pq(ntile * TH * DK), pk(ntile * TH * DK), pa(ntile * TH * DK),
       pb(ntile * TH);
   Args<float> a{q.data(), k.data(), v.data(), al.data(), be.data(),
                 has_s0 ? s0.data() : nullptr, d_o.data(), has_dsf ? dsf.data() : nullptr,
-                dv.data(), pq.data(), pk.data(), pa.data(), pb.data(), ds0.data(),
-                ck.data(), H, DV, TH, scale};
-  std::vector<float> sm(Layout<DK, DVT>::FLOATS);
+                dv.data(), pq.data(), pk.data(), pa.data(), pb.data(), ds0.data(), H, DV, TH,
+                scale};
   HostExec x;
-  for (int tile = 0; tile < ntile; ++tile)
-    for (int n = 0; n < N; ++n)
-      for (int h = 0; h < H; ++h) {
-        const int bos = varlen ? cu[n] : n * T, eos = varlen ? cu[n + 1] : bos + T;
-        bwd_chunk_program<HostExec, HostIO, float, DK, DVT>(x, a, sm.data(), h, n, tile, bos,
-                                                           eos, bos / C + n);
-      }
+  auto bounds = [&](int n, int &bos, int &eos) {
+    bos = varlen ? cu[n] : n * T;
+    eos = varlen ? cu[n + 1] : bos + T;
+  };
+  {
+    const size_t sl = slots * H;
+    std::vector<float> cks(sl * DK * DV), ckd(sl * DK * DV), gc(sl * DK), ab(sl * C * C);
+    std::vector<float> wt(TH * DK), kb(TH * DK), wb(TH * DK), qs(TH * DK), bk(TH * DK);
+    std::vector<float> ut(TH * DV), xt(TH * DV), uu(TH * DV), dr(TH * DV);
+    SplitWs w{cks.data(), ckd.data(), gc.data(), ab.data(), wt.data(), kb.data(), wb.data(),
+              qs.data(), bk.data(), ut.data(), xt.data(), uu.data(), dr.data()};
+    // the chunk of slot g, as the kernels find it
+    auto slot_rows = [&](int g, int &t0, int &L) {
+      int n, ci, bos, eos;
+      if (!slot_chunk(varlen ? cu.data() : nullptr, N, T, g, n, ci)) return false;
+      bounds(n, bos, eos);
+      if (ci >= (eos - bos + C - 1) / C) return false;
+      t0 = bos + C * ci;
+      L = eos - t0 < C ? eos - t0 : C;
+      return true;
+    };
+    std::vector<float> psm(PrepLayout<DK, DVT>::FLOATS), ssm(ScanLayout<DK, DVT>::FLOATS),
+        gsm(Layout<DK, DVT>::FLOATS);
+    int t0, L;
+    for (int h = 0; h < H; ++h)
+      for (int g = 0; g < (int)slots; ++g)
+        if (slot_rows(g, t0, L))
+          prep_program<HostExec, HostIO, float, DK, DVT>(x, a, w, psm.data(), h, t0, L, g);
+    for (int pass = 0; pass < 2; ++pass)
+      for (int tile = 0; tile < ntile; ++tile)
+        for (int n = 0; n < N; ++n)
+          for (int h = 0; h < H; ++h) {
+            int bos, eos;
+            bounds(n, bos, eos);
+            if (pass == 0)
+              scan1_program<HostExec, HostIO, float, DK, DVT>(x, a, w, ssm.data(), h, n, tile,
+                                                             bos, eos, bos / C + n);
+            else
+              scan2_program<HostExec, HostIO, float, DK, DVT>(x, a, w, ssm.data(), h, n, tile,
+                                                             bos, eos, bos / C + n);
+          }
+    for (int tile = 0; tile < ntile; ++tile)
+      for (int h = 0; h < H; ++h)
+        for (int g = 0; g < (int)slots; ++g)
+          if (slot_rows(g, t0, L))
+            grads_program<HostExec, HostIO, float, DK, DVT>(x, a, w, gsm.data(), h, tile, t0, L,
+                                                           g);
+  }
   std::vector<float> dq(TH * DK), dk(TH * DK), da(TH * DK), db(TH);
   for (size_t i = 0; i < TH * DK; ++i)
     for (int t = 0; t < ntile; ++t) {

@@ -1,10 +1,11 @@
-"""The chunkwise backward's per-CTA program (csrc/ckda_bwd_chunk.cuh), run
-on the CPU through its host executor (emu_bwd_chunk.cpp, built here with
-AddressSanitizer and UBSan), against the oracle's fp64 adjoint.
+"""The chunkwise backward's four per-CTA programs (csrc/ckda_bwd_split.cuh,
+built from the pieces of csrc/ckda_bwd_chunk.cuh), run on the CPU through
+their host executor (emu_bwd_chunk.cpp, built here with AddressSanitizer and
+UBSan), against the oracle's fp64 adjoint.
 
-This checks the program's algebra and its index arithmetic (chunks, ragged
-and empty sequences, column tiles, checkpoint slots, partials) before the
-kernel runs on a GPU; it is not a GPU parity claim. Cases and the fp32 bound
+This checks the programs' algebra and index arithmetic (chunks, ragged and
+empty sequences, column tiles, checkpoint slots, the slot-to-chunk search,
+partials) before the kernels run on a GPU; it is not a GPU parity claim. Cases and the fp32 bound
 (BWD_FP32_REL * rms of the reference) are those of the GPU backward tests.
 """
 import dataclasses
