@@ -303,6 +303,9 @@ def main():
     ap.add_argument("--bwd-impl", default="serial", choices=["serial", "chunked"],
                     help="backward entry point: ckda_bwd (token-serial) or ckda_bwd_chunked")
     ap.add_argument("--complex-steps", type=int, default=5)
+    ap.add_argument("--complex-impl", default="serial", choices=["serial", "chunked"],
+                    help="complex-gate entry point: ckda_fwd_complex (token-serial) or "
+                         "ckda_fwd_complex_chunked")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -457,10 +460,17 @@ def main():
     co = torch.empty((T_total, H, dv), dtype=torch.complex64, device="cuda")
     csf = torch.empty((N, H, dk, dv), dtype=torch.complex64, device="cuda")
 
+    cchunked = args.complex_impl == "chunked"
+    cws = None
+    if cchunked:
+        cws = torch.empty(ckda.ckda_fwd_complex_chunked_workspace_bytes(N, T_total, H, dk, dv,
+                                                                         True),
+                          dtype=torch.uint8, device="cuda")
+
     def complex_step():
         ckda.ckda_fwd_complex(cin["q"], cin["k"], cin["v"], cin["alpha"], cin["theta"],
                               cin["beta"], cin["initial_state"], csf, co, cin["cu_seqlens"],
-                              None, stream=stream)
+                              None, stream=stream, chunked=cchunked, workspace=cws)
 
     cms = time_loop(complex_step, args.complex_steps, 3, stream, barrier)
     if ckda.ckda_last_error() != ckda.CKDA_OK:
@@ -472,8 +482,13 @@ def main():
                                  "peak": pk["hbm_gbs"], "unit": "GB/s",
                                  "frac": cbytes / (cms / 1e3) / 1e9 / pk["hbm_gbs"],
                                  "traffic": None, "algorithmic_bytes_per_launch": cbytes},
-                    "kernel": "token-serial complex recurrence on CUDA cores, fp32",
-                    "gpu_launches": args.complex_steps}
+                    "kernel": ("chunked (16-token chunk-WY, complex) on CUDA cores, fp32: "
+                               "a prep over all chunks and a state scan" if cchunked else
+                               "token-serial complex recurrence on CUDA cores, fp32"),
+                    "entry_point": ("ckda_fwd_complex_chunked" if cchunked
+                                    else "ckda_fwd_complex"),
+                    "gpu_launches": (2 if cchunked else 1) * args.complex_steps}
+    del cws
     del cin, co, csf
 
     # ---------------- decode step

@@ -87,6 +87,11 @@ def load(path: str | None = None):
     lib.ckda_bwd_chunked.argtypes = lib.ckda_bwd.argtypes
     lib.ckda_fwd_complex.restype = ctypes.c_int
     lib.ckda_fwd_complex.argtypes = [vp] * 11 + [i32] * 5 + [f32, vp]
+    lib.ckda_fwd_complex_chunked.restype = ctypes.c_int
+    lib.ckda_fwd_complex_chunked.argtypes = [vp] * 11 + [i32] * 5 + [f32, vp, ctypes.c_size_t,
+                                                                     vp]
+    lib.ckda_fwd_complex_chunked_workspace_bytes.restype = ctypes.c_size_t
+    lib.ckda_fwd_complex_chunked_workspace_bytes.argtypes = [i32] * 6
     lib.ckda_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.ckda_bwd_workspace_bytes.argtypes = [i32] * 6
     lib.ckda_bwd_chunked_workspace_bytes.restype = ctypes.c_size_t
@@ -404,13 +409,20 @@ def fwd_chunked_gated(q, k_raw, v, a_logit, c_logit, gates: GateParams,
     return o, sf
 
 
+def ckda_fwd_complex_chunked_workspace_bytes(N, T, H, d_k, d_v, varlen=False) -> int:
+    """Scratch bytes ckda_fwd_complex_chunked needs (see include/ckda.h)."""
+    return int(load().ckda_fwd_complex_chunked_workspace_bytes(
+        int(N), int(T), int(H), int(d_k), int(d_v), int(bool(varlen))))
+
+
 def ckda_fwd_complex(q, k, v, alpha, theta, beta, initial_state, final_state, o,
                      cu_seqlens=None, cu_seqlens_host=None, N=None, T=None,
-                     scale: float = 1.0, stream=None):
-    """Marshal tensors into ckda_fwd_complex (see include/ckda.h): q, k
-    [T_total, H, d_k] and v, o [T_total, H, d_v] complex64; alpha, theta
-    [T_total, H, d_k] and beta [T_total, H] fp32; states [N, H, d_k, d_v]
-    complex64 or None."""
+                     scale: float = 1.0, stream=None, chunked: bool = False, workspace=None):
+    """Marshal tensors into ckda_fwd_complex, or ckda_fwd_complex_chunked when
+    ``chunked`` (see include/ckda.h): q, k [T_total, H, d_k] and v, o
+    [T_total, H, d_v] complex64; alpha, theta [T_total, H, d_k] and beta
+    [T_total, H] fp32; states [N, H, d_k, d_v] complex64 or None. The chunked
+    call allocates its workspace with torch unless one is given."""
     lib = load()
     for t, nme in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, nme, torch.complex64, 3)
@@ -434,17 +446,26 @@ def ckda_fwd_complex(q, k, v, alpha, theta, beta, initial_state, final_state, o,
                 or not cu_seqlens_host.is_contiguous():
             raise ValueError("cu_seqlens_host must be a contiguous CPU int32 tensor")
         host_ptr = ctypes.c_void_p(cu_seqlens_host.data_ptr())
-    st = lib.ckda_fwd_complex(_p(q), _p(k), _p(v), _p(alpha), _p(theta), _p(beta),
-                              _p(initial_state), _p(final_state), _p(o), _p(cu_seqlens), host_ptr,
-                              int(N), int(T), int(H), int(d_k), int(d_v), float(scale),
-                              _stream(stream))
-    _check(st, "ckda_fwd_complex")
+    args = (_p(q), _p(k), _p(v), _p(alpha), _p(theta), _p(beta), _p(initial_state),
+            _p(final_state), _p(o), _p(cu_seqlens), host_ptr, int(N), int(T), int(H), int(d_k),
+            int(d_v), float(scale))
+    if not chunked:
+        _check(lib.ckda_fwd_complex(*args, _stream(stream)), "ckda_fwd_complex")
+        return
+    need = ckda_fwd_complex_chunked_workspace_bytes(N, T, H, d_k, d_v, cu_seqlens is not None)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ckda_fwd_complex_chunked(*args, _p(workspace), ws_bytes, _stream(stream)),
+           "ckda_fwd_complex_chunked")
 
 
 def fwd_complex(q, k, v, alpha, theta, beta, initial_state=None, cu_seqlens=None,
-                cu_seqlens_host=None, N=None, T=None, scale: float = 1.0, stream=None):
+                cu_seqlens_host=None, N=None, T=None, scale: float = 1.0, stream=None,
+                chunked: bool = False):
     """The complex-phase gate: allocate o and the final state (complex64) with
-    torch, then call ckda_fwd_complex. Returns (o, final_state)."""
+    torch, then call ckda_fwd_complex (ckda_fwd_complex_chunked when
+    ``chunked``). Returns (o, final_state)."""
     T_total, H, d_k = q.shape
     d_v = v.shape[2]
     if cu_seqlens is not None:
@@ -454,7 +475,7 @@ def fwd_complex(q, k, v, alpha, theta, beta, initial_state=None, cu_seqlens=None
     o = torch.empty((T_total, H, d_v), dtype=torch.complex64, device=q.device)
     sf = torch.empty((N, H, d_k, d_v), dtype=torch.complex64, device=q.device)
     ckda_fwd_complex(q, k, v, alpha, theta, beta, initial_state, sf, o, cu_seqlens,
-                     cu_seqlens_host, N, T, scale, stream)
+                     cu_seqlens_host, N, T, scale, stream, chunked)
     return o, sf
 
 

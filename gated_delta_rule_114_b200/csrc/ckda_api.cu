@@ -23,6 +23,13 @@ cudaError_t launch_fwd_simt(int dk, int dv, int chunk, const void *q,
                             int T_total, int H, float scale, GateArgs g,
                             unsigned int *err, cudaStream_t st);
 size_t bwd_workspace_bytes(int N, int T_total, int H, int dk, int dv);
+size_t complex_chunk_workspace_bytes(int N, int T_total, int H, int dk, int dv);
+cudaError_t launch_fwd_complex_chunked(int dk, int dv, const void *q, const void *k,
+                                       const void *v, const float *alpha, const float *theta,
+                                       const float *beta, const void *s0, void *sf, void *o,
+                                       const int32_t *cu, int N, int T, int T_total, int H,
+                                       float scale, void *ws, unsigned int *err,
+                                       cudaStream_t st);
 cudaError_t launch_fwd_complex(int dk, int dv, const void *q, const void *k, const void *v,
                                const float *alpha, const float *theta, const float *beta,
                                const void *s0, void *sf, void *o, const int32_t *cu, int N,
@@ -179,24 +186,35 @@ ckda_status ckda_last_error(cudaStream_t stream) {
   return w ? CKDA_ERR_DEVICE : CKDA_OK;
 }
 
-ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const float *alpha,
-                             const float *theta, const float *beta, const void *initial_state,
-                             void *final_state, void *o, const int32_t *cu_seqlens,
-                             const int32_t *cu_seqlens_host, int32_t N, int32_t T, int32_t H,
-                             int32_t d_k, int32_t d_v, float scale, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// ckda_fwd_complex (token-serial kernel, chunked = false) and
+// ckda_fwd_complex_chunked: one validation, then the chosen launch.
+ckda_status complex_impl(const void *q, const void *k, const void *v, const float *alpha,
+                         const float *theta, const float *beta, const void *initial_state,
+                         void *final_state, void *o, const int32_t *cu_seqlens,
+                         const int32_t *cu_seqlens_host, int32_t N, int32_t T, int32_t H,
+                         int32_t d_k, int32_t d_v, float scale, void *workspace,
+                         size_t workspace_bytes, cudaStream_t stream, bool chunked) {
   if (!supported_dim(d_k) || !supported_dim(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (N < 0 || T < 0 || H <= 0) return CKDA_ERR_ARG;
   if (!grid_fits(N, H)) return CKDA_ERR_UNSUPPORTED;
   if (!q || !k || !v || !alpha || !theta || !beta || !o) return CKDA_ERR_ARG;
-  const void *ptrs[] = {q, k, v, alpha, theta, beta, initial_state, final_state, o, cu_seqlens};
+  const void *ptrs[] = {q, k, v, alpha, theta, beta, initial_state, final_state, o, cu_seqlens,
+                        workspace};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return CKDA_ERR_ARG;
   int64_t T_total;
   if (!token_rows(cu_seqlens, cu_seqlens_host, N, T, T_total)) return CKDA_ERR_ARG;
-  // complex64 = 8 bytes per element; no output may overlap an input or the other output
+  // complex64 = 8 bytes per element; no output may overlap an input, the other
+  // output or the workspace
   const size_t th = (size_t)T_total * H;
   const size_t kb = th * d_k * 8, vb = th * d_v * 8, rb = th * d_k * sizeof(float);
   const size_t sb = (size_t)N * H * d_k * d_v * 8;
+  const size_t need =
+      chunked && N > 0 ? ckda::complex_chunk_workspace_bytes(N, (int)T_total, H, d_k, d_v) : 0;
   struct R { const void *p; size_t n; };
   const R ins[] = {{q, kb}, {k, kb}, {v, vb}, {alpha, rb}, {theta, rb}, {beta, th * sizeof(float)},
                    {initial_state, sb}};
@@ -208,11 +226,56 @@ ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const 
   if (final_state && initial_state && final_state != initial_state &&
       overlaps(final_state, sb, initial_state, sb))
     return CKDA_ERR_ARG;
+  if (chunked) {
+    for (const R &x : ins)
+      if (overlaps(workspace, need, x.p, x.n)) return CKDA_ERR_ARG;
+    if (overlaps(workspace, need, o, vb) || overlaps(workspace, need, final_state, sb))
+      return CKDA_ERR_ARG;
+  }
   if (N == 0) return CKDA_OK;
-  const cudaError_t e = ckda::launch_fwd_complex(d_k, d_v, q, k, v, alpha, theta, beta,
+  if (chunked && (!workspace || workspace_bytes < need)) return CKDA_ERR_ARG;
+  const cudaError_t e =
+      chunked ? ckda::launch_fwd_complex_chunked(d_k, d_v, q, k, v, alpha, theta, beta,
                                                  initial_state, final_state, o, cu_seqlens, N, T,
-                                                 (int)T_total, H, scale, error_word_ptr(), stream);
+                                                 (int)T_total, H, scale, workspace,
+                                                 error_word_ptr(), stream)
+              : ckda::launch_fwd_complex(d_k, d_v, q, k, v, alpha, theta, beta, initial_state,
+                                         final_state, o, cu_seqlens, N, T, (int)T_total, H,
+                                         scale, error_word_ptr(), stream);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const float *alpha,
+                             const float *theta, const float *beta, const void *initial_state,
+                             void *final_state, void *o, const int32_t *cu_seqlens,
+                             const int32_t *cu_seqlens_host, int32_t N, int32_t T, int32_t H,
+                             int32_t d_k, int32_t d_v, float scale, cudaStream_t stream) {
+  return complex_impl(q, k, v, alpha, theta, beta, initial_state, final_state, o, cu_seqlens,
+                      cu_seqlens_host, N, T, H, d_k, d_v, scale, nullptr, 0, stream, false);
+}
+
+ckda_status ckda_fwd_complex_chunked(const void *q, const void *k, const void *v,
+                                     const float *alpha, const float *theta, const float *beta,
+                                     const void *initial_state, void *final_state, void *o,
+                                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                     int32_t N, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                     float scale, void *workspace, size_t workspace_bytes,
+                                     cudaStream_t stream) {
+  return complex_impl(q, k, v, alpha, theta, beta, initial_state, final_state, o, cu_seqlens,
+                      cu_seqlens_host, N, T, H, d_k, d_v, scale, workspace, workspace_bytes,
+                      stream, true);
+}
+
+size_t ckda_fwd_complex_chunked_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                                int32_t d_v, int32_t varlen) {
+  if (N <= 0 || T < 0 || H <= 0 || !supported_dim(d_k) || !supported_dim(d_v)) return 0;
+  const int64_t T_total = varlen ? (int64_t)T : (int64_t)N * T;
+  if (T_total > INT32_MAX) return 0;
+  return ckda::complex_chunk_workspace_bytes(N, (int)T_total, H, d_k, d_v);
 }
 
 size_t ckda_bwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,

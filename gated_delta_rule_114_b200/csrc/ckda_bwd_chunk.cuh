@@ -314,7 +314,8 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
     g = 1.f;  // G_{i<-r}
     for (int i = r; i < C; ++i) {
       if (i > r) g *= al[i * KS + c];
-      dk += g * (sm[Ly::DM + i * CS + r] * qq[i * KS + c] + sm[Ly::DA + i * CS + r] * kk[i * KS + c]);
+      dk += g * (sm[Ly::DM + i * CS + r] * qq[i * KS + c] +
+                 sm[Ly::DA + i * CS + r] * kk[i * KS + c]);
     }
     if (r < L) {
       const size_t pi = ((size_t)tile * a.TH + (size_t)(t0 + r) * H + h) * DK + c;

@@ -226,7 +226,8 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
     x.par(DK * DVT, [&](int e) {  // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
       const int c = e / DVT, v = e - c * DVT;
       float s = GC[c] * DS[c * VS + v];
-      for (int i = 0; i < C; ++i) s += QS[i * KS + c] * DO[i * VS + v] - BK[i * KS + c] * DR[i * VS + v];
+      for (int i = 0; i < C; ++i)
+        s += QS[i * KS + c] * DO[i * VS + v] - BK[i * KS + c] * DR[i * VS + v];
       DS[c * VS + v] = s;
     });
   }

@@ -1,0 +1,262 @@
+// The complex-phase gate's forward in 16-token chunks: per-CTA programs.
+//
+// "Semidirect Fourier Delta Attention" §3, eqs. (13)-(14): S' = Lambda_t S,
+// Lambda_t = diag(lambda_t), lambda_t = alpha_t exp(i theta_t);
+// S_t = S' + beta_t k_t (conj(v_t) - k_t^* S')^T; o_t = scale S_t^* q_t. The
+// chunk-WY form of §2.2 eqs. (9)-(10) carries over with conjugates where k^*
+// and q^* stand (rows i, j in 0..C-1 of a chunk; entry state S;
+// G_{i<-j} = prod_{s=j+1..i} diag(lambda_s); gamma_i = G_{i<-(-1)};
+// sigma_j = G_{C-1<-j}):
+//   A_ij = beta_i k_i^* G_{i<-j} k_j (j < i),   M_ij = q_i^* G_{i<-j} k_j (j <= i)
+//   T = (I + A)^-1,  W = T diag(beta) Khat,  Utilde = T diag(beta) conj(V)
+//   U = Utilde - W S,  conj(O) = scale (Qhat S + M U),
+//   S <- diag(gamma_{C-1}) S + Kbar^T U,
+// with Khat_i = gamma_i conj(k_i), Qhat_i = gamma_i conj(q_i), Kbar_j = sigma_j k_j.
+// Two programs:
+//   prep (per chunk and head): lambda, gamma, sigma, A and M (per-pair running
+//        products of lambda over at most 15 tokens), T by forward substitution,
+//        then W, Kbar, Qhat (token-major [T, H, d_k]), Utilde ([T, H, d_v]),
+//        M and gamma_{C-1} per checkpoint slot;
+//   scan (per sequence, head, tile of DVT complex columns): per chunk
+//        U = Utilde - W S, the outputs, the state update.
+// Complex numbers are interleaved (real, imaginary) fp32 pairs, in global and
+// in shared memory. The same executor contract as ckda_bwd_chunk.cuh: each
+// phase is x.par(n, f) over independent items, then a barrier, so the programs
+// also run as plain host loops in the tests.
+#pragma once
+
+#include <math.h>
+
+#include "ckda_bwd_chunk.cuh"
+
+namespace ckda {
+namespace cplx {
+
+using bwdc::C;
+
+struct cf {
+  float r, i;
+};
+CKDA_PROG cf cmul(cf a, cf b) { return cf{a.r * b.r - a.i * b.i, a.r * b.i + a.i * b.r}; }
+// conj(a) b
+CKDA_PROG cf cmulc(cf a, cf b) { return cf{a.r * b.r + a.i * b.i, a.r * b.i - a.i * b.r}; }
+CKDA_PROG cf cadd(cf a, cf b) { return cf{a.r + b.r, a.i + b.i}; }
+CKDA_PROG cf csub(cf a, cf b) { return cf{a.r - b.r, a.i - b.i}; }
+CKDA_PROG cf cscale(float s, cf a) { return cf{s * a.r, s * a.i}; }
+CKDA_PROG cf cconj(cf a) { return cf{a.r, -a.i}; }
+CKDA_PROG cf cld(const float *p) { return cf{p[0], p[1]}; }
+CKDA_PROG void cst(float *p, cf x) {
+  p[0] = x.r;
+  p[1] = x.i;
+}
+
+// Pointers and sizes of one call: q, k [T_total, H, d_k] and v, o [T_total,
+// H, d_v] complex; alpha, theta [T_total, H, d_k] and beta [T_total, H] fp32;
+// states [N, H, d_k, d_v] complex (s0, sf may be null).
+struct Args {
+  const float *q, *k, *v, *alpha, *theta, *beta, *s0;
+  float *sf, *o;
+  int H, DVF;
+  float scale;
+};
+
+// Workspace (complex unless noted): W, Kbar, Qhat [T_total H][d_k];
+// Utilde [T_total H][d_v]; M [slots][H][C][C]; gamma_{C-1} [slots][H][d_k].
+struct Ws {
+  float *wt, *kb, *qh, *ut, *mm, *gc;
+};
+
+template <int DK, int DVT>
+struct PrepLayout {
+  static constexpr int KS = 2 * (DK + 1), VS = 2 * (DVT + 1), CS = 2 * (C + 1);
+  // C x DK complex: q, k, lambda, gamma, sigma; C x DVT complex: conj(v)
+  static constexpr int Q = 0, K = Q + C * KS, LM = K + C * KS, GM = LM + C * KS,
+                       SG = GM + C * KS, V = SG + C * KS;
+  // C x C complex: A, M, T; beta [C]
+  static constexpr int A = V + C * VS, M = A + C * CS, TT = M + C * CS, BE = TT + C * CS;
+  static constexpr int FLOATS = BE + C;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+template <class X, int DK, int DVT>
+CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, int t0, int L,
+                            int slot) {
+  using Ly = PrepLayout<DK, DVT>;
+  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
+  const int H = a.H, DVF = a.DVF;
+  float *be = sm + Ly::BE;
+  // stage q, k (complex), lambda = alpha (cos theta, sin theta), beta; rows
+  // L..C-1 are inert (q = k = 0, lambda = 1, beta = 0)
+  x.par(C * DK, [&](int e) {
+    const int i = e / DK, c = e - i * DK;
+    cf qv{0.f, 0.f}, kv{0.f, 0.f}, lv{1.f, 0.f};
+    if (i < L) {
+      const size_t g = ((size_t)(t0 + i) * H + h) * DK + c;
+      qv = cld(a.q + 2 * g);
+      kv = cld(a.k + 2 * g);
+      const float al = a.alpha[g], th = a.theta[g];
+      lv = cf{al * cosf(th), al * sinf(th)};
+    }
+    cst(sm + Ly::Q + i * KS + 2 * c, qv);
+    cst(sm + Ly::K + i * KS + 2 * c, kv);
+    cst(sm + Ly::LM + i * KS + 2 * c, lv);
+    if (e < C) be[e] = e < L ? a.beta[(size_t)(t0 + e) * H + h] : 0.f;
+  });
+  x.par(DK, [&](int c) {  // gamma (prefix products), sigma (suffix products)
+    cf g{1.f, 0.f};
+    for (int i = 0; i < C; ++i) {
+      g = cmul(g, cld(sm + Ly::LM + i * KS + 2 * c));
+      cst(sm + Ly::GM + i * KS + 2 * c, g);
+    }
+    g = cf{1.f, 0.f};
+    for (int j = C - 1; j >= 0; --j) {
+      cst(sm + Ly::SG + j * KS + 2 * c, g);
+      g = cmul(g, cld(sm + Ly::LM + j * KS + 2 * c));
+    }
+  });
+  x.par(C * C, [&](int e) {  // A (without beta) and M
+    const int i = e / C, j = e - i * C;
+    cf ak{0.f, 0.f}, m{0.f, 0.f};
+    if (j <= i) {
+      for (int c = 0; c < DK; ++c) {
+        cf g{1.f, 0.f};
+        for (int s = j + 1; s <= i; ++s) g = cmul(g, cld(sm + Ly::LM + s * KS + 2 * c));
+        const cf gk = cmul(g, cld(sm + Ly::K + j * KS + 2 * c));
+        ak = cadd(ak, cmulc(cld(sm + Ly::K + i * KS + 2 * c), gk));
+        m = cadd(m, cmulc(cld(sm + Ly::Q + i * KS + 2 * c), gk));
+      }
+      if (j == i) ak = cf{0.f, 0.f};
+    }
+    cst(sm + Ly::A + i * CS + 2 * j, ak);
+    cst(sm + Ly::M + i * CS + 2 * j, m);
+    w.mm[(((size_t)slot * H + h) * C * C + e) * 2] = m.r;
+    w.mm[(((size_t)slot * H + h) * C * C + e) * 2 + 1] = m.i;
+  });
+  x.par(C, [&](int j) {  // column j of T = (I + diag(beta) A)^-1
+    float *tt = sm + Ly::TT;
+    for (int i = 0; i < j; ++i) cst(tt + i * CS + 2 * j, cf{0.f, 0.f});
+    cst(tt + j * CS + 2 * j, cf{1.f, 0.f});
+    for (int i = j + 1; i < C; ++i) {
+      cf s{0.f, 0.f};
+      for (int m = j; m < i; ++m)
+        s = cadd(s, cmul(cld(sm + Ly::A + i * CS + 2 * m), cld(tt + m * CS + 2 * j)));
+      cst(tt + i * CS + 2 * j, cscale(-be[i], s));
+    }
+  });
+  // W = T diag(beta) Khat, Kbar, Qhat; gamma_{C-1}
+  x.par(C * DK, [&](int e) {
+    const int i = e / DK, c = e - i * DK;
+    if (e < DK) {
+      const cf g = cld(sm + Ly::GM + (C - 1) * KS + 2 * c);
+      cst(w.gc + (((size_t)slot * H + h) * DK + c) * 2, g);
+    }
+    if (i >= L) return;
+    cf wt{0.f, 0.f};
+    for (int m = 0; m <= i; ++m) {
+      const cf kh =
+          cmul(cld(sm + Ly::GM + m * KS + 2 * c), cconj(cld(sm + Ly::K + m * KS + 2 * c)));
+      wt = cadd(wt, cscale(be[m], cmul(cld(sm + Ly::TT + i * CS + 2 * m), kh)));
+    }
+    const size_t o = (((size_t)(t0 + i) * H + h) * DK + c) * 2;
+    cst(w.wt + o, wt);
+    cst(w.kb + o, cmul(cld(sm + Ly::SG + i * KS + 2 * c), cld(sm + Ly::K + i * KS + 2 * c)));
+    cst(w.qh + o,
+        cmul(cld(sm + Ly::GM + i * KS + 2 * c), cconj(cld(sm + Ly::Q + i * KS + 2 * c))));
+  });
+  // Utilde = T diag(beta) conj(V), one column tile at a time
+  for (int c0 = 0; c0 < DVF; c0 += DVT) {
+    x.par(C * DVT, [&](int e) {
+      const int i = e / DVT, v = e - i * DVT;
+      const cf vv = i < L ? cld(a.v + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2)
+                          : cf{0.f, 0.f};
+      cst(sm + Ly::V + i * VS + 2 * v, cconj(vv));
+    });
+    x.par(C * DVT, [&](int e) {
+      const int i = e / DVT, v = e - i * DVT;
+      cf u{0.f, 0.f};
+      for (int m = 0; m <= i; ++m)
+        u = cadd(u, cscale(be[m], cmul(cld(sm + Ly::TT + i * CS + 2 * m),
+                                       cld(sm + Ly::V + m * VS + 2 * v))));
+      if (i < L) cst(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2, u);
+    });
+  }
+}
+
+template <int DK, int DVT>
+struct ScanLayout {
+  static constexpr int KS = 2 * (DK + 1), VS = 2 * (DVT + 1), CS = 2 * (C + 1);
+  // DK x DVT complex state; C x DK complex W, Kbar, Qhat; C x DVT complex U;
+  // C x C complex M; gamma_{C-1} [DK] complex
+  static constexpr int S = 0, WT = S + DK * VS, KB = WT + C * KS, QH = KB + C * KS,
+                       U = QH + C * KS, M = U + C * VS, GC = M + C * CS;
+  static constexpr int FLOATS = GC + 2 * DK;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+template <class X, int DK, int DVT>
+CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, int n, int tile,
+                            int bos, int eos, int slot0) {
+  using Ly = ScanLayout<DK, DVT>;
+  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
+  const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
+  const int nck = (eos - bos + C - 1) / C;
+  const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;  // complex elements
+  float *S = sm + Ly::S, *U = sm + Ly::U;
+  x.par(DK * DVT, [&](int e) {
+    const int c = e / DVT, v = e - c * DVT;
+    const cf s = a.s0 ? cld(a.s0 + (st_base + (size_t)c * DVF + v) * 2) : cf{0.f, 0.f};
+    cst(S + c * VS + 2 * v, s);
+  });
+  for (int ci = 0; ci < nck; ++ci) {
+    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
+    const size_t sl = (size_t)(slot0 + ci) * H + h;
+    x.par(C * DK, [&](int e) {  // the chunk's factors; rows L..C-1 zero
+      const int i = e / DK, c = e - i * DK;
+      const size_t o = (((size_t)(t0 + i) * H + h) * DK + c) * 2;
+      const bool in = i < L;
+      cst(sm + Ly::WT + i * KS + 2 * c, in ? cld(w.wt + o) : cf{0.f, 0.f});
+      cst(sm + Ly::KB + i * KS + 2 * c, in ? cld(w.kb + o) : cf{0.f, 0.f});
+      cst(sm + Ly::QH + i * KS + 2 * c, in ? cld(w.qh + o) : cf{0.f, 0.f});
+      if (e < C * C)
+        cst(sm + Ly::M + (e / C) * CS + 2 * (e % C), cld(w.mm + (sl * C * C + e) * 2));
+      if (e < DK) cst(sm + Ly::GC + 2 * e, cld(w.gc + (sl * DK + e) * 2));
+    });
+    x.par(C * DVT, [&](int e) {  // U = Utilde - W S
+      const int i = e / DVT, v = e - i * DVT;
+      if (i >= L) {
+        cst(U + i * VS + 2 * v, cf{0.f, 0.f});
+        return;
+      }
+      cf u = cld(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
+      for (int c = 0; c < DK; ++c)
+        u = csub(u, cmul(cld(sm + Ly::WT + i * KS + 2 * c), cld(S + c * VS + 2 * v)));
+      cst(U + i * VS + 2 * v, u);
+    });
+    x.par(C * DVT, [&](int e) {  // o = conj(scale (Qhat S + M U))
+      const int i = e / DVT, v = e - i * DVT;
+      if (i >= L) return;
+      cf s{0.f, 0.f};
+      for (int c = 0; c < DK; ++c)
+        s = cadd(s, cmul(cld(sm + Ly::QH + i * KS + 2 * c), cld(S + c * VS + 2 * v)));
+      for (int j = 0; j <= i; ++j)
+        s = cadd(s, cmul(cld(sm + Ly::M + i * CS + 2 * j), cld(U + j * VS + 2 * v)));
+      cst(a.o + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2, cconj(cscale(a.scale, s)));
+    });
+    x.par(DK * DVT, [&](int e) {  // S <- diag(gamma_{C-1}) S + Kbar^T U
+      const int c = e / DVT, v = e - c * DVT;
+      cf s = cmul(cld(sm + Ly::GC + 2 * c), cld(S + c * VS + 2 * v));
+      for (int i = 0; i < C; ++i)
+        s = cadd(s, cmul(cld(sm + Ly::KB + i * KS + 2 * c), cld(U + i * VS + 2 * v)));
+      cst(S + c * VS + 2 * v, s);
+    });
+  }
+  if (a.sf) {
+    x.par(DK * DVT, [&](int e) {
+      const int c = e / DVT, v = e - c * DVT;
+      cst(a.sf + (st_base + (size_t)c * DVF + v) * 2, cld(S + c * VS + 2 * v));
+    });
+  }
+}
+
+}  // namespace cplx
+}  // namespace ckda

@@ -326,6 +326,36 @@ ckda_status ckda_fwd_complex(const void *q, const void *k, const void *v, const 
                              int32_t d_k, int32_t d_v, float scale, cudaStream_t stream);
 
 /*
+ * ckda_fwd_complex_chunked: the outputs of ckda_fwd_complex (the same
+ * arguments, layouts and errors, plus a workspace) computed 16 tokens at a
+ * time in the chunk-WY form of "Semidirect Fourier Delta Attention" §2.2
+ * eqs. (9)-(10) with complex gates lambda = alpha exp(i theta):
+ *   A_ij = beta_i k_i^* G_ij k_j (j < i),  M_ij = q_i^* G_ij k_j (j <= i),
+ *   T = (I + A)^-1,  U = T diag(beta) (conj(V) - Khat S),
+ *   conj(O) = scale (Qhat S + M U),  S <- diag(gamma) S + Kbar^T U,
+ * where G_ij is the product of the lambdas over (j, i], gamma and sigma the
+ * chunk's prefix and suffix products, Khat = gamma conj(k), Qhat = gamma conj(q),
+ * Kbar = sigma k. A prep kernel over all chunks forms T, W = T diag(beta) Khat,
+ * T diag(beta) conj(V), Kbar, Qhat and M; a scan per (sequence, head, tile of
+ * up to 32 complex columns) carries the state through U = T diag(beta) conj(V)
+ * - W S and the update. fp32 arithmetic on CUDA cores, deterministic.
+ *   workspace   device scratch of at least
+ *               ckda_fwd_complex_chunked_workspace_bytes() bytes, owned by the
+ *               caller; required when N > 0; must not overlap any tensor.
+ */
+ckda_status ckda_fwd_complex_chunked(const void *q, const void *k, const void *v,
+                                     const float *alpha, const float *theta, const float *beta,
+                                     const void *initial_state, void *final_state, void *o,
+                                     const int32_t *cu_seqlens, const int32_t *cu_seqlens_host,
+                                     int32_t N, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                     float scale, void *workspace, size_t workspace_bytes,
+                                     cudaStream_t stream);
+
+/* Scratch that ckda_fwd_complex_chunked needs (arguments as ckda_bwd_workspace_bytes). */
+size_t ckda_fwd_complex_chunked_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
+                                                int32_t d_v, int32_t varlen);
+
+/*
  * ckda_bwd_workspace_bytes, ckda_bwd_chunked_workspace_bytes: scratch that
  * ckda_bwd and ckda_bwd_chunked need (T as in ckda_bwd; varlen nonzero when
  * cu_seqlens is given, so that T is total_T). 0 for unsupported or invalid

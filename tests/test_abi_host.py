@@ -285,7 +285,11 @@ def test_bwd_zero_sequences_is_a_noop(lib):
 
 
 def cplx(lib, q=P, k=P2, v=P3, a=P4, th=P5, b=P6, s0=NULL, sf=NULL,
-         o=ctypes.c_void_p(0x70000), cu=NULL, cuh=NULL, N=1, T=8, H=1, dk=16, dv=16):
+         o=ctypes.c_void_p(0x70000), cu=NULL, cuh=NULL, N=1, T=8, H=1, dk=16, dv=16,
+         chunked=False, ws=ctypes.c_void_p(0x100000), wsb=1 << 30):
+    if chunked:
+        return lib.ckda_fwd_complex_chunked(q, k, v, a, th, b, s0, sf, o, cu, cuh, N, T, H, dk,
+                                            dv, 1.0, ws, wsb, None)
     return lib.ckda_fwd_complex(q, k, v, a, th, b, s0, sf, o, cu, cuh, N, T, H, dk, dv, 1.0,
                                 None)
 
@@ -304,9 +308,29 @@ def cplx(lib, q=P, k=P2, v=P3, a=P4, th=P5, b=P6, s0=NULL, sf=NULL,
     # host cu_seqlens without a device copy
     (dict(cuh=ctypes.cast((ctypes.c_int32 * 2)(0, 8), ctypes.c_void_p)), ckda.CKDA_ERR_ARG),
 ])
-def test_complex_rejects(lib, kw, want):
-    assert cplx(lib, **kw) == want
+@pytest.mark.parametrize("chunked", [False, True])
+def test_complex_rejects(lib, kw, want, chunked):
+    assert cplx(lib, chunked=chunked, **kw) == want
 
 
-def test_complex_zero_sequences_is_a_noop(lib):
-    assert cplx(lib, N=0, T=0) == ckda.CKDA_OK
+@pytest.mark.parametrize("kw", [dict(ws=NULL), dict(wsb=64), dict(ws=P)])
+def test_complex_chunked_rejects_bad_workspace(lib, kw):
+    """missing, too small, or over an input"""
+    assert cplx(lib, chunked=True, **kw) == ckda.CKDA_ERR_ARG
+
+
+def test_complex_chunked_workspace_query(lib):
+    # complex64 (8 bytes): W, Kbar, Qhat per token-head (d_k each), Utilde (d_v);
+    # per 16-token chunk slot and head: M (16 x 16) and gamma (d_k)
+    def want(N, T_total, H, dk, dv):
+        sl, th = (T_total // 16 + N) * H, T_total * H
+        return 8 * (th * (3 * dk + dv) + sl * (256 + dk))
+    q = lib.ckda_fwd_complex_chunked_workspace_bytes
+    assert q(2, 40, 3, 32, 64, 0) == want(2, 80, 3, 32, 64)
+    assert q(2, 40, 3, 32, 64, 1) == want(2, 40, 3, 32, 64)
+    assert q(1, 8, 1, 24, 16, 0) == 0 and q(0, 8, 1, 16, 16, 0) == 0
+
+
+@pytest.mark.parametrize("chunked", [False, True])
+def test_complex_zero_sequences_is_a_noop(lib, chunked):
+    assert cplx(lib, N=0, T=0, chunked=chunked, ws=NULL, wsb=0) == ckda.CKDA_OK
