@@ -28,9 +28,9 @@
 // over columns (dq, dk, dalpha, dbeta) is linear in per-column terms, so each
 // column tile writes fp32 partials that a second kernel adds in tile order.
 //
-// Every program is a fixed sequence of data-parallel phases. Executor X runs
-// one phase, x.par(n, f): f(i) for every i in [0, n), the calls independent
-// of one another, then a barrier. Every value that outlives a phase sits in
+// Every program is a fixed sequence of data-parallel phases. par<N>(x, f)
+// runs one phase on executor X: f(i) for every i in [0, N), the calls
+// independent of one another, then a barrier. Every value that outlives a phase sits in
 // the shared-memory block `sm` (or in global memory), so the same source runs
 // as a CUDA kernel (threads stride over i, __syncthreads between phases) and,
 // for tests, as plain host loops. Gate products inside a 16-token chunk are
@@ -45,9 +45,11 @@
 #ifdef __CUDACC__
 #define CKDA_PROG __device__ __forceinline__
 #define CKDA_UNROLL _Pragma("unroll")
+#define CKDA_LDG(p) __ldg(p)
 #else
 #define CKDA_PROG inline
 #define CKDA_UNROLL
+#define CKDA_LDG(p) (*(p))
 #endif
 #endif
 
@@ -55,6 +57,14 @@ namespace ckda {
 namespace bwdc {
 
 constexpr int C = 16;  // tokens per chunk
+
+// One phase: f(i) for every i in [0, N), the calls independent of one
+// another, then a barrier. N is a compile-time count so that a CUDA thread
+// can unroll its share of the items and issue all of their loads at once.
+template <int N, class X, class F>
+CKDA_PROG void par(X &x, F f) {
+  x.template run<N>(f);
+}
 
 // Shared-memory layout (floats) of the per-chunk gradient program. Rows are
 // padded to an odd stride so that a warp reading down a column, or along rows
@@ -105,15 +115,15 @@ CKDA_PROG void stage(X &x, const Args<IOT> &a, float *sm, int h, int c0, int t0,
                      bool with_do) {
   constexpr int DK = Ly::dk, DVT = Ly::dvt;
   constexpr int NW = DK > DVT ? DK : DVT;  // items per row: the wider of d_k and the tile
-  x.par(C * NW, [&](int e) {
+  par<C * NW>(x, [&](int e) {
     const int i = e / NW, c = e - i * NW;
     if (c < DK) {
       float qv = 0.f, kv = 0.f, av = 1.f;
       if (i < L) {
         const size_t g = ((size_t)(t0 + i) * a.H + h) * DK + c;
-        qv = IOL::ld(a.q + g);
-        kv = IOL::ld(a.k + g);
-        av = a.alpha[g];
+        qv = IOL::ldg(a.q + g);
+        kv = IOL::ldg(a.k + g);
+        av = CKDA_LDG(a.alpha + g);
       }
       sm[Ly::Q + i * Ly::KS + c] = qv;
       sm[Ly::K + i * Ly::KS + c] = kv;
@@ -123,13 +133,13 @@ CKDA_PROG void stage(X &x, const Args<IOT> &a, float *sm, int h, int c0, int t0,
       float vv = 0.f, dd = 0.f;
       if (i < L) {
         const size_t g = ((size_t)(t0 + i) * a.H + h) * a.DVF + c0 + c;
-        vv = IOL::ld(a.v + g);
-        if (with_do) dd = IOL::ld(a.d_o + g);
+        vv = IOL::ldg(a.v + g);
+        if (with_do) dd = IOL::ldg(a.d_o + g);
       }
       sm[Ly::V + i * Ly::VS + c] = vv;
       sm[Ly::DO + i * Ly::VS + c] = dd;
     }
-    if (e < C) sm[Ly::BE + e] = e < L ? a.beta[(size_t)(t0 + e) * a.H + h] : 0.f;
+    if (e < C) sm[Ly::BE + e] = e < L ? CKDA_LDG(a.beta + (size_t)(t0 + e) * a.H + h) : 0.f;
   });
 }
 
@@ -138,7 +148,7 @@ template <class X, class Ly>
 CKDA_PROG void chunk_gates(X &x, float *sm) {
   constexpr int DK = Ly::dk, KS = Ly::KS;
   const float *al = sm + Ly::AL;
-  x.par(DK, [&](int c) {
+  par<DK>(x, [&](int c) {
     float g = 1.f;
     for (int i = 0; i < C; ++i) {
       g *= al[i * KS + c];
@@ -157,7 +167,7 @@ template <class X, class Ly>
 CKDA_PROG void chunk_grams_solve(X &x, float *sm, bool want_m) {
   constexpr int DK = Ly::dk, KS = Ly::KS, CS = Ly::CS;
   const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q, *be = sm + Ly::BE;
-  x.par(C * C, [&](int e) {
+  par<C * C>(x, [&](int e) {
     const int i = e / C, j = e - i * C;
     float ab = 0.f, m = 0.f;
     if (j <= i) {
@@ -173,7 +183,7 @@ CKDA_PROG void chunk_grams_solve(X &x, float *sm, bool want_m) {
     sm[Ly::AB + i * CS + j] = ab;
     if (want_m) sm[Ly::M + i * CS + j] = m;
   });
-  x.par(C, [&](int j) {  // column j of T by forward substitution
+  par<C>(x, [&](int j) {  // column j of T by forward substitution
     float *tt = sm + Ly::TT;
     const float *ab = sm + Ly::AB;
     for (int i = 0; i < j; ++i) tt[i * CS + j] = 0.f;
@@ -191,7 +201,7 @@ template <class X, class Ly>
 CKDA_PROG void chunk_khat_s(X &x, float *sm) {
   constexpr int DK = Ly::dk, DVT = Ly::dvt, KS = Ly::KS, VS = Ly::VS;
   const float *kk = sm + Ly::K;
-  x.par(C * DVT, [&](int e) {
+  par<C * DVT>(x, [&](int e) {
     const int i = e / DVT, v = e - i * DVT;
     float ks = 0.f;
     for (int c = 0; c < DK; ++c)
@@ -252,7 +262,7 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
   const float *be = sm + Ly::BE;
   const float *S = sm + Ly::S, *DS = sm + Ly::DS;
   // w = V - Khat S - Abar U (over the Khat S rows); dv = diag(beta) dR
-  x.par(C * DVT, [&](int e) {
+  par<C * DVT>(x, [&](int e) {
     const int i = e / DVT, v = e - i * DVT;
     float s = 0.f;
     for (int m = 0; m < i; ++m) s += sm[Ly::AB + i * CS + m] * sm[Ly::U + m * VS + v];
@@ -262,7 +272,7 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
               be[i] * sm[Ly::DR + i * VS + v]);
   });
   // dbeta (this tile's share); dM and dAbar
-  x.par(C * C, [&](int e) {
+  par<C * C>(x, [&](int e) {
     const int i = e / C, j = e - i * C;
     if (j == 0 && i < L) {
       float s = 0.f;
@@ -282,7 +292,7 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
   });
   // the state-side terms: dQhat = scale dO S^T, dKhat = -diag(beta) dR S^T,
   // dKbar = U dS_C^T; dq and dk start from them, E0 and EX keep the gate parts
-  x.par(C * DK, [&](int e) {
+  par<C * DK>(x, [&](int e) {
     const int i = e / DK, c = e - i * DK;
     float xq = 0.f, xk = 0.f, xb = 0.f;
     for (int v = 0; v < DVT; ++v) {
@@ -299,7 +309,7 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
     sm[Ly::EX + i * KS + c] = sm[Ly::K + i * KS + c] * xb;
   });
   // gated Gram terms of dq and dk; write this tile's dq, dk partials
-  x.par(C * DK, [&](int e) {
+  par<C * DK>(x, [&](int e) {
     const int r = e / DK, c = e - r * DK;
     const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
     float dq = sm[Ly::DQ + r * KS + c], dk = sm[Ly::DKK + r * KS + c];
@@ -324,7 +334,7 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
     }
   });
   // dalpha (this tile's share), one channel per item
-  x.par(DK, [&](int c) {
+  par<DK>(x, [&](int c) {
     float sds = 0.f;
     for (int v = 0; v < DVT; ++v) sds += S[c * VS + v] * DS[c * VS + v];
     float da[C];

@@ -26,10 +26,17 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// One phase: this thread's items threadIdx.x + r * kThreads, fully unrolled,
+// then the CTA's barrier.
 struct DeviceExec {
-  template <class F>
-  __device__ __forceinline__ void par(int n, F f) {
-    for (int i = threadIdx.x; i < n; i += kThreads) f(i);
+  template <int N, class F>
+  __device__ __forceinline__ void run(F f) {
+    constexpr int R = (N + kThreads - 1) / kThreads;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int i = threadIdx.x + r * kThreads;
+      if (N % kThreads == 0 || i < N) f(i);
+    }
     __syncthreads();
   }
 };

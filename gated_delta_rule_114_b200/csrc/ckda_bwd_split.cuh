@@ -74,7 +74,7 @@ CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *s
   chunk_gates<X, Ly>(x, sm);
   chunk_grams_solve<X, Ly>(x, sm, true);
   // the d_k-wide factors, gamma_C and Abar
-  x.par(C * DK, [&](int e) {
+  par<C * DK>(x, [&](int e) {
     const int i = e / DK, c = e - i * DK;
     if (e < DK) w.gc[((size_t)slot * H + h) * DK + c] = sm[Ly::GM + (C - 1) * KS + c];
     if (e < C * C) w.ab[((size_t)slot * H + h) * C * C + e] = sm[Ly::AB + (e / C) * CS + e % C];
@@ -95,19 +95,19 @@ CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *s
   // Utilde = T diag(beta) V and X = T^T (scale M^T dO), one column tile at a time
   for (int c0 = 0; c0 < DVF; c0 += DVT) {
     if (c0 > 0) {
-      x.par(C * DVT, [&](int e) {
+      par<C * DVT>(x, [&](int e) {
         const int i = e / DVT, v = e - i * DVT;
         float vv = 0.f, dd = 0.f;
         if (i < L) {
           const size_t g = ((size_t)(t0 + i) * H + h) * DVF + c0 + v;
-          vv = IOL::ld(a.v + g);
-          dd = IOL::ld(a.d_o + g);
+          vv = IOL::ldg(a.v + g);
+          dd = IOL::ldg(a.d_o + g);
         }
         sm[Ly::V + i * VS + v] = vv;
         sm[Ly::DO + i * VS + v] = dd;
       });
     }
-    x.par(C * DVT, [&](int e) {  // Utilde; Y = scale M^T dO into the R rows
+    par<C * DVT>(x, [&](int e) {  // Utilde; Y = scale M^T dO into the R rows
       const int i = e / DVT, v = e - i * DVT;
       float u = 0.f, y = 0.f;
       for (int m = 0; m <= i; ++m) u += tt[i * CS + m] * be[m] * sm[Ly::V + m * VS + v];
@@ -115,7 +115,7 @@ CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *s
       sm[Ly::RD + i * VS + v] = scale * y;
       if (i < L) w.ut[((size_t)(t0 + i) * H + h) * DVF + c0 + v] = u;
     });
-    x.par(C * DVT, [&](int e) {  // X = T^T Y
+    par<C * DVT>(x, [&](int e) {  // X = T^T Y
       const int j = e / DVT, v = e - j * DVT;
       float s = 0.f;
       for (int i = j; i < C; ++i) s += tt[i * CS + j] * sm[Ly::RD + i * VS + v];
@@ -135,49 +135,50 @@ struct ScanLayout {
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
-// rows [t0, t0 + L) of a token-major [T_total H][width] array into C padded rows
-template <class X>
-CKDA_PROG void load_rows(X &x, float *dst, int stride, const float *src, int width, int col0,
-                         int ncol, int t0, int L, int H, int h) {
-  x.par(C * ncol, [&](int e) {
-    const int i = e / ncol, c = e - i * ncol;
-    dst[i * stride + c] = i < L ? src[((size_t)(t0 + i) * H + h) * width + col0 + c] : 0.f;
-  });
-}
-
 template <class X, class IOL, typename IOT, int DK, int DVT>
 CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
                              int n, int tile, int bos, int eos, int slot0) {
   using Ly = ScanLayout<DK, DVT>;
   constexpr int KS = Ly::KS, VS = Ly::VS;
+  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of the load phase
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
   float *S = sm + Ly::S, *WT = sm + Ly::F0, *KB = sm + Ly::F1, *U = sm + Ly::R0;
   float *GC = sm + Ly::GC;
-  x.par(DK * DVT, [&](int e) {
+  par<DK * DVT>(x, [&](int e) {
     const int c = e / DVT, v = e - c * DVT;
     S[c * VS + v] = a.s0 ? a.s0[st_base + (size_t)c * DVF + v] : 0.f;
   });
   for (int ci = 0; ci < nck; ++ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t slot = (size_t)(slot0 + ci) * H + h;
-    x.par(DK * DVT, [&](int e) {
-      const int c = e / DVT, v = e - c * DVT;
-      w.cks[slot * DK * DVF + (size_t)c * DVF + c0 + v] = S[c * VS + v];
-      if (e < DK) GC[e] = w.gc[slot * DK + e];
+    // checkpoint S; load the chunk's W, Kbar, Utilde (rows L..C-1 zero) and gamma_C
+    par<NL>(x, [&](int e) {
+      if (e < DK * DVT) {
+        const int c = e / DVT, v = e - c * DVT;
+        w.cks[slot * DK * DVF + (size_t)c * DVF + c0 + v] = S[c * VS + v];
+      }
+      if (e < C * DK) {
+        const int i = e / DK, c = e - i * DK;
+        const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
+        WT[i * KS + c] = i < L ? CKDA_LDG(w.wt + o) : 0.f;
+        KB[i * KS + c] = i < L ? CKDA_LDG(w.kb + o) : 0.f;
+      }
+      if (e < C * DVT) {
+        const int i = e / DVT, v = e - i * DVT;
+        U[i * VS + v] = i < L ? CKDA_LDG(w.ut + ((size_t)(t0 + i) * H + h) * DVF + c0 + v) : 0.f;
+      }
+      if (e < DK) GC[e] = CKDA_LDG(w.gc + slot * DK + e);
     });
-    load_rows(x, WT, KS, w.wt, DK, 0, DK, t0, L, H, h);
-    load_rows(x, KB, KS, w.kb, DK, 0, DK, t0, L, H, h);
-    load_rows(x, U, VS, w.ut, DVF, c0, DVT, t0, L, H, h);
-    x.par(C * DVT, [&](int e) {  // U = Utilde - W S
+    par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
       const int i = e / DVT, v = e - i * DVT;
       float s = U[i * VS + v];
       for (int c = 0; c < DK; ++c) s -= WT[i * KS + c] * S[c * VS + v];
       U[i * VS + v] = s;
       if (i < L) w.uu[((size_t)(t0 + i) * H + h) * DVF + c0 + v] = s;
     });
-    x.par(DK * DVT, [&](int e) {  // S <- diag(gamma_C) S + Kbar^T U
+    par<DK * DVT>(x, [&](int e) {  // S <- diag(gamma_C) S + Kbar^T U
       const int c = e / DVT, v = e - c * DVT;
       float s = GC[c] * S[c * VS + v];
       for (int i = 0; i < C; ++i) s += KB[i * KS + c] * U[i * VS + v];
@@ -191,39 +192,48 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
                              int n, int tile, int bos, int eos, int slot0) {
   using Ly = ScanLayout<DK, DVT>;
   constexpr int KS = Ly::KS, VS = Ly::VS;
+  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of the load phase
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
   float *DS = sm + Ly::S, *WB = sm + Ly::F0, *QS = sm + Ly::F1, *BK = sm + Ly::F2;
   float *DR = sm + Ly::R0, *DO = sm + Ly::R1, *GC = sm + Ly::GC;
-  x.par(DK * DVT, [&](int e) {
+  par<DK * DVT>(x, [&](int e) {
     const int c = e / DVT, v = e - c * DVT;
     DS[c * VS + v] = a.dsf ? a.dsf[st_base + (size_t)c * DVF + v] : 0.f;
   });
   for (int ci = nck - 1; ci >= 0; --ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t slot = (size_t)(slot0 + ci) * H + h;
-    x.par(DK * DVT, [&](int e) {
-      const int c = e / DVT, v = e - c * DVT;
-      w.ckd[slot * DK * DVF + (size_t)c * DVF + c0 + v] = DS[c * VS + v];
-      if (e < DK) GC[e] = w.gc[slot * DK + e];
+    // checkpoint dS_C; load the chunk's Wb, Qs, BK, X, dO (rows L..C-1 zero) and gamma_C
+    par<NL>(x, [&](int e) {
+      if (e < DK * DVT) {
+        const int c = e / DVT, v = e - c * DVT;
+        w.ckd[slot * DK * DVF + (size_t)c * DVF + c0 + v] = DS[c * VS + v];
+      }
+      if (e < C * DK) {
+        const int i = e / DK, c = e - i * DK;
+        const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
+        WB[i * KS + c] = i < L ? CKDA_LDG(w.wb + o) : 0.f;
+        QS[i * KS + c] = i < L ? CKDA_LDG(w.qs + o) : 0.f;
+        BK[i * KS + c] = i < L ? CKDA_LDG(w.bk + o) : 0.f;
+      }
+      if (e < C * DVT) {
+        const int i = e / DVT, v = e - i * DVT;
+        const size_t o = ((size_t)(t0 + i) * H + h) * DVF + c0 + v;
+        DR[i * VS + v] = i < L ? CKDA_LDG(w.xt + o) : 0.f;
+        DO[i * VS + v] = i < L ? IOL::ldg(a.d_o + o) : 0.f;
+      }
+      if (e < DK) GC[e] = CKDA_LDG(w.gc + slot * DK + e);
     });
-    load_rows(x, WB, KS, w.wb, DK, 0, DK, t0, L, H, h);
-    load_rows(x, QS, KS, w.qs, DK, 0, DK, t0, L, H, h);
-    load_rows(x, BK, KS, w.bk, DK, 0, DK, t0, L, H, h);
-    load_rows(x, DR, VS, w.xt, DVF, c0, DVT, t0, L, H, h);
-    x.par(C * DVT, [&](int e) {
-      const int i = e / DVT, v = e - i * DVT;
-      DO[i * VS + v] = i < L ? IOL::ld(a.d_o + ((size_t)(t0 + i) * H + h) * DVF + c0 + v) : 0.f;
-    });
-    x.par(C * DVT, [&](int e) {  // dR = X + Wb dS_C
+    par<C * DVT>(x, [&](int e) {  // dR = X + Wb dS_C
       const int j = e / DVT, v = e - j * DVT;
       float s = DR[j * VS + v];
       for (int c = 0; c < DK; ++c) s += WB[j * KS + c] * DS[c * VS + v];
       DR[j * VS + v] = s;
       if (j < L) w.dr[((size_t)(t0 + j) * H + h) * DVF + c0 + v] = s;
     });
-    x.par(DK * DVT, [&](int e) {  // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
+    par<DK * DVT>(x, [&](int e) {  // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
       const int c = e / DVT, v = e - c * DVT;
       float s = GC[c] * DS[c * VS + v];
       for (int i = 0; i < C; ++i)
@@ -232,7 +242,7 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
     });
   }
   if (a.ds0) {
-    x.par(DK * DVT, [&](int e) {
+    par<DK * DVT>(x, [&](int e) {
       const int c = e / DVT, v = e - c * DVT;
       a.ds0[st_base + (size_t)c * DVF + v] = DS[c * VS + v];
     });
@@ -249,15 +259,20 @@ CKDA_PROG void grads_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
   const size_t sl = (size_t)slot * H + h;
   stage<X, IOL, IOT, Ly>(x, a, sm, h, c0, t0, L, true);
   chunk_gates<X, Ly>(x, sm);
-  x.par(DK * DVT, [&](int e) {
+  // the chunk's S, dS_C, Abar and its rows of U and dR (rows L..C-1 zero)
+  par<DK * DVT>(x, [&](int e) {
     const int c = e / DVT, v = e - c * DVT;
     const size_t o = sl * DK * DVF + (size_t)c * DVF + c0 + v;
-    sm[Ly::S + c * VS + v] = w.cks[o];
-    sm[Ly::DS + c * VS + v] = w.ckd[o];
-    if (e < C * C) sm[Ly::AB + (e / C) * CS + e % C] = w.ab[sl * C * C + e];
+    sm[Ly::S + c * VS + v] = CKDA_LDG(w.cks + o);
+    sm[Ly::DS + c * VS + v] = CKDA_LDG(w.ckd + o);
+    if (e < C * C) sm[Ly::AB + (e / C) * CS + e % C] = CKDA_LDG(w.ab + sl * C * C + e);
+    if (e < C * DVT) {
+      const int i = e / DVT, u = e - i * DVT;
+      const size_t r = ((size_t)(t0 + i) * H + h) * DVF + c0 + u;
+      sm[Ly::U + i * VS + u] = i < L ? CKDA_LDG(w.uu + r) : 0.f;
+      sm[Ly::DR + i * VS + u] = i < L ? CKDA_LDG(w.dr + r) : 0.f;
+    }
   });
-  load_rows(x, sm + Ly::U, VS, w.uu, DVF, c0, DVT, t0, L, H, h);
-  load_rows(x, sm + Ly::DR, VS, w.dr, DVF, c0, DVT, t0, L, H, h);
   chunk_khat_s<X, Ly>(x, sm);
   chunk_grads<X, IOL, IOT, DK, DVT>(x, a, sm, h, tile, t0, L);
 }

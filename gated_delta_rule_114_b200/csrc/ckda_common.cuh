@@ -50,6 +50,8 @@ __device__ __forceinline__ float key_rnorm(const GateArgs &g, float sumsq) {
 template <typename T> struct IO;
 template <> struct IO<float> {
   static __device__ __forceinline__ float ld(const float *p) { return *p; }
+  // read-only data (not written while the kernel runs)
+  static __device__ __forceinline__ float ldg(const float *p) { return __ldg(p); }
   static __device__ __forceinline__ void st(float *p, float x) { *p = x; }
   // 4 consecutive elements (16-byte aligned for float)
   static __device__ __forceinline__ float4 ld4(const float *p) {
@@ -62,6 +64,9 @@ template <> struct IO<float> {
 template <> struct IO<__nv_bfloat16> {
   static __device__ __forceinline__ float ld(const __nv_bfloat16 *p) {
     return __bfloat162float(*p);
+  }
+  static __device__ __forceinline__ float ldg(const __nv_bfloat16 *p) {
+    return __bfloat162float(__ldg(p));
   }
   static __device__ __forceinline__ void st(__nv_bfloat16 *p, float x) {
     *p = __float2bfloat16_rn(x);

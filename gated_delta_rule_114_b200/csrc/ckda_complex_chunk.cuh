@@ -21,8 +21,8 @@
 //        U = Utilde - W S, the outputs, the state update.
 // Complex numbers are interleaved (real, imaginary) fp32 pairs, in global and
 // in shared memory. The same executor contract as ckda_bwd_chunk.cuh: each
-// phase is x.par(n, f) over independent items, then a barrier, so the programs
-// also run as plain host loops in the tests.
+// phase is par<N>(x, f) over independent items, then a barrier, so the
+// programs also run as plain host loops in the tests.
 #pragma once
 
 #include <math.h>
@@ -33,6 +33,7 @@ namespace ckda {
 namespace cplx {
 
 using bwdc::C;
+using bwdc::par;
 
 struct cf {
   float r, i;
@@ -45,6 +46,8 @@ CKDA_PROG cf csub(cf a, cf b) { return cf{a.r - b.r, a.i - b.i}; }
 CKDA_PROG cf cscale(float s, cf a) { return cf{s * a.r, s * a.i}; }
 CKDA_PROG cf cconj(cf a) { return cf{a.r, -a.i}; }
 CKDA_PROG cf cld(const float *p) { return cf{p[0], p[1]}; }
+// read-only global data
+CKDA_PROG cf cldg(const float *p) { return cf{CKDA_LDG(p), CKDA_LDG(p + 1)}; }
 CKDA_PROG void cst(float *p, cf x) {
   p[0] = x.r;
   p[1] = x.i;
@@ -87,22 +90,22 @@ CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
   float *be = sm + Ly::BE;
   // stage q, k (complex), lambda = alpha (cos theta, sin theta), beta; rows
   // L..C-1 are inert (q = k = 0, lambda = 1, beta = 0)
-  x.par(C * DK, [&](int e) {
+  par<C * DK>(x, [&](int e) {
     const int i = e / DK, c = e - i * DK;
     cf qv{0.f, 0.f}, kv{0.f, 0.f}, lv{1.f, 0.f};
     if (i < L) {
       const size_t g = ((size_t)(t0 + i) * H + h) * DK + c;
-      qv = cld(a.q + 2 * g);
-      kv = cld(a.k + 2 * g);
-      const float al = a.alpha[g], th = a.theta[g];
+      qv = cldg(a.q + 2 * g);
+      kv = cldg(a.k + 2 * g);
+      const float al = CKDA_LDG(a.alpha + g), th = CKDA_LDG(a.theta + g);
       lv = cf{al * cosf(th), al * sinf(th)};
     }
     cst(sm + Ly::Q + i * KS + 2 * c, qv);
     cst(sm + Ly::K + i * KS + 2 * c, kv);
     cst(sm + Ly::LM + i * KS + 2 * c, lv);
-    if (e < C) be[e] = e < L ? a.beta[(size_t)(t0 + e) * H + h] : 0.f;
+    if (e < C) be[e] = e < L ? CKDA_LDG(a.beta + (size_t)(t0 + e) * H + h) : 0.f;
   });
-  x.par(DK, [&](int c) {  // gamma (prefix products), sigma (suffix products)
+  par<DK>(x, [&](int c) {  // gamma (prefix products), sigma (suffix products)
     cf g{1.f, 0.f};
     for (int i = 0; i < C; ++i) {
       g = cmul(g, cld(sm + Ly::LM + i * KS + 2 * c));
@@ -114,7 +117,7 @@ CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
       g = cmul(g, cld(sm + Ly::LM + j * KS + 2 * c));
     }
   });
-  x.par(C * C, [&](int e) {  // A (without beta) and M
+  par<C * C>(x, [&](int e) {  // A (without beta) and M
     const int i = e / C, j = e - i * C;
     cf ak{0.f, 0.f}, m{0.f, 0.f};
     if (j <= i) {
@@ -132,7 +135,7 @@ CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
     w.mm[(((size_t)slot * H + h) * C * C + e) * 2] = m.r;
     w.mm[(((size_t)slot * H + h) * C * C + e) * 2 + 1] = m.i;
   });
-  x.par(C, [&](int j) {  // column j of T = (I + diag(beta) A)^-1
+  par<C>(x, [&](int j) {  // column j of T = (I + diag(beta) A)^-1
     float *tt = sm + Ly::TT;
     for (int i = 0; i < j; ++i) cst(tt + i * CS + 2 * j, cf{0.f, 0.f});
     cst(tt + j * CS + 2 * j, cf{1.f, 0.f});
@@ -144,7 +147,7 @@ CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
     }
   });
   // W = T diag(beta) Khat, Kbar, Qhat; gamma_{C-1}
-  x.par(C * DK, [&](int e) {
+  par<C * DK>(x, [&](int e) {
     const int i = e / DK, c = e - i * DK;
     if (e < DK) {
       const cf g = cld(sm + Ly::GM + (C - 1) * KS + 2 * c);
@@ -165,13 +168,13 @@ CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
   });
   // Utilde = T diag(beta) conj(V), one column tile at a time
   for (int c0 = 0; c0 < DVF; c0 += DVT) {
-    x.par(C * DVT, [&](int e) {
+    par<C * DVT>(x, [&](int e) {
       const int i = e / DVT, v = e - i * DVT;
-      const cf vv = i < L ? cld(a.v + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2)
+      const cf vv = i < L ? cldg(a.v + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2)
                           : cf{0.f, 0.f};
       cst(sm + Ly::V + i * VS + 2 * v, cconj(vv));
     });
-    x.par(C * DVT, [&](int e) {
+    par<C * DVT>(x, [&](int e) {
       const int i = e / DVT, v = e - i * DVT;
       cf u{0.f, 0.f};
       for (int m = 0; m <= i; ++m)
@@ -202,37 +205,38 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;  // complex elements
   float *S = sm + Ly::S, *U = sm + Ly::U;
-  x.par(DK * DVT, [&](int e) {
+  par<DK * DVT>(x, [&](int e) {
     const int c = e / DVT, v = e - c * DVT;
+    // plain load: the final state may overwrite the initial one in place
     const cf s = a.s0 ? cld(a.s0 + (st_base + (size_t)c * DVF + v) * 2) : cf{0.f, 0.f};
     cst(S + c * VS + 2 * v, s);
   });
   for (int ci = 0; ci < nck; ++ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t sl = (size_t)(slot0 + ci) * H + h;
-    x.par(C * DK, [&](int e) {  // the chunk's factors; rows L..C-1 zero
+    par<C * DK>(x, [&](int e) {  // the chunk's factors; rows L..C-1 zero
       const int i = e / DK, c = e - i * DK;
       const size_t o = (((size_t)(t0 + i) * H + h) * DK + c) * 2;
       const bool in = i < L;
-      cst(sm + Ly::WT + i * KS + 2 * c, in ? cld(w.wt + o) : cf{0.f, 0.f});
-      cst(sm + Ly::KB + i * KS + 2 * c, in ? cld(w.kb + o) : cf{0.f, 0.f});
-      cst(sm + Ly::QH + i * KS + 2 * c, in ? cld(w.qh + o) : cf{0.f, 0.f});
+      cst(sm + Ly::WT + i * KS + 2 * c, in ? cldg(w.wt + o) : cf{0.f, 0.f});
+      cst(sm + Ly::KB + i * KS + 2 * c, in ? cldg(w.kb + o) : cf{0.f, 0.f});
+      cst(sm + Ly::QH + i * KS + 2 * c, in ? cldg(w.qh + o) : cf{0.f, 0.f});
       if (e < C * C)
-        cst(sm + Ly::M + (e / C) * CS + 2 * (e % C), cld(w.mm + (sl * C * C + e) * 2));
-      if (e < DK) cst(sm + Ly::GC + 2 * e, cld(w.gc + (sl * DK + e) * 2));
+        cst(sm + Ly::M + (e / C) * CS + 2 * (e % C), cldg(w.mm + (sl * C * C + e) * 2));
+      if (e < DK) cst(sm + Ly::GC + 2 * e, cldg(w.gc + (sl * DK + e) * 2));
     });
-    x.par(C * DVT, [&](int e) {  // U = Utilde - W S
+    par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
       const int i = e / DVT, v = e - i * DVT;
       if (i >= L) {
         cst(U + i * VS + 2 * v, cf{0.f, 0.f});
         return;
       }
-      cf u = cld(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
+      cf u = cldg(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
       for (int c = 0; c < DK; ++c)
         u = csub(u, cmul(cld(sm + Ly::WT + i * KS + 2 * c), cld(S + c * VS + 2 * v)));
       cst(U + i * VS + 2 * v, u);
     });
-    x.par(C * DVT, [&](int e) {  // o = conj(scale (Qhat S + M U))
+    par<C * DVT>(x, [&](int e) {  // o = conj(scale (Qhat S + M U))
       const int i = e / DVT, v = e - i * DVT;
       if (i >= L) return;
       cf s{0.f, 0.f};
@@ -242,7 +246,7 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
         s = cadd(s, cmul(cld(sm + Ly::M + i * CS + 2 * j), cld(U + j * VS + 2 * v)));
       cst(a.o + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2, cconj(cscale(a.scale, s)));
     });
-    x.par(DK * DVT, [&](int e) {  // S <- diag(gamma_{C-1}) S + Kbar^T U
+    par<DK * DVT>(x, [&](int e) {  // S <- diag(gamma_{C-1}) S + Kbar^T U
       const int c = e / DVT, v = e - c * DVT;
       cf s = cmul(cld(sm + Ly::GC + 2 * c), cld(S + c * VS + 2 * v));
       for (int i = 0; i < C; ++i)
@@ -251,7 +255,7 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
     });
   }
   if (a.sf) {
-    x.par(DK * DVT, [&](int e) {
+    par<DK * DVT>(x, [&](int e) {
       const int c = e / DVT, v = e - c * DVT;
       cst(a.sf + (st_base + (size_t)c * DVF + v) * 2, cld(S + c * VS + 2 * v));
     });

@@ -19,14 +19,15 @@
 namespace {
 
 struct HostExec {
-  template <class F>
-  void par(int n, F f) {
-    for (int i = 0; i < n; ++i) f(i);
+  template <int N, class F>
+  void run(F f) {
+    for (int i = 0; i < N; ++i) f(i);
   }
 };
 
 struct HostIO {
   static float ld(const float *p) { return *p; }
+  static float ldg(const float *p) { return *p; }
   static void st(float *p, float x) { *p = x; }
 };
 

@@ -21,9 +21,9 @@
 namespace {
 
 struct HostExec {
-  template <class F>
-  void par(int n, F f) {
-    for (int i = 0; i < n; ++i) f(i);
+  template <int N, class F>
+  void run(F f) {
+    for (int i = 0; i < N; ++i) f(i);
   }
 };
 
