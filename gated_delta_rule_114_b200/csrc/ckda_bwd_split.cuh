@@ -135,6 +135,51 @@ struct ScanLayout {
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
+// The scans' state update over one chunk, in 4 x 4 register tiles (each item
+// owns rows 4cg..4cg+3 and columns 4vg..4vg+3 of the d_k x DVT tile):
+//   Z[c][v] <- g[c] Z[c][v] + sum_i A[i][c] B[i][v]   (minus sum_i A2[i][c] B2[i][v]
+// when A2 is given), rows of A, A2 with stride KS and of B, B2 and Z with stride VS.
+template <int DK, int DVT, class X>
+CKDA_PROG void state_update(X &x, float *Z, const float *g, const float *A, const float *B,
+                            const float *A2, const float *B2) {
+  constexpr int KS = DK + 1, VS = DVT + 1, NV = DVT / 4;
+  static_assert(DK % 4 == 0 && DVT % 4 == 0, "4 x 4 tiles");
+  par<(DK / 4) * NV>(x, [&](int e) {
+    const int c0 = 4 * (e / NV), v0 = 4 * (e % NV);
+    float acc[4][4];
+CKDA_UNROLL
+    for (int r = 0; r < 4; ++r)
+CKDA_UNROLL
+      for (int j = 0; j < 4; ++j) acc[r][j] = g[c0 + r] * Z[(c0 + r) * VS + v0 + j];
+CKDA_UNROLL
+    for (int i = 0; i < C; ++i) {
+      float av[4], bv[4];
+CKDA_UNROLL
+      for (int r = 0; r < 4; ++r) av[r] = A[i * KS + c0 + r];
+CKDA_UNROLL
+      for (int j = 0; j < 4; ++j) bv[j] = B[i * VS + v0 + j];
+CKDA_UNROLL
+      for (int r = 0; r < 4; ++r)
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) acc[r][j] += av[r] * bv[j];
+      if (A2) {
+CKDA_UNROLL
+        for (int r = 0; r < 4; ++r) av[r] = A2[i * KS + c0 + r];
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) bv[j] = B2[i * VS + v0 + j];
+CKDA_UNROLL
+        for (int r = 0; r < 4; ++r)
+CKDA_UNROLL
+          for (int j = 0; j < 4; ++j) acc[r][j] -= av[r] * bv[j];
+      }
+    }
+CKDA_UNROLL
+    for (int r = 0; r < 4; ++r)
+CKDA_UNROLL
+      for (int j = 0; j < 4; ++j) Z[(c0 + r) * VS + v0 + j] = acc[r][j];
+  });
+}
+
 template <class X, class IOL, typename IOT, int DK, int DVT>
 CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
                              int n, int tile, int bos, int eos, int slot0) {
@@ -178,12 +223,8 @@ CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
       U[i * VS + v] = s;
       if (i < L) w.uu[((size_t)(t0 + i) * H + h) * DVF + c0 + v] = s;
     });
-    par<DK * DVT>(x, [&](int e) {  // S <- diag(gamma_C) S + Kbar^T U
-      const int c = e / DVT, v = e - c * DVT;
-      float s = GC[c] * S[c * VS + v];
-      for (int i = 0; i < C; ++i) s += KB[i * KS + c] * U[i * VS + v];
-      S[c * VS + v] = s;
-    });
+    // S <- diag(gamma_C) S + Kbar^T U
+    state_update<DK, DVT>(x, S, GC, KB, U, nullptr, nullptr);
   }
 }
 
@@ -233,13 +274,8 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
       DR[j * VS + v] = s;
       if (j < L) w.dr[((size_t)(t0 + j) * H + h) * DVF + c0 + v] = s;
     });
-    par<DK * DVT>(x, [&](int e) {  // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
-      const int c = e / DVT, v = e - c * DVT;
-      float s = GC[c] * DS[c * VS + v];
-      for (int i = 0; i < C; ++i)
-        s += QS[i * KS + c] * DO[i * VS + v] - BK[i * KS + c] * DR[i * VS + v];
-      DS[c * VS + v] = s;
-    });
+    // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
+    state_update<DK, DVT>(x, DS, GC, QS, DO, BK, DR);
   }
   if (a.ds0) {
     par<DK * DVT>(x, [&](int e) {
