@@ -75,11 +75,10 @@ struct Layout {
   static constexpr int KS = DK + 1;   // C x DK rows
   static constexpr int VS = DVT + 1;  // C x DVT and DK x DVT rows
   static constexpr int CS = C + 1;    // C x C rows
-  // C x DK: inputs q, k, alpha; gamma, sigma; dq, dk accumulators; the
-  // gate-gradient coefficients of the chunk entry (E0) and exit (EX)
+  // C x DK: inputs q, k, alpha; gamma, sigma; the gate-gradient coefficients
+  // of the chunk entry (E0) and exit (EX)
   static constexpr int Q = 0, K = Q + C * KS, AL = K + C * KS, GM = AL + C * KS,
-                       SG = GM + C * KS, DQ = SG + C * KS, DKK = DQ + C * KS,
-                       E0 = DKK + C * KS, EX = E0 + C * KS;
+                       SG = GM + C * KS, E0 = SG + C * KS, EX = E0 + C * KS;
   // C x DVT: v, dO, Khat S then w, U, dR
   static constexpr int V = EX + C * KS, DO = V + C * VS, KSW = DO + C * VS, U = KSW + C * VS,
                        DR = U + C * VS;
@@ -290,29 +289,24 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
     sm[Ly::DM + i * CS + j] = scale * m;
     sm[Ly::DA + i * CS + j] = j < i ? -be[i] * d : 0.f;
   });
-  // the state-side terms: dQhat = scale dO S^T, dKhat = -diag(beta) dR S^T,
-  // dKbar = U dS_C^T; dq and dk start from them, E0 and EX keep the gate parts
-  par<C * DK>(x, [&](int e) {
-    const int i = e / DK, c = e - i * DK;
-    float xq = 0.f, xk = 0.f, xb = 0.f;
-    for (int v = 0; v < DVT; ++v) {
-      const float s = S[c * VS + v];
-      xq += sm[Ly::DO + i * VS + v] * s;
-      xk += sm[Ly::DR + i * VS + v] * s;
-      xb += sm[Ly::U + i * VS + v] * DS[c * VS + v];
-    }
-    const float dqh = scale * xq, dkh = -be[i] * xk;
-    const float gm = sm[Ly::GM + i * KS + c], sg = sm[Ly::SG + i * KS + c];
-    sm[Ly::DQ + i * KS + c] = gm * dqh;
-    sm[Ly::DKK + i * KS + c] = gm * dkh + sg * xb;
-    sm[Ly::E0 + i * KS + c] = sm[Ly::Q + i * KS + c] * dqh + sm[Ly::K + i * KS + c] * dkh;
-    sm[Ly::EX + i * KS + c] = sm[Ly::K + i * KS + c] * xb;
-  });
-  // gated Gram terms of dq and dk; write this tile's dq, dk partials
+  // per (row r, channel c): the state-side terms dQhat = scale dO S^T,
+  // dKhat = -diag(beta) dR S^T, dKbar = U dS_C^T (E0 and EX keep their gate
+  // parts), then the gated Gram terms of dq and dk; this tile's dq, dk partials
   par<C * DK>(x, [&](int e) {
     const int r = e / DK, c = e - r * DK;
     const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
-    float dq = sm[Ly::DQ + r * KS + c], dk = sm[Ly::DKK + r * KS + c];
+    float xq = 0.f, xk = 0.f, xb = 0.f;
+    for (int v = 0; v < DVT; ++v) {
+      const float sv = S[c * VS + v];
+      xq += sm[Ly::DO + r * VS + v] * sv;
+      xk += sm[Ly::DR + r * VS + v] * sv;
+      xb += sm[Ly::U + r * VS + v] * DS[c * VS + v];
+    }
+    const float dqh = scale * xq, dkh = -be[r] * xk;
+    const float gm = sm[Ly::GM + r * KS + c], sg = sm[Ly::SG + r * KS + c];
+    sm[Ly::E0 + r * KS + c] = qq[r * KS + c] * dqh + kk[r * KS + c] * dkh;
+    sm[Ly::EX + r * KS + c] = kk[r * KS + c] * xb;
+    float dq = gm * dqh, dk = gm * dkh + sg * xb;
     float g = 1.f;  // G_{r<-j}
     dq += sm[Ly::DM + r * CS + r] * kk[r * KS + c];
     for (int j = r - 1; j >= 0; --j) {

@@ -84,7 +84,7 @@ bwd_scan_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ 
 }
 
 template <typename IOT, int DK, int DVT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 bwd_grads_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ cu, int N,
                  int T, int T_total, unsigned int *err) {
   extern __shared__ float sm[];
