@@ -161,26 +161,39 @@ CKDA_PROG void chunk_gates(X &x, float *sm) {
   });
 }
 
-// Abar and M (with M only when want_m); T = (I + diag(beta) Abar)^-1
+// Abar and M, then T = (I + diag(beta) Abar)^-1. A (row i, column j, channel
+// group g) item sums channels g, g + NG, g + 2 NG, ... (strided so that the
+// groups of one pair read different banks); a second phase adds the NG
+// partials in a fixed order. Needs Ly::PG, 2 C C NG floats.
 template <class X, class Ly>
-CKDA_PROG void chunk_grams_solve(X &x, float *sm, bool want_m) {
-  constexpr int DK = Ly::dk, KS = Ly::KS, CS = Ly::CS;
+CKDA_PROG void chunk_grams_solve(X &x, float *sm) {
+  constexpr int DK = Ly::dk, KS = Ly::KS, CS = Ly::CS, NG = Ly::NG;
   const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q, *be = sm + Ly::BE;
-  par<C * C>(x, [&](int e) {
-    const int i = e / C, j = e - i * C;
+  par<C * C * NG>(x, [&](int e) {
+    const int g = e % NG, p = e / NG, i = p / C, j = p - i * C;
     float ab = 0.f, m = 0.f;
     if (j <= i) {
-      for (int c = 0; c < DK; ++c) {
-        float g = 1.f;
-        for (int s = j + 1; s <= i; ++s) g *= al[s * KS + c];
-        const float gk = g * kk[j * KS + c];
+      for (int c = g; c < DK; c += NG) {
+        float gp = 1.f;
+        for (int s = j + 1; s <= i; ++s) gp *= al[s * KS + c];
+        const float gk = gp * kk[j * KS + c];
         ab += kk[i * KS + c] * gk;
         m += qq[i * KS + c] * gk;
       }
-      if (j == i) ab = 0.f;
     }
-    sm[Ly::AB + i * CS + j] = ab;
-    if (want_m) sm[Ly::M + i * CS + j] = m;
+    sm[Ly::PG + 2 * e] = ab;
+    sm[Ly::PG + 2 * e + 1] = m;
+  });
+  par<C * C>(x, [&](int e) {
+    const int i = e / C, j = e - i * C;
+    float ab = 0.f, m = 0.f;
+CKDA_UNROLL
+    for (int g = 0; g < NG; ++g) {
+      ab += sm[Ly::PG + 2 * (e * NG + g)];
+      m += sm[Ly::PG + 2 * (e * NG + g) + 1];
+    }
+    sm[Ly::AB + i * CS + j] = j < i ? ab : 0.f;
+    sm[Ly::M + i * CS + j] = m;
   });
   par<C>(x, [&](int j) {  // column j of T by forward substitution
     float *tt = sm + Ly::TT;

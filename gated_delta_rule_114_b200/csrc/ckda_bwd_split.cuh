@@ -57,7 +57,8 @@ struct PrepLayout {
                        SG = GM + C * KS;
   static constexpr int V = SG + C * KS, DO = V + C * VS, RD = DO + C * VS;
   static constexpr int AB = RD + C * VS, M = AB + C * CS, TT = M + C * CS;
-  static constexpr int BE = TT + C * CS;
+  static constexpr int NG = 4;  // channel groups of the Gram phase
+  static constexpr int PG = TT + C * CS, BE = PG + 2 * C * C * NG;
   static constexpr int FLOATS = BE + C;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
@@ -72,7 +73,7 @@ CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *s
   const float *be = sm + Ly::BE, *tt = sm + Ly::TT;
   stage<X, IOL, IOT, Ly>(x, a, sm, h, 0, t0, L, true);
   chunk_gates<X, Ly>(x, sm);
-  chunk_grams_solve<X, Ly>(x, sm, true);
+  chunk_grams_solve<X, Ly>(x, sm);
   // the d_k-wide factors, gamma_C and Abar
   par<C * DK>(x, [&](int e) {
     const int i = e / DK, c = e - i * DK;

@@ -75,8 +75,10 @@ struct PrepLayout {
   // C x DK complex: q, k, lambda, gamma, sigma; C x DVT complex: conj(v)
   static constexpr int Q = 0, K = Q + C * KS, LM = K + C * KS, GM = LM + C * KS,
                        SG = GM + C * KS, V = SG + C * KS;
-  // C x C complex: A, M, T; beta [C]
-  static constexpr int A = V + C * VS, M = A + C * CS, TT = M + C * CS, BE = TT + C * CS;
+  // C x C complex: A, M, T; the Gram phase's per-group partials; beta [C]
+  static constexpr int NG = 2;  // channel groups of the Gram phase
+  static constexpr int A = V + C * VS, M = A + C * CS, TT = M + C * CS, PG = TT + C * CS,
+                       BE = PG + 4 * C * C * NG;
   static constexpr int FLOATS = BE + C;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
@@ -117,19 +119,33 @@ CKDA_PROG void prep_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
       g = cmul(g, cld(sm + Ly::LM + j * KS + 2 * c));
     }
   });
-  par<C * C>(x, [&](int e) {  // A (without beta) and M
-    const int i = e / C, j = e - i * C;
+  // A (without beta) and M: item (pair, channel group g) sums channels g, g + NG, ...;
+  // then the NG partials are added in a fixed order
+  constexpr int NG = Ly::NG;
+  par<C * C * NG>(x, [&](int e) {
+    const int g = e % NG, p = e / NG, i = p / C, j = p - i * C;
     cf ak{0.f, 0.f}, m{0.f, 0.f};
     if (j <= i) {
-      for (int c = 0; c < DK; ++c) {
-        cf g{1.f, 0.f};
-        for (int s = j + 1; s <= i; ++s) g = cmul(g, cld(sm + Ly::LM + s * KS + 2 * c));
-        const cf gk = cmul(g, cld(sm + Ly::K + j * KS + 2 * c));
+      for (int c = g; c < DK; c += NG) {
+        cf gp{1.f, 0.f};
+        for (int s = j + 1; s <= i; ++s) gp = cmul(gp, cld(sm + Ly::LM + s * KS + 2 * c));
+        const cf gk = cmul(gp, cld(sm + Ly::K + j * KS + 2 * c));
         ak = cadd(ak, cmulc(cld(sm + Ly::K + i * KS + 2 * c), gk));
         m = cadd(m, cmulc(cld(sm + Ly::Q + i * KS + 2 * c), gk));
       }
-      if (j == i) ak = cf{0.f, 0.f};
     }
+    cst(sm + Ly::PG + 4 * e, ak);
+    cst(sm + Ly::PG + 4 * e + 2, m);
+  });
+  par<C * C>(x, [&](int e) {
+    const int i = e / C, j = e - i * C;
+    cf ak{0.f, 0.f}, m{0.f, 0.f};
+CKDA_UNROLL
+    for (int g = 0; g < NG; ++g) {
+      ak = cadd(ak, cld(sm + Ly::PG + 4 * (e * NG + g)));
+      m = cadd(m, cld(sm + Ly::PG + 4 * (e * NG + g) + 2));
+    }
+    if (j >= i) ak = cf{0.f, 0.f};
     cst(sm + Ly::A + i * CS + 2 * j, ak);
     cst(sm + Ly::M + i * CS + 2 * j, m);
     w.mm[(((size_t)slot * H + h) * C * C + e) * 2] = m.r;
