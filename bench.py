@@ -247,6 +247,75 @@ def cpu_baseline_prefill(w, inp_cpu, target_s=12.0):
                        % (h, H, T, tok_heads, dt, H))}
 
 
+def chunked_legs(args, w, inp_cpu, T_total, H, N, dk, dv, stream, pk, world):
+    """The chunked backward and complex-gate entry points on the bench's shape,
+    timed on this rank alone (no collective), after every other leg. Any
+    failure is recorded in the returned dict instead of ending the run."""
+    out = {}
+    try:
+        dev = {key: (val.cuda() if isinstance(val, torch.Tensor) else val)
+               for key, val in inp_cpu.items()}
+        if args.bwd_impl != "chunked":
+            bg = make_bwd_grads(w, T_total, H, N)
+            bdo, bdsf = bg["d_o"].cuda(), bg["d_final_state"].cuda()
+            bout = [torch.empty_like(dev["q"]), torch.empty_like(dev["k"]),
+                    torch.empty_like(dev["v"]), torch.empty_like(dev["alpha"]),
+                    torch.empty_like(dev["beta"]),
+                    torch.empty((N, H, dk, dv), dtype=torch.float32, device="cuda")]
+            bws = torch.empty(ckda.ckda_bwd_workspace_bytes(N, T_total, H, dk, dv, True, True),
+                              dtype=torch.uint8, device="cuda")
+
+            def bstep():
+                ckda.ckda_bwd(dev["q"], dev["k"], dev["v"], dev["alpha"], dev["beta"],
+                              dev["initial_state"], bdo, bdsf, *bout, dev["cu_seqlens"], None,
+                              stream=stream, workspace=bws, chunked=True)
+
+            ms = time_loop(bstep, args.bwd_steps, 3, stream)
+            if ckda.ckda_last_error() != ckda.CKDA_OK:
+                raise RuntimeError("kernel reported an error")
+            nb = bwd_bytes(inp_cpu)
+            out["backward_chunked"] = {
+                "entry_point": "ckda_bwd_chunked", "ms_per_step": ms,
+                "tokens_per_s": T_total / (ms / 1e3), "steps": args.bwd_steps, "warmup": 3,
+                "roofline": {"bound": "hbm", "achieved": nb / (ms / 1e3) / 1e9,
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                             "algorithmic_bytes_per_launch": nb},
+                "timing": "this rank alone", "gpu_launches": 5 * args.bwd_steps}
+            del bws, bout, bdo, bdsf
+        if args.complex_impl != "chunked":
+            cin = {key: val.cuda() for key, val in
+                   make_complex_inputs(w, inp_cpu["cu_seqlens"], H).items()}
+            co = torch.empty((T_total, H, dv), dtype=torch.complex64, device="cuda")
+            csf = torch.empty((N, H, dk, dv), dtype=torch.complex64, device="cuda")
+            cws = torch.empty(ckda.ckda_fwd_complex_chunked_workspace_bytes(N, T_total, H, dk, dv,
+                                                                             True),
+                              dtype=torch.uint8, device="cuda")
+
+            def cstep():
+                ckda.ckda_fwd_complex(cin["q"], cin["k"], cin["v"], cin["alpha"], cin["theta"],
+                                      cin["beta"], cin["initial_state"], csf, co,
+                                      cin["cu_seqlens"], None, stream=stream, chunked=True,
+                                      workspace=cws)
+
+            ms = time_loop(cstep, args.complex_steps, 3, stream)
+            if ckda.ckda_last_error() != ckda.CKDA_OK:
+                raise RuntimeError("kernel reported an error")
+            nb = complex_bytes(T_total, H, N, dk, dv)
+            out["complex_gate_chunked"] = {
+                "entry_point": "ckda_fwd_complex_chunked", "ms_per_step": ms,
+                "tokens_per_s": T_total / (ms / 1e3), "steps": args.complex_steps, "warmup": 3,
+                "roofline": {"bound": "hbm", "achieved": nb / (ms / 1e3) / 1e9,
+                             "peak": pk["hbm_gbs"], "unit": "GB/s",
+                             "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
+                             "algorithmic_bytes_per_launch": nb},
+                "timing": "this rank alone", "gpu_launches": 2 * args.complex_steps}
+            del cws, cin, co, csf
+    except Exception as e:  # recorded, not fatal: these legs come after every other one
+        out["chunked_legs_error"] = "%s: %s" % (type(e).__name__, e)
+    return out
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -307,6 +376,8 @@ def main():
                     help="complex-gate entry point: ckda_fwd_complex (token-serial) or "
                          "ckda_fwd_complex_chunked")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-chunked-legs", action="store_true",
+                    help="skip the extra timing of the chunked backward and complex paths")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -519,6 +590,10 @@ def main():
                            "algorithmic_bytes_per_launch": dbytes},
               "gpu_launches": args.decode_steps, "clocks": dclk.summary()}
 
+    extra = {}
+    if not args.no_chunked_legs:
+        extra = chunked_legs(args, w, inp_cpu, T_total, H, N, dk, dv, stream, pk, world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_prefill(w, inp_cpu)
@@ -543,6 +618,7 @@ def main():
         "gpu_launches": 3 * args.steps, "clocks": clk.summary(), "decode": decode,
         "prefill_fused_prologue": gated, "backward": backward, "complex_gate": complex_gate,
     }
+    line.update(extra)
     print(json.dumps(line), flush=True)
     return 0
 
