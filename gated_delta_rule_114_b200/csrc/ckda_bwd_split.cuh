@@ -132,9 +132,48 @@ struct ScanLayout {
   static constexpr int KS = DK + 1, VS = DVT + 1;
   static constexpr int S = 0, F0 = S + DK * VS, F1 = F0 + C * KS, F2 = F1 + C * KS,
                        R0 = F2 + C * KS, R1 = R0 + C * VS, GC = R1 + C * VS;
-  static constexpr int FLOATS = GC + DK;
+  static constexpr int P = GC + DK;  // partial products, C x DVT x 4
+  static constexpr int FLOATS = P + 4 * C * DVT;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
+
+// Partial products of the C x DVT result A B (A: C x DK rows of stride DK + 1;
+// B: the DK x DVT state tile, rows of stride DVT + 1): item (row pair, 4
+// columns, quarter q) sums channels q, q + 4, q + 8, ... in a 2 x 4 register
+// tile into P; rows_state_sum adds the four quarters in a fixed order.
+template <int DK, int DVT, class X>
+CKDA_PROG void rows_state_partials(X &x, float *P, const float *A, const float *B) {
+  constexpr int KS = DK + 1, VS = DVT + 1, NV = DVT / 4;
+  par<(C / 2) * NV * 4>(x, [&](int e) {
+    const int q = e % 4, rest = e / 4, vg = rest % NV, ip = rest / NV;
+    const int i0 = 2 * ip, v0 = 4 * vg;
+    float acc[2][4] = {};
+    for (int c = q; c < DK; c += 4) {
+      const float a0 = A[i0 * KS + c], a1 = A[(i0 + 1) * KS + c];
+CKDA_UNROLL
+      for (int j = 0; j < 4; ++j) {
+        const float b = B[c * VS + v0 + j];
+        acc[0][j] += a0 * b;
+        acc[1][j] += a1 * b;
+      }
+    }
+CKDA_UNROLL
+    for (int r = 0; r < 2; ++r)
+CKDA_UNROLL
+      for (int j = 0; j < 4; ++j) P[(e * 2 + r) * 4 + j] = acc[r][j];
+  });
+}
+
+// (A B)[i][v] from rows_state_partials' P
+template <int DVT>
+CKDA_PROG float rows_state_sum(const float *P, int i, int v) {
+  constexpr int NV = DVT / 4;
+  const int e0 = (((i / 2) * NV + v / 4) * 4) * 2 + (i % 2), j = v % 4;
+  float s = 0.f;
+CKDA_UNROLL
+  for (int q = 0; q < 4; ++q) s += P[(e0 + 2 * q) * 4 + j];
+  return s;
+}
 
 // The scans' state update over one chunk, in 4 x 4 register tiles (each item
 // owns rows 4cg..4cg+3 and columns 4vg..4vg+3 of the d_k x DVT tile):
@@ -217,10 +256,10 @@ CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
       }
       if (e < DK) GC[e] = CKDA_LDG(w.gc + slot * DK + e);
     });
+    rows_state_partials<DK, DVT>(x, sm + Ly::P, WT, S);
     par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
       const int i = e / DVT, v = e - i * DVT;
-      float s = U[i * VS + v];
-      for (int c = 0; c < DK; ++c) s -= WT[i * KS + c] * S[c * VS + v];
+      const float s = U[i * VS + v] - rows_state_sum<DVT>(sm + Ly::P, i, v);
       U[i * VS + v] = s;
       if (i < L) w.uu[((size_t)(t0 + i) * H + h) * DVF + c0 + v] = s;
     });
@@ -268,10 +307,10 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
       }
       if (e < DK) GC[e] = CKDA_LDG(w.gc + slot * DK + e);
     });
+    rows_state_partials<DK, DVT>(x, sm + Ly::P, WB, DS);
     par<C * DVT>(x, [&](int e) {  // dR = X + Wb dS_C
       const int j = e / DVT, v = e - j * DVT;
-      float s = DR[j * VS + v];
-      for (int c = 0; c < DK; ++c) s += WB[j * KS + c] * DS[c * VS + v];
+      const float s = DR[j * VS + v] + rows_state_sum<DVT>(sm + Ly::P, j, v);
       DR[j * VS + v] = s;
       if (j < L) w.dr[((size_t)(t0 + j) * H + h) * DVF + c0 + v] = s;
     });

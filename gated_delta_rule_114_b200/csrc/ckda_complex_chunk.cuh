@@ -208,7 +208,9 @@ struct ScanLayout {
   // C x C complex M; gamma_{C-1} [DK] complex
   static constexpr int S = 0, WT = S + DK * VS, KB = WT + C * KS, QH = KB + C * KS,
                        U = QH + C * KS, M = U + C * VS, GC = M + C * CS;
-  static constexpr int FLOATS = GC + 2 * DK;
+  // partial products of W S and Qhat S: 4 quarters of C x DVT complex each
+  static constexpr int PW = GC + 2 * DK, PQ = PW + 8 * C * DVT;
+  static constexpr int FLOATS = PQ + 8 * C * DVT;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
@@ -216,7 +218,7 @@ template <class X, int DK, int DVT>
 CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, int n, int tile,
                             int bos, int eos, int slot0) {
   using Ly = ScanLayout<DK, DVT>;
-  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
+  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS, NV = DVT / 4;
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;  // complex elements
@@ -241,33 +243,88 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
         cst(sm + Ly::M + (e / C) * CS + 2 * (e % C), cldg(w.mm + (sl * C * C + e) * 2));
       if (e < DK) cst(sm + Ly::GC + 2 * e, cldg(w.gc + (sl * DK + e) * 2));
     });
+    // W S and Qhat S in one pass over S: item (row pair, 4 columns, quarter q)
+    // sums channels q, q + 4, ... in 2 x 4 complex register tiles
+    par<(C / 2) * NV * 4>(x, [&](int e) {
+      const int q = e % 4, rest = e / 4, vg = rest % NV, ip = rest / NV;
+      const int i0 = 2 * ip, v0 = 4 * vg;
+      cf aw[2][4], aq[2][4];
+CKDA_UNROLL
+      for (int r = 0; r < 2; ++r)
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) aw[r][j] = aq[r][j] = cf{0.f, 0.f};
+      for (int c = q; c < DK; c += 4) {
+        const cf w0 = cld(sm + Ly::WT + i0 * KS + 2 * c);
+        const cf w1 = cld(sm + Ly::WT + (i0 + 1) * KS + 2 * c);
+        const cf q0 = cld(sm + Ly::QH + i0 * KS + 2 * c);
+        const cf q1 = cld(sm + Ly::QH + (i0 + 1) * KS + 2 * c);
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) {
+          const cf sv = cld(S + c * VS + 2 * (v0 + j));
+          aw[0][j] = cadd(aw[0][j], cmul(w0, sv));
+          aw[1][j] = cadd(aw[1][j], cmul(w1, sv));
+          aq[0][j] = cadd(aq[0][j], cmul(q0, sv));
+          aq[1][j] = cadd(aq[1][j], cmul(q1, sv));
+        }
+      }
+CKDA_UNROLL
+      for (int r = 0; r < 2; ++r)
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) {
+          cst(sm + Ly::PW + ((e * 2 + r) * 4 + j) * 2, aw[r][j]);
+          cst(sm + Ly::PQ + ((e * 2 + r) * 4 + j) * 2, aq[r][j]);
+        }
+    });
+    // the four quarters of (row i, column v) in a fixed order
+    auto quarters = [&](int base, int i, int v) {
+      const int e0 = (((i / 2) * NV + v / 4) * 4) * 2 + (i % 2), j = v % 4;
+      cf s{0.f, 0.f};
+CKDA_UNROLL
+      for (int q4 = 0; q4 < 4; ++q4) s = cadd(s, cld(sm + base + ((e0 + 2 * q4) * 4 + j) * 2));
+      return s;
+    };
     par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
       const int i = e / DVT, v = e - i * DVT;
       if (i >= L) {
         cst(U + i * VS + 2 * v, cf{0.f, 0.f});
         return;
       }
-      cf u = cldg(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
-      for (int c = 0; c < DK; ++c)
-        u = csub(u, cmul(cld(sm + Ly::WT + i * KS + 2 * c), cld(S + c * VS + 2 * v)));
-      cst(U + i * VS + 2 * v, u);
+      const cf u = cldg(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
+      cst(U + i * VS + 2 * v, csub(u, quarters(Ly::PW, i, v)));
     });
     par<C * DVT>(x, [&](int e) {  // o = conj(scale (Qhat S + M U))
       const int i = e / DVT, v = e - i * DVT;
       if (i >= L) return;
-      cf s{0.f, 0.f};
-      for (int c = 0; c < DK; ++c)
-        s = cadd(s, cmul(cld(sm + Ly::QH + i * KS + 2 * c), cld(S + c * VS + 2 * v)));
+      cf s = quarters(Ly::PQ, i, v);
       for (int j = 0; j <= i; ++j)
         s = cadd(s, cmul(cld(sm + Ly::M + i * CS + 2 * j), cld(U + j * VS + 2 * v)));
       cst(a.o + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2, cconj(cscale(a.scale, s)));
     });
-    par<DK * DVT>(x, [&](int e) {  // S <- diag(gamma_{C-1}) S + Kbar^T U
-      const int c = e / DVT, v = e - c * DVT;
-      cf s = cmul(cld(sm + Ly::GC + 2 * c), cld(S + c * VS + 2 * v));
-      for (int i = 0; i < C; ++i)
-        s = cadd(s, cmul(cld(sm + Ly::KB + i * KS + 2 * c), cld(U + i * VS + 2 * v)));
-      cst(S + c * VS + 2 * v, s);
+    // S <- diag(gamma_{C-1}) S + Kbar^T U, in 2 x 4 complex register tiles
+    par<(DK / 2) * NV>(x, [&](int e) {
+      const int cg = e / NV, vg = e - cg * NV, cc = 2 * cg, v0 = 4 * vg;
+      cf acc[2][4];
+CKDA_UNROLL
+      for (int r = 0; r < 2; ++r) {
+        const cf g = cld(sm + Ly::GC + 2 * (cc + r));
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) acc[r][j] = cmul(g, cld(S + (cc + r) * VS + 2 * (v0 + j)));
+      }
+CKDA_UNROLL
+      for (int i = 0; i < C; ++i) {
+        const cf k0 = cld(sm + Ly::KB + i * KS + 2 * cc);
+        const cf k1 = cld(sm + Ly::KB + i * KS + 2 * (cc + 1));
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) {
+          const cf uv = cld(U + i * VS + 2 * (v0 + j));
+          acc[0][j] = cadd(acc[0][j], cmul(k0, uv));
+          acc[1][j] = cadd(acc[1][j], cmul(k1, uv));
+        }
+      }
+CKDA_UNROLL
+      for (int r = 0; r < 2; ++r)
+CKDA_UNROLL
+        for (int j = 0; j < 4; ++j) cst(S + (cc + r) * VS + 2 * (v0 + j), acc[r][j]);
     });
   }
   if (a.sf) {
