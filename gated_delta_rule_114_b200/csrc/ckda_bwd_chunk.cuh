@@ -302,42 +302,70 @@ CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile,
     sm[Ly::DM + i * CS + j] = scale * m;
     sm[Ly::DA + i * CS + j] = j < i ? -be[i] * d : 0.f;
   });
-  // per (row r, channel c): the state-side terms dQhat = scale dO S^T,
-  // dKhat = -diag(beta) dR S^T, dKbar = U dS_C^T (E0 and EX keep their gate
-  // parts), then the gated Gram terms of dq and dk; this tile's dq, dk partials
-  par<C * DK>(x, [&](int e) {
-    const int r = e / DK, c = e - r * DK;
+  // per (row r, channels cq + t DK/4 for t < 4): the state-side terms
+  // dQhat = scale dO S^T, dKhat = -diag(beta) dR S^T, dKbar = U dS_C^T (E0 and EX
+  // keep their gate parts), then the gated Gram terms of dq and dk; this tile's
+  // dq, dk partials. The row's dO, dR, U, dM and dAbar values serve all four
+  // channels; channels at stride DK/4 keep a warp's accesses on distinct banks.
+  constexpr int NQ = DK / 4;
+  par<C * NQ>(x, [&](int e) {
+    const int r = e / NQ, cq = e - r * NQ;
     const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
-    float xq = 0.f, xk = 0.f, xb = 0.f;
+    float xq[4] = {}, xk[4] = {}, xb[4] = {};
     for (int v = 0; v < DVT; ++v) {
-      const float sv = S[c * VS + v];
-      xq += sm[Ly::DO + r * VS + v] * sv;
-      xk += sm[Ly::DR + r * VS + v] * sv;
-      xb += sm[Ly::U + r * VS + v] * DS[c * VS + v];
+      const float dov = sm[Ly::DO + r * VS + v], drv = sm[Ly::DR + r * VS + v];
+      const float uv = sm[Ly::U + r * VS + v];
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        const int c = cq + t * NQ;
+        const float sv = S[c * VS + v];
+        xq[t] += dov * sv;
+        xk[t] += drv * sv;
+        xb[t] += uv * DS[c * VS + v];
+      }
     }
-    const float dqh = scale * xq, dkh = -be[r] * xk;
-    const float gm = sm[Ly::GM + r * KS + c], sg = sm[Ly::SG + r * KS + c];
-    sm[Ly::E0 + r * KS + c] = qq[r * KS + c] * dqh + kk[r * KS + c] * dkh;
-    sm[Ly::EX + r * KS + c] = kk[r * KS + c] * xb;
-    float dq = gm * dqh, dk = gm * dkh + sg * xb;
-    float g = 1.f;  // G_{r<-j}
-    dq += sm[Ly::DM + r * CS + r] * kk[r * KS + c];
+    float dq[4], dk[4];
+    const float dmrr = sm[Ly::DM + r * CS + r];
+CKDA_UNROLL
+    for (int t = 0; t < 4; ++t) {
+      const int c = cq + t * NQ;
+      const float dqh = scale * xq[t], dkh = -be[r] * xk[t];
+      const float gm = sm[Ly::GM + r * KS + c], sg = sm[Ly::SG + r * KS + c];
+      sm[Ly::E0 + r * KS + c] = qq[r * KS + c] * dqh + kk[r * KS + c] * dkh;
+      sm[Ly::EX + r * KS + c] = kk[r * KS + c] * xb[t];
+      dq[t] = gm * dqh + dmrr * kk[r * KS + c];
+      dk[t] = gm * dkh + sg * xb[t];
+    }
+    float g[4] = {1.f, 1.f, 1.f, 1.f};  // G_{r<-j} per channel
     for (int j = r - 1; j >= 0; --j) {
-      g *= al[(j + 1) * KS + c];
-      const float gk = g * kk[j * KS + c];
-      dq += sm[Ly::DM + r * CS + j] * gk;
-      dk += sm[Ly::DA + r * CS + j] * gk;
+      const float dm = sm[Ly::DM + r * CS + j], da = sm[Ly::DA + r * CS + j];
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        const int c = cq + t * NQ;
+        g[t] *= al[(j + 1) * KS + c];
+        const float gk = g[t] * kk[j * KS + c];
+        dq[t] += dm * gk;
+        dk[t] += da * gk;
+      }
     }
-    g = 1.f;  // G_{i<-r}
+CKDA_UNROLL
+    for (int t = 0; t < 4; ++t) g[t] = 1.f;  // G_{i<-r} per channel
     for (int i = r; i < C; ++i) {
-      if (i > r) g *= al[i * KS + c];
-      dk += g * (sm[Ly::DM + i * CS + r] * qq[i * KS + c] +
-                 sm[Ly::DA + i * CS + r] * kk[i * KS + c]);
+      const float dm = sm[Ly::DM + i * CS + r], da = sm[Ly::DA + i * CS + r];
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        const int c = cq + t * NQ;
+        if (i > r) g[t] *= al[i * KS + c];
+        dk[t] += g[t] * (dm * qq[i * KS + c] + da * kk[i * KS + c]);
+      }
     }
     if (r < L) {
-      const size_t pi = ((size_t)tile * a.TH + (size_t)(t0 + r) * H + h) * DK + c;
-      a.pq[pi] = dq;
-      a.pk[pi] = dk;
+      const size_t pi = ((size_t)tile * a.TH + (size_t)(t0 + r) * H + h) * DK;
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        a.pq[pi + cq + t * NQ] = dq[t];
+        a.pk[pi + cq + t * NQ] = dk[t];
+      }
     }
   });
   // dalpha (this tile's share), one channel per item
