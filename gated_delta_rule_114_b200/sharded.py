@@ -129,14 +129,15 @@ def _gather_parts(parts, cu_seqlens_host, world, group):
     return tuple(out)
 
 
-def _cuda_bwd(q, k, v, alpha, beta, s0, d_o, dsf, cu_local, scale):
+def _cuda_bwd(q, k, v, alpha, beta, s0, d_o, dsf, cu_local, scale, chunked=False):
     return ckda.bwd(q, k, v, alpha, beta, d_o, s0, dsf, cu_seqlens=cu_local.to(q.device),
-                    cu_seqlens_host=cu_local, scale=scale)
+                    cu_seqlens_host=cu_local, scale=scale, chunked=chunked)
 
 
 def bwd_sharded(q, k, v, alpha, beta, d_o, initial_state, d_final_state, cu_seqlens_host,
                 rank: int | None = None, world: int | None = None, *, scale: float = 1.0,
-                gather: bool = False, group=None, bwd: Callable | None = None):
+                gather: bool = False, group=None, bwd: Callable | None = None,
+                chunked: bool = False):
     """This rank's shard of a packed varlen backward pass.
 
     Inputs are the whole batch (as for fwd_chunked_sharded, plus d_o
@@ -144,13 +145,15 @@ def bwd_sharded(q, k, v, alpha, beta, d_o, initial_state, d_final_state, cu_seql
     reads only its own sequences' rows. Returns (dq, dk, dv, dalpha, dbeta,
     d_initial_state) for this rank's token rows and sequences and (n0, n1);
     with gather=True, the whole batch's gradients on every rank instead.
-    `bwd` replaces the CUDA backward (same arguments as the default) for
-    host-side tests."""
+    `chunked` selects ckda_bwd_chunked for the shard; `bwd` replaces the CUDA
+    backward (same arguments as the default) for host-side tests."""
     if rank is None:
         rank = dist.get_rank(group) if dist.is_initialized() else 0
     if world is None:
         world = dist.get_world_size(group) if dist.is_initialized() else 1
-    bwd = bwd or _cuda_bwd
+    if bwd is None:
+        def bwd(*args):
+            return _cuda_bwd(*args, chunked=chunked)
     n0, n1 = plan_shards(cu_seqlens_host, world)[rank]
     qs, ks, vs, as_, bs, s0, cu_local = shard_inputs(q, k, v, alpha, beta, initial_state,
                                                      cu_seqlens_host, n0, n1)
