@@ -22,11 +22,11 @@
 // special. Only dS crosses chunks.
 //
 // This file holds the pieces one chunk needs (staging, gate products, Grams
-// and the UT solve, Khat S and U, the gradients of a chunk from S, dS_C, U
-// and dR); ckda_bwd_split.cuh composes them into the four programs of the
-// backward. The columns of S and dS are independent; everything that sums
-// over columns (dq, dk, dalpha, dbeta) is linear in per-column terms, so each
-// column tile writes fp32 partials that a second kernel adds in tile order.
+// and the UT solve, Khat S, the per-channel gate gradient); ckda_bwd_split.cuh
+// composes them into the four programs of the backward. The columns of S and
+// dS are independent; everything that sums over columns (dq, dk, dalpha,
+// dbeta) is linear in per-column terms, so the gradient program adds the
+// column tiles of one chunk in a fixed order.
 //
 // Every program is a fixed sequence of data-parallel phases. par<N>(x, f)
 // runs one phase on executor X: f(i) for every i in [0, N), the calls
@@ -66,44 +66,18 @@ CKDA_PROG void par(X &x, F f) {
   x.template run<N>(f);
 }
 
-// Shared-memory layout (floats) of the per-chunk gradient program. Rows are
-// padded to an odd stride so that a warp reading down a column, or along rows
-// indexed by its lanes, touches distinct banks.
-template <int DK, int DVT>
-struct Layout {
-  static constexpr int dk = DK, dvt = DVT;
-  static constexpr int KS = DK + 1;   // C x DK rows
-  static constexpr int VS = DVT + 1;  // C x DVT and DK x DVT rows
-  static constexpr int CS = C + 1;    // C x C rows
-  // C x DK: inputs q, k, alpha; gamma, sigma; the gate-gradient coefficients
-  // of the chunk entry (E0) and exit (EX)
-  static constexpr int Q = 0, K = Q + C * KS, AL = K + C * KS, GM = AL + C * KS,
-                       SG = GM + C * KS, E0 = SG + C * KS, EX = E0 + C * KS;
-  // C x DVT: v, dO, Khat S then w, U, dR
-  static constexpr int V = EX + C * KS, DO = V + C * VS, KSW = DO + C * VS, U = KSW + C * VS,
-                       DR = U + C * VS;
-  // DK x DVT: the entry state tile and the exit-state gradient tile
-  static constexpr int S = DR + C * VS, DS = S + DK * VS;
-  // C x C: Abar, dM, dAbar
-  static constexpr int AB = DS + DK * VS, DM = AB + C * CS, DA = DM + C * CS;
-  static constexpr int BE = DA + C * CS;  // beta [C]
-  static constexpr int FLOATS = BE + C;
-  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
-};
-
-// Pointers and sizes of one call. Token-major [T_total, H, .] tensors; states
-// [N, H, d_k, d_v]; partials [ntile, T_total H, d_k] (dq, dk, dalpha) and
-// [ntile, T_total H] (dbeta).
+// Pointers and sizes of one call. Token-major [T_total, H, .] tensors (q, k,
+// v, dO and dq, dk, dv in the I/O type; alpha, dalpha [T_total, H, d_k] and
+// beta, dbeta [T_total, H] fp32); states [N, H, d_k, d_v] fp32.
 template <typename IOT>
 struct Args {
   const IOT *q, *k, *v;
   const float *alpha, *beta, *s0;
   const IOT *d_o;
   const float *dsf;
-  IOT *dv;
-  float *pq, *pk, *pa, *pb, *ds0;
-  int H, DVF;   // heads; full d_v (the tiles' columns are c0 .. c0 + DVT - 1)
-  size_t TH;    // T_total * H
+  IOT *dq, *dk, *dv;
+  float *dalpha, *dbeta, *ds0;
+  int H, DVF;  // heads; full d_v
   float scale;
 };
 
@@ -227,9 +201,8 @@ CKDA_PROG void chunk_khat_s(X &x, float *sm) {
 // positions (q, p]. F_s(p) = sum_{q<s} G_{s-1<-q} E(p, q) grows as
 // F_{s+1} = alpha_s F_s + E(., s); dalpha_s = sum_{p>=s} G_{p<-s} F_s(p), a
 // Horner pass from p = C down.
-template <int DK, int DVT>
+template <class Ly>
 CKDA_PROG void gate_grad_channel(const float *sm, int c, float sds, float *out) {
-  using Ly = Layout<DK, DVT>;
   constexpr int KS = Ly::KS, CS = Ly::CS;
   const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
   const float *dm = sm + Ly::DM, *da = sm + Ly::DA;
@@ -258,126 +231,6 @@ CKDA_UNROLL
     for (int p = C - 1; p >= s; --p) hsum = al[p * KS + c] * hsum + F[p];
     out[s - 1] = hsum;
   }
-}
-
-// The gradients of one chunk from the staged inputs, gamma and sigma, Abar,
-// the entry state S, the exit-state gradient dS_C (in the DS rows), U, dR and
-// Khat S (in the Khat S rows): dv; dbeta, dq, dk and dalpha as this tile's
-// partials. Leaves Khat S replaced by w; S, dS_C, U and dR unchanged.
-template <class X, class IOL, typename IOT, int DK, int DVT>
-CKDA_PROG void chunk_grads(X &x, const Args<IOT> &a, float *sm, int h, int tile, int t0,
-                            int L) {
-  using Ly = Layout<DK, DVT>;
-  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS;
-  const int c0 = tile * DVT, H = a.H;
-  const float scale = a.scale;
-  const float *be = sm + Ly::BE;
-  const float *S = sm + Ly::S, *DS = sm + Ly::DS;
-  // w = V - Khat S - Abar U (over the Khat S rows); dv = diag(beta) dR
-  par<C * DVT>(x, [&](int e) {
-    const int i = e / DVT, v = e - i * DVT;
-    float s = 0.f;
-    for (int m = 0; m < i; ++m) s += sm[Ly::AB + i * CS + m] * sm[Ly::U + m * VS + v];
-    sm[Ly::KSW + i * VS + v] = sm[Ly::V + i * VS + v] - sm[Ly::KSW + i * VS + v] - s;
-    if (i < L)
-      IOL::st(a.dv + ((size_t)(t0 + i) * H + h) * a.DVF + c0 + v,
-              be[i] * sm[Ly::DR + i * VS + v]);
-  });
-  // dbeta (this tile's share); dM and dAbar
-  par<C * C>(x, [&](int e) {
-    const int i = e / C, j = e - i * C;
-    if (j == 0 && i < L) {
-      float s = 0.f;
-      for (int v = 0; v < DVT; ++v) s += sm[Ly::DR + i * VS + v] * sm[Ly::KSW + i * VS + v];
-      a.pb[(size_t)tile * a.TH + (size_t)(t0 + i) * H + h] = s;
-    }
-    float m = 0.f, d = 0.f;
-    if (j <= i) {
-      for (int v = 0; v < DVT; ++v) {
-        const float u = sm[Ly::U + j * VS + v];
-        m += sm[Ly::DO + i * VS + v] * u;
-        d += sm[Ly::DR + i * VS + v] * u;
-      }
-    }
-    sm[Ly::DM + i * CS + j] = scale * m;
-    sm[Ly::DA + i * CS + j] = j < i ? -be[i] * d : 0.f;
-  });
-  // per (row r, channels cq + t DK/4 for t < 4): the state-side terms
-  // dQhat = scale dO S^T, dKhat = -diag(beta) dR S^T, dKbar = U dS_C^T (E0 and EX
-  // keep their gate parts), then the gated Gram terms of dq and dk; this tile's
-  // dq, dk partials. The row's dO, dR, U, dM and dAbar values serve all four
-  // channels; channels at stride DK/4 keep a warp's accesses on distinct banks.
-  constexpr int NQ = DK / 4;
-  par<C * NQ>(x, [&](int e) {
-    const int r = e / NQ, cq = e - r * NQ;
-    const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
-    float xq[4] = {}, xk[4] = {}, xb[4] = {};
-    for (int v = 0; v < DVT; ++v) {
-      const float dov = sm[Ly::DO + r * VS + v], drv = sm[Ly::DR + r * VS + v];
-      const float uv = sm[Ly::U + r * VS + v];
-CKDA_UNROLL
-      for (int t = 0; t < 4; ++t) {
-        const int c = cq + t * NQ;
-        const float sv = S[c * VS + v];
-        xq[t] += dov * sv;
-        xk[t] += drv * sv;
-        xb[t] += uv * DS[c * VS + v];
-      }
-    }
-    float dq[4], dk[4];
-    const float dmrr = sm[Ly::DM + r * CS + r];
-CKDA_UNROLL
-    for (int t = 0; t < 4; ++t) {
-      const int c = cq + t * NQ;
-      const float dqh = scale * xq[t], dkh = -be[r] * xk[t];
-      const float gm = sm[Ly::GM + r * KS + c], sg = sm[Ly::SG + r * KS + c];
-      sm[Ly::E0 + r * KS + c] = qq[r * KS + c] * dqh + kk[r * KS + c] * dkh;
-      sm[Ly::EX + r * KS + c] = kk[r * KS + c] * xb[t];
-      dq[t] = gm * dqh + dmrr * kk[r * KS + c];
-      dk[t] = gm * dkh + sg * xb[t];
-    }
-    float g[4] = {1.f, 1.f, 1.f, 1.f};  // G_{r<-j} per channel
-    for (int j = r - 1; j >= 0; --j) {
-      const float dm = sm[Ly::DM + r * CS + j], da = sm[Ly::DA + r * CS + j];
-CKDA_UNROLL
-      for (int t = 0; t < 4; ++t) {
-        const int c = cq + t * NQ;
-        g[t] *= al[(j + 1) * KS + c];
-        const float gk = g[t] * kk[j * KS + c];
-        dq[t] += dm * gk;
-        dk[t] += da * gk;
-      }
-    }
-CKDA_UNROLL
-    for (int t = 0; t < 4; ++t) g[t] = 1.f;  // G_{i<-r} per channel
-    for (int i = r; i < C; ++i) {
-      const float dm = sm[Ly::DM + i * CS + r], da = sm[Ly::DA + i * CS + r];
-CKDA_UNROLL
-      for (int t = 0; t < 4; ++t) {
-        const int c = cq + t * NQ;
-        if (i > r) g[t] *= al[i * KS + c];
-        dk[t] += g[t] * (dm * qq[i * KS + c] + da * kk[i * KS + c]);
-      }
-    }
-    if (r < L) {
-      const size_t pi = ((size_t)tile * a.TH + (size_t)(t0 + r) * H + h) * DK;
-CKDA_UNROLL
-      for (int t = 0; t < 4; ++t) {
-        a.pq[pi + cq + t * NQ] = dq[t];
-        a.pk[pi + cq + t * NQ] = dk[t];
-      }
-    }
-  });
-  // dalpha (this tile's share), one channel per item
-  par<DK>(x, [&](int c) {
-    float sds = 0.f;
-    for (int v = 0; v < DVT; ++v) sds += S[c * VS + v] * DS[c * VS + v];
-    float da[C];
-    gate_grad_channel<DK, DVT>(sm, c, sds, da);
-CKDA_UNROLL
-    for (int i = 0; i < C; ++i)  // static indices keep da in registers
-      if (i < L) a.pa[((size_t)tile * a.TH + (size_t)(t0 + i) * H + h) * DK + c] = da[i];
-  });
 }
 
 }  // namespace bwdc

@@ -1,10 +1,10 @@
 // The split chunkwise backward (ckda_bwd_split.cuh) as four kernels on CUDA
-// cores (sm_100a), plus the tile reduction shared with the other backward
-// kernels:
-//   prep   grid (checkpoint slots, H)           256 threads, parallel over chunks
-//   scan1  grid (H, N, d_v tiles)               entry states and U, chunk by chunk
-//   scan2  grid (H, N, d_v tiles)               exit-state gradients and dR, in reverse
-//   grads  grid (checkpoint slots, H, d_v tiles) parallel over chunks
+// cores (sm_100a):
+//   prep   grid (checkpoint slots, H)   256 threads, parallel over chunks
+//   scan1  grid (H, N, d_v tiles)       entry states and U, chunk by chunk
+//   scan2  grid (H, N, d_v tiles)       exit-state gradients and dR, in reverse
+//   grads  grid (checkpoint slots, H)   every gradient of a chunk, its columns
+//                                       in 16-column tiles added in order
 // A slot that starts no chunk (slots are floor(cu[n] / 16) + n + chunk) exits
 // at once, before any barrier, on every thread of its CTA.
 #include <cuda_bf16.h>
@@ -17,12 +17,9 @@
 
 namespace ckda {
 
-template <typename IOT>
-cudaError_t launch_bwd_reduce(const float *pq, const float *pk, const float *pa,
-                              const float *pb, void *dq, void *dk, float *dalpha, float *dbeta,
-                              size_t n_tk, size_t n_t, int ntile, cudaStream_t st);
-
 namespace {
+
+constexpr int kGradTile = 16;  // columns per tile of the gradient program
 
 constexpr int kThreads = 256;
 
@@ -83,7 +80,7 @@ bwd_scan_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ 
                                                            bos / CK + n);
 }
 
-template <typename IOT, int DK, int DVT>
+template <typename IOT, int DK>
 __global__ void __launch_bounds__(kThreads, 2)
 bwd_grads_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ cu, int N,
                  int T, int T_total, unsigned int *err) {
@@ -91,8 +88,8 @@ bwd_grads_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__
   int t0, L;
   if (!slot_rows(cu, N, T, T_total, err, t0, L)) return;
   DeviceExec x;
-  bwdc::grads_program<DeviceExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, blockIdx.y, blockIdx.z,
-                                                         t0, L, blockIdx.x);
+  bwdc::grads_program<DeviceExec, IO<IOT>, IOT, DK, kGradTile>(x, a, w, sm, blockIdx.y, t0, L,
+                                                               blockIdx.x);
 }
 
 template <class K>
@@ -107,44 +104,36 @@ cudaError_t launch_dims(const bwdc::Args<IOT> &a, const bwdc::SplitWs &w, const 
   const int ntile = a.DVF / DVT;
   using PL = bwdc::PrepLayout<DK, DVT>;
   using SL = bwdc::ScanLayout<DK, DVT>;
-  using GL = bwdc::Layout<DK, DVT>;
+  using GL = bwdc::GradLayout<DK, kGradTile>;
   cudaError_t e;
   if ((e = set_smem(bwd_prep_kernel<IOT, DK, DVT>, PL::BYTES)) != cudaSuccess) return e;
   if ((e = set_smem(bwd_scan_kernel<IOT, DK, DVT, false>, SL::BYTES)) != cudaSuccess) return e;
   if ((e = set_smem(bwd_scan_kernel<IOT, DK, DVT, true>, SL::BYTES)) != cudaSuccess) return e;
-  if ((e = set_smem(bwd_grads_kernel<IOT, DK, DVT>, GL::BYTES)) != cudaSuccess) return e;
+  if ((e = set_smem(bwd_grads_kernel<IOT, DK>, GL::BYTES)) != cudaSuccess) return e;
   bwd_prep_kernel<IOT, DK, DVT><<<dim3(slots, a.H), kThreads, PL::BYTES, st>>>(a, w, cu, N, T,
                                                                               T_total, err);
   bwd_scan_kernel<IOT, DK, DVT, false><<<dim3(a.H, N, ntile), kThreads, SL::BYTES, st>>>(
       a, w, cu, T, T_total, err);
   bwd_scan_kernel<IOT, DK, DVT, true><<<dim3(a.H, N, ntile), kThreads, SL::BYTES, st>>>(
       a, w, cu, T, T_total, err);
-  bwd_grads_kernel<IOT, DK, DVT><<<dim3(slots, a.H, ntile), kThreads, GL::BYTES, st>>>(
-      a, w, cu, N, T, T_total, err);
+  bwd_grads_kernel<IOT, DK><<<dim3(slots, a.H), kThreads, GL::BYTES, st>>>(a, w, cu, N, T,
+                                                                          T_total, err);
   return cudaGetLastError();
 }
 
 // Workspace pieces, in order: checkpoints S and dS | gamma_C | Abar | W, Kbar,
-// Wb, Qs, BK | Utilde, X, U, dR | partials dq, dk, dalpha [ntile][T_total H]
-// [d_k] | dbeta [ntile][T_total H] (float counts).
-constexpr int kPieces = 17;
+// Wb, Qs, BK | Utilde, X, U, dR (float counts).
+constexpr int kPieces = 13;
 
 void piece_sizes(int N, int T_total, int H, int dk, int dv, size_t (&n)[kPieces]) {
   const size_t slots = (size_t)T_total / CK + (size_t)N, th = (size_t)T_total * H;
-  const size_t ntile = (size_t)(dv / (dv < 32 ? dv : 32));
   const size_t sizes[kPieces] = {slots * H * dk * dv, slots * H * dk * dv, slots * H * dk,
                                  slots * H * CK * CK, th * dk, th * dk, th * dk, th * dk,
-                                 th * dk, th * dv, th * dv, th * dv, th * dv,
-                                 ntile * th * dk, ntile * th * dk, ntile * th * dk, ntile * th};
+                                 th * dk, th * dv, th * dv, th * dv, th * dv};
   for (int i = 0; i < kPieces; ++i) n[i] = sizes[i];
 }
 
-struct Carve {
-  bwdc::SplitWs w;
-  float *pq, *pk, *pa, *pb;
-};
-
-Carve carve(float *base, int N, int T_total, int H, int dk, int dv) {
+bwdc::SplitWs carve(float *base, int N, int T_total, int H, int dk, int dv) {
   size_t n[kPieces];
   piece_sizes(N, T_total, H, dk, dv, n);
   float *p[kPieces];
@@ -152,14 +141,8 @@ Carve carve(float *base, int N, int T_total, int H, int dk, int dv) {
     p[i] = base;
     base += n[i];
   }
-  Carve c;
-  c.w = bwdc::SplitWs{p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7], p[8],
-                      p[9], p[10], p[11], p[12]};
-  c.pq = p[13];
-  c.pk = p[14];
-  c.pa = p[15];
-  c.pb = p[16];
-  return c;
+  return bwdc::SplitWs{p[0], p[1], p[2], p[3], p[4], p[5], p[6],
+                       p[7], p[8], p[9], p[10], p[11], p[12]};
 }
 
 }  // namespace
@@ -179,22 +162,19 @@ cudaError_t launch_bwd_split(int dk_, int dv_, const void *q, const void *k, con
                              int T, int T_total, int H, float scale, void *ws,
                              unsigned int *err, cudaStream_t st) {
   const int dvt = dv_ < 32 ? dv_ : 32;
-  const size_t th = (size_t)T_total * H, ntile = (size_t)(dv_ / dvt);
-  const Carve c = carve(static_cast<float *>(ws), N, T_total, H, dk_, dv_);
-  bwdc::Args<IOT> a{static_cast<const IOT *>(q), static_cast<const IOT *>(k),
-                    static_cast<const IOT *>(v), alpha, beta, s0,
-                    static_cast<const IOT *>(d_o), dsf, static_cast<IOT *>(dv), c.pq, c.pk,
-                    c.pa, c.pb, ds0, H, dv_, th, scale};
-  cudaError_t e = cudaErrorInvalidValue;
-#define CKDA_BWDS_DK(X)                                                        \
-  if (dk_ == X)                                                                \
-    e = dvt == 16 ? launch_dims<IOT, X, 16>(a, c.w, cu, N, T, T_total, err, st) \
-                  : launch_dims<IOT, X, 32>(a, c.w, cu, N, T, T_total, err, st);
+  const bwdc::SplitWs w = carve(static_cast<float *>(ws), N, T_total, H, dk_, dv_);
+  bwdc::Args<IOT> a{static_cast<const IOT *>(q),  static_cast<const IOT *>(k),
+                    static_cast<const IOT *>(v),  alpha, beta, s0,
+                    static_cast<const IOT *>(d_o), dsf,
+                    static_cast<IOT *>(dq),       static_cast<IOT *>(dk),
+                    static_cast<IOT *>(dv),       dalpha, dbeta, ds0, H, dv_, scale};
+#define CKDA_BWDS_DK(X)                                                      \
+  if (dk_ == X)                                                              \
+    return dvt == 16 ? launch_dims<IOT, X, 16>(a, w, cu, N, T, T_total, err, st) \
+                     : launch_dims<IOT, X, 32>(a, w, cu, N, T, T_total, err, st);
   CKDA_BWDS_DK(16) CKDA_BWDS_DK(32) CKDA_BWDS_DK(64) CKDA_BWDS_DK(128)
 #undef CKDA_BWDS_DK
-  if (e != cudaSuccess) return e;
-  return launch_bwd_reduce<IOT>(c.pq, c.pk, c.pa, c.pb, dq, dk, dalpha, dbeta, th * dk_, th,
-                                (int)ntile, st);
+  return cudaErrorInvalidValue;
 }
 
 template cudaError_t launch_bwd_split<float>(int, int, const void *, const void *, const void *,

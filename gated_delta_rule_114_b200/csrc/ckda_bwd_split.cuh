@@ -13,7 +13,7 @@
 //   prep   (per chunk and head)            the factors above, Abar, gamma_C;
 //   scan1  (per sequence, head, col. tile) entry states S per chunk, and U;
 //   scan2  (per sequence, head, col. tile) exit-state gradients dS_C, and dR;
-//   grads  (per chunk, head, col. tile)    chunk_grads from (S, dS_C, U, dR).
+//   grads  (per chunk and head)            all gradients from (S, dS_C, U, dR).
 // Per-chunk values (S, dS_C, gamma_C, Abar) sit in checkpoint slots
 // (slot = floor(cu[n] / C) + n + chunk, at most floor(T_total / C) + N
 // slots); per-token values in token-major [T_total, H, .] fp32 arrays.
@@ -325,32 +325,214 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
   }
 }
 
-// The gradients of one (chunk, head, column tile) from the scans' outputs.
-template <class X, class IOL, typename IOT, int DK, int DVT>
+// Shared memory of the gradient program: one (chunk, head), the columns in
+// tiles of GT. Rows are padded to an odd stride so that a warp reading down a
+// column, or along rows indexed by its lanes, touches distinct banks.
+template <int DK, int GT>
+struct GradLayout {
+  static constexpr int dk = DK, dvt = GT;
+  static constexpr int KS = DK + 1, VS = GT + 1, CS = C + 1;
+  // C x DK: q, k, alpha; gamma, sigma; the column sums of dO S^T, dR S^T and
+  // U dS_C^T, overwritten by the gate-gradient coefficients E0 (over XQ) and
+  // EX (over XB)
+  static constexpr int Q = 0, K = Q + C * KS, AL = K + C * KS, GM = AL + C * KS,
+                       SG = GM + C * KS, XQ = SG + C * KS, XK = XQ + C * KS, XB = XK + C * KS;
+  static constexpr int E0 = XQ, EX = XB;
+  // C x GT: v, dO, Khat S then w, U, dR of the current column tile
+  static constexpr int V = XB + C * KS, DO = V + C * VS, KSW = DO + C * VS, U = KSW + C * VS,
+                       DR = U + C * VS;
+  // DK x GT: the tile of the entry state and of the exit-state gradient
+  static constexpr int S = DR + C * VS, DS = S + DK * VS;
+  // C x C: Abar, dM and dAbar (summed over the tiles)
+  static constexpr int AB = DS + DK * VS, DM = AB + C * CS, DA = DM + C * CS;
+  // beta [C], dbeta [C], sum_v S dS_C per channel [DK]
+  static constexpr int BE = DA + C * CS, DB = BE + C, SDS = DB + C;
+  static constexpr int FLOATS = SDS + DK;
+  static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
+};
+
+// The gradients of one (chunk, head) from the scans' outputs (S, dS_C, U, dR
+// per chunk). dv is written tile by tile; everything that sums over the
+// columns (dM, dAbar, dbeta and the state-side terms of dq, dk, dalpha)
+// accumulates over the column tiles in a fixed order, then dq, dk (with the
+// gated Gram terms), dalpha and dbeta are written once.
+template <class X, class IOL, typename IOT, int DK, int GT>
 CKDA_PROG void grads_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
-                             int tile, int t0, int L, int slot) {
-  using Ly = Layout<DK, DVT>;
-  constexpr int VS = Ly::VS, CS = Ly::CS;
-  const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
+                             int t0, int L, int slot) {
+  using Ly = GradLayout<DK, GT>;
+  constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS, NQ = DK / 4;
+  const int H = a.H, DVF = a.DVF;
+  const float scale = a.scale;
   const size_t sl = (size_t)slot * H + h;
-  stage<X, IOL, IOT, Ly>(x, a, sm, h, c0, t0, L, true);
+  const float *be = sm + Ly::BE;
+  const float *al = sm + Ly::AL, *kk = sm + Ly::K, *qq = sm + Ly::Q;
+  // q, k, alpha, beta (rows L..C-1 inert); zero the sums; Abar
+  par<C * DK>(x, [&](int e) {
+    const int i = e / DK, c = e - i * DK;
+    float qv = 0.f, kv = 0.f, av = 1.f;
+    if (i < L) {
+      const size_t g = ((size_t)(t0 + i) * H + h) * DK + c;
+      qv = IOL::ldg(a.q + g);
+      kv = IOL::ldg(a.k + g);
+      av = CKDA_LDG(a.alpha + g);
+    }
+    sm[Ly::Q + i * KS + c] = qv;
+    sm[Ly::K + i * KS + c] = kv;
+    sm[Ly::AL + i * KS + c] = av;
+    sm[Ly::XQ + i * KS + c] = 0.f;
+    sm[Ly::XK + i * KS + c] = 0.f;
+    sm[Ly::XB + i * KS + c] = 0.f;
+    if (e < C * C) {
+      sm[Ly::AB + (e / C) * CS + e % C] = CKDA_LDG(w.ab + sl * C * C + e);
+      sm[Ly::DM + (e / C) * CS + e % C] = 0.f;
+      sm[Ly::DA + (e / C) * CS + e % C] = 0.f;
+    }
+    if (e < C) {
+      sm[Ly::BE + e] = e < L ? CKDA_LDG(a.beta + (size_t)(t0 + e) * H + h) : 0.f;
+      sm[Ly::DB + e] = 0.f;
+    }
+    if (e < DK) sm[Ly::SDS + e] = 0.f;
+  });
   chunk_gates<X, Ly>(x, sm);
-  // the chunk's S, dS_C, Abar and its rows of U and dR (rows L..C-1 zero)
-  par<DK * DVT>(x, [&](int e) {
-    const int c = e / DVT, v = e - c * DVT;
-    const size_t o = sl * DK * DVF + (size_t)c * DVF + c0 + v;
-    sm[Ly::S + c * VS + v] = CKDA_LDG(w.cks + o);
-    sm[Ly::DS + c * VS + v] = CKDA_LDG(w.ckd + o);
-    if (e < C * C) sm[Ly::AB + (e / C) * CS + e % C] = CKDA_LDG(w.ab + sl * C * C + e);
-    if (e < C * DVT) {
-      const int i = e / DVT, u = e - i * DVT;
-      const size_t r = ((size_t)(t0 + i) * H + h) * DVF + c0 + u;
-      sm[Ly::U + i * VS + u] = i < L ? CKDA_LDG(w.uu + r) : 0.f;
-      sm[Ly::DR + i * VS + u] = i < L ? CKDA_LDG(w.dr + r) : 0.f;
+  for (int c0 = 0; c0 < DVF; c0 += GT) {
+    // the tile's S, dS_C and rows of U, dR, v, dO (rows L..C-1 zero)
+    par<DK * GT>(x, [&](int e) {
+      const int c = e / GT, v = e - c * GT;
+      const size_t o = sl * DK * DVF + (size_t)c * DVF + c0 + v;
+      sm[Ly::S + c * VS + v] = CKDA_LDG(w.cks + o);
+      sm[Ly::DS + c * VS + v] = CKDA_LDG(w.ckd + o);
+      if (e < C * GT) {
+        const int i = e / GT, u = e - i * GT;
+        const bool in = i < L;
+        const size_t r = ((size_t)(t0 + i) * H + h) * DVF + c0 + u;
+        sm[Ly::U + i * VS + u] = in ? CKDA_LDG(w.uu + r) : 0.f;
+        sm[Ly::DR + i * VS + u] = in ? CKDA_LDG(w.dr + r) : 0.f;
+        sm[Ly::V + i * VS + u] = in ? IOL::ldg(a.v + r) : 0.f;
+        sm[Ly::DO + i * VS + u] = in ? IOL::ldg(a.d_o + r) : 0.f;
+      }
+    });
+    chunk_khat_s<X, Ly>(x, sm);
+    // w = V - Khat S - Abar U (over the Khat S rows); dv = diag(beta) dR
+    par<C * GT>(x, [&](int e) {
+      const int i = e / GT, v = e - i * GT;
+      float s = 0.f;
+      for (int m = 0; m < i; ++m) s += sm[Ly::AB + i * CS + m] * sm[Ly::U + m * VS + v];
+      sm[Ly::KSW + i * VS + v] = sm[Ly::V + i * VS + v] - sm[Ly::KSW + i * VS + v] - s;
+      if (i < L)
+        IOL::st(a.dv + ((size_t)(t0 + i) * H + h) * DVF + c0 + v, be[i] * sm[Ly::DR + i * VS + v]);
+    });
+    // the tile's share of dO U^T, dR U^T and dR . w
+    par<C * C>(x, [&](int e) {
+      const int i = e / C, j = e - i * C;
+      if (j == 0) {
+        float s = 0.f;
+        for (int v = 0; v < GT; ++v) s += sm[Ly::DR + i * VS + v] * sm[Ly::KSW + i * VS + v];
+        sm[Ly::DB + i] += s;
+      }
+      if (j <= i) {
+        float m = 0.f, d = 0.f;
+        for (int v = 0; v < GT; ++v) {
+          const float u = sm[Ly::U + j * VS + v];
+          m += sm[Ly::DO + i * VS + v] * u;
+          d += sm[Ly::DR + i * VS + v] * u;
+        }
+        sm[Ly::DM + i * CS + j] += m;
+        sm[Ly::DA + i * CS + j] += d;
+      }
+    });
+    // the tile's share of dO S^T, dR S^T, U dS_C^T and of sum_v S dS_C, per
+    // (row r, channels cq + t DK/4)
+    par<C * NQ>(x, [&](int e) {
+      const int r = e / NQ, cq = e - r * NQ;
+      float xq[4] = {}, xk[4] = {}, xb[4] = {}, sd[4] = {};
+      for (int v = 0; v < GT; ++v) {
+        const float dov = sm[Ly::DO + r * VS + v], drv = sm[Ly::DR + r * VS + v];
+        const float uv = sm[Ly::U + r * VS + v];
+CKDA_UNROLL
+        for (int t = 0; t < 4; ++t) {
+          const int c = cq + t * NQ;
+          const float sv = sm[Ly::S + c * VS + v], dsv = sm[Ly::DS + c * VS + v];
+          xq[t] += dov * sv;
+          xk[t] += drv * sv;
+          xb[t] += uv * dsv;
+          sd[t] += sv * dsv;
+        }
+      }
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        const int c = cq + t * NQ;
+        sm[Ly::XQ + r * KS + c] += xq[t];
+        sm[Ly::XK + r * KS + c] += xk[t];
+        sm[Ly::XB + r * KS + c] += xb[t];
+        if (r == 0) sm[Ly::SDS + c] += sd[t];
+      }
+    });
+  }
+  // dM = scale dO U^T (j <= i), dAbar = -diag(beta) dR U^T (j < i)
+  par<C * C>(x, [&](int e) {
+    const int i = e / C, j = e - i * C;
+    sm[Ly::DM + i * CS + j] *= scale;
+    sm[Ly::DA + i * CS + j] = j < i ? -be[i] * sm[Ly::DA + i * CS + j] : 0.f;
+  });
+  // per (row r, channels cq + t DK/4): dQhat = scale (dO S^T), dKhat =
+  // -diag(beta) (dR S^T), dKbar = U dS_C^T; E0, EX over their sums; dq and dk
+  // with the gated Gram terms, written once
+  par<C * NQ>(x, [&](int e) {
+    const int r = e / NQ, cq = e - r * NQ;
+    float dq[4], dk[4];
+    const float dmrr = sm[Ly::DM + r * CS + r];
+CKDA_UNROLL
+    for (int t = 0; t < 4; ++t) {
+      const int c = cq + t * NQ;
+      const float dqh = scale * sm[Ly::XQ + r * KS + c], dkh = -be[r] * sm[Ly::XK + r * KS + c];
+      const float xb = sm[Ly::XB + r * KS + c];
+      const float gm = sm[Ly::GM + r * KS + c], sg = sm[Ly::SG + r * KS + c];
+      sm[Ly::E0 + r * KS + c] = qq[r * KS + c] * dqh + kk[r * KS + c] * dkh;
+      sm[Ly::EX + r * KS + c] = kk[r * KS + c] * xb;
+      dq[t] = gm * dqh + dmrr * kk[r * KS + c];
+      dk[t] = gm * dkh + sg * xb;
+    }
+    float g[4] = {1.f, 1.f, 1.f, 1.f};  // G_{r<-j} per channel
+    for (int j = r - 1; j >= 0; --j) {
+      const float dm = sm[Ly::DM + r * CS + j], da = sm[Ly::DA + r * CS + j];
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        const int c = cq + t * NQ;
+        g[t] *= al[(j + 1) * KS + c];
+        const float gk = g[t] * kk[j * KS + c];
+        dq[t] += dm * gk;
+        dk[t] += da * gk;
+      }
+    }
+CKDA_UNROLL
+    for (int t = 0; t < 4; ++t) g[t] = 1.f;  // G_{i<-r} per channel
+    for (int i = r; i < C; ++i) {
+      const float dm = sm[Ly::DM + i * CS + r], da = sm[Ly::DA + i * CS + r];
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        const int c = cq + t * NQ;
+        if (i > r) g[t] *= al[i * KS + c];
+        dk[t] += g[t] * (dm * qq[i * KS + c] + da * kk[i * KS + c]);
+      }
+    }
+    if (r < L) {
+      const size_t o = ((size_t)(t0 + r) * H + h) * DK;
+CKDA_UNROLL
+      for (int t = 0; t < 4; ++t) {
+        IOL::st(a.dq + o + cq + t * NQ, dq[t]);
+        IOL::st(a.dk + o + cq + t * NQ, dk[t]);
+      }
     }
   });
-  chunk_khat_s<X, Ly>(x, sm);
-  chunk_grads<X, IOL, IOT, DK, DVT>(x, a, sm, h, tile, t0, L);
+  // dalpha, one channel per item; dbeta
+  par<DK>(x, [&](int c) {
+    float da[C];
+    gate_grad_channel<Ly>(sm, c, sm[Ly::SDS + c], da);
+CKDA_UNROLL
+    for (int i = 0; i < C; ++i)  // static indices keep da in registers
+      if (i < L) a.dalpha[((size_t)(t0 + i) * H + h) * DK + c] = da[i];
+    if (c < L) a.dbeta[(size_t)(t0 + c) * H + h] = sm[Ly::DB + c];
+  });
 }
 
 }  // namespace bwdc

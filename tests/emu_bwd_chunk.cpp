@@ -70,13 +70,10 @@ void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool 
   if (has_dsf) dsf = load(dir + "/dsf.bin", st);
   const int ntile = DV / DVT;
   const size_t slots = (size_t)T_total / C + N;
-  std::vector<float> dv(TH * DV), ds0(st);
-  std::vector<float> pq(ntile * TH * DK), pk(ntile * TH * DK), pa(ntile * TH * DK),
-      pb(ntile * TH);
-  Args<float> a{q.data(), k.data(), v.data(), al.data(), be.data(),
+  std::vector<float> dq(TH * DK), dk(TH * DK), dv(TH * DV), da(TH * DK), db(TH), ds0(st);
+  Args<float> a{q.data(),  k.data(),  v.data(),  al.data(), be.data(),
                 has_s0 ? s0.data() : nullptr, d_o.data(), has_dsf ? dsf.data() : nullptr,
-                dv.data(), pq.data(), pk.data(), pa.data(), pb.data(), ds0.data(), H, DV, TH,
-                scale};
+                dq.data(), dk.data(), dv.data(), da.data(), db.data(), ds0.data(), H, DV, scale};
   HostExec x;
   auto bounds = [&](int n, int &bos, int &eos) {
     bos = varlen ? cu[n] : n * T;
@@ -99,8 +96,9 @@ void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool 
       L = eos - t0 < C ? eos - t0 : C;
       return true;
     };
+    constexpr int GT = 16;  // columns per tile of the gradient program
     std::vector<float> psm(PrepLayout<DK, DVT>::FLOATS), ssm(ScanLayout<DK, DVT>::FLOATS),
-        gsm(Layout<DK, DVT>::FLOATS);
+        gsm(GradLayout<DK, GT>::FLOATS);
     int t0, L;
     for (int h = 0; h < H; ++h)
       for (int g = 0; g < (int)slots; ++g)
@@ -119,22 +117,11 @@ void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool 
               scan2_program<HostExec, HostIO, float, DK, DVT>(x, a, w, ssm.data(), h, n, tile,
                                                              bos, eos, bos / C + n);
           }
-    for (int tile = 0; tile < ntile; ++tile)
-      for (int h = 0; h < H; ++h)
-        for (int g = 0; g < (int)slots; ++g)
-          if (slot_rows(g, t0, L))
-            grads_program<HostExec, HostIO, float, DK, DVT>(x, a, w, gsm.data(), h, tile, t0, L,
-                                                           g);
+    for (int h = 0; h < H; ++h)
+      for (int g = 0; g < (int)slots; ++g)
+        if (slot_rows(g, t0, L))
+          grads_program<HostExec, HostIO, float, DK, GT>(x, a, w, gsm.data(), h, t0, L, g);
   }
-  std::vector<float> dq(TH * DK), dk(TH * DK), da(TH * DK), db(TH);
-  for (size_t i = 0; i < TH * DK; ++i)
-    for (int t = 0; t < ntile; ++t) {
-      dq[i] += pq[t * TH * DK + i];
-      dk[i] += pk[t * TH * DK + i];
-      da[i] += pa[t * TH * DK + i];
-    }
-  for (size_t i = 0; i < TH; ++i)
-    for (int t = 0; t < ntile; ++t) db[i] += pb[t * TH + i];
   save(dir + "/dq.bin", dq);
   save(dir + "/dk.bin", dk);
   save(dir + "/dv.bin", dv);

@@ -265,11 +265,10 @@ def test_bwd_chunked_workspace_query(lib):
     # per 16-token chunk slot (floor(T_total / 16) + N of them) and head: an
     # entry state and an exit-state gradient (d_k x d_v), gamma over the chunk
     # (d_k) and Abar (16 x 16); per token-head: W, Kbar, Wb, Qs, BK (d_k each)
-    # and Utilde, X, U, dR (d_v each); then the tiles' partials (d_v = 64: 2)
+    # and Utilde, X, U, dR (d_v each)
     def want(N, T_total, H, dk, dv):
-        sl, th, nt = (T_total // 16 + N) * H, T_total * H, dv // min(dv, 32)
-        return 4 * (sl * (2 * dk * dv + dk + 256) + th * (5 * dk + 4 * dv)
-                    + nt * th * (3 * dk + 1))
+        sl, th = (T_total // 16 + N) * H, T_total * H
+        return 4 * (sl * (2 * dk * dv + dk + 256) + th * (5 * dk + 4 * dv))
     assert lib.ckda_bwd_chunked_workspace_bytes(2, 40, 3, 32, 64, 0) == want(2, 80, 3, 32, 64)
     assert lib.ckda_bwd_chunked_workspace_bytes(2, 40, 3, 32, 64, 1) == want(2, 40, 3, 32, 64)
     assert lib.ckda_bwd_chunked_workspace_bytes(1, 8, 1, 16, 16, 0) == want(1, 8, 1, 16, 16)
