@@ -281,7 +281,7 @@ def chunked_legs(args, w, inp_cpu, T_total, H, N, dk, dv, stream, pk, world):
                              "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": nb / (ms / 1e3) / 1e9 / pk["hbm_gbs"], "traffic": None,
                              "algorithmic_bytes_per_launch": nb},
-                "timing": "this rank alone", "gpu_launches": 5 * args.bwd_steps}
+                "timing": "this rank alone", "gpu_launches": 4 * args.bwd_steps}
             del bws, bout, bdo, bdsf
         if args.complex_impl != "chunked":
             cin = {key: val.cuda() for key, val in
@@ -520,9 +520,9 @@ def main():
                            "32-column tile), plus a tile reduction" if args.bwd_impl == "serial"
                            else "chunkwise (16-token chunk-WY reverse) on CUDA cores: prep and "
                                 "gradients over all chunks, two scans per (sequence, head, "
-                                "32-column tile), plus a tile reduction"),
+                                "32-column tile)"),
                 "entry_point": "ckda_bwd_chunked" if args.bwd_impl == "chunked" else "ckda_bwd",
-                "gpu_launches": (2 if args.bwd_impl == "serial" else 5) * args.bwd_steps}
+                "gpu_launches": (2 if args.bwd_impl == "serial" else 4) * args.bwd_steps}
     del bws, bout
 
     # ---------------- the complex-phase gate on the same shape (complex64)

@@ -283,13 +283,13 @@ ckda_status ckda_bwd(const void *q, const void *k, const void *v, const float *a
  * dS = scale Qhat^T dO + diag(gamma) dS_C - Khat^T diag(beta) dR passes from
  * chunk to chunk. Four kernels: a prep over all chunks, a forward scan and a
  * reverse scan per (sequence, head, tile of up to 32 state columns) that
- * carry only the state products, and the per-chunk gradients over all
- * chunks; then the tiles' partials are added in a fixed order. fp32
- * arithmetic on CUDA cores, deterministic.
+ * carry only the state products, and the gradients per (chunk, head), whose
+ * column tiles are added in a fixed order. fp32 arithmetic on CUDA cores,
+ * deterministic.
  *   workspace   device scratch of at least ckda_bwd_chunked_workspace_bytes()
  *               bytes, owned by the caller (one entry state and one exit-state
- *               gradient per 16-token chunk, the chunks' factors, the tiles'
- *               partials); required when N > 0.
+ *               gradient per 16-token chunk and the chunks' factors); required
+ *               when N > 0.
  */
 ckda_status ckda_bwd_chunked(const void *q, const void *k, const void *v, const float *alpha,
                              const float *beta, const float *initial_state, const void *d_o,
