@@ -130,21 +130,25 @@ CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *s
 template <int DK, int DVT>
 struct ScanLayout {
   static constexpr int KS = DK + 1, VS = DVT + 1;
-  static constexpr int S = 0, F0 = S + DK * VS, F1 = F0 + C * KS, F2 = F1 + C * KS,
-                       R0 = F2 + C * KS, R1 = R0 + C * VS, GC = R1 + C * VS;
-  static constexpr int P = GC + DK;  // partial products, C x DVT x 4
+  // two sets of a chunk's factors (chunk i in set i & 1, so that the next
+  // chunk's loads overlap this chunk's products): three C x DK, two C x DVT
+  // and gamma_C; offsets within a set
+  static constexpr int F0 = 0, F1 = F0 + C * KS, F2 = F1 + C * KS, R0 = F2 + C * KS,
+                       R1 = R0 + C * VS, GC = R1 + C * VS, SET = GC + DK;
+  static constexpr int S = 0, SETS = S + DK * VS;
+  static constexpr int P = SETS + 2 * SET;  // partial products, C x DVT x 4
   static constexpr int FLOATS = P + 4 * C * DVT;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
 // Partial products of the C x DVT result A B (A: C x DK rows of stride DK + 1;
-// B: the DK x DVT state tile, rows of stride DVT + 1): item (row pair, 4
-// columns, quarter q) sums channels q, q + 4, q + 8, ... in a 2 x 4 register
-// tile into P; rows_state_sum adds the four quarters in a fixed order.
-template <int DK, int DVT, class X>
-CKDA_PROG void rows_state_partials(X &x, float *P, const float *A, const float *B) {
+// B: the DK x DVT state tile, rows of stride DVT + 1): item e (row pair, 4
+// columns, quarter q; PartialItems of them) sums channels q, q + 4, ... in
+// a 2 x 4 register tile into P; rows_state_sum adds the quarters in order.
+template <int DK, int DVT>
+CKDA_PROG void rows_state_partial_item(int e, float *P, const float *A, const float *B) {
   constexpr int KS = DK + 1, VS = DVT + 1, NV = DVT / 4;
-  par<(C / 2) * NV * 4>(x, [&](int e) {
+  {
     const int q = e % 4, rest = e / 4, vg = rest % NV, ip = rest / NV;
     const int i0 = 2 * ip, v0 = 4 * vg;
     float acc[2][4] = {};
@@ -161,10 +165,16 @@ CKDA_UNROLL
     for (int r = 0; r < 2; ++r)
 CKDA_UNROLL
       for (int j = 0; j < 4; ++j) P[(e * 2 + r) * 4 + j] = acc[r][j];
-  });
+  }
 }
 
-// (A B)[i][v] from rows_state_partials' P
+// items of rows_state_partial_item
+template <int DVT>
+struct PartialItems {
+  static constexpr int value = (C / 2) * (DVT / 4) * 4;
+};
+
+// (A B)[i][v] from the partial products of rows_state_partial_item
 template <int DVT>
 CKDA_PROG float rows_state_sum(const float *P, int i, int v) {
   constexpr int NV = DVT / 4;
@@ -224,39 +234,51 @@ template <class X, class IOL, typename IOT, int DK, int DVT>
 CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
                              int n, int tile, int bos, int eos, int slot0) {
   using Ly = ScanLayout<DK, DVT>;
-  constexpr int KS = Ly::KS, VS = Ly::VS;
-  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of the load phase
+  constexpr int KS = Ly::KS, VS = Ly::VS, NP = PartialItems<DVT>::value;
+  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of a load phase
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
-  float *S = sm + Ly::S, *WT = sm + Ly::F0, *KB = sm + Ly::F1, *U = sm + Ly::R0;
-  float *GC = sm + Ly::GC;
-  par<DK * DVT>(x, [&](int e) {
-    const int c = e / DVT, v = e - c * DVT;
-    S[c * VS + v] = a.s0 ? a.s0[st_base + (size_t)c * DVF + v] : 0.f;
+  float *S = sm + Ly::S;
+  // item e of loading chunk ci's W, Kbar, Utilde (rows past its end zero) and
+  // gamma_C into set ci & 1
+  auto load = [&](int e, int ci) {
+    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
+    if (e < C * DK) {
+      const int i = e / DK, c = e - i * DK;
+      const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
+      f[Ly::F0 + i * KS + c] = i < L ? CKDA_LDG(w.wt + o) : 0.f;
+      f[Ly::F1 + i * KS + c] = i < L ? CKDA_LDG(w.kb + o) : 0.f;
+    }
+    if (e < C * DVT) {
+      const int i = e / DVT, v = e - i * DVT;
+      f[Ly::R0 + i * VS + v] =
+          i < L ? CKDA_LDG(w.ut + ((size_t)(t0 + i) * H + h) * DVF + c0 + v) : 0.f;
+    }
+    if (e < DK) f[Ly::GC + e] = CKDA_LDG(w.gc + ((size_t)(slot0 + ci) * H + h) * DK + e);
+  };
+  par<NL>(x, [&](int e) {  // the initial state; chunk 0's factors
+    if (e < DK * DVT) {
+      const int c = e / DVT, v = e - c * DVT;
+      S[c * VS + v] = a.s0 ? a.s0[st_base + (size_t)c * DVF + v] : 0.f;
+    }
+    if (nck > 0) load(e, 0);
   });
   for (int ci = 0; ci < nck; ++ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t slot = (size_t)(slot0 + ci) * H + h;
-    // checkpoint S; load the chunk's W, Kbar, Utilde (rows L..C-1 zero) and gamma_C
+    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    float *WT = f + Ly::F0, *KB = f + Ly::F1, *U = f + Ly::R0, *GC = f + Ly::GC;
+    // checkpoint S; the partial products of W S; chunk ci + 1's factors
     par<NL>(x, [&](int e) {
       if (e < DK * DVT) {
         const int c = e / DVT, v = e - c * DVT;
         w.cks[slot * DK * DVF + (size_t)c * DVF + c0 + v] = S[c * VS + v];
       }
-      if (e < C * DK) {
-        const int i = e / DK, c = e - i * DK;
-        const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
-        WT[i * KS + c] = i < L ? CKDA_LDG(w.wt + o) : 0.f;
-        KB[i * KS + c] = i < L ? CKDA_LDG(w.kb + o) : 0.f;
-      }
-      if (e < C * DVT) {
-        const int i = e / DVT, v = e - i * DVT;
-        U[i * VS + v] = i < L ? CKDA_LDG(w.ut + ((size_t)(t0 + i) * H + h) * DVF + c0 + v) : 0.f;
-      }
-      if (e < DK) GC[e] = CKDA_LDG(w.gc + slot * DK + e);
+      if (e < NP) rows_state_partial_item<DK, DVT>(e, sm + Ly::P, WT, S);
+      if (ci + 1 < nck) load(e, ci + 1);
     });
-    rows_state_partials<DK, DVT>(x, sm + Ly::P, WT, S);
     par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
       const int i = e / DVT, v = e - i * DVT;
       const float s = U[i * VS + v] - rows_state_sum<DVT>(sm + Ly::P, i, v);
@@ -272,42 +294,54 @@ template <class X, class IOL, typename IOT, int DK, int DVT>
 CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *sm, int h,
                              int n, int tile, int bos, int eos, int slot0) {
   using Ly = ScanLayout<DK, DVT>;
-  constexpr int KS = Ly::KS, VS = Ly::VS;
-  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of the load phase
+  constexpr int KS = Ly::KS, VS = Ly::VS, NP = PartialItems<DVT>::value;
+  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of a load phase
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
-  float *DS = sm + Ly::S, *WB = sm + Ly::F0, *QS = sm + Ly::F1, *BK = sm + Ly::F2;
-  float *DR = sm + Ly::R0, *DO = sm + Ly::R1, *GC = sm + Ly::GC;
-  par<DK * DVT>(x, [&](int e) {
-    const int c = e / DVT, v = e - c * DVT;
-    DS[c * VS + v] = a.dsf ? a.dsf[st_base + (size_t)c * DVF + v] : 0.f;
+  float *DS = sm + Ly::S;
+  // item e of loading chunk ci's Wb, Qs, BK, X, dO (rows past its end zero)
+  // and gamma_C into set ci & 1
+  auto load = [&](int e, int ci) {
+    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
+    if (e < C * DK) {
+      const int i = e / DK, c = e - i * DK;
+      const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
+      f[Ly::F0 + i * KS + c] = i < L ? CKDA_LDG(w.wb + o) : 0.f;
+      f[Ly::F1 + i * KS + c] = i < L ? CKDA_LDG(w.qs + o) : 0.f;
+      f[Ly::F2 + i * KS + c] = i < L ? CKDA_LDG(w.bk + o) : 0.f;
+    }
+    if (e < C * DVT) {
+      const int i = e / DVT, v = e - i * DVT;
+      const size_t o = ((size_t)(t0 + i) * H + h) * DVF + c0 + v;
+      f[Ly::R0 + i * VS + v] = i < L ? CKDA_LDG(w.xt + o) : 0.f;
+      f[Ly::R1 + i * VS + v] = i < L ? IOL::ldg(a.d_o + o) : 0.f;
+    }
+    if (e < DK) f[Ly::GC + e] = CKDA_LDG(w.gc + ((size_t)(slot0 + ci) * H + h) * DK + e);
+  };
+  par<NL>(x, [&](int e) {  // the final-state gradient; the last chunk's factors
+    if (e < DK * DVT) {
+      const int c = e / DVT, v = e - c * DVT;
+      DS[c * VS + v] = a.dsf ? a.dsf[st_base + (size_t)c * DVF + v] : 0.f;
+    }
+    if (nck > 0) load(e, nck - 1);
   });
   for (int ci = nck - 1; ci >= 0; --ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t slot = (size_t)(slot0 + ci) * H + h;
-    // checkpoint dS_C; load the chunk's Wb, Qs, BK, X, dO (rows L..C-1 zero) and gamma_C
+    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    float *WB = f + Ly::F0, *QS = f + Ly::F1, *BK = f + Ly::F2, *DR = f + Ly::R0,
+          *DO = f + Ly::R1, *GC = f + Ly::GC;
+    // checkpoint dS_C; the partial products of Wb dS_C; chunk ci - 1's factors
     par<NL>(x, [&](int e) {
       if (e < DK * DVT) {
         const int c = e / DVT, v = e - c * DVT;
         w.ckd[slot * DK * DVF + (size_t)c * DVF + c0 + v] = DS[c * VS + v];
       }
-      if (e < C * DK) {
-        const int i = e / DK, c = e - i * DK;
-        const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
-        WB[i * KS + c] = i < L ? CKDA_LDG(w.wb + o) : 0.f;
-        QS[i * KS + c] = i < L ? CKDA_LDG(w.qs + o) : 0.f;
-        BK[i * KS + c] = i < L ? CKDA_LDG(w.bk + o) : 0.f;
-      }
-      if (e < C * DVT) {
-        const int i = e / DVT, v = e - i * DVT;
-        const size_t o = ((size_t)(t0 + i) * H + h) * DVF + c0 + v;
-        DR[i * VS + v] = i < L ? CKDA_LDG(w.xt + o) : 0.f;
-        DO[i * VS + v] = i < L ? IOL::ldg(a.d_o + o) : 0.f;
-      }
-      if (e < DK) GC[e] = CKDA_LDG(w.gc + slot * DK + e);
+      if (e < NP) rows_state_partial_item<DK, DVT>(e, sm + Ly::P, WB, DS);
+      if (ci > 0) load(e, ci - 1);
     });
-    rows_state_partials<DK, DVT>(x, sm + Ly::P, WB, DS);
     par<C * DVT>(x, [&](int e) {  // dR = X + Wb dS_C
       const int j = e / DVT, v = e - j * DVT;
       const float s = DR[j * VS + v] + rows_state_sum<DVT>(sm + Ly::P, j, v);

@@ -204,12 +204,15 @@ CKDA_UNROLL
 template <int DK, int DVT>
 struct ScanLayout {
   static constexpr int KS = 2 * (DK + 1), VS = 2 * (DVT + 1), CS = 2 * (C + 1);
-  // DK x DVT complex state; C x DK complex W, Kbar, Qhat; C x DVT complex U;
-  // C x C complex M; gamma_{C-1} [DK] complex
-  static constexpr int S = 0, WT = S + DK * VS, KB = WT + C * KS, QH = KB + C * KS,
-                       U = QH + C * KS, M = U + C * VS, GC = M + C * CS;
-  // partial products of W S and Qhat S: 4 quarters of C x DVT complex each
-  static constexpr int PW = GC + 2 * DK, PQ = PW + 8 * C * DVT;
+  // two sets of a chunk's factors (chunk i in set i & 1, so that the next
+  // chunk's loads overlap this chunk's products): C x DK complex W, Kbar, Qhat;
+  // C x DVT complex Utilde (then U); C x C complex M; gamma_{C-1} [DK]
+  // complex; offsets within a set
+  static constexpr int WT = 0, KB = WT + C * KS, QH = KB + C * KS, UT = QH + C * KS,
+                       M = UT + C * VS, GC = M + C * CS, SET = GC + 2 * DK;
+  // DK x DVT complex state; the sets; partial products of W S and Qhat S (4
+  // quarters of C x DVT complex each)
+  static constexpr int S = 0, SETS = S + DK * VS, PW = SETS + 2 * SET, PQ = PW + 8 * C * DVT;
   static constexpr int FLOATS = PQ + 8 * C * DVT;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
@@ -219,85 +222,101 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
                             int bos, int eos, int slot0) {
   using Ly = ScanLayout<DK, DVT>;
   constexpr int KS = Ly::KS, VS = Ly::VS, CS = Ly::CS, NV = DVT / 4;
+  constexpr int NP = (C / 2) * NV * 4;                       // items of the W S, Qhat S pass
+  constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of a load phase
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;  // complex elements
-  float *S = sm + Ly::S, *U = sm + Ly::U;
-  par<DK * DVT>(x, [&](int e) {
-    const int c = e / DVT, v = e - c * DVT;
-    // plain load: the final state may overwrite the initial one in place
-    const cf s = a.s0 ? cld(a.s0 + (st_base + (size_t)c * DVF + v) * 2) : cf{0.f, 0.f};
-    cst(S + c * VS + 2 * v, s);
-  });
-  for (int ci = 0; ci < nck; ++ci) {
+  float *S = sm + Ly::S;
+  const cf zero{0.f, 0.f};
+  // item e of loading chunk ci's factors (rows past its end zero) into set ci & 1
+  auto load = [&](int e, int ci) {
+    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t sl = (size_t)(slot0 + ci) * H + h;
-    par<C * DK>(x, [&](int e) {  // the chunk's factors; rows L..C-1 zero
+    if (e < C * DK) {
       const int i = e / DK, c = e - i * DK;
       const size_t o = (((size_t)(t0 + i) * H + h) * DK + c) * 2;
       const bool in = i < L;
-      cst(sm + Ly::WT + i * KS + 2 * c, in ? cldg(w.wt + o) : cf{0.f, 0.f});
-      cst(sm + Ly::KB + i * KS + 2 * c, in ? cldg(w.kb + o) : cf{0.f, 0.f});
-      cst(sm + Ly::QH + i * KS + 2 * c, in ? cldg(w.qh + o) : cf{0.f, 0.f});
-      if (e < C * C)
-        cst(sm + Ly::M + (e / C) * CS + 2 * (e % C), cldg(w.mm + (sl * C * C + e) * 2));
-      if (e < DK) cst(sm + Ly::GC + 2 * e, cldg(w.gc + (sl * DK + e) * 2));
-    });
+      cst(f + Ly::WT + i * KS + 2 * c, in ? cldg(w.wt + o) : zero);
+      cst(f + Ly::KB + i * KS + 2 * c, in ? cldg(w.kb + o) : zero);
+      cst(f + Ly::QH + i * KS + 2 * c, in ? cldg(w.qh + o) : zero);
+    }
+    if (e < C * DVT) {
+      const int i = e / DVT, v = e - i * DVT;
+      cst(f + Ly::UT + i * VS + 2 * v,
+          i < L ? cldg(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2) : zero);
+    }
+    if (e < C * C) cst(f + Ly::M + (e / C) * CS + 2 * (e % C), cldg(w.mm + (sl * C * C + e) * 2));
+    if (e < DK) cst(f + Ly::GC + 2 * e, cldg(w.gc + (sl * DK + e) * 2));
+  };
+  par<NL>(x, [&](int e) {  // the initial state; chunk 0's factors
+    if (e < DK * DVT) {
+      const int c = e / DVT, v = e - c * DVT;
+      // plain load: the final state may overwrite the initial one in place
+      const cf s = a.s0 ? cld(a.s0 + (st_base + (size_t)c * DVF + v) * 2) : zero;
+      cst(S + c * VS + 2 * v, s);
+    }
+    if (nck > 0) load(e, 0);
+  });
+  for (int ci = 0; ci < nck; ++ci) {
+    const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
+    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    float *U = f + Ly::UT;
     // W S and Qhat S in one pass over S: item (row pair, 4 columns, quarter q)
-    // sums channels q, q + 4, ... in 2 x 4 complex register tiles
-    par<(C / 2) * NV * 4>(x, [&](int e) {
-      const int q = e % 4, rest = e / 4, vg = rest % NV, ip = rest / NV;
-      const int i0 = 2 * ip, v0 = 4 * vg;
-      cf aw[2][4], aq[2][4];
+    // sums channels q, q + 4, ... in 2 x 4 complex register tiles; chunk
+    // ci + 1's factors load meanwhile
+    par<NL>(x, [&](int e) {
+      if (e < NP) {
+        const int q = e % 4, rest = e / 4, vg = rest % NV, ip = rest / NV;
+        const int i0 = 2 * ip, v0 = 4 * vg;
+        cf aw[2][4], aq[2][4];
 CKDA_UNROLL
-      for (int r = 0; r < 2; ++r)
+        for (int r = 0; r < 2; ++r)
 CKDA_UNROLL
-        for (int j = 0; j < 4; ++j) aw[r][j] = aq[r][j] = cf{0.f, 0.f};
-      for (int c = q; c < DK; c += 4) {
-        const cf w0 = cld(sm + Ly::WT + i0 * KS + 2 * c);
-        const cf w1 = cld(sm + Ly::WT + (i0 + 1) * KS + 2 * c);
-        const cf q0 = cld(sm + Ly::QH + i0 * KS + 2 * c);
-        const cf q1 = cld(sm + Ly::QH + (i0 + 1) * KS + 2 * c);
+          for (int j = 0; j < 4; ++j) aw[r][j] = aq[r][j] = zero;
+        for (int c = q; c < DK; c += 4) {
+          const cf w0 = cld(f + Ly::WT + i0 * KS + 2 * c);
+          const cf w1 = cld(f + Ly::WT + (i0 + 1) * KS + 2 * c);
+          const cf q0 = cld(f + Ly::QH + i0 * KS + 2 * c);
+          const cf q1 = cld(f + Ly::QH + (i0 + 1) * KS + 2 * c);
 CKDA_UNROLL
-        for (int j = 0; j < 4; ++j) {
-          const cf sv = cld(S + c * VS + 2 * (v0 + j));
-          aw[0][j] = cadd(aw[0][j], cmul(w0, sv));
-          aw[1][j] = cadd(aw[1][j], cmul(w1, sv));
-          aq[0][j] = cadd(aq[0][j], cmul(q0, sv));
-          aq[1][j] = cadd(aq[1][j], cmul(q1, sv));
+          for (int j = 0; j < 4; ++j) {
+            const cf sv = cld(S + c * VS + 2 * (v0 + j));
+            aw[0][j] = cadd(aw[0][j], cmul(w0, sv));
+            aw[1][j] = cadd(aw[1][j], cmul(w1, sv));
+            aq[0][j] = cadd(aq[0][j], cmul(q0, sv));
+            aq[1][j] = cadd(aq[1][j], cmul(q1, sv));
+          }
         }
+CKDA_UNROLL
+        for (int r = 0; r < 2; ++r)
+CKDA_UNROLL
+          for (int j = 0; j < 4; ++j) {
+            cst(sm + Ly::PW + ((e * 2 + r) * 4 + j) * 2, aw[r][j]);
+            cst(sm + Ly::PQ + ((e * 2 + r) * 4 + j) * 2, aq[r][j]);
+          }
       }
-CKDA_UNROLL
-      for (int r = 0; r < 2; ++r)
-CKDA_UNROLL
-        for (int j = 0; j < 4; ++j) {
-          cst(sm + Ly::PW + ((e * 2 + r) * 4 + j) * 2, aw[r][j]);
-          cst(sm + Ly::PQ + ((e * 2 + r) * 4 + j) * 2, aq[r][j]);
-        }
+      if (ci + 1 < nck) load(e, ci + 1);
     });
     // the four quarters of (row i, column v) in a fixed order
     auto quarters = [&](int base, int i, int v) {
       const int e0 = (((i / 2) * NV + v / 4) * 4) * 2 + (i % 2), j = v % 4;
-      cf s{0.f, 0.f};
+      cf s = zero;
 CKDA_UNROLL
       for (int q4 = 0; q4 < 4; ++q4) s = cadd(s, cld(sm + base + ((e0 + 2 * q4) * 4 + j) * 2));
       return s;
     };
-    par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
+    par<C * DVT>(x, [&](int e) {  // U = Utilde - W S (rows past the end stay zero)
       const int i = e / DVT, v = e - i * DVT;
-      if (i >= L) {
-        cst(U + i * VS + 2 * v, cf{0.f, 0.f});
-        return;
-      }
-      const cf u = cldg(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
-      cst(U + i * VS + 2 * v, csub(u, quarters(Ly::PW, i, v)));
+      if (i < L) cst(U + i * VS + 2 * v, csub(cld(U + i * VS + 2 * v), quarters(Ly::PW, i, v)));
     });
     par<C * DVT>(x, [&](int e) {  // o = conj(scale (Qhat S + M U))
       const int i = e / DVT, v = e - i * DVT;
       if (i >= L) return;
       cf s = quarters(Ly::PQ, i, v);
       for (int j = 0; j <= i; ++j)
-        s = cadd(s, cmul(cld(sm + Ly::M + i * CS + 2 * j), cld(U + j * VS + 2 * v)));
+        s = cadd(s, cmul(cld(f + Ly::M + i * CS + 2 * j), cld(U + j * VS + 2 * v)));
       cst(a.o + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2, cconj(cscale(a.scale, s)));
     });
     // S <- diag(gamma_{C-1}) S + Kbar^T U, in 2 x 4 complex register tiles
@@ -306,14 +325,14 @@ CKDA_UNROLL
       cf acc[2][4];
 CKDA_UNROLL
       for (int r = 0; r < 2; ++r) {
-        const cf g = cld(sm + Ly::GC + 2 * (cc + r));
+        const cf g = cld(f + Ly::GC + 2 * (cc + r));
 CKDA_UNROLL
         for (int j = 0; j < 4; ++j) acc[r][j] = cmul(g, cld(S + (cc + r) * VS + 2 * (v0 + j)));
       }
 CKDA_UNROLL
       for (int i = 0; i < C; ++i) {
-        const cf k0 = cld(sm + Ly::KB + i * KS + 2 * cc);
-        const cf k1 = cld(sm + Ly::KB + i * KS + 2 * (cc + 1));
+        const cf k0 = cld(f + Ly::KB + i * KS + 2 * cc);
+        const cf k1 = cld(f + Ly::KB + i * KS + 2 * (cc + 1));
 CKDA_UNROLL
         for (int j = 0; j < 4; ++j) {
           const cf uv = cld(U + i * VS + 2 * (v0 + j));
