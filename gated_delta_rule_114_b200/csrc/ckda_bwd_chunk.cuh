@@ -22,7 +22,7 @@
 // special. Only dS crosses chunks.
 //
 // This file holds the pieces one chunk needs (staging, gate products, Grams
-// and the UT solve, Khat S, the per-channel gate gradient); ckda_bwd_split.cuh
+// and the UT solve, the per-channel gate gradient); ckda_bwd_split.cuh
 // composes them into the four programs of the backward. The columns of S and
 // dS are independent; everything that sums over columns (dq, dk, dalpha,
 // dbeta) is linear in per-column terms, so the gradient program adds the
@@ -179,20 +179,6 @@ CKDA_UNROLL
       for (int m = j; m < i; ++m) s += ab[i * CS + m] * tt[m * CS + j];
       tt[i * CS + j] = -be[i] * s;
     }
-  });
-}
-
-// Khat S (into the Khat S rows)
-template <class X, class Ly>
-CKDA_PROG void chunk_khat_s(X &x, float *sm) {
-  constexpr int DK = Ly::dk, DVT = Ly::dvt, KS = Ly::KS, VS = Ly::VS;
-  const float *kk = sm + Ly::K;
-  par<C * DVT>(x, [&](int e) {
-    const int i = e / DVT, v = e - i * DVT;
-    float ks = 0.f;
-    for (int c = 0; c < DK; ++c)
-      ks += sm[Ly::GM + i * KS + c] * kk[i * KS + c] * sm[Ly::S + c * VS + v];
-    sm[Ly::KSW + i * VS + v] = ks;
   });
 }
 

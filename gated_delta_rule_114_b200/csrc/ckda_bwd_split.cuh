@@ -370,18 +370,19 @@ struct GradLayout {
   // U dS_C^T, overwritten by the gate-gradient coefficients E0 (over XQ) and
   // EX (over XB)
   static constexpr int Q = 0, K = Q + C * KS, AL = K + C * KS, GM = AL + C * KS,
-                       SG = GM + C * KS, XQ = SG + C * KS, XK = XQ + C * KS, XB = XK + C * KS;
+                       SG = GM + C * KS, XQ = SG + C * KS, XK = XQ + C * KS, XB = XK + C * KS,
+                       KH = XB + C * KS;  // KH: Khat = gamma * k
   static constexpr int E0 = XQ, EX = XB;
   // C x GT: v, dO, Khat S then w, U, dR of the current column tile
-  static constexpr int V = XB + C * KS, DO = V + C * VS, KSW = DO + C * VS, U = KSW + C * VS,
+  static constexpr int V = KH + C * KS, DO = V + C * VS, KSW = DO + C * VS, U = KSW + C * VS,
                        DR = U + C * VS;
   // DK x GT: the tile of the entry state and of the exit-state gradient
   static constexpr int S = DR + C * VS, DS = S + DK * VS;
   // C x C: Abar, dM and dAbar (summed over the tiles)
   static constexpr int AB = DS + DK * VS, DM = AB + C * CS, DA = DM + C * CS;
-  // beta [C], dbeta [C], sum_v S dS_C per channel [DK]
-  static constexpr int BE = DA + C * CS, DB = BE + C, SDS = DB + C;
-  static constexpr int FLOATS = SDS + DK;
+  // beta [C], dbeta [C], sum_v S dS_C per channel [DK]; partial products of Khat S
+  static constexpr int BE = DA + C * CS, DB = BE + C, SDS = DB + C, P = SDS + DK;
+  static constexpr int FLOATS = P + 4 * C * GT;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
 
@@ -428,6 +429,10 @@ CKDA_PROG void grads_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
     if (e < DK) sm[Ly::SDS + e] = 0.f;
   });
   chunk_gates<X, Ly>(x, sm);
+  par<C * DK>(x, [&](int e) {  // Khat = gamma * k
+    const int i = e / DK, c = e - i * DK;
+    sm[Ly::KH + i * KS + c] = sm[Ly::GM + i * KS + c] * kk[i * KS + c];
+  });
   for (int c0 = 0; c0 < DVF; c0 += GT) {
     // the tile's S, dS_C and rows of U, dR, v, dO (rows L..C-1 zero)
     par<DK * GT>(x, [&](int e) {
@@ -445,13 +450,15 @@ CKDA_PROG void grads_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
         sm[Ly::DO + i * VS + u] = in ? IOL::ldg(a.d_o + r) : 0.f;
       }
     });
-    chunk_khat_s<X, Ly>(x, sm);
-    // w = V - Khat S - Abar U (over the Khat S rows); dv = diag(beta) dR
+    // Khat S in 2 x 4 register tiles (split d_k sums); then
+    // w = V - Khat S - Abar U (into the Khat S rows) and dv = diag(beta) dR
+    par<PartialItems<GT>::value>(
+        x, [&](int e) { rows_state_partial_item<DK, GT>(e, sm + Ly::P, sm + Ly::KH, sm + Ly::S); });
     par<C * GT>(x, [&](int e) {
       const int i = e / GT, v = e - i * GT;
-      float s = 0.f;
+      float s = rows_state_sum<GT>(sm + Ly::P, i, v);
       for (int m = 0; m < i; ++m) s += sm[Ly::AB + i * CS + m] * sm[Ly::U + m * VS + v];
-      sm[Ly::KSW + i * VS + v] = sm[Ly::V + i * VS + v] - sm[Ly::KSW + i * VS + v] - s;
+      sm[Ly::KSW + i * VS + v] = sm[Ly::V + i * VS + v] - s;
       if (i < L)
         IOL::st(a.dv + ((size_t)(t0 + i) * H + h) * DVF + c0 + v, be[i] * sm[Ly::DR + i * VS + v]);
     });
@@ -475,30 +482,41 @@ CKDA_PROG void grads_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
       }
     });
     // the tile's share of dO S^T, dR S^T, U dS_C^T and of sum_v S dS_C, per
-    // (row r, channels cq + t DK/4)
-    par<C * NQ>(x, [&](int e) {
-      const int r = e / NQ, cq = e - r * NQ;
-      float xq[4] = {}, xk[4] = {}, xb[4] = {}, sd[4] = {};
+    // (rows 2rp, 2rp + 1; channels cq + t DK/4): each S, dS_C load serves both rows
+    par<(C / 2) * NQ>(x, [&](int e) {
+      const int rp = e / NQ, cq = e - rp * NQ, r0 = 2 * rp;
+      float xq[2][4] = {}, xk[2][4] = {}, xb[2][4] = {}, sd[4] = {};
       for (int v = 0; v < GT; ++v) {
-        const float dov = sm[Ly::DO + r * VS + v], drv = sm[Ly::DR + r * VS + v];
-        const float uv = sm[Ly::U + r * VS + v];
+        float dov[2], drv[2], uv[2];
+CKDA_UNROLL
+        for (int r = 0; r < 2; ++r) {
+          dov[r] = sm[Ly::DO + (r0 + r) * VS + v];
+          drv[r] = sm[Ly::DR + (r0 + r) * VS + v];
+          uv[r] = sm[Ly::U + (r0 + r) * VS + v];
+        }
 CKDA_UNROLL
         for (int t = 0; t < 4; ++t) {
           const int c = cq + t * NQ;
           const float sv = sm[Ly::S + c * VS + v], dsv = sm[Ly::DS + c * VS + v];
-          xq[t] += dov * sv;
-          xk[t] += drv * sv;
-          xb[t] += uv * dsv;
+CKDA_UNROLL
+          for (int r = 0; r < 2; ++r) {
+            xq[r][t] += dov[r] * sv;
+            xk[r][t] += drv[r] * sv;
+            xb[r][t] += uv[r] * dsv;
+          }
           sd[t] += sv * dsv;
         }
       }
 CKDA_UNROLL
       for (int t = 0; t < 4; ++t) {
         const int c = cq + t * NQ;
-        sm[Ly::XQ + r * KS + c] += xq[t];
-        sm[Ly::XK + r * KS + c] += xk[t];
-        sm[Ly::XB + r * KS + c] += xb[t];
-        if (r == 0) sm[Ly::SDS + c] += sd[t];
+CKDA_UNROLL
+        for (int r = 0; r < 2; ++r) {
+          sm[Ly::XQ + (r0 + r) * KS + c] += xq[r][t];
+          sm[Ly::XK + (r0 + r) * KS + c] += xk[r][t];
+          sm[Ly::XB + (r0 + r) * KS + c] += xb[r][t];
+        }
+        if (rp == 0) sm[Ly::SDS + c] += sd[t];
       }
     });
   }
