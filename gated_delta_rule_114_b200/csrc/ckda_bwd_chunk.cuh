@@ -30,10 +30,10 @@
 //
 // Every program is a fixed sequence of data-parallel phases. par<N>(x, f)
 // runs one phase on executor X: f(i) for every i in [0, N), the calls
-// independent of one another, then a barrier. Every value that outlives a phase sits in
-// the shared-memory block `sm` (or in global memory), so the same source runs
-// as a CUDA kernel (threads stride over i, __syncthreads between phases) and,
-// for tests, as plain host loops. Gate products inside a 16-token chunk are
+// independent of one another, then a barrier. Every value that outlives a
+// phase sits in the shared-memory block `sm` (or in global memory), so the
+// same source runs as a CUDA kernel (threads stride over i, __syncthreads
+// between phases) and, for tests, as plain host loops. Gate products inside a 16-token chunk are
 // short running products (at most 15 factors), so every factor keeps its sign
 // and its zeros exactly. fp32 throughout.
 #pragma once
