@@ -20,10 +20,15 @@
 
 namespace {
 
+// Runs a phase's items in index order, or in reverse when `reverse` is set:
+// the two orders give bit-identical results only if no item reads what
+// another item of the same phase writes, which is what the GPU's concurrent
+// threads need.
 struct HostExec {
+  bool reverse = false;
   template <int N, class F>
   void run(F f) {
-    for (int i = 0; i < N; ++i) f(i);
+    for (int i = 0; i < N; ++i) f(reverse ? N - 1 - i : i);
   }
 };
 
@@ -75,6 +80,7 @@ void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool 
     eos = varlen ? cu[n + 1] : bos + T;
   };
   HostExec x;
+  x.reverse = std::getenv("EMU_REVERSE_ITEMS") != nullptr;
   std::vector<float> psm(cplx::PrepLayout<DK, DVT>::FLOATS), ssm(cplx::ScanLayout<DK, DVT>::FLOATS);
   for (int h = 0; h < H; ++h)
     for (int g = 0; g < (int)slots; ++g) {

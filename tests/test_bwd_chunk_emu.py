@@ -63,7 +63,7 @@ def f32(x):
     return np.ascontiguousarray(x.numpy() if hasattr(x, "numpy") else x, dtype=np.float32)
 
 
-def run_emu(exe, tmp, inp, grads, scale, varlen=True, N=None, T=None):
+def run_emu(exe, tmp, inp, grads, scale, varlen=True, N=None, T=None, reverse=False):
     q = f32(inp["q"])
     Tt, H, dk = q.shape
     dv = inp["v"].shape[2]
@@ -79,8 +79,13 @@ def run_emu(exe, tmp, inp, grads, scale, varlen=True, N=None, T=None):
     if varlen:
         cu.tofile(os.path.join(tmp, "cu.bin"))
         N, T = len(cu) - 1, Tt
+    env = dict(os.environ)
+    env.pop("EMU_REVERSE_ITEMS", None)
+    if reverse:
+        env["EMU_REVERSE_ITEMS"] = "1"
     subprocess.check_call([exe, tmp, str(N), str(T), str(H), str(dk), str(dv), repr(scale),
-                           str(int(varlen)), str(int("s0" in files)), str(int("dsf" in files))])
+                           str(int(varlen)), str(int("s0" in files)), str(int("dsf" in files))],
+                          env=env)
 
     def rd(name, shape):
         return np.fromfile(os.path.join(tmp, name + ".bin"), dtype=np.float32).reshape(shape)
@@ -147,3 +152,15 @@ def test_degenerate_gates(emu, tmp_path, kind):
         a = np.where((u >= 0.2) & (u < 0.25), 1e-6 * rng.normal(size=shape), a)
     inp["alpha"] = torch.from_numpy(a.astype(np.float32))
     compare(run_emu(emu, str(tmp_path), inp, grads, 1.0), run_ref(inp, grads, 1.0))
+
+
+def test_items_of_a_phase_are_independent(emu, tmp_path):
+    """Every phase's items in reverse order give bit-identical gradients: no
+    item reads what another item of its phase writes (the GPU runs them at
+    once)."""
+    w = custom("ckda_B1_H32_T8192_d128", dtype="f32", d_k=64, d_v=64, seed=830)
+    inp, grads = make_case(w, [37, 16, 5], H=2)
+    fwd = run_emu(emu, str(tmp_path), inp, grads, 0.9)
+    rev = run_emu(emu, str(tmp_path), inp, grads, 0.9, reverse=True)
+    for name, x, y in zip(NAMES, fwd, rev):
+        assert np.array_equal(x, y), name

@@ -53,7 +53,7 @@ def c64(x):
     return np.ascontiguousarray(torch.view_as_real(x.to(torch.complex64)).numpy())
 
 
-def run_emu(exe, tmp, inp, scale, with_s0=True, varlen=True, N=None, T=None):
+def run_emu(exe, tmp, inp, scale, with_s0=True, varlen=True, N=None, T=None, reverse=False):
     Tt, H, dk = inp["q"].shape
     dv = inp["v"].shape[2]
     for name in ("q", "k", "v"):
@@ -67,8 +67,12 @@ def run_emu(exe, tmp, inp, scale, with_s0=True, varlen=True, N=None, T=None):
     if varlen:
         cu.tofile(os.path.join(tmp, "cu.bin"))
         N, T = len(cu) - 1, Tt
+    env = dict(os.environ)
+    env.pop("EMU_REVERSE_ITEMS", None)
+    if reverse:
+        env["EMU_REVERSE_ITEMS"] = "1"
     subprocess.check_call([exe, tmp, str(N), str(T), str(H), str(dk), str(dv), repr(scale),
-                           str(int(varlen)), str(int(with_s0))])
+                           str(int(varlen)), str(int(with_s0))], env=env)
     o = np.fromfile(os.path.join(tmp, "o.bin"), dtype=np.float32).reshape(Tt, H, dv, 2)
     sf = np.fromfile(os.path.join(tmp, "sf.bin"), dtype=np.float32).reshape(N, H, dk, dv, 2)
     return o, sf
@@ -120,3 +124,13 @@ def test_degenerate_gates(emu, tmp_path, kind):
         a = torch.sign(a)
     inp["alpha"] = a.contiguous()
     check(run_emu(emu, str(tmp_path), inp, 1.0), inp, 1.0)
+
+
+def test_items_of_a_phase_are_independent(emu, tmp_path):
+    """Every phase's items in reverse order give bit-identical outputs: no item
+    reads what another item of its phase writes (the GPU runs them at once)."""
+    w = custom(d_k=64, d_v=64, seed=950)
+    inp = make_complex_inputs(w, lens_cu([37, 16, 5]), H=2, ranges="ckda")
+    fwd = run_emu(emu, str(tmp_path), inp, 0.9)
+    rev = run_emu(emu, str(tmp_path), inp, 0.9, reverse=True)
+    assert np.array_equal(fwd[0], rev[0]) and np.array_equal(fwd[1], rev[1])
