@@ -1,8 +1,8 @@
 // The split chunkwise backward (ckda_bwd_split.cuh) as four kernels on CUDA
 // cores (sm_100a):
 //   prep   grid (checkpoint slots, H)   256 threads, parallel over chunks
-//   scan1  grid (H, N, d_v tiles)       entry states and U, chunk by chunk
-//   scan2  grid (H, N, d_v tiles)       exit-state gradients and dR, in reverse
+//   scan1  grid (H, N, d_v / 16)        entry states and U, chunk by chunk
+//   scan2  grid (H, N, d_v / 16)        exit-state gradients and dR, in reverse
 //   grads  grid (checkpoint slots, H)   every gradient of a chunk, its columns
 //                                       in 16-column tiles added in order
 // A slot that starts no chunk (slots are floor(cu[n] / 16) + n + chunk) exits
@@ -20,6 +20,7 @@ namespace ckda {
 namespace {
 
 constexpr int kGradTile = 16;  // columns per tile of the gradient program
+constexpr int kScanTile = 16;  // columns per CTA of the scans (and per tile of prep)
 
 constexpr int kThreads = 256;
 
@@ -161,19 +162,20 @@ cudaError_t launch_bwd_split(int dk_, int dv_, const void *q, const void *k, con
                              float *dalpha, float *dbeta, float *ds0, const int32_t *cu, int N,
                              int T, int T_total, int H, float scale, void *ws,
                              unsigned int *err, cudaStream_t st) {
-  const int dvt = dv_ < 32 ? dv_ : 32;
   const bwdc::SplitWs w = carve(static_cast<float *>(ws), N, T_total, H, dk_, dv_);
   bwdc::Args<IOT> a{static_cast<const IOT *>(q),  static_cast<const IOT *>(k),
                     static_cast<const IOT *>(v),  alpha, beta, s0,
                     static_cast<const IOT *>(d_o), dsf,
                     static_cast<IOT *>(dq),       static_cast<IOT *>(dk),
                     static_cast<IOT *>(dv),       dalpha, dbeta, ds0, H, dv_, scale};
-#define CKDA_BWDS_DK(X)                                                      \
-  if (dk_ == X)                                                              \
-    return dvt == 16 ? launch_dims<IOT, X, 16>(a, w, cu, N, T, T_total, err, st) \
-                     : launch_dims<IOT, X, 32>(a, w, cu, N, T, T_total, err, st);
-  CKDA_BWDS_DK(16) CKDA_BWDS_DK(32) CKDA_BWDS_DK(64) CKDA_BWDS_DK(128)
-#undef CKDA_BWDS_DK
+  // the scans take 16-column tiles: twice the CTAs of 32-column ones (d_v / 16
+  // per sequence and head), each with half the work per chunk, up to three per SM
+  switch (dk_) {
+    case 16: return launch_dims<IOT, 16, kScanTile>(a, w, cu, N, T, T_total, err, st);
+    case 32: return launch_dims<IOT, 32, kScanTile>(a, w, cu, N, T, T_total, err, st);
+    case 64: return launch_dims<IOT, 64, kScanTile>(a, w, cu, N, T, T_total, err, st);
+    case 128: return launch_dims<IOT, 128, kScanTile>(a, w, cu, N, T, T_total, err, st);
+  }
   return cudaErrorInvalidValue;
 }
 

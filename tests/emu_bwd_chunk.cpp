@@ -148,13 +148,12 @@ int main(int argc, char **argv) {
   const int dk = std::atoi(argv[5]), dv = std::atoi(argv[6]);
   const float scale = (float)std::atof(argv[7]);
   const bool varlen = std::atoi(argv[8]), s0 = std::atoi(argv[9]), dsf = std::atoi(argv[10]);
-#define EMU_CASE(DK, DVT)                                       \
-  if (dk == DK && (dv < 32 ? dv : 32) == DVT) {                 \
-    run<DK, DVT>(dir, N, T, H, dv, scale, varlen, s0, dsf);     \
-    return 0;                                                   \
+#define EMU_CASE(DK)                                          \
+  if (dk == DK) { /* 16-column scan tiles, as the kernels */  \
+    run<DK, 16>(dir, N, T, H, dv, scale, varlen, s0, dsf);    \
+    return 0;                                                 \
   }
-  EMU_CASE(16, 16) EMU_CASE(16, 32) EMU_CASE(32, 16) EMU_CASE(32, 32)
-  EMU_CASE(64, 16) EMU_CASE(64, 32) EMU_CASE(128, 16) EMU_CASE(128, 32)
+  EMU_CASE(16) EMU_CASE(32) EMU_CASE(64) EMU_CASE(128)
 #undef EMU_CASE
   std::fprintf(stderr, "unsupported d_k=%d d_v=%d\n", dk, dv);
   return 1;
