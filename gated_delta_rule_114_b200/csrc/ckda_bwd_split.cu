@@ -13,6 +13,7 @@
 #include "ckda.h"
 #include "ckda_bwd_split.cuh"
 #include "ckda_common.cuh"
+#include "ckda_exec.cuh"
 #include "ckda_rowcol.cuh"
 
 namespace ckda {
@@ -24,20 +25,7 @@ constexpr int kScanTile = 16;  // columns per CTA of the scans (and per tile of 
 
 constexpr int kThreads = 256;
 
-// One phase: this thread's items threadIdx.x + r * kThreads, fully unrolled,
-// then the CTA's barrier.
-struct DeviceExec {
-  template <int N, class F>
-  __device__ __forceinline__ void run(F f) {
-    constexpr int R = (N + kThreads - 1) / kThreads;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int i = threadIdx.x + r * kThreads;
-      if (N % kThreads == 0 || i < N) f(i);
-    }
-    __syncthreads();
-  }
-};
+using Exec = DeviceExec<kThreads>;  // one phase per barrier, kThreads threads
 
 // the chunk of slot blockIdx.x: token rows [t0, t0 + L); false if none
 __device__ __forceinline__ bool slot_rows(const int32_t *cu, int N, int T, int T_total,
@@ -59,8 +47,8 @@ bwd_prep_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ 
   extern __shared__ float sm[];
   int t0, L;
   if (!slot_rows(cu, N, T, T_total, err, t0, L)) return;
-  DeviceExec x;
-  bwdc::prep_program<DeviceExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, blockIdx.y, t0, L,
+  Exec x;
+  bwdc::prep_program<Exec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, blockIdx.y, t0, L,
                                                         blockIdx.x);
 }
 
@@ -72,12 +60,12 @@ bwd_scan_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ 
   const int h = blockIdx.x, n = blockIdx.y, tile = blockIdx.z;
   int bos, eos;
   seq_bounds(cu, n, T, T_total, err, bos, eos);
-  DeviceExec x;
+  Exec x;
   if (REVERSE)
-    bwdc::scan2_program<DeviceExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
+    bwdc::scan2_program<Exec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
                                                            bos / CK + n);
   else
-    bwdc::scan1_program<DeviceExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
+    bwdc::scan1_program<Exec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
                                                            bos / CK + n);
 }
 
@@ -88,8 +76,8 @@ bwd_grads_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__
   extern __shared__ float sm[];
   int t0, L;
   if (!slot_rows(cu, N, T, T_total, err, t0, L)) return;
-  DeviceExec x;
-  bwdc::grads_program<DeviceExec, IO<IOT>, IOT, DK, kGradTile>(x, a, w, sm, blockIdx.y, t0, L,
+  Exec x;
+  bwdc::grads_program<Exec, IO<IOT>, IOT, DK, kGradTile>(x, a, w, sm, blockIdx.y, t0, L,
                                                                blockIdx.x);
 }
 

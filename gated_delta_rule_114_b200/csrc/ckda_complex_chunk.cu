@@ -9,6 +9,7 @@
 #include "ckda.h"
 #include "ckda_bwd_split.cuh"
 #include "ckda_common.cuh"
+#include "ckda_exec.cuh"
 #include "ckda_complex_chunk.cuh"
 #include "ckda_rowcol.cuh"
 
@@ -17,20 +18,7 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// One phase: this thread's items threadIdx.x + r * kThreads, fully unrolled,
-// then the CTA's barrier.
-struct DeviceExec {
-  template <int N, class F>
-  __device__ __forceinline__ void run(F f) {
-    constexpr int R = (N + kThreads - 1) / kThreads;
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const int i = threadIdx.x + r * kThreads;
-      if (N % kThreads == 0 || i < N) f(i);
-    }
-    __syncthreads();
-  }
-};
+using Exec = DeviceExec<kThreads>;  // one phase per barrier, kThreads threads
 
 template <int DK, int DVT>
 __global__ void __launch_bounds__(kThreads)
@@ -43,8 +31,8 @@ complex_prep_kernel(cplx::Args a, cplx::Ws w, const int32_t *__restrict__ cu, in
   seq_bounds(cu, n, T, T_total, err, bos, eos);
   if (ci >= (eos - bos + CK - 1) / CK) return;
   const int t0 = bos + CK * ci, L = eos - t0 < CK ? eos - t0 : CK;
-  DeviceExec x;
-  cplx::prep_program<DeviceExec, DK, DVT>(x, a, w, sm, blockIdx.y, t0, L, blockIdx.x);
+  Exec x;
+  cplx::prep_program<Exec, DK, DVT>(x, a, w, sm, blockIdx.y, t0, L, blockIdx.x);
 }
 
 template <int DK, int DVT>
@@ -55,8 +43,8 @@ complex_scan_kernel(cplx::Args a, cplx::Ws w, const int32_t *__restrict__ cu, in
   const int h = blockIdx.x, n = blockIdx.y, tile = blockIdx.z;
   int bos, eos;
   seq_bounds(cu, n, T, T_total, err, bos, eos);
-  DeviceExec x;
-  cplx::scan_program<DeviceExec, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos, bos / CK + n);
+  Exec x;
+  cplx::scan_program<Exec, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos, bos / CK + n);
 }
 
 template <int DK, int DVT>
