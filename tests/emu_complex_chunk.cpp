@@ -81,7 +81,8 @@ void run(const std::string &dir, int N, int T, int H, int DV, float scale, bool 
   };
   HostExec x;
   x.reverse = std::getenv("EMU_REVERSE_ITEMS") != nullptr;
-  std::vector<float> psm(cplx::PrepLayout<DK, DVT>::FLOATS), ssm(cplx::ScanLayout<DK, DVT>::FLOATS);
+  std::vector<float> psm(cplx::PrepLayout<DK, DVT>::FLOATS);
+  std::vector<float> ssm(cplx::ScanLayout<DK, DVT>::FLOATS);
   for (int h = 0; h < H; ++h)
     for (int g = 0; g < (int)slots; ++g) {
       int n, ci, bos, eos;
