@@ -164,3 +164,47 @@ def test_items_of_a_phase_are_independent(emu, tmp_path):
     rev = run_emu(emu, str(tmp_path), inp, grads, 0.9, reverse=True)
     for name, x, y in zip(NAMES, fwd, rev):
         assert np.array_equal(x, y), name
+
+
+@pytest.fixture(scope="module")
+def slot_map(tmp_path_factory):
+    cxx = shutil.which("g++")
+    if cxx is None:
+        pytest.skip("no host C++ compiler")
+    out = str(tmp_path_factory.mktemp("slots") / "emu_slot_map")
+    subprocess.check_call([cxx, "-std=c++17", "-O1", "-I", CSRC,
+                           os.path.join(HERE, "emu_slot_map.cpp"), "-o", out])
+    return out
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_every_slot_finds_its_chunk(slot_map, seed):
+    """slot_chunk, the per-chunk grids' map from checkpoint slot to (sequence,
+    chunk), against an enumeration: every chunk's slot maps back to it, and
+    every other slot is one the kernels skip (no sequence, or past its last
+    chunk), so no chunk runs twice and none is missed."""
+    rng = np.random.default_rng(seed)
+    N = int(rng.integers(1, 9))
+    lens = rng.choice([0, 1, 15, 16, 17, 31, 32, 33, 64, 100], size=N)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(int)
+    cases = [(N, 0, list(cu)), (N, int(lens[0]), None)]  # varlen; N equal sequences
+    for n_seq, T, offsets in cases:
+        if offsets is None:
+            offsets = [i * T for i in range(n_seq + 1)]
+        args = [slot_map, str(n_seq), str(T)] + ([str(c) for c in offsets] if T == 0 else [])
+        out = subprocess.run(args, check=True, capture_output=True, text=True).stdout.split("\n")
+        got = {int(g): (int(n), int(ci), int(ok))
+               for g, n, ci, ok in (line.split() for line in out if line)}
+        want = {}
+        for n in range(n_seq):
+            b, e = offsets[n], offsets[n + 1]
+            for ci in range((e - b + 15) // 16):
+                want[b // 16 + n + ci] = (n, ci)
+        assert len(got) == offsets[-1] // 16 + n_seq
+        assert all(g in got for g in want)  # every chunk's slot is inside the grid
+        for g, (n, ci, ok) in got.items():
+            nck = (offsets[n + 1] - offsets[n] + 15) // 16 if 0 <= n < n_seq else 0
+            runs = bool(ok) and ci < nck
+            assert runs == (g in want), (g, n, ci, ok)
+            if runs:
+                assert (n, ci) == want[g], g
