@@ -13,6 +13,16 @@ collective sits on the data path); value = all ranks' tokens / max time.
 
 --impl reference runs the fp64 CPU oracle on the host cores instead, on a
 bounded sample of the same workload (rank 0 only).
+
+    python bench.py --case prefill|decode|bwd|complex [--T 4096] [--H 32] [--N 64]
+                    [--iters 3] [--chunked]
+
+runs one entry point a few times on one workload and times nothing (a
+command for a profiler to wrap): prefill uses the CKDA long-prefill recipe
+with T tokens per head, decode the decode recipe with N sequences, bwd the
+backward pass on the prefill recipe with seeded upstream gradients, complex
+the complex-phase gate on complex64 inputs of the same shape; --chunked
+selects the chunked entry point of bwd or complex.
 """
 from __future__ import annotations
 
@@ -361,6 +371,49 @@ def run_reference(args):
     return 0
 
 
+def run_case(args):
+    """One entry point, args.iters calls, no timing (see the module doc)."""
+    ckda.load()
+    T, H = args.T, args.H
+    if args.case in ("prefill", "bwd", "complex"):
+        w = WORKLOADS[PREFILL]
+        cu = torch.tensor([0, T], dtype=torch.int32)
+    if args.case == "prefill":
+        inp = make_fwd_inputs(w, cu_seqlens=cu, H=H)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        for _ in range(args.iters):
+            ckda.fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                             d["initial_state"], d["cu_seqlens"], chunk=w.chunk)
+        shape = "T=%d H=%d d=128" % (T, H)
+    elif args.case == "bwd":
+        inp = make_fwd_inputs(w, cu_seqlens=cu, H=H)
+        d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+        g = {k: v.cuda() for k, v in make_bwd_grads(w, T, H, 1).items()}
+        for _ in range(args.iters):
+            ckda.bwd(d["q"], d["k"], d["v"], d["alpha"], d["beta"], g["d_o"],
+                     d["initial_state"], g["d_final_state"], cu_seqlens=d["cu_seqlens"],
+                     chunked=args.chunked)
+        shape = "T=%d H=%d d=128" % (T, H)
+    elif args.case == "complex":
+        c = {k: v.cuda() for k, v in make_complex_inputs(w, cu, H).items()}
+        for _ in range(args.iters):
+            ckda.fwd_complex(c["q"], c["k"], c["v"], c["alpha"], c["theta"], c["beta"],
+                             c["initial_state"], cu_seqlens=c["cu_seqlens"], chunked=args.chunked)
+        shape = "T=%d H=%d d=128 complex64" % (T, H)
+    else:
+        w = WORKLOADS[DECODE]
+        state = make_decode_state(w, N=args.N).cuda()
+        tok = {k: v.cuda() for k, v in make_decode_tokens(w, 0, N=args.N).items()}
+        for _ in range(args.iters):
+            ckda.decode_step(tok["q"], tok["k"], tok["v"], tok["alpha"], tok["beta"], state)
+        shape = "N=%d H=32 d=128" % args.N
+    torch.cuda.synchronize()
+    if ckda.ckda_last_error() != ckda.CKDA_OK:
+        raise RuntimeError("kernel reported an error")
+    print("case %s %s iters=%d ok" % (args.case, shape, args.iters))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,7 +432,17 @@ def main():
     ap.add_argument("--no-chunked-legs", action="store_true",
                     help="skip the extra timing of the chunked backward and complex paths")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["prefill", "decode", "bwd", "complex"], default=None,
+                    help="run one entry point --iters times for a profiler; no timing")
+    ap.add_argument("--T", type=int, default=4096, help="--case: tokens per head")
+    ap.add_argument("--H", type=int, default=32, help="--case: heads")
+    ap.add_argument("--N", type=int, default=64, help="--case decode: sequences")
+    ap.add_argument("--iters", type=int, default=3, help="--case: calls")
+    ap.add_argument("--chunked", action="store_true",
+                    help="--case bwd / complex: the chunked entry point")
     args = ap.parse_args()
+    if args.case:
+        return run_case(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

@@ -137,9 +137,10 @@ size_t ckda_fwd_workspace_bytes(int32_t N, int32_t T, int32_t H, int32_t d_k,
  * process exits. The function allocates nothing.
  *  - Limit: calls whose ckda_fwd_workspace_bytes() exceeds
  *    CKDA_NOALLOC_SCRATCH_BYTES return CKDA_ERR_UNSUPPORTED and launch
- *    nothing (with d_v = 128, 64 MiB holds about 400 (chunk slot, head)
- *    pairs, e.g. 32 heads x 768 tokens). Calls that need no scratch run as in
- *    ckda_fwd_chunked.
+ *    nothing. With d_v = 128 the need is (floor(T_total / 64) + N) * H
+ *    blocks of 164,864 bytes plus a small slot table: one sequence of 767
+ *    tokens with 32 heads (12 x 32 blocks) fits, 768 tokens (13 x 32) do
+ *    not. Calls that need no scratch run as in ckda_fwd_chunked.
  *  - The first call on each device looks up the array's device address (a
  *    cudaGetSymbolAddress on the current device); make that first call before
  *    any stream capture.

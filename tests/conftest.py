@@ -40,3 +40,26 @@ def cuda_lib():
     from gated_delta_rule_114_b200 import ckda
     ckda.load()
     return ckda
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the literal max|x - x_ref| / rms(x_ref) of every parity check the
+    session ran (the largest per test and output; step numbers folded), next
+    to its bound, so a passing run shows its margins."""
+    import re
+    try:
+        from parity_util import RECORDED
+    except ImportError:
+        return
+    if not RECORDED:
+        return
+    worst = {}
+    for test_id, what, ratio, rel, store in RECORDED:
+        key = (test_id, re.sub(r"\d+", "#", what))
+        if key not in worst or ratio > worst[key][0]:
+            worst[key] = (ratio, rel, store)
+    tr = terminalreporter
+    tr.section("parity margins: literal max|x - x_ref| / rms(x_ref)")
+    for (test_id, what), (ratio, rel, store) in worst.items():
+        allow = "%.0e rms" % rel + (" + 2^-8|x_ref|" if store else "")
+        tr.write_line("%-9.3e  (bound %s)  %s  [%s]" % (ratio, allow, test_id, what))

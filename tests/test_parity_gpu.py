@@ -148,25 +148,15 @@ def test_ckda_long_prefill_full(cuda_lib):
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
 
 
-def test_ckda_varlen_full_sampled(cuda_lib):
-    """32 packed sequences, U[128,4096] tokens, H=32 at full size on the GPU;
-    the oracle recomputes a seeded sample of 6 sequences (all heads),
-    including the longest and the shortest."""
+def test_ckda_varlen_full(cuda_lib):
+    """32 packed sequences, U[128,4096] tokens, H=32 at full size: every output
+    row of every sequence and every final state against the oracle."""
     w = WORKLOADS["ckda_varlen_N32_H32_d128"]
     inp = make_fwd_inputs(w)
     o, sf = run_fwd(inp, chunk=w.chunk)
-    cu = inp["cu_seqlens"].numpy()
-    lens = np.diff(cu)
-    rng = np.random.default_rng(4)
-    pick = sorted(set([int(lens.argmax()), int(lens.argmin())] +
-                      list(rng.choice(len(lens), 4, replace=False))))
-    sub_rows = np.concatenate([np.arange(cu[n], cu[n + 1]) for n in pick])
-    sub = {key: inp[key][sub_rows] for key in ("q", "k", "v", "alpha", "beta")}
-    sub["initial_state"] = inp["initial_state"][pick]
-    sub["cu_seqlens"] = lens_cu(lens[pick])
-    o_ref, sf_ref = ref_fwd(sub)
-    check_bf16_out(o.cpu()[torch.from_numpy(sub_rows)], o_ref)
-    check_close(sf.cpu()[pick], sf_ref, 1e-2, 0.0, "final_state")
+    o_ref, sf_ref = ref_fwd(inp)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
 
 
 def test_bf16_ragged_small(cuda_lib):
