@@ -506,7 +506,13 @@ def main():
                            "frac": flops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
                            "useful_flops_per_launch": flops}}
 
-    # ---------------- end to end through the C ABI with host buffers
+    # ---------------- end to end through the C ABI with host buffers. Every
+    # step copies its inputs from pinned host memory, runs the forward and
+    # copies o and the final state back. Copies in, compute and copies out sit
+    # on three streams with two device buffer sets, so step i + 1's inputs
+    # cross the link while step i computes and step i - 1's outputs return
+    # (the link's two directions and the GPU work overlap, as in a serving
+    # loop); the timed region is every step's copies and compute.
     pinned = {key: (val.pin_memory() if isinstance(val, torch.Tensor) else val)
               for key, val in inp_cpu.items()}
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -514,19 +520,72 @@ def main():
     h2d = sum(v.numel() * v.element_size() for k_, v in pinned.items()
               if isinstance(v, torch.Tensor))
     d2h = o_host.numel() * o_host.element_size() + sf_host.numel() * 4
+    sets = [dev, {key: (torch.empty_like(val) if isinstance(val, torch.Tensor) else val)
+                  for key, val in dev.items()}]
+    outs = [(o, sf), (torch.empty_like(o), torch.empty_like(sf))]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_back = [torch.cuda.Event() for _ in range(2)]
+    e2e_state = {"i": 0}
 
     def e2e_step():
-        for key, val in pinned.items():
-            if isinstance(val, torch.Tensor):
-                dev[key].copy_(val, non_blocking=True)
-        prefill()
-        o_host.copy_(o, non_blocking=True)
-        sf_host.copy_(sf, non_blocking=True)
+        b = e2e_state["i"] & 1
+        e2e_state["i"] += 1
+        d, (ob, sfb) = sets[b], outs[b]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_done[b])       # step i - 2 has read these inputs
+            for key, val in pinned.items():
+                if isinstance(val, torch.Tensor):
+                    d[key].copy_(val, non_blocking=True)
+            ev_in[b].record(s_in)
+        stream.wait_event(ev_in[b])
+        stream.wait_event(ev_back[b])         # step i - 2's outputs are home
+        ckda.ckda_fwd_chunked(d["q"], d["k"], d["v"], d["alpha"], d["beta"],
+                              d["initial_state"], sfb, ob, d["cu_seqlens"], None,
+                              chunk=w.chunk, stream=stream, workspace=ws)
+        ev_done[b].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[b])
+            o_host.copy_(ob, non_blocking=True)
+            sf_host.copy_(sfb, non_blocking=True)
+            ev_back[b].record(s_out)
 
-    e2e_ms = time_loop(e2e_step, args.e2e_steps, 3, stream, barrier)
+    def e2e_loop(steps):
+        for _ in range(steps):
+            e2e_step()
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+
+    for ev in ev_done + ev_back:
+        ev.record(stream)
+    e2e_loop(3)
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    torch.cuda.synchronize()
+    st_ev, en_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st_ev.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
+    e2e_loop(args.e2e_steps)
+    en_ev.record(stream)
+    en_ev.synchronize()
+    torch.cuda.synchronize()
+    if barrier:
+        barrier()
+    if ckda.ckda_last_error() != ckda.CKDA_OK:
+        raise RuntimeError("kernel reported an error")
+    e2e_ms = st_ev.elapsed_time(en_ev) / args.e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
     e2e = {"value": T_total * world / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": e2e_ms}
+           "ms_per_step": e2e_ms,
+           "pipeline": "copies in, forward and copies out on three streams, two buffer sets"}
+    del sets[1], outs[1]
 
     # ---------------- the same workload through the fused input prologue
     ginp = make_gated_fwd_inputs(w)
