@@ -53,6 +53,7 @@
 #endif
 #endif
 
+
 namespace ckda {
 namespace bwdc {
 

@@ -126,17 +126,22 @@ CKDA_PROG void prep_program(X &x, const Args<IOT> &a, const SplitWs &w, float *s
 }
 
 // Shared memory of the two scans: one state (or state gradient) tile and the
-// chunk's per-token factors.
+// chunks' per-token factors.
 template <int DK, int DVT>
 struct ScanLayout {
   static constexpr int KS = DK + 1, VS = DVT + 1;
-  // two sets of a chunk's factors (chunk i in set i & 1, so that the next
-  // chunk's loads overlap this chunk's products): three C x DK, two C x DVT
-  // and gamma_C; offsets within a set
+  // three sets of a chunk's factors: the k-th chunk a scan visits sits in set
+  // k % 3, its copies started two chunks ahead (asynchronous copies, waited
+  // for at the chunk's start), so their latency overlaps two chunks' work.
+  // Per set: three C x DK, two C x DVT, gamma_C, and the raw I/O-type pairs of
+  // a C x DVT tile (dO in bf16, converted in place once it has landed);
+  // offsets within a set
   static constexpr int F0 = 0, F1 = F0 + C * KS, F2 = F1 + C * KS, R0 = F2 + C * KS,
-                       R1 = R0 + C * VS, GC = R1 + C * VS, SET = GC + DK;
+                       R1 = R0 + C * VS, GC = R1 + C * VS, RAW = GC + DK,
+                       SET = RAW + C * DVT / 2;
+  static constexpr int NSETS = 3;
   static constexpr int S = 0, SETS = S + DK * VS;
-  static constexpr int P = SETS + 2 * SET;  // partial products, C x DVT x 4
+  static constexpr int P = SETS + NSETS * SET;  // partial products, C x DVT x 4
   static constexpr int FLOATS = P + 4 * C * DVT;
   static constexpr size_t BYTES = (size_t)FLOATS * sizeof(float);
 };
@@ -240,45 +245,59 @@ CKDA_PROG void scan1_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
   float *S = sm + Ly::S;
-  // item e of loading chunk ci's W, Kbar, Utilde (rows past its end zero) and
-  // gamma_C into set ci & 1
+  // item e of starting the copies of chunk ci's W, Kbar, Utilde and gamma_C
+  // into set ci % 3 (rows past its end are written as zero at once)
   auto load = [&](int e, int ci) {
-    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    if (ci >= nck) return;
+    float *f = sm + Ly::SETS + (ci % Ly::NSETS) * Ly::SET;
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     if (e < C * DK) {
       const int i = e / DK, c = e - i * DK;
       const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
-      f[Ly::F0 + i * KS + c] = i < L ? CKDA_LDG(w.wt + o) : 0.f;
-      f[Ly::F1 + i * KS + c] = i < L ? CKDA_LDG(w.kb + o) : 0.f;
+      if (i < L) {
+        x.acopy4(f + Ly::F0 + i * KS + c, w.wt + o);
+        x.acopy4(f + Ly::F1 + i * KS + c, w.kb + o);
+      } else {
+        f[Ly::F0 + i * KS + c] = 0.f;
+        f[Ly::F1 + i * KS + c] = 0.f;
+      }
     }
     if (e < C * DVT) {
       const int i = e / DVT, v = e - i * DVT;
-      f[Ly::R0 + i * VS + v] =
-          i < L ? CKDA_LDG(w.ut + ((size_t)(t0 + i) * H + h) * DVF + c0 + v) : 0.f;
+      if (i < L)
+        x.acopy4(f + Ly::R0 + i * VS + v, w.ut + ((size_t)(t0 + i) * H + h) * DVF + c0 + v);
+      else
+        f[Ly::R0 + i * VS + v] = 0.f;
     }
-    if (e < DK) f[Ly::GC + e] = CKDA_LDG(w.gc + ((size_t)(slot0 + ci) * H + h) * DK + e);
+    if (e < DK) x.acopy4(f + Ly::GC + e, w.gc + ((size_t)(slot0 + ci) * H + h) * DK + e);
   };
-  par<NL>(x, [&](int e) {  // the initial state; chunk 0's factors
+  par<NL>(x, [&](int e) {  // the initial state; chunks 0 and 1 start coming in
     if (e < DK * DVT) {
       const int c = e / DVT, v = e - c * DVT;
       S[c * VS + v] = a.s0 ? a.s0[st_base + (size_t)c * DVF + v] : 0.f;
     }
-    if (nck > 0) load(e, 0);
+    load(e, 0);
+    load(e, 1);
   });
+  x.commit();
   for (int ci = 0; ci < nck; ++ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t slot = (size_t)(slot0 + ci) * H + h;
-    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    float *f = sm + Ly::SETS + (ci % Ly::NSETS) * Ly::SET;
     float *WT = f + Ly::F0, *KB = f + Ly::F1, *U = f + Ly::R0, *GC = f + Ly::GC;
-    // checkpoint S; the partial products of W S; chunk ci + 1's factors
+    // chunk ci has landed (only chunk ci + 1's group may still be in flight)
+    if (ci == 0) x.template wait_copies<0>();
+    else x.template wait_copies<1>();
+    // checkpoint S; the partial products of W S; chunk ci + 2's copies start
     par<NL>(x, [&](int e) {
       if (e < DK * DVT) {
         const int c = e / DVT, v = e - c * DVT;
         w.cks[slot * DK * DVF + (size_t)c * DVF + c0 + v] = S[c * VS + v];
       }
       if (e < NP) rows_state_partial_item<DK, DVT>(e, sm + Ly::P, WT, S);
-      if (ci + 1 < nck) load(e, ci + 1);
+      load(e, ci + 2);
     });
+    x.commit();
     par<C * DVT>(x, [&](int e) {  // U = Utilde - W S
       const int i = e / DVT, v = e - i * DVT;
       const float s = U[i * VS + v] - rows_state_sum<DVT>(sm + Ly::P, i, v);
@@ -296,57 +315,90 @@ CKDA_PROG void scan2_program(X &x, const Args<IOT> &a, const SplitWs &w, float *
   using Ly = ScanLayout<DK, DVT>;
   constexpr int KS = Ly::KS, VS = Ly::VS, NP = PartialItems<DVT>::value;
   constexpr int NL = DK * DVT > C * DK ? DK * DVT : C * DK;  // items of a load phase
+  constexpr bool RAW_DO = sizeof(IOT) != sizeof(float);  // dO arrives as bf16 pairs
   const int c0 = tile * DVT, H = a.H, DVF = a.DVF;
   const int nck = (eos - bos + C - 1) / C;
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;
   float *DS = sm + Ly::S;
-  // item e of loading chunk ci's Wb, Qs, BK, X, dO (rows past its end zero)
-  // and gamma_C into set ci & 1
-  auto load = [&](int e, int ci) {
-    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+  // item e of starting the copies of the k-th chunk from the end (chunk
+  // nck - 1 - k): Wb, Qs, BK, X, dO and gamma_C into set k % 3 (rows past its
+  // end are written as zero at once)
+  auto load = [&](int e, int k) {
+    if (k >= nck) return;
+    const int ci = nck - 1 - k;
+    float *f = sm + Ly::SETS + (k % Ly::NSETS) * Ly::SET;
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     if (e < C * DK) {
       const int i = e / DK, c = e - i * DK;
       const size_t o = ((size_t)(t0 + i) * H + h) * DK + c;
-      f[Ly::F0 + i * KS + c] = i < L ? CKDA_LDG(w.wb + o) : 0.f;
-      f[Ly::F1 + i * KS + c] = i < L ? CKDA_LDG(w.qs + o) : 0.f;
-      f[Ly::F2 + i * KS + c] = i < L ? CKDA_LDG(w.bk + o) : 0.f;
+      if (i < L) {
+        x.acopy4(f + Ly::F0 + i * KS + c, w.wb + o);
+        x.acopy4(f + Ly::F1 + i * KS + c, w.qs + o);
+        x.acopy4(f + Ly::F2 + i * KS + c, w.bk + o);
+      } else {
+        f[Ly::F0 + i * KS + c] = 0.f;
+        f[Ly::F1 + i * KS + c] = 0.f;
+        f[Ly::F2 + i * KS + c] = 0.f;
+      }
     }
     if (e < C * DVT) {
       const int i = e / DVT, v = e - i * DVT;
       const size_t o = ((size_t)(t0 + i) * H + h) * DVF + c0 + v;
-      f[Ly::R0 + i * VS + v] = i < L ? CKDA_LDG(w.xt + o) : 0.f;
-      f[Ly::R1 + i * VS + v] = i < L ? IOL::ldg(a.d_o + o) : 0.f;
+      if (i < L) {
+        x.acopy4(f + Ly::R0 + i * VS + v, w.xt + o);
+        if constexpr (RAW_DO) {  // a pair of bf16 per 4-byte copy
+          if ((v & 1) == 0)
+            x.acopy4(f + Ly::RAW + i * (DVT / 2) + v / 2, reinterpret_cast<const float *>(a.d_o + o));
+        } else {
+          x.acopy4(f + Ly::R1 + i * VS + v, reinterpret_cast<const float *>(a.d_o + o));
+        }
+      } else {
+        f[Ly::R0 + i * VS + v] = 0.f;
+        f[Ly::R1 + i * VS + v] = 0.f;
+        if constexpr (RAW_DO) if ((v & 1) == 0) f[Ly::RAW + i * (DVT / 2) + v / 2] = 0.f;
+      }
     }
-    if (e < DK) f[Ly::GC + e] = CKDA_LDG(w.gc + ((size_t)(slot0 + ci) * H + h) * DK + e);
+    if (e < DK) x.acopy4(f + Ly::GC + e, w.gc + ((size_t)(slot0 + ci) * H + h) * DK + e);
   };
-  par<NL>(x, [&](int e) {  // the final-state gradient; the last chunk's factors
+  par<NL>(x, [&](int e) {  // the final-state gradient; the last two chunks start coming in
     if (e < DK * DVT) {
       const int c = e / DVT, v = e - c * DVT;
       DS[c * VS + v] = a.dsf ? a.dsf[st_base + (size_t)c * DVF + v] : 0.f;
     }
-    if (nck > 0) load(e, nck - 1);
+    load(e, 0);
+    load(e, 1);
   });
-  for (int ci = nck - 1; ci >= 0; --ci) {
+  x.commit();
+  for (int k = 0; k < nck; ++k) {
+    const int ci = nck - 1 - k;
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     const size_t slot = (size_t)(slot0 + ci) * H + h;
-    float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
+    float *f = sm + Ly::SETS + (k % Ly::NSETS) * Ly::SET;
     float *WB = f + Ly::F0, *QS = f + Ly::F1, *BK = f + Ly::F2, *DR = f + Ly::R0,
           *DO = f + Ly::R1, *GC = f + Ly::GC;
-    // checkpoint dS_C; the partial products of Wb dS_C; chunk ci - 1's factors
+    // this chunk has landed (only the next one's group may still be in flight)
+    if (k == 0) x.template wait_copies<0>();
+    else x.template wait_copies<1>();
+    // checkpoint dS_C; the partial products of Wb dS_C; the copies of the
+    // chunk two ahead start
     par<NL>(x, [&](int e) {
       if (e < DK * DVT) {
         const int c = e / DVT, v = e - c * DVT;
         w.ckd[slot * DK * DVF + (size_t)c * DVF + c0 + v] = DS[c * VS + v];
       }
       if (e < NP) rows_state_partial_item<DK, DVT>(e, sm + Ly::P, WB, DS);
-      if (ci > 0) load(e, ci - 1);
+      load(e, k + 2);
     });
-    par<C * DVT>(x, [&](int e) {  // dR = X + Wb dS_C
+    x.commit();
+    par<C * DVT>(x, [&](int e) {  // dR = X + Wb dS_C; dO to fp32 (bf16 pairs)
       const int j = e / DVT, v = e - j * DVT;
       const float s = DR[j * VS + v] + rows_state_sum<DVT>(sm + Ly::P, j, v);
       DR[j * VS + v] = s;
       if (j < L) w.dr[((size_t)(t0 + j) * H + h) * DVF + c0 + v] = s;
+      if constexpr (RAW_DO) {
+        const float pair = f[Ly::RAW + j * (DVT / 2) + v / 2];
+        DO[j * VS + v] = IOL::pair_half(pair, v & 1);
+      }
     });
     // dS <- diag(gamma_C) dS_C + Qs^T dO - BK^T dR
     state_update<DK, DVT>(x, DS, GC, QS, DO, BK, DR);

@@ -71,6 +71,11 @@ template <> struct IO<__nv_bfloat16> {
   static __device__ __forceinline__ void st(__nv_bfloat16 *p, float x) {
     *p = __float2bfloat16_rn(x);
   }
+  // element `hi` (0 or 1) of a bf16 pair held in the 4 bytes of `pair`
+  static __device__ __forceinline__ float pair_half(float pair, int hi) {
+    const uint32_t b = __float_as_uint(pair);
+    return __uint_as_float(hi ? (b & 0xffff0000u) : (b << 16));
+  }
   // 4 consecutive elements (8-byte aligned)
   static __device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
     uint2 raw = *reinterpret_cast<const uint2 *>(p);

@@ -204,8 +204,9 @@ CKDA_UNROLL
 template <int DK, int DVT>
 struct ScanLayout {
   static constexpr int KS = 2 * (DK + 1), VS = 2 * (DVT + 1), CS = 2 * (C + 1);
-  // two sets of a chunk's factors (chunk i in set i & 1, so that the next
-  // chunk's loads overlap this chunk's products): C x DK complex W, Kbar, Qhat;
+  // two sets of a chunk's factors (chunk i in set i & 1; chunk i + 1's
+  // asynchronous copies land while chunk i is worked on, and are waited for
+  // at chunk i + 1's start): C x DK complex W, Kbar, Qhat;
   // C x DVT complex Utilde (then U); C x C complex M; gamma_{C-1} [DK]
   // complex; offsets within a set
   static constexpr int WT = 0, KB = WT + C * KS, QH = KB + C * KS, UT = QH + C * KS,
@@ -229,7 +230,13 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
   const size_t st_base = ((size_t)n * H + h) * DK * DVF + c0;  // complex elements
   float *S = sm + Ly::S;
   const cf zero{0.f, 0.f};
-  // item e of loading chunk ci's factors (rows past its end zero) into set ci & 1
+  // one complex element (two floats) copied in the background
+  auto acopy = [&](float *dst, const float *src) {
+    x.acopy4(dst, src);
+    x.acopy4(dst + 1, src + 1);
+  };
+  // item e of starting the copies of chunk ci's factors into set ci & 1
+  // (rows past its end are written as zero at once)
   auto load = [&](int e, int ci) {
     float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
@@ -237,18 +244,25 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
     if (e < C * DK) {
       const int i = e / DK, c = e - i * DK;
       const size_t o = (((size_t)(t0 + i) * H + h) * DK + c) * 2;
-      const bool in = i < L;
-      cst(f + Ly::WT + i * KS + 2 * c, in ? cldg(w.wt + o) : zero);
-      cst(f + Ly::KB + i * KS + 2 * c, in ? cldg(w.kb + o) : zero);
-      cst(f + Ly::QH + i * KS + 2 * c, in ? cldg(w.qh + o) : zero);
+      if (i < L) {
+        acopy(f + Ly::WT + i * KS + 2 * c, w.wt + o);
+        acopy(f + Ly::KB + i * KS + 2 * c, w.kb + o);
+        acopy(f + Ly::QH + i * KS + 2 * c, w.qh + o);
+      } else {
+        cst(f + Ly::WT + i * KS + 2 * c, zero);
+        cst(f + Ly::KB + i * KS + 2 * c, zero);
+        cst(f + Ly::QH + i * KS + 2 * c, zero);
+      }
     }
     if (e < C * DVT) {
       const int i = e / DVT, v = e - i * DVT;
-      cst(f + Ly::UT + i * VS + 2 * v,
-          i < L ? cldg(w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2) : zero);
+      if (i < L)
+        acopy(f + Ly::UT + i * VS + 2 * v, w.ut + (((size_t)(t0 + i) * H + h) * DVF + c0 + v) * 2);
+      else
+        cst(f + Ly::UT + i * VS + 2 * v, zero);
     }
-    if (e < C * C) cst(f + Ly::M + (e / C) * CS + 2 * (e % C), cldg(w.mm + (sl * C * C + e) * 2));
-    if (e < DK) cst(f + Ly::GC + 2 * e, cldg(w.gc + (sl * DK + e) * 2));
+    if (e < C * C) acopy(f + Ly::M + (e / C) * CS + 2 * (e % C), w.mm + (sl * C * C + e) * 2);
+    if (e < DK) acopy(f + Ly::GC + 2 * e, w.gc + (sl * DK + e) * 2);
   };
   par<NL>(x, [&](int e) {  // the initial state; chunk 0's factors
     if (e < DK * DVT) {
@@ -259,10 +273,12 @@ CKDA_PROG void scan_program(X &x, const Args &a, const Ws &w, float *sm, int h, 
     }
     if (nck > 0) load(e, 0);
   });
+  x.commit();
   for (int ci = 0; ci < nck; ++ci) {
     const int t0 = bos + C * ci, L = eos - t0 < C ? eos - t0 : C;
     float *f = sm + Ly::SETS + (ci & 1) * Ly::SET;
     float *U = f + Ly::UT;
+    x.template wait_copies<0>();  // chunk ci has landed
     // W S and Qhat S in one pass over S: item (row pair, 4 columns, quarter q)
     // sums channels q, q + 4, ... in 2 x 4 complex register tiles; chunk
     // ci + 1's factors load meanwhile
@@ -299,6 +315,7 @@ CKDA_UNROLL
       }
       if (ci + 1 < nck) load(e, ci + 1);
     });
+    x.commit();
     // the four quarters of (row i, column v) in a fixed order
     auto quarters = [&](int base, int i, int v) {
       const int e0 = (((i / 2) * NV + v / 4) * 4) * 2 + (i % 2), j = v % 4;

@@ -11,7 +11,9 @@
 // raw .bin files; writes dq dk dv dalpha dbeta ds0 (.bin, float32) there.
 #include <cstdio>
 #include <cstdlib>
+#include <deque>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "ckda_bwd_split.cuh"
@@ -27,6 +29,23 @@ struct HostExec {
   template <int N, class F>
   void run(F f) {
     for (int i = 0; i < N; ++i) f(reverse ? N - 1 - i : i);
+  }
+  // Asynchronous copies as the GPU may see them: each lands only when a
+  // wait_copies that covers its group runs, so a program that reads a copy's
+  // destination before waiting for it reads the old contents here too.
+  std::vector<std::pair<float *, const float *>> open_group;
+  std::deque<std::vector<std::pair<float *, const float *>>> groups;
+  void acopy4(float *dst, const float *src) { open_group.emplace_back(dst, src); }
+  void commit() {
+    groups.push_back(std::move(open_group));
+    open_group.clear();
+  }
+  template <int pending>
+  void wait_copies() {
+    while (groups.size() > (size_t)pending) {
+      for (auto &c : groups.front()) *c.first = *c.second;
+      groups.pop_front();
+    }
   }
 };
 
