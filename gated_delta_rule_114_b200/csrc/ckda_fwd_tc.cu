@@ -53,7 +53,7 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64, DK = 128, DVT = 32;
-constexpr int PF_STEP = 128;  // bytes per L2 prefetch of the next item's rows
+constexpr int PF_STEP = 128;  // bytes per L2 prefetch of the next item's gate logits
 constexpr int AL_S = 132;  // fp32 row stride of alpha / Qhat
 
 // Float offset of (row i, channel c) in the alpha / Qhat buffer: the 16-byte
@@ -241,6 +241,46 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
+  // An item's q, k, v rows, beta (or its logits) and, without the fused
+  // prologue, alpha arrive by per-thread asynchronous copies (cp.async) into
+  // their shared buffers, issued during the previous item once each buffer's
+  // last reader is done: q, k, v while D5 runs (after [M ; I] x T, their last
+  // reader), alpha and beta after the epilogue has read Qhat. Rows past the
+  // chunk's end read as zero (alpha: 1). An item whose copies were not issued
+  // ahead (the first, or one after empty slots) issues them at its start.
+  const int nvp = DV / 8, lnv = __ffs(nvp) - 1;  // 16-byte pieces of a v row (a power of 2)
+  auto issue_qkv = [&](int t0r, int Lr, int hr) {
+    for (int idx = tid; idx < 2 * C * 16; idx += NTP) {  // q, k: 64 rows x 16 pieces
+      const int kt = idx >> 10, i = (idx >> 4) & (C - 1), w = idx & 15;
+      const uint32_t nb = i < Lr ? 16u : 0u;  // 0: zero fill, nothing read
+      const size_t off = ((size_t)(t0r + (i < Lr ? i : 0)) * H + hr) * DK + w * 8;
+      cp_async16(sm + (kt ? P_K : P_Q) + i * 256 + w * 16, (kt ? k : q) + off, nb);
+    }
+    for (int idx = tid; idx < C * nvp; idx += NTP) {  // v: 64 rows x DV / 8 pieces
+      const int i = idx >> lnv, w = idx & (nvp - 1);
+      const uint32_t nb = i < Lr ? 16u : 0u;
+      const size_t off = ((size_t)(t0r + (i < Lr ? i : 0)) * H + hr) * DV + w * 8;
+      cp_async16(sm + P_V + i * DV * 2 + w * 16, v + off, nb);
+    }
+    cp_async_commit();
+  };
+  auto issue_gates = [&](int t0r, int Lr, int hr) {  // alpha (no fused prologue), beta
+    if constexpr (!GATED) {
+      for (int idx = tid; idx < C * 32; idx += NTP) {  // 64 rows x 32 pieces of 4 floats
+        const int i = idx >> 5, c4 = (idx & 31) * 4;
+        float *dst = sAl + al_off(i, c4);
+        if (i < Lr) cp_async16(dst, alpha + ((size_t)(t0r + i) * H + hr) * DK + c4, 16u);
+        else *reinterpret_cast<float4 *>(dst) = make_float4(1.f, 1.f, 1.f, 1.f);
+      }
+    }
+    if (tid < C) {
+      if (tid < Lr) cp_async4(sB + tid, beta + (size_t)(t0r + tid) * H + hr);
+      else sB[tid] = 0.f;
+    }
+    cp_async_commit();
+  };
+  int raw_for = -1;  // item whose row copies were issued ahead (CTA-uniform)
+
   // Persistent: items (slot, head) = it / H, it % H, strided by the grid.
   // Each mbarrier completes once per non-empty item: parity `ph`.
   uint32_t ph = 0;
@@ -259,25 +299,17 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   uint8_t *wsb = ws + ((size_t)slot * H + h) * ws_block_bytes(DV);
 
   do {  // one pass; `break` leaves on a timed-out wait
-    // ---------------- 1. load the chunk: all global loads in flight at once
+    // ---------------- 1. load the chunk: q, k, v, beta and (without the fused
+    // prologue) alpha have been copied in asynchronously; the gate logits of
+    // the fused prologue come through registers
+    if (raw_for != it) {
+      issue_qkv(t0, L, h);
+      issue_gates(t0, L, h);
+    }
+    raw_for = -1;
     {
-      uint4 qv[2], kv[2];
-      float4 av[4];
-      (void)av;
-      uint4 vr[2];
-      float bv = 0.f;
-      const int nv = DV / 8;  // 16-byte pieces of a v row
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {  // q, k: 64 rows x 16 pieces of 16 bytes
-        const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
-        qv[u] = kv[u] = make_uint4(0, 0, 0, 0);
-        if (i < L) {
-          const size_t off = ((size_t)(t0 + i) * H + h) * DK + ch * 8;
-          qv[u] = __ldg(reinterpret_cast<const uint4 *>(q + off));
-          kv[u] = __ldg(reinterpret_cast<const uint4 *>(k + off));
-        }
-      }
       uint4 al[2];  // GATED: 64 rows x 16 pieces of 8 bf16 logits
+      (void)al;
       if constexpr (GATED) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
@@ -286,35 +318,10 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           if (i < L)
             al[u] = __ldg(reinterpret_cast<const uint4 *>(alogit + ((size_t)(t0 + i) * H + h) * DK + ch * 8));
         }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {  // alpha: 64 rows x 32 float4
-          const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
-          av[u] = make_float4(1.f, 1.f, 1.f, 1.f);
-          if (i < L)
-            av[u] = __ldg(reinterpret_cast<const float4 *>(alpha + ((size_t)(t0 + i) * H + h) * DK + c4));
-        }
       }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {  // v: 64 rows x DV/8 pieces of 16 bytes
-        const int idx = tid + u * NTP, i = idx / nv, p8 = idx % nv;
-        vr[u] = make_uint4(0, 0, 0, 0);
-        if (idx < C * nv && i < L)
-          vr[u] = __ldg(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + i) * H + h) * DV + 8 * p8));
-      }
-      if (tid < L) {
-        bv = __ldg(beta + (size_t)(t0 + tid) * H + h);
-        if constexpr (GATED) bv = gate_beta(ga, bv);
-      }
-      // (the previous item's bulk stores may still read its staging, which
-      // lies outside every buffer written here)
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
-        *reinterpret_cast<uint4 *>(sm + P_Q + i * 256 + ch * 16) = qv[u];
-        *reinterpret_cast<uint4 *>(sm + P_K + i * 256 + ch * 16) = kv[u];
-      }
+      cp_async_wait_all();
       if constexpr (GATED) {
+        __syncthreads();  // every thread's k rows have landed
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
@@ -331,7 +338,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           *reinterpret_cast<float4 *>(sAl + al_off(i, 8 * ch)) = make_float4(x[0], x[1], x[2], x[3]);
           *reinterpret_cast<float4 *>(sAl + al_off(i, 8 * ch + 4)) = make_float4(x[4], x[5], x[6], x[7]);
           // key row inverse norm: 16 lanes hold row i's 128 channels
-          const uint32_t kw[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+          const uint4 kq = *reinterpret_cast<const uint4 *>(sm + P_K + i * 256 + ch * 16);
+          const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w};
           float ss = 0.f;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -342,45 +350,25 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           for (int m = 8; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
           if (ch == 0) sRN[i] = (i < L) ? key_rnorm(ga, ss) : 0.f;
         }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int idx = tid + u * NTP, i = idx >> 5, c4 = (idx & 31) * 4;
-          *reinterpret_cast<float4 *>(sAl + al_off(i, c4)) = av[u];
-        }
+        if (tid < L) sB[tid] = gate_beta(ga, sB[tid]);  // beta from its logit
       }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int idx = tid + u * NTP;
-        if (idx < C * nv) *reinterpret_cast<uint4 *>(sm + P_V + idx * 16) = vr[u];
-      }
-      if (tid < C) sB[tid] = bv;
       // the gate pass writes over the staging: the stores must have read it
       if (tid == 0) bulk_wait_read0();
     }
     __syncthreads();
 
-    // the next item's rows into L2 (one PF_STEP-byte piece per thread and
-    // step; plain prefetches, which leave the bulk-copy unit to the workspace
-    // stores), while this item is computed. Every address lies inside its
-    // row: q, k bf16, the gate input (fp32 alpha or bf16 logits), v bf16.
-    if (nxt.y > 0) {
-      const int nh = nit % H;
-      constexpr int AW = GATED ? 2 : 4;  // bytes per gate element
-      constexpr int lq = DK * 2 / PF_STEP, la = DK * AW / PF_STEP;
-      const int lv = (DV * 2 + PF_STEP - 1) / PF_STEP;
-      const int per = 2 * lq + la + lv;  // pieces per token row
-      const char *gate_in = reinterpret_cast<const char *>(alpha_in);
-      for (int t = tid; t < nxt.y * per; t += NTP) {
-        const int r = t / per, w = t % per;
-        const size_t tok = (size_t)(nxt.x + r) * H + nh;
-        const char *p;
-        if (w < lq) p = reinterpret_cast<const char *>(q + tok * DK) + PF_STEP * w;
-        else if (w < 2 * lq) p = reinterpret_cast<const char *>(k + tok * DK) + PF_STEP * (w - lq);
-        else if (w < 2 * lq + la) p = gate_in + tok * DK * AW + PF_STEP * (w - 2 * lq);
-        else p = reinterpret_cast<const char *>(v + tok * DV) + PF_STEP * (w - 2 * lq - la);
-        prefetch_line_l2(p);
-        if (w == 0) prefetch_line_l2(beta + tok);
+    // the next item's gate logits (fused prologue) into L2 (plain line
+    // prefetches) while this item is computed; every address lies inside its
+    // row
+    if constexpr (GATED) {
+      if (nxt.y > 0) {
+        const int nh = nit % H;
+        constexpr int la = DK * 2 / PF_STEP;  // pieces of a logit row
+        const char *gate_in = reinterpret_cast<const char *>(alpha_in);
+        for (int t = tid; t < nxt.y * la; t += NTP) {
+          const int r = t / la, w = t % la;
+          prefetch_line_l2(gate_in + ((size_t)(nxt.x + r) * H + nh) * DK * 2 + PF_STEP * w);
+        }
       }
     }
 
@@ -945,6 +933,12 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
                     desc_k_sw128_f32(sb + P_GA, DK + DV, kk), id5, kk > 0);
       mma_commit(&bar[2]);
     }
+    // while D5 runs: the q, k, v buffers' last reader ([M ; I] x T) is done,
+    // so the next item's rows may come in
+    if (nxt.y > 0) {
+      issue_qkv(nxt.x, nxt.y, nit % H);
+      raw_for = nit;
+    }
     if (!wait_all(&bar[2], ph, s_abort)) break;
     {
       const int qw = warp & 3, cg = warp >> 2, row = 32 * qw + lane;
@@ -981,12 +975,15 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
       bulk_s2g(wsb + WS_OU + 64u * DV * 4u, sm + P_A, 64u * DV * 4u);
       bulk_commit();
     }
+    // Qhat and beta have been read: the next item's gates may come in
+    if (nxt.y > 0) issue_gates(nxt.x, nxt.y, nit % H);
   } while (0);
   if (*s_abort) break;  // CTA-uniform: read after a barrier
   ph ^= 1u;
   cur = nxt;
   }  // item loop
 
+  cp_async_wait_all();  // copies issued ahead land before shared memory is released
   if (tid == 0) {
     if (*s_abort) flag_error(err, kErrMbarTimeout);
     bulk_wait_read0();  // shared memory stays valid until the stores read it
