@@ -77,12 +77,15 @@ def esize(dt):
 # capture, its command and the scaling are in profiles/. Set to None whenever
 # a kernel changes after its capture.
 NCU_TRAFFIC = {
-    # prep + scan at T=2048, H=32 (1024 chunk-heads): 375.9 MB, x4 for T=8192
-    "prefill": 4 * 375.9e6,
+    # prep + scan at T=2048, H=32 (1024 chunk-heads): 374.6 MB, x4 for T=8192
+    "prefill": 4 * 374.6e6,
     # N=64 (2048 pairs): 214.8 MB, x4 for N=256
     "decode": 4 * 214.8e6,
-    # backward (both kernels) at T=512, H=32: 356.3 MB, x16 for T=8192
+    # token-serial backward (both kernels) at T=512, H=32: 356.3 MB, x16 for T=8192
     "backward": 16 * 356.3e6,
+    # chunked backward (prep, two scans, gradients) at T=2048, H=32: 1944.9 MB,
+    # x4 for T=8192
+    "backward_chunked": 4 * 1944.9e6,
 }
 
 
@@ -422,10 +425,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-steps", type=int, default=200)
     ap.add_argument("--bwd-steps", type=int, default=5)
-    ap.add_argument("--bwd-impl", default="serial", choices=["serial", "chunked"],
+    ap.add_argument("--bwd-impl", default="chunked", choices=["serial", "chunked"],
                     help="backward entry point: ckda_bwd (token-serial) or ckda_bwd_chunked")
     ap.add_argument("--complex-steps", type=int, default=5)
-    ap.add_argument("--complex-impl", default="serial", choices=["serial", "chunked"],
+    ap.add_argument("--complex-impl", default="chunked", choices=["serial", "chunked"],
                     help="complex-gate entry point: ckda_fwd_complex (token-serial) or "
                          "ckda_fwd_complex_chunked")
     ap.add_argument("--e2e-steps", type=int, default=10)
@@ -501,9 +504,13 @@ def main():
                 "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                 "traffic": NCU_TRAFFIC["prefill"], "peak_source": pk["source"],
                 "algorithmic_bytes_per_launch": nbytes,
+                # every tensor-core product is tf32: its peak is the measured bf16
+                # peak times the nominal tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s)
                 "tensor": {"achieved_tflops": flops / (ms / 1e3) / 1e12,
-                           "peak_tflops": pk["bf16_tflops"],
-                           "frac": flops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
+                           "peak_tflops": pk["bf16_tflops"] * 1.1 / 2.25,
+                           "peak_source": "measured bf16 x 1.1/2.25 (tf32 operands)",
+                           "frac": flops / (ms / 1e3) / 1e12 / (pk["bf16_tflops"] * 1.1 / 2.25),
+                           "frac_of_bf16_peak": flops / (ms / 1e3) / 1e12 / pk["bf16_tflops"],
                            "useful_flops_per_launch": flops}}
 
     # ---------------- end to end through the C ABI with host buffers. Every
@@ -634,15 +641,14 @@ def main():
                 "roofline": {"bound": "hbm", "achieved": bbytes / (bms / 1e3) / 1e9,
                              "peak": pk["hbm_gbs"], "unit": "GB/s",
                              "frac": bbytes / (bms / 1e3) / 1e9 / pk["hbm_gbs"],
-                             # counters were taken on the token-serial kernel
-                             "traffic": (NCU_TRAFFIC["backward"] if args.bwd_impl == "serial"
-                                         else None),
+                             "traffic": NCU_TRAFFIC["backward" if args.bwd_impl == "serial"
+                                                    else "backward_chunked"],
                              "algorithmic_bytes_per_launch": bbytes},
                 "kernel": ("token-serial adjoint on CUDA cores, one CTA per (sequence, head, "
                            "32-column tile), plus a tile reduction" if args.bwd_impl == "serial"
                            else "chunkwise (16-token chunk-WY reverse) on CUDA cores: prep and "
                                 "gradients over all chunks, two scans per (sequence, head, "
-                                "32-column tile)"),
+                                "16-column tile) fed by asynchronous copies two chunks ahead"),
                 "entry_point": "ckda_bwd_chunked" if args.bwd_impl == "chunked" else "ckda_bwd",
                 "gpu_launches": (2 if args.bwd_impl == "serial" else 4) * args.bwd_steps}
     del bws, bout
