@@ -159,6 +159,46 @@ def test_ckda_varlen_full(cuda_lib):
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
 
 
+def test_ckda_long_sequence_large_workspace(cuda_lib):
+    """One 32768-token sequence with 32 heads: 2.7 GB of chunk workspace, so
+    its byte offsets pass 2^31. The first and the last head are checked in
+    full against the oracle; every output of every head must be finite."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=909)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([32768]), H=32)
+    o, sf = run_fwd(inp)
+    assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(sf).all())
+    heads = [0, 31]
+    sub = {key: inp[key][:, heads].contiguous() for key in ("q", "k", "v", "alpha", "beta")}
+    sub["initial_state"] = inp["initial_state"][:, heads].contiguous()
+    sub["cu_seqlens"] = inp["cu_seqlens"]
+    o_ref, sf_ref = ref_fwd(sub)
+    check_bf16_out(o.cpu()[:, heads], o_ref)
+    check_close(sf.cpu()[:, heads], sf_ref, 1e-2, 0.0, "final_state")
+
+
+# Final states of sequences a few tokens long are the initial state (rms 0.15)
+# plus one chunk's update, and tf32 operands round that update at 2^-11 of its
+# own size: the rounding model of the kernels' data flow (precision_sim.py)
+# puts max|S - S_ref| at 1.18e-2 * rms(S_ref) for the case below. The GPU
+# measures the same. The bound derived for such states is 2e-2 * rms; the
+# pages' workloads (sequences of 128 tokens and more) keep the 1e-2 of the
+# output's rule.
+SHORT_STATE_REL = 2e-2
+
+
+def test_many_short_sequences(cuda_lib):
+    """3000 sequences of 0 to 9 tokens (most of them shorter than one chunk,
+    some empty), 4 heads: the slot table, partial chunks and per-sequence
+    states at scale, every output against the oracle."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=1234)
+    lens = np.random.default_rng(5).integers(0, 10, size=3000)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu(lens), H=4)
+    o, sf = run_fwd(inp)
+    o_ref, sf_ref = ref_fwd(inp)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, SHORT_STATE_REL, 0.0, "final_state")
+
+
 def test_bf16_ragged_small(cuda_lib):
     """bf16 path on ragged lengths (partial chunks, empty and 1-token
     sequences), scale != 1."""
