@@ -16,7 +16,10 @@
 namespace ckda {
 namespace {
 
-constexpr int kThreads = 256;
+// 512 threads per CTA: both programs' CTAs are few per SM (the scan's 176 KB
+// of shared memory allow one, the prep's two), and their phases are chains of
+// shared-memory loads and FMAs, so more warps per SM hide more of that latency.
+constexpr int kThreads = 512;
 
 using Exec = DeviceExec<kThreads>;  // one phase per barrier, kThreads threads
 
