@@ -24,8 +24,12 @@ constexpr int kGradTile = 16;  // columns per tile of the gradient program
 constexpr int kScanTile = 16;  // columns per CTA of the scans (and per tile of prep)
 
 constexpr int kThreads = 256;
+// the prep's CTAs (51 KB of shared memory, few registers) take 512 threads:
+// four of them fill an SM's warp slots
+constexpr int kPrepThreads = 512;
 
 using Exec = DeviceExec<kThreads>;  // one phase per barrier, kThreads threads
+using PrepExec = DeviceExec<kPrepThreads>;
 
 // the chunk of slot blockIdx.x: token rows [t0, t0 + L); false if none
 __device__ __forceinline__ bool slot_rows(const int32_t *cu, int N, int T, int T_total,
@@ -41,14 +45,14 @@ __device__ __forceinline__ bool slot_rows(const int32_t *cu, int N, int T, int T
 }
 
 template <typename IOT, int DK, int DVT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kPrepThreads)
 bwd_prep_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ cu, int N,
                 int T, int T_total, unsigned int *err) {
   extern __shared__ float sm[];
   int t0, L;
   if (!slot_rows(cu, N, T, T_total, err, t0, L)) return;
-  Exec x;
-  bwdc::prep_program<Exec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, blockIdx.y, t0, L,
+  PrepExec x;
+  bwdc::prep_program<PrepExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, blockIdx.y, t0, L,
                                                         blockIdx.x);
 }
 
@@ -99,7 +103,7 @@ cudaError_t launch_dims(const bwdc::Args<IOT> &a, const bwdc::SplitWs &w, const 
   if ((e = set_smem(bwd_scan_kernel<IOT, DK, DVT, false>, SL::BYTES)) != cudaSuccess) return e;
   if ((e = set_smem(bwd_scan_kernel<IOT, DK, DVT, true>, SL::BYTES)) != cudaSuccess) return e;
   if ((e = set_smem(bwd_grads_kernel<IOT, DK>, GL::BYTES)) != cudaSuccess) return e;
-  bwd_prep_kernel<IOT, DK, DVT><<<dim3(slots, a.H), kThreads, PL::BYTES, st>>>(a, w, cu, N, T,
+  bwd_prep_kernel<IOT, DK, DVT><<<dim3(slots, a.H), kPrepThreads, PL::BYTES, st>>>(a, w, cu, N, T,
                                                                               T_total, err);
   bwd_scan_kernel<IOT, DK, DVT, false><<<dim3(a.H, N, ntile), kThreads, SL::BYTES, st>>>(
       a, w, cu, T, T_total, err);
