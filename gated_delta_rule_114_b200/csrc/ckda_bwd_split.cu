@@ -25,11 +25,14 @@ constexpr int kScanTile = 16;  // columns per CTA of the scans (and per tile of 
 
 constexpr int kThreads = 256;
 // the prep's CTAs (51 KB of shared memory, few registers) take 512 threads:
-// four of them fill an SM's warp slots
+// four of them fill an SM's warp slots; so do the scans' (97 KB, two per SM,
+// at most 64 registers a thread)
 constexpr int kPrepThreads = 512;
+constexpr int kScanThreads = 512;
 
 using Exec = DeviceExec<kThreads>;  // one phase per barrier, kThreads threads
 using PrepExec = DeviceExec<kPrepThreads>;
+using ScanExec = DeviceExec<kScanThreads>;
 
 // the chunk of slot blockIdx.x: token rows [t0, t0 + L); false if none
 __device__ __forceinline__ bool slot_rows(const int32_t *cu, int N, int T, int T_total,
@@ -57,20 +60,20 @@ bwd_prep_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ 
 }
 
 template <typename IOT, int DK, int DVT, bool REVERSE>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kScanThreads, 2)
 bwd_scan_kernel(bwdc::Args<IOT> a, bwdc::SplitWs w, const int32_t *__restrict__ cu, int T,
                 int T_total, unsigned int *err) {
   extern __shared__ float sm[];
   const int h = blockIdx.x, n = blockIdx.y, tile = blockIdx.z;
   int bos, eos;
   seq_bounds(cu, n, T, T_total, err, bos, eos);
-  Exec x;
+  ScanExec x;
   if (REVERSE)
-    bwdc::scan2_program<Exec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
-                                                           bos / CK + n);
+    bwdc::scan2_program<ScanExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
+                                                               bos / CK + n);
   else
-    bwdc::scan1_program<Exec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
-                                                           bos / CK + n);
+    bwdc::scan1_program<ScanExec, IO<IOT>, IOT, DK, DVT>(x, a, w, sm, h, n, tile, bos, eos,
+                                                               bos / CK + n);
 }
 
 template <typename IOT, int DK>
@@ -105,9 +108,9 @@ cudaError_t launch_dims(const bwdc::Args<IOT> &a, const bwdc::SplitWs &w, const 
   if ((e = set_smem(bwd_grads_kernel<IOT, DK>, GL::BYTES)) != cudaSuccess) return e;
   bwd_prep_kernel<IOT, DK, DVT><<<dim3(slots, a.H), kPrepThreads, PL::BYTES, st>>>(a, w, cu, N, T,
                                                                               T_total, err);
-  bwd_scan_kernel<IOT, DK, DVT, false><<<dim3(a.H, N, ntile), kThreads, SL::BYTES, st>>>(
+  bwd_scan_kernel<IOT, DK, DVT, false><<<dim3(a.H, N, ntile), kScanThreads, SL::BYTES, st>>>(
       a, w, cu, T, T_total, err);
-  bwd_scan_kernel<IOT, DK, DVT, true><<<dim3(a.H, N, ntile), kThreads, SL::BYTES, st>>>(
+  bwd_scan_kernel<IOT, DK, DVT, true><<<dim3(a.H, N, ntile), kScanThreads, SL::BYTES, st>>>(
       a, w, cu, T, T_total, err);
   bwd_grads_kernel<IOT, DK><<<dim3(slots, a.H), kThreads, GL::BYTES, st>>>(a, w, cu, N, T,
                                                                           T_total, err);
