@@ -15,7 +15,7 @@ import oracle
 from gated_delta_rule_114_b200 import ckda
 from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,
                                               make_decode_tokens,
-                                              make_fwd_inputs, seqlens)
+                                              make_fwd_inputs)
 from parity_util import as_f64, check_bf16_out, check_close, check_fp32, to_dev
 
 pytestmark = pytest.mark.gpu
