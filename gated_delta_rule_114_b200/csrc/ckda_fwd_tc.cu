@@ -6,7 +6,7 @@
 //
 //  * ckda_chunk_prep_kernel: persistent, one CTA per SM, walking the (chunk,
 //    head) items of all sequences (a small kernel first tabulates which
-//    chunk each slot holds). For each item it builds everything that does not
+//    chunk each slot holds); q, k and v come in by tensor-map copies. For each item it builds everything that does not
 //    depend on the state entering it (the chunk-WY / UT-transform factors of
 //    the product of diagonal-plus-rank-one transitions, Semidirect Fourier
 //    Delta Attention §2.2, and the affine chunk transfer's write summary, §1
@@ -38,7 +38,9 @@
 // adds up to about 2-3% of rms(o) on the CKDA and KDA workloads, above the
 // 1e-2 rms bound; tf32 operands keep it near 2e-3. Every MMA is kind::tf32,
 // operands rounded to tf32 when they are written.
+#include <cuda.h>  // CUtensorMap (the encoder is reached through the runtime)
 #include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <mutex>
@@ -137,7 +139,7 @@ constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
 constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68] (with P_M: staged Ut rows, epilogue)
 constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
 constexpr uint32_t P_B = 216064;      //   256 beta
-constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..3] + TMEM address + flag
+constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..3], TMEM address, flag, input mbarrier
 constexpr uint32_t P_P = 216384;      //  2048 gate products of whole sub-blocks [4][128]
 constexpr uint32_t P_RN = 218432;     //   256 key row inverse norms (fused prologue)
 constexpr uint32_t P_SMEM = 218688 + 1024;
@@ -196,14 +198,13 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase,
 // the diagonal sub-blocks), which is the same as using the normalised keys.
 template <bool GATED>
 __global__ void __launch_bounds__(NTP, 1)
-ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
-                       const __nv_bfloat16 *__restrict__ k,
-                       const __nv_bfloat16 *__restrict__ v,
-                       const void *__restrict__ alpha_in,
+ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
                        const float *__restrict__ beta,
                        const int2 *__restrict__ slot_tab, int n_items,
                        int H, int DV, GateArgs ga, uint8_t *__restrict__ ws,
-                       unsigned int *err) {
+                       unsigned int *err, const __grid_constant__ CUtensorMap map_q,
+                       const __grid_constant__ CUtensorMap map_k,
+                       const __grid_constant__ CUtensorMap map_v) {
   const float *__restrict__ alpha = reinterpret_cast<const float *>(alpha_in);
   const __nv_bfloat16 *__restrict__ alogit = reinterpret_cast<const __nv_bfloat16 *>(alpha_in);
   extern __shared__ uint8_t smem_raw[];
@@ -224,6 +225,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..3]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
+  uint64_t *bin = reinterpret_cast<uint64_t *>(sm + P_BAR + 40);  // q, k, v copies
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (warp == 0) {
@@ -232,6 +234,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   }
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
+    mbar_init(bin, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -241,28 +244,25 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
-  // An item's q, k, v rows, beta (or its logits) and, without the fused
-  // prologue, alpha arrive by per-thread asynchronous copies (cp.async) into
-  // their shared buffers, issued during the previous item once each buffer's
-  // last reader is done: q, k, v while D5 runs (after [M ; I] x T, their last
-  // reader), alpha and beta after the epilogue has read Qhat. Rows past the
-  // chunk's end read as zero (alpha: 1). An item whose copies were not issued
-  // ahead (the first, or one after empty slots) issues them at its start.
+  // An item's q, k and v rows arrive by tensor-map copies (one box of 64
+  // token rows per input, issued by thread 0 and counted on mbarrier bin);
+  // beta (or its logits) and, without the fused prologue, alpha by per-thread
+  // asynchronous copies (cp.async). They are issued during the previous item
+  // once each buffer's last reader is done: q, k, v while D5 runs (after
+  // [M ; I] x T, their last reader), alpha and beta after the epilogue has
+  // read Qhat. An item whose copies were not issued ahead (the first, or one
+  // after empty slots) issues them at its start. Box rows past the chunk's end
+  // hold the next sequence's tokens (zeros past the last token) until the
+  // item's start overwrites them with zeros; alpha and beta rows past the end
+  // are written as 1 and 0 directly.
   const int nvp = DV / 8, lnv = __ffs(nvp) - 1;  // 16-byte pieces of a v row (a power of 2)
-  auto issue_qkv = [&](int t0r, int Lr, int hr) {
-    for (int idx = tid; idx < 2 * C * 16; idx += NTP) {  // q, k: 64 rows x 16 pieces
-      const int kt = idx >> 10, i = (idx >> 4) & (C - 1), w = idx & 15;
-      const uint32_t nb = i < Lr ? 16u : 0u;  // 0: zero fill, nothing read
-      const size_t off = ((size_t)(t0r + (i < Lr ? i : 0)) * H + hr) * DK + w * 8;
-      cp_async16(sm + (kt ? P_K : P_Q) + i * 256 + w * 16, (kt ? k : q) + off, nb);
+  auto issue_qkv = [&](int t0r, int hr) {
+    if (tid == 0) {
+      mbar_arrive_expect_tx(bin, (uint32_t)C * (2 * DK + DV) * 2u);
+      tma_load_3d(sm + P_Q, &map_q, 0, hr, t0r, bin);
+      tma_load_3d(sm + P_K, &map_k, 0, hr, t0r, bin);
+      tma_load_3d(sm + P_V, &map_v, 0, hr, t0r, bin);
     }
-    for (int idx = tid; idx < C * nvp; idx += NTP) {  // v: 64 rows x DV / 8 pieces
-      const int i = idx >> lnv, w = idx & (nvp - 1);
-      const uint32_t nb = i < Lr ? 16u : 0u;
-      const size_t off = ((size_t)(t0r + (i < Lr ? i : 0)) * H + hr) * DV + w * 8;
-      cp_async16(sm + P_V + i * DV * 2 + w * 16, v + off, nb);
-    }
-    cp_async_commit();
   };
   auto issue_gates = [&](int t0r, int Lr, int hr) {  // alpha (no fused prologue), beta
     if constexpr (!GATED) {
@@ -303,7 +303,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     // prologue) alpha have been copied in asynchronously; the gate logits of
     // the fused prologue come through registers
     if (raw_for != it) {
-      issue_qkv(t0, L, h);
+      issue_qkv(t0, h);
       issue_gates(t0, L, h);
     }
     raw_for = -1;
@@ -319,6 +319,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
             al[u] = __ldg(reinterpret_cast<const uint4 *>(alogit + ((size_t)(t0 + i) * H + h) * DK + ch * 8));
         }
       }
+      if (!mbar_wait(bin, ph)) *s_abort = 1;
       cp_async_wait_all();
       if constexpr (GATED) {
         __syncthreads();  // every thread's k rows have landed
@@ -338,7 +339,8 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           *reinterpret_cast<float4 *>(sAl + al_off(i, 8 * ch)) = make_float4(x[0], x[1], x[2], x[3]);
           *reinterpret_cast<float4 *>(sAl + al_off(i, 8 * ch + 4)) = make_float4(x[4], x[5], x[6], x[7]);
           // key row inverse norm: 16 lanes hold row i's 128 channels
-          const uint4 kq = *reinterpret_cast<const uint4 *>(sm + P_K + i * 256 + ch * 16);
+          uint4 kq = make_uint4(0, 0, 0, 0);
+          if (i < L) kq = *reinterpret_cast<const uint4 *>(sm + P_K + i * 256 + ch * 16);
           const uint32_t kw[4] = {kq.x, kq.y, kq.z, kq.w};
           float ss = 0.f;
 #pragma unroll
@@ -351,6 +353,20 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
           if (ch == 0) sRN[i] = (i < L) ? key_rnorm(ga, ss) : 0.f;
         }
         if (tid < L) sB[tid] = gate_beta(ga, sB[tid]);  // beta from its logit
+      }
+      // rows past the chunk's end: q, k, v zero (the fused prologue reads no
+      // k row past the end before this)
+      if (L < C) {
+        const int nr = C - L;
+        for (int idx = tid; idx < nr * 16; idx += NTP) {
+          const int i = L + (idx >> 4), w = idx & 15;
+          *reinterpret_cast<uint4 *>(sm + P_Q + i * 256 + w * 16) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4 *>(sm + P_K + i * 256 + w * 16) = make_uint4(0, 0, 0, 0);
+        }
+        for (int idx = tid; idx < nr * nvp; idx += NTP) {
+          const int i = L + (idx >> lnv), w = idx & (nvp - 1);
+          *reinterpret_cast<uint4 *>(sm + P_V + i * DV * 2 + w * 16) = make_uint4(0, 0, 0, 0);
+        }
       }
       // the gate pass writes over the staging: the stores must have read it
       if (tid == 0) bulk_wait_read0();
@@ -936,7 +952,7 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
     // while D5 runs: the q, k, v buffers' last reader ([M ; I] x T) is done,
     // so the next item's rows may come in
     if (nxt.y > 0) {
-      issue_qkv(nxt.x, nxt.y, nit % H);
+      issue_qkv(nxt.x, nit % H);
       raw_for = nit;
     }
     if (!wait_all(&bar[2], ph, s_abort)) break;
@@ -983,6 +999,11 @@ ckda_chunk_prep_kernel(const __nv_bfloat16 *__restrict__ q,
   cur = nxt;
   }  // item loop
 
+  // After an abort, q, k, v copies still in flight land before shared memory
+  // is released: those issued for the next item (raw_for >= 0 only then)
+  // complete phase ph ^ 1; otherwise the item's own, if waiting for them is
+  // what timed out, phase ph (an already completed phase is not waited for).
+  if (*s_abort) mbar_wait(bin, raw_for >= 0 ? ph ^ 1u : ph);
   cp_async_wait_all();  // copies issued ahead land before shared memory is released
   if (tid == 0) {
     if (*s_abort) flag_error(err, kErrMbarTimeout);
@@ -1291,6 +1312,37 @@ static int sm_count() {
   return cache[dev];
 }
 
+// cuTensorMapEncodeTiled, reached through the runtime (no link against the
+// driver library).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Tensor map over a [T_total, H, d] bf16 row-major tensor (dims d, H,
+// T_total, innermost first) whose box is one head's row of d channels by 64
+// tokens, laid out densely in shared memory.
+static bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int T_total) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T_total};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)d, 1u, (cuuint32_t)C};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
                           const void *alpha, const float *beta,
                           const float *s0, float *sf, void *o,
@@ -1315,9 +1367,12 @@ cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
     const long long items = (long long)slots * H;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(items, (long long)sm_count());
-    prep<<<grid, NTP, P_SMEM, st>>>(
-        (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-        alpha, beta, tab, (int)items, H, dv, g, (uint8_t *)ws, err);
+    CUtensorMap mq, mk, mv;
+    if (!encode_rows(&mq, q, DK, H, T_total) || !encode_rows(&mk, k, DK, H, T_total) ||
+        !encode_rows(&mv, v, dv, H, T_total))
+      return cudaErrorInvalidValue;
+    prep<<<grid, NTP, P_SMEM, st>>>(alpha, beta, tab, (int)items, H, dv, g, (uint8_t *)ws, err,
+                                     mq, mk, mv);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

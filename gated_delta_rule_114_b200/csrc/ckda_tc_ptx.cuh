@@ -336,6 +336,20 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32
       : "memory");
 }
 
+// Tiled 3-D tensor copy global -> shared (this CTA, no multicast) through a
+// tensor map `map` (a __grid_constant__ kernel parameter), box origin
+// (x, y, z) in elements, innermost first; x * element size must be a multiple
+// of 16 bytes. Elements outside the tensor are written as zero. Completion:
+// the whole box's bytes are counted on the mbarrier.
+__device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *map, int x, int y, int z,
+                                            uint64_t *mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst_smem)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(mbar))
+      : "memory");
+}
+
 // Bulk copy shared (this CTA) -> global, tracked in this thread's bulk
 // async-group. Both addresses 16-byte aligned, bytes % 16 == 0.
 __device__ __forceinline__ void bulk_s2g(void *dst, const void *src_smem, uint32_t bytes) {
