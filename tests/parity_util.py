@@ -77,3 +77,26 @@ def to_dev(inp: dict, device="cuda") -> dict:
     for key, val in inp.items():
         out[key] = val.to(device).contiguous() if isinstance(val, torch.Tensor) else val
     return out
+
+
+def poison(inp: dict, a: int, b: int, keys) -> None:
+    """Overwrite tokens a .. b-1 of the inputs named by `keys` with NaN (the
+    first few with +inf), in place."""
+    for key in keys:
+        x = inp[key].clone()
+        x[a:b] = float("nan")
+        x[a:min(b, a + 5)] = float("inf")
+        inp[key] = x
+
+
+def select_seqs(inp: dict, keep, keys):
+    """The packed inputs of sequences `keep` only (their token rows, initial
+    states and cu_seqlens), and the token rows they came from."""
+    cu = inp["cu_seqlens"].tolist()
+    idx = torch.cat([torch.arange(cu[n], cu[n + 1]) for n in keep])
+    sub = {key: inp[key][idx] for key in keys}
+    lens = [cu[n + 1] - cu[n] for n in keep]
+    sub["cu_seqlens"] = torch.from_numpy(np.concatenate([[0], np.cumsum(lens)]).astype(np.int32))
+    s0 = inp.get("initial_state")
+    sub["initial_state"] = None if s0 is None else s0[list(keep)]
+    return sub, idx

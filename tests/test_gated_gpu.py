@@ -13,7 +13,8 @@ from gated_delta_rule_114_b200 import ckda
 from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,
                                               make_gated_decode_tokens,
                                               make_gated_fwd_inputs)
-from parity_util import check_bf16_out, check_close, check_fp32, to_dev
+from parity_util import (check_bf16_out, check_close, check_fp32, poison, select_seqs,
+                         to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -55,6 +56,21 @@ def test_gated_tensor_core_bf16(cuda_lib, gname, d_v):
     o_ref, sf_ref = ref_gated(inp, GATES[gname], 0.9)
     check_bf16_out(o, o_ref)
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
+def test_gated_partial_chunk_ignores_the_next_sequence(cuda_lib):
+    """As in the plain forward: with the sequence after a partial chunk full
+    of NaN and inf (q, raw k, v and both gate logits), the sequences around
+    it match the oracle run on them alone."""
+    keys = ("q", "k_raw", "v", "a_logit", "c_logit")
+    w = custom("ckda_B1_H32_T8192_d128", seed=8300)
+    inp = make_gated_fwd_inputs(w, cu_seqlens=lens_cu([100, 70, 29]), H=4)
+    poison(inp, 100, 170, keys)
+    o, sf = run_gated(inp, GATES["ckda"], 64, 1.0)
+    sub, idx = select_seqs(inp, [0, 2], keys)
+    o_ref, sf_ref = ref_gated(sub, GATES["ckda"], 1.0)
+    check_bf16_out(o[idx], o_ref)
+    check_close(sf[[0, 2]], sf_ref, 1e-2, 0.0, "final_state")
 
 
 def test_gated_tensor_core_bf16_long(cuda_lib):

@@ -16,7 +16,8 @@ from gated_delta_rule_114_b200 import ckda
 from gated_delta_rule_114_b200.inputs import (WORKLOADS, make_decode_state,
                                               make_decode_tokens,
                                               make_fwd_inputs)
-from parity_util import as_f64, check_bf16_out, check_close, check_fp32, to_dev
+from parity_util import (as_f64, check_bf16_out, check_close, check_fp32, poison,
+                         select_seqs, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -209,6 +210,22 @@ def test_bf16_ragged_small(cuda_lib):
     o_ref, sf_ref = ref_fwd(inp, scale=1.5)
     check_bf16_out(o, o_ref)
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
+
+
+def test_partial_chunk_ignores_the_next_sequence(cuda_lib):
+    """The tensor-core prep loads q, k and v in whole 64-token boxes, so the
+    rows past the end of a sequence's last (partial) chunk first hold the next
+    sequence's tokens, until the kernel clears them. With that next sequence
+    full of NaN and inf (q, k, v, alpha, beta), the sequences before and after
+    it must still match the oracle run on them alone."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=4343)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([100, 70, 29]), H=4)
+    poison(inp, 100, 170, ("q", "k", "v", "alpha", "beta"))
+    o, sf = run_fwd(inp)
+    sub, idx = select_seqs(inp, [0, 2], ("q", "k", "v", "alpha", "beta"))
+    o_ref, sf_ref = ref_fwd(sub)
+    check_bf16_out(o[idx], o_ref)
+    check_close(sf[[0, 2]], sf_ref, 1e-2, 0.0, "final_state")
 
 
 @pytest.mark.parametrize("d_k,d_v,chunk", [(128, 32, 64), (128, 64, 64), (64, 64, 64),
