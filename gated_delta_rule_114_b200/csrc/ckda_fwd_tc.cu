@@ -6,7 +6,7 @@
 //
 //  * ckda_chunk_prep_kernel: persistent, one CTA per SM, walking the (chunk,
 //    head) items of all sequences (a small kernel first tabulates which
-//    chunk each slot holds); q, k and v come in by tensor-map copies. For each item it builds everything that does not
+//    chunk each slot holds); q, k, v and alpha come in by tensor-map copies. For each item it builds everything that does not
 //    depend on the state entering it (the chunk-WY / UT-transform factors of
 //    the product of diagonal-plus-rank-one transitions, Semidirect Fourier
 //    Delta Attention §2.2, and the affine chunk transfer's write summary, §1
@@ -43,6 +43,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "ckda.h"
@@ -58,14 +59,11 @@ constexpr int C = 64, DK = 128, DVT = 32;
 constexpr int PF_STEP = 128;  // bytes per L2 prefetch of the next item's gate logits
 constexpr int AL_S = 132;  // fp32 row stride of alpha / Qhat
 
-// Float offset of (row i, channel c) in the alpha / Qhat buffer: the 16-byte
-// piece p = c / 4 of a row sits at p ^ ((p >> 3) & 1), so that the 16 lanes
-// of a half-warp reading pieces 2 sl (or 2 sl + 1) of one row hit every bank
-// group twice, not half of them four times.
-__device__ __forceinline__ int al_off(int i, int c) {
-  const int p = c >> 2;
-  return i * AL_S + 4 * (p ^ ((p >> 3) & 1)) + (c & 3);
-}
+// Float offset of (row i, channel c) in the alpha / Qhat buffer: rows of 128
+// channels padded to 132 floats (the tensor-map copy of alpha fills the
+// padding with zeros), so that 16-byte reads of one channel block by the
+// threads of 32 consecutive rows fall into different banks.
+__device__ __forceinline__ int al_off(int i, int c) { return i * AL_S + c; }
 
 // ---------------------------------------------------------------- workspace
 // One block per (chunk slot, head); chunk c of sequence n sits in slot
@@ -139,16 +137,17 @@ constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
 constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68] (with P_M: staged Ut rows, epilogue)
 constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
 constexpr uint32_t P_B = 216064;      //   256 beta
-constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..3], TMEM address, flag, input mbarrier
+constexpr uint32_t P_BAR = 216320;    //    64 mbarriers [0..3], TMEM address, flag, input mbarriers [2]
 constexpr uint32_t P_P = 216384;      //  2048 gate products of whole sub-blocks [4][128]
 constexpr uint32_t P_RN = 218432;     //   256 key row inverse norms (fused prologue)
 constexpr uint32_t P_SMEM = 218688 + 1024;
 
 // TMEM columns of the prep kernel (512 allocated; one CTA per SM)
 constexpr uint32_t TP_G = 0;      //  96 Gram accumulator
-constexpr uint32_t TP_AD5 = 96;   //  64 [M T ; T] (A of D5)
-constexpr uint32_t TP_D5 = 160;   // 256 [M W | M Ut ; W | Ut]
-constexpr uint32_t TP_G4 = 416;   //  96 Gram inside the 16-token sub-blocks
+constexpr uint32_t TP_G4 = 96;    //  96 Gram inside the 16-token sub-blocks
+constexpr uint32_t TP_QH = 0;     // 128 Qhat (lanes 0..63), once both Grams are read
+constexpr uint32_t TP_AD5 = 192;  //  64 [M T ; T] (A of D5)
+constexpr uint32_t TP_D5 = 256;   // 256 [M W | M Ut ; W | Ut]
 constexpr uint32_t TP_COLS = 512;
 
 constexpr uint32_t ID_G = idesc_tf32(128, 96, 1, 1);
@@ -204,8 +203,8 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
                        int H, int DV, GateArgs ga, uint8_t *__restrict__ ws,
                        unsigned int *err, const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
-                       const __grid_constant__ CUtensorMap map_v) {
-  const float *__restrict__ alpha = reinterpret_cast<const float *>(alpha_in);
+                       const __grid_constant__ CUtensorMap map_v,
+                       const __grid_constant__ CUtensorMap map_a) {
   const __nv_bfloat16 *__restrict__ alogit = reinterpret_cast<const __nv_bfloat16 *>(alpha_in);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
@@ -225,7 +224,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..3]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
-  uint64_t *bin = reinterpret_cast<uint64_t *>(sm + P_BAR + 40);  // q, k, v copies
+  uint64_t *bin = reinterpret_cast<uint64_t *>(sm + P_BAR + 40);  // input copies: [0] q, k, v; [1] alpha
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (warp == 0) {
@@ -234,7 +233,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   }
   if (tid == 0) {
     for (int i = 0; i < 4; ++i) mbar_init(&bar[i], 1);
-    mbar_init(bin, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&bin[i], 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -244,33 +243,32 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
-  // An item's q, k and v rows arrive by tensor-map copies (one box of 64
-  // token rows per input, issued by thread 0 and counted on mbarrier bin);
-  // beta (or its logits) and, without the fused prologue, alpha by per-thread
-  // asynchronous copies (cp.async). They are issued during the previous item
-  // once each buffer's last reader is done: q, k, v while D5 runs (after
-  // [M ; I] x T, their last reader), alpha and beta after the epilogue has
-  // read Qhat. An item whose copies were not issued ahead (the first, or one
-  // after empty slots) issues them at its start. Box rows past the chunk's end
-  // hold the next sequence's tokens (zeros past the last token) until the
-  // item's start overwrites them with zeros; alpha and beta rows past the end
-  // are written as 1 and 0 directly.
+  // An item's q, k and v rows and, without the fused prologue, alpha arrive
+  // by tensor-map copies (one box of 64 token rows per input, issued by
+  // thread 0, counted on mbarrier bin[0] or bin[1]); beta (or its logits) by
+  // per-thread copies (cp.async). They are issued during the previous item
+  // once each buffer's last reader is done: alpha and beta when the [M ; I]
+  // and T operands are built (Qhat has moved to tensor memory, and gamma and
+  // beta were last read by the WY operand build), q, k, v while D5 runs
+  // ([M ; I] x T was their last reader). An item whose copies were not issued
+  // ahead (the first, or one after empty slots) issues them at its start. Box
+  // rows past the chunk's end hold the next sequence's tokens (zeros past the
+  // last token) until the item's start overwrites them (q, k, v: 0, alpha: 1);
+  // beta rows past the end are written as 0.
   const int nvp = DV / 8, lnv = __ffs(nvp) - 1;  // 16-byte pieces of a v row (a power of 2)
   auto issue_qkv = [&](int t0r, int hr) {
     if (tid == 0) {
-      mbar_arrive_expect_tx(bin, (uint32_t)C * (2 * DK + DV) * 2u);
-      tma_load_3d(sm + P_Q, &map_q, 0, hr, t0r, bin);
-      tma_load_3d(sm + P_K, &map_k, 0, hr, t0r, bin);
-      tma_load_3d(sm + P_V, &map_v, 0, hr, t0r, bin);
+      mbar_arrive_expect_tx(&bin[0], (uint32_t)C * (2 * DK + DV) * 2u);
+      tma_load_3d(sm + P_Q, &map_q, 0, hr, t0r, &bin[0]);
+      tma_load_3d(sm + P_K, &map_k, 0, hr, t0r, &bin[0]);
+      tma_load_3d(sm + P_V, &map_v, 0, hr, t0r, &bin[0]);
     }
   };
   auto issue_gates = [&](int t0r, int Lr, int hr) {  // alpha (no fused prologue), beta
     if constexpr (!GATED) {
-      for (int idx = tid; idx < C * 32; idx += NTP) {  // 64 rows x 32 pieces of 4 floats
-        const int i = idx >> 5, c4 = (idx & 31) * 4;
-        float *dst = sAl + al_off(i, c4);
-        if (i < Lr) cp_async16(dst, alpha + ((size_t)(t0r + i) * H + hr) * DK + c4, 16u);
-        else *reinterpret_cast<float4 *>(dst) = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&bin[1], (uint32_t)C * AL_S * 4u);
+        tma_load_3d(sAl, &map_a, 0, hr, t0r, &bin[1]);
       }
     }
     if (tid < C) {
@@ -279,6 +277,12 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
     }
     cp_async_commit();
   };
+  auto wait_in = [&](int b, uint32_t parity) {  // all threads
+    if (!mbar_wait(&bin[b], parity)) *s_abort = 1;
+  };
+  // copy groups issued for the next item and not yet waited for (bit 0: q, k,
+  // v; bit 1: alpha); looked at only when an abort ends the loop
+  int ahead = 0;
   int raw_for = -1;  // item whose row copies were issued ahead (CTA-uniform)
 
   // Persistent: items (slot, head) = it / H, it % H, strided by the grid.
@@ -319,7 +323,9 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
             al[u] = __ldg(reinterpret_cast<const uint4 *>(alogit + ((size_t)(t0 + i) * H + h) * DK + ch * 8));
         }
       }
-      if (!mbar_wait(bin, ph)) *s_abort = 1;
+      wait_in(0, ph);
+      if constexpr (!GATED) wait_in(1, ph);
+      ahead = 0;
       cp_async_wait_all();
       if constexpr (GATED) {
         __syncthreads();  // every thread's k rows have landed
@@ -354,8 +360,8 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
         }
         if (tid < L) sB[tid] = gate_beta(ga, sB[tid]);  // beta from its logit
       }
-      // rows past the chunk's end: q, k, v zero (the fused prologue reads no
-      // k row past the end before this)
+      // rows past the chunk's end: q, k, v zero, alpha one (the fused
+      // prologue has set its alpha rows and reads no k row past the end)
       if (L < C) {
         const int nr = C - L;
         for (int idx = tid; idx < nr * 16; idx += NTP) {
@@ -366,6 +372,12 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
         for (int idx = tid; idx < nr * nvp; idx += NTP) {
           const int i = L + (idx >> lnv), w = idx & (nvp - 1);
           *reinterpret_cast<uint4 *>(sm + P_V + i * DV * 2 + w * 16) = make_uint4(0, 0, 0, 0);
+        }
+        if constexpr (!GATED) {
+          for (int idx = tid; idx < nr * 32; idx += NTP) {
+            const int i = L + (idx >> 5), c4 = (idx & 31) * 4;
+            *reinterpret_cast<float4 *>(sAl + al_off(i, c4)) = make_float4(1.f, 1.f, 1.f, 1.f);
+          }
         }
       }
       // the gate pass writes over the staging: the stores must have read it
@@ -475,21 +487,28 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
     }
     // ... and, meanwhile on CUDA cores, the pairs inside each 4-token group
     // (j <= i, same group). A half-warp owns row i (lane sl: channels
-    // 8 sl .. 8 sl + 7) and walks j = i, i-1, ... down the group carrying
+    // 4 sl .. 4 sl + 3 and 64 + 4 sl .. 64 + 4 sl + 3, so that the 8 lanes
+    // of each 16-byte access phase read 128 consecutive bytes of a row) and
+    // walks j = i, i-1, ... down the group carrying
     // G_{i<-j} (paired fp32); a reduce-scatter butterfly over the 16 lanes
     // then leaves entry sl / 2 of [A row | M row] (4 + 4 entries) in lanes
     // sl. Warp w takes group 2 (w / 2) + half and its rows {0, 3} (w even) or
     // {1, 2} (w odd), so every half-warp walks 5 steps.
     {
-      const int sl = lane & 15, c8 = 8 * sl;
+      const int sl = lane & 15, c4 = 4 * sl;
+      auto ld8 = [&](const __nv_bfloat16 *row) {  // this lane's 8 channels of a bf16 row
+        const uint2 lo = *reinterpret_cast<const uint2 *>(row + c4);
+        const uint2 hi = *reinterpret_cast<const uint2 *>(row + 64 + c4);
+        return make_uint4(lo.x, lo.y, hi.x, hi.y);
+      };
       const int r0 = 4 * (2 * (warp >> 1) + (lane >> 4));
 #pragma unroll 1
       for (int pass = 0; pass < 2; ++pass) {
         const int ii = (warp & 1) ? 1 + pass : 3 * pass, i = r0 + ii;
         uint64_t ki[4], qi[4], g[4];
         {
-          const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + i * DK + c8);
-          const uint4 qr = *reinterpret_cast<const uint4 *>(sQr + i * DK + c8);
+          const uint4 kr = ld8(sKr + i * DK);
+          const uint4 qr = ld8(sQr + i * DK);
           ki[0] = bf2_to_f2(kr.x); ki[1] = bf2_to_f2(kr.y);
           ki[2] = bf2_to_f2(kr.z); ki[3] = bf2_to_f2(kr.w);
           qi[0] = bf2_to_f2(qr.x); qi[1] = bf2_to_f2(qr.y);
@@ -509,9 +528,9 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
         for (int jj = 3; jj >= 0; --jj) {
           if (jj <= ii) {
             const int j = r0 + jj;
-            const uint4 kr = *reinterpret_cast<const uint4 *>(sKr + j * DK + c8);
-            const float4 a0 = *reinterpret_cast<const float4 *>(sAl + al_off(j, c8));
-            const float4 a1 = *reinterpret_cast<const float4 *>(sAl + al_off(j, c8 + 4));
+            const uint4 kr = ld8(sKr + j * DK);
+            const float4 a0 = *reinterpret_cast<const float4 *>(sAl + al_off(j, c4));
+            const float4 a1 = *reinterpret_cast<const float4 *>(sAl + al_off(j, 64 + c4));
             const uint64_t x0 = f2mul(g[0], bf2_to_f2(kr.x)), x1 = f2mul(g[1], bf2_to_f2(kr.y));
             const uint64_t x2 = f2mul(g[2], bf2_to_f2(kr.z)), x3 = f2mul(g[3], bf2_to_f2(kr.w));
             uint64_t sa = f2mul(ki[0], x0), sq = f2mul(qi[0], x0);
@@ -890,6 +909,25 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
           st4_f32(GA + off_k_sw128_f32(DK + cv + (sw ? 0 : 1), j0 + g, DK + DV), x1[0], x1[1], x1[2], x1[3]);
         }
       }
+      // Qhat rows 0..63 into tensor memory (lanes 0..63, columns TP_QH ..
+      // TP_QH + 127), so that alpha's buffer is free from here on: warps 8, 9
+      // take columns 0..63 and warps 12, 13 columns 64..127, a row per lane
+      named_bar_sync(2, NTP / 2);  // every Qhat value of this phase is in place
+      if ((warp & 3) < 2) {
+        const int row = 32 * (warp & 3) + lane, c0 = 64 * ((warp >> 2) & 1);
+#pragma unroll
+        for (int hh = 0; hh < 64; hh += 32) {
+          float x[32];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 qv = *reinterpret_cast<const float4 *>(sAl + al_off(row, c0 + hh + e));
+            x[e] = qv.x; x[e + 1] = qv.y; x[e + 2] = qv.z; x[e + 3] = qv.w;
+          }
+          tmem_st32(tm + lane_base + TP_QH + (uint32_t)(c0 + hh), x);
+        }
+        tmem_wait_st();
+      }
+      fence_before_sync();
     }
     __syncthreads();
 
@@ -926,6 +964,13 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
                     desc_mn_sw128b32_f32(sb + P_B0, C, kk), ID_D0, kk > 0);
       mma_commit(&bar[1]);
     }
+    // gamma, Qhat (now in tensor memory) and beta have had their last reads:
+    // the next item's alpha and beta may come in
+    if (nxt.y > 0) {
+      issue_gates(nxt.x, nxt.y, nit % H);
+      raw_for = nit;
+      if constexpr (!GATED) ahead |= 2;
+    }
     if (!wait_all(&bar[1], ph, s_abort)) break;
     if ((warp & 3) < 2) {  // rows of M T: round the fp32 accumulator to tf32
       const uint32_t ta = tm + lane_base + TP_AD5 + (uint32_t)(16 * (warp >> 2));
@@ -953,7 +998,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
     // so the next item's rows may come in
     if (nxt.y > 0) {
       issue_qkv(nxt.x, nit % H);
-      raw_for = nit;
+      ahead |= 1;
     }
     if (!wait_all(&bar[2], ph, s_abort)) break;
     {
@@ -962,13 +1007,11 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
         float x[32];
         tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)cb, x);
         if (cb < DK) {  // [Qtil ; W] rows, tf32, K-major sw128 image
-          if (row < C) {
+          if (row < C) {  // warp-uniform (lane quarters 0, 1)
+            float qh[32];
+            tmem_ld32(tm + lane_base + TP_QH + (uint32_t)cb, qh);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 qh = *reinterpret_cast<const float4 *>(sAl + al_off(row, cb + e));
-              x[e] = qh.x - x[e]; x[e + 1] = qh.y - x[e + 1];
-              x[e + 2] = qh.z - x[e + 2]; x[e + 3] = qh.w - x[e + 3];
-            }
+            for (int e = 0; e < 32; ++e) x[e] = qh[e] - x[e];
           }
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
@@ -991,19 +1034,19 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
       bulk_s2g(wsb + WS_OU + 64u * DV * 4u, sm + P_A, 64u * DV * 4u);
       bulk_commit();
     }
-    // Qhat and beta have been read: the next item's gates may come in
-    if (nxt.y > 0) issue_gates(nxt.x, nxt.y, nit % H);
   } while (0);
   if (*s_abort) break;  // CTA-uniform: read after a barrier
   ph ^= 1u;
   cur = nxt;
   }  // item loop
 
-  // After an abort, q, k, v copies still in flight land before shared memory
-  // is released: those issued for the next item (raw_for >= 0 only then)
-  // complete phase ph ^ 1; otherwise the item's own, if waiting for them is
-  // what timed out, phase ph (an already completed phase is not waited for).
-  if (*s_abort) mbar_wait(bin, raw_for >= 0 ? ph ^ 1u : ph);
+  // After an abort, copies still in flight land before shared memory is
+  // released: those issued for the next item complete phase ph ^ 1; an
+  // item's own, if waiting for them is what timed out, phase ph (an already
+  // completed phase is not waited for).
+  if (*s_abort) {
+    for (int b = 0; b < (GATED ? 1 : 2); ++b) wait_in(b, ((ahead >> b) & 1) ? ph ^ 1u : ph);
+  }
   cp_async_wait_all();  // copies issued ahead land before shared memory is released
   if (tid == 0) {
     if (*s_abort) flag_error(err, kErrMbarTimeout);
@@ -1328,18 +1371,20 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Tensor map over a [T_total, H, d] bf16 row-major tensor (dims d, H,
-// T_total, innermost first) whose box is one head's row of d channels by 64
-// tokens, laid out densely in shared memory.
-static bool encode_rows(CUtensorMap *m, const void *base, int d, int H, int T_total) {
+// Tensor map over a [T_total, H, d] row-major tensor (dims d, H, T_total,
+// innermost first) whose box is `box0` elements of one head's row by 64
+// tokens, laid out densely in shared memory. box0 may exceed d: those
+// elements are filled with zeros.
+static bool encode_rows(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize,
+                        int d, int H, int T_total, int box0) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T_total};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)d, 1u, (cuuint32_t)C};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * esize, (cuuint64_t)H * d * esize};
+  const cuuint32_t box[3] = {(cuuint32_t)box0, 1u, (cuuint32_t)C};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+  return enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1367,12 +1412,18 @@ cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
     const long long items = (long long)slots * H;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(items, (long long)sm_count());
-    CUtensorMap mq, mk, mv;
-    if (!encode_rows(&mq, q, DK, H, T_total) || !encode_rows(&mk, k, DK, H, T_total) ||
-        !encode_rows(&mv, v, dv, H, T_total))
+    // input boxes: q, k (128 channels), v (d_v), alpha (128 channels padded to
+    // the 132-float shared row); the fused prologue reads its gate logits itself
+    CUtensorMap mq, mk, mv, ma;
+    std::memset(&ma, 0, sizeof(ma));
+    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_rows(&mq, q, bf, 2, DK, H, T_total, DK) ||
+        !encode_rows(&mk, k, bf, 2, DK, H, T_total, DK) ||
+        !encode_rows(&mv, v, bf, 2, dv, H, T_total, dv) ||
+        (!g.on && !encode_rows(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, H, T_total, AL_S)))
       return cudaErrorInvalidValue;
     prep<<<grid, NTP, P_SMEM, st>>>(alpha, beta, tab, (int)items, H, dv, g, (uint8_t *)ws, err,
-                                     mq, mk, mv);
+                                     mq, mk, mv, ma);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -366,17 +366,10 @@ __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
 
-// Per-thread asynchronous 16-byte copy global -> shared (cp.async, no
-// registers in between); `bytes` < 16 reads only that many bytes and fills
-// the rest of the 16 with zeros (0: nothing is read). Both addresses 16-byte
-// aligned. Completion: cp_async_commit() groups this thread's copies,
+// Per-thread asynchronous copy of one 4-byte element global -> shared
+// (cp.async, no registers in between; both addresses 4-byte aligned).
+// Completion: cp_async_commit() groups this thread's copies,
 // cp_async_wait_all() waits for all of them.
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)),
-               "l"(src), "r"(bytes)
-               : "memory");
-}
-// The same for one 4-byte element (both addresses 4-byte aligned).
 __device__ __forceinline__ void cp_async4(void *dst_smem, const void *src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src)
                : "memory");
