@@ -264,6 +264,10 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
       tma_load_3d(sm + P_V, &map_v, 0, hr, t0r, &bin[0]);
     }
   };
+  // Beta is copied by threads BT .. BT + 63, not by thread 0: thread 0
+  // commits the workspace's bulk stores, and its cp.async wait was measured
+  // to last until those stores had finished.
+  constexpr int BT = 64;
   auto issue_gates = [&](int t0r, int Lr, int hr) {  // alpha (no fused prologue), beta
     if constexpr (!GATED) {
       if (tid == 0) {
@@ -271,11 +275,12 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
         tma_load_3d(sAl, &map_a, 0, hr, t0r, &bin[1]);
       }
     }
-    if (tid < C) {
-      if (tid < Lr) cp_async4(sB + tid, beta + (size_t)(t0r + tid) * H + hr);
-      else sB[tid] = 0.f;
+    if (tid >= BT && tid < BT + C) {  // beta: threads BT .. BT + 63
+      const int j = tid - BT;
+      if (j < Lr) cp_async4(sB + j, beta + (size_t)(t0r + j) * H + hr);
+      else sB[j] = 0.f;
+      cp_async_commit();
     }
-    cp_async_commit();
   };
   auto wait_in = [&](int b, uint32_t parity) {  // all threads
     if (!mbar_wait(&bin[b], parity)) *s_abort = 1;
@@ -326,7 +331,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
       wait_in(0, ph);
       if constexpr (!GATED) wait_in(1, ph);
       ahead = 0;
-      cp_async_wait_all();
+      if (tid >= BT && tid < BT + C) cp_async_wait_all();
       if constexpr (GATED) {
         __syncthreads();  // every thread's k rows have landed
 #pragma unroll
@@ -380,8 +385,10 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
           }
         }
       }
-      // the gate pass writes over the staging: the stores must have read it
-      if (tid == 0) bulk_wait_read0();
+      // The previous item's workspace stores read their staging in three
+      // groups, committed in the order this item writes over them. The gate
+      // pass's Gram rows go over group 1 ([Qtil ; W] columns 0..95).
+      if (tid == 0) bulk_wait_read<2>();
     }
     __syncthreads();
 
@@ -443,6 +450,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
         sfx *= a[u];
       }
       sP[gq * DK + gc] = p;
+      if (tid == 0) bulk_wait_read<1>();  // the R stack goes over group 2
       __syncthreads();
       float P[4];
 #pragma unroll
@@ -473,6 +481,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
                         to_tf32(suf * kr[u + 2]), to_tf32(suf * kr[u + 3]));
       if (gq == 3) reinterpret_cast<float *>(wsb + ws_gamma_off(DV))[gc] = pre * p;
     }
+    if (tid == 0) bulk_wait_read<0>();  // the sweep's A and M go over group 3
     fence_async_smem();
     __syncthreads();
 
@@ -1029,8 +1038,14 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
-      bulk_s2g(wsb + WS_A1, sm + P_GA, 65536);
+      // three groups, in the order the next item writes over their sources:
+      // [Qtil ; W] columns 0..95 (the Gram rows' buffer); its columns 96..127
+      // and the M Ut rows (the R stack's); the Ut rows (over A and M)
+      bulk_s2g(wsb + WS_A1, sm + P_GA, 49152);
+      bulk_commit();
+      bulk_s2g(wsb + WS_A1 + 49152, sm + P_GA + 49152, 16384);
       bulk_s2g(wsb + WS_OU, sm + P_OU, 64u * DV * 4u);
+      bulk_commit();
       bulk_s2g(wsb + WS_OU + 64u * DV * 4u, sm + P_A, 64u * DV * 4u);
       bulk_commit();
     }

@@ -365,6 +365,13 @@ __device__ __forceinline__ void bulk_commit() {
 __device__ __forceinline__ void bulk_wait_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
+// Wait until at most N of this thread's most recently committed bulk groups
+// are still reading their shared-memory sources (groups complete in commit
+// order, so every older group has finished reading).
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
 
 // Per-thread asynchronous copy of one 4-byte element global -> shared
 // (cp.async, no registers in between; both addresses 4-byte aligned).
