@@ -1012,38 +1012,47 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
     if (!wait_all(&bar[2], ph, s_abort)) break;
     {
       const int qw = warp & 3, cg = warp >> 2, row = 32 * qw + lane;
-      for (int cb = 32 * cg; cb < DK + DV; cb += 128) {
+      {  // [Qtil ; W] columns 32 cg .. 32 cg + 31, tf32, K-major sw128 image
+        const int cb = 32 * cg;
         float x[32];
         tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)cb, x);
-        if (cb < DK) {  // [Qtil ; W] rows, tf32, K-major sw128 image
-          if (row < C) {  // warp-uniform (lane quarters 0, 1)
-            float qh[32];
-            tmem_ld32(tm + lane_base + TP_QH + (uint32_t)cb, qh);
+        if (row < C) {  // warp-uniform (lane quarters 0, 1)
+          float qh[32];
+          tmem_ld32(tm + lane_base + TP_QH + (uint32_t)cb, qh);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] = qh[e] - x[e];
-          }
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            st4_f32(sm + P_GA + off_k_sw128_f32(row, cb + e, DK), x[e], x[e + 1], x[e + 2], x[e + 3]);
-        } else {  // [M Ut ; Ut] rows, fp32, pieces swizzled by row (Ut rows over A, M)
-          uint8_t *dst = row < C ? sm + P_OU + (size_t)row * DV * 4 : sm + P_A + (size_t)(row - C) * DV * 4;
-          const int pc0 = (cb - DK) >> 2;
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4 *>(dst + 16 * ou_piece(row, pc0 + (e >> 2))) =
-                make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+          for (int e = 0; e < 32; ++e) x[e] = qh[e] - x[e];
         }
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          st4_f32(sm + P_GA + off_k_sw128_f32(row, cb + e, DK), x[e], x[e + 1], x[e + 2], x[e + 3]);
+      }
+      // The workspace stores go in three groups, in the order the next item
+      // writes over their sources: [Qtil ; W] columns 0..95 (the Gram rows'
+      // buffer); its columns 96..127 and the M Ut rows (the R stack's); the Ut
+      // rows (over A and M). The [Qtil ; W] image is complete here, so its
+      // stores start while the [M Ut ; Ut] rows are staged.
+      fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        bulk_s2g(wsb + WS_A1, sm + P_GA, 49152);
+        bulk_commit();
+        bulk_s2g(wsb + WS_A1 + 49152, sm + P_GA + 49152, 16384);
+      }
+      // [M Ut ; Ut] rows, fp32, pieces swizzled by row (Ut rows over A, M)
+      for (int cb = 32 * cg + DK; cb < DK + DV; cb += 128) {
+        float x[32];
+        tmem_ld32(tm + lane_base + TP_D5 + (uint32_t)cb, x);
+        uint8_t *dst = row < C ? sm + P_OU + (size_t)row * DV * 4 : sm + P_A + (size_t)(row - C) * DV * 4;
+        const int pc0 = (cb - DK) >> 2;
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4 *>(dst + 16 * ou_piece(row, pc0 + (e >> 2))) =
+              make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
       }
     }
     fence_async_smem();
     __syncthreads();
     if (tid == 0) {
-      // three groups, in the order the next item writes over their sources:
-      // [Qtil ; W] columns 0..95 (the Gram rows' buffer); its columns 96..127
-      // and the M Ut rows (the R stack's); the Ut rows (over A and M)
-      bulk_s2g(wsb + WS_A1, sm + P_GA, 49152);
-      bulk_commit();
-      bulk_s2g(wsb + WS_A1 + 49152, sm + P_GA + 49152, 16384);
       bulk_s2g(wsb + WS_OU, sm + P_OU, 64u * DV * 4u);
       bulk_commit();
       bulk_s2g(wsb + WS_OU + 64u * DV * 4u, sm + P_A, 64u * DV * 4u);
