@@ -6,11 +6,12 @@
 //
 //  * ckda_chunk_prep_kernel: persistent, one CTA per SM, walking the (chunk,
 //    head) items of all sequences (a small kernel first tabulates which
-//    chunk each slot holds); q, k, v and alpha come in by tensor-map copies. For each item it builds everything that does not
-//    depend on the state entering it (the chunk-WY / UT-transform factors of
-//    the product of diagonal-plus-rank-one transitions, Semidirect Fourier
-//    Delta Attention §2.2, and the affine chunk transfer's write summary, §1
-//    contribution 4), and stores the serial step's operands in a workspace:
+//    chunk each slot holds); q, k, v and alpha come in by tensor-map copies.
+//    For each item it builds everything that does not depend on the state
+//    entering it (the chunk-WY / UT-transform factors of the product of
+//    diagonal-plus-rank-one transitions, Semidirect Fourier Delta Attention
+//    §2.2, and the affine chunk transfer's write summary, §1 contribution 4),
+//    and stores the serial step's operands in a workspace:
 //        [Qtil ; W]   = [Qhat - M W ; T diag(beta) Khat]       128 x d_k
 //        Kbar^T                                                d_k x 64
 //        [M Ut ; Ut]  = [M T ; T] diag(beta) V                 128 x d_v
