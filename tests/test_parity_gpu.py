@@ -212,6 +212,19 @@ def test_bf16_ragged_small(cuda_lib):
     check_close(sf, sf_ref, 1e-2, 0.0, "final_state")
 
 
+@pytest.mark.parametrize("H", [1, 3])
+def test_batch_shorter_than_one_box(cuda_lib, H):
+    """A whole packed batch of 5 tokens: every 64-token input box of the
+    tensor-core prep reaches past the last token (those rows read as zeros,
+    then are cleared), with one head and with three."""
+    w = custom("ckda_B1_H32_T8192_d128", seed=4400 + H)
+    inp = make_fwd_inputs(w, cu_seqlens=lens_cu([5]), H=H)
+    o, sf = run_fwd(inp)
+    o_ref, sf_ref = ref_fwd(inp)
+    check_bf16_out(o, o_ref)
+    check_close(sf, sf_ref, SHORT_STATE_REL, 0.0, "final_state")
+
+
 def test_partial_chunk_ignores_the_next_sequence(cuda_lib):
     """The tensor-core prep loads q, k and v in whole 64-token boxes, so the
     rows past the end of a sequence's last (partial) chunk first hold the next
