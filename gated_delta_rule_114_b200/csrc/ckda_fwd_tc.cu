@@ -44,7 +44,6 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
-#include <cstring>
 #include <mutex>
 
 #include "ckda.h"
@@ -57,7 +56,6 @@ namespace {
 using namespace tc;
 
 constexpr int C = 64, DK = 128, DVT = 32;
-constexpr int PF_STEP = 128;  // bytes per L2 prefetch of the next item's gate logits
 constexpr int AL_S = 132;  // fp32 row stride of alpha / Qhat
 
 // Float offset of (row i, channel c) in the alpha / Qhat buffer: rows of 128
@@ -135,6 +133,7 @@ constexpr uint32_t P_Q = 114688;      // 16384 raw q bf16 [64][128]
 constexpr uint32_t P_K = 131072;      // 16384 raw k bf16 [64][128]
 constexpr uint32_t P_A0 = 114688;     // 32768 [M ; I] (128 x 64 K-major), over raw q and k
 constexpr uint32_t P_AL = 147456;     // 33792 alpha fp32 [64][132] -> Qhat fp32
+constexpr uint32_t P_AL_LOGIT = 17408; // fused prologue: the bf16 gate logits [64][128] land here in alpha's buffer
 constexpr uint32_t P_A = 181248;      // 17408 A fp32 [64][68] (with P_M: staged Ut rows, epilogue)
 constexpr uint32_t P_M = 198656;      // 17408 M fp32 [64][68]
 constexpr uint32_t P_B = 216064;      //   256 beta
@@ -192,21 +191,20 @@ __device__ __forceinline__ bool wait_all(uint64_t *bar, uint32_t phase,
   return *s_abort == 0;
 }
 
-// GATED: the fused input prologue (GateArgs): `alpha` holds bf16 gate
-// logits, `beta` fp32 logits and `k` raw keys; the key row inverse norms rn
-// are applied to every product k enters (Gram rows, R, Kbar, beta Khat and
-// the diagonal sub-blocks), which is the same as using the normalised keys.
+// GATED: the fused input prologue (GateArgs): the alpha tensor map is over
+// bf16 gate logits, `beta` holds fp32 logits and `k` raw keys; the key row
+// inverse norms rn are applied to every product k enters (Gram rows, R, Kbar,
+// beta Khat and the diagonal sub-blocks), which is the same as using the
+// normalised keys.
 template <bool GATED>
 __global__ void __launch_bounds__(NTP, 1)
-ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
-                       const float *__restrict__ beta,
+ckda_chunk_prep_kernel(const float *__restrict__ beta,
                        const int2 *__restrict__ slot_tab, int n_items,
                        int H, int DV, GateArgs ga, uint8_t *__restrict__ ws,
                        unsigned int *err, const __grid_constant__ CUtensorMap map_q,
                        const __grid_constant__ CUtensorMap map_k,
                        const __grid_constant__ CUtensorMap map_v,
                        const __grid_constant__ CUtensorMap map_a) {
-  const __nv_bfloat16 *__restrict__ alogit = reinterpret_cast<const __nv_bfloat16 *>(alpha_in);
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -225,7 +223,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   uint64_t *bar = reinterpret_cast<uint64_t *>(sm + P_BAR);  // [0..3]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_BAR + 32);
   volatile int *s_abort = reinterpret_cast<volatile int *>(sm + P_BAR + 36);
-  uint64_t *bin = reinterpret_cast<uint64_t *>(sm + P_BAR + 40);  // input copies: [0] q, k, v; [1] alpha
+  uint64_t *bin = reinterpret_cast<uint64_t *>(sm + P_BAR + 40);  // input copies: [0] q, k, v; [1] alpha (or its logits)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (warp == 0) {
@@ -244,10 +242,11 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   const uint32_t tm = *s_tmem;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
 
-  // An item's q, k and v rows and, without the fused prologue, alpha arrive
-  // by tensor-map copies (one box of 64 token rows per input, issued by
-  // thread 0, counted on mbarrier bin[0] or bin[1]); beta (or its logits) by
-  // per-thread copies (cp.async). They are issued during the previous item
+  // An item's q, k and v rows and alpha (with the fused prologue, alpha's bf16
+  // logits, into the upper half of alpha's buffer) arrive by tensor-map copies
+  // (one box of 64 token rows per input, issued by thread 0, counted on
+  // mbarrier bin[0] or bin[1]); beta (or its logits) by per-thread copies
+  // (cp.async). They are issued during the previous item
   // once each buffer's last reader is done: alpha and beta when the [M ; I]
   // and T operands are built (Qhat has moved to tensor memory, and gamma and
   // beta were last read by the WY operand build), q, k, v while D5 runs
@@ -269,9 +268,12 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   // commits the workspace's bulk stores, and its cp.async wait was measured
   // to last until those stores had finished.
   constexpr int BT = 64;
-  auto issue_gates = [&](int t0r, int Lr, int hr) {  // alpha (no fused prologue), beta
-    if constexpr (!GATED) {
-      if (tid == 0) {
+  auto issue_gates = [&](int t0r, int Lr, int hr) {  // alpha (or its logits), beta
+    if (tid == 0) {
+      if constexpr (GATED) {
+        mbar_arrive_expect_tx(&bin[1], (uint32_t)C * DK * 2u);
+        tma_load_3d(sm + P_AL + P_AL_LOGIT, &map_a, 0, hr, t0r, &bin[1]);
+      } else {
         mbar_arrive_expect_tx(&bin[1], (uint32_t)C * AL_S * 4u);
         tma_load_3d(sAl, &map_a, 0, hr, t0r, &bin[1]);
       }
@@ -309,32 +311,30 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   uint8_t *wsb = ws + ((size_t)slot * H + h) * ws_block_bytes(DV);
 
   do {  // one pass; `break` leaves on a timed-out wait
-    // ---------------- 1. load the chunk: q, k, v, beta and (without the fused
-    // prologue) alpha have been copied in asynchronously; the gate logits of
-    // the fused prologue come through registers
+    // ---------------- 1. load the chunk: q, k, v, alpha (or its logits) and
+    // beta have been copied in asynchronously
     if (raw_for != it) {
       issue_qkv(t0, h);
       issue_gates(t0, L, h);
     }
     raw_for = -1;
     {
-      uint4 al[2];  // GATED: 64 rows x 16 pieces of 8 bf16 logits
+      wait_in(0, ph);
+      wait_in(1, ph);
+      ahead = 0;
+      uint4 al[2];  // GATED: 64 rows x 16 pieces of 8 bf16 logits, read before alpha overwrites them
       (void)al;
       if constexpr (GATED) {
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
           al[u] = make_uint4(0, 0, 0, 0);
-          if (i < L)
-            al[u] = __ldg(reinterpret_cast<const uint4 *>(alogit + ((size_t)(t0 + i) * H + h) * DK + ch * 8));
+          if (i < L) al[u] = *reinterpret_cast<const uint4 *>(sm + P_AL + P_AL_LOGIT + i * 256 + ch * 16);
         }
       }
-      wait_in(0, ph);
-      if constexpr (!GATED) wait_in(1, ph);
-      ahead = 0;
       if (tid >= BT && tid < BT + C) cp_async_wait_all();
       if constexpr (GATED) {
-        __syncthreads();  // every thread's k rows have landed
+        __syncthreads();  // every thread's logits are read (alpha goes over them)
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int idx = tid + u * NTP, i = idx >> 4, ch = idx & 15;
@@ -392,21 +392,6 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
       if (tid == 0) bulk_wait_read<2>();
     }
     __syncthreads();
-
-    // the next item's gate logits (fused prologue) into L2 (plain line
-    // prefetches) while this item is computed; every address lies inside its
-    // row
-    if constexpr (GATED) {
-      if (nxt.y > 0) {
-        const int nh = nit % H;
-        constexpr int la = DK * 2 / PF_STEP;  // pieces of a logit row
-        const char *gate_in = reinterpret_cast<const char *>(alpha_in);
-        for (int t = tid; t < nxt.y * la; t += NTP) {
-          const int r = t / la, w = t % la;
-          prefetch_line_l2(gate_in + ((size_t)(nxt.x + r) * H + nh) * DK * 2 + PF_STEP * w);
-        }
-      }
-    }
 
     // ---------------- 2. gate pass: thread (16-token sub-block g, channel c)
     // forms the sub-block prefix products p_u = prod_{s=16g..16g+u} alpha_s
@@ -979,7 +964,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
     if (nxt.y > 0) {
       issue_gates(nxt.x, nxt.y, nit % H);
       raw_for = nit;
-      if constexpr (!GATED) ahead |= 2;
+      ahead |= 2;
     }
     if (!wait_all(&bar[1], ph, s_abort)) break;
     if ((warp & 3) < 2) {  // rows of M T: round the fp32 accumulator to tf32
@@ -1070,7 +1055,7 @@ ckda_chunk_prep_kernel(const void *__restrict__ alpha_in,
   // item's own, if waiting for them is what timed out, phase ph (an already
   // completed phase is not waited for).
   if (*s_abort) {
-    for (int b = 0; b < (GATED ? 1 : 2); ++b) wait_in(b, ((ahead >> b) & 1) ? ph ^ 1u : ph);
+    for (int b = 0; b < 2; ++b) wait_in(b, ((ahead >> b) & 1) ? ph ^ 1u : ph);
   }
   cp_async_wait_all();  // copies issued ahead land before shared memory is released
   if (tid == 0) {
@@ -1437,17 +1422,17 @@ cudaError_t launch_fwd_tc(int dv, const void *q, const void *k, const void *v,
     const long long items = (long long)slots * H;
     if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
     const int grid = (int)std::min<long long>(items, (long long)sm_count());
-    // input boxes: q, k (128 channels), v (d_v), alpha (128 channels padded to
-    // the 132-float shared row); the fused prologue reads its gate logits itself
+    // input boxes: q, k (128 channels), v (d_v), and alpha (128 channels padded
+    // to the 132-float shared row) or, with the fused prologue, its bf16 logits
     CUtensorMap mq, mk, mv, ma;
-    std::memset(&ma, 0, sizeof(ma));
     const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!encode_rows(&mq, q, bf, 2, DK, H, T_total, DK) ||
         !encode_rows(&mk, k, bf, 2, DK, H, T_total, DK) ||
         !encode_rows(&mv, v, bf, 2, dv, H, T_total, dv) ||
-        (!g.on && !encode_rows(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, H, T_total, AL_S)))
+        !(g.on ? encode_rows(&ma, alpha, bf, 2, DK, H, T_total, DK)
+               : encode_rows(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, H, T_total, AL_S)))
       return cudaErrorInvalidValue;
-    prep<<<grid, NTP, P_SMEM, st>>>(alpha, beta, tab, (int)items, H, dv, g, (uint8_t *)ws, err,
+    prep<<<grid, NTP, P_SMEM, st>>>(beta, tab, (int)items, H, dv, g, (uint8_t *)ws, err,
                                      mq, mk, mv, ma);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
