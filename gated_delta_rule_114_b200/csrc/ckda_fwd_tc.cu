@@ -1224,12 +1224,6 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
     for (int c = 0; c < nch; ++c) {
       const int b = c & 1;
       const int t0 = bos + C * c, L = min(C, eos - t0);
-      float ou[DVT];
-#pragma unroll
-      for (int e = 0; e < DVT; ++e) ou[e] = ou_next[e];
-      const float gc = gc_next;
-      if (c + 1 < nch) load_rows(c + 1);
-
       if (tid == ISS || tid == ISS2) {  // D1 = [Qtil ; W] x S, K split over two issuers
         const int h2 = tid == ISS2;
         if (!mbar_wait(&bar[B_READY + b], (uint32_t)(c >> 1) & 1u)) *s_abort = 1;
@@ -1240,6 +1234,13 @@ ckda_chunk_scan_kernel(const float *__restrict__ s0, float *__restrict__ sfin,
                       desc_mn_sw128b32_f32(sb + S_S, DK, kk + 8 * h2), ID_D1, kk > 0);
         mma_commit(&bar[B_D1]);
       }
+      // this chunk's rows (loaded one chunk ahead) and the next chunk's loads
+      // come after the MMA issue, so that the issuing threads reach it first
+      float ou[DVT];
+#pragma unroll
+      for (int e = 0; e < DVT; ++e) ou[e] = ou_next[e];
+      const float gc = gc_next;
+      if (c + 1 < nch) load_rows(c + 1);
       if (!mbar_wait(&bar[B_D1], (uint32_t)c & 1u)) *s_abort = 1;
       fence_after_sync();
       float d1[32];
