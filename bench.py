@@ -76,8 +76,8 @@ def esize(dt):
 # capture, its command and the scaling are in profiles/. Set to None whenever
 # a kernel changes after its capture.
 NCU_TRAFFIC = {
-    # prep + scan at T=2048, H=32 (1024 chunk-heads): 193.3 + 178.4 MB, x4 for T=8192
-    "prefill": 4 * 371.7e6,
+    # prep + scan at T=2048, H=32 (1024 chunk-heads): 193.3 + 178.5 MB, x4 for T=8192
+    "prefill": 4 * 371.8e6,
     # N=64 (2048 pairs): 214.8 MB, x4 for N=256
     "decode": 4 * 214.8e6,
     # token-serial backward (both kernels) at T=512, H=32: 356.3 MB, x16 for T=8192
