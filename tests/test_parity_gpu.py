@@ -225,13 +225,15 @@ def test_batch_shorter_than_one_box(cuda_lib, H):
     check_close(sf, sf_ref, SHORT_STATE_REL, 0.0, "final_state")
 
 
-def test_partial_chunk_ignores_the_next_sequence(cuda_lib):
+@pytest.mark.parametrize("d_v", [128, 64, 32])
+def test_partial_chunk_ignores_the_next_sequence(cuda_lib, d_v):
     """The tensor-core prep loads q, k and v in whole 64-token boxes, so the
     rows past the end of a sequence's last (partial) chunk first hold the next
     sequence's tokens, until the kernel clears them. With that next sequence
     full of NaN and inf (q, k, v, alpha, beta), the sequences before and after
-    it must still match the oracle run on them alone."""
-    w = custom("ckda_B1_H32_T8192_d128", seed=4343)
+    it must still match the oracle run on them alone, for every d_v the
+    tensor-core path takes."""
+    w = custom("ckda_B1_H32_T8192_d128", d_v=d_v, seed=4343 + d_v)
     inp = make_fwd_inputs(w, cu_seqlens=lens_cu([100, 70, 29]), H=4)
     poison(inp, 100, 170, ("q", "k", "v", "alpha", "beta"))
     o, sf = run_fwd(inp)
