@@ -4,7 +4,8 @@ A CPU restatement of the chunk-WY data flow of the tensor-core path (64-token
 chunks, Grams factored at the 16-token sub-block and 4-token group boundaries,
 T = (I + A)^-1, the two WY products, then the state chain) in fp64, rounding
 the operands of each tensor-core product to a chosen format (fp32, tf32 with
-round-to-nearest-away as cvt.rna.tf32.f32 does, or bf16 round-to-nearest-even)
+round-to-nearest-away as cvt.rna.tf32.f32 does, tf32 cut off (what an MMA
+reading an unrounded fp32 value uses), or bf16 round-to-nearest-even)
 and keeping the accumulations exact. It compares o and the final state with
 the fp64 token oracle on the CKDA long-prefill distribution. It is neither the
 oracle nor the CUDA path: it only tells which operand precision each product
@@ -44,6 +45,9 @@ def rnd(x, kind):
         b = x.astype(np.float32).view(np.uint32).astype(np.uint64)
         b = (b + 0x1000) & 0xFFFFE000
         return b.astype(np.uint32).view(np.float32).astype(np.float64)
+    if kind == "tf32t":  # keep 10 mantissa bits, the rest cut off
+        b = x.astype(np.float32).view(np.uint32) & np.uint32(0xFFFFE000)
+        return b.view(np.float32).astype(np.float64)
     if kind == "bf16":
         return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
     raise ValueError(kind)
@@ -86,7 +90,7 @@ def chunk(S, q, k, v, al, be, P):
     MT = rnd(M, P["mt"]) @ rnd(T, P["mt"])
     bK = rnd(be[..., None] * gam * k, P["wy"])
     bV = rnd(be[..., None] * v, P["wy"])
-    Tq, MTq = rnd(T, P["wy"]), rnd(MT, P["wy"])
+    Tq, MTq = rnd(T, P["wy"]), rnd(MT, P.get("mtq", P["wy"]))
     W, Ut, MW, MUt = Tq @ bK, Tq @ bV, MTq @ bK, MTq @ bV
     Qt = gam * q - MW
     Sq = rnd(S, P["state"])
@@ -123,6 +127,8 @@ VARIANTS = {
     "tf32 everywhere (the kernels)": dict(gram="tf32", mt="tf32", wy="tf32", scan="tf32", state="tf32"),
     "bf16 Gram operands": dict(gram="bf16", mt="tf32", wy="tf32", scan="tf32", state="tf32"),
     "bf16 [M;I] x T": dict(gram="tf32", mt="bf16", wy="tf32", scan="tf32", state="tf32"),
+    "[MT;T] truncated as D5's A operand": dict(gram="tf32", mt="tf32", wy="tf32", mtq="tf32t",
+                                               scan="tf32", state="tf32"),
     "bf16 WY product": dict(gram="tf32", mt="tf32", wy="bf16", scan="tf32", state="tf32"),
     "bf16 chain A operands, tf32 S and U": dict(gram="tf32", mt="tf32", wy="tf32", scan="bf16", state="tf32"),
     "bf16 chain (A and S, U)": dict(gram="tf32", mt="tf32", wy="tf32", scan="bf16", state="bf16"),
